@@ -1,0 +1,366 @@
+"""Benchmark of the NF4-LoRA hot path on B200.
+
+Workload (one GPU): the Llama-7B q_proj shape -- W 4096 x 4096 stored NF4 with
+double quantization (E4M3 absmax, groups of 256), X 8192 x 4096 bf16 (batch 4 x
+seq 2048), rank 16, alpha 32, forward + backward (dX, dL1, dL2).
+
+One timed step runs every step of the path once on that batch:
+  nf4_quantize(W, dq)                  quantize + double-quantize the scales
+  nf4_layer_error_rank([W], K=0)       per-layer NF4 error + ranking
+  qlora_linear_fwd                     T = X L1; Y = X W^T + s T L2 (fused dequant GEMM)
+  qlora_linear_bwd                     U, dL2, dL1, dX = dY W + s U L1^T (fused dequant GEMM)
+`value` counts only the algorithmic fwd+bwd flops (4 M h o + 6 M r (h + o))
+over the whole step time; per-leg times are reported beside it.
+
+With torchrun (N > 1 GPUs) every rank runs the same step on its own batch of
+8192 tokens (weak scaling) and the adapter gradients dL1 / dL2 are summed
+across ranks with an NCCL all-reduce, the one exchange a data-parallel step has.
+
+`--impl reference` times the CPU oracle (the plain fp64 restatement of the
+method used by the tests) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NF4-LoRA linear fwd+bwd TFLOP/s (frac of bf16 peak); NF4 quant/error GB/s"
+UNIT = "TFLOP/s"
+WORKLOAD = "llama7b-q_proj: W 4096x4096 NF4 blocksize 64 + double-quant (e4m3 absmax, group 256), X 8192x4096 bf16, r=16, alpha=32, fwd+bwd"
+
+
+def flops_fwd_bwd(M, h, o, r):
+    return 4.0 * M * h * o + 6.0 * M * r * (h + o)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def config_dict(args, world):
+    return {"workload": WORKLOAD, "M_per_gpu": args.M, "in": 4096, "out": 4096, "r": 16, "alpha": 32,
+            "global_tokens": args.M * world, "l2": "flushed between timed steps (256 MiB write)",
+            "parallelism": f"dp{world}" if world > 1 else "single-gpu"}
+
+
+# --------------------------------------------------------------------------- CPU oracle leg
+
+def run_oracle_sample(rows: int, seed: int = 0):
+    """Times the oracle on the q_proj workload: full W quantize (+DQ) and error,
+    fwd+bwd on `rows` token rows. Returns (seconds, flops_counted, description)."""
+    import numpy as np
+    from oracle import layer_error, lora, nf4
+    from quantized_lora_fine_b200 import synth
+
+    case = synth.case_q_proj(seed=seed, M=rows)
+    d = case.make()
+    Wb = synth.bf16_bits(d["W"])
+    X, L1, L2, dY = (nf4.f32_from_bf16_bits(synth.bf16_bits(d[k])).astype(np.float64) for k in ("X", "L1", "L2", "dY"))
+    t0 = time.perf_counter()
+    qw = nf4.quantize(nf4.f32_from_bf16_bits(Wb).reshape(d["W"].shape), double_quant=True)
+    What = nf4.f32_from_bf16_bits(nf4.dequantize_bf16_bits(qw)).astype(np.float64).reshape(d["W"].shape)
+    layer_error.layer_error(Wb, True)
+    Y, T = lora.forward(X, What, L1, L2, case.scale)
+    lora.backward(X, What, L1, L2, dY, case.scale)
+    dt = time.perf_counter() - t0
+    return dt, flops_fwd_bwd(rows, 4096, 4096, 16), (
+        f"oracle (numpy fp64) on {rows} of 8192 token rows: full 4096x4096 quantize+DQ, error pass, "
+        f"fwd+bwd; rate = fwd+bwd flops of the rows / wall time")
+
+
+def cpu_threads():
+    try:
+        import numpy as np  # noqa: F401
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info()]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def reference_main(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = 256
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm state worth priming beyond its table cache
+    run_oracle_sample(16)  # builds the NF4 table cache
+    times = []
+    for _ in range(max(1, args.steps)):
+        dt, fl, desc = run_oracle_sample(rows)
+        times.append(dt)
+    dt = statistics.median(times)
+    tf = fl / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": tf, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(args, 1),
+            "cpu_baseline": {"value": tf, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": desc},
+            "e2e": {"value": tf, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU leg
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"qlb_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for ln in open(self.path):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), reasons=parts[4:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = set()
+        for r in rows:
+            for nm, v in zip(names, r["reasons"][1:]):
+                if v.lower() in ("active", "0x1", "1", "yes"):
+                    seen.add(nm)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(seen), "samples": len(rows)}
+
+
+def gpu_main(args):
+    import ctypes
+
+    import torch
+    import torch.distributed as dist
+
+    from quantized_lora_fine_b200 import _lib, api, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    lib = _lib.load()
+    peaks = load_peaks()
+
+    M, h, o, r, alpha = args.M, 4096, 4096, 16, 32.0
+    s = alpha / r
+    case = synth.case_q_proj(seed=0, M=M)
+    # weak scaling: each rank draws its own batch (matrix index offset) over the same weights
+    d = case.make(device="cpu")
+    if world > 1 and rank > 0:
+        import dataclasses
+        d2 = dataclasses.replace(case, index=rank).make(device="cpu")
+        d["X"], d["dY"] = d2["X"], d2["dY"]
+    g = {k: v.to(dev) for k, v in d.items()}
+    stream = torch.cuda.current_stream()
+
+    def run_step(W, X, dY, L1, L2):
+        w = api.quantize(W, double_quant=True)
+        api.layer_error_rank([W], 0, double_quant=True)
+        Y, T = api.linear_fwd(w, X, L1, L2, s)
+        dX, dL1, dL2 = api.linear_bwd(w, X, dY, L1, L2, s, T=T)
+        if world > 1:
+            dist.all_reduce(dL1)
+            dist.all_reduce(dL2)
+        return Y, dX, dL1, dL2
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    prof = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    # legs, measured once per step with events between the calls
+    for _ in range(max(3, args.warmup)):
+        run_step(g["W"], g["X"], g["dY"], g["L1"], g["L2"])
+    torch.cuda.synchronize()
+    assert api.status() == 0, "device status set during warm-up"
+
+    lib.qlora_profile_events(ctypes.c_void_p(prof[0].cuda_event), ctypes.c_void_p(prof[1].cuda_event),
+                             ctypes.c_void_p(prof[2].cuda_event), ctypes.c_void_p(prof[3].cuda_event))
+    step_ms, legs = [], {"quantize": [], "error_rank": [], "fwd": [], "bwd": [], "fwd_gemm": [], "dx_gemm": []}
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        ev[0].record(stream)
+        w = api.quantize(g["W"], double_quant=True)
+        ev[1].record(stream)
+        api.layer_error_rank([g["W"]], 0, double_quant=True)
+        ev[2].record(stream)
+        Y, T = api.linear_fwd(w, g["X"], g["L1"], g["L2"], s)
+        ev[3].record(stream)
+        dX, dL1, dL2 = api.linear_bwd(w, g["X"], g["dY"], g["L1"], g["L2"], s, T=T)
+        if world > 1:
+            dist.all_reduce(dL1)
+            dist.all_reduce(dL2)
+        ev[4].record(stream)
+        ev[4].synchronize()
+        step_ms.append(ev[0].elapsed_time(ev[4]))
+        legs["quantize"].append(ev[0].elapsed_time(ev[1]))
+        legs["error_rank"].append(ev[1].elapsed_time(ev[2]))
+        legs["fwd"].append(ev[2].elapsed_time(ev[3]))
+        legs["bwd"].append(ev[3].elapsed_time(ev[4]))
+        legs["fwd_gemm"].append(prof[0].elapsed_time(prof[1]))
+        legs["dx_gemm"].append(prof[2].elapsed_time(prof[3]))
+    clk = clocks.stop()
+    lib.qlora_profile_events(None, None, None, None)
+    torch.cuda.synchronize()
+    assert api.status() == 0, "device status set during timing"
+
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / args.steps
+    fl = flops_fwd_bwd(M, h, o, r)
+    value = fl * world / (ms * 1e-3) / 1e12
+
+    med = {k: statistics.median(v) for k, v in legs.items()}
+    fl_fwd_gemm = 2.0 * M * h * o + 2.0 * M * r * o
+    fl_dx_gemm = 2.0 * M * o * h + 2.0 * M * r * h
+    fwd_tf = fl_fwd_gemm / (med["fwd_gemm"] * 1e-3) / 1e12
+    dx_tf = fl_dx_gemm / (med["dx_gemm"] * 1e-3) / 1e12
+    # dominant kernel = the longer of the two fused GEMMs
+    dom = ("qlora_fwd_gemm (tc_gemm_kernel FwdNF4)", fwd_tf, med["fwd_gemm"]) if med["fwd_gemm"] >= med["dx_gemm"] \
+        else ("qlora_bwd_dx_gemm (tc_gemm_kernel DxNF4)", dx_tf, med["dx_gemm"])
+    n = M * h  # placeholder not used
+    numel = h * o
+    quant_bytes = numel * 2 + numel // 2 + numel // 64 + 4 * (numel // 64 // 256)
+    err_bytes = numel * 2
+    roofline = {"kernel": dom[0], "bound": "tensor", "achieved": dom[1], "peak": peaks["bf16_sus"],
+                "unit": "TFLOP/s", "frac": dom[1] / peaks["bf16_sus"],
+                "peak_kind": f"bf16 sustained ({peaks['source']})",
+                "frac_of_burst": dom[1] / peaks["bf16"], "traffic": None,
+                "per_launch_flops": fl_fwd_gemm if dom[0].startswith("qlora_fwd") else fl_dx_gemm}
+    legs_out = {
+        "quantize": {"ms": med["quantize"], "GB/s": quant_bytes / (med["quantize"] * 1e-3) / 1e9,
+                     "frac_hbm": quant_bytes / (med["quantize"] * 1e-3) / 1e9 / peaks["hbm"]},
+        "error_rank": {"ms": med["error_rank"], "GB/s": err_bytes / (med["error_rank"] * 1e-3) / 1e9,
+                       "frac_hbm": err_bytes / (med["error_rank"] * 1e-3) / 1e9 / peaks["hbm"]},
+        "fwd": {"ms": med["fwd"]}, "bwd": {"ms": med["bwd"]},
+        "fwd_gemm": {"ms": med["fwd_gemm"], "TFLOP/s": fwd_tf}, "dx_gemm": {"ms": med["dx_gemm"], "TFLOP/s": dx_tf},
+    }
+
+    # ------------------------------------------------ end to end with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = {k: v.cpu().pin_memory() for k, v in d.items()}
+        outs = {"Y": torch.empty((M, o), dtype=torch.bfloat16).pin_memory(),
+                "dX": torch.empty((M, h), dtype=torch.bfloat16).pin_memory(),
+                "dL1": torch.empty((h, r), dtype=torch.float32).pin_memory(),
+                "dL2": torch.empty((r, o), dtype=torch.float32).pin_memory()}
+        h2d = sum(t.numel() * t.element_size() for t in pin.values())
+        d2h = sum(t.numel() * t.element_size() for t in outs.values())
+        dev_in = {k: torch.empty_like(v, device=dev) for k, v in pin.items()}
+        e2e_ms = []
+        for i in range(args.e2e_steps + 2):
+            flush.zero_()
+            ev[0].record(stream)
+            for k in pin:
+                dev_in[k].copy_(pin[k], non_blocking=True)
+            Y, dX, dL1, dL2 = run_step(dev_in["W"], dev_in["X"], dev_in["dY"], dev_in["L1"], dev_in["L2"])
+            outs["Y"].copy_(Y, non_blocking=True)
+            outs["dX"].copy_(dX, non_blocking=True)
+            outs["dL1"].copy_(dL1, non_blocking=True)
+            outs["dL2"].copy_(dL2, non_blocking=True)
+            ev[1].record(stream)
+            ev[1].synchronize()
+            if i >= 2:
+                e2e_ms.append(ev[0].elapsed_time(ev[1]))
+        em = sum(e2e_ms) / len(e2e_ms)
+        if world > 1:
+            t = torch.tensor([em], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            em = float(t.item())
+        e2e = {"value": fl * world / (em * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": em,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        run_oracle_sample(16)
+        dt, cfl, desc = run_oracle_sample(args.cpu_rows)
+        cpu = {"value": cfl / dt / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": desc,
+               "seconds": dt}
+
+    launches_per_step = 1 + 3 + 5 + 9
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args, world),
+            "roofline": roofline, "legs": legs_out, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clk,
+            "peaks": {"bf16_tflops": peaks["bf16"], "bf16_tflops_sustained": peaks["bf16_sus"],
+                      "hbm_gbs": peaks["hbm"], "source": peaks["source"]}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--M", type=int, default=8192)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return reference_main(args)
+    return gpu_main(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,212 @@
+/*
+ * qlora_b200.h -- C ABI of the NF4-LoRA hot path for NVIDIA B200 (sm_100a).
+ *
+ * The operations and the pages that define them:
+ *   nf4_quantize / nf4_dequantize
+ *       "QLoRA: How to fine-tune large language models with less memory",
+ *       sections "1. NormalFloat" (16 normal-shaped 4-bit codes, one scale per
+ *       block of weights, dequantized to BFloat16 before the matmul) and
+ *       "2. Double quantization" (8-bit first-level scales, a higher-precision
+ *       scale per group of 256); AQLoRA summary page, section 3.1 (64-element
+ *       blocks).
+ *   qlora_linear_fwd
+ *       Same QLoRA page, "The algebra", eq. (3): Y = X W + s X L1 L2, with the
+ *       scaling s = alpha / r of "LoRA: Fine-tuning a model by learning a small
+ *       update", eq. (3).
+ *   qlora_linear_bwd
+ *       Gradients of eq. (3) with the base frozen: gradient reaches X through
+ *       the dequantized W, no gradient is formed for W ("Lesson 17. What QLoRA
+ *       Actually Costs", warm-up; QLoRA page, "One training step").
+ *   nf4_layer_error_rank
+ *       AQLoRA summary page, sections 3.1-3.2: per-layer NF4 reconstruction
+ *       error, ranking, top-K kept in 16-bit.
+ *
+ * Conventions (all entry points):
+ *   - Every tensor is dense, row-major, and lives in device memory owned by the
+ *     caller. The library never allocates device memory on these calls; scratch
+ *     comes from a caller workspace sized by the matching *_workspace_size().
+ *   - bf16 tensors are passed as uint16_t* (bit patterns).
+ *   - Weights are stored out x in (nn.Linear layout): W_s = W^T of eq. (3).
+ *     Quantization blocks of 64 run along `in` (the flattened row-major order).
+ *   - Work is enqueued on `stream` and runs asynchronously; pointers must stay
+ *     valid until it completes. Host-side argument checks run before any
+ *     launch and return an error without touching device memory.
+ *   - Device-side conditions (non-finite weights, an internal wait that ran
+ *     out) are recorded in an int32 status word at the start of the
+ *     workspace. The word is sticky: it keeps the first error until
+ *     qlora_reset_status(). A fresh workspace must be zeroed (or reset) once.
+ *   - No call aborts the process or throws.
+ */
+#ifndef QLORA_B200_H
+#define QLORA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* qlora_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_NULL = 1,        /* a required pointer is NULL                         */
+  QLORA_ERR_SHAPE = 2,       /* a size or a size combination is not supported      */
+  QLORA_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                   */
+  QLORA_ERR_DTYPE = 4,       /* unknown dtype code                                 */
+  QLORA_ERR_UNSUPPORTED = 5, /* device is not sm_100, or a config value unsupported */
+  QLORA_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed                  */
+  QLORA_ERR_WORKSPACE = 7,   /* workspace NULL, misaligned or too small            */
+  QLORA_ERR_NONFINITE = 8,   /* device: a weight was NaN or +-Inf                  */
+  QLORA_ERR_TIMEOUT = 9      /* device: a pipeline wait exceeded its limit         */
+} qlora_status;
+
+enum { QLORA_DTYPE_BF16 = 0, QLORA_DTYPE_F32 = 1 };
+
+/* Quantization config: blocksize must be 64 and dq_blocksize 256 (the values
+ * the pages give); double_quant is 0 or 1. */
+typedef struct {
+  int32_t blocksize;
+  int32_t double_quant;
+  int32_t dq_blocksize;
+} nf4_qconfig;
+
+/* Descriptor of one frozen linear weight, stored out x in.
+ *   is_bf16 = 0: NF4 storage.
+ *     codes    uint8 [out*in/2]; byte k holds element 2k in its high nibble and
+ *              element 2k+1 in its low nibble; a nibble is the index (0..15) of
+ *              the code in the ascending NF4 table.
+ *     absmax   fp32 [out*in/64]          (double_quant = 0)
+ *     absmax_q uint8 [out*in/64], E4M3   (double_quant = 1)
+ *     absmax2  fp32 [ceil(out*in/64/256)] (double_quant = 1)
+ *   is_bf16 = 1: a protected layer kept in 16-bit (AQLoRA section 3.2);
+ *     w_bf16 bf16 [out*in]; the NF4 fields are ignored.
+ */
+typedef struct {
+  int64_t out;
+  int64_t in;
+  nf4_qconfig q;
+  int32_t is_bf16;
+  const uint8_t* codes;
+  const float* absmax;
+  const uint8_t* absmax_q;
+  const float* absmax2;
+  const uint16_t* w_bf16;
+} qlora_weight;
+
+/* ------------------------------------------------------------------ status */
+
+const char* qlora_status_str(qlora_status s);
+
+/* Synchronizes `stream` and returns the device status word in `workspace`
+ * (QLORA_OK if no device-side error was recorded). */
+qlora_status qlora_read_status(const void* workspace, qlora_stream_t stream);
+
+/* Clears the device status word (stream-ordered). */
+qlora_status qlora_reset_status(void* workspace, qlora_stream_t stream);
+
+/* Checks that device `device` is an sm_100 part and that the library's kernels
+ * can be loaded on it. */
+qlora_status qlora_device_check(int device);
+
+/* Profiling aid (not part of the method): when set, cudaEvent_t handles that
+ * the library records on the caller's stream right before and right after the
+ * main tensor-core GEMM of qlora_linear_fwd (fwd_*) and of qlora_linear_bwd
+ * (dx_*). Pass NULL to disable. Process-wide; not thread-safe. */
+qlora_status qlora_profile_events(void* fwd_begin, void* fwd_end, void* dx_begin, void* dx_end);
+
+/* ------------------------------------------------------------ NF4 codec */
+
+/* Bytes of workspace nf4_quantize needs (the status word only). */
+size_t nf4_quantize_workspace_size(int64_t numel);
+
+/* Blockwise NF4 quantization of W (numel = out*in elements, any even count;
+ * a short last block uses the elements present).
+ *   W        device, bf16 (w_dtype QLORA_DTYPE_BF16) or fp32, 16-byte aligned
+ *   codes    device out, uint8 [numel/2]
+ *   absmax   device out, fp32 [ceil(numel/64)]; required when double_quant = 0,
+ *            optional (may be NULL) when double_quant = 1
+ *   absmax_q device out, uint8 [ceil(numel/64)]      (double_quant = 1)
+ *   absmax2  device out, fp32 [ceil(numel/64/256)]   (double_quant = 1)
+ * Per block b: a_b = max|w| (fp32); n = w / a_b (IEEE fp32 division); code =
+ * #{j : n > m_j} over the 15 fp32 midpoints of adjacent codes. With double
+ * quantization, per group of 256 scales: G = max a_b, q_b =
+ * E4M3_rn_satfinite(a_b * fp32(448/G)), absmax2 = fp32(G/448); codes always use
+ * the exact a_b. A NaN/Inf weight sets QLORA_ERR_NONFINITE in the status word
+ * (codes of that block are then unspecified; the call still completes). */
+qlora_status nf4_quantize(const void* W, int32_t w_dtype, int64_t out, int64_t in, nf4_qconfig q,
+                          uint8_t* codes, float* absmax, uint8_t* absmax_q, float* absmax2,
+                          void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* Dequantization to bf16: W_out[i] = bf16_rn(fp32_rn(code[idx_i] * a)) with a the
+ * block's absmax, or with double quantization a = fp32_rn(fp32(q_b) * absmax2[g]).
+ *   w      host pointer to a descriptor with is_bf16 = 0 (device buffers inside)
+ *   W_out  device out, bf16 [out*in], 16-byte aligned */
+qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream_t stream);
+
+/* --------------------------------------------------------- NF4-LoRA linear */
+
+/* Shape rules for the linear: in % 256 == 0, out % 256 == 0, M >= 1 (any),
+ * r % 8 == 0 and 8 <= r <= 256; every pointer 16-byte aligned. */
+size_t qlora_fwd_workspace_size(int64_t M, int64_t out, int64_t in, int32_t r);
+size_t qlora_bwd_workspace_size(int64_t M, int64_t out, int64_t in, int32_t r);
+
+/* Forward, eq. (3) in stored layout:
+ *   T = X L1             (M x r; fp32 accumulation, rounded once to bf16)
+ *   Y = X W_s^T + s T L2 (M x out; fp32 accumulation in tensor memory, one bf16
+ *                         rounding at the end)
+ *   w       host pointer to the weight descriptor (NF4 or protected bf16)
+ *   X       device bf16 [M x in]     L1 device bf16 [in x r]   L2 device bf16 [r x out]
+ *   scale   s (alpha / r, or any value)
+ *   Y       device out, bf16 [M x out]
+ *   T_save  device out, bf16 [M x r] (T, unscaled), or NULL to keep it in the
+ *           workspace only.
+ * The NF4 weight is dequantized tile by tile inside the GEMM; no dequantized
+ * copy of W is written to memory. */
+qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t M,
+                              const uint16_t* L1, const uint16_t* L2, int32_t r, float scale,
+                              uint16_t* Y, uint16_t* T_save,
+                              void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* Backward of the forward above (no gradient for W):
+ *   U   = dY L2^T                 (M x r, bf16 after fp32 accumulation)
+ *   dX  = dY W_s + s U L1^T       (M x in, bf16)          -- skipped if dX == NULL
+ *   dL2 = s T^T dY                (r x out, fp32)
+ *   dL1 = s X^T U                 (in x r, fp32)
+ *   T_saved  device bf16 [M x r] from the forward, or NULL to recompute T = X L1.
+ * dX == NULL expresses an early backward stop below the lowest adapted layer
+ * (AQLoRA section 3.3). dL1/dL2 are overwritten, not accumulated. Their
+ * reductions run in a fixed order, so repeated calls give identical bits. */
+qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const uint16_t* dY, int64_t M,
+                              const uint16_t* L1, const uint16_t* L2, int32_t r, float scale,
+                              const uint16_t* T_saved, uint16_t* dX, float* dL1, float* dL2,
+                              void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* ------------------------------------------------------ AQLoRA allocation */
+
+/* Workspace for nf4_layer_error_rank over n_layers matrices of the given
+ * element counts (host array). */
+size_t nf4_layer_error_rank_workspace_size(int32_t n_layers, const int64_t* numel);
+
+/* Per-layer NF4 reconstruction error, ranking and top-K selection.
+ *   W_ptrs   HOST array of n_layers DEVICE pointers, each a bf16 matrix
+ *            (w_dtype must be QLORA_DTYPE_BF16), 16-byte aligned
+ *   numel    HOST array of element counts (each a positive multiple of 64)
+ *   q        quantization config used for every layer (double_quant 0 or 1)
+ *   K        number of layers to keep (0 <= K <= n_layers)
+ *   err      device out, fp64 [n_layers]: e = sqrt(sum (w - w_hat)^2 / sum w^2)
+ *            with w_hat the bf16 dequantized weight (0 for an all-zero matrix)
+ *   order    device out, int32 [n_layers]: layer ids by (err desc, id asc)
+ *   keep     device out, uint8 [n_layers]: 1 for the first K of `order`
+ * 1 <= n_layers <= 1024. Sums run in fp64 in a fixed order (deterministic). */
+qlora_status nf4_layer_error_rank(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
+                                  int32_t w_dtype, nf4_qconfig q, int32_t K,
+                                  double* err, int32_t* order, uint8_t* keep,
+                                  void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_B200_H */

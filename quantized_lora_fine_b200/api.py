@@ -1,0 +1,183 @@
+"""Torch-facing binding of the C ABI: tensors in, tensors out.
+
+PyTorch supplies device memory and the current stream; the arithmetic of every
+step runs in libqlora_b200.so. Functions mirror the C entry points:
+
+    quantize(W, double_quant)              -> NF4Weight        (nf4_quantize)
+    dequantize(w)                          -> bf16 tensor      (nf4_dequantize)
+    linear_fwd(w, X, L1, L2, scale)        -> (Y, T)           (qlora_linear_fwd)
+    linear_bwd(w, X, dY, L1, L2, scale, T) -> (dX, dL1, dL2)   (qlora_linear_bwd)
+    layer_error_rank(Ws, K, double_quant)  -> (err, order, keep) (nf4_layer_error_rank)
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import DTYPE_BF16, DTYPE_F32, NF4QConfig, QLoraWeight, check
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class Workspace:
+    """A grow-only device scratch buffer per device, zeroed at allocation (its
+    first 4 bytes are the library's sticky device status word)."""
+
+    _bufs = {}
+
+    @classmethod
+    def get(cls, nbytes: int, device: torch.device) -> torch.Tensor:
+        key = torch.device(device).index or 0
+        buf = cls._bufs.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+            cls._bufs[key] = buf
+        return buf
+
+
+def read_status(ws: torch.Tensor) -> int:
+    return _lib.load().qlora_read_status(ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(_stream()))
+
+
+def reset_status(ws: torch.Tensor) -> None:
+    check(_lib.load().qlora_reset_status(ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(_stream())), "reset_status")
+
+
+@dataclasses.dataclass
+class NF4Weight:
+    """An NF4 (or protected bf16) frozen weight stored out x in."""
+    out: int
+    inp: int
+    double_quant: bool
+    codes: Optional[torch.Tensor] = None
+    absmax: Optional[torch.Tensor] = None
+    absmax_q: Optional[torch.Tensor] = None
+    absmax2: Optional[torch.Tensor] = None
+    w_bf16: Optional[torch.Tensor] = None
+
+    @property
+    def is_bf16(self) -> bool:
+        return self.w_bf16 is not None
+
+    @staticmethod
+    def protected(W: torch.Tensor) -> "NF4Weight":
+        _need(W, torch.bfloat16, "W")
+        return NF4Weight(W.shape[0], W.shape[1], False, w_bf16=W)
+
+    def c_struct(self) -> QLoraWeight:
+        s = QLoraWeight()
+        s.out, s.in_ = self.out, self.inp
+        s.q = NF4QConfig(64, 1 if self.double_quant else 0, 256)
+        s.is_bf16 = 1 if self.is_bf16 else 0
+        s.codes = _ptr(self.codes)
+        s.absmax = _ptr(self.absmax)
+        s.absmax_q = _ptr(self.absmax_q)
+        s.absmax2 = _ptr(self.absmax2)
+        s.w_bf16 = _ptr(self.w_bf16)
+        return s
+
+
+def quantize(W: torch.Tensor, double_quant: bool = False, keep_absmax: bool = False) -> NF4Weight:
+    """NF4-quantize a 2-D bf16 or fp32 CUDA tensor stored out x in."""
+    if W.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("W must be bf16 or fp32")
+    _need(W, W.dtype, "W")
+    lib = _lib.load()
+    out, inp = W.shape
+    n = W.numel()
+    nb = (n + 63) // 64
+    dev = W.device
+    codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(nb, dtype=torch.float32, device=dev) if (not double_quant or keep_absmax) else None
+    absmax_q = torch.empty(nb, dtype=torch.uint8, device=dev) if double_quant else None
+    absmax2 = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev) if double_quant else None
+    ws = Workspace.get(lib.nf4_quantize_workspace_size(n), dev)
+    check(lib.nf4_quantize(_ptr(W), DTYPE_BF16 if W.dtype == torch.bfloat16 else DTYPE_F32, out, inp,
+                           NF4QConfig(64, 1 if double_quant else 0, 256), _ptr(codes), _ptr(absmax),
+                           _ptr(absmax_q), _ptr(absmax2), _ptr(ws), ws.numel(), _stream()), "nf4_quantize")
+    return NF4Weight(out, inp, double_quant, codes=codes, absmax=absmax, absmax_q=absmax_q, absmax2=absmax2)
+
+
+def dequantize(w: NF4Weight) -> torch.Tensor:
+    lib = _lib.load()
+    out = torch.empty((w.out, w.inp), dtype=torch.bfloat16, device=w.codes.device)
+    cs = w.c_struct()
+    check(lib.nf4_dequantize(ctypes.byref(cs), _ptr(out), _stream()), "nf4_dequantize")
+    return out
+
+
+def linear_fwd(w: NF4Weight, X: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, scale: float,
+               save_T: bool = True, Y: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    for t, nm in ((X, "X"), (L1, "L1"), (L2, "L2")):
+        _need(t, torch.bfloat16, nm)
+    lib = _lib.load()
+    M, r = X.shape[0], L1.shape[1]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, w.out), dtype=torch.bfloat16, device=dev)
+    T = torch.empty((M, r), dtype=torch.bfloat16, device=dev) if save_T else None
+    ws = Workspace.get(lib.qlora_fwd_workspace_size(M, w.out, w.inp, r), dev)
+    cs = w.c_struct()
+    check(lib.qlora_linear_fwd(ctypes.byref(cs), _ptr(X), M, _ptr(L1), _ptr(L2), r, float(scale), _ptr(Y), _ptr(T),
+                               _ptr(ws), ws.numel(), _stream()), "qlora_linear_fwd")
+    return Y, T
+
+
+def linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, scale: float,
+               T: Optional[torch.Tensor] = None, need_dX: bool = True):
+    for t, nm in ((X, "X"), (dY, "dY"), (L1, "L1"), (L2, "L2")):
+        _need(t, torch.bfloat16, nm)
+    lib = _lib.load()
+    M, r = X.shape[0], L1.shape[1]
+    dev = X.device
+    dX = torch.empty((M, w.inp), dtype=torch.bfloat16, device=dev) if need_dX else None
+    dL1 = torch.empty((w.inp, r), dtype=torch.float32, device=dev)
+    dL2 = torch.empty((r, w.out), dtype=torch.float32, device=dev)
+    ws = Workspace.get(lib.qlora_bwd_workspace_size(M, w.out, w.inp, r), dev)
+    cs = w.c_struct()
+    check(lib.qlora_linear_bwd(ctypes.byref(cs), _ptr(X), _ptr(dY), M, _ptr(L1), _ptr(L2), r, float(scale), _ptr(T),
+                               _ptr(dX), _ptr(dL1), _ptr(dL2), _ptr(ws), ws.numel(), _stream()), "qlora_linear_bwd")
+    return dX, dL1, dL2
+
+
+def layer_error_rank(Ws: Sequence[torch.Tensor], K: int, double_quant: bool = False):
+    lib = _lib.load()
+    L = len(Ws)
+    for i, W in enumerate(Ws):
+        _need(W, torch.bfloat16, f"W[{i}]")
+    dev = Ws[0].device
+    ptrs = (ctypes.c_void_p * L)(*[W.data_ptr() for W in Ws])
+    numel = (ctypes.c_int64 * L)(*[W.numel() for W in Ws])
+    err = torch.empty(L, dtype=torch.float64, device=dev)
+    order = torch.empty(L, dtype=torch.int32, device=dev)
+    keep = torch.empty(L, dtype=torch.uint8, device=dev)
+    ws = Workspace.get(lib.nf4_layer_error_rank_workspace_size(L, numel), dev)
+    check(lib.nf4_layer_error_rank(L, ptrs, numel, DTYPE_BF16, NF4QConfig(64, 1 if double_quant else 0, 256), K,
+                                   _ptr(err), _ptr(order), _ptr(keep), _ptr(ws), ws.numel(), _stream()),
+          "nf4_layer_error_rank")
+    return err, order, keep
+
+
+def status() -> int:
+    """Device status word of this device's shared workspace (synchronizes)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    return read_status(Workspace.get(256, dev))

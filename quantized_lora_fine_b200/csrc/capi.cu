@@ -1,0 +1,419 @@
+// C entry points: host-side validation, workspace carving and the launch
+// sequence of each operation. Every compute step runs in this library's kernels.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "gemm.cuh"
+#include "internal.cuh"
+
+using namespace qlb;
+
+namespace {
+
+constexpr int kThinTargetCtas = 296;  // split-K target for the thin LoRA products (fixed: results do not
+                                      // depend on the device's SM count)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+inline cudaStream_t S(qlora_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+qlora_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  static int checked_dev = -1;
+  static qlora_status cached = QLORA_OK;
+  if (checked_dev == dev) return cached;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  cached = (major == 10 && minor == 0) ? QLORA_OK : QLORA_ERR_UNSUPPORTED;
+  checked_dev = dev;
+  return cached;
+}
+
+bool qconfig_ok(const nf4_qconfig& q) {
+  return q.blocksize == 64 && q.dq_blocksize == 256 && (q.double_quant == 0 || q.double_quant == 1);
+}
+
+struct ThinSplit {
+  int tiles, splits, kps;
+};
+
+ThinSplit thin_split(int64_t rows, int64_t ksteps) {
+  ThinSplit t;
+  t.tiles = int((rows + 127) / 128);
+  int sp = std::max(1, int((kThinTargetCtas + t.tiles - 1) / t.tiles));
+  sp = int(std::min<int64_t>(sp, ksteps));
+  t.kps = int((ksteps + sp - 1) / sp);
+  t.splits = int((ksteps + t.kps - 1) / t.kps);
+  return t;
+}
+
+int thin_bn(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
+
+// ---- workspace layouts
+
+struct FwdLayout {
+  size_t scales, l2t, t, part, total;
+};
+
+FwdLayout fwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
+  FwdLayout L;
+  size_t off = kStatusBytes;
+  L.scales = off; off += up256(size_t(out) * size_t(in / 64) * 4);
+  L.l2t = off;    off += up256(size_t(out) * r * 2);
+  L.t = off;      off += up256(size_t(M) * r * 2);
+  const ThinSplit ts = thin_split(M, in / 64);
+  L.part = off;   off += up256(size_t(ts.splits) * size_t(M) * r * 4);
+  L.total = off;
+  return L;
+}
+
+struct BwdLayout {
+  size_t scales, l1s, t, u, part, total;
+};
+
+BwdLayout bwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
+  BwdLayout L;
+  size_t off = kStatusBytes;
+  L.scales = off; off += up256(size_t(out) * size_t(in / 64) * 4);
+  L.l1s = off;    off += up256(size_t(in) * r * 2);
+  L.t = off;      off += up256(size_t(M) * r * 2);
+  L.u = off;      off += up256(size_t(M) * r * 2);
+  const ThinSplit a = thin_split(M, in / 64), b = thin_split(M, out / 64);
+  const ThinSplit c = thin_split(out, (M + 63) / 64), d = thin_split(in, (M + 63) / 64);
+  size_t part = std::max({size_t(a.splits) * M * r, size_t(b.splits) * M * r, size_t(c.splits) * out * r,
+                          size_t(d.splits) * in * r}) * 4;
+  L.part = off;   off += up256(part);
+  L.total = off;
+  return L;
+}
+
+qlora_status check_linear(const qlora_weight* w, int64_t M, int32_t r) {
+  if (!w) return QLORA_ERR_NULL;
+  if (w->out <= 0 || w->in <= 0 || M <= 0) return QLORA_ERR_SHAPE;
+  if (w->in % 256 || w->out % 256) return QLORA_ERR_SHAPE;
+  if (w->in > (int64_t(1) << 30) || w->out > (int64_t(1) << 30) || M > (int64_t(1) << 30)) return QLORA_ERR_SHAPE;
+  if (r < 8 || r > 256 || r % 8) return QLORA_ERR_SHAPE;
+  if (w->is_bf16) {
+    if (!w->w_bf16) return QLORA_ERR_NULL;
+    if (!aligned16(w->w_bf16)) return QLORA_ERR_ALIGN;
+  } else {
+    if (!qconfig_ok(w->q)) return QLORA_ERR_UNSUPPORTED;
+    if (!w->codes) return QLORA_ERR_NULL;
+    if (!aligned16(w->codes)) return QLORA_ERR_ALIGN;
+    if (w->q.double_quant) {
+      if (!w->absmax_q || !w->absmax2) return QLORA_ERR_NULL;
+    } else if (!w->absmax) {
+      return QLORA_ERR_NULL;
+    }
+  }
+  return QLORA_OK;
+}
+
+// thin product into fp32 partials then a reduction
+struct Thin {
+  GemmKind kind;
+  const void* a; int64_t a_inner, a_outer;  // A tensor as stored: inner x outer (row-major)
+  const void* b; int64_t b_inner, b_outer;
+  int64_t rows;        // D rows
+  int64_t ksteps;      // K / 64 (ceil)
+  int r;
+};
+
+qlora_status run_thin(const Thin& t, float* part, int* status, cudaStream_t s, int* splits_out) {
+  const ThinSplit ts = thin_split(t.rows, t.ksteps);
+  const int bn = thin_bn(t.r);
+  GemmOperands o;
+  std::memset(&o, 0, sizeof(o));
+  const bool a_mn = t.kind == GemmKind::ThinMM;
+  const bool b_mn = t.kind != GemmKind::ThinKK;
+  if (!make_tmap_2d(&o.A, t.a, TmapType::BF16, t.a_inner, t.a_outer, t.a_inner * 2, 64, a_mn ? 64 : 128, true))
+    return QLORA_ERR_CUDA;
+  if (!make_tmap_2d(&o.B, t.b, TmapType::BF16, t.b_inner, t.b_outer, t.b_inner * 2, 64, b_mn ? 64 : bn, true))
+    return QLORA_ERR_CUDA;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = int(t.rows);
+  p.N = t.r;
+  p.num_k_main = int(t.ksteps);
+  p.num_k_ext = 0;
+  p.tiles_m = ts.tiles;
+  p.tiles_n = 1;
+  p.splits = ts.splits;
+  p.ksteps_per_split = ts.kps;
+  p.out = part;
+  p.ld_out = t.r;
+  p.split_stride = t.rows * t.r;
+  p.status = status;
+  *splits_out = ts.splits;
+  return launch_gemm(t.kind, bn, o, p, s);
+}
+
+#define QLB_TRY(x)                         \
+  do {                                     \
+    qlora_status _st = (x);                \
+    if (_st != QLORA_OK) return _st;       \
+  } while (0)
+
+cudaEvent_t g_prof[4] = {nullptr, nullptr, nullptr, nullptr};
+
+// main GEMM with NF4 or bf16 weight and the LoRA extension
+qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t M, const uint16_t* Ax,
+                      const uint16_t* Bx, int32_t r, const float* scales_t, uint16_t* out, int* status,
+                      cudaStream_t s) {
+  const int64_t o_ = w->out, h = w->in;
+  const int64_t Kdim = dx ? o_ : h;   // reduction length
+  const int64_t Ndim = dx ? h : o_;   // output columns
+  GemmOperands op;
+  std::memset(&op, 0, sizeof(op));
+  if (!make_tmap_2d(&op.A, A, TmapType::BF16, Kdim, M, Kdim * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d(&op.Ax, Ax, TmapType::BF16, r, M, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d(&op.Bx, Bx, TmapType::BF16, r, Ndim, int64_t(r) * 2, 64, 256, true)) return QLORA_ERR_CUDA;
+  GemmKind kind;
+  if (w->is_bf16) {
+    if (!dx) {
+      if (!make_tmap_2d(&op.B, w->w_bf16, TmapType::BF16, h, o_, h * 2, 64, 256, true)) return QLORA_ERR_CUDA;
+      kind = GemmKind::FwdBF16;
+    } else {
+      if (!make_tmap_2d(&op.B, w->w_bf16, TmapType::BF16, h, o_, h * 2, 64, 64, true)) return QLORA_ERR_CUDA;
+      kind = GemmKind::DxBF16;
+    }
+  } else {
+    if (!dx) {
+      if (!make_tmap_2d(&op.codes, w->codes, TmapType::U8, h / 2, o_, h / 2, 32, 256, false)) return QLORA_ERR_CUDA;
+      if (!make_tmap_2d(&op.scales, scales_t, TmapType::F32, o_, h / 64, o_ * 4, 256, 1, false)) return QLORA_ERR_CUDA;
+      kind = GemmKind::FwdNF4;
+    } else {
+      if (!make_tmap_2d(&op.codes, w->codes, TmapType::U8, h / 2, o_, h / 2, 128, 64, true)) return QLORA_ERR_CUDA;
+      if (!make_tmap_2d(&op.scales, scales_t, TmapType::F32, o_, h / 64, o_ * 4, 64, 4, false)) return QLORA_ERR_CUDA;
+      kind = GemmKind::DxNF4;
+    }
+  }
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = int(M);
+  p.N = int(Ndim);
+  p.num_k_main = int(Kdim / 64);
+  p.num_k_ext = (r + 63) / 64;
+  p.tiles_m = int((M + 127) / 128);
+  p.tiles_n = int(Ndim / 256);
+  p.splits = 1;
+  p.ksteps_per_split = p.num_k_main;
+  p.out = out;
+  p.ld_out = Ndim;
+  p.split_stride = 0;
+  p.status = status;
+  cudaEvent_t eb = g_prof[dx ? 2 : 0], ee = g_prof[dx ? 3 : 1];
+  if (eb) cudaEventRecord(eb, s);
+  const qlora_status st = launch_gemm(kind, 256, op, p, s);
+  if (ee) cudaEventRecord(ee, s);
+  return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qlora_status_str(qlora_status s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_NULL: return "null pointer";
+    case QLORA_ERR_SHAPE: return "unsupported shape";
+    case QLORA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case QLORA_ERR_DTYPE: return "unknown dtype";
+    case QLORA_ERR_UNSUPPORTED: return "unsupported device or configuration";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case QLORA_ERR_NONFINITE: return "non-finite weight";
+    case QLORA_ERR_TIMEOUT: return "device pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+qlora_status qlora_profile_events(void* fwd_begin, void* fwd_end, void* dx_begin, void* dx_end) {
+  g_prof[0] = static_cast<cudaEvent_t>(fwd_begin);
+  g_prof[1] = static_cast<cudaEvent_t>(fwd_end);
+  g_prof[2] = static_cast<cudaEvent_t>(dx_begin);
+  g_prof[3] = static_cast<cudaEvent_t>(dx_end);
+  return QLORA_OK;
+}
+
+qlora_status qlora_device_check(int device) {
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return (major == 10 && minor == 0) ? QLORA_OK : QLORA_ERR_UNSUPPORTED;
+}
+
+qlora_status qlora_read_status(const void* workspace, qlora_stream_t stream) {
+  if (!workspace) return QLORA_ERR_WORKSPACE;
+  int v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, S(stream)) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return QLORA_ERR_CUDA;
+  return static_cast<qlora_status>(v);
+}
+
+qlora_status qlora_reset_status(void* workspace, qlora_stream_t stream) {
+  if (!workspace) return QLORA_ERR_WORKSPACE;
+  return cudaMemsetAsync(workspace, 0, sizeof(int), S(stream)) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+size_t nf4_quantize_workspace_size(int64_t) { return kStatusBytes; }
+
+qlora_status nf4_quantize(const void* W, int32_t w_dtype, int64_t out, int64_t in, nf4_qconfig q, uint8_t* codes,
+                          float* absmax, uint8_t* absmax_q, float* absmax2, void* workspace, size_t workspace_bytes,
+                          qlora_stream_t stream) {
+  if (w_dtype != QLORA_DTYPE_BF16 && w_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
+  if (!qconfig_ok(q)) return QLORA_ERR_UNSUPPORTED;
+  if (out <= 0 || in <= 0) return QLORA_ERR_SHAPE;
+  const int64_t numel = out * in;
+  if (numel % 2) return QLORA_ERR_SHAPE;
+  if (!W || !codes) return QLORA_ERR_NULL;
+  if (q.double_quant ? (!absmax_q || !absmax2) : !absmax) return QLORA_ERR_NULL;
+  if (!aligned16(W)) return QLORA_ERR_ALIGN;
+  if (!aligned16(codes)) return QLORA_ERR_ALIGN;
+  if (!workspace || workspace_bytes < kStatusBytes || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  QLB_TRY(check_device());
+  return launch_quantize(W, w_dtype, numel, q.double_quant != 0, codes, absmax, absmax_q, absmax2,
+                         static_cast<int*>(workspace), S(stream));
+}
+
+qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream_t stream) {
+  if (!w || !W_out) return QLORA_ERR_NULL;
+  if (w->is_bf16) return QLORA_ERR_UNSUPPORTED;
+  if (!qconfig_ok(w->q)) return QLORA_ERR_UNSUPPORTED;
+  if (w->out <= 0 || w->in <= 0) return QLORA_ERR_SHAPE;
+  const int64_t numel = w->out * w->in;
+  if (numel % 2) return QLORA_ERR_SHAPE;
+  if (!w->codes) return QLORA_ERR_NULL;
+  if (w->q.double_quant ? (!w->absmax_q || !w->absmax2) : !w->absmax) return QLORA_ERR_NULL;
+  if (!aligned16(w->codes) || !aligned16(W_out)) return QLORA_ERR_ALIGN;
+  QLB_TRY(check_device());
+  return launch_dequantize(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, numel, W_out,
+                           S(stream));
+}
+
+size_t qlora_fwd_workspace_size(int64_t M, int64_t out, int64_t in, int32_t r) {
+  if (M <= 0 || out <= 0 || in <= 0 || r <= 0) return 0;
+  return fwd_layout(M, out, in, r).total;
+}
+
+size_t qlora_bwd_workspace_size(int64_t M, int64_t out, int64_t in, int32_t r) {
+  if (M <= 0 || out <= 0 || in <= 0 || r <= 0) return 0;
+  return bwd_layout(M, out, in, r).total;
+}
+
+qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t M, const uint16_t* L1,
+                              const uint16_t* L2, int32_t r, float scale, uint16_t* Y, uint16_t* T_save,
+                              void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  QLB_TRY(check_linear(w, M, r));
+  if (!X || !L1 || !L2 || !Y) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(L1) || !aligned16(L2) || !aligned16(Y) || (T_save && !aligned16(T_save)))
+    return QLORA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  const FwdLayout L = fwd_layout(M, w->out, w->in, r);
+  if (workspace_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  QLB_TRY(check_device());
+  cudaStream_t s = S(stream);
+  char* ws = static_cast<char*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  float* scales_t = reinterpret_cast<float*>(ws + L.scales);
+  uint16_t* l2t = reinterpret_cast<uint16_t*>(ws + L.l2t);
+  uint16_t* T = T_save ? T_save : reinterpret_cast<uint16_t*>(ws + L.t);
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  const int64_t h = w->in, o_ = w->out;
+  if (!w->is_bf16)
+    QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
+                                 scales_t, s));
+  QLB_TRY(launch_scale_lora(L2, r, o_, scale, /*transpose=*/true, l2t, s));
+  // T = X L1 : A = X (K-major), B = L1 as [h x r] (MN-major for B)
+  Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
+  int splits = 0;
+  QLB_TRY(run_thin(tt, part, status, s, &splits));
+  QLB_TRY(launch_reduce_bf16(part, splits, M, r, T, s));
+  return run_main(false, w, X, M, T, l2t, r, scales_t, Y, status, s);
+}
+
+qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const uint16_t* dY, int64_t M,
+                              const uint16_t* L1, const uint16_t* L2, int32_t r, float scale,
+                              const uint16_t* T_saved, uint16_t* dX, float* dL1, float* dL2, void* workspace,
+                              size_t workspace_bytes, qlora_stream_t stream) {
+  QLB_TRY(check_linear(w, M, r));
+  if (!X || !dY || !L1 || !L2 || !dL1 || !dL2) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(L1) || !aligned16(L2) || !aligned16(dL1) || !aligned16(dL2) ||
+      (dX && !aligned16(dX)) || (T_saved && !aligned16(T_saved)))
+    return QLORA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  const BwdLayout L = bwd_layout(M, w->out, w->in, r);
+  if (workspace_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  QLB_TRY(check_device());
+  cudaStream_t s = S(stream);
+  char* ws = static_cast<char*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  float* scales_t = reinterpret_cast<float*>(ws + L.scales);
+  uint16_t* l1s = reinterpret_cast<uint16_t*>(ws + L.l1s);
+  uint16_t* U = reinterpret_cast<uint16_t*>(ws + L.u);
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  const int64_t h = w->in, o_ = w->out;
+  const int64_t mk = (M + 63) / 64;
+  int splits = 0;
+  const uint16_t* T = T_saved;
+  if (!T) {
+    uint16_t* Tw = reinterpret_cast<uint16_t*>(ws + L.t);
+    Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
+    QLB_TRY(run_thin(tt, part, status, s, &splits));
+    QLB_TRY(launch_reduce_bf16(part, splits, M, r, Tw, s));
+    T = Tw;
+  }
+  // U = dY L2^T : A = dY (K-major, K = out), B = L2 [r x out] (K-major)
+  Thin tu{GemmKind::ThinKK, dY, o_, M, L2, o_, r, M, o_ / 64, r};
+  QLB_TRY(run_thin(tu, part, status, s, &splits));
+  QLB_TRY(launch_reduce_bf16(part, splits, M, r, U, s));
+  // dL2^T = dY^T T  (out x r): A = dY^T (MN-major), B = T (MN-major); K = M
+  Thin t2{GemmKind::ThinMM, dY, o_, M, T, r, M, o_, mk, r};
+  QLB_TRY(run_thin(t2, part, status, s, &splits));
+  QLB_TRY(launch_reduce_f32(part, splits, o_, r, scale, /*transpose=*/true, dL2, s));
+  // dL1 = X^T U (in x r): A = X^T (MN-major), B = U (MN-major); K = M
+  Thin t1{GemmKind::ThinMM, X, h, M, U, r, M, h, mk, r};
+  QLB_TRY(run_thin(t1, part, status, s, &splits));
+  QLB_TRY(launch_reduce_f32(part, splits, h, r, scale, /*transpose=*/false, dL1, s));
+  if (dX) {
+    if (!w->is_bf16)
+      QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
+                                   scales_t, s));
+    QLB_TRY(launch_scale_lora(L1, h, r, scale, /*transpose=*/false, l1s, s));
+    QLB_TRY(run_main(true, w, dY, M, U, l1s, r, scales_t, dX, status, s));
+  }
+  return QLORA_OK;
+}
+
+size_t nf4_layer_error_rank_workspace_size(int32_t n_layers, const int64_t* numel) {
+  if (n_layers <= 0 || !numel) return 0;
+  return layer_error_ws_bytes(n_layers, numel);
+}
+
+qlora_status nf4_layer_error_rank(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
+                                  int32_t w_dtype, nf4_qconfig q, int32_t K, double* err, int32_t* order,
+                                  uint8_t* keep, void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  if (w_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_DTYPE;
+  if (!qconfig_ok(q)) return QLORA_ERR_UNSUPPORTED;
+  if (n_layers < 1 || n_layers > 1024 || K < 0 || K > n_layers) return QLORA_ERR_SHAPE;
+  if (!W_ptrs || !numel || !err || !order || !keep) return QLORA_ERR_NULL;
+  for (int i = 0; i < n_layers; ++i) {
+    if (!W_ptrs[i]) return QLORA_ERR_NULL;
+    if (numel[i] <= 0 || numel[i] % 64) return QLORA_ERR_SHAPE;
+    if (!aligned16(W_ptrs[i])) return QLORA_ERR_ALIGN;
+  }
+  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  QLB_TRY(check_device());
+  return launch_layer_error_rank(n_layers, W_ptrs, numel, q.double_quant != 0, K, err, order, keep, workspace,
+                                 workspace_bytes, static_cast<int*>(workspace), S(stream));
+}
+
+}  // extern "C"

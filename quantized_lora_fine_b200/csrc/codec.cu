@@ -1,0 +1,292 @@
+// NF4 quantizer, dequantizer and the small elementwise / reduction kernels of
+// the LoRA path. All HBM-bound: 128-bit loads and stores, warp shuffles.
+#include <algorithm>
+#include <cfloat>
+#include <cuda_bf16.h>
+
+#include "internal.cuh"
+#include "nf4_device.cuh"
+
+namespace qlb {
+
+// ------------------------------------------------------------------ quantize
+//
+// One CTA of 256 threads per group of 256 blocks (16384 elements). In each of 8
+// slices, lane l of warp w handles elements [8*(l%8), 8*(l%8)+8) of block
+// (slice*32 + 4*w + l/8): a warp reads 512 contiguous bytes of bf16 per slice.
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* W, int64_t e0, int64_t numel, float (&w)[8]);
+
+template <>
+__device__ __forceinline__ void load8<uint16_t>(const uint16_t* W, int64_t e0, int64_t numel, float (&w)[8]) {
+  if (e0 + 8 <= numel) {
+    uint4 v = __ldg(reinterpret_cast<const uint4*>(W + e0));
+    uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { w[2 * i] = bf16_lo(u[i]); w[2 * i + 1] = bf16_hi(u[i]); }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = (e0 + i < numel) ? __uint_as_float(uint32_t(W[e0 + i]) << 16) : 0.f;
+  }
+}
+
+template <>
+__device__ __forceinline__ void load8<float>(const float* W, int64_t e0, int64_t numel, float (&w)[8]) {
+  if (e0 + 8 <= numel) {
+    float4 a = __ldg(reinterpret_cast<const float4*>(W + e0));
+    float4 b = __ldg(reinterpret_cast<const float4*>(W + e0 + 4));
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = (e0 + i < numel) ? W[e0 + i] : 0.f;
+  }
+}
+
+template <typename T, bool DQ>
+__global__ void __launch_bounds__(256) nf4_quantize_kernel(const T* __restrict__ W, int64_t numel,
+                                                           uint8_t* __restrict__ codes, float* __restrict__ absmax,
+                                                           uint8_t* __restrict__ absmax_q,
+                                                           float* __restrict__ absmax2, int* status) {
+  __shared__ float s_amax[256];
+  __shared__ float s_red[8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t nb = (numel + kBlock - 1) / kBlock;
+  const int64_t g = blockIdx.x;
+  bool bad = false;
+#pragma unroll 1
+  for (int it = 0; it < 8; ++it) {
+    const int bi = it * 32 + warp * 4 + (lane >> 3);
+    const int64_t blk = g * kDQBlock + bi;
+    const int64_t e0 = blk * kBlock + (lane & 7) * 8;
+    float w[8];
+    const bool live = blk < nb && e0 < numel;
+    if (live) load8<T>(W, e0, numel, w);
+    else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = 0.f;
+    }
+    float am = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float aw = fabsf(w[i]);
+      bad |= !(aw <= FLT_MAX);
+      am = fmaxf(am, aw);
+    }
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+    if ((lane & 7) == 0) {
+      s_amax[bi] = am;
+      if (blk < nb && absmax != nullptr) absmax[blk] = am;
+    }
+    if (live) {
+      uint32_t idx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) idx[i] = (am > 0.f) ? nf4_index(__fdiv_rn(w[i], am)) : 7u;
+      if (e0 + 8 <= numel) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) word |= ((idx[2 * k] << 4) | idx[2 * k + 1]) << (8 * k);
+        *reinterpret_cast<uint32_t*>(codes + e0 / 2) = word;
+      } else {
+        for (int k = 0; 2 * k < numel - e0; ++k) codes[e0 / 2 + k] = uint8_t((idx[2 * k] << 4) | idx[2 * k + 1]);
+      }
+    }
+  }
+  if (bad) set_status(status, QLORA_ERR_NONFINITE);
+  if constexpr (DQ) {
+    __syncthreads();
+    const int64_t nblk_g = (int64_t(kDQBlock) < nb - g * kDQBlock ? int64_t(kDQBlock) : nb - g * kDQBlock);
+    float v = (tid < nblk_g) ? s_amax[tid] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) s_red[warp] = v;
+    __syncthreads();
+    float G = s_red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) G = fmaxf(G, s_red[i]);
+    if (tid < nblk_g) {
+      uint8_t q = 0;
+      if (G > 0.f) {
+        const float inv = __fdiv_rn(448.f, G);
+        q = f32_to_e4m3_satfinite(__fmul_rn(s_amax[tid], inv));
+      }
+      absmax_q[g * kDQBlock + tid] = q;
+    }
+    if (tid == 0) absmax2[g] = (G > 0.f) ? __fdiv_rn(G, 448.f) : 0.f;
+  }
+}
+
+qlora_status launch_quantize(const void* W, int w_dtype, int64_t numel, bool dq, uint8_t* codes, float* absmax,
+                             uint8_t* absmax_q, float* absmax2, int* status, cudaStream_t s) {
+  const int64_t nb = (numel + kBlock - 1) / kBlock;
+  const int64_t groups = (nb + kDQBlock - 1) / kDQBlock;
+  if (groups <= 0) return QLORA_OK;
+  dim3 grid(static_cast<unsigned>(groups));
+  if (w_dtype == QLORA_DTYPE_BF16) {
+    if (dq) nf4_quantize_kernel<uint16_t, true><<<grid, 256, 0, s>>>((const uint16_t*)W, numel, codes, absmax, absmax_q, absmax2, status);
+    else nf4_quantize_kernel<uint16_t, false><<<grid, 256, 0, s>>>((const uint16_t*)W, numel, codes, absmax, absmax_q, absmax2, status);
+  } else {
+    if (dq) nf4_quantize_kernel<float, true><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
+    else nf4_quantize_kernel<float, false><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
+  }
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- dequantize
+//
+// Each thread turns 16 code bytes (32 elements, half a block) into 64 bytes of
+// bf16 through the per-block product table.
+
+__device__ __forceinline__ float block_scale(int64_t blk, const float* absmax, const uint8_t* absmax_q,
+                                             const float* absmax2, bool dq) {
+  if (!dq) return __ldg(absmax + blk);
+  return __fmul_rn(e4m3_to_f32(__ldg(absmax_q + blk)), __ldg(absmax2 + blk / kDQBlock));
+}
+
+__global__ void __launch_bounds__(256) nf4_dequantize_kernel(const uint8_t* __restrict__ codes,
+                                                             const float* __restrict__ absmax,
+                                                             const uint8_t* __restrict__ absmax_q,
+                                                             const float* __restrict__ absmax2, int dq,
+                                                             int64_t numel, uint16_t* __restrict__ out) {
+  const int64_t n_units = (numel + 31) / 32;
+  for (int64_t u = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; u < n_units; u += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t e0 = u * 32;
+    const int64_t blk = e0 / kBlock;
+    const float a = block_scale(blk, absmax, absmax_q, absmax2, dq != 0);
+    const NF4Lut t = nf4_make_lut(a);
+    if (e0 + 32 <= numel) {
+      const uint4 c = __ldg(reinterpret_cast<const uint4*>(codes + e0 / 2));
+      const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+      uint4* dst = reinterpret_cast<uint4*>(out + e0);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) dst[k] = nf4_dequant_word(cw[k], t);
+    } else {
+      for (int64_t e = e0; e < numel; ++e) {
+        const uint8_t b = codes[e / 2];
+        const uint32_t j = (e & 1) ? (b & 0xF) : (b >> 4);
+        const float v = __fmul_rn(nf4_code(j), a);
+        __nv_bfloat16 h = __float2bfloat16_rn(v);
+        out[e] = *reinterpret_cast<uint16_t*>(&h);
+      }
+    }
+  }
+}
+
+qlora_status launch_dequantize(const uint8_t* codes, const float* absmax, const uint8_t* absmax_q,
+                               const float* absmax2, bool dq, int64_t numel, uint16_t* out, cudaStream_t s) {
+  const int64_t n_units = (numel + 31) / 32;
+  if (n_units == 0) return QLORA_OK;
+  const int64_t blocks = std::min<int64_t>((n_units + 255) / 256, int64_t(num_sms()) * 16);
+  nf4_dequantize_kernel<<<unsigned(blocks), 256, 0, s>>>(codes, absmax, absmax_q, absmax2, dq ? 1 : 0, numel, out);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// ------------------------------------------------------- expanded GEMM scales
+
+__global__ void expand_scales_kernel(const float* __restrict__ absmax, const uint8_t* __restrict__ absmax_q,
+                                     const float* __restrict__ absmax2, int dq, int64_t out, int64_t nbr,
+                                     float* __restrict__ scales_t) {
+  // scales_t[kb][o] = scale of block (o, kb)
+  __shared__ float tile[32][33];
+  const int64_t o0 = int64_t(blockIdx.x) * 32, k0 = int64_t(blockIdx.y) * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  for (int j = ty; j < 32; j += 8) {
+    const int64_t o = o0 + j, kb = k0 + tx;
+    float v = 0.f;
+    if (o < out && kb < nbr) v = block_scale(o * nbr + kb, absmax, absmax_q, absmax2, dq != 0);
+    tile[j][tx] = v;
+  }
+  __syncthreads();
+  for (int j = ty; j < 32; j += 8) {
+    const int64_t kb = k0 + j, o = o0 + tx;
+    if (o < out && kb < nbr) scales_t[kb * out + o] = tile[tx][j];
+  }
+}
+
+qlora_status launch_expand_scales(const uint8_t*, const float* absmax, const uint8_t* absmax_q,
+                                  const float* absmax2, bool dq, int64_t out, int64_t in, float* scales_t,
+                                  cudaStream_t s) {
+  const int64_t nbr = in / kBlock;
+  dim3 grid(unsigned((out + 31) / 32), unsigned((nbr + 31) / 32));
+  expand_scales_kernel<<<grid, dim3(32, 8), 0, s>>>(absmax, absmax_q, absmax2, dq ? 1 : 0, out, nbr, scales_t);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------- LoRA prep / reduce
+
+__global__ void scale_lora_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t cols, float scale,
+                                  int transpose, uint16_t* __restrict__ dst) {
+  const int64_t n = rows * cols;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    // non-transposed: dst[i] = s*src[i]; transposed: src is rows x cols, dst is cols x rows
+    int64_t d = i;
+    if (transpose) {
+      const int64_t rr = i / cols, cc = i % cols;
+      d = cc * rows + rr;
+    }
+    const float v = __fmul_rn(__uint_as_float(uint32_t(src[i]) << 16), scale);
+    __nv_bfloat16 h = __float2bfloat16_rn(v);
+    dst[d] = *reinterpret_cast<uint16_t*>(&h);
+  }
+}
+
+qlora_status launch_scale_lora(const uint16_t* src, int64_t rows, int64_t cols, float scale, bool transpose,
+                               uint16_t* dst, cudaStream_t s) {
+  const int64_t n = rows * cols;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 4096);
+  scale_lora_kernel<<<unsigned(blocks), 256, 0, s>>>(src, rows, cols, scale, transpose ? 1 : 0, dst);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+__global__ void reduce_bf16_kernel(const float* __restrict__ part, int splits, int64_t n, uint16_t* __restrict__ out) {
+  // 4 consecutive elements per thread
+  const int64_t n4 = n / 4;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n4; i += int64_t(gridDim.x) * blockDim.x) {
+    float4 acc = __ldg(reinterpret_cast<const float4*>(part) + i);
+    for (int p = 1; p < splits; ++p) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(part + p * n) + i);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    uint2 o;
+    o.x = pack_bf16x2(acc.x, acc.y);
+    o.y = pack_bf16x2(acc.z, acc.w);
+    reinterpret_cast<uint2*>(out)[i] = o;
+  }
+}
+
+qlora_status launch_reduce_bf16(const float* part, int splits, int64_t rows, int64_t cols, uint16_t* out,
+                                cudaStream_t s) {
+  const int64_t n = rows * cols;  // cols % 8 == 0 by the shape rules
+  const int64_t blocks = std::min<int64_t>((n / 4 + 255) / 256, int64_t(num_sms()) * 8);
+  reduce_bf16_kernel<<<unsigned(std::max<int64_t>(blocks, 1)), 256, 0, s>>>(part, splits, n, out);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+__global__ void reduce_f32_kernel(const float* __restrict__ part, int splits, int64_t rows, int64_t cols,
+                                  float scale, int transpose, float* __restrict__ out) {
+  const int64_t n = rows * cols;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    float acc = part[i];
+    for (int p = 1; p < splits; ++p) acc += part[p * n + i];
+    acc = __fmul_rn(acc, scale);
+    if (transpose) {
+      const int64_t rr = i / cols, cc = i % cols;
+      out[cc * rows + rr] = acc;
+    } else {
+      out[i] = acc;
+    }
+  }
+}
+
+qlora_status launch_reduce_f32(const float* part, int splits, int64_t rows, int64_t cols, float scale,
+                               bool transpose, float* out, cudaStream_t s) {
+  const int64_t n = rows * cols;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, int64_t(num_sms()) * 8);
+  reduce_f32_kernel<<<unsigned(std::max<int64_t>(blocks, 1)), 256, 0, s>>>(part, splits, rows, cols, scale,
+                                                                          transpose ? 1 : 0, out);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+}  // namespace qlb

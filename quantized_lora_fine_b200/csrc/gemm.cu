@@ -1,0 +1,439 @@
+// tcgen05 GEMM engine for sm_100a.
+//
+//   D[M x N] = A[M x K] * B[N x K]^T  (+ A_ext[M x r] * B_ext[N x r]^T)
+//
+// Tiles of 128 x BN x 64 (bf16 in, fp32 accumulate in tensor memory), a
+// persistent grid, warp-specialised roles:
+//   warp 0      TMA producer (one elected lane): A tiles, and either B tiles
+//               (bf16 operand) or packed NF4 codes + expanded scales
+//   warp 1      TMEM allocator and MMA issuer (one elected lane)
+//   warps 2-5   epilogue: tcgen05.ld -> registers -> global (bf16 or fp32)
+//   warps 6-13  (NF4 operand only) dequantizers: packed codes in shared memory
+//               -> bf16 B tile in the 128-byte-swizzled UMMA layout, through a
+//               per-block 16-entry product table (prmt byte lookups)
+// Stage hand-off uses mbarriers; MMA completion is signalled with
+// tcgen05.commit; the accumulator is double-buffered in TMEM so that the
+// epilogue of one tile overlaps the mainloop of the next.
+//
+// Operand layouts in shared memory (all 128-byte swizzle, 1024-byte aligned):
+//   K-major  : rows x 64 elements (128 B per row); 8-row groups 1024 B apart.
+//   MN-major : [MN/64 chunks][64 K rows][64 elements]; chunk stride 8 KB.
+// The LoRA term is appended as extra K steps whose A and B tiles are loaded by
+// TMA (T or U, and the scaled L2^T or L1), zero-filled beyond r.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "gemm.cuh"
+#include "internal.cuh"
+#include "nf4_device.cuh"
+#include "ptx.cuh"
+
+namespace qlb {
+
+// --------------------------------------------------------------- config
+
+template <int BN_, bool A_MN_, bool B_MN_, bool NF4_, bool OUT_F32_, int STAGES_>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64, BN = BN_;
+  static constexpr bool A_MN = A_MN_, B_MN = B_MN_, NF4 = NF4_, OUT_F32 = OUT_F32_;
+  static constexpr int STAGES = STAGES_;
+  static constexpr int kA = BM * BK * 2;
+  static constexpr int kB = BN * BK * 2;
+  static constexpr int kCodes = NF4 ? BN * BK / 2 : 0;
+  static constexpr int kScales = NF4 ? BN * 4 : 0;  // fwd: BN scales; dX: 64 rows x BN/64 blocks
+  static constexpr int kCodesOff = kA + kB;
+  static constexpr int kScalesOff = kCodesOff + ((kCodes + 1023) / 1024) * 1024;
+  static constexpr int kStage = kScalesOff + ((kScales + 1023) / 1024) * 1024;
+  static constexpr int kDequantWarps = NF4 ? 8 : 0;
+  static constexpr int kThreads = (6 + kDequantWarps) * 32;
+  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                   : (2 * BN <= 256) ? 256 : 512;
+  static constexpr int kBarBytes = 8 * (3 * STAGES + 5) + 16;
+  static constexpr int kSmem = STAGES * kStage + kBarBytes + 1024;  // + alignment slack
+  static_assert(BN % 16 == 0 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0, N <= 256");
+  static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are 64-element chunks");
+  static_assert(!NF4 || BN == 256, "dequant mapping assumes BN = 256");
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+// --------------------------------------------------------------- tile decode
+
+struct TileInfo {
+  int m0, n0, split, kb, ke;  // main k-step range [kb, ke)
+  int n_ext;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int t) {
+  TileInfo ti;
+  const int per_split = p.tiles_m * p.tiles_n;
+  ti.split = t / per_split;
+  const int r = t - ti.split * per_split;
+  const int mb = r / p.tiles_n, nb = r - mb * p.tiles_n;
+  ti.m0 = mb * 128;
+  ti.n0 = nb * p.bn;
+  ti.kb = ti.split * p.ksteps_per_split;
+  ti.ke = min(p.num_k_main, ti.kb + p.ksteps_per_split);
+  ti.n_ext = (p.splits == 1) ? p.num_k_ext : 0;
+  return ti;
+}
+
+// --------------------------------------------------------------- dequant stage
+
+// fwd (K-major B): thread t owns B row n = t (one 64-element block per stage).
+// dX  (MN-major B): thread t owns K row (t % 64) and 64-column chunk (t / 64).
+template <bool B_MN>
+__device__ __forceinline__ void dequant_stage(uint32_t t, const uint8_t* codes_s, const float* scales_s,
+                                              uint32_t b_tile) {
+  uint32_t row, chunk, code_off0, code_off1;
+  float a;
+  if constexpr (!B_MN) {
+    row = t;
+    chunk = 0;
+    code_off0 = t * 32;
+    code_off1 = t * 32 + 16;
+    a = scales_s[t];
+  } else {
+    row = t & 63u;
+    chunk = t >> 6;
+    const uint32_t sw = row & 7u;
+    code_off0 = row * 128 + (((2 * chunk) ^ sw) << 4);
+    code_off1 = row * 128 + (((2 * chunk + 1) ^ sw) << 4);
+    a = scales_s[chunk * 64 + row];
+  }
+  const uint4 c0 = *reinterpret_cast<const uint4*>(codes_s + code_off0);
+  const uint4 c1 = *reinterpret_cast<const uint4*>(codes_s + code_off1);
+  const NF4Lut lut = nf4_make_lut(a);
+  const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const uint32_t sw = row & 7u;
+  const uint32_t row_base = b_tile + (B_MN ? chunk * 8192u : 0u) + (row >> 3) * 1024u + sw * 128u;
+#pragma unroll
+  for (uint32_t c = 0; c < 8; ++c) {
+    const uint4 v = nf4_dequant_word(words[c], lut);
+    const uint32_t addr = row_base + ((c ^ sw) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+  }
+}
+
+// --------------------------------------------------------------- kernel
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmScales,
+                   const __grid_constant__ CUtensorMap tmAx, const __grid_constant__ CUtensorMap tmBx,
+                   const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::kStage);
+  const uint32_t bar_base = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto deq_bar = [&](int s) { return bar_base + 8u * (C::STAGES + s); };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (2 * C::STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar_base + 8u * (3 * C::STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar_base + 8u * (3 * C::STAGES + 2 + a); };
+  const uint32_t drain_bar = bar_base + 8u * (3 * C::STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 5);
+
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(deq_bar(s), C::kDequantWarps > 0 ? C::kDequantWarps : 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbarrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = p.tiles_m * p.tiles_n * p.splits;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      if (!C::NF4) tma_prefetch_desc(&tmB);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile(p, t);
+        const int nsteps = (ti.ke - ti.kb) + ti.n_ext;
+        for (int j = 0; j < nsteps; ++j, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          if (!mbar_wait(empty_bar(s), ph ^ 1u)) { set_status(p.status, QLORA_ERR_TIMEOUT); ok = false; break; }
+          const uint32_t st = smem_base + s * C::kStage;
+          const uint32_t a_s = st, b_s = st + C::kA;
+          if (j < ti.ke - ti.kb) {
+            const int ks = ti.kb + j;
+            const int k0 = ks * 64;
+            const uint32_t bytes = C::kA + (C::NF4 ? (C::kCodes + C::kScales) : C::kB);
+            mbar_arrive_expect_tx(full_bar(s), bytes);
+            if constexpr (!C::A_MN) {
+              tma_load_2d(a_s, &tmA, full_bar(s), k0, ti.m0);
+            } else {
+              tma_load_2d(a_s, &tmA, full_bar(s), ti.m0, k0);
+              tma_load_2d(a_s + 8192, &tmA, full_bar(s), ti.m0 + 64, k0);
+            }
+            if constexpr (C::NF4) {
+              if constexpr (!C::B_MN) {
+                tma_load_2d(st + C::kCodesOff, &tmCodes, full_bar(s), k0 / 2, ti.n0);
+                tma_load_2d(st + C::kScalesOff, &tmScales, full_bar(s), ti.n0, ks);
+              } else {
+                tma_load_2d(st + C::kCodesOff, &tmCodes, full_bar(s), ti.n0 / 2, k0);
+                tma_load_2d(st + C::kScalesOff, &tmScales, full_bar(s), k0, ti.n0 / 64);
+              }
+            } else {
+              if constexpr (!C::B_MN) {
+                tma_load_2d(b_s, &tmB, full_bar(s), k0, ti.n0);
+              } else {
+#pragma unroll
+                for (int c = 0; c < C::BN / 64; ++c) tma_load_2d(b_s + c * 8192, &tmB, full_bar(s), ti.n0 + 64 * c, k0);
+              }
+            }
+          } else {
+            const int kx = (j - (ti.ke - ti.kb)) * 64;
+            mbar_arrive_expect_tx(full_bar(s), C::kA + C::kB);
+            tma_load_2d(a_s, &tmAx, full_bar(s), kx, ti.m0);
+            tma_load_2d(b_s, &tmBx, full_bar(s), kx, ti.n0);
+          }
+        }
+      }
+      // Do not leave while copies this thread issued may still be landing.
+      if (it > 0) {
+        const uint32_t last = it - 1;
+        for (int k = 0; k < C::STAGES && k <= int(last); ++k) {
+          const uint32_t i2 = last - k;
+          mbar_wait(full_bar(i2 % C::STAGES), (i2 / C::STAGES) & 1u, 100000000ull);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_main = make_idesc_bf16(128, C::BN, C::A_MN ? 1 : 0, C::B_MN ? 1 : 0);
+      constexpr uint32_t idesc_ext = make_idesc_bf16(128, C::BN, 0, 0);
+      // K advance per 16-element MMA step: 32 B inside a K-major row; 2 x 8-row
+      // groups (2048 B) in an MN-major tile.
+      constexpr uint32_t a_adv = C::A_MN ? 2048u : 32u;
+      constexpr uint32_t b_adv = C::B_MN ? 2048u : 32u;
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tcount) {
+        const TileInfo ti = decode_tile(p, t);
+        const int nsteps = (ti.ke - ti.kb) + ti.n_ext;
+        const uint32_t acc = tcount & 1u, tph = (tcount >> 1) & 1u;
+        if (!mbar_wait(tempty_bar(acc), tph ^ 1u)) { set_status(p.status, QLORA_ERR_TIMEOUT); ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * C::BN;
+        for (int j = 0; j < nsteps; ++j, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          if (!mbar_wait(full_bar(s), ph)) { set_status(p.status, QLORA_ERR_TIMEOUT); ok = false; break; }
+          if (C::NF4 && !mbar_wait(deq_bar(s), ph)) { set_status(p.status, QLORA_ERR_TIMEOUT); ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = smem_base + s * C::kStage;
+          const bool ext = j >= ti.ke - ti.kb;
+          const uint32_t a_lbo = (!ext && C::A_MN) ? 8192u : 16u;
+          const uint32_t b_lbo = (!ext && C::B_MN) ? 8192u : 16u;
+          const uint64_t adesc = make_smem_desc(st, a_lbo, 1024u, kSwizzle128B);
+          const uint64_t bdesc = make_smem_desc(st + C::kA, b_lbo, 1024u, kSwizzle128B);
+          const uint32_t aadv = ext ? 32u : a_adv, badv = ext ? 32u : b_adv;
+          const uint32_t idesc = ext ? idesc_ext : idesc_main;
+#pragma unroll
+          for (uint32_t kk = 0; kk < 4; ++kk) {
+            tc_mma_bf16(d_tmem, adesc + uint64_t((kk * aadv) >> 4), bdesc + uint64_t((kk * badv) >> 4), idesc,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(empty_bar(s));
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+      }
+      // all MMAs issued by this thread are complete once drain_bar flips
+      tc_commit(drain_bar);
+      mbar_wait(drain_bar, 0, 100000000ull);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t q = warp & 3u;
+    const uint32_t row = q * 32 + lane;
+    uint32_t tcount = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tcount) {
+      const TileInfo ti = decode_tile(p, t);
+      const uint32_t acc = tcount & 1u, tph = (tcount >> 1) & 1u;
+      if (!mbar_wait(tfull_bar(acc), tph)) { set_status(p.status, QLORA_ERR_TIMEOUT); break; }
+      tc_fence_after();
+      const int grow = ti.m0 + int(row);
+      const uint32_t tbase = tmem_base + ((q * 32u) << 16) + acc * C::BN;
+#pragma unroll 1
+      for (int c = 0; c < C::BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + c * 32, v);
+        tmem_ld_wait();
+        const int col0 = ti.n0 + c * 32;
+        if (grow < p.M) {
+          if constexpr (C::OUT_F32) {
+            float* dst = reinterpret_cast<float*>(p.out) + int64_t(ti.split) * p.split_stride +
+                         int64_t(grow) * p.ld_out + col0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              if (col0 + 4 * i + 4 <= p.N)
+                reinterpret_cast<float4*>(dst)[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                                __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            }
+          } else {
+            uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) + int64_t(grow) * p.ld_out + col0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (col0 + 8 * i + 8 <= p.N) {
+                uint4 o;
+                o.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+                o.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+                o.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+                o.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+                reinterpret_cast<uint4*>(dst)[i] = o;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+    }
+  } else {
+    // ------------------------------------------------------------ dequantizers
+    if constexpr (C::NF4) {
+      const uint32_t dt = threadIdx.x - 192;
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile(p, t);
+        const int nsteps = (ti.ke - ti.kb) + ti.n_ext;
+        for (int j = 0; j < nsteps; ++j, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          if (!mbar_wait(full_bar(s), ph)) { set_status(p.status, QLORA_ERR_TIMEOUT); ok = false; break; }
+          if (j < ti.ke - ti.kb) {
+            uint8_t* st = smem + s * C::kStage;
+            dequant_stage<C::B_MN>(dt, st + C::kCodesOff, reinterpret_cast<const float*>(st + C::kScalesOff),
+                                   smem_base + s * C::kStage + C::kA);
+            fence_proxy_async_smem();
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(deq_bar(s));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// --------------------------------------------------------------- host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+bool make_tmap_2d(CUtensorMap* m, const void* base, TmapType type, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (type == TmapType::U8) dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if (type == TmapType::F32) dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <class C>
+static qlora_status launch_cfg(const GemmOperands& o, GemmParams p, int ctas_per_sm, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(tc_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+        cudaSuccess)
+      return QLORA_ERR_CUDA;
+    attr_set = true;
+  }
+  p.bn = C::BN;
+  const int num_tiles = p.tiles_m * p.tiles_n * p.splits;
+  const int grid = std::max(1, std::min(num_tiles, num_sms() * ctas_per_sm));
+  tc_gemm_kernel<C><<<grid, C::kThreads, C::kSmem, s>>>(o.A, o.B, o.codes, o.scales, o.Ax, o.Bx, p);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status launch_gemm(GemmKind kind, int bn, const GemmOperands& o, const GemmParams& p, cudaStream_t s) {
+  switch (kind) {
+    case GemmKind::FwdNF4: return launch_cfg<GemmCfg<256, false, false, true, false, 3>>(o, p, 1, s);
+    case GemmKind::DxNF4: return launch_cfg<GemmCfg<256, false, true, true, false, 3>>(o, p, 1, s);
+    case GemmKind::FwdBF16: return launch_cfg<GemmCfg<256, false, false, false, false, 4>>(o, p, 1, s);
+    case GemmKind::DxBF16: return launch_cfg<GemmCfg<256, false, true, false, false, 4>>(o, p, 1, s);
+    case GemmKind::ThinKK:  // A K-major, B K-major, fp32 partials
+      if (bn <= 64) return launch_cfg<GemmCfg<64, false, false, false, true, 4>>(o, p, 2, s);
+      if (bn <= 128) return launch_cfg<GemmCfg<128, false, false, false, true, 4>>(o, p, 2, s);
+      return launch_cfg<GemmCfg<256, false, false, false, true, 4>>(o, p, 1, s);
+    case GemmKind::ThinKM:  // A K-major, B MN-major
+      if (bn <= 64) return launch_cfg<GemmCfg<64, false, true, false, true, 4>>(o, p, 2, s);
+      if (bn <= 128) return launch_cfg<GemmCfg<128, false, true, false, true, 4>>(o, p, 2, s);
+      return launch_cfg<GemmCfg<256, false, true, false, true, 4>>(o, p, 1, s);
+    case GemmKind::ThinMM:  // A MN-major, B MN-major
+      if (bn <= 64) return launch_cfg<GemmCfg<64, true, true, false, true, 4>>(o, p, 2, s);
+      if (bn <= 128) return launch_cfg<GemmCfg<128, true, true, false, true, 4>>(o, p, 2, s);
+      return launch_cfg<GemmCfg<256, true, true, false, true, 4>>(o, p, 1, s);
+  }
+  return QLORA_ERR_UNSUPPORTED;
+}
+
+}  // namespace qlb

@@ -1,0 +1,49 @@
+// Internal declarations shared by the translation units of libqlora_b200.so.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/qlora_b200.h"
+
+namespace qlb {
+
+constexpr int kBlock = 64;        // NF4 block (elements per absmax)
+constexpr int kDQBlock = 256;     // absmax values per second-level scale
+constexpr size_t kStatusBytes = 256;
+
+__device__ __forceinline__ void set_status(int* st, int code) {
+  if (st) atomicCAS(st, 0, code);
+}
+
+// ---- codec.cu
+qlora_status launch_quantize(const void* W, int w_dtype, int64_t numel, bool dq, uint8_t* codes, float* absmax,
+                             uint8_t* absmax_q, float* absmax2, int* status, cudaStream_t s);
+qlora_status launch_dequantize(const uint8_t* codes, const float* absmax, const uint8_t* absmax_q,
+                               const float* absmax2, bool dq, int64_t numel, uint16_t* out, cudaStream_t s);
+// Scales of an out x in NF4 weight, expanded to fp32 and laid out [in/64][out].
+qlora_status launch_expand_scales(const uint8_t* unused, const float* absmax, const uint8_t* absmax_q,
+                                  const float* absmax2, bool dq, int64_t out, int64_t in, float* scales_t,
+                                  cudaStream_t s);
+// dst[i][q] = bf16(s * src[i][q]), rows x r  (transpose = 0)
+// dst[n][q] = bf16(s * src[q][n]), src r x cols (transpose = 1)
+qlora_status launch_scale_lora(const uint16_t* src, int64_t rows, int64_t cols, float scale, bool transpose,
+                               uint16_t* dst, cudaStream_t s);
+// out[m][c] = bf16(sum_p part[p][m][c])
+qlora_status launch_reduce_bf16(const float* part, int splits, int64_t rows, int64_t cols, uint16_t* out,
+                                cudaStream_t s);
+// out = scale * sum_p part[p]; transpose: part is [rows x cols], out is [cols x rows]
+qlora_status launch_reduce_f32(const float* part, int splits, int64_t rows, int64_t cols, float scale,
+                               bool transpose, float* out, cudaStream_t s);
+
+// ---- layer_error.cu
+size_t layer_error_ws_bytes(int n_layers, const int64_t* numel);
+qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
+                                     int K, double* err, int32_t* order, uint8_t* keep, void* ws, size_t ws_bytes,
+                                     int* status, cudaStream_t s);
+
+// ---- gemm.cu
+int num_sms();
+// Operand descriptions for the tcgen05 GEMM engine.
+struct GemmPlan;
+}  // namespace qlb

@@ -1,0 +1,94 @@
+// Device-side NF4 helpers shared by the codec, error-pass and GEMM kernels.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "nf4_constants.cuh"
+
+namespace qlb {
+
+__device__ __forceinline__ float nf4_code(int j) { return __uint_as_float(kNF4CodeBits[j]); }
+
+// Index of the nearest code for a normalised value n: #{j : n > m_j}.
+__device__ __forceinline__ uint32_t nf4_index(float n) {
+  uint32_t idx = 0;
+#pragma unroll
+  for (int j = 0; j < 15; ++j) idx += (n > __uint_as_float(kNF4MidBits[j])) ? 1u : 0u;
+  return idx;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t bitselect(uint32_t a, uint32_t b, uint32_t m) {
+  // (a & ~m) | (b & m); lut 0xCA = (x & y) | (~x & z) with x = m, y = b, z = a
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xCA;" : "=r"(d) : "r"(m), "r"(b), "r"(a));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Per-block dequantization table: the 16 products bf16_rn(fp32_rn(c_j * a)) split
+// into a low-byte table (lo[0..3], byte j = low byte of entry j) and a high-byte
+// table (hi[0..3]).
+struct NF4Lut {
+  uint32_t lo[4];
+  uint32_t hi[4];
+};
+
+__device__ __forceinline__ NF4Lut nf4_make_lut(float a) {
+  uint32_t p[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) p[j] = pack_bf16x2(nf4_code(2 * j) * a, nf4_code(2 * j + 1) * a);
+  NF4Lut t;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    t.lo[q] = prmt(p[2 * q], p[2 * q + 1], 0x6420u);
+    t.hi[q] = prmt(p[2 * q], p[2 * q + 1], 0x7531u);
+  }
+  return t;
+}
+
+// Dequantize 8 packed codes (one little-endian 32-bit word = 4 code bytes; byte k
+// holds element 2k in its high nibble) into 8 bf16 values (a 16-byte chunk, element
+// 0 in the lowest half-word).
+__device__ __forceinline__ uint4 nf4_dequant_word(uint32_t w, const NF4Lut& t) {
+  const uint32_t s = w & 0x77777777u;                                   // table index within a half
+  const uint32_t sm = (w & 0x88888888u) | ((w >> 3) & 0x11111111u);      // sign-replicate selector
+  uint32_t out[4];
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const uint32_t sg = g ? (s >> 16) : s;
+    const uint32_t mg = g ? (sm >> 16) : sm;
+    const uint32_t m = prmt(0x00008000u, 0u, mg);   // byte i = 0xFF iff nibble i >= 8
+    const uint32_t lo = bitselect(prmt(t.lo[0], t.lo[1], sg), prmt(t.lo[2], t.lo[3], sg), m);
+    const uint32_t hi = bitselect(prmt(t.hi[0], t.hi[1], sg), prmt(t.hi[2], t.hi[3], sg), m);
+    // nibble order within a byte pair is (odd, even); reorder to (even, odd)
+    out[2 * g] = prmt(lo, hi, 0x4051u);
+    out[2 * g + 1] = prmt(lo, hi, 0x6273u);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// fp32 value of an E4M3 scale byte (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint8_t q) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(q), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+__device__ __forceinline__ uint8_t f32_to_e4m3_satfinite(float x) {
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+
+}  // namespace qlb

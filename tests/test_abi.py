@@ -1,0 +1,89 @@
+"""The C ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before touching a device (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_lora_fine_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*([a-z][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_five_operations():
+    names = declared_functions()
+    for op in ("nf4_quantize", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "nf4_layer_error_rank"):
+        assert op in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(_lib.SIGNATURES), set(names) - set(_lib.SIGNATURES)
+
+
+def test_status_strings(lib):
+    assert lib.qlora_status_str(0) == b"ok"
+    assert b"time" in lib.qlora_status_str(9)
+
+
+def test_workspace_sizes_are_host_only(lib):
+    assert lib.qlora_fwd_workspace_size(8192, 4096, 4096, 16) > 4096 * 64 * 4
+    assert lib.qlora_bwd_workspace_size(8192, 4096, 4096, 16) > 0
+    assert lib.qlora_fwd_workspace_size(0, 4096, 4096, 16) == 0
+    n = (ctypes.c_int64 * 2)(4096 * 4096, 11008 * 4096)
+    assert lib.nf4_layer_error_rank_workspace_size(2, n) > 0
+
+
+def test_host_validation_before_any_launch(lib):
+    q = _lib.NF4QConfig(64, 0, 256)
+    # NULL weight pointer
+    assert lib.nf4_quantize(None, 0, 64, 64, q, None, None, None, None, None, 0, None) == 1
+    # bad dtype
+    assert lib.nf4_quantize(None, 7, 64, 64, q, None, None, None, None, None, 0, None) == 4
+    # unsupported blocksize
+    assert lib.nf4_quantize(None, 0, 64, 64, _lib.NF4QConfig(32, 0, 256), None, None, None, None, None, 0, None) == 5
+    # linear: bad shapes are refused on the host
+    w = _lib.QLoraWeight()
+    w.out, w.in_ = 4096, 1000
+    w.q = q
+    assert lib.qlora_linear_fwd(ctypes.byref(w), None, 8, None, None, 16, 2.0, None, None, None, 0, None) == 2
+    w.in_ = 4096
+    assert lib.qlora_linear_fwd(ctypes.byref(w), None, 8, None, None, 12, 2.0, None, None, None, 0, None) == 2
+    # missing codes
+    assert lib.qlora_linear_fwd(ctypes.byref(w), None, 8, None, None, 16, 2.0, None, None, None, 0, None) == 1
+    # misaligned weight pointer
+    w.codes = 0x1001
+    w.absmax = 0x2000
+    assert lib.qlora_linear_fwd(ctypes.byref(w), None, 8, None, None, 16, 2.0, None, None, None, 0, None) == 3
+    # layer error: K out of range, numel not a multiple of 64
+    ptrs = (ctypes.c_void_p * 1)(0x1000)
+    n = (ctypes.c_int64 * 1)(100)
+    assert lib.nf4_layer_error_rank(1, ptrs, n, 0, q, 2, None, None, None, None, 0, None) == 2
+    assert lib.nf4_layer_error_rank(1, ptrs, n, 0, q, 1, 0x10, 0x10, 0x10, None, 0, None) == 2
+
+
+def test_product_path_refuses_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(RuntimeError):
+        _lib.load(str(tmp_path / "missing.so"))

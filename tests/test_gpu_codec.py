@@ -1,0 +1,82 @@
+"""GPU parity: NF4 quantize / dequantize are bit-exact with the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import nf4
+from quantized_lora_fine_b200 import api, synth
+from tests.gpu_helpers import bits
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_quant(W: torch.Tensor, dq: bool):
+    qw = nf4.quantize(nf4.f32_from_bf16_bits(bits(W)).reshape(W.shape), double_quant=dq)
+    g = api.quantize(W.cuda(), double_quant=dq, keep_absmax=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(g.codes.cpu().numpy(), qw["codes"]), "codes differ"
+    assert np.array_equal(g.absmax.cpu().numpy().view(np.uint32), qw["absmax"].view(np.uint32)), "absmax differ"
+    if dq:
+        assert np.array_equal(g.absmax_q.cpu().numpy(), qw["absmax_q"]), "absmax_q differ"
+        assert np.array_equal(g.absmax2.cpu().numpy().view(np.uint32), qw["absmax2"].view(np.uint32)), "absmax2 differ"
+    deq = api.dequantize(g)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(deq).reshape(-1), nf4.dequantize_bf16_bits(qw).reshape(-1)), "dequantized values differ"
+    assert api.status() == 0
+
+
+def test_quant_small_case(cuda_device):
+    d = synth.case_small().make()
+    _check_quant(d["W"], dq=False)
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_quant_q_proj_shape(cuda_device, dq):
+    W = synth.normal_bf16((4096, 4096), 0.02, 0, synth.STREAM_W)
+    _check_quant(W, dq)
+
+
+def test_quant_student_t_ragged_groups(cuda_device):
+    # 11008 x 256: 44032 blocks = 172 groups exactly; plus a shape whose last DQ group is partial
+    _check_quant(synth.student_t_bf16((11008, 256), 5.0, 0.02, 0, synth.STREAM_W), dq=True)
+    _check_quant(synth.student_t_bf16((300, 192), 3.0, 0.02, 1, synth.STREAM_W), dq=True)
+
+
+def test_quant_partial_tail_block(cuda_device):
+    W = synth.normal_bf16((7, 38), 0.5, 2, synth.STREAM_W)   # 266 elements: 4 full blocks + 10
+    _check_quant(W, dq=False)
+    _check_quant(W, dq=True)
+
+
+def test_quant_adversarial_blocks(cuda_device):
+    C = nf4.nf4_code_table()
+    mids = nf4.nf4_midpoints()
+    rows = []
+    rows.append(np.zeros(64, np.float32))                                   # all-zero block
+    r = np.zeros(64, np.float32); r[5] = 3.0; rows.append(r)                 # one non-zero
+    r = np.full(64, -0.0, np.float32); rows.append(r)                        # negative zeros
+    r = np.concatenate([[1.0], mids, -mids, C, np.nextafter(mids, 2), np.nextafter(mids, -2)]).astype(np.float32)
+    rows.append(np.resize(r, 64))
+    rows.append(np.resize(np.concatenate([[1.0], np.nextafter(mids, 2)]), 64).astype(np.float32))
+    r = (C[np.arange(64) % 16] * np.float32(0.75)).astype(np.float32); rows.append(r)
+    r = np.full(64, 2.0 ** -130, np.float32); r[0] = 2.0 ** -126; rows.append(r)   # subnormal range
+    r = np.linspace(-3e38, 3e38, 64).astype(np.float32); rows.append(r)            # huge
+    W32 = np.stack(rows)
+    Wb = synth.from_bf16_bits(nf4.bf16_bits_from_f32(W32))
+    _check_quant(Wb, dq=False)
+    _check_quant(Wb, dq=True)
+    # fp32 input path
+    qw = nf4.quantize(W32)
+    g = api.quantize(torch.from_numpy(W32).cuda(), double_quant=False)
+    assert np.array_equal(g.codes.cpu().numpy(), qw["codes"])
+
+
+def test_nonfinite_sets_status(cuda_device):
+    W = torch.zeros((4, 64), dtype=torch.bfloat16)
+    W[2, 7] = float("nan")
+    ws = api.Workspace.get(256, torch.device("cuda:0"))
+    api.reset_status(ws)
+    api.quantize(W.cuda())
+    assert api.read_status(ws) == 8
+    api.reset_status(ws)
+    assert api.read_status(ws) == 0

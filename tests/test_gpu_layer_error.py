@@ -1,0 +1,52 @@
+"""GPU parity: AQLoRA per-layer NF4 error (within 1e-6 relative) and ranks
+(bit-exact) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import layer_error
+from quantized_lora_fine_b200 import api, synth
+from tests.gpu_helpers import bits
+
+pytestmark = pytest.mark.gpu
+
+
+def _compare(Ws, K, dq):
+    ref_err = np.array([layer_error.layer_error(bits(W), dq) for W in Ws])
+    ref_order = layer_error.rank_layers(ref_err)
+    ref_keep = layer_error.keep_mask(ref_order, K)
+    err, order, keep = api.layer_error_rank([W.cuda() for W in Ws], K, double_quant=dq)
+    torch.cuda.synchronize()
+    err = err.cpu().numpy()
+    nz = ref_err > 0
+    assert np.all(np.abs(err[nz] - ref_err[nz]) <= 1e-6 * ref_err[nz])
+    assert np.all(err[~nz] == 0)
+    assert np.array_equal(order.cpu().numpy(), ref_order)
+    assert np.array_equal(keep.cpu().numpy(), ref_keep)
+    assert api.status() == 0
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_small_stack(cuda_device, dq):
+    mats = synth.stack_matrices(n_layers=4, linears=(("a", 256, 512), ("b", 512, 256), ("c", 64, 320)))
+    Ws = [synth.stack_weight(m) for m in mats]
+    _compare(Ws, K=5, dq=dq)
+
+
+def test_degenerate_layers(cuda_device):
+    Ws = [torch.zeros((64, 64), dtype=torch.bfloat16),
+          synth.normal_bf16((64, 128), 0.02, 0, 1, 0),
+          synth.normal_bf16((64, 128), 0.02, 0, 1, 0),   # exact duplicate: tie resolved by index
+          synth.student_t_bf16((128, 64), 3.0, 0.01, 0, 1, 1)]
+    _compare(Ws, K=0, dq=False)
+    _compare(Ws, K=4, dq=False)
+    _compare(Ws, K=2, dq=True)
+
+
+def test_llama_stack_sampled_layers(cuda_device):
+    """A few full-size matrices of the 32-layer Llama-7B-shaped stack (per-layer
+    Student-t with nu in [3,30], scale in [0.005,0.05]); K = 3."""
+    mats = synth.stack_matrices()
+    pick = [mats[i] for i in (0, 4, 6, 100, 223)]
+    Ws = [synth.stack_weight(m) for m in pick]
+    _compare(Ws, K=3, dq=False)

@@ -1,0 +1,104 @@
+"""GPU parity: NF4-LoRA linear forward / backward against the fp64 oracle."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lora
+from quantized_lora_fine_b200 import api, synth
+from tests.gpu_helpers import assert_close, f64_of_bf16, gpu_case, oracle_qweight, oracle_what
+
+pytestmark = pytest.mark.gpu
+
+
+def run_and_compare(case: synth.LinearCase, protected=False, rows=None, need_dX=True, save_T=True):
+    d = case.make()
+    s = case.scale
+    if protected:
+        What = f64_of_bf16(d["W"])
+    else:
+        What = oracle_what(oracle_qweight(d["W"], case.double_quant))
+    X, L1, L2, dY = (f64_of_bf16(d[k]) for k in ("X", "L1", "L2", "dY"))
+    g, w = gpu_case(d, case.double_quant, protected)
+    Y, T = api.linear_fwd(w, g["X"], g["L1"], g["L2"], s, save_T=save_T)
+    dX, dL1, dL2 = api.linear_bwd(w, g["X"], g["dY"], g["L1"], g["L2"], s, T=T, need_dX=need_dX)
+    torch.cuda.synchronize()
+    assert api.status() == 0
+    sel = np.arange(case.M) if rows is None else rows
+    Yref, Tref = lora.forward(X[sel], What, L1, L2, s)
+    out = {}
+    out["Y"] = assert_close(f64_of_bf16(Y)[sel], Yref, "Y")
+    if T is not None:
+        out["T"] = assert_close(f64_of_bf16(T)[sel], Tref, "T")
+    # gradients: dL1/dL2 reduce over all M rows; dX is checked on the sampled rows
+    T_full = X @ L1
+    U_full = dY @ L2.T
+    out["dL2"] = assert_close(dL2.cpu().numpy(), s * (T_full.T @ dY), "dL2")
+    out["dL1"] = assert_close(dL1.cpu().numpy(), s * (X.T @ U_full), "dL1")
+    if need_dX:
+        dXref = dY[sel] @ What + s * (U_full[sel] @ L1.T)
+        out["dX"] = assert_close(f64_of_bf16(dX)[sel], dXref, "dX")
+    else:
+        assert dX is None
+    return out
+
+
+def test_small_case_fwd_bwd(cuda_device):
+    run_and_compare(synth.case_small())
+
+
+@pytest.mark.parametrize("M", [1, 77, 200, 384])
+def test_ragged_token_counts(cuda_device, M):
+    run_and_compare(dataclasses.replace(synth.case_small(), M=M))
+
+
+@pytest.mark.parametrize("r", [8, 16, 32, 64, 128, 256])
+def test_ranks(cuda_device, r):
+    c = dataclasses.replace(synth.case_small(), M=256, out=768, inp=512, r=r, alpha=2.0 * r, double_quant=(r % 16 == 0))
+    run_and_compare(c)
+
+
+def test_protected_bf16_layer(cuda_device):
+    c = dataclasses.replace(synth.case_small(), M=300, out=512, inp=768, r=16, alpha=32.0)
+    run_and_compare(c, protected=True)
+
+
+def test_early_stop_and_recompute_T(cuda_device):
+    c = dataclasses.replace(synth.case_small(), M=192, r=16, alpha=32.0)
+    run_and_compare(c, need_dX=False, save_T=False)
+
+
+def test_zero_adapter_is_plain_gemm(cuda_device):
+    c = synth.case_small()
+    d = c.make()
+    d["L2"] = torch.zeros_like(d["L2"])
+    g, w = gpu_case(d, False)
+    Y, _ = api.linear_fwd(w, g["X"], g["L1"], g["L2"], c.scale)
+    What = oracle_what(oracle_qweight(d["W"], False))
+    assert_close(f64_of_bf16(Y), f64_of_bf16(d["X"]) @ What.T, "Y(L2=0)")
+
+
+def test_deterministic_gradients(cuda_device):
+    c = dataclasses.replace(synth.case_small(), M=512, r=16, alpha=32.0)
+    d = c.make()
+    g, w = gpu_case(d, False)
+    a = api.linear_bwd(w, g["X"], g["dY"], g["L1"], g["L2"], c.scale)
+    b = api.linear_bwd(w, g["X"], g["dY"], g["L1"], g["L2"], c.scale)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_q_proj_full_size_sampled(cuda_device):
+    """Llama-7B q_proj shape at full size (M=8192, 4096^2, DQ, r=16): Y and dX on
+    sampled rows, dL1 / dL2 over all rows."""
+    rows = np.random.default_rng(0).choice(8192, 192, replace=False)
+    rows.sort()
+    run_and_compare(synth.case_q_proj(), rows=rows)
+
+
+@pytest.mark.parametrize("idx", [0, 2])
+def test_mlp_full_size_sampled(cuda_device, idx):
+    rows = np.random.default_rng(1).choice(8192, 96, replace=False)
+    rows.sort()
+    run_and_compare(synth.cases_mlp()[idx], rows=rows)
