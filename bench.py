@@ -58,27 +58,43 @@ def config_dict(args, world):
 
 # --------------------------------------------------------------------------- CPU oracle leg
 
-def run_oracle_sample(rows: int, seed: int = 0):
-    """Times the oracle on the q_proj workload: full W quantize (+DQ) and error,
-    fwd+bwd on `rows` token rows. Returns (seconds, flops_counted, description)."""
+def run_oracle_sample(rows: int, out_rows: int = 4096, seed: int = 0):
+    """Times the oracle on a sub-problem of the q_proj workload: the first
+    `out_rows` output rows of W (all 4096 inputs) quantized with double
+    quantization, their NF4 error, and fwd+bwd on `rows` token rows.
+    Returns (seconds, fwd+bwd flops of the sub-problem, description)."""
     import numpy as np
     from oracle import layer_error, lora, nf4
     from quantized_lora_fine_b200 import synth
 
     case = synth.case_q_proj(seed=seed, M=rows)
     d = case.make()
-    Wb = synth.bf16_bits(d["W"])
-    X, L1, L2, dY = (nf4.f32_from_bf16_bits(synth.bf16_bits(d[k])).astype(np.float64) for k in ("X", "L1", "L2", "dY"))
+    W = d["W"][:out_rows].contiguous()
+    L2 = d["L2"][:, :out_rows].contiguous()
+    dYt = d["dY"][:, :out_rows].contiguous()
+    Wb = synth.bf16_bits(W)
+    X, L1, L2, dY = (nf4.f32_from_bf16_bits(synth.bf16_bits(t)).astype(np.float64) for t in (d["X"], d["L1"], L2, dYt))
     t0 = time.perf_counter()
-    qw = nf4.quantize(nf4.f32_from_bf16_bits(Wb).reshape(d["W"].shape), double_quant=True)
-    What = nf4.f32_from_bf16_bits(nf4.dequantize_bf16_bits(qw)).astype(np.float64).reshape(d["W"].shape)
+    qw = nf4.quantize(nf4.f32_from_bf16_bits(Wb).reshape(W.shape), double_quant=True)
+    What = nf4.f32_from_bf16_bits(nf4.dequantize_bf16_bits(qw)).astype(np.float64).reshape(W.shape)
     layer_error.layer_error(Wb, True)
-    Y, T = lora.forward(X, What, L1, L2, case.scale)
+    lora.forward(X, What, L1, L2, case.scale)
     lora.backward(X, What, L1, L2, dY, case.scale)
     dt = time.perf_counter() - t0
-    return dt, flops_fwd_bwd(rows, 4096, 4096, 16), (
-        f"oracle (numpy fp64) on {rows} of 8192 token rows: full 4096x4096 quantize+DQ, error pass, "
-        f"fwd+bwd; rate = fwd+bwd flops of the rows / wall time")
+    return dt, flops_fwd_bwd(rows, 4096, out_rows, 16), (
+        f"oracle (numpy fp64): {out_rows}x4096 slice of W quantized with DQ + its error pass + fwd+bwd on "
+        f"{rows} of 8192 token rows; rate = fwd+bwd flops of that sub-problem / wall time")
+
+
+def oracle_rate(min_seconds: float, rows: int, out_rows: int):
+    run_oracle_sample(16, 64)  # NF4 table cache
+    tot_t = tot_f = 0.0
+    desc = ""
+    while tot_t < min_seconds:
+        dt, fl, desc = run_oracle_sample(rows, out_rows)
+        tot_t += dt
+        tot_f += fl
+    return tot_f / tot_t / 1e12, tot_t, desc
 
 
 def cpu_threads():
@@ -95,15 +111,15 @@ def reference_main(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    rows = 256
+    rows, out_rows = 256, 512
+    run_oracle_sample(16, 64)  # NF4 table cache
     for _ in range(args.warmup):
-        pass  # the oracle has no warm state worth priming beyond its table cache
-    run_oracle_sample(16)  # builds the NF4 table cache
-    times = []
+        run_oracle_sample(rows, out_rows)
+    times, desc, fl = [], "", 0.0
     for _ in range(max(1, args.steps)):
-        dt, fl, desc = run_oracle_sample(rows)
+        dt, fl, desc = run_oracle_sample(rows, out_rows)
         times.append(dt)
-    dt = statistics.median(times)
+    dt = sum(times) / len(times)
     tf = fl / dt / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": tf, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
@@ -215,6 +231,9 @@ def gpu_main(args):
     torch.cuda.synchronize()
     assert api.status() == 0, "device status set during warm-up"
 
+    for e in prof:  # torch creates the CUDA event on first record
+        e.record(stream)
+    torch.cuda.synchronize()
     lib.qlora_profile_events(ctypes.c_void_p(prof[0].cuda_event), ctypes.c_void_p(prof[1].cuda_event),
                              ctypes.c_void_p(prof[2].cuda_event), ctypes.c_void_p(prof[3].cuda_event))
     step_ms, legs = [], {"quantize": [], "error_rank": [], "fwd": [], "bwd": [], "fwd_gemm": [], "dx_gemm": []}
@@ -268,7 +287,6 @@ def gpu_main(args):
     # dominant kernel = the longer of the two fused GEMMs
     dom = ("qlora_fwd_gemm (tc_gemm_kernel FwdNF4)", fwd_tf, med["fwd_gemm"]) if med["fwd_gemm"] >= med["dx_gemm"] \
         else ("qlora_bwd_dx_gemm (tc_gemm_kernel DxNF4)", dx_tf, med["dx_gemm"])
-    n = M * h  # placeholder not used
     numel = h * o
     quant_bytes = numel * 2 + numel // 2 + numel // 64 + 4 * (numel // 64 // 256)
     err_bytes = numel * 2
@@ -323,10 +341,9 @@ def gpu_main(args):
     # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        run_oracle_sample(16)
-        dt, cfl, desc = run_oracle_sample(args.cpu_rows)
-        cpu = {"value": cfl / dt / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": desc,
-               "seconds": dt}
+        rate, secs, desc = oracle_rate(args.cpu_seconds, args.cpu_rows, 4096)
+        cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": desc + f"; repeated for {secs:.1f} s", "seconds": secs}
 
     launches_per_step = 1 + 3 + 5 + 9
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -353,6 +370,7 @@ def main():
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
