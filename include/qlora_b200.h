@@ -205,6 +205,35 @@ qlora_status nf4_layer_error_rank(int32_t n_layers, const uint16_t* const* W_ptr
                                   double* err, int32_t* order, uint8_t* keep,
                                   void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
+/* Allocation-free variant of nf4_layer_error_rank (the paper has no
+ * counterpart; this is a convenience of the library).
+ *
+ * For callers that cannot allocate device memory at the point of the call:
+ * runtimes that hand out device memory only from a fixed pool fixed at start-up
+ * (so a workspace of this size may not exist), code running in a host callback
+ * or an allocator hook where cudaMalloc is not allowed, and pipelines that
+ * cannot afford cudaMalloc/cudaFree because those calls synchronize the device.
+ * It takes the same inputs and outputs as nf4_layer_error_rank and no
+ * workspace: the per-chunk partial sums live in a 16 MiB array inside the
+ * library (one per GPU, kept until the process exits).
+ *
+ * Limits and behaviour:
+ *   - at most 2^20 chunks of 16384 weights per call (sum over layers of
+ *     ceil(numel/16384) <= 1048576, about 1.7e10 weights); larger calls return
+ *     QLORA_ERR_SHAPE before any device work;
+ *   - the first call on a device looks up the array's device address (with that
+ *     device current) and caches it; make that first call before capturing any
+ *     stream;
+ *   - every call on a device uses the same array, so calls that overlap on the
+ *     GPU (different streams or host threads) race and must be serialized by the
+ *     caller; nothing needs clearing between calls;
+ *   - there is no device status word: a layer that contains NaN or +-Inf gets
+ *     err = NaN.
+ * Allocates no device memory and calls no allocating routine. */
+qlora_status nf4_layer_error_rank_noalloc(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
+                                          int32_t w_dtype, nf4_qconfig q, int32_t K,
+                                          double* err, int32_t* order, uint8_t* keep, qlora_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -416,4 +416,22 @@ qlora_status nf4_layer_error_rank(int32_t n_layers, const uint16_t* const* W_ptr
                                  workspace_bytes, static_cast<int*>(workspace), S(stream));
 }
 
+qlora_status nf4_layer_error_rank_noalloc(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
+                                          int32_t w_dtype, nf4_qconfig q, int32_t K, double* err, int32_t* order,
+                                          uint8_t* keep, qlora_stream_t stream) {
+  if (w_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_DTYPE;
+  if (!qconfig_ok(q)) return QLORA_ERR_UNSUPPORTED;
+  if (n_layers < 1 || n_layers > 1024 || K < 0 || K > n_layers) return QLORA_ERR_SHAPE;
+  if (!W_ptrs || !numel || !err || !order || !keep) return QLORA_ERR_NULL;
+  for (int i = 0; i < n_layers; ++i) {
+    if (!W_ptrs[i]) return QLORA_ERR_NULL;
+    if (numel[i] <= 0 || numel[i] % 64) return QLORA_ERR_SHAPE;
+    if (!aligned16(W_ptrs[i])) return QLORA_ERR_ALIGN;
+  }
+  if (noalloc_chunks(n_layers, numel) > (int64_t(1) << 20)) return QLORA_ERR_SHAPE;
+  QLB_TRY(check_device());
+  return launch_layer_error_rank_noalloc(n_layers, W_ptrs, numel, q.double_quant != 0, K, err, order, keep,
+                                         S(stream));
+}
+
 }  // extern "C"

@@ -42,6 +42,12 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
                                      int K, double* err, int32_t* order, uint8_t* keep, void* ws, size_t ws_bytes,
                                      int* status, cudaStream_t s);
 
+// Allocation-free variant: partial sums in a file-scope device array (see layer_error.cu).
+int64_t noalloc_chunks(int n_layers, const int64_t* numel);
+qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
+                                             bool dq, int K, double* err, int32_t* order, uint8_t* keep,
+                                             cudaStream_t s);
+
 // ---- gemm.cu
 int num_sms();
 // Operand descriptions for the tcgen05 GEMM engine.

@@ -9,6 +9,8 @@
 #include <cfloat>
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "internal.cuh"
 #include "nf4_device.cuh"
 
@@ -182,6 +184,77 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
   else layer_error_chunk_kernel<false><<<unsigned(c), 256, 0, s>>>(tab, partial, status);
   if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
   layer_error_finish_kernel<<<(n_layers + 255) / 256, 256, 0, s>>>(partial, first_dev, n_layers, err);
+  rank_topk_kernel<<<1, 1024, 0, s>>>(err, n_layers, K, order, keep);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------
+// Allocation-free variant.
+//
+// Same three passes, but the per-chunk partial sums live in a file-scope device
+// array instead of a caller workspace, and the chunk table reaches the finish
+// pass as a kernel parameter, so a call needs no device memory beyond its
+// inputs and outputs. The array is 16 MiB (2^20 chunks of 16384 weights, i.e.
+// up to 2^34 weights per call); every GPU that loads the library keeps it
+// until the process exits. All calls share it: calls that overlap on the GPU
+// (two streams, two host threads) race on it. Each call overwrites every
+// partial it reads, so nothing has to be cleared between calls.
+
+constexpr int64_t kNoAllocMaxChunks = int64_t(1) << 20;
+static __device__ __align__(256) double2 g_noalloc_partials[kNoAllocMaxChunks];
+
+__global__ void layer_error_finish_table_kernel(const double2* __restrict__ partial,
+                                                const __grid_constant__ LayerTable tab, double* __restrict__ err) {
+  const int l = blockIdx.x * blockDim.x + threadIdx.x;
+  if (l >= tab.n_layers) return;
+  double sd = 0.0, sw = 0.0;
+  for (int c = tab.first_chunk[l]; c < tab.first_chunk[l + 1]; ++c) { sd += partial[c].x; sw += partial[c].y; }
+  err[l] = (sw > 0.0) ? sqrt(sd / sw) : 0.0;
+}
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+LayerTable g_noalloc_tab;  // host staging of the by-value parameter, guarded by g_noalloc_mu
+}  // namespace
+
+int64_t noalloc_chunks(int n_layers, const int64_t* numel) {
+  int64_t c = 0;
+  for (int i = 0; i < n_layers; ++i) c += chunks_of(numel[i]);
+  return c;
+}
+
+qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
+                                             bool dq, int K, double* err, int32_t* order, uint8_t* keep,
+                                             cudaStream_t s) {
+  if (noalloc_chunks(n_layers, numel) > kNoAllocMaxChunks) return QLORA_ERR_SHAPE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return QLORA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    // One-time set-up on this device (the current one): the host-side name of the
+    // array is only a stand-in, the kernels need its device address.
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_partials) != cudaSuccess || ptr == nullptr) return QLORA_ERR_CUDA;
+    g_noalloc_addr[dev] = ptr;
+  }
+  double2* partial = static_cast<double2*>(g_noalloc_addr[dev]);
+  LayerTable& tab = g_noalloc_tab;
+  tab.n_layers = n_layers;
+  int32_t c = 0;
+  for (int i = 0; i < n_layers; ++i) {
+    tab.ptr[i] = W_ptrs[i];
+    tab.numel[i] = numel[i];
+    tab.first_chunk[i] = c;
+    c += chunks_of(numel[i]);
+  }
+  tab.first_chunk[n_layers] = c;
+  if (dq) layer_error_chunk_kernel<true><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr);
+  else layer_error_chunk_kernel<false><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr);
+  if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
+  layer_error_finish_table_kernel<<<(n_layers + 255) / 256, 256, 0, s>>>(partial, tab, err);
   rank_topk_kernel<<<1, 1024, 0, s>>>(err, n_layers, K, order, keep);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
