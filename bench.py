@@ -225,17 +225,60 @@ def gpu_main(args):
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
     prof = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
 
-    # legs, measured once per step with events between the calls
+    # Warm up eagerly (sizes the workspace, sets kernel attributes), then capture
+    # one whole step -- and each leg on its own -- into CUDA graphs; timing
+    # replays removes host launch gaps from the device time.
     for _ in range(max(3, args.warmup)):
         run_step(g["W"], g["X"], g["dY"], g["L1"], g["L2"])
     torch.cuda.synchronize()
     assert api.status() == 0, "device status set during warm-up"
-
     for e in prof:  # torch creates the CUDA event on first record
         e.record(stream)
     torch.cuda.synchronize()
     lib.qlora_profile_events(ctypes.c_void_p(prof[0].cuda_event), ctypes.c_void_p(prof[1].cuda_event),
                              ctypes.c_void_p(prof[2].cuda_event), ctypes.c_void_p(prof[3].cuda_event))
+    state = {}
+
+    def leg_quant():
+        state["w"] = api.quantize(g["W"], double_quant=True)
+
+    def leg_err():
+        api.layer_error_rank([g["W"]], 0, double_quant=True)
+
+    def leg_fwd():
+        state["Y"], state["T"] = api.linear_fwd(state["w"], g["X"], g["L1"], g["L2"], s)
+
+    def leg_bwd():
+        state["dX"], state["dL1"], state["dL2"] = api.linear_bwd(state["w"], g["X"], g["dY"], g["L1"], g["L2"], s,
+                                                                  T=state["T"])
+        if world > 1:
+            dist.all_reduce(state["dL1"])
+            dist.all_reduce(state["dL2"])
+
+    def whole_step():
+        leg_quant(); leg_err(); leg_fwd(); leg_bwd()
+
+    use_graphs = not args.eager and world == 1
+    graphs = {}
+    if use_graphs:
+        try:
+            for name, fn in (("step", whole_step), ("quantize", leg_quant), ("error_rank", leg_err),
+                             ("fwd", leg_fwd), ("bwd", leg_bwd)):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr):
+                    fn()
+                graphs[name] = gr
+            torch.cuda.synchronize()
+        except Exception as exc:  # fall back to eager timing
+            print(f"graph capture failed ({exc}); timing eagerly", file=sys.stderr)
+            graphs, use_graphs = {}, False
+
+    def run(name, fn):
+        if use_graphs:
+            graphs[name].replay()
+        else:
+            fn()
+
     step_ms, legs = [], {"quantize": [], "error_rank": [], "fwd": [], "bwd": [], "fwd_gemm": [], "dx_gemm": []}
     if world > 1:
         dist.barrier()
@@ -246,29 +289,25 @@ def gpu_main(args):
     for i in range(args.steps):
         flush.zero_()
         ev[0].record(stream)
-        w = api.quantize(g["W"], double_quant=True)
+        run("step", whole_step)
         ev[1].record(stream)
-        api.layer_error_rank([g["W"]], 0, double_quant=True)
-        ev[2].record(stream)
-        Y, T = api.linear_fwd(w, g["X"], g["L1"], g["L2"], s)
-        ev[3].record(stream)
-        dX, dL1, dL2 = api.linear_bwd(w, g["X"], g["dY"], g["L1"], g["L2"], s, T=T)
-        if world > 1:
-            dist.all_reduce(dL1)
-            dist.all_reduce(dL2)
-        ev[4].record(stream)
-        ev[4].synchronize()
-        step_ms.append(ev[0].elapsed_time(ev[4]))
-        legs["quantize"].append(ev[0].elapsed_time(ev[1]))
-        legs["error_rank"].append(ev[1].elapsed_time(ev[2]))
-        legs["fwd"].append(ev[2].elapsed_time(ev[3]))
-        legs["bwd"].append(ev[3].elapsed_time(ev[4]))
+        ev[1].synchronize()
+        step_ms.append(ev[0].elapsed_time(ev[1]))
         legs["fwd_gemm"].append(prof[0].elapsed_time(prof[1]))
         legs["dx_gemm"].append(prof[2].elapsed_time(prof[3]))
     clk = clocks.stop()
+    for name, fn in (("quantize", leg_quant), ("error_rank", leg_err), ("fwd", leg_fwd), ("bwd", leg_bwd)):
+        for i in range(max(5, min(args.steps, 50))):
+            flush.zero_()
+            ev[2].record(stream)
+            run(name, fn)
+            ev[3].record(stream)
+            ev[3].synchronize()
+            legs[name].append(ev[2].elapsed_time(ev[3]))
     lib.qlora_profile_events(None, None, None, None)
     torch.cuda.synchronize()
     assert api.status() == 0, "device status set during timing"
+    graphs.clear()
 
     total_ms = sum(step_ms)
     if world > 1:
@@ -345,12 +384,13 @@ def gpu_main(args):
         cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": desc + f"; repeated for {secs:.1f} s", "seconds": secs}
 
-    launches_per_step = 1 + 3 + 5 + 9
+    launches_per_step = 1 + 3 + 4 + 6  # quantize; error chunk/finish/rank; fwd (scales, L2 prep, T, GEMM); bwd (U, dL2, dL1, scales, L1 prep, dX GEMM)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args, world),
             "roofline": roofline, "legs": legs_out, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
+            "timing": "cuda-graph replay of the step" if use_graphs else "eager API calls",
             "peaks": {"bf16_tflops": peaks["bf16"], "bf16_tflops_sustained": peaks["bf16_sus"],
                       "hbm_gbs": peaks["hbm"], "source": peaks["source"]}}
     if rank == 0:
@@ -372,6 +412,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager API calls instead of CUDA-graph replays")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

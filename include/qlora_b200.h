@@ -106,8 +106,7 @@ qlora_status qlora_read_status(const void* workspace, qlora_stream_t stream);
 /* Clears the device status word (stream-ordered). */
 qlora_status qlora_reset_status(void* workspace, qlora_stream_t stream);
 
-/* Checks that device `device` is an sm_100 part and that the library's kernels
- * can be loaded on it. */
+/* Checks that device `device` is an sm_100 (B200-class) part. */
 qlora_status qlora_device_check(int device);
 
 /* Profiling aid (not part of the method): when set, cudaEvent_t handles that
@@ -147,8 +146,10 @@ qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream
 
 /* --------------------------------------------------------- NF4-LoRA linear */
 
-/* Shape rules for the linear: in % 256 == 0, out % 256 == 0, M >= 1 (any),
- * r % 8 == 0 and 8 <= r <= 256; every pointer 16-byte aligned. */
+/* Shape rules for the linear: in % 256 == 0, out % 256 == 0, 1 <= M <= 2^21,
+ * r % 8 == 0 and 8 <= r <= 256; every pointer 16-byte aligned. The workspace
+ * holds, after the status word, 64 KiB of split-K tile counters that the
+ * kernels leave at zero: zero a fresh workspace once before its first use. */
 size_t qlora_fwd_workspace_size(int64_t M, int64_t out, int64_t in, int32_t r);
 size_t qlora_bwd_workspace_size(int64_t M, int64_t out, int64_t in, int32_t r);
 

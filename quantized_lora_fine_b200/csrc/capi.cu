@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 
 #include "gemm.cuh"
@@ -45,7 +46,7 @@ struct ThinSplit {
 ThinSplit thin_split(int64_t rows, int64_t ksteps) {
   ThinSplit t;
   t.tiles = int((rows + 127) / 128);
-  int sp = std::max(1, int((kThinTargetCtas + t.tiles - 1) / t.tiles));
+  int sp = std::max(1, int(kThinTargetCtas / t.tiles));  // one wave of CTAs
   sp = int(std::min<int64_t>(sp, ksteps));
   t.kps = int((ksteps + sp - 1) / sp);
   t.splits = int((ksteps + t.kps - 1) / t.kps);
@@ -57,12 +58,13 @@ int thin_bn(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
 // ---- workspace layouts
 
 struct FwdLayout {
-  size_t scales, l2t, t, part, total;
+  size_t scales, l2t, t, part, counters, total;
 };
 
 FwdLayout fwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
   FwdLayout L;
-  size_t off = kStatusBytes;
+  L.counters = kStatusBytes;
+  size_t off = kReservedBytes;
   L.scales = off; off += up256(size_t(out) * size_t(in / 64) * 4);
   L.l2t = off;    off += up256(size_t(out) * r * 2);
   L.t = off;      off += up256(size_t(M) * r * 2);
@@ -73,12 +75,13 @@ FwdLayout fwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
 }
 
 struct BwdLayout {
-  size_t scales, l1s, t, u, part, total;
+  size_t scales, l1s, t, u, part, counters, total;
 };
 
 BwdLayout bwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
   BwdLayout L;
-  size_t off = kStatusBytes;
+  L.counters = kStatusBytes;
+  size_t off = kReservedBytes;
   L.scales = off; off += up256(size_t(out) * size_t(in / 64) * 4);
   L.l1s = off;    off += up256(size_t(in) * r * 2);
   L.t = off;      off += up256(size_t(M) * r * 2);
@@ -97,6 +100,8 @@ qlora_status check_linear(const qlora_weight* w, int64_t M, int32_t r) {
   if (w->out <= 0 || w->in <= 0 || M <= 0) return QLORA_ERR_SHAPE;
   if (w->in % 256 || w->out % 256) return QLORA_ERR_SHAPE;
   if (w->in > (int64_t(1) << 30) || w->out > (int64_t(1) << 30) || M > (int64_t(1) << 30)) return QLORA_ERR_SHAPE;
+  // split-K tile counters: one per 128 rows of M, out or in
+  if ((std::max({M, w->out, w->in}) + 127) / 128 > kMaxCounterTiles) return QLORA_ERR_SHAPE;
   if (r < 8 || r > 256 || r % 8) return QLORA_ERR_SHAPE;
   if (w->is_bf16) {
     if (!w->w_bf16) return QLORA_ERR_NULL;
@@ -124,7 +129,8 @@ struct Thin {
   int r;
 };
 
-qlora_status run_thin(const Thin& t, float* part, int* status, cudaStream_t s, int* splits_out) {
+qlora_status run_thin(const Thin& t, float* part, int* counters, void* fin_out, int fin_mode, float fin_scale,
+                      int* status, cudaStream_t s) {
   const ThinSplit ts = thin_split(t.rows, t.ksteps);
   const int bn = thin_bn(t.r);
   GemmOperands o;
@@ -149,7 +155,10 @@ qlora_status run_thin(const Thin& t, float* part, int* status, cudaStream_t s, i
   p.ld_out = t.r;
   p.split_stride = t.rows * t.r;
   p.status = status;
-  *splits_out = ts.splits;
+  p.counters = counters;
+  p.fin_out = fin_out;
+  p.fin_mode = fin_mode;
+  p.fin_scale = fin_scale;
   return launch_gemm(t.kind, bn, o, p, s);
 }
 
@@ -160,6 +169,29 @@ qlora_status run_thin(const Thin& t, float* part, int* status, cudaStream_t s, i
   } while (0)
 
 cudaEvent_t g_prof[4] = {nullptr, nullptr, nullptr, nullptr};
+
+// Profiling events are recorded as timestamp nodes when the stream is being
+// captured into a CUDA graph.
+void record_prof(cudaEvent_t e, cudaStream_t s) {
+  if (!e) return;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, s);
+}
+
+// The NF4 GEMMs run on the single-CTA kernel unless QLORA_B200_GEMM=pair selects
+// the CTA-pair kernel (both compute the same values; kept side by side for
+// measurement).
+bool use_pair_kernel() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("QLORA_B200_GEMM");
+    v = (e && std::strcmp(e, "pair") == 0) ? 1 : 0;
+  }
+  return v == 1;
+}
 
 // main GEMM with NF4 or bf16 weight and the LoRA extension
 qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t M, const uint16_t* Ax,
@@ -173,6 +205,39 @@ qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
   if (!make_tmap_2d(&op.A, A, TmapType::BF16, Kdim, M, Kdim * 2, 64, 128, true)) return QLORA_ERR_CUDA;
   if (!make_tmap_2d(&op.Ax, Ax, TmapType::BF16, r, M, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
   if (!make_tmap_2d(&op.Bx, Bx, TmapType::BF16, r, Ndim, int64_t(r) * 2, 64, 256, true)) return QLORA_ERR_CUDA;
+  if (!w->is_bf16 && use_pair_kernel()) {
+    // CTA-pair fused kernel: 512 x 128 tiles; each CTA holds two 128-row A tiles
+    // and 64 rows (fwd) or columns (dX) of B.
+    GemmOperands pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.A = op.A;
+    pp.Ax = op.Ax;
+    if (!make_tmap_2d(&pp.Bx, Bx, TmapType::BF16, r, Ndim, int64_t(r) * 2, 64, 64, true)) return QLORA_ERR_CUDA;
+    if (!dx) {
+      if (!make_tmap_2d_sw(&pp.codes, w->codes, TmapType::U8, h / 2, o_, h / 2, 32, 64, 32)) return QLORA_ERR_CUDA;
+      if (!make_tmap_2d(&pp.scales, scales_t, TmapType::F32, o_, h / 64, o_ * 4, 64, 1, false)) return QLORA_ERR_CUDA;
+    } else {
+      if (!make_tmap_2d_sw(&pp.codes, w->codes, TmapType::U8, h / 2, o_, h / 2, 32, 64, 32)) return QLORA_ERR_CUDA;
+      if (!make_tmap_2d(&pp.scales, scales_t, TmapType::F32, o_, h / 64, o_ * 4, 64, 1, false)) return QLORA_ERR_CUDA;
+    }
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = int(M);
+    p.N = int(Ndim);
+    p.num_k_main = int(Kdim / 64);
+    p.num_k_ext = (r + 63) / 64;
+    p.tiles_m = int((M + 511) / 512);
+    p.tiles_n = int(Ndim / 128);
+    p.splits = 1;
+    p.ksteps_per_split = p.num_k_main;
+    p.out = out;
+    p.ld_out = Ndim;
+    p.status = status;
+    record_prof(g_prof[dx ? 2 : 0], s);
+    const qlora_status st = launch_gemm_pair(dx, pp, p, s);
+    record_prof(g_prof[dx ? 3 : 1], s);
+    return st;
+  }
   GemmKind kind;
   if (w->is_bf16) {
     if (!dx) {
@@ -207,10 +272,9 @@ qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
   p.ld_out = Ndim;
   p.split_stride = 0;
   p.status = status;
-  cudaEvent_t eb = g_prof[dx ? 2 : 0], ee = g_prof[dx ? 3 : 1];
-  if (eb) cudaEventRecord(eb, s);
+  record_prof(g_prof[dx ? 2 : 0], s);
   const qlora_status st = launch_gemm(kind, 256, op, p, s);
-  if (ee) cudaEventRecord(ee, s);
+  record_prof(g_prof[dx ? 3 : 1], s);
   return st;
 }
 
@@ -333,10 +397,9 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t 
                                  scales_t, s));
   QLB_TRY(launch_scale_lora(L2, r, o_, scale, /*transpose=*/true, l2t, s));
   // T = X L1 : A = X (K-major), B = L1 as [h x r] (MN-major for B)
+  int* counters = reinterpret_cast<int*>(ws + L.counters);
   Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
-  int splits = 0;
-  QLB_TRY(run_thin(tt, part, status, s, &splits));
-  QLB_TRY(launch_reduce_bf16(part, splits, M, r, T, s));
+  QLB_TRY(run_thin(tt, part, counters, T, 0, 1.f, status, s));
   return run_main(false, w, X, M, T, l2t, r, scales_t, Y, status, s);
 }
 
@@ -362,27 +425,23 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const ui
   float* part = reinterpret_cast<float*>(ws + L.part);
   const int64_t h = w->in, o_ = w->out;
   const int64_t mk = (M + 63) / 64;
-  int splits = 0;
+  int* counters = reinterpret_cast<int*>(ws + L.counters);
   const uint16_t* T = T_saved;
   if (!T) {
     uint16_t* Tw = reinterpret_cast<uint16_t*>(ws + L.t);
     Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
-    QLB_TRY(run_thin(tt, part, status, s, &splits));
-    QLB_TRY(launch_reduce_bf16(part, splits, M, r, Tw, s));
+    QLB_TRY(run_thin(tt, part, counters, Tw, 0, 1.f, status, s));
     T = Tw;
   }
   // U = dY L2^T : A = dY (K-major, K = out), B = L2 [r x out] (K-major)
   Thin tu{GemmKind::ThinKK, dY, o_, M, L2, o_, r, M, o_ / 64, r};
-  QLB_TRY(run_thin(tu, part, status, s, &splits));
-  QLB_TRY(launch_reduce_bf16(part, splits, M, r, U, s));
-  // dL2^T = dY^T T  (out x r): A = dY^T (MN-major), B = T (MN-major); K = M
+  QLB_TRY(run_thin(tu, part, counters, U, 0, 1.f, status, s));
+  // dL2 = s (dY^T T)^T : A = dY^T (MN-major), B = T (MN-major); K = M; written transposed
   Thin t2{GemmKind::ThinMM, dY, o_, M, T, r, M, o_, mk, r};
-  QLB_TRY(run_thin(t2, part, status, s, &splits));
-  QLB_TRY(launch_reduce_f32(part, splits, o_, r, scale, /*transpose=*/true, dL2, s));
-  // dL1 = X^T U (in x r): A = X^T (MN-major), B = U (MN-major); K = M
+  QLB_TRY(run_thin(t2, part, counters, dL2, 2, scale, status, s));
+  // dL1 = s X^T U (in x r): A = X^T (MN-major), B = U (MN-major); K = M
   Thin t1{GemmKind::ThinMM, X, h, M, U, r, M, h, mk, r};
-  QLB_TRY(run_thin(t1, part, status, s, &splits));
-  QLB_TRY(launch_reduce_f32(part, splits, h, r, scale, /*transpose=*/false, dL1, s));
+  QLB_TRY(run_thin(t1, part, counters, dL1, 1, scale, status, s));
   if (dX) {
     if (!w->is_bf16)
       QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,

@@ -43,11 +43,96 @@ __device__ __forceinline__ void load8<float>(const float* W, int64_t e0, int64_t
   }
 }
 
-template <typename T, bool DQ>
-__global__ void __launch_bounds__(256) nf4_quantize_kernel(const T* __restrict__ W, int64_t numel,
-                                                           uint8_t* __restrict__ codes, float* __restrict__ absmax,
-                                                           uint8_t* __restrict__ absmax_q,
-                                                           float* __restrict__ absmax2, int* status) {
+// Shared tail of both quantizer variants: double quantization of the group's
+// 256 absmax values held in s_amax.
+__device__ __forceinline__ void dq_group(const float* s_amax, float* s_red, int64_t nb, int64_t g,
+                                         uint8_t* __restrict__ absmax_q, float* __restrict__ absmax2) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __syncthreads();
+  const int64_t nblk_g = (int64_t(kDQBlock) < nb - g * kDQBlock ? int64_t(kDQBlock) : nb - g * kDQBlock);
+  float v = (tid < nblk_g) ? s_amax[tid] : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  float G = s_red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) G = fmaxf(G, s_red[i]);
+  if (tid < nblk_g) {
+    uint8_t q = 0;
+    if (G > 0.f) {
+      const float inv = __fdiv_rn(448.f, G);
+      q = f32_to_e4m3_satfinite(__fmul_rn(s_amax[tid], inv));
+    }
+    absmax_q[g * kDQBlock + tid] = q;
+  }
+  if (tid == 0) absmax2[g] = (G > 0.f) ? __fdiv_rn(G, 448.f) : 0.f;
+}
+
+// bf16 weights, full chunks of 8: integer absmax on packed pairs, reciprocal
+// division (exact for bf16 operands), cell-table code lookup.
+template <bool DQ>
+__global__ void __launch_bounds__(256) nf4_quantize_bf16_kernel(const uint16_t* __restrict__ W, int64_t numel,
+                                                                uint8_t* __restrict__ codes,
+                                                                float* __restrict__ absmax,
+                                                                uint8_t* __restrict__ absmax_q,
+                                                                float* __restrict__ absmax2, int* status) {
+  __shared__ float s_amax[256];
+  __shared__ float s_red[8];
+  __shared__ NF4CellSmem s_cells;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  nf4_cells_load(s_cells, tid);
+  const int64_t nb = (numel + kBlock - 1) / kBlock;
+  const int64_t g = blockIdx.x;
+  // Prefetch all 8 slices of this thread (one 16-byte load each).
+  uint4 raw[8];
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int64_t e0 = (g * kDQBlock + it * 32 + warp * 4 + (lane >> 3)) * kBlock + (lane & 7) * 8;
+    raw[it] = (e0 + 8 <= numel) ? __ldg(reinterpret_cast<const uint4*>(W + e0)) : make_uint4(0, 0, 0, 0);
+    if (e0 < numel && e0 + 8 > numel) {  // ragged tail chunk
+      uint16_t tmp[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int i = 0; i < 8; ++i) if (e0 + i < numel) tmp[i] = W[e0 + i];
+      raw[it] = make_uint4(tmp[0] | (uint32_t(tmp[1]) << 16), tmp[2] | (uint32_t(tmp[3]) << 16),
+                           tmp[4] | (uint32_t(tmp[5]) << 16), tmp[6] | (uint32_t(tmp[7]) << 16));
+    }
+  }
+  __syncthreads();
+  uint32_t bad = 0;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int bi = it * 32 + warp * 4 + (lane >> 3);
+    const int64_t blk = g * kDQBlock + bi;
+    const int64_t e0 = blk * kBlock + (lane & 7) * 8;
+    const uint32_t amb = block_max8_lanes(absmax8_bf16_bits(raw[it]));
+    bad |= amb >= 0x7F80u;
+    const float am = __uint_as_float(amb << 16);
+    if ((lane & 7) == 0) {
+      s_amax[bi] = am;
+      if (blk < nb && absmax != nullptr) absmax[blk] = am;
+    }
+    if (e0 < numel) {
+      uint32_t idx[8];
+      const uint32_t word = (am > 0.f) ? quant8_bf16(raw[it], am, s_cells, idx) : 0x77777777u;
+      if (e0 + 8 <= numel) {
+        *reinterpret_cast<uint32_t*>(codes + e0 / 2) = word;
+      } else {
+        for (int k = 0; 2 * k < numel - e0; ++k) codes[e0 / 2 + k] = uint8_t(word >> (8 * k));
+      }
+    }
+  }
+  if (bad) set_status(status, QLORA_ERR_NONFINITE);
+  if constexpr (DQ) dq_group(s_amax, s_red, nb, g, absmax_q, absmax2);
+}
+
+// fp32 weights: IEEE division per element, linear midpoint count (kept simple:
+// the workloads quantize bf16 weights).
+template <bool DQ>
+__global__ void __launch_bounds__(256) nf4_quantize_f32_kernel(const float* __restrict__ W, int64_t numel,
+                                                               uint8_t* __restrict__ codes,
+                                                               float* __restrict__ absmax,
+                                                               uint8_t* __restrict__ absmax_q,
+                                                               float* __restrict__ absmax2, int* status) {
   __shared__ float s_amax[256];
   __shared__ float s_red[8];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -61,7 +146,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const T* __restrict__
     const int64_t e0 = blk * kBlock + (lane & 7) * 8;
     float w[8];
     const bool live = blk < nb && e0 < numel;
-    if (live) load8<T>(W, e0, numel, w);
+    if (live) load8<float>(W, e0, numel, w);
     else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) w[i] = 0.f;
@@ -95,27 +180,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const T* __restrict__
     }
   }
   if (bad) set_status(status, QLORA_ERR_NONFINITE);
-  if constexpr (DQ) {
-    __syncthreads();
-    const int64_t nblk_g = (int64_t(kDQBlock) < nb - g * kDQBlock ? int64_t(kDQBlock) : nb - g * kDQBlock);
-    float v = (tid < nblk_g) ? s_amax[tid] : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (lane == 0) s_red[warp] = v;
-    __syncthreads();
-    float G = s_red[0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) G = fmaxf(G, s_red[i]);
-    if (tid < nblk_g) {
-      uint8_t q = 0;
-      if (G > 0.f) {
-        const float inv = __fdiv_rn(448.f, G);
-        q = f32_to_e4m3_satfinite(__fmul_rn(s_amax[tid], inv));
-      }
-      absmax_q[g * kDQBlock + tid] = q;
-    }
-    if (tid == 0) absmax2[g] = (G > 0.f) ? __fdiv_rn(G, 448.f) : 0.f;
-  }
+  if constexpr (DQ) dq_group(s_amax, s_red, nb, g, absmax_q, absmax2);
 }
 
 qlora_status launch_quantize(const void* W, int w_dtype, int64_t numel, bool dq, uint8_t* codes, float* absmax,
@@ -125,11 +190,11 @@ qlora_status launch_quantize(const void* W, int w_dtype, int64_t numel, bool dq,
   if (groups <= 0) return QLORA_OK;
   dim3 grid(static_cast<unsigned>(groups));
   if (w_dtype == QLORA_DTYPE_BF16) {
-    if (dq) nf4_quantize_kernel<uint16_t, true><<<grid, 256, 0, s>>>((const uint16_t*)W, numel, codes, absmax, absmax_q, absmax2, status);
-    else nf4_quantize_kernel<uint16_t, false><<<grid, 256, 0, s>>>((const uint16_t*)W, numel, codes, absmax, absmax_q, absmax2, status);
+    if (dq) nf4_quantize_bf16_kernel<true><<<grid, 256, 0, s>>>((const uint16_t*)W, numel, codes, absmax, absmax_q, absmax2, status);
+    else nf4_quantize_bf16_kernel<false><<<grid, 256, 0, s>>>((const uint16_t*)W, numel, codes, absmax, absmax_q, absmax2, status);
   } else {
-    if (dq) nf4_quantize_kernel<float, true><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
-    else nf4_quantize_kernel<float, false><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
+    if (dq) nf4_quantize_f32_kernel<true><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
+    else nf4_quantize_f32_kernel<false><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
   }
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
@@ -237,55 +302,6 @@ qlora_status launch_scale_lora(const uint16_t* src, int64_t rows, int64_t cols, 
   const int64_t n = rows * cols;
   const int64_t blocks = std::min<int64_t>((n + 255) / 256, 4096);
   scale_lora_kernel<<<unsigned(blocks), 256, 0, s>>>(src, rows, cols, scale, transpose ? 1 : 0, dst);
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
-}
-
-__global__ void reduce_bf16_kernel(const float* __restrict__ part, int splits, int64_t n, uint16_t* __restrict__ out) {
-  // 4 consecutive elements per thread
-  const int64_t n4 = n / 4;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n4; i += int64_t(gridDim.x) * blockDim.x) {
-    float4 acc = __ldg(reinterpret_cast<const float4*>(part) + i);
-    for (int p = 1; p < splits; ++p) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(part + p * n) + i);
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
-    uint2 o;
-    o.x = pack_bf16x2(acc.x, acc.y);
-    o.y = pack_bf16x2(acc.z, acc.w);
-    reinterpret_cast<uint2*>(out)[i] = o;
-  }
-}
-
-qlora_status launch_reduce_bf16(const float* part, int splits, int64_t rows, int64_t cols, uint16_t* out,
-                                cudaStream_t s) {
-  const int64_t n = rows * cols;  // cols % 8 == 0 by the shape rules
-  const int64_t blocks = std::min<int64_t>((n / 4 + 255) / 256, int64_t(num_sms()) * 8);
-  reduce_bf16_kernel<<<unsigned(std::max<int64_t>(blocks, 1)), 256, 0, s>>>(part, splits, n, out);
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
-}
-
-__global__ void reduce_f32_kernel(const float* __restrict__ part, int splits, int64_t rows, int64_t cols,
-                                  float scale, int transpose, float* __restrict__ out) {
-  const int64_t n = rows * cols;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
-    float acc = part[i];
-    for (int p = 1; p < splits; ++p) acc += part[p * n + i];
-    acc = __fmul_rn(acc, scale);
-    if (transpose) {
-      const int64_t rr = i / cols, cc = i % cols;
-      out[cc * rows + rr] = acc;
-    } else {
-      out[i] = acc;
-    }
-  }
-}
-
-qlora_status launch_reduce_f32(const float* part, int splits, int64_t rows, int64_t cols, float scale,
-                               bool transpose, float* out, cudaStream_t s) {
-  const int64_t n = rows * cols;
-  const int64_t blocks = std::min<int64_t>((n + 255) / 256, int64_t(num_sms()) * 8);
-  reduce_f32_kernel<<<unsigned(std::max<int64_t>(blocks, 1)), 256, 0, s>>>(part, splits, rows, cols, scale,
-                                                                          transpose ? 1 : 0, out);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * C::STAGES + 5);
 
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ uint32_t s_last;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         for (int j = 0; j < nsteps; ++j, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!mbar_wait(empty_bar(s), ph ^ 1u)) { set_status(p.status, QLORA_ERR_TIMEOUT); ok = false; break; }
+          if (!mbar_wait(empty_bar(s), ph ^ 1u)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 1); ok = false; break; }
           const uint32_t st = smem_base + s * C::kStage;
           const uint32_t a_s = st, b_s = st + C::kA;
           if (j < ti.ke - ti.kb) {
@@ -242,14 +243,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         const TileInfo ti = decode_tile(p, t);
         const int nsteps = (ti.ke - ti.kb) + ti.n_ext;
         const uint32_t acc = tcount & 1u, tph = (tcount >> 1) & 1u;
-        if (!mbar_wait(tempty_bar(acc), tph ^ 1u)) { set_status(p.status, QLORA_ERR_TIMEOUT); ok = false; break; }
+        if (!mbar_wait(tempty_bar(acc), tph ^ 1u)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 2); ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::BN;
         for (int j = 0; j < nsteps; ++j, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!mbar_wait(full_bar(s), ph)) { set_status(p.status, QLORA_ERR_TIMEOUT); ok = false; break; }
-          if (C::NF4 && !mbar_wait(deq_bar(s), ph)) { set_status(p.status, QLORA_ERR_TIMEOUT); ok = false; break; }
+          if (!mbar_wait(full_bar(s), ph)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 3); ok = false; break; }
+          if (C::NF4 && !mbar_wait(deq_bar(s), ph)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 4); ok = false; break; }
           tc_fence_after();
           const uint32_t st = smem_base + s * C::kStage;
           const bool ext = j >= ti.ke - ti.kb;
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tcount) {
       const TileInfo ti = decode_tile(p, t);
       const uint32_t acc = tcount & 1u, tph = (tcount >> 1) & 1u;
-      if (!mbar_wait(tfull_bar(acc), tph)) { set_status(p.status, QLORA_ERR_TIMEOUT); break; }
+      if (!mbar_wait(tfull_bar(acc), tph)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 5); break; }
       tc_fence_after();
       const int grow = ti.m0 + int(row);
       const uint32_t tbase = tmem_base + ((q * 32u) << 16) + acc * C::BN;
@@ -320,6 +321,46 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if constexpr (C::OUT_F32) {
+        if (p.counters != nullptr) {
+          // Split-K finish: the last of the `splits` CTAs of this M tile reduces.
+          const int mt = t % (p.tiles_m * p.tiles_n);
+          __threadfence();
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (warp == 2 && lane == 0) s_last = (atomicAdd(p.counters + mt, 1) == p.splits - 1) ? 1u : 0u;
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (s_last) {
+            __threadfence();
+            if (grow < p.M) {
+              const float* src = reinterpret_cast<const float*>(p.out) + int64_t(grow) * p.ld_out;
+              for (int c4 = 0; c4 < p.N; c4 += 4) {
+                float4 acc4 = *reinterpret_cast<const float4*>(src + c4);
+                for (int sp = 1; sp < p.splits; ++sp) {
+                  const float4 v4 = *reinterpret_cast<const float4*>(src + int64_t(sp) * p.split_stride + c4);
+                  acc4.x += v4.x; acc4.y += v4.y; acc4.z += v4.z; acc4.w += v4.w;
+                }
+                if (p.fin_mode == 0) {
+                  uint2 o2;
+                  o2.x = pack_bf16x2(acc4.x, acc4.y);
+                  o2.y = pack_bf16x2(acc4.z, acc4.w);
+                  *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.fin_out) + int64_t(grow) * p.N + c4) = o2;
+                } else if (p.fin_mode == 1) {
+                  float* d = reinterpret_cast<float*>(p.fin_out) + int64_t(grow) * p.N + c4;
+                  *reinterpret_cast<float4*>(d) = make_float4(__fmul_rn(acc4.x, p.fin_scale), __fmul_rn(acc4.y, p.fin_scale),
+                                                              __fmul_rn(acc4.z, p.fin_scale), __fmul_rn(acc4.w, p.fin_scale));
+                } else {
+                  float* d = reinterpret_cast<float*>(p.fin_out);
+                  d[int64_t(c4 + 0) * p.M + grow] = __fmul_rn(acc4.x, p.fin_scale);
+                  d[int64_t(c4 + 1) * p.M + grow] = __fmul_rn(acc4.y, p.fin_scale);
+                  d[int64_t(c4 + 2) * p.M + grow] = __fmul_rn(acc4.z, p.fin_scale);
+                  d[int64_t(c4 + 3) * p.M + grow] = __fmul_rn(acc4.w, p.fin_scale);
+                }
+              }
+            }
+            if (warp == 2 && lane == 0) p.counters[mt] = 0;
+          }
+        }
+      }
     }
   } else {
     // ------------------------------------------------------------ dequantizers
@@ -333,7 +374,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         for (int j = 0; j < nsteps; ++j, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!mbar_wait(full_bar(s), ph)) { set_status(p.status, QLORA_ERR_TIMEOUT); ok = false; break; }
+          if (!mbar_wait(full_bar(s), ph)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 6); ok = false; break; }
           if (j < ti.ke - ti.kb) {
             uint8_t* st = smem + s * C::kStage;
             dequant_stage<C::B_MN>(dt, st + C::kCodesOff, reinterpret_cast<const float*>(st + C::kScalesOff),
@@ -355,6 +396,344 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   }
 }
 
+// =============================================================== CTA-pair kernel
+//
+// Fused NF4 GEMM on a pair of CTAs (cluster of 2, tcgen05 cta_group::2).
+// One pair tile is 512 (M) x 128 (N): two M = 256 accumulators share every
+// dequantized B tile, so each SM dequantizes one weight per 512 output rows.
+//
+// Shared memory holds three rings so that the dequantization latency does not
+// sit inside the A operand's load-to-release cycle:
+//   A ring (SA slots)  A0, A1: this CTA's 128-row halves of the two 256-row MMA
+//                      tiles (or the LoRA T/U rows in the extension steps)
+//   C ring (SC slots)  packed codes + expanded scales of this CTA's half of B;
+//                      loaded ahead of the A ring, consumed by the dequantizers
+//   B ring (SB slots)  bf16 B half (64 rows fwd / 64 columns dX), read by MMA
+// Every ring slot has exactly one writer that fills its rounds in order (the A
+// producer, the C producer, and dequantizer group g for B slot g, which also
+// issues the TMA load of the LoRA steps' B tile), so a parity wait can never be
+// satisfied by a phase two rounds old.
+// Warp roles: 0 A producer, 1 MMA issuer (even CTA) / relay (odd CTA) and TMEM
+// allocation, 2 C producer, 3-6 epilogue, 7.. dequantizer groups. The odd CTA's
+// relay forwards "B slot ready" to the even CTA once per step (one
+// cluster-scope release per step).
+
+template <bool B_MN_>
+struct PairCfg {
+  static constexpr bool B_MN = B_MN_;
+  static constexpr int SA = 5, SB = 4, SC = 8;
+  static constexpr int kA = 128 * 64 * 2;       // one 128-row A tile: 16 KB
+  static constexpr int kASlot = 2 * kA;         // A0 + A1
+  static constexpr int kB = 64 * 64 * 2;        // 8 KB
+  static constexpr int kCodes = 64 * 32;        // 2 KB
+  static constexpr int kScales = 64 * 4;        // 256 B
+  static constexpr int kCSlot = 3072;
+  static constexpr int kAOff = 0;
+  static constexpr int kBOff = kAOff + SA * kASlot;
+  static constexpr int kCOff = kBOff + SB * kB;
+  static constexpr int kBarOff = kCOff + SC * kCSlot;
+  static constexpr int kGroups = SB;            // group g owns B slot g
+  static constexpr int kWarpsPerGroup = 2;      // 64 threads: one 64-element block each per step
+  static constexpr int kDeqWarps = kGroups * kWarpsPerGroup;
+  static constexpr int kThreads = (7 + kDeqWarps) * 32;
+  static constexpr int kTmemCols = 512;         // 2 buffers x 2 accumulators x 128 columns
+  static constexpr int kNumBars = 2 * SA + 2 * SC + 3 * SB + 5;
+  static constexpr int kSmem = kBarOff + 8 * kNumBars + 16 + 1024;
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+// One thread turns one 64-element block of this CTA's B half into bf16.
+//   fwd (K-major): t = B row (0..63); dX (MN-major): t = K row of the single
+//   64-column chunk. Both read 64 rows x 32 B of codes (32-byte swizzle).
+__device__ __forceinline__ void dequant_block_pair(uint32_t t, const uint8_t* codes_s, const float* scales_s,
+                                                   uint32_t b_tile) {
+  const uint32_t csw = (t >> 2) & 1u;
+  const uint4 c0 = *reinterpret_cast<const uint4*>(codes_s + t * 32 + ((0u ^ csw) << 4));
+  const uint4 c1 = *reinterpret_cast<const uint4*>(codes_s + t * 32 + ((1u ^ csw) << 4));
+  const NF4Lut lut = nf4_make_lut(scales_s[t]);
+  const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const uint32_t sw = t & 7u;
+  const uint32_t row_base = b_tile + (t >> 3) * 1024u + sw * 128u;
+#pragma unroll
+  for (uint32_t c = 0; c < 8; ++c) {
+    const uint4 v = nf4_dequant_word(words[c], lut);
+    const uint32_t addr = row_base + ((c ^ sw) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+  }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1)
+    tc_gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmCodes,
+                            const __grid_constant__ CUtensorMap tmScales, const __grid_constant__ CUtensorMap tmAx,
+                            const __grid_constant__ CUtensorMap tmBx, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_base = smem_base + C::kBarOff;
+  auto afull = [&](int i) { return bar_base + 8u * i; };
+  auto aempty = [&](int i) { return bar_base + 8u * (C::SA + i); };
+  auto cfull = [&](int i) { return bar_base + 8u * (2 * C::SA + i); };
+  auto cempty = [&](int i) { return bar_base + 8u * (2 * C::SA + C::SC + i); };
+  auto bfull = [&](int i) { return bar_base + 8u * (2 * C::SA + 2 * C::SC + i); };
+  auto bready = [&](int i) { return bar_base + 8u * (2 * C::SA + 2 * C::SC + C::SB + i); };
+  auto bempty = [&](int i) { return bar_base + 8u * (2 * C::SA + 2 * C::SC + 2 * C::SB + i); };
+  const int kT0 = 2 * C::SA + 2 * C::SC + 3 * C::SB;
+  auto tfull = [&](int b) { return bar_base + 8u * (kT0 + b); };
+  auto tempty = [&](int b) { return bar_base + 8u * (kT0 + 2 + b); };
+  const uint32_t drain_bar = bar_base + 8u * (kT0 + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * C::kNumBars);
+  auto a_slot = [&](uint32_t i) { return smem_base + C::kAOff + (i % C::SA) * C::kASlot; };
+  auto b_slot = [&](uint32_t i) { return smem_base + C::kBOff + (i % C::SB) * C::kB; };
+  auto c_slot = [&](uint32_t i) { return C::kCOff + (i % C::SC) * C::kCSlot; };  // offset from smem
+
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::SA; ++i) { mbar_init(afull(i), 1); mbar_init(aempty(i), 1); }
+    for (int i = 0; i < C::SC; ++i) { mbar_init(cfull(i), 1); mbar_init(cempty(i), C::kWarpsPerGroup); }
+    for (int i = 0; i < C::SB; ++i) {
+      mbar_init(bfull(i), C::kWarpsPerGroup);
+      mbar_init(bready(i), 1);
+      mbar_init(bempty(i), 1);
+    }
+    for (int b = 0; b < 2; ++b) { mbar_init(tfull(b), 1); mbar_init(tempty(b), 8); }
+    mbar_init(drain_bar, 1);
+    fence_mbarrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = p.tiles_m * p.tiles_n;   // tiles of 512 x 128
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int nsteps = p.num_k_main + p.num_k_ext;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ A producer (both CTAs)
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += npairs) {
+        const int mb = t / p.tiles_n;
+        const int m0 = mb * 512 + int(rank) * 128;
+        for (int j = 0; j < nsteps; ++j, ++it) {
+          if (!mbar_wait(aempty(it % C::SA), ((it / C::SA) & 1u) ^ 1u)) {
+            set_status_site(p.status, QLORA_ERR_TIMEOUT, 101); ok = false; break;
+          }
+          const uint32_t dst = a_slot(it), bar = afull(it % C::SA);
+          mbar_arrive_expect_tx(bar, C::kASlot);
+          if (j < p.num_k_main) {
+            tma_load_2d(dst, &tmA, bar, j * 64, m0);
+            tma_load_2d(dst + C::kA, &tmA, bar, j * 64, m0 + 256);
+          } else {
+            const int kx = (j - p.num_k_main) * 64;
+            tma_load_2d(dst, &tmAx, bar, kx, m0);
+            tma_load_2d(dst + C::kA, &tmAx, bar, kx, m0 + 256);
+          }
+        }
+      }
+      if (it > 0) {  // let the last copies land before leaving
+        for (int k = 0; k < C::SA && k < int(it); ++k) {
+          const uint32_t i2 = it - 1 - k;
+          mbar_wait(afull(i2 % C::SA), (i2 / C::SA) & 1u, 100000000ull);
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ C producer (both CTAs)
+    if (lane == 0) {
+      tma_prefetch_desc(&tmCodes);
+      tma_prefetch_desc(&tmScales);
+      uint32_t it = 0, ic = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += npairs) {
+        const int nb = t % p.tiles_n;
+        const int nc0 = nb * 128 + int(rank) * 64;
+        for (int j = 0; j < nsteps; ++j, ++it) {
+          if (j >= p.num_k_main) continue;
+          if (!mbar_wait(cempty(ic % C::SC), ((ic / C::SC) & 1u) ^ 1u)) {
+            set_status_site(p.status, QLORA_ERR_TIMEOUT, 102); ok = false; break;
+          }
+          const uint32_t dst = smem_base + c_slot(ic), bar = cfull(ic % C::SC);
+          mbar_arrive_expect_tx(bar, C::kCodes + C::kScales);
+          if constexpr (!C::B_MN) {
+            tma_load_2d(dst, &tmCodes, bar, j * 32, nc0);
+            tma_load_2d(dst + C::kCodes, &tmScales, bar, nc0, j);
+          } else {
+            tma_load_2d(dst, &tmCodes, bar, nc0 / 2, j * 64);
+            tma_load_2d(dst + C::kCodes, &tmScales, bar, j * 64, nc0 / 64);
+          }
+          ++ic;
+        }
+      }
+      if (ic > 0) {
+        for (int k = 0; k < C::SC && k < int(ic); ++k) {
+          const uint32_t i2 = ic - 1 - k;
+          mbar_wait(cfull(i2 % C::SC), (i2 / C::SC) & 1u, 100000000ull);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0) {
+      // ------------------------------------------------------------ MMA issuer (even CTA)
+      if (lane == 0) {
+        constexpr uint32_t idesc_main = make_idesc_bf16(256, 128, 0, C::B_MN ? 1 : 0);
+        constexpr uint32_t idesc_ext = make_idesc_bf16(256, 128, 0, 0);
+        constexpr uint32_t b_adv = C::B_MN ? 2048u : 32u;
+        uint32_t it = 0, tcount = 0;
+        bool ok = true;
+        for (int t = pair; t < num_tiles && ok; t += npairs, ++tcount) {
+          const uint32_t buf = tcount & 1u, tph = (tcount >> 1) & 1u;
+          if (!mbar_wait_cluster(tempty(buf), tph ^ 1u)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 104); ok = false; break; }
+          tc_fence_after();
+          const uint32_t d0 = tmem_base + buf * 256u, d1 = d0 + 128u;
+          for (int j = 0; j < nsteps; ++j, ++it) {
+            const uint32_t pa = (it / C::SA) & 1u, pb = (it / C::SB) & 1u;
+            const int site = !mbar_wait(afull(it % C::SA), pa) ? 105
+                             : !mbar_wait(bfull(it % C::SB), pb) ? 115
+                             : !mbar_wait_cluster(bready(it % C::SB), pb) ? 125 : 0;
+            if (site) { set_status_site(p.status, QLORA_ERR_TIMEOUT, site); ok = false; break; }
+            tc_fence_after();
+            const bool ext = j >= p.num_k_main;
+            const uint32_t as = a_slot(it);
+            const uint64_t a0 = make_smem_desc(as, 16u, 1024u, kSwizzle128B);
+            const uint64_t a1 = make_smem_desc(as + C::kA, 16u, 1024u, kSwizzle128B);
+            const uint64_t bd = make_smem_desc(b_slot(it), 16u, 1024u, kSwizzle128B);
+            const uint32_t badv = ext ? 32u : b_adv;
+            const uint32_t idesc = ext ? idesc_ext : idesc_main;
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+              const uint64_t boff = uint64_t((kk * badv) >> 4), aoff = uint64_t((kk * 32u) >> 4);
+              tc_mma_bf16_pair(d0, a0 + aoff, bd + boff, idesc, acc);
+              tc_mma_bf16_pair(d1, a1 + aoff, bd + boff, idesc, acc);
+            }
+            tc_commit_pair_mc(aempty(it % C::SA), 0x3);
+            tc_commit_pair_mc(bempty(it % C::SB), 0x3);
+          }
+          if (!ok) break;
+          tc_commit_pair_mc(tfull(buf), 0x3);
+        }
+        tc_commit_pair_mc(drain_bar, 0x1);
+        mbar_wait(drain_bar, 0, 100000000ull);
+      }
+    } else {
+      // ------------------------------------------------------------ relay (odd CTA)
+      if (lane == 0) {
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = pair; t < num_tiles && ok; t += npairs) {
+          for (int j = 0; j < nsteps; ++j, ++it) {
+            if (!mbar_wait(bfull(it % C::SB), (it / C::SB) & 1u)) {
+              set_status_site(p.status, QLORA_ERR_TIMEOUT, 106); ok = false; break;
+            }
+            mbar_arrive_cluster(mapa_shared(bready(it % C::SB), 0));
+          }
+        }
+      }
+    }
+  } else if (warp < 7) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const uint32_t q = warp & 3u;
+    const uint32_t row = q * 32 + lane;
+    const uint32_t tempty_remote0 = mapa_shared(tempty(0), 0), tempty_remote1 = mapa_shared(tempty(1), 0);
+    uint32_t tcount = 0;
+    for (int t = pair; t < num_tiles; t += npairs, ++tcount) {
+      const int mb = t / p.tiles_n, nb = t - mb * p.tiles_n;
+      const uint32_t buf = tcount & 1u, tph = (tcount >> 1) & 1u;
+      if (!mbar_wait_cluster(tfull(buf), tph)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 107); break; }
+      tc_fence_after();
+#pragma unroll 1
+      for (int a = 0; a < 2; ++a) {
+        const int grow = mb * 512 + a * 256 + int(rank) * 128 + int(row);
+        const uint32_t tbase = tmem_base + ((q * 32u) << 16) + buf * 256u + uint32_t(a) * 128u;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+          if (grow < p.M) {
+            uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) + int64_t(grow) * p.ld_out + nb * 128 + c * 32;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+              o.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+              o.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+              o.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+              reinterpret_cast<uint4*>(dst)[i] = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(buf ? tempty_remote1 : tempty_remote0);
+    }
+  } else {
+    // ------------------------------------------------------------ dequantizers (both CTAs)
+    const uint32_t dwarp = warp - 7;
+    const uint32_t group = dwarp / C::kWarpsPerGroup;              // owns B slot `group`
+    const uint32_t sub = dwarp % C::kWarpsPerGroup;
+    const uint32_t dt = sub * 32 + lane;                           // 0..63
+    uint32_t it = 0, ic = 0;
+    bool ok = true;
+    for (int t = pair; t < num_tiles && ok; t += npairs) {
+      const int nc0 = (t % p.tiles_n) * 128 + int(rank) * 64;
+      for (int j = 0; j < nsteps; ++j, ++it) {
+        const bool main_step = j < p.num_k_main;
+        const uint32_t my = main_step ? ic++ : 0u;
+        if ((it % C::SB) != group) continue;
+        const uint32_t sb = it % C::SB;
+        if (!mbar_wait(bempty(sb), ((it / C::SB) & 1u) ^ 1u)) {
+          set_status_site(p.status, QLORA_ERR_TIMEOUT, 118); ok = false; break;
+        }
+        if (main_step) {
+          if (!mbar_wait(cfull(my % C::SC), (my / C::SC) & 1u)) {
+            set_status_site(p.status, QLORA_ERR_TIMEOUT, 108); ok = false; break;
+          }
+          const uint8_t* cs = smem + c_slot(my);
+          dequant_block_pair(dt, cs, reinterpret_cast<const float*>(cs + C::kCodes), b_slot(it));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(cempty(my % C::SC));
+            mbar_arrive(bfull(sb));
+          }
+        } else if (lane == 0) {
+          // LoRA step: this group's slot is filled by TMA (one expect_tx arrival plus
+          // the other warp's plain arrival).
+          if (sub == 0) {
+            mbar_arrive_expect_tx(bfull(sb), C::kB);
+            tma_load_2d(b_slot(it), &tmBx, bfull(sb), (j - p.num_k_main) * 64, nc0);
+          } else {
+            mbar_arrive(bfull(sb));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+}
+
 // --------------------------------------------------------------- host side
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -372,6 +751,11 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool make_tmap_2d(CUtensorMap* m, const void* base, TmapType type, uint64_t inner, uint64_t outer,
                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  return make_tmap_2d_sw(m, base, type, inner, outer, row_bytes, box_inner, box_outer, swizzle128 ? 128 : 0);
+}
+
+bool make_tmap_2d_sw(CUtensorMap* m, const void* base, TmapType type, uint64_t inner, uint64_t outer,
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes) {
   auto fn = encode_fn();
   if (!fn) return false;
   CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -382,7 +766,9 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, TmapType type, uint64_t inne
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                  : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                  : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -412,6 +798,58 @@ static qlora_status launch_cfg(const GemmOperands& o, GemmParams p, int ctas_per
   const int grid = std::max(1, std::min(num_tiles, num_sms() * ctas_per_sm));
   tc_gemm_kernel<C><<<grid, C::kThreads, C::kSmem, s>>>(o.A, o.B, o.codes, o.scales, o.Ax, o.Bx, p);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+template <class C>
+static qlora_status launch_pair_cfg(const GemmOperands& o, GemmParams p, cudaStream_t s) {
+  static bool attr_set = false;
+  static int max_pairs = 0;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(tc_gemm_nf4_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+        cudaSuccess)
+      return QLORA_ERR_CUDA;
+    cudaLaunchConfig_t qc = {};
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    qc.gridDim = dim3(2 * 74, 1, 1);
+    qc.blockDim = dim3(C::kThreads, 1, 1);
+    qc.dynamicSmemBytes = C::kSmem;
+    qc.attrs = qa;
+    qc.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_nf4_pair_kernel<C>, &qc) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    max_pairs = n;
+    attr_set = true;
+  }
+  p.bn = 128;
+  const int num_tiles = p.tiles_m * p.tiles_n;
+  const int pairs = std::max(1, std::min(num_tiles, max_pairs));
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, tc_gemm_nf4_pair_kernel<C>, o.A, o.codes, o.scales, o.Ax, o.Bx, p) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status launch_gemm_pair(bool dx, const GemmOperands& o, const GemmParams& p, cudaStream_t s) {
+  if (!dx) return launch_pair_cfg<PairCfg<false>>(o, p, s);
+  return launch_pair_cfg<PairCfg<true>>(o, p, s);
 }
 
 qlora_status launch_gemm(GemmKind kind, int bn, const GemmOperands& o, const GemmParams& p, cudaStream_t s) {

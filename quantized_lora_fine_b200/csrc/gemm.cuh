@@ -21,6 +21,15 @@ struct GemmParams {
   int64_t ld_out;
   int64_t split_stride;   // elements between split partials
   int* status;            // device status word
+  // Fused split-K reduction (thin products): when counters != nullptr, the last
+  // CTA to finish a tile sums the split partials in split order and writes
+  //   fin_mode 0: bf16 [M x N]            fin_mode 1: fp32 [M x N] * fin_scale
+  //   fin_mode 2: fp32 [N x M] * fin_scale (transposed)
+  // Counters (one int per M tile) must start at zero; the kernel leaves them zero.
+  int* counters;
+  void* fin_out;
+  int fin_mode;
+  float fin_scale;
 };
 
 struct GemmOperands {
@@ -43,7 +52,16 @@ enum class TmapType { BF16, U8, F32 };
 // `row_bytes` between rows; box of box_inner x box_outer elements.
 bool make_tmap_2d(CUtensorMap* m, const void* base, TmapType type, uint64_t inner, uint64_t outer,
                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+// Same with an explicit swizzle: 0 none, 32, 64 or 128 (bytes).
+bool make_tmap_2d_sw(CUtensorMap* m, const void* base, TmapType type, uint64_t inner, uint64_t outer,
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes);
 
 qlora_status launch_gemm(GemmKind kind, int bn, const GemmOperands& o, const GemmParams& p, cudaStream_t s);
+
+// Fused NF4 GEMM on CTA pairs (256 x 256 tiles). Operands: A (box 64 x 128),
+// codes (fwd: box 32 B x 128 rows; dX: box 64 B x 64 rows, 64-byte swizzle),
+// scales (fwd: box 128 x 1; dX: box 64 x 2), Ax (box 64 x 128), Bx (box 64 x 128).
+// Requires N % 256 == 0.
+qlora_status launch_gemm_pair(bool dx, const GemmOperands& o, const GemmParams& p, cudaStream_t s);
 
 }  // namespace qlb

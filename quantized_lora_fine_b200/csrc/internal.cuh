@@ -11,9 +11,21 @@ namespace qlb {
 constexpr int kBlock = 64;        // NF4 block (elements per absmax)
 constexpr int kDQBlock = 256;     // absmax values per second-level scale
 constexpr size_t kStatusBytes = 256;
+// Workspace layout shared by every entry point: [0, 256) status word,
+// [256, 256 + 64 KiB) split-K tile counters (only ever used as counters, which
+// the kernels return to zero), then per-call scratch.
+constexpr size_t kCounterBytes = 65536;
+constexpr size_t kReservedBytes = kStatusBytes + kCounterBytes;
+constexpr int64_t kMaxCounterTiles = int64_t(kCounterBytes / 4);
 
 __device__ __forceinline__ void set_status(int* st, int code) {
   if (st) atomicCAS(st, 0, code);
+}
+
+// Records the first error and, next to it, which wait gave up (a site number
+// chosen by the kernel), for diagnosing a stalled pipeline.
+__device__ __forceinline__ void set_status_site(int* st, int code, int site) {
+  if (st && atomicCAS(st, 0, code) == 0) atomicExch(st + 1, site);
 }
 
 // ---- codec.cu
@@ -29,13 +41,6 @@ qlora_status launch_expand_scales(const uint8_t* unused, const float* absmax, co
 // dst[n][q] = bf16(s * src[q][n]), src r x cols (transpose = 1)
 qlora_status launch_scale_lora(const uint16_t* src, int64_t rows, int64_t cols, float scale, bool transpose,
                                uint16_t* dst, cudaStream_t s);
-// out[m][c] = bf16(sum_p part[p][m][c])
-qlora_status launch_reduce_bf16(const float* part, int splits, int64_t rows, int64_t cols, uint16_t* out,
-                                cudaStream_t s);
-// out = scale * sum_p part[p]; transpose: part is [rows x cols], out is [cols x rows]
-qlora_status launch_reduce_f32(const float* part, int splits, int64_t rows, int64_t cols, float scale,
-                               bool transpose, float* out, cudaStream_t s);
-
 // ---- layer_error.cu
 size_t layer_error_ws_bytes(int n_layers, const int64_t* numel);
 qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,

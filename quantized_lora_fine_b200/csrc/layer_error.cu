@@ -25,6 +25,30 @@ struct LayerTable {
   int32_t n_layers;
 };
 
+// Error contribution of 8 bf16 weights of one block: codes from the exact absmax
+// a, reconstruction with ahat (= a, or the double-quantized scale). w and w_hat
+// are bf16 values within a small exponent range of each other (or w_hat = 0),
+// so d = w - w_hat and the squares d^2, w^2 are exact in fp32; the 8-term
+// partial sums carry at most 8 roundings before they are added in fp64.
+__device__ __forceinline__ void err8_bf16(uint4 v, float a, float ahat, const NF4CellSmem& cells, const float* s_code,
+                                          float& sd8, float& sw8) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  uint32_t idx[8];
+  if (a > 0.f) quant8_bf16(v, a, cells, idx);
+  else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) idx[i] = 7u;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float w = (i & 1) ? __uint_as_float(u[i >> 1] & 0xFFFF0000u) : __uint_as_float(u[i >> 1] << 16);
+    const float wh = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_code[idx[i]], ahat)));
+    const float d = __fsub_rn(w, wh);
+    sd8 = __fmaf_rn(d, d, sd8);
+    sw8 = __fmaf_rn(w, w, sw8);
+  }
+}
+
 template <bool DQ>
 __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_constant__ LayerTable tab,
                                                                 double2* __restrict__ partial, int* status) {
@@ -33,43 +57,45 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
   __shared__ float s_red[8];
   __shared__ float s_code[16];
   __shared__ double s_sum[2][8];
+  __shared__ NF4CellSmem s_cells;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  nf4_cells_load(s_cells, tid);
+  if (tid < 16) s_code[tid] = nf4_code(tid);
   const int chunk = blockIdx.x;
-  // find the layer owning this chunk
-  int lo = 0, hi = tab.n_layers - 1;
+  int lo = 0, hi = tab.n_layers - 1;  // layer owning this chunk
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (tab.first_chunk[mid] <= chunk) lo = mid; else hi = mid - 1;
   }
-  const int layer = lo;
-  const uint16_t* W = tab.ptr[layer];
-  const int64_t numel = tab.numel[layer];
-  const int64_t g = chunk - tab.first_chunk[layer];
-  const int64_t nb = numel / kBlock;
-  if (tid < 16) s_code[tid] = nf4_code(tid);
-
+  const uint16_t* W = tab.ptr[lo];
+  const int64_t nb = tab.numel[lo] / kBlock;
+  const int64_t g = chunk - tab.first_chunk[lo];
+  auto load = [&](int it) -> uint4 {
+    const int64_t blk = g * kDQBlock + it * 32 + warp * 4 + (lane >> 3);
+    return (blk < nb) ? __ldg(reinterpret_cast<const uint4*>(W + blk * kBlock + (lane & 7) * 8)) : make_uint4(0, 0, 0, 0);
+  };
   uint4 raw[8];
+#pragma unroll
+  for (int it = 0; it < 8; ++it) raw[it] = load(it);
+  __syncthreads();
+  uint32_t bad = 0;
+  double sd = 0.0, sw = 0.0;
   float am_slice[8];
-  bool bad = false;
 #pragma unroll
   for (int it = 0; it < 8; ++it) {
     const int bi = it * 32 + warp * 4 + (lane >> 3);
-    const int64_t blk = g * kDQBlock + bi;
-    raw[it] = make_uint4(0, 0, 0, 0);
-    if (blk < nb) raw[it] = __ldg(reinterpret_cast<const uint4*>(W + blk * kBlock + (lane & 7) * 8));
-    const uint32_t u[4] = {raw[it].x, raw[it].y, raw[it].z, raw[it].w};
-    float am = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float a0 = fabsf(bf16_lo(u[i])), a1 = fabsf(bf16_hi(u[i]));
-      bad |= !(a0 <= FLT_MAX) || !(a1 <= FLT_MAX);
-      am = fmaxf(am, fmaxf(a0, a1));
-    }
-    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+    const uint32_t amb = block_max8_lanes(absmax8_bf16_bits(raw[it]));
+    bad |= amb >= 0x7F80u;
+    const float am = __uint_as_float(amb << 16);
     am_slice[it] = am;
-    if ((lane & 7) == 0) s_amax[bi] = am;
+    if constexpr (DQ) {
+      if ((lane & 7) == 0) s_amax[bi] = am;
+    } else {
+      float sd8 = 0.f, sw8 = 0.f;
+      err8_bf16(raw[it], am, am, s_cells, s_code, sd8, sw8);
+      sd += double(sd8);
+      sw += double(sw8);
+    }
   }
   if (bad) set_status(status, QLORA_ERR_NONFINITE);
   if constexpr (DQ) {
@@ -90,23 +116,14 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
       ah = __fmul_rn(e4m3_to_f32(q), __fdiv_rn(G, 448.f));
     }
     s_ahat[tid] = ah;
-  }
-  __syncthreads();
-  double sd = 0.0, sw = 0.0;
+    __syncthreads();
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int bi = it * 32 + warp * 4 + (lane >> 3);
-    const float a = am_slice[it];
-    const float ahat = DQ ? s_ahat[bi] : a;
-    const uint32_t u[4] = {raw[it].x, raw[it].y, raw[it].z, raw[it].w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float w = (i & 1) ? bf16_hi(u[i >> 1]) : bf16_lo(u[i >> 1]);
-      const uint32_t j = (a > 0.f) ? nf4_index(__fdiv_rn(w, a)) : 7u;
-      const float wh = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_code[j], ahat)));
-      const double d = double(w) - double(wh);
-      sd = fma(d, d, sd);
-      sw = fma(double(w), double(w), sw);
+    for (int it = 0; it < 8; ++it) {
+      const int bi = it * 32 + warp * 4 + (lane >> 3);
+      float sd8 = 0.f, sw8 = 0.f;
+      err8_bf16(raw[it], am_slice[it], s_ahat[bi], s_cells, s_code, sd8, sw8);
+      sd += double(sd8);
+      sw += double(sw8);
     }
   }
 #pragma unroll
@@ -123,13 +140,21 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
   }
 }
 
-__global__ void layer_error_finish_kernel(const double2* __restrict__ partial, const int32_t* __restrict__ first,
-                                          int n_layers, double* __restrict__ err) {
-  const int l = blockIdx.x * blockDim.x + threadIdx.x;
-  if (l >= n_layers) return;
-  double sd = 0.0, sw = 0.0;
-  for (int c = first[l]; c < first[l + 1]; ++c) { sd += partial[c].x; sw += partial[c].y; }
-  err[l] = (sw > 0.0) ? sqrt(sd / sw) : 0.0;
+// One CTA per layer: thread t sums chunks first+t, first+t+256, ... in order, then a
+// fixed-shape tree combines the 256 partials -- deterministic for a given layout.
+__device__ __forceinline__ void finish_layer(const double2* __restrict__ partial, int c0, int c1,
+                                             double* __restrict__ err_out) {
+  __shared__ double s_a[256], s_b[256];
+  double a = 0.0, b = 0.0;
+  for (int c = c0 + threadIdx.x; c < c1; c += 256) { a += partial[c].x; b += partial[c].y; }
+  s_a[threadIdx.x] = a;
+  s_b[threadIdx.x] = b;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) { s_a[threadIdx.x] += s_a[threadIdx.x + o]; s_b[threadIdx.x] += s_b[threadIdx.x + o]; }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *err_out = (s_b[0] > 0.0) ? sqrt(s_a[0] / s_b[0]) : 0.0;
 }
 
 __global__ void __launch_bounds__(1024) rank_topk_kernel(const double* __restrict__ err, int n_layers, int K,
@@ -149,6 +174,10 @@ __global__ void __launch_bounds__(1024) rank_topk_kernel(const double* __restric
   }
 }
 
+__global__ void __launch_bounds__(256) layer_error_finish_table_kernel(const double2* __restrict__ partial,
+                                                                       const __grid_constant__ LayerTable tab,
+                                                                       double* __restrict__ err);
+
 static int32_t chunks_of(int64_t numel) {
   const int64_t nb = numel / kBlock;
   return static_cast<int32_t>((nb + kDQBlock - 1) / kDQBlock);
@@ -157,13 +186,17 @@ static int32_t chunks_of(int64_t numel) {
 size_t layer_error_ws_bytes(int n_layers, const int64_t* numel) {
   int64_t chunks = 0;
   for (int i = 0; i < n_layers; ++i) chunks += chunks_of(numel[i]);
-  return kStatusBytes + size_t(chunks) * sizeof(double2) + size_t(n_layers + 1) * sizeof(int32_t) + 256;
+  return kReservedBytes + size_t(chunks) * sizeof(double2);
 }
 
 qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
                                      int K, double* err, int32_t* order, uint8_t* keep, void* ws, size_t ws_bytes,
                                      int* status, cudaStream_t s) {
-  static LayerTable tab;  // host staging of the by-value kernel parameter
+  // The chunk table travels as a by-value kernel parameter (no host-to-device
+  // copy), so this call can be captured into a CUDA graph.
+  static std::mutex mu;
+  static LayerTable tab;
+  std::lock_guard<std::mutex> lock(mu);
   tab.n_layers = n_layers;
   int32_t c = 0;
   for (int i = 0; i < n_layers; ++i) {
@@ -174,16 +207,11 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
   }
   tab.first_chunk[n_layers] = c;
   if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
-  char* base = static_cast<char*>(ws) + kStatusBytes;
-  double2* partial = reinterpret_cast<double2*>(base);
-  int32_t* first_dev = reinterpret_cast<int32_t*>(base + size_t(c) * sizeof(double2));
-  if (cudaMemcpyAsync(first_dev, tab.first_chunk, size_t(n_layers + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, s) !=
-      cudaSuccess)
-    return QLORA_ERR_CUDA;
+  double2* partial = reinterpret_cast<double2*>(static_cast<char*>(ws) + kReservedBytes);
   if (dq) layer_error_chunk_kernel<true><<<unsigned(c), 256, 0, s>>>(tab, partial, status);
   else layer_error_chunk_kernel<false><<<unsigned(c), 256, 0, s>>>(tab, partial, status);
   if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
-  layer_error_finish_kernel<<<(n_layers + 255) / 256, 256, 0, s>>>(partial, first_dev, n_layers, err);
+  layer_error_finish_table_kernel<<<n_layers, 256, 0, s>>>(partial, tab, err);
   rank_topk_kernel<<<1, 1024, 0, s>>>(err, n_layers, K, order, keep);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
@@ -203,13 +231,12 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
 constexpr int64_t kNoAllocMaxChunks = int64_t(1) << 20;
 static __device__ __align__(256) double2 g_noalloc_partials[kNoAllocMaxChunks];
 
-__global__ void layer_error_finish_table_kernel(const double2* __restrict__ partial,
-                                                const __grid_constant__ LayerTable tab, double* __restrict__ err) {
-  const int l = blockIdx.x * blockDim.x + threadIdx.x;
+__global__ void __launch_bounds__(256) layer_error_finish_table_kernel(const double2* __restrict__ partial,
+                                                                       const __grid_constant__ LayerTable tab,
+                                                                       double* __restrict__ err) {
+  const int l = blockIdx.x;
   if (l >= tab.n_layers) return;
-  double sd = 0.0, sw = 0.0;
-  for (int c = tab.first_chunk[l]; c < tab.first_chunk[l + 1]; ++c) { sd += partial[c].x; sw += partial[c].y; }
-  err[l] = (sw > 0.0) ? sqrt(sd / sw) : 0.0;
+  finish_layer(partial, tab.first_chunk[l], tab.first_chunk[l + 1], err + l);
 }
 
 namespace {
@@ -254,7 +281,7 @@ qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const
   if (dq) layer_error_chunk_kernel<true><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr);
   else layer_error_chunk_kernel<false><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr);
   if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
-  layer_error_finish_table_kernel<<<(n_layers + 255) / 256, 256, 0, s>>>(partial, tab, err);
+  layer_error_finish_table_kernel<<<n_layers, 256, 0, s>>>(partial, tab, err);
   rank_topk_kernel<<<1, 1024, 0, s>>>(err, n_layers, K, order, keep);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }

@@ -18,6 +18,103 @@ __device__ __forceinline__ uint32_t nf4_index(float n) {
   return idx;
 }
 
+// Shared-memory copy of the cell tables (64 thresholds + 64 base indices).
+struct NF4CellSmem {
+  float thr[64];
+  uint32_t base[64];
+};
+
+__device__ __forceinline__ void nf4_cells_load(NF4CellSmem& t, int tid) {
+  if (tid < 64) {
+    t.thr[tid] = __uint_as_float(kNF4CellThrBits[tid]);
+    t.base[tid] = kNF4CellBase[tid];
+  }
+}
+
+// Same result as nf4_index(n) for every fp32 n (NaN maps to some index; callers
+// flag non-finite input separately): the cell of n holds at most one midpoint.
+__device__ __forceinline__ uint32_t nf4_index_cell(float n, const NF4CellSmem& t) {
+  const uint32_t c = (__float_as_uint(__fadd_rn(n, 3.0f)) >> 18) & 63u;
+  return t.base[c] + ((n > t.thr[c]) ? 1u : 0u);
+}
+
+// Correctly rounded w / a from r = RN(1/a) with one residual correction
+// (Markstein's division step: q0 = RN(w r), e = w - q0 a exactly by FMA,
+// q = RN(q0 + e r)). Requires a normal, finite a with 1/a normal; the callers
+// rescale tiny blocks by 2^64 first. Checked against IEEE division for every
+// (bf16 w, bf16 a) significand / exponent-gap combination by the GPU tests.
+__device__ __forceinline__ float div_by_recip(float w, float a, float r) {
+  const float q0 = __fmul_rn(w, r);
+  const float e = __fmaf_rn(-q0, a, w);
+  return __fmaf_rn(e, r, q0);
+}
+
+// Normalised value n = RN(w / a) for a block with absmax a > 0. bf16 inputs take
+// the reciprocal path (exact for every bf16 pair, see div_by_recip); fp32 inputs
+// use IEEE division directly.
+template <typename T>
+struct BlockDiv {
+  float a, r;
+  __device__ __forceinline__ BlockDiv(float am) {
+    // Tiny blocks: rescale by 2^64 (exact) so that 1/a stays a normal number.
+    a = (am < 0x1p-100f) ? am * 0x1p64f : am;
+    r = __frcp_rn(a);
+  }
+  __device__ __forceinline__ float operator()(float w, float am) const {
+    if constexpr (sizeof(T) == 2) {
+      return div_by_recip((am < 0x1p-100f) ? w * 0x1p64f : w, a, r);
+    } else {
+      return __fdiv_rn(w, am);
+    }
+  }
+};
+
+// bf16 bit pattern of max |w| over 8 elements held as 4 packed bf16 pairs.
+// Comparing magnitudes as unsigned integers orders +Inf and NaN above every
+// finite value, so a result >= 0x7F80 flags a non-finite element.
+__device__ __forceinline__ uint32_t absmax8_bf16_bits(uint4 v) {
+  const uint32_t a = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+  const uint32_t b = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
+  const uint32_t m = __vmaxu2(a, b);
+  return max(m >> 16, m & 0xFFFFu);
+}
+
+// Max over the 8 lanes (l ^ 1, l ^ 2, l ^ 4) that share one 64-element block.
+__device__ __forceinline__ uint32_t block_max8_lanes(uint32_t v) {
+  v = max(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  v = max(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  v = max(v, __shfl_xor_sync(0xffffffffu, v, 4));
+  return v;
+}
+
+// Codes of 8 bf16 weights (4 packed pairs) of a block with absmax a > 0, packed in
+// storage order (byte k = idx[2k] << 4 | idx[2k + 1]).
+__device__ __forceinline__ uint32_t quant8_bf16(uint4 v, float a, const NF4CellSmem& cells, uint32_t (&idx)[8]) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  float w[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) { w[2 * i] = __uint_as_float(u[i] << 16); w[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u); }
+  float as = a;
+  if (a < 0x1p-100f) {  // tiny block: rescale by 2^64 (exact) so that 1/a stays normal
+    as = a * 0x1p64f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] *= 0x1p64f;
+  }
+  const float r = __frcp_rn(as);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) idx[i] = nf4_index_cell(div_by_recip(w[i], as, r), cells);
+  // byte k = idx[2k] << 4 | idx[2k+1]; integer multiply-adds keep this off the ALU pipe
+  uint32_t word = idx[1];
+  word = idx[0] * 16u + word;
+  word = idx[3] * 256u + word;
+  word = idx[2] * 4096u + word;
+  word = idx[5] * 65536u + word;
+  word = idx[4] * 1048576u + word;
+  word = idx[7] * 16777216u + word;
+  word = idx[6] * 268435456u + word;
+  return word;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

@@ -80,3 +80,27 @@ def test_nonfinite_sets_status(cuda_device):
     assert api.read_status(ws) == 8
     api.reset_status(ws)
     assert api.read_status(ws) == 0
+
+
+def _exhaustive_blocks(exp: int, sigs) -> np.ndarray:
+    """Blocks [a, x_1..x_63] for every bf16 x with |x| <= a, a = (1 + s/128) 2^exp."""
+    allb = nf4.f32_from_bf16_bits(np.arange(65536, dtype=np.uint32).astype(np.uint16))
+    allb = allb[np.isfinite(allb)]
+    blocks = []
+    for s in sigs:
+        a = np.float32((1 + s / 128.0) * 2.0 ** exp)
+        x = allb[np.abs(allb) <= a]
+        pad = (-x.size) % 63
+        x = np.concatenate([x, np.zeros(pad, np.float32)]).reshape(-1, 63)
+        blocks.append(np.concatenate([np.full((x.shape[0], 1), a, np.float32), x], axis=1))
+    return np.concatenate(blocks)
+
+
+@pytest.mark.parametrize("exp,sigs", [(0, range(128)), (-120, range(0, 128, 9)), (100, range(0, 128, 13))])
+def test_quant_every_bf16_pair(cuda_device, exp, sigs):
+    """Every (bf16 w, bf16 absmax) significand pair and exponent gap: the GPU's
+    reciprocal-based division and cell-table code lookup give the oracle's codes
+    (IEEE division, 15 midpoint comparisons)."""
+    W32 = _exhaustive_blocks(exp, sigs)
+    Wb = synth.from_bf16_bits(nf4.bf16_bits_from_f32(W32))
+    _check_quant(Wb, dq=False)
