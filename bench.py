@@ -324,8 +324,9 @@ def gpu_main(args):
     fwd_tf = fl_fwd_gemm / (med["fwd_gemm"] * 1e-3) / 1e12
     dx_tf = fl_dx_gemm / (med["dx_gemm"] * 1e-3) / 1e12
     # dominant kernel = the longer of the two fused GEMMs
-    dom = ("qlora_fwd_gemm (tc_gemm_kernel FwdNF4)", fwd_tf, med["fwd_gemm"]) if med["fwd_gemm"] >= med["dx_gemm"] \
-        else ("qlora_bwd_dx_gemm (tc_gemm_kernel DxNF4)", dx_tf, med["dx_gemm"])
+    engine = "tc_gemm_kernel" if os.environ.get("QLORA_B200_GEMM") == "1cta" else "tc_gemm_nf4_pair_kernel"
+    dom = (f"qlora_fwd_gemm ({engine} fwd)", fwd_tf, med["fwd_gemm"]) if med["fwd_gemm"] >= med["dx_gemm"] \
+        else (f"qlora_bwd_dx_gemm ({engine} dX)", dx_tf, med["dx_gemm"])
     numel = h * o
     quant_bytes = numel * 2 + numel // 2 + numel // 64 + 4 * (numel // 64 // 256)
     err_bytes = numel * 2

@@ -181,14 +181,14 @@ void record_prof(cudaEvent_t e, cudaStream_t s) {
     cudaEventRecord(e, s);
 }
 
-// The NF4 GEMMs run on the single-CTA kernel unless QLORA_B200_GEMM=pair selects
-// the CTA-pair kernel (both compute the same values; kept side by side for
+// The NF4 GEMMs run on the CTA-pair kernel unless QLORA_B200_GEMM=1cta selects
+// the single-CTA kernel (both compute the same values; kept side by side for
 // measurement).
 bool use_pair_kernel() {
   static int v = -1;
   if (v < 0) {
     const char* e = std::getenv("QLORA_B200_GEMM");
-    v = (e && std::strcmp(e, "pair") == 0) ? 1 : 0;
+    v = (e && std::strcmp(e, "1cta") == 0) ? 0 : 1;
   }
   return v == 1;
 }

@@ -282,7 +282,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tcount) {
       const TileInfo ti = decode_tile(p, t);
       const uint32_t acc = tcount & 1u, tph = (tcount >> 1) & 1u;
-      if (!mbar_wait(tfull_bar(acc), tph)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 5); break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(acc), tph))) {
+        set_status_site(p.status, QLORA_ERR_TIMEOUT, 5); break;
+      }
       tc_fence_after();
       const int grow = ti.m0 + int(row);
       const uint32_t tbase = tmem_base + ((q * 32u) << 16) + acc * C::BN;
@@ -374,7 +376,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         for (int j = 0; j < nsteps; ++j, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!mbar_wait(full_bar(s), ph)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 6); ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph))) {
+            set_status_site(p.status, QLORA_ERR_TIMEOUT, 6); ok = false; break;
+          }
           if (j < ti.ke - ti.kb) {
             uint8_t* st = smem + s * C::kStage;
             dequant_stage<C::B_MN>(dt, st + C::kCodesOff, reinterpret_cast<const float*>(st + C::kScalesOff),
@@ -402,42 +406,43 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 // One pair tile is 512 (M) x 128 (N): two M = 256 accumulators share every
 // dequantized B tile, so each SM dequantizes one weight per 512 output rows.
 //
-// Shared memory holds three rings so that the dequantization latency does not
-// sit inside the A operand's load-to-release cycle:
-//   A ring (SA slots)  A0, A1: this CTA's 128-row halves of the two 256-row MMA
-//                      tiles (or the LoRA T/U rows in the extension steps)
-//   C ring (SC slots)  packed codes + expanded scales of this CTA's half of B;
-//                      loaded ahead of the A ring, consumed by the dequantizers
-//   B ring (SB slots)  bf16 B half (64 rows fwd / 64 columns dX), read by MMA
-// Every ring slot has exactly one writer that fills its rounds in order (the A
-// producer, the C producer, and dequantizer group g for B slot g, which also
-// issues the TMA load of the LoRA steps' B tile), so a parity wait can never be
-// satisfied by a phase two rounds old.
-// Warp roles: 0 A producer, 1 MMA issuer (even CTA) / relay (odd CTA) and TMEM
-// allocation, 2 C producer, 3-6 epilogue, 7.. dequantizer groups. The odd CTA's
-// relay forwards "B slot ready" to the even CTA once per step (one
-// cluster-scope release per step).
+// Shared memory per CTA:
+//   S slots   A0, A1 (this CTA's 128-row halves of the two 256-row MMA tiles,
+//             or the LoRA T/U rows in the extension steps) and this CTA's bf16
+//             half of B (64 rows fwd / 64 columns dX)
+//   SC slots  packed codes + expanded scales of that B half, loaded ahead
+// Slot s of step `it` is it % S. Every slot has exactly one writer per role
+// (the A producer for A, dequantizer warp it % S for B, which also issues the
+// TMA of the LoRA steps' B tile) and all writers wait for the slot's previous
+// round to be consumed, so a parity wait never matches a phase two rounds old.
+//
+// Barriers (same offsets in both CTAs):
+//   ready[s]  even CTA: A bytes (TMA) + its slot owners + the odd CTA's slot
+//             owner (remote arrival, sent after the odd CTA's own ready[s]
+//             completed); odd CTA: A bytes + its slot owners
+//   empty[s]  one multicast tcgen05.commit per step from the even CTA's MMA
+//   cfull / cempty   code ring
+//   tfull[b] / tempty[b]  accumulator double buffer
+// Warp roles: 0 A producer, 1 MMA issuer (even CTA) and TMEM allocation, 2 C
+// producer, 3-6 epilogue, 7.. dequantizers (kWarpsPerSlot warps per slot).
 
 template <bool B_MN_>
 struct PairCfg {
   static constexpr bool B_MN = B_MN_;
-  static constexpr int SA = 5, SB = 4, SC = 8;
+  static constexpr int S = 5, SC = 8;
   static constexpr int kA = 128 * 64 * 2;       // one 128-row A tile: 16 KB
-  static constexpr int kASlot = 2 * kA;         // A0 + A1
   static constexpr int kB = 64 * 64 * 2;        // 8 KB
+  static constexpr int kSlot = 2 * kA + kB;     // 40 KB
   static constexpr int kCodes = 64 * 32;        // 2 KB
   static constexpr int kScales = 64 * 4;        // 256 B
   static constexpr int kCSlot = 3072;
-  static constexpr int kAOff = 0;
-  static constexpr int kBOff = kAOff + SA * kASlot;
-  static constexpr int kCOff = kBOff + SB * kB;
+  static constexpr int kCOff = S * kSlot;
   static constexpr int kBarOff = kCOff + SC * kCSlot;
-  static constexpr int kGroups = SB;            // group g owns B slot g
-  static constexpr int kWarpsPerGroup = 2;      // 64 threads: one 64-element block each per step
-  static constexpr int kDeqWarps = kGroups * kWarpsPerGroup;
+  static constexpr int kWarpsPerSlot = 2;       // the warps of slot w dequantize 32 rows each
+  static constexpr int kDeqWarps = S * kWarpsPerSlot;
   static constexpr int kThreads = (7 + kDeqWarps) * 32;
   static constexpr int kTmemCols = 512;         // 2 buffers x 2 accumulators x 128 columns
-  static constexpr int kNumBars = 2 * SA + 2 * SC + 3 * SB + 5;
+  static constexpr int kNumBars = 2 * S + 2 * SC + 5;
   static constexpr int kSmem = kBarOff + 8 * kNumBars + 16 + 1024;
   static_assert(kSmem <= 232448, "shared memory budget");
 };
@@ -472,33 +477,27 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t bar_base = smem_base + C::kBarOff;
-  auto afull = [&](int i) { return bar_base + 8u * i; };
-  auto aempty = [&](int i) { return bar_base + 8u * (C::SA + i); };
-  auto cfull = [&](int i) { return bar_base + 8u * (2 * C::SA + i); };
-  auto cempty = [&](int i) { return bar_base + 8u * (2 * C::SA + C::SC + i); };
-  auto bfull = [&](int i) { return bar_base + 8u * (2 * C::SA + 2 * C::SC + i); };
-  auto bready = [&](int i) { return bar_base + 8u * (2 * C::SA + 2 * C::SC + C::SB + i); };
-  auto bempty = [&](int i) { return bar_base + 8u * (2 * C::SA + 2 * C::SC + 2 * C::SB + i); };
-  const int kT0 = 2 * C::SA + 2 * C::SC + 3 * C::SB;
+  auto ready = [&](int i) { return bar_base + 8u * i; };
+  auto empty = [&](int i) { return bar_base + 8u * (C::S + i); };
+  auto cfull = [&](int i) { return bar_base + 8u * (2 * C::S + i); };
+  auto cempty = [&](int i) { return bar_base + 8u * (2 * C::S + C::SC + i); };
+  const int kT0 = 2 * C::S + 2 * C::SC;
   auto tfull = [&](int b) { return bar_base + 8u * (kT0 + b); };
   auto tempty = [&](int b) { return bar_base + 8u * (kT0 + 2 + b); };
   const uint32_t drain_bar = bar_base + 8u * (kT0 + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * C::kNumBars);
-  auto a_slot = [&](uint32_t i) { return smem_base + C::kAOff + (i % C::SA) * C::kASlot; };
-  auto b_slot = [&](uint32_t i) { return smem_base + C::kBOff + (i % C::SB) * C::kB; };
-  auto c_slot = [&](uint32_t i) { return C::kCOff + (i % C::SC) * C::kCSlot; };  // offset from smem
+  auto slot = [&](uint32_t i) { return smem_base + (i % C::S) * C::kSlot; };          // A0 | A1 | B
+  auto c_off = [&](uint32_t i) { return C::kCOff + (i % C::SC) * C::kCSlot; };         // from smem
 
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::SA; ++i) { mbar_init(afull(i), 1); mbar_init(aempty(i), 1); }
-    for (int i = 0; i < C::SC; ++i) { mbar_init(cfull(i), 1); mbar_init(cempty(i), C::kWarpsPerGroup); }
-    for (int i = 0; i < C::SB; ++i) {
-      mbar_init(bfull(i), C::kWarpsPerGroup);
-      mbar_init(bready(i), 1);
-      mbar_init(bempty(i), 1);
+    for (int i = 0; i < C::S; ++i) {
+      mbar_init(ready(i), 1 + C::kWarpsPerSlot + (rank == 0 ? 1 : 0));
+      mbar_init(empty(i), 1);
     }
+    for (int i = 0; i < C::SC; ++i) { mbar_init(cfull(i), 1); mbar_init(cempty(i), C::kWarpsPerSlot); }
     for (int b = 0; b < 2; ++b) { mbar_init(tfull(b), 1); mbar_init(tempty(b), 8); }
     mbar_init(drain_bar, 1);
     fence_mbarrier_init();
@@ -525,47 +524,36 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += npairs) {
-        const int mb = t / p.tiles_n;
-        const int m0 = mb * 512 + int(rank) * 128;
+        const int m0 = (t / p.tiles_n) * 512 + int(rank) * 128;
         for (int j = 0; j < nsteps; ++j, ++it) {
-          if (!mbar_wait(aempty(it % C::SA), ((it / C::SA) & 1u) ^ 1u)) {
+          if (!mbar_wait(empty(it % C::S), ((it / C::S) & 1u) ^ 1u)) {
             set_status_site(p.status, QLORA_ERR_TIMEOUT, 101); ok = false; break;
           }
-          const uint32_t dst = a_slot(it), bar = afull(it % C::SA);
-          mbar_arrive_expect_tx(bar, C::kASlot);
-          if (j < p.num_k_main) {
-            tma_load_2d(dst, &tmA, bar, j * 64, m0);
-            tma_load_2d(dst + C::kA, &tmA, bar, j * 64, m0 + 256);
-          } else {
-            const int kx = (j - p.num_k_main) * 64;
-            tma_load_2d(dst, &tmAx, bar, kx, m0);
-            tma_load_2d(dst + C::kA, &tmAx, bar, kx, m0 + 256);
-          }
+          const uint32_t dst = slot(it), bar = ready(it % C::S);
+          mbar_arrive_expect_tx(bar, 2 * C::kA);
+          const CUtensorMap* m = (j < p.num_k_main) ? &tmA : &tmAx;
+          const int kx = (j < p.num_k_main ? j : j - p.num_k_main) * 64;
+          tma_load_2d(dst, m, bar, kx, m0);
+          tma_load_2d(dst + C::kA, m, bar, kx, m0 + 256);
         }
       }
-      if (it > 0) {  // let the last copies land before leaving
-        for (int k = 0; k < C::SA && k < int(it); ++k) {
-          const uint32_t i2 = it - 1 - k;
-          mbar_wait(afull(i2 % C::SA), (i2 / C::SA) & 1u, 100000000ull);
-        }
-      }
+      // let the last copies land before leaving
+      mbar_wait(empty(it % C::S), ((it / C::S) & 1u) ^ 1u, 100000000ull);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ C producer (both CTAs)
     if (lane == 0) {
       tma_prefetch_desc(&tmCodes);
       tma_prefetch_desc(&tmScales);
-      uint32_t it = 0, ic = 0;
+      uint32_t ic = 0;
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += npairs) {
-        const int nb = t % p.tiles_n;
-        const int nc0 = nb * 128 + int(rank) * 64;
-        for (int j = 0; j < nsteps; ++j, ++it) {
-          if (j >= p.num_k_main) continue;
+        const int nc0 = (t % p.tiles_n) * 128 + int(rank) * 64;
+        for (int j = 0; j < p.num_k_main; ++j, ++ic) {
           if (!mbar_wait(cempty(ic % C::SC), ((ic / C::SC) & 1u) ^ 1u)) {
             set_status_site(p.status, QLORA_ERR_TIMEOUT, 102); ok = false; break;
           }
-          const uint32_t dst = smem_base + c_slot(ic), bar = cfull(ic % C::SC);
+          const uint32_t dst = smem_base + c_off(ic), bar = cfull(ic % C::SC);
           mbar_arrive_expect_tx(bar, C::kCodes + C::kScales);
           if constexpr (!C::B_MN) {
             tma_load_2d(dst, &tmCodes, bar, j * 32, nc0);
@@ -574,74 +562,53 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             tma_load_2d(dst, &tmCodes, bar, nc0 / 2, j * 64);
             tma_load_2d(dst + C::kCodes, &tmScales, bar, j * 64, nc0 / 64);
           }
-          ++ic;
         }
       }
-      if (ic > 0) {
-        for (int k = 0; k < C::SC && k < int(ic); ++k) {
-          const uint32_t i2 = ic - 1 - k;
-          mbar_wait(cfull(i2 % C::SC), (i2 / C::SC) & 1u, 100000000ull);
-        }
+      for (int k = 0; k < C::SC && k < int(ic); ++k) {
+        const uint32_t i2 = ic - 1 - k;
+        mbar_wait(cfull(i2 % C::SC), (i2 / C::SC) & 1u, 100000000ull);
       }
     }
   } else if (warp == 1) {
-    if (rank == 0) {
-      // ------------------------------------------------------------ MMA issuer (even CTA)
-      if (lane == 0) {
-        constexpr uint32_t idesc_main = make_idesc_bf16(256, 128, 0, C::B_MN ? 1 : 0);
-        constexpr uint32_t idesc_ext = make_idesc_bf16(256, 128, 0, 0);
-        constexpr uint32_t b_adv = C::B_MN ? 2048u : 32u;
-        uint32_t it = 0, tcount = 0;
-        bool ok = true;
-        for (int t = pair; t < num_tiles && ok; t += npairs, ++tcount) {
-          const uint32_t buf = tcount & 1u, tph = (tcount >> 1) & 1u;
-          if (!mbar_wait_cluster(tempty(buf), tph ^ 1u)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 104); ok = false; break; }
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc_main = make_idesc_bf16(256, 128, 0, C::B_MN ? 1 : 0);
+      constexpr uint32_t idesc_ext = make_idesc_bf16(256, 128, 0, 0);
+      constexpr uint32_t b_adv = C::B_MN ? (2048u >> 4) : (32u >> 4);
+      // descriptors are linear in the start address (bits 0..13 hold addr >> 4)
+      const uint64_t da0_base = make_smem_desc(slot(0), 16u, 1024u, kSwizzle128B);
+      const uint64_t db_base = make_smem_desc(slot(0) + 2 * C::kA, 16u, 1024u, kSwizzle128B);
+      constexpr uint64_t kA1Adv = uint64_t(C::kA >> 4), kSlotAdv = uint64_t(C::kSlot >> 4);
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += npairs, ++tcount) {
+        const uint32_t buf = tcount & 1u, tph = (tcount >> 1) & 1u;
+        if (!mbar_wait_cluster(tempty(buf), tph ^ 1u)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 104); ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + buf * 256u, d1 = d0 + 128u;
+        for (int j = 0; j < nsteps; ++j, ++it) {
+          const uint32_t si = it % C::S;
+          if (!mbar_wait_cluster(ready(si), (it / C::S) & 1u)) {
+            set_status_site(p.status, QLORA_ERR_TIMEOUT, 105); ok = false; break;
+          }
           tc_fence_after();
-          const uint32_t d0 = tmem_base + buf * 256u, d1 = d0 + 128u;
-          for (int j = 0; j < nsteps; ++j, ++it) {
-            const uint32_t pa = (it / C::SA) & 1u, pb = (it / C::SB) & 1u;
-            const int site = !mbar_wait(afull(it % C::SA), pa) ? 105
-                             : !mbar_wait(bfull(it % C::SB), pb) ? 115
-                             : !mbar_wait_cluster(bready(it % C::SB), pb) ? 125 : 0;
-            if (site) { set_status_site(p.status, QLORA_ERR_TIMEOUT, site); ok = false; break; }
-            tc_fence_after();
-            const bool ext = j >= p.num_k_main;
-            const uint32_t as = a_slot(it);
-            const uint64_t a0 = make_smem_desc(as, 16u, 1024u, kSwizzle128B);
-            const uint64_t a1 = make_smem_desc(as + C::kA, 16u, 1024u, kSwizzle128B);
-            const uint64_t bd = make_smem_desc(b_slot(it), 16u, 1024u, kSwizzle128B);
-            const uint32_t badv = ext ? 32u : b_adv;
-            const uint32_t idesc = ext ? idesc_ext : idesc_main;
+          const bool ext = j >= p.num_k_main;
+          const uint64_t a0 = da0_base + si * kSlotAdv, a1 = a0 + kA1Adv, bd = db_base + si * kSlotAdv;
+          const uint32_t badv = ext ? (32u >> 4) : b_adv;
+          const uint32_t idesc = ext ? idesc_ext : idesc_main;
 #pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-              const uint64_t boff = uint64_t((kk * badv) >> 4), aoff = uint64_t((kk * 32u) >> 4);
-              tc_mma_bf16_pair(d0, a0 + aoff, bd + boff, idesc, acc);
-              tc_mma_bf16_pair(d1, a1 + aoff, bd + boff, idesc, acc);
-            }
-            tc_commit_pair_mc(aempty(it % C::SA), 0x3);
-            tc_commit_pair_mc(bempty(it % C::SB), 0x3);
+          for (uint32_t kk = 0; kk < 4; ++kk) {
+            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+            tc_mma_bf16_pair(d0, a0 + 2 * kk, bd + kk * badv, idesc, acc);
+            tc_mma_bf16_pair(d1, a1 + 2 * kk, bd + kk * badv, idesc, acc);
           }
-          if (!ok) break;
-          tc_commit_pair_mc(tfull(buf), 0x3);
+          tc_commit_pair_mc(empty(si), 0x3);
         }
-        tc_commit_pair_mc(drain_bar, 0x1);
-        mbar_wait(drain_bar, 0, 100000000ull);
+        if (!ok) break;
+        tc_commit_pair_mc(tfull(buf), 0x3);
       }
-    } else {
-      // ------------------------------------------------------------ relay (odd CTA)
-      if (lane == 0) {
-        uint32_t it = 0;
-        bool ok = true;
-        for (int t = pair; t < num_tiles && ok; t += npairs) {
-          for (int j = 0; j < nsteps; ++j, ++it) {
-            if (!mbar_wait(bfull(it % C::SB), (it / C::SB) & 1u)) {
-              set_status_site(p.status, QLORA_ERR_TIMEOUT, 106); ok = false; break;
-            }
-            mbar_arrive_cluster(mapa_shared(bready(it % C::SB), 0));
-          }
-        }
-      }
+      tc_commit_pair_mc(drain_bar, 0x1);
+      mbar_wait(drain_bar, 0, 100000000ull);
     }
   } else if (warp < 7) {
     // ------------------------------------------------------------ epilogue (both CTAs)
@@ -652,7 +619,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     for (int t = pair; t < num_tiles; t += npairs, ++tcount) {
       const int mb = t / p.tiles_n, nb = t - mb * p.tiles_n;
       const uint32_t buf = tcount & 1u, tph = (tcount >> 1) & 1u;
-      if (!mbar_wait_cluster(tfull(buf), tph)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 107); break; }
+      if (!__all_sync(0xffffffffu, mbar_wait_cluster(tfull(buf), tph))) {
+        set_status_site(p.status, QLORA_ERR_TIMEOUT, 107); break;
+      }
       tc_fence_after();
 #pragma unroll 1
       for (int a = 0; a < 2; ++a) {
@@ -683,10 +652,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ dequantizers (both CTAs)
-    const uint32_t dwarp = warp - 7;
-    const uint32_t group = dwarp / C::kWarpsPerGroup;              // owns B slot `group`
-    const uint32_t sub = dwarp % C::kWarpsPerGroup;
-    const uint32_t dt = sub * 32 + lane;                           // 0..63
+    const uint32_t own = (warp - 7) / C::kWarpsPerSlot;   // slot this warp fills
+    const uint32_t sub = (warp - 7) % C::kWarpsPerSlot;   // rows [32 sub, 32 sub + 32)
+    const uint32_t ready_remote = mapa_shared(ready(own), 0);
     uint32_t it = 0, ic = 0;
     bool ok = true;
     for (int t = pair; t < num_tiles && ok; t += npairs) {
@@ -694,33 +662,47 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       for (int j = 0; j < nsteps; ++j, ++it) {
         const bool main_step = j < p.num_k_main;
         const uint32_t my = main_step ? ic++ : 0u;
-        if ((it % C::SB) != group) continue;
-        const uint32_t sb = it % C::SB;
-        if (!mbar_wait(bempty(sb), ((it / C::SB) & 1u) ^ 1u)) {
+        if ((it % C::S) != own) continue;
+        const uint32_t round = it / C::S;
+        if (!__all_sync(0xffffffffu, mbar_wait(empty(own), (round & 1u) ^ 1u))) {
           set_status_site(p.status, QLORA_ERR_TIMEOUT, 118); ok = false; break;
         }
+        const uint32_t b_tile = slot(it) + 2 * C::kA;
         if (main_step) {
-          if (!mbar_wait(cfull(my % C::SC), (my / C::SC) & 1u)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(cfull(my % C::SC), (my / C::SC) & 1u))) {
             set_status_site(p.status, QLORA_ERR_TIMEOUT, 108); ok = false; break;
           }
-          const uint8_t* cs = smem + c_slot(my);
-          dequant_block_pair(dt, cs, reinterpret_cast<const float*>(cs + C::kCodes), b_slot(it));
+          const uint8_t* cs = smem + c_off(my);
+#pragma unroll
+          for (uint32_t r = sub * 32 + lane; r < 64; r += 32 * C::kWarpsPerSlot)
+            dequant_block_pair(r, cs, reinterpret_cast<const float*>(cs + C::kCodes), b_tile);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
             mbar_arrive(cempty(my % C::SC));
-            mbar_arrive(bfull(sb));
+            mbar_arrive(ready(own));
           }
         } else if (lane == 0) {
-          // LoRA step: this group's slot is filled by TMA (one expect_tx arrival plus
-          // the other warp's plain arrival).
+          // LoRA step: B half by TMA, counted on the slot's ready barrier
           if (sub == 0) {
-            mbar_arrive_expect_tx(bfull(sb), C::kB);
-            tma_load_2d(b_slot(it), &tmBx, bfull(sb), (j - p.num_k_main) * 64, nc0);
+            mbar_arrive_expect_tx(ready(own), C::kB);
+            tma_load_2d(b_tile, &tmBx, ready(own), (j - p.num_k_main) * 64, nc0);
           } else {
-            mbar_arrive(bfull(sb));
+            mbar_arrive(ready(own));
           }
         }
+        if (rank != 0 && sub == 0) {
+          // odd CTA: once this CTA's A and B halves are in place, tell the even CTA
+          int fail = 0;
+          if (lane == 0) {
+            if (mbar_wait(ready(own), round & 1u)) mbar_arrive_cluster(ready_remote);
+            else fail = 1;
+          }
+          if (__shfl_sync(0xffffffffu, fail, 0)) {
+            set_status_site(p.status, QLORA_ERR_TIMEOUT, 128); ok = false; break;
+          }
+        }
+        __syncwarp();
       }
     }
   }
