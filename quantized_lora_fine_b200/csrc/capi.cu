@@ -206,19 +206,19 @@ qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
   if (!make_tmap_2d(&op.Ax, Ax, TmapType::BF16, r, M, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
   if (!make_tmap_2d(&op.Bx, Bx, TmapType::BF16, r, Ndim, int64_t(r) * 2, 64, 256, true)) return QLORA_ERR_CUDA;
   if (!w->is_bf16 && use_pair_kernel()) {
-    // CTA-pair fused kernel: 512 x 128 tiles; each CTA holds two 128-row A tiles
-    // and 64 rows (fwd) or columns (dX) of B.
+    // CTA-pair fused kernel: 256 x 256 tiles; each CTA holds 128 A rows and
+    // 128 rows (fwd) or columns (dX) of B.
     GemmOperands pp;
     std::memset(&pp, 0, sizeof(pp));
     pp.A = op.A;
     pp.Ax = op.Ax;
-    if (!make_tmap_2d(&pp.Bx, Bx, TmapType::BF16, r, Ndim, int64_t(r) * 2, 64, 64, true)) return QLORA_ERR_CUDA;
+    if (!make_tmap_2d(&pp.Bx, Bx, TmapType::BF16, r, Ndim, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
     if (!dx) {
-      if (!make_tmap_2d_sw(&pp.codes, w->codes, TmapType::U8, h / 2, o_, h / 2, 32, 64, 32)) return QLORA_ERR_CUDA;
-      if (!make_tmap_2d(&pp.scales, scales_t, TmapType::F32, o_, h / 64, o_ * 4, 64, 1, false)) return QLORA_ERR_CUDA;
+      if (!make_tmap_2d_sw(&pp.codes, w->codes, TmapType::U8, h / 2, o_, h / 2, 32, 128, 32)) return QLORA_ERR_CUDA;
+      if (!make_tmap_2d(&pp.scales, scales_t, TmapType::F32, o_, h / 64, o_ * 4, 128, 1, false)) return QLORA_ERR_CUDA;
     } else {
-      if (!make_tmap_2d_sw(&pp.codes, w->codes, TmapType::U8, h / 2, o_, h / 2, 32, 64, 32)) return QLORA_ERR_CUDA;
-      if (!make_tmap_2d(&pp.scales, scales_t, TmapType::F32, o_, h / 64, o_ * 4, 64, 1, false)) return QLORA_ERR_CUDA;
+      if (!make_tmap_2d_sw(&pp.codes, w->codes, TmapType::U8, h / 2, o_, h / 2, 64, 64, 64)) return QLORA_ERR_CUDA;
+      if (!make_tmap_2d(&pp.scales, scales_t, TmapType::F32, o_, h / 64, o_ * 4, 64, 2, false)) return QLORA_ERR_CUDA;
     }
     GemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -226,8 +226,8 @@ qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
     p.N = int(Ndim);
     p.num_k_main = int(Kdim / 64);
     p.num_k_ext = (r + 63) / 64;
-    p.tiles_m = int((M + 511) / 512);
-    p.tiles_n = int(Ndim / 128);
+    p.tiles_m = int((M + 255) / 256);
+    p.tiles_n = int(Ndim / 256);
     p.splits = 1;
     p.ksteps_per_split = p.num_k_main;
     p.out = out;

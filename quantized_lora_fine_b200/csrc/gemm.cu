@@ -403,23 +403,29 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 // =============================================================== CTA-pair kernel
 //
 // Fused NF4 GEMM on a pair of CTAs (cluster of 2, tcgen05 cta_group::2).
-// One pair tile is 512 (M) x 128 (N): two M = 256 accumulators share every
-// dequantized B tile, so each SM dequantizes one weight per 512 output rows.
+// One pair tile is 256 (M) x 256 (N), one M = 256, N = 256 accumulator (double
+// buffered in TMEM). Each CTA stages its 128 rows of A by TMA and dequantizes its
+// 128-wide half of B; every MMA reads 4 KB of A and 4 KB of B per CTA per 128
+// tensor cycles, and each A byte fetched from L2 feeds 256 output columns.
 //
 // Shared memory per CTA:
-//   S slots   A0, A1 (this CTA's 128-row halves of the two 256-row MMA tiles,
-//             or the LoRA T/U rows in the extension steps) and this CTA's bf16
-//             half of B (64 rows fwd / 64 columns dX)
-//   SC slots  packed codes + expanded scales of that B half, loaded ahead
-// Slot s of step `it` is it % S. Every slot has exactly one writer per role
-// (the A producer for A, dequantizer warp it % S for B, which also issues the
-// TMA of the LoRA steps' B tile) and all writers wait for the slot's previous
-// round to be consumed, so a parity wait never matches a phase two rounds old.
+//   S slots   A (this CTA's 128 rows, or the LoRA T/U rows in the extension
+//             steps) and this CTA's bf16 half of B (128 rows fwd, K-major /
+//             128 columns dX, MN-major in two 64-column chunks)
+//   SC slots  packed codes + expanded scales of that B half
+// Slot s of step `it` is it % S, and so is its code slot. Every slot has exactly
+// one writer per role (the A producer for A, the two dequantizer warps that own
+// slot it % S for B, which also issue the TMA of the LoRA steps' B half) and all
+// writers wait for the slot's previous round to be consumed, so a parity wait
+// never matches a phase two rounds old.
 //
 // Barriers (same offsets in both CTAs):
-//   ready[s]  even CTA: A bytes (TMA) + its slot owners + the odd CTA's slot
-//             owner (remote arrival, sent after the odd CTA's own ready[s]
-//             completed); odd CTA: A bytes + its slot owners
+//   ready[s]  even CTA only: one arrival from the even A producer, which also
+//             posts every byte the step needs (both CTAs' A tiles, loaded with
+//             2-SM TMA that signals the even CTA, and the LoRA steps' B halves),
+//             plus one arrival per slot owner of either CTA (the odd CTA's owners
+//             arrive across the cluster with release semantics once their B
+//             rows are written and fenced for the async proxy).
 //   empty[s]  one multicast tcgen05.commit per step from the even CTA's MMA
 //   cfull / cempty   code ring
 //   tfull[b] / tempty[b]  accumulator double buffer
@@ -429,39 +435,71 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 template <bool B_MN_>
 struct PairCfg {
   static constexpr bool B_MN = B_MN_;
-  static constexpr int S = 5, SC = 8;
-  static constexpr int kA = 128 * 64 * 2;       // one 128-row A tile: 16 KB
-  static constexpr int kB = 64 * 64 * 2;        // 8 KB
-  static constexpr int kSlot = 2 * kA + kB;     // 40 KB
-  static constexpr int kCodes = 64 * 32;        // 2 KB
-  static constexpr int kScales = 64 * 4;        // 256 B
-  static constexpr int kCSlot = 3072;
+  static constexpr int S = 6, SC = S;           // code slot = B slot: one reader pair per slot
+  static constexpr int kA = 128 * 64 * 2;       // this CTA's 128 A rows: 16 KB
+  static constexpr int kB = 128 * 64 * 2;       // this CTA's B half: 16 KB
+  static constexpr int kSlot = kA + kB;         // 32 KB
+  static constexpr int kCodes = 128 * 32;       // 4 KB
+  static constexpr int kScales = 128 * 4;       // 512 B
+  static constexpr int kCSlot = kCodes + kScales;
   static constexpr int kCOff = S * kSlot;
   static constexpr int kBarOff = kCOff + SC * kCSlot;
-  static constexpr int kWarpsPerSlot = 2;       // the warps of slot w dequantize 32 rows each
+  static constexpr int kWarpsPerSlot = 2;       // each thread dequantizes two 64-element blocks
   static constexpr int kDeqWarps = S * kWarpsPerSlot;
   static constexpr int kThreads = (7 + kDeqWarps) * 32;
-  static constexpr int kTmemCols = 512;         // 2 buffers x 2 accumulators x 128 columns
+  static constexpr int kTmemCols = 512;         // 2 buffers x 256 columns
   static constexpr int kNumBars = 2 * S + 2 * SC + 5;
   static constexpr int kSmem = kBarOff + 8 * kNumBars + 16 + 1024;
   static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(kCSlot % 512 == 0, "code slots keep the 64-byte swizzle alignment");
 };
 
-// One thread turns one 64-element block of this CTA's B half into bf16.
-//   fwd (K-major): t = B row (0..63); dX (MN-major): t = K row of the single
-//   64-column chunk. Both read 64 rows x 32 B of codes (32-byte swizzle).
-__device__ __forceinline__ void dequant_block_pair(uint32_t t, const uint8_t* codes_s, const float* scales_s,
-                                                   uint32_t b_tile) {
-  const uint32_t csw = (t >> 2) & 1u;
-  const uint4 c0 = *reinterpret_cast<const uint4*>(codes_s + t * 32 + ((0u ^ csw) << 4));
-  const uint4 c1 = *reinterpret_cast<const uint4*>(codes_s + t * 32 + ((1u ^ csw) << 4));
-  const NF4Lut lut = nf4_make_lut(scales_s[t]);
-  const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-  const uint32_t sw = t & 7u;
-  const uint32_t row_base = b_tile + (t >> 3) * 1024u + sw * 128u;
+// One thread turns two 64-element blocks of this CTA's B half into bf16.
+//   fwd (K-major B, 128 rows x 64 K): blocks are B rows t and t + 64; their codes
+//     are rows of 32 bytes (32-byte swizzle), one scale each.
+//   dX (MN-major B, 64 K rows x 128 columns): blocks are K row t of the column
+//     chunks 0 and 1; codes are rows of 64 bytes (64-byte swizzle), scales are
+//     stored [chunk][K row].
+// The codes and the blocks' product tables are loaded first (they arrive early,
+// on their own ring); the stores wait until the B slot is free. The code slot is
+// released only after the B stores and the proxy fence: a slot released right
+// after the generic loads was measured to be overwritten by the next TMA before
+// those loads had read it (a generic-read / async-write hazard needs the fence).
+struct PairBlock {
+  uint32_t w[8];
+  NF4Lut lut;
+};
+
+template <bool B_MN>
+__device__ __forceinline__ void dequant_load_pair(uint32_t t, uint32_t blk, const uint8_t* codes_s,
+                                                  const float* scales_s, PairBlock& b) {
+  uint4 c0, c1;
+  float a;
+  if constexpr (!B_MN) {
+    const uint32_t row = t + 64u * blk, csw = (row >> 2) & 1u;
+    c0 = *reinterpret_cast<const uint4*>(codes_s + row * 32 + ((0u ^ csw) << 4));
+    c1 = *reinterpret_cast<const uint4*>(codes_s + row * 32 + ((1u ^ csw) << 4));
+    a = scales_s[row];
+  } else {
+    const uint32_t csw = (t >> 1) & 3u;
+    c0 = *reinterpret_cast<const uint4*>(codes_s + t * 64 + (((2u * blk) ^ csw) << 4));
+    c1 = *reinterpret_cast<const uint4*>(codes_s + t * 64 + (((2u * blk + 1u) ^ csw) << 4));
+    a = scales_s[blk * 64u + t];
+  }
+  b.lut = nf4_make_lut(a);
+  b.w[0] = c0.x; b.w[1] = c0.y; b.w[2] = c0.z; b.w[3] = c0.w;
+  b.w[4] = c1.x; b.w[5] = c1.y; b.w[6] = c1.z; b.w[7] = c1.w;
+}
+
+// Writes block `blk` of thread t as one 128-byte swizzled row of the B half.
+template <bool B_MN>
+__device__ __forceinline__ void dequant_store_pair(uint32_t t, uint32_t blk, const PairBlock& b, uint32_t b_tile) {
+  const uint32_t row = B_MN ? t : t + 64u * blk;
+  const uint32_t sw = row & 7u;
+  const uint32_t row_base = b_tile + (B_MN ? blk * 8192u : 0u) + (row >> 3) * 1024u + sw * 128u;
 #pragma unroll
   for (uint32_t c = 0; c < 8; ++c) {
-    const uint4 v = nf4_dequant_word(words[c], lut);
+    const uint4 v = nf4_dequant_word(b.w[c], b.lut);
     const uint32_t addr = row_base + ((c ^ sw) << 4);
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
@@ -486,7 +524,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   auto tempty = [&](int b) { return bar_base + 8u * (kT0 + 2 + b); };
   const uint32_t drain_bar = bar_base + 8u * (kT0 + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * C::kNumBars);
-  auto slot = [&](uint32_t i) { return smem_base + (i % C::S) * C::kSlot; };          // A0 | A1 | B
+  auto slot = [&](uint32_t i) { return smem_base + (i % C::S) * C::kSlot; };          // A | B half
   auto c_off = [&](uint32_t i) { return C::kCOff + (i % C::SC) * C::kCSlot; };         // from smem
 
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -494,7 +532,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::S; ++i) {
-      mbar_init(ready(i), 1 + C::kWarpsPerSlot + (rank == 0 ? 1 : 0));
+      mbar_init(ready(i), 1 + 2 * C::kWarpsPerSlot);   // used in the even CTA only
       mbar_init(empty(i), 1);
     }
     for (int i = 0; i < C::SC; ++i) { mbar_init(cfull(i), 1); mbar_init(cempty(i), C::kWarpsPerSlot); }
@@ -513,7 +551,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_tiles = p.tiles_m * p.tiles_n;   // tiles of 512 x 128
+  const int num_tiles = p.tiles_m * p.tiles_n;   // tiles of 256 x 256
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int nsteps = p.num_k_main + p.num_k_ext;
 
@@ -524,17 +562,22 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += npairs) {
-        const int m0 = (t / p.tiles_n) * 512 + int(rank) * 128;
+        const int m0 = (t / p.tiles_n) * 256 + int(rank) * 128;
         for (int j = 0; j < nsteps; ++j, ++it) {
           if (!mbar_wait(empty(it % C::S), ((it / C::S) & 1u) ^ 1u)) {
             set_status_site(p.status, QLORA_ERR_TIMEOUT, 101); ok = false; break;
           }
+          const bool main_step = j < p.num_k_main;
           const uint32_t dst = slot(it), bar = ready(it % C::S);
-          mbar_arrive_expect_tx(bar, 2 * C::kA);
-          const CUtensorMap* m = (j < p.num_k_main) ? &tmA : &tmAx;
-          const int kx = (j < p.num_k_main ? j : j - p.num_k_main) * 64;
-          tma_load_2d(dst, m, bar, kx, m0);
-          tma_load_2d(dst + C::kA, m, bar, kx, m0 + 256);
+          const CUtensorMap* m = main_step ? &tmA : &tmAx;
+          const int kx = (main_step ? j : j - p.num_k_main) * 64;
+          if (rank == 0) {
+            // bytes of the whole step: both CTAs' A tiles and, in LoRA steps, B halves
+            mbar_arrive_expect_tx(bar, 2 * C::kA + (main_step ? 0u : uint32_t(2 * C::kB)));
+            tma_load_2d(dst, m, bar, kx, m0);
+          } else {
+            tma_load_2d_pair(dst, m, mapa_shared(bar, 0), kx, m0);
+          }
         }
       }
       // let the last copies land before leaving
@@ -545,20 +588,23 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmCodes);
       tma_prefetch_desc(&tmScales);
+      // one code slot per step, LoRA steps included (their slot is released
+      // without a load), so slot i % SC is read only by the warps that own B slot i % S
       uint32_t ic = 0;
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += npairs) {
-        const int nc0 = (t % p.tiles_n) * 128 + int(rank) * 64;
-        for (int j = 0; j < p.num_k_main; ++j, ++ic) {
+        const int nc0 = (t % p.tiles_n) * 256 + int(rank) * 128;
+        for (int j = 0; j < nsteps; ++j, ++ic) {
           if (!mbar_wait(cempty(ic % C::SC), ((ic / C::SC) & 1u) ^ 1u)) {
             set_status_site(p.status, QLORA_ERR_TIMEOUT, 102); ok = false; break;
           }
           const uint32_t dst = smem_base + c_off(ic), bar = cfull(ic % C::SC);
+          if (j >= p.num_k_main) { mbar_arrive(bar); continue; }
           mbar_arrive_expect_tx(bar, C::kCodes + C::kScales);
-          if constexpr (!C::B_MN) {
+          if constexpr (!C::B_MN) {   // codes box 32 B x 128 rows, scales box 128 x 1
             tma_load_2d(dst, &tmCodes, bar, j * 32, nc0);
             tma_load_2d(dst + C::kCodes, &tmScales, bar, nc0, j);
-          } else {
+          } else {                     // codes box 64 B x 64 rows, scales box 64 x 2
             tma_load_2d(dst, &tmCodes, bar, nc0 / 2, j * 64);
             tma_load_2d(dst + C::kCodes, &tmScales, bar, j * 64, nc0 / 64);
           }
@@ -572,20 +618,22 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (rank == 0 && lane == 0) {
-      constexpr uint32_t idesc_main = make_idesc_bf16(256, 128, 0, C::B_MN ? 1 : 0);
-      constexpr uint32_t idesc_ext = make_idesc_bf16(256, 128, 0, 0);
+      constexpr uint32_t idesc_main = make_idesc_bf16(256, 256, 0, C::B_MN ? 1 : 0);
+      constexpr uint32_t idesc_ext = make_idesc_bf16(256, 256, 0, 0);
       constexpr uint32_t b_adv = C::B_MN ? (2048u >> 4) : (32u >> 4);
-      // descriptors are linear in the start address (bits 0..13 hold addr >> 4)
-      const uint64_t da0_base = make_smem_desc(slot(0), 16u, 1024u, kSwizzle128B);
-      const uint64_t db_base = make_smem_desc(slot(0) + 2 * C::kA, 16u, 1024u, kSwizzle128B);
-      constexpr uint64_t kA1Adv = uint64_t(C::kA >> 4), kSlotAdv = uint64_t(C::kSlot >> 4);
+      // descriptors are linear in the start address (bits 0..13 hold addr >> 4);
+      // the MN-major B half is two 64-column chunks 8 KB apart (leading offset),
+      // which a K-major operand ignores
+      const uint64_t da_base = make_smem_desc(slot(0), 16u, 1024u, kSwizzle128B);
+      const uint64_t db_base = make_smem_desc(slot(0) + C::kA, 8192u, 1024u, kSwizzle128B);
+      constexpr uint64_t kSlotAdv = uint64_t(C::kSlot >> 4);
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += npairs, ++tcount) {
         const uint32_t buf = tcount & 1u, tph = (tcount >> 1) & 1u;
         if (!mbar_wait_cluster(tempty(buf), tph ^ 1u)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 104); ok = false; break; }
         tc_fence_after();
-        const uint32_t d0 = tmem_base + buf * 256u, d1 = d0 + 128u;
+        const uint32_t d = tmem_base + buf * 256u;
         for (int j = 0; j < nsteps; ++j, ++it) {
           const uint32_t si = it % C::S;
           if (!mbar_wait_cluster(ready(si), (it / C::S) & 1u)) {
@@ -593,15 +641,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           }
           tc_fence_after();
           const bool ext = j >= p.num_k_main;
-          const uint64_t a0 = da0_base + si * kSlotAdv, a1 = a0 + kA1Adv, bd = db_base + si * kSlotAdv;
+          const uint64_t ad = da_base + si * kSlotAdv, bd = db_base + si * kSlotAdv;
           const uint32_t badv = ext ? (32u >> 4) : b_adv;
           const uint32_t idesc = ext ? idesc_ext : idesc_main;
 #pragma unroll
-          for (uint32_t kk = 0; kk < 4; ++kk) {
-            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-            tc_mma_bf16_pair(d0, a0 + 2 * kk, bd + kk * badv, idesc, acc);
-            tc_mma_bf16_pair(d1, a1 + 2 * kk, bd + kk * badv, idesc, acc);
-          }
+          for (uint32_t kk = 0; kk < 4; ++kk)
+            tc_mma_bf16_pair(d, ad + 2 * kk, bd + kk * badv, idesc, (j > 0 || kk > 0) ? 1u : 0u);
           tc_commit_pair_mc(empty(si), 0x3);
         }
         if (!ok) break;
@@ -623,17 +668,16 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         set_status_site(p.status, QLORA_ERR_TIMEOUT, 107); break;
       }
       tc_fence_after();
+      {
+        const int grow = mb * 256 + int(rank) * 128 + int(row);
+        const uint32_t tbase = tmem_base + ((q * 32u) << 16) + buf * 256u;
 #pragma unroll 1
-      for (int a = 0; a < 2; ++a) {
-        const int grow = mb * 512 + a * 256 + int(rank) * 128 + int(row);
-        const uint32_t tbase = tmem_base + ((q * 32u) << 16) + buf * 256u + uint32_t(a) * 128u;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 8; ++c) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tbase + c * 32, v);
           tmem_ld_wait();
           if (grow < p.M) {
-            uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) + int64_t(grow) * p.ld_out + nb * 128 + c * 32;
+            uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) + int64_t(grow) * p.ld_out + nb * 256 + c * 32;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               uint4 o;
@@ -653,53 +697,54 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   } else {
     // ------------------------------------------------------------ dequantizers (both CTAs)
     const uint32_t own = (warp - 7) / C::kWarpsPerSlot;   // slot this warp fills
-    const uint32_t sub = (warp - 7) % C::kWarpsPerSlot;   // rows [32 sub, 32 sub + 32)
-    const uint32_t ready_remote = mapa_shared(ready(own), 0);
-    uint32_t it = 0, ic = 0;
+    const uint32_t sub = (warp - 7) % C::kWarpsPerSlot;   // threads t in [32 sub, 32 sub + 32)
+    const uint32_t row = sub * 32 + lane;
+    const uint32_t ready_even = mapa_shared(ready(own), 0);
+    uint32_t it = 0;
     bool ok = true;
     for (int t = pair; t < num_tiles && ok; t += npairs) {
-      const int nc0 = (t % p.tiles_n) * 128 + int(rank) * 64;
+      const int nc0 = (t % p.tiles_n) * 256 + int(rank) * 128;
       for (int j = 0; j < nsteps; ++j, ++it) {
         const bool main_step = j < p.num_k_main;
-        const uint32_t my = main_step ? ic++ : 0u;
         if ((it % C::S) != own) continue;
         const uint32_t round = it / C::S;
-        if (!__all_sync(0xffffffffu, mbar_wait(empty(own), (round & 1u) ^ 1u))) {
-          set_status_site(p.status, QLORA_ERR_TIMEOUT, 118); ok = false; break;
+        const uint32_t b_tile = slot(it) + C::kA;
+        if (!__all_sync(0xffffffffu, mbar_wait(cfull(it % C::SC), (it / C::SC) & 1u))) {
+          set_status_site(p.status, QLORA_ERR_TIMEOUT, 108); ok = false; break;
         }
-        const uint32_t b_tile = slot(it) + 2 * C::kA;
         if (main_step) {
-          if (!__all_sync(0xffffffffu, mbar_wait(cfull(my % C::SC), (my / C::SC) & 1u))) {
-            set_status_site(p.status, QLORA_ERR_TIMEOUT, 108); ok = false; break;
+          const uint8_t* cs = smem + c_off(it);
+          const float* ss = reinterpret_cast<const float*>(cs + C::kCodes);
+          PairBlock blk;
+          dequant_load_pair<C::B_MN>(row, 0, cs, ss, blk);
+          if (!__all_sync(0xffffffffu, mbar_wait(empty(own), (round & 1u) ^ 1u))) {
+            set_status_site(p.status, QLORA_ERR_TIMEOUT, 118); ok = false; break;
           }
-          const uint8_t* cs = smem + c_off(my);
-#pragma unroll
-          for (uint32_t r = sub * 32 + lane; r < 64; r += 32 * C::kWarpsPerSlot)
-            dequant_block_pair(r, cs, reinterpret_cast<const float*>(cs + C::kCodes), b_tile);
+          dequant_store_pair<C::B_MN>(row, 0, blk, b_tile);
+          dequant_load_pair<C::B_MN>(row, 1, cs, ss, blk);
+          dequant_store_pair<C::B_MN>(row, 1, blk, b_tile);
           fence_proxy_async_smem();
           __syncwarp();
+          if (lane == 0) mbar_arrive(cempty(it % C::SC));
           if (lane == 0) {
-            mbar_arrive(cempty(my % C::SC));
-            mbar_arrive(ready(own));
+            if (rank == 0) mbar_arrive(ready(own));
+            else mbar_arrive_cluster(ready_even);
           }
-        } else if (lane == 0) {
-          // LoRA step: B half by TMA, counted on the slot's ready barrier
-          if (sub == 0) {
-            mbar_arrive_expect_tx(ready(own), C::kB);
-            tma_load_2d(b_tile, &tmBx, ready(own), (j - p.num_k_main) * 64, nc0);
-          } else {
-            mbar_arrive(ready(own));
+        } else {
+          if (lane == 0) mbar_arrive(cempty(it % C::SC));
+          if (!__all_sync(0xffffffffu, mbar_wait(empty(own), (round & 1u) ^ 1u))) {
+            set_status_site(p.status, QLORA_ERR_TIMEOUT, 118); ok = false; break;
           }
-        }
-        if (rank != 0 && sub == 0) {
-          // odd CTA: once this CTA's A and B halves are in place, tell the even CTA
-          int fail = 0;
+          // LoRA step: B half by TMA; its bytes were posted by the even A producer
           if (lane == 0) {
-            if (mbar_wait(ready(own), round & 1u)) mbar_arrive_cluster(ready_remote);
-            else fail = 1;
-          }
-          if (__shfl_sync(0xffffffffu, fail, 0)) {
-            set_status_site(p.status, QLORA_ERR_TIMEOUT, 128); ok = false; break;
+            const int kx = (j - p.num_k_main) * 64;
+            if (rank == 0) {
+              if (sub == 0) tma_load_2d(b_tile, &tmBx, ready(own), kx, nc0);
+              mbar_arrive(ready(own));
+            } else {
+              if (sub == 0) tma_load_2d_pair(b_tile, &tmBx, ready_even, kx, nc0);
+              mbar_arrive_cluster(ready_even);
+            }
           }
         }
         __syncwarp();
@@ -809,7 +854,7 @@ static qlora_status launch_pair_cfg(const GemmOperands& o, GemmParams p, cudaStr
     max_pairs = n;
     attr_set = true;
   }
-  p.bn = 128;
+  p.bn = 256;
   const int num_tiles = p.tiles_m * p.tiles_n;
   const int pairs = std::max(1, std::min(num_tiles, max_pairs));
   cudaLaunchConfig_t cfg = {};
