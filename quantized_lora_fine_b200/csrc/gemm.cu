@@ -449,7 +449,9 @@ struct PairCfg {
   static constexpr int kThreads = (7 + kDeqWarps) * 32;
   static constexpr int kTmemCols = 512;         // 2 buffers x 256 columns
   static constexpr int kNumBars = 2 * S + 2 * SC + 5;
-  static constexpr int kSmem = kBarOff + 8 * kNumBars + 16 + 1024;
+  static constexpr int kSigOff = kBarOff + 8 * kNumBars + 16;   // 4 bytes per dequantizer warp
+  static constexpr int kSigBytes = 4;
+  static constexpr int kSmem = kSigOff + kDeqWarps * kSigBytes + 1024;
   static_assert(kSmem <= 232448, "shared memory budget");
   static_assert(kCSlot % 512 == 0, "code slots keep the 64-byte swizzle alignment");
 };
@@ -532,7 +534,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::S; ++i) {
-      mbar_init(ready(i), 1 + 2 * C::kWarpsPerSlot);   // used in the even CTA only
+      mbar_init(ready(i), 1 + C::kWarpsPerSlot);   // used in the even CTA only
       mbar_init(empty(i), 1);
     }
     for (int i = 0; i < C::SC; ++i) { mbar_init(cfull(i), 1); mbar_init(cempty(i), C::kWarpsPerSlot); }
@@ -573,7 +575,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           const int kx = (main_step ? j : j - p.num_k_main) * 64;
           if (rank == 0) {
             // bytes of the whole step: both CTAs' A tiles and, in LoRA steps, B halves
-            mbar_arrive_expect_tx(bar, 2 * C::kA + (main_step ? 0u : uint32_t(2 * C::kB)));
+            mbar_arrive_expect_tx(bar, 2 * C::kA + (main_step ? uint32_t(C::kWarpsPerSlot * C::kSigBytes)
+                                                          : uint32_t(2 * C::kB)));
             tma_load_2d(dst, m, bar, kx, m0);
           } else {
             tma_load_2d_pair(dst, m, mapa_shared(bar, 0), kx, m0);
@@ -700,6 +703,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     const uint32_t sub = (warp - 7) % C::kWarpsPerSlot;   // threads t in [32 sub, 32 sub + 32)
     const uint32_t row = sub * 32 + lane;
     const uint32_t ready_even = mapa_shared(ready(own), 0);
+    const uint32_t sig_even = mapa_shared(smem_base + C::kSigOff + (warp - 7) * C::kSigBytes, 0);
     uint32_t it = 0;
     bool ok = true;
     for (int t = pair; t < num_tiles && ok; t += npairs) {
@@ -728,7 +732,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           if (lane == 0) mbar_arrive(cempty(it % C::SC));
           if (lane == 0) {
             if (rank == 0) mbar_arrive(ready(own));
-            else mbar_arrive_cluster(ready_even);
+            else st_async_signal(sig_even, ready_even);
           }
         } else {
           if (lane == 0) mbar_arrive(cempty(it % C::SC));
@@ -743,7 +747,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
               mbar_arrive(ready(own));
             } else {
               if (sub == 0) tma_load_2d_pair(b_tile, &tmBx, ready_even, kx, nc0);
-              mbar_arrive_cluster(ready_even);
             }
           }
         }

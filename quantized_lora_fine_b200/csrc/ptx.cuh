@@ -94,6 +94,16 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
+// Stores 4 bytes into another CTA's shared memory and counts them on that CTA's
+// mbarrier; the complete-tx has release semantics at cluster scope, so the
+// issuing thread's earlier writes (fenced for the async proxy) are visible to a
+// thread that observes the phase.
+__device__ __forceinline__ void st_async_signal(uint32_t dst_cluster, uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(dst_cluster), "r"(1u),
+               "r"(bar_cluster)
+               : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
