@@ -213,13 +213,6 @@ qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
     pp.A = op.A;
     pp.Ax = op.Ax;
     if (!make_tmap_2d(&pp.Bx, Bx, TmapType::BF16, r, Ndim, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
-    if (!dx) {
-      if (!make_tmap_2d_sw(&pp.codes, w->codes, TmapType::U8, h / 2, o_, h / 2, 32, 128, 32)) return QLORA_ERR_CUDA;
-      if (!make_tmap_2d(&pp.scales, scales_t, TmapType::F32, o_, h / 64, o_ * 4, 128, 1, false)) return QLORA_ERR_CUDA;
-    } else {
-      if (!make_tmap_2d_sw(&pp.codes, w->codes, TmapType::U8, h / 2, o_, h / 2, 64, 64, 64)) return QLORA_ERR_CUDA;
-      if (!make_tmap_2d(&pp.scales, scales_t, TmapType::F32, o_, h / 64, o_ * 4, 64, 2, false)) return QLORA_ERR_CUDA;
-    }
     GemmParams p;
     std::memset(&p, 0, sizeof(p));
     p.M = int(M);
@@ -228,6 +221,10 @@ qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
     p.num_k_ext = (r + 63) / 64;
     p.tiles_m = int((M + 255) / 256);
     p.tiles_n = int(Ndim / 256);
+    p.codes = w->codes;
+    p.scales = scales_t;
+    p.codes_ld = h / 2;
+    p.scales_ld = o_;
     p.splits = 1;
     p.ksteps_per_split = p.num_k_main;
     p.out = out;

@@ -408,100 +408,95 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 // 128-wide half of B; every MMA reads 4 KB of A and 4 KB of B per CTA per 128
 // tensor cycles, and each A byte fetched from L2 feeds 256 output columns.
 //
-// Shared memory per CTA:
-//   S slots   A (this CTA's 128 rows, or the LoRA T/U rows in the extension
-//             steps) and this CTA's bf16 half of B (128 rows fwd, K-major /
-//             128 columns dX, MN-major in two 64-column chunks)
-//   SC slots  packed codes + expanded scales of that B half
-// Slot s of step `it` is it % S, and so is its code slot. Every slot has exactly
-// one writer per role (the A producer for A, the two dequantizer warps that own
-// slot it % S for B, which also issue the TMA of the LoRA steps' B half) and all
-// writers wait for the slot's previous round to be consumed, so a parity wait
-// never matches a phase two rounds old.
+// Shared memory per CTA: S slots, each holding A (this CTA's 128 rows, or the
+// LoRA T/U rows in the extension steps) and this CTA's bf16 half of B (128 rows
+// fwd, K-major / 128 columns dX, MN-major in two 64-column chunks). Slot s of
+// step `it` is it % S. Every slot has exactly one writer per role (the A producer
+// for A; the two dequantizer warps that own slot it % S for B, which also issue
+// the TMA of the LoRA steps' B half) and all writers wait for the slot's previous
+// round to be consumed, so a parity wait never matches a phase two rounds old.
+// The dequantizers read packed codes and scales from global memory (L2) into
+// registers one owned step ahead; shared memory holds only the MMA operands.
 //
 // Barriers (same offsets in both CTAs):
 //   ready[s]  even CTA only: one arrival from the even A producer, which also
 //             posts every byte the step needs (both CTAs' A tiles, loaded with
-//             2-SM TMA that signals the even CTA, and the LoRA steps' B halves),
-//             plus one arrival per slot owner of either CTA (the odd CTA's owners
-//             arrive across the cluster with release semantics once their B
-//             rows are written and fenced for the async proxy).
+//             2-SM TMA that signals the even CTA; the LoRA steps' B halves; a
+//             4-byte st.async from each odd slot owner), plus one arrival per
+//             even slot owner. The odd owners' st.async completes on the even
+//             barrier with release semantics at cluster scope once their B rows
+//             are written and fenced for the async proxy.
 //   empty[s]  one multicast tcgen05.commit per step from the even CTA's MMA
-//   cfull / cempty   code ring
 //   tfull[b] / tempty[b]  accumulator double buffer
-// Warp roles: 0 A producer, 1 MMA issuer (even CTA) and TMEM allocation, 2 C
-// producer, 3-6 epilogue, 7.. dequantizers (kWarpsPerSlot warps per slot).
+// Warp roles: 0 A producer, 1 MMA issuer (even CTA) and TMEM allocation, 2-5
+// epilogue, 6.. dequantizers (kWarpsPerSlot warps per slot).
 
 template <bool B_MN_>
 struct PairCfg {
   static constexpr bool B_MN = B_MN_;
-  static constexpr int S = 6, SC = S;           // code slot = B slot: one reader pair per slot
+  static constexpr int S = 7;                   // ring slots (one K step each)
   static constexpr int kA = 128 * 64 * 2;       // this CTA's 128 A rows: 16 KB
   static constexpr int kB = 128 * 64 * 2;       // this CTA's B half: 16 KB
   static constexpr int kSlot = kA + kB;         // 32 KB
-  static constexpr int kCodes = 128 * 32;       // 4 KB
-  static constexpr int kScales = 128 * 4;       // 512 B
-  static constexpr int kCSlot = kCodes + kScales;
-  static constexpr int kCOff = S * kSlot;
-  static constexpr int kBarOff = kCOff + SC * kCSlot;
+  static constexpr int kBarOff = S * kSlot;
   static constexpr int kWarpsPerSlot = 2;       // each thread dequantizes two 64-element blocks
   static constexpr int kDeqWarps = S * kWarpsPerSlot;
-  static constexpr int kThreads = (7 + kDeqWarps) * 32;
+  static constexpr int kFirstDeqWarp = 6;       // 0 A producer, 1 MMA, 2-5 epilogue
+  static constexpr int kThreads = (kFirstDeqWarp + kDeqWarps) * 32;
   static constexpr int kTmemCols = 512;         // 2 buffers x 256 columns
-  static constexpr int kNumBars = 2 * S + 2 * SC + 5;
+  static constexpr int kNumBars = 2 * S + 5;
   static constexpr int kSigOff = kBarOff + 8 * kNumBars + 16;   // 4 bytes per dequantizer warp
   static constexpr int kSigBytes = 4;
   static constexpr int kSmem = kSigOff + kDeqWarps * kSigBytes + 1024;
   static_assert(kSmem <= 232448, "shared memory budget");
-  static_assert(kCSlot % 512 == 0, "code slots keep the 64-byte swizzle alignment");
 };
 
 // One thread turns two 64-element blocks of this CTA's B half into bf16.
-//   fwd (K-major B, 128 rows x 64 K): blocks are B rows t and t + 64; their codes
-//     are rows of 32 bytes (32-byte swizzle), one scale each.
-//   dX (MN-major B, 64 K rows x 128 columns): blocks are K row t of the column
-//     chunks 0 and 1; codes are rows of 64 bytes (64-byte swizzle), scales are
-//     stored [chunk][K row].
-// The codes and the blocks' product tables are loaded first (they arrive early,
-// on their own ring); the stores wait until the B slot is free. The code slot is
-// released only after the B stores and the proxy fence: a slot released right
-// after the generic loads was measured to be overwritten by the next TMA before
-// those loads had read it (a generic-read / async-write hazard needs the fence).
-struct PairBlock {
-  uint32_t w[8];
-  NF4Lut lut;
+//   fwd (K-major B, 128 rows x 64 K): blocks are B rows t and t + 64 (weight rows
+//     nc0 + t, nc0 + t + 64 at K block j).
+//   dX (MN-major B, 64 K rows x 128 columns): blocks are K row t (weight row
+//     64 j + t) of the column chunks 0 and 1 (weight columns nc0 .. nc0 + 127).
+// The packed codes and scales are read straight from global memory (L2) into
+// registers one owned step ahead, so they are in place when the slot frees; the
+// product tables are built after the slot wait.
+struct PairRaw {
+  uint4 c[2][2];   // 32 code bytes per block
+  float a[2];      // block scales
 };
 
 template <bool B_MN>
-__device__ __forceinline__ void dequant_load_pair(uint32_t t, uint32_t blk, const uint8_t* codes_s,
-                                                  const float* scales_s, PairBlock& b) {
-  uint4 c0, c1;
-  float a;
-  if constexpr (!B_MN) {
-    const uint32_t row = t + 64u * blk, csw = (row >> 2) & 1u;
-    c0 = *reinterpret_cast<const uint4*>(codes_s + row * 32 + ((0u ^ csw) << 4));
-    c1 = *reinterpret_cast<const uint4*>(codes_s + row * 32 + ((1u ^ csw) << 4));
-    a = scales_s[row];
-  } else {
-    const uint32_t csw = (t >> 1) & 3u;
-    c0 = *reinterpret_cast<const uint4*>(codes_s + t * 64 + (((2u * blk) ^ csw) << 4));
-    c1 = *reinterpret_cast<const uint4*>(codes_s + t * 64 + (((2u * blk + 1u) ^ csw) << 4));
-    a = scales_s[blk * 64u + t];
+__device__ __forceinline__ void pair_load_raw(const GemmParams& p, uint32_t t, int j, int nc0, PairRaw& r) {
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    const uint8_t* cp;
+    const float* sp;
+    if constexpr (!B_MN) {
+      const int64_t n = nc0 + int64_t(t) + 64 * b;
+      cp = p.codes + n * p.codes_ld + int64_t(j) * 32;
+      sp = p.scales + int64_t(j) * p.scales_ld + n;
+    } else {
+      const int64_t kr = int64_t(j) * 64 + t;
+      cp = p.codes + kr * p.codes_ld + (nc0 + 64 * b) / 2;
+      sp = p.scales + int64_t(nc0 / 64 + b) * p.scales_ld + kr;
+    }
+    r.c[b][0] = __ldg(reinterpret_cast<const uint4*>(cp));
+    r.c[b][1] = __ldg(reinterpret_cast<const uint4*>(cp + 16));
+    r.a[b] = __ldg(sp);
   }
-  b.lut = nf4_make_lut(a);
-  b.w[0] = c0.x; b.w[1] = c0.y; b.w[2] = c0.z; b.w[3] = c0.w;
-  b.w[4] = c1.x; b.w[5] = c1.y; b.w[6] = c1.z; b.w[7] = c1.w;
 }
 
 // Writes block `blk` of thread t as one 128-byte swizzled row of the B half.
 template <bool B_MN>
-__device__ __forceinline__ void dequant_store_pair(uint32_t t, uint32_t blk, const PairBlock& b, uint32_t b_tile) {
+__device__ __forceinline__ void pair_store_block(uint32_t t, uint32_t blk, const PairRaw& r, uint32_t b_tile) {
+  const NF4Lut lut = nf4_make_lut(r.a[blk]);
+  const uint32_t w[8] = {r.c[blk][0].x, r.c[blk][0].y, r.c[blk][0].z, r.c[blk][0].w,
+                         r.c[blk][1].x, r.c[blk][1].y, r.c[blk][1].z, r.c[blk][1].w};
   const uint32_t row = B_MN ? t : t + 64u * blk;
   const uint32_t sw = row & 7u;
   const uint32_t row_base = b_tile + (B_MN ? blk * 8192u : 0u) + (row >> 3) * 1024u + sw * 128u;
 #pragma unroll
   for (uint32_t c = 0; c < 8; ++c) {
-    const uint4 v = nf4_dequant_word(b.w[c], b.lut);
+    const uint4 v = nf4_dequant_word(w[c], lut);
     const uint32_t addr = row_base + ((c ^ sw) << 4);
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
@@ -510,8 +505,7 @@ __device__ __forceinline__ void dequant_store_pair(uint32_t t, uint32_t blk, con
 
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, 1)
-    tc_gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmCodes,
-                            const __grid_constant__ CUtensorMap tmScales, const __grid_constant__ CUtensorMap tmAx,
+    tc_gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAx,
                             const __grid_constant__ CUtensorMap tmBx, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -519,15 +513,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   const uint32_t bar_base = smem_base + C::kBarOff;
   auto ready = [&](int i) { return bar_base + 8u * i; };
   auto empty = [&](int i) { return bar_base + 8u * (C::S + i); };
-  auto cfull = [&](int i) { return bar_base + 8u * (2 * C::S + i); };
-  auto cempty = [&](int i) { return bar_base + 8u * (2 * C::S + C::SC + i); };
-  const int kT0 = 2 * C::S + 2 * C::SC;
+  const int kT0 = 2 * C::S;
   auto tfull = [&](int b) { return bar_base + 8u * (kT0 + b); };
   auto tempty = [&](int b) { return bar_base + 8u * (kT0 + 2 + b); };
   const uint32_t drain_bar = bar_base + 8u * (kT0 + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * C::kNumBars);
   auto slot = [&](uint32_t i) { return smem_base + (i % C::S) * C::kSlot; };          // A | B half
-  auto c_off = [&](uint32_t i) { return C::kCOff + (i % C::SC) * C::kCSlot; };         // from smem
 
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -537,7 +528,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       mbar_init(ready(i), 1 + C::kWarpsPerSlot);   // used in the even CTA only
       mbar_init(empty(i), 1);
     }
-    for (int i = 0; i < C::SC; ++i) { mbar_init(cfull(i), 1); mbar_init(cempty(i), C::kWarpsPerSlot); }
     for (int b = 0; b < 2; ++b) { mbar_init(tfull(b), 1); mbar_init(tempty(b), 8); }
     mbar_init(drain_bar, 1);
     fence_mbarrier_init();
@@ -586,38 +576,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       // let the last copies land before leaving
       mbar_wait(empty(it % C::S), ((it / C::S) & 1u) ^ 1u, 100000000ull);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ C producer (both CTAs)
-    if (lane == 0) {
-      tma_prefetch_desc(&tmCodes);
-      tma_prefetch_desc(&tmScales);
-      // one code slot per step, LoRA steps included (their slot is released
-      // without a load), so slot i % SC is read only by the warps that own B slot i % S
-      uint32_t ic = 0;
-      bool ok = true;
-      for (int t = pair; t < num_tiles && ok; t += npairs) {
-        const int nc0 = (t % p.tiles_n) * 256 + int(rank) * 128;
-        for (int j = 0; j < nsteps; ++j, ++ic) {
-          if (!mbar_wait(cempty(ic % C::SC), ((ic / C::SC) & 1u) ^ 1u)) {
-            set_status_site(p.status, QLORA_ERR_TIMEOUT, 102); ok = false; break;
-          }
-          const uint32_t dst = smem_base + c_off(ic), bar = cfull(ic % C::SC);
-          if (j >= p.num_k_main) { mbar_arrive(bar); continue; }
-          mbar_arrive_expect_tx(bar, C::kCodes + C::kScales);
-          if constexpr (!C::B_MN) {   // codes box 32 B x 128 rows, scales box 128 x 1
-            tma_load_2d(dst, &tmCodes, bar, j * 32, nc0);
-            tma_load_2d(dst + C::kCodes, &tmScales, bar, nc0, j);
-          } else {                     // codes box 64 B x 64 rows, scales box 64 x 2
-            tma_load_2d(dst, &tmCodes, bar, nc0 / 2, j * 64);
-            tma_load_2d(dst + C::kCodes, &tmScales, bar, j * 64, nc0 / 64);
-          }
-        }
-      }
-      for (int k = 0; k < C::SC && k < int(ic); ++k) {
-        const uint32_t i2 = ic - 1 - k;
-        mbar_wait(cfull(i2 % C::SC), (i2 / C::SC) & 1u, 100000000ull);
-      }
-    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (rank == 0 && lane == 0) {
@@ -658,7 +616,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       tc_commit_pair_mc(drain_bar, 0x1);
       mbar_wait(drain_bar, 0, 100000000ull);
     }
-  } else if (warp < 7) {
+  } else if (warp < uint32_t(C::kFirstDeqWarp)) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const uint32_t q = warp & 3u;
     const uint32_t row = q * 32 + lane;
@@ -699,59 +657,52 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ dequantizers (both CTAs)
-    const uint32_t own = (warp - 7) / C::kWarpsPerSlot;   // slot this warp fills
-    const uint32_t sub = (warp - 7) % C::kWarpsPerSlot;   // threads t in [32 sub, 32 sub + 32)
+    const uint32_t dw = warp - uint32_t(C::kFirstDeqWarp);
+    const uint32_t own = dw / C::kWarpsPerSlot;   // slot this warp fills
+    const uint32_t sub = dw % C::kWarpsPerSlot;   // threads t in [32 sub, 32 sub + 32)
     const uint32_t row = sub * 32 + lane;
     const uint32_t ready_even = mapa_shared(ready(own), 0);
-    const uint32_t sig_even = mapa_shared(smem_base + C::kSigOff + (warp - 7) * C::kSigBytes, 0);
-    uint32_t it = 0;
-    bool ok = true;
-    for (int t = pair; t < num_tiles && ok; t += npairs) {
-      const int nc0 = (t % p.tiles_n) * 256 + int(rank) * 128;
-      for (int j = 0; j < nsteps; ++j, ++it) {
-        const bool main_step = j < p.num_k_main;
-        if ((it % C::S) != own) continue;
-        const uint32_t round = it / C::S;
-        const uint32_t b_tile = slot(it) + C::kA;
-        if (!__all_sync(0xffffffffu, mbar_wait(cfull(it % C::SC), (it / C::SC) & 1u))) {
-          set_status_site(p.status, QLORA_ERR_TIMEOUT, 108); ok = false; break;
-        }
-        if (main_step) {
-          const uint8_t* cs = smem + c_off(it);
-          const float* ss = reinterpret_cast<const float*>(cs + C::kCodes);
-          PairBlock blk;
-          dequant_load_pair<C::B_MN>(row, 0, cs, ss, blk);
-          if (!__all_sync(0xffffffffu, mbar_wait(empty(own), (round & 1u) ^ 1u))) {
-            set_status_site(p.status, QLORA_ERR_TIMEOUT, 118); ok = false; break;
-          }
-          dequant_store_pair<C::B_MN>(row, 0, blk, b_tile);
-          dequant_load_pair<C::B_MN>(row, 1, cs, ss, blk);
-          dequant_store_pair<C::B_MN>(row, 1, blk, b_tile);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(cempty(it % C::SC));
-          if (lane == 0) {
-            if (rank == 0) mbar_arrive(ready(own));
-            else st_async_signal(sig_even, ready_even);
-          }
-        } else {
-          if (lane == 0) mbar_arrive(cempty(it % C::SC));
-          if (!__all_sync(0xffffffffu, mbar_wait(empty(own), (round & 1u) ^ 1u))) {
-            set_status_site(p.status, QLORA_ERR_TIMEOUT, 118); ok = false; break;
-          }
-          // LoRA step: B half by TMA; its bytes were posted by the even A producer
-          if (lane == 0) {
-            const int kx = (j - p.num_k_main) * 64;
-            if (rank == 0) {
-              if (sub == 0) tma_load_2d(b_tile, &tmBx, ready(own), kx, nc0);
-              mbar_arrive(ready(own));
-            } else {
-              if (sub == 0) tma_load_2d_pair(b_tile, &tmBx, ready_even, kx, nc0);
-            }
-          }
-        }
-        __syncwarp();
+    const uint32_t sig_even = mapa_shared(smem_base + C::kSigOff + dw * C::kSigBytes, 0);
+    // this pair's steps are numbered it = (tile of the pair) * nsteps + j; this
+    // warp owns it = own, own + S, ...
+    const uint32_t total = uint32_t((num_tiles - pair + npairs - 1) / npairs) * uint32_t(nsteps);
+    auto tile_of = [&](uint32_t i) { return pair + int(i / uint32_t(nsteps)) * npairs; };
+    auto nc0_of = [&](int t) { return (t % p.tiles_n) * 256 + int(rank) * 128; };
+    PairRaw raw;
+    if (own < total && int(own % uint32_t(nsteps)) < p.num_k_main)
+      pair_load_raw<C::B_MN>(p, row, int(own % uint32_t(nsteps)), nc0_of(tile_of(own)), raw);
+    for (uint32_t it = own; it < total; it += C::S) {
+      const int t = tile_of(it), j = int(it % uint32_t(nsteps));
+      const uint32_t round = it / C::S;
+      const uint32_t b_tile = slot(it) + C::kA;
+      if (!__all_sync(0xffffffffu, mbar_wait(empty(own), (round & 1u) ^ 1u))) {
+        set_status_site(p.status, QLORA_ERR_TIMEOUT, 118);
+        break;
       }
+      if (j < p.num_k_main) {
+        pair_store_block<C::B_MN>(row, 0, raw, b_tile);
+        pair_store_block<C::B_MN>(row, 1, raw, b_tile);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(ready(own));
+          else st_async_signal(sig_even, ready_even);
+        }
+      } else if (lane == 0) {
+        // LoRA step: B half by TMA; its bytes were posted by the even A producer
+        const int kx = (j - p.num_k_main) * 64;
+        if (rank == 0) {
+          if (sub == 0) tma_load_2d(b_tile, &tmBx, ready(own), kx, nc0_of(t));
+          mbar_arrive(ready(own));
+        } else if (sub == 0) {
+          tma_load_2d_pair(b_tile, &tmBx, ready_even, kx, nc0_of(t));
+        }
+      }
+      // codes of this warp's next step, in flight while it waits for that slot
+      const uint32_t nx = it + C::S;
+      if (nx < total && int(nx % uint32_t(nsteps)) < p.num_k_main)
+        pair_load_raw<C::B_MN>(p, row, int(nx % uint32_t(nsteps)), nc0_of(tile_of(nx)), raw);
+      __syncwarp();
     }
   }
 
@@ -872,7 +823,7 @@ static qlora_status launch_pair_cfg(const GemmOperands& o, GemmParams p, cudaStr
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, tc_gemm_nf4_pair_kernel<C>, o.A, o.codes, o.scales, o.Ax, o.Bx, p) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, tc_gemm_nf4_pair_kernel<C>, o.A, o.Ax, o.Bx, p) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }

@@ -30,6 +30,12 @@ struct GemmParams {
   void* fin_out;
   int fin_mode;
   float fin_scale;
+  // CTA-pair NF4 kernel: packed codes [out x in/2] and expanded scales S_t
+  // [in/64 x out] read directly by the dequantizer warps
+  const uint8_t* codes;
+  const float* scales;
+  int64_t codes_ld;   // bytes between code rows (in / 2)
+  int64_t scales_ld;  // floats between S_t rows (out)
 };
 
 struct GemmOperands {
