@@ -75,7 +75,7 @@ FwdLayout fwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
 }
 
 struct BwdLayout {
-  size_t scales, l1s, t, u, part, counters, total;
+  size_t scales, l1s, t, u, su, part, counters, total;
 };
 
 BwdLayout bwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
@@ -86,6 +86,7 @@ BwdLayout bwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
   L.l1s = off;    off += up256(size_t(in) * r * 2);
   L.t = off;      off += up256(size_t(M) * r * 2);
   L.u = off;      off += up256(size_t(M) * r * 2);
+  L.su = off;     off += up256(size_t(M) * r * 2);
   const ThinSplit a = thin_split(M, in / 64), b = thin_split(M, out / 64);
   const ThinSplit c = thin_split(out, (M + 63) / 64), d = thin_split(in, (M + 63) / 64);
   size_t part = std::max({size_t(a.splits) * M * r, size_t(b.splits) * M * r, size_t(c.splits) * out * r,
@@ -130,7 +131,7 @@ struct Thin {
 };
 
 qlora_status run_thin(const Thin& t, float* part, int* counters, void* fin_out, int fin_mode, float fin_scale,
-                      int* status, cudaStream_t s) {
+                      int* status, cudaStream_t s, void* fin_out2 = nullptr) {
   const ThinSplit ts = thin_split(t.rows, t.ksteps);
   const int bn = thin_bn(t.r);
   GemmOperands o;
@@ -159,6 +160,7 @@ qlora_status run_thin(const Thin& t, float* part, int* counters, void* fin_out, 
   p.fin_out = fin_out;
   p.fin_mode = fin_mode;
   p.fin_scale = fin_scale;
+  p.fin_out2 = fin_out2;
   return launch_gemm(t.kind, bn, o, p, s);
 }
 
@@ -193,6 +195,45 @@ bool use_pair_kernel() {
   return v == 1;
 }
 
+// Fused NF4 GEMM on CTA pairs (256 x 256 tiles): out = A . W' + Ax . Bx^T, where
+// the LoRA step reads Bx as [N x r] rows: Ax = T with Bx = s.L2^T (fwd), or
+// Ax = s.U with Bx = L1 as stored (dX). Codes are read in place, scales from S_t.
+// (An MN-major LoRA B read straight from L2 [r x out] was measured 12 us slower
+// per forward GEMM on the q_proj workload than this transposed copy.)
+qlora_status run_pair(bool dx, const qlora_weight* w, const uint16_t* A, int64_t M, const uint16_t* Ax,
+                      const uint16_t* Bx, int32_t r, const float* scales_t, uint16_t* out, int* status,
+                      cudaStream_t s) {
+  const int64_t o_ = w->out, h = w->in;
+  const int64_t Kdim = dx ? o_ : h;
+  const int64_t Ndim = dx ? h : o_;
+  GemmOperands pp;
+  std::memset(&pp, 0, sizeof(pp));
+  if (!make_tmap_2d(&pp.A, A, TmapType::BF16, Kdim, M, Kdim * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d(&pp.Ax, Ax, TmapType::BF16, r, M, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d(&pp.Bx, Bx, TmapType::BF16, r, Ndim, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = int(M);
+  p.N = int(Ndim);
+  p.num_k_main = int(Kdim / 64);
+  p.num_k_ext = (r + 63) / 64;
+  p.tiles_m = int((M + 255) / 256);
+  p.tiles_n = int(Ndim / 256);
+  p.splits = 1;
+  p.ksteps_per_split = p.num_k_main;
+  p.out = out;
+  p.ld_out = Ndim;
+  p.status = status;
+  p.codes = w->codes;
+  p.codes_ld = h / 2;
+  p.scales = scales_t;
+  p.scales_ld = o_;
+  record_prof(g_prof[dx ? 2 : 0], s);
+  const qlora_status st = launch_gemm_pair(dx, pp, p, s);
+  record_prof(g_prof[dx ? 3 : 1], s);
+  return st;
+}
+
 // main GEMM with NF4 or bf16 weight and the LoRA extension
 qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t M, const uint16_t* Ax,
                       const uint16_t* Bx, int32_t r, const float* scales_t, uint16_t* out, int* status,
@@ -205,36 +246,6 @@ qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
   if (!make_tmap_2d(&op.A, A, TmapType::BF16, Kdim, M, Kdim * 2, 64, 128, true)) return QLORA_ERR_CUDA;
   if (!make_tmap_2d(&op.Ax, Ax, TmapType::BF16, r, M, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
   if (!make_tmap_2d(&op.Bx, Bx, TmapType::BF16, r, Ndim, int64_t(r) * 2, 64, 256, true)) return QLORA_ERR_CUDA;
-  if (!w->is_bf16 && use_pair_kernel()) {
-    // CTA-pair fused kernel: 256 x 256 tiles; each CTA holds 128 A rows and
-    // 128 rows (fwd) or columns (dX) of B.
-    GemmOperands pp;
-    std::memset(&pp, 0, sizeof(pp));
-    pp.A = op.A;
-    pp.Ax = op.Ax;
-    if (!make_tmap_2d(&pp.Bx, Bx, TmapType::BF16, r, Ndim, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
-    GemmParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.M = int(M);
-    p.N = int(Ndim);
-    p.num_k_main = int(Kdim / 64);
-    p.num_k_ext = (r + 63) / 64;
-    p.tiles_m = int((M + 255) / 256);
-    p.tiles_n = int(Ndim / 256);
-    p.codes = w->codes;
-    p.scales = scales_t;
-    p.codes_ld = h / 2;
-    p.scales_ld = o_;
-    p.splits = 1;
-    p.ksteps_per_split = p.num_k_main;
-    p.out = out;
-    p.ld_out = Ndim;
-    p.status = status;
-    record_prof(g_prof[dx ? 2 : 0], s);
-    const qlora_status st = launch_gemm_pair(dx, pp, p, s);
-    record_prof(g_prof[dx ? 3 : 1], s);
-    return st;
-  }
   GemmKind kind;
   if (w->is_bf16) {
     if (!dx) {
@@ -389,14 +400,15 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t 
   uint16_t* T = T_save ? T_save : reinterpret_cast<uint16_t*>(ws + L.t);
   float* part = reinterpret_cast<float*>(ws + L.part);
   const int64_t h = w->in, o_ = w->out;
+  int* counters = reinterpret_cast<int*>(ws + L.counters);
+  // T = X L1 : A = X (K-major), B = L1 as [h x r] (MN-major for B)
+  Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
   if (!w->is_bf16)
     QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
                                  scales_t, s));
   QLB_TRY(launch_scale_lora(L2, r, o_, scale, /*transpose=*/true, l2t, s));
-  // T = X L1 : A = X (K-major), B = L1 as [h x r] (MN-major for B)
-  int* counters = reinterpret_cast<int*>(ws + L.counters);
-  Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
   QLB_TRY(run_thin(tt, part, counters, T, 0, 1.f, status, s));
+  if (!w->is_bf16 && use_pair_kernel()) return run_pair(false, w, X, M, T, l2t, r, scales_t, Y, status, s);
   return run_main(false, w, X, M, T, l2t, r, scales_t, Y, status, s);
 }
 
@@ -430,15 +442,24 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const ui
     QLB_TRY(run_thin(tt, part, counters, Tw, 0, 1.f, status, s));
     T = Tw;
   }
-  // U = dY L2^T : A = dY (K-major, K = out), B = L2 [r x out] (K-major)
+  // U = dY L2^T : A = dY (K-major, K = out), B = L2 [r x out] (K-major); with
+  // the pair engine also s.U, the dX LoRA step's A
+  const bool pair = !w->is_bf16 && use_pair_kernel();
+  uint16_t* sU = reinterpret_cast<uint16_t*>(ws + L.su);
   Thin tu{GemmKind::ThinKK, dY, o_, M, L2, o_, r, M, o_ / 64, r};
-  QLB_TRY(run_thin(tu, part, counters, U, 0, 1.f, status, s));
+  if (pair && dX) QLB_TRY(run_thin(tu, part, counters, U, 3, scale, status, s, sU));
+  else QLB_TRY(run_thin(tu, part, counters, U, 0, 1.f, status, s));
   // dL2 = s (dY^T T)^T : A = dY^T (MN-major), B = T (MN-major); K = M; written transposed
   Thin t2{GemmKind::ThinMM, dY, o_, M, T, r, M, o_, mk, r};
   QLB_TRY(run_thin(t2, part, counters, dL2, 2, scale, status, s));
   // dL1 = s X^T U (in x r): A = X^T (MN-major), B = U (MN-major); K = M
   Thin t1{GemmKind::ThinMM, X, h, M, U, r, M, h, mk, r};
   QLB_TRY(run_thin(t1, part, counters, dL1, 1, scale, status, s));
+  if (dX && pair) {
+    QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
+                                 scales_t, s));
+    return run_pair(true, w, dY, M, sU, L1, r, scales_t, dX, status, s);
+  }
   if (dX) {
     if (!w->is_bf16)
       QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,

@@ -346,6 +346,18 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                   o2.x = pack_bf16x2(acc4.x, acc4.y);
                   o2.y = pack_bf16x2(acc4.z, acc4.w);
                   *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.fin_out) + int64_t(grow) * p.N + c4) = o2;
+                } else if (p.fin_mode == 3) {
+                  uint2 o2;
+                  o2.x = pack_bf16x2(acc4.x, acc4.y);
+                  o2.y = pack_bf16x2(acc4.z, acc4.w);
+                  *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.fin_out) + int64_t(grow) * p.N + c4) = o2;
+                  // the same bf16 values times the LoRA scale, rounded once more to bf16
+                  uint2 s2;
+                  s2.x = pack_bf16x2(__fmul_rn(__uint_as_float(o2.x << 16), p.fin_scale),
+                                     __fmul_rn(__uint_as_float(o2.x & 0xFFFF0000u), p.fin_scale));
+                  s2.y = pack_bf16x2(__fmul_rn(__uint_as_float(o2.y << 16), p.fin_scale),
+                                     __fmul_rn(__uint_as_float(o2.y & 0xFFFF0000u), p.fin_scale));
+                  *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.fin_out2) + int64_t(grow) * p.N + c4) = s2;
                 } else if (p.fin_mode == 1) {
                   float* d = reinterpret_cast<float*>(p.fin_out) + int64_t(grow) * p.N + c4;
                   *reinterpret_cast<float4*>(d) = make_float4(__fmul_rn(acc4.x, p.fin_scale), __fmul_rn(acc4.y, p.fin_scale),
@@ -456,9 +468,11 @@ struct PairCfg {
 //     nc0 + t, nc0 + t + 64 at K block j).
 //   dX (MN-major B, 64 K rows x 128 columns): blocks are K row t (weight row
 //     64 j + t) of the column chunks 0 and 1 (weight columns nc0 .. nc0 + 127).
-// The packed codes and scales are read straight from global memory (L2) into
-// registers one owned step ahead, so they are in place when the slot frees; the
-// product tables are built after the slot wait.
+// The packed codes and expanded scales are read straight from global memory (L2)
+// into registers one owned step ahead, so they are in place when the slot frees;
+// the product tables are built after the slot wait. (Reading the E4M3 scales in
+// place instead was measured slower: the per-row scale bytes are 64 bytes apart,
+// so every warp load touches 32 sectors.)
 struct PairRaw {
   uint4 c[2][2];   // 32 code bytes per block
   float a[2];      // block scales
@@ -580,8 +594,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (rank == 0 && lane == 0) {
       constexpr uint32_t idesc_main = make_idesc_bf16(256, 256, 0, C::B_MN ? 1 : 0);
+      // the LoRA steps' B is K-major in both directions ([N x r] rows)
       constexpr uint32_t idesc_ext = make_idesc_bf16(256, 256, 0, 0);
       constexpr uint32_t b_adv = C::B_MN ? (2048u >> 4) : (32u >> 4);
+      constexpr uint32_t b_adv_ext = 32u >> 4;
       // descriptors are linear in the start address (bits 0..13 hold addr >> 4);
       // the MN-major B half is two 64-column chunks 8 KB apart (leading offset),
       // which a K-major operand ignores
@@ -603,7 +619,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           tc_fence_after();
           const bool ext = j >= p.num_k_main;
           const uint64_t ad = da_base + si * kSlotAdv, bd = db_base + si * kSlotAdv;
-          const uint32_t badv = ext ? (32u >> 4) : b_adv;
+          const uint32_t badv = ext ? b_adv_ext : b_adv;
           const uint32_t idesc = ext ? idesc_ext : idesc_main;
 #pragma unroll
           for (uint32_t kk = 0; kk < 4; ++kk)
@@ -690,13 +706,13 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         }
       } else if (lane == 0) {
         // LoRA step: B half by TMA; its bytes were posted by the even A producer
-        const int kx = (j - p.num_k_main) * 64;
-        if (rank == 0) {
-          if (sub == 0) tma_load_2d(b_tile, &tmBx, ready(own), kx, nc0_of(t));
-          mbar_arrive(ready(own));
-        } else if (sub == 0) {
-          tma_load_2d_pair(b_tile, &tmBx, ready_even, kx, nc0_of(t));
+        const int kx = (j - p.num_k_main) * 64, n0 = nc0_of(t);
+        const uint32_t bar = rank == 0 ? ready(own) : ready_even;
+        if (sub == 0) {   // [N x r] rows n0.. (s.L2^T for the forward pass, L1 for dX)
+          if (rank == 0) tma_load_2d(b_tile, &tmBx, bar, kx, n0);
+          else tma_load_2d_pair(b_tile, &tmBx, bar, kx, n0);
         }
+        if (rank == 0) mbar_arrive(ready(own));
       }
       // codes of this warp's next step, in flight while it waits for that slot
       const uint32_t nx = it + C::S;

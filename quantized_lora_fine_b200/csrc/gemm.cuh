@@ -28,13 +28,15 @@ struct GemmParams {
   // Counters (one int per M tile) must start at zero; the kernel leaves them zero.
   int* counters;
   void* fin_out;
-  int fin_mode;
+  int fin_mode;       // 3: bf16 [M x N] to fin_out and bf16(fin_scale * that) to fin_out2
   float fin_scale;
-  // CTA-pair NF4 kernel: packed codes [out x in/2] and expanded scales S_t
-  // [in/64 x out] read directly by the dequantizer warps
+  void* fin_out2;
+  // CTA-pair NF4 kernel: packed codes [out x in/2] and expanded block scales S_t
+  // [in/64 x out] (S_t[j][n] = scale of weight row n, block j), read directly by
+  // the dequantizer warps (coalesced in both orientations)
   const uint8_t* codes;
-  const float* scales;
   int64_t codes_ld;   // bytes between code rows (in / 2)
+  const float* scales;
   int64_t scales_ld;  // floats between S_t rows (out)
 };
 
