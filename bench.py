@@ -180,6 +180,48 @@ class ClockSampler:
                 "reasons": sorted(seen), "samples": len(rows)}
 
 
+def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3):
+    """Quantize-all and error/rank over the 224-matrix Llama-7B-shaped stack."""
+    mats = synth.stack_matrices()
+    Ws = [synth.stack_weight(m, device=str(dev)) for m in mats]
+    numel = sum(w.numel() for w in Ws)
+    nb = numel // 64
+    q_bytes = numel * 2 + numel // 2 + nb * 4              # bf16 in; codes, fp32 absmax out (no double quant)
+    e_bytes = numel * 2
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    outs = []
+    for w in Ws:   # outputs allocated once, outside the timed region
+        outs.append((torch.empty(w.numel() // 2, dtype=torch.uint8, device=dev),
+                     torch.empty(w.numel() // 64, dtype=torch.float32, device=dev)))
+    q_ms, e_ms = [], []
+    for i in range(reps + 1):
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for w, (c, a) in zip(Ws, outs):
+            api.quantize(w, codes=c, absmax=a)
+        e1.record(stream)
+        e1.synchronize()
+        if i:
+            q_ms.append(e0.elapsed_time(e1))
+        e0.record(stream)
+        err, order, keep = api.layer_error_rank(Ws, 16, double_quant=False)
+        e1.record(stream)
+        e1.synchronize()
+        if i:
+            e_ms.append(e0.elapsed_time(e1))
+    assert api.status() == 0, "device status set in the codec legs"
+    qm, em = min(q_ms), min(e_ms)
+    del Ws, outs
+    torch.cuda.empty_cache()
+    return {"workload": "llama7b stack: 224 matrices (32 x q,k,v,o 4096^2, gate/up 11008x4096, down 4096x11008), "
+                        "6.48 G weights, per-matrix scale * Student-t(nu), NF4 blocksize 64, no double quant",
+            "quantize_all": {"ms": qm, "bytes": q_bytes, "GB/s": q_bytes / (qm * 1e-3) / 1e9,
+                             "frac_hbm": q_bytes / (qm * 1e-3) / 1e9 / peaks["hbm"], "launches": len(mats)},
+            "error_rank_all": {"ms": em, "bytes": e_bytes, "GB/s": e_bytes / (em * 1e-3) / 1e9,
+                               "frac_hbm": e_bytes / (em * 1e-3) / 1e9 / peaks["hbm"], "launches": 1},
+            "timing": f"best of {reps} (inputs 12.95 GB, far above L2)"}
+
+
 def gpu_main(args):
     import ctypes
 
@@ -378,6 +420,16 @@ def gpu_main(args):
         e2e = {"value": fl * world / (em * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": em,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    # ------------------------------------------------ codec kernels at full model scale
+    # The q_proj weight (33.5 MB) fits in L2 and its kernels last tens of
+    # microseconds; the HBM roofline of the quantizer and the error pass is taken
+    # on the Llama-7B-shaped stack instead: 224 matrices, 6.48 G weights (12.95 GB
+    # of bf16), quantize every matrix (one call each) and one error/rank call over
+    # all of them, as the allocation pass does.
+    hbm = None
+    if rank == 0 and world == 1 and not args.no_hbm_legs:
+        hbm = hbm_legs(api, synth, torch, dev, stream, peaks)
+
     # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -385,11 +437,11 @@ def gpu_main(args):
         cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": desc + f"; repeated for {secs:.1f} s", "seconds": secs}
 
-    launches_per_step = 1 + 3 + 4 + 6  # quantize; error chunk/finish/rank; fwd (scales, L2 prep, T, GEMM); bwd (U, dL2, dL1, scales, L1 prep, dX GEMM)
+    launches_per_step = 1 + 1 + 4 + 5  # quantize; error/rank; fwd (scales, s.L2^T, T, GEMM); bwd (U + s.U, dL2, dL1, scales, dX GEMM)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args, world),
-            "roofline": roofline, "legs": legs_out, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "legs": legs_out, "hbm_legs": hbm, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
             "timing": "cuda-graph replay of the step" if use_graphs else "eager API calls",
             "peaks": {"bf16_tflops": peaks["bf16"], "bf16_tflops_sustained": peaks["bf16_sus"],
@@ -413,6 +465,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-hbm-legs", action="store_true", help="skip the full-stack quantizer / error-pass legs")
     ap.add_argument("--eager", action="store_true", help="time eager API calls instead of CUDA-graph replays")
     args = ap.parse_args()
     if args.warmup < 3:

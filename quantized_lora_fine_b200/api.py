@@ -96,8 +96,10 @@ class NF4Weight:
         return s
 
 
-def quantize(W: torch.Tensor, double_quant: bool = False, keep_absmax: bool = False) -> NF4Weight:
-    """NF4-quantize a 2-D bf16 or fp32 CUDA tensor stored out x in."""
+def quantize(W: torch.Tensor, double_quant: bool = False, keep_absmax: bool = False,
+             codes: Optional[torch.Tensor] = None, absmax: Optional[torch.Tensor] = None) -> NF4Weight:
+    """NF4-quantize a 2-D bf16 or fp32 CUDA tensor stored out x in. `codes` and
+    `absmax` may be given as preallocated outputs (no double quant)."""
     if W.dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("W must be bf16 or fp32")
     _need(W, W.dtype, "W")
@@ -106,8 +108,14 @@ def quantize(W: torch.Tensor, double_quant: bool = False, keep_absmax: bool = Fa
     n = W.numel()
     nb = (n + 63) // 64
     dev = W.device
-    codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev)
-    absmax = torch.empty(nb, dtype=torch.float32, device=dev) if (not double_quant or keep_absmax) else None
+    if codes is None:
+        codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev)
+    elif codes.numel() < (n + 1) // 2 or codes.dtype != torch.uint8 or not codes.is_contiguous():
+        raise ValueError("codes: need a contiguous uint8 tensor of (numel + 1) // 2 bytes")
+    if absmax is None:
+        absmax = torch.empty(nb, dtype=torch.float32, device=dev) if (not double_quant or keep_absmax) else None
+    elif absmax.numel() < nb or absmax.dtype != torch.float32 or not absmax.is_contiguous():
+        raise ValueError("absmax: need a contiguous fp32 tensor of one value per 64 weights")
     absmax_q = torch.empty(nb, dtype=torch.uint8, device=dev) if double_quant else None
     absmax2 = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev) if double_quant else None
     ws = Workspace.get(lib.nf4_quantize_workspace_size(n), dev)

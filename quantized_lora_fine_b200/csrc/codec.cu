@@ -69,57 +69,118 @@ __device__ __forceinline__ void dq_group(const float* s_amax, float* s_red, int6
   if (tid == 0) absmax2[g] = (G > 0.f) ? __fdiv_rn(G, 448.f) : 0.f;
 }
 
-// bf16 weights, full chunks of 8: integer absmax on packed pairs, reciprocal
-// division (exact for bf16 operands), cell-table code lookup.
+// bf16 weights. One CTA of 256 threads per group of 256 blocks (16384 elements);
+// in each of 4 passes a thread takes 16 consecutive elements (4 threads per block,
+// a CTA covers 8 KB contiguous per pass), loading the next pass while it codes the
+// current one. Per block: integer absmax on packed bf16 pairs (4-lane shuffle
+// max) and one IEEE reciprocal. Per element pair: Markstein division in packed
+// fp32 (exact RN(w / a) for bf16 operands); per element the code index comes from
+// the 33-cell table on the FMA pipe (cell address by RZ multiply-add, one
+// shared-memory load, a saturating FMA for the midpoint test) and is accumulated
+// as fp32 nibble weights.
+__device__ __forceinline__ void quant_load16(const uint16_t* __restrict__ W, int64_t e, int64_t numel,
+                                             uint4 (&r)[2]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t eh = e + 8 * h;
+    if (eh + 8 <= numel) {
+      r[h] = __ldg(reinterpret_cast<const uint4*>(W + eh));
+    } else {
+      uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;
+      if (eh + 0 < numel) t0 |= uint32_t(W[eh + 0]);
+      if (eh + 1 < numel) t0 |= uint32_t(W[eh + 1]) << 16;
+      if (eh + 2 < numel) t1 |= uint32_t(W[eh + 2]);
+      if (eh + 3 < numel) t1 |= uint32_t(W[eh + 3]) << 16;
+      if (eh + 4 < numel) t2 |= uint32_t(W[eh + 4]);
+      if (eh + 5 < numel) t2 |= uint32_t(W[eh + 5]) << 16;
+      if (eh + 6 < numel) t3 |= uint32_t(W[eh + 6]);
+      if (eh + 7 < numel) t3 |= uint32_t(W[eh + 7]) << 16;
+      r[h] = make_uint4(t0, t1, t2, t3);
+    }
+  }
+}
+
+// Codes of 16 bf16 weights (8 packed pairs) of a block with absmax am > 0, as two
+// words in storage order (byte k = idx[2k] << 4 | idx[2k + 1]).
+__device__ __forceinline__ uint2 quant16_bf16(const uint32_t (&u)[8], float am, uint32_t tbl) {
+  float a = am;
+  uint64_t wp[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) wp[i] = f2_from_bf16x2(u[i]);
+  if (am < 0x1p-100f) {   // tiny block: rescale by 2^64 (exact) so that 1/a stays normal
+    a = am * 0x1p64f;
+    const uint64_t s64 = f2_splat(0x1p64f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wp[i] = f2_mul(wp[i], s64);
+  }
+  const uint64_t r2 = f2_splat(__frcp_rn(a)), na2 = f2_splat(-a);
+  uint32_t word[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    // within a 16-bit half the 4 elements weigh 16, 1, 4096, 256 (storage order)
+    float acc[2] = {0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint64_t q = f2_div_by_recip(wp[4 * h + i], na2, r2);
+      const float n0 = f2_lo(q), n1 = f2_hi(q);
+      const float2 t0 = lds_f2(coarse_addr<8>(n0, tbl)), t1 = lds_f2(coarse_addr<8>(n1, tbl));
+      const float w0 = (i & 1) ? 4096.f : 16.f, w1 = (i & 1) ? 256.f : 1.f;
+      acc[i >> 1] = __fmaf_rn(t0.y + sat_fma(n0, 0x1p100f, t0.x), w0, acc[i >> 1]);
+      acc[i >> 1] = __fmaf_rn(t1.y + sat_fma(n1, 0x1p100f, t1.x), w1, acc[i >> 1]);
+    }
+    word[h] = prmt(nibbles_from_f32(acc[0]), nibbles_from_f32(acc[1]), 0x5410u);
+  }
+  return make_uint2(word[0], word[1]);
+}
+
 template <bool DQ>
 __global__ void __launch_bounds__(256) nf4_quantize_bf16_kernel(const uint16_t* __restrict__ W, int64_t numel,
                                                                 uint8_t* __restrict__ codes,
                                                                 float* __restrict__ absmax,
                                                                 uint8_t* __restrict__ absmax_q,
                                                                 float* __restrict__ absmax2, int* status) {
+  __shared__ __align__(16) float2 s_tbl[33];
   __shared__ float s_amax[256];
   __shared__ float s_red[8];
-  __shared__ NF4CellSmem s_cells;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  nf4_cells_load(s_cells, tid);
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (tid < 33) s_tbl[tid] = make_float2(__uint_as_float(kNF4CoarseQ[2 * tid]), __uint_as_float(kNF4CoarseQ[2 * tid + 1]));
+  const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(s_tbl));
+  __syncthreads();
   const int64_t nb = (numel + kBlock - 1) / kBlock;
   const int64_t g = blockIdx.x;
-  // Prefetch all 8 slices of this thread (one 16-byte load each).
-  uint4 raw[8];
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int64_t e0 = (g * kDQBlock + it * 32 + warp * 4 + (lane >> 3)) * kBlock + (lane & 7) * 8;
-    raw[it] = (e0 + 8 <= numel) ? __ldg(reinterpret_cast<const uint4*>(W + e0)) : make_uint4(0, 0, 0, 0);
-    if (e0 < numel && e0 + 8 > numel) {  // ragged tail chunk
-      uint16_t tmp[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int i = 0; i < 8; ++i) if (e0 + i < numel) tmp[i] = W[e0 + i];
-      raw[it] = make_uint4(tmp[0] | (uint32_t(tmp[1]) << 16), tmp[2] | (uint32_t(tmp[3]) << 16),
-                           tmp[4] | (uint32_t(tmp[5]) << 16), tmp[6] | (uint32_t(tmp[7]) << 16));
-    }
-  }
-  __syncthreads();
+  const int64_t g0 = g * int64_t(kDQBlock * kBlock);   // first element of the group
   uint32_t bad = 0;
+  uint4 cur[2], nxt[2];
+  quant_load16(W, g0 + int64_t(tid) * 16, numel, cur);
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int bi = it * 32 + warp * 4 + (lane >> 3);
+  for (int k = 0; k < 4; ++k) {
+    if (k < 3) quant_load16(W, g0 + int64_t((k + 1) * 256 + tid) * 16, numel, nxt);
+    const int bi = (k * 256 + tid) >> 2;               // block within the group
     const int64_t blk = g * kDQBlock + bi;
-    const int64_t e0 = blk * kBlock + (lane & 7) * 8;
-    const uint32_t amb = block_max8_lanes(absmax8_bf16_bits(raw[it]));
+    const int64_t e0 = g0 + int64_t(k * 256 + tid) * 16;
+    const uint32_t u[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+    uint32_t m = __vmaxu2(u[0] & 0x7FFF7FFFu, u[1] & 0x7FFF7FFFu);
+#pragma unroll
+    for (int i = 2; i < 8; ++i) m = __vmaxu2(m, u[i] & 0x7FFF7FFFu);
+    uint32_t amb = max(m >> 16, m & 0xFFFFu);
+    amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 1));
+    amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 2));
     bad |= amb >= 0x7F80u;
     const float am = __uint_as_float(amb << 16);
-    if ((lane & 7) == 0) {
-      s_amax[bi] = am;
-      if (blk < nb && absmax != nullptr) absmax[blk] = am;
+    if ((lane & 3) == 0) {
+      if constexpr (DQ) s_amax[bi] = am;
+      if (absmax != nullptr && blk < nb) absmax[blk] = am;
     }
     if (e0 < numel) {
-      uint32_t idx[8];
-      const uint32_t word = (am > 0.f) ? quant8_bf16(raw[it], am, s_cells, idx) : 0x77777777u;
-      if (e0 + 8 <= numel) {
-        *reinterpret_cast<uint32_t*>(codes + e0 / 2) = word;
+      const uint2 word = (am > 0.f) ? quant16_bf16(u, am, tbl) : make_uint2(0x77777777u, 0x77777777u);
+      if (e0 + 16 <= numel) {
+        *reinterpret_cast<uint2*>(codes + e0 / 2) = word;
       } else {
-        for (int k = 0; 2 * k < numel - e0; ++k) codes[e0 / 2 + k] = uint8_t(word >> (8 * k));
+        const uint64_t both = (uint64_t(word.y) << 32) | word.x;
+        for (int kb = 0; 2 * kb < numel - e0; ++kb) codes[e0 / 2 + kb] = uint8_t(both >> (8 * kb));
       }
     }
+    if (k < 3) { cur[0] = nxt[0]; cur[1] = nxt[1]; }
   }
   if (bad) set_status(status, QLORA_ERR_NONFINITE);
   if constexpr (DQ) dq_group(s_amax, s_red, nb, g, absmax_q, absmax2);

@@ -3,9 +3,12 @@
 //
 // Pass 1: one CTA per chunk of 256 blocks (16384 elements) of some layer;
 //         quantizes, dequantizes and accumulates sum (w - w_hat)^2 and sum w^2
-//         in fp64; writes one partial pair per chunk (nothing else is written).
+//         in fp64; writes one partial pair per chunk.
 // Pass 2: per layer, sums its chunk partials in chunk order -> err.
 // Pass 3: one CTA ranks all layers by (err desc, id asc).
+// The workspace entry point runs all three in one launch (the last chunk CTA of a
+// layer does pass 2 for it, the last layer's finisher does pass 3); the
+// allocation-free entry point, which has no counters, launches them separately.
 #include <cfloat>
 #include <cuda_bf16.h>
 
@@ -25,79 +28,122 @@ struct LayerTable {
   int32_t n_layers;
 };
 
-// Error contribution of 8 bf16 weights of one block: codes from the exact absmax
-// a, reconstruction with ahat (= a, or the double-quantized scale). w and w_hat
-// are bf16 values within a small exponent range of each other (or w_hat = 0),
-// so d = w - w_hat and the squares d^2, w^2 are exact in fp32; the 8-term
-// partial sums carry at most 8 roundings before they are added in fp64.
-__device__ __forceinline__ void err8_bf16(uint4 v, float a, float ahat, const NF4CellSmem& cells, const float* s_code,
-                                          float& sd8, float& sw8) {
-  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-  uint32_t idx[8];
-  if (a > 0.f) quant8_bf16(v, a, cells, idx);
-  else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) idx[i] = 7u;
-  }
+// Error contribution of 16 bf16 weights (8 packed pairs) of one block: codes
+// from the exact absmax a (same arithmetic as the quantizer), reconstruction
+// w_hat = bf16(fp32(code * ahat)) with ahat = a, or the double-quantized scale.
+// Squares are summed per pair lane in fp32 (8 terms) before the fp64 total.
+template <bool kTiny>
+__device__ __forceinline__ void err16_core(const uint32_t (&u)[8], float a, float ahat, uint32_t tbl, double& sd,
+                                           double& sw) {
+  // tiny blocks: the division operands are rescaled by 2^64 (exact) so 1/a stays normal
+  const float as = kTiny ? a * 0x1p64f : a;
+  const uint64_t r2 = f2_splat(__frcp_rn(as)), na2 = f2_splat(-as), ah2 = f2_splat(ahat);
+  uint64_t sd2 = 0, sw2 = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float w = (i & 1) ? __uint_as_float(u[i >> 1] & 0xFFFF0000u) : __uint_as_float(u[i >> 1] << 16);
-    const float wh = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_code[idx[i]], ahat)));
-    const float d = __fsub_rn(w, wh);
-    sd8 = __fmaf_rn(d, d, sd8);
-    sw8 = __fmaf_rn(w, w, sw8);
+    const uint64_t w = f2_from_bf16x2(u[i]);
+    const uint64_t q = f2_div_by_recip(kTiny ? f2_mul(w, f2_splat(0x1p64f)) : w, na2, r2);
+    const float n0 = f2_lo(q), n1 = f2_hi(q);
+    // cell entry {code[base], code[base + 1]}; RN(lo + hi) is twice the cell's midpoint
+    const float2 e0 = lds_f2(coarse_addr<8>(n0, tbl)), e1 = lds_f2(coarse_addr<8>(n1, tbl));
+    const float s0 = sat_fma(__fadd_rn(e0.x, e0.y), -0x1p99f, __fmul_rn(n0, 0x1p100f));
+    const float s1 = sat_fma(__fadd_rn(e1.x, e1.y), -0x1p99f, __fmul_rn(n1, 0x1p100f));
+    const float c0 = __fmaf_rn(s0, __fsub_rn(e0.y, e0.x), e0.x);   // code value (exact)
+    const float c1 = __fmaf_rn(s1, __fsub_rn(e1.y, e1.x), e1.x);
+    const uint64_t p = f2_mul((uint64_t(__float_as_uint(c1)) << 32) | __float_as_uint(c0), ah2);
+    const uint64_t wh = f2_from_bf16x2(pack_bf16x2(f2_lo(p), f2_hi(p)));
+    const uint64_t d = f2_sub(w, wh);
+    sd2 = f2_fma(d, d, sd2);
+    sw2 = f2_fma(w, w, sw2);
   }
+  sd += double(f2_lo(sd2)) + double(f2_hi(sd2));
+  sw += double(f2_lo(sw2)) + double(f2_hi(sw2));
 }
 
+__device__ __forceinline__ void err16_bf16(const uint32_t (&u)[8], float a, float ahat, uint32_t tbl, double& sd,
+                                           double& sw) {
+  if (!(a > 0.f)) return;   // all-zero block: every w and w_hat is 0
+  if (a < 0x1p-100f) err16_core<true>(u, a, ahat, tbl, sd, sw);
+  else err16_core<false>(u, a, ahat, tbl, sd, sw);
+}
+
+// absmax (bf16 bits) of 16 weights, over the 4 lanes that share the block
+__device__ __forceinline__ uint32_t absmax16_lanes(const uint32_t (&u)[8]) {
+  uint32_t m = __vmaxu2(u[0] & 0x7FFF7FFFu, u[1] & 0x7FFF7FFFu);
+#pragma unroll
+  for (int i = 2; i < 8; ++i) m = __vmaxu2(m, u[i] & 0x7FFF7FFFu);
+  uint32_t amb = max(m >> 16, m & 0xFFFFu);
+  amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 1));
+  amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 2));
+  return amb;
+}
+
+__device__ __forceinline__ void finish_layer(const double2* __restrict__ partial, int c0, int c1,
+                                             double* __restrict__ err_out);
+
+// Pass 1 (and, with counters, passes 2-3 fused): one CTA per chunk of 256 blocks
+// of some layer; in each of 4 passes a thread takes 16 consecutive weights (4
+// threads per block). The chunk's (sum d^2, sum w^2) goes to partial[chunk]. With
+// counters (zero on entry, left zero): the last chunk CTA of a layer sums that
+// layer's partials in chunk order into err[layer], and the last layer to finish
+// ranks all layers and writes order / keep.
 template <bool DQ>
 __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_constant__ LayerTable tab,
-                                                                double2* __restrict__ partial, int* status) {
+                                                                double2* __restrict__ partial, int* status,
+                                                                int* counters, double* __restrict__ err, int K,
+                                                                int32_t* __restrict__ order, uint8_t* __restrict__ keep) {
+  __shared__ __align__(16) float2 s_tbl[33];
   __shared__ float s_amax[256];
   __shared__ float s_ahat[256];
   __shared__ float s_red[8];
-  __shared__ float s_code[16];
   __shared__ double s_sum[2][8];
-  __shared__ NF4CellSmem s_cells;
+  __shared__ int s_flag;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  nf4_cells_load(s_cells, tid);
-  if (tid < 16) s_code[tid] = nf4_code(tid);
+  if (tid < 33) s_tbl[tid] = make_float2(__uint_as_float(kNF4CoarseC[2 * tid]), __uint_as_float(kNF4CoarseC[2 * tid + 1]));
+  const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(s_tbl));
   const int chunk = blockIdx.x;
   int lo = 0, hi = tab.n_layers - 1;  // layer owning this chunk
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (tab.first_chunk[mid] <= chunk) lo = mid; else hi = mid - 1;
   }
-  const uint16_t* W = tab.ptr[lo];
-  const int64_t nb = tab.numel[lo] / kBlock;
-  const int64_t g = chunk - tab.first_chunk[lo];
-  auto load = [&](int it) -> uint4 {
-    const int64_t blk = g * kDQBlock + it * 32 + warp * 4 + (lane >> 3);
-    return (blk < nb) ? __ldg(reinterpret_cast<const uint4*>(W + blk * kBlock + (lane & 7) * 8)) : make_uint4(0, 0, 0, 0);
+  const int layer = lo;
+  const uint16_t* W = tab.ptr[layer];
+  const int64_t nb = tab.numel[layer] / kBlock;
+  const int64_t g = chunk - tab.first_chunk[layer];
+  // task k of this thread: weights [16 (tid & 3), +16) of block 64 k + tid / 4
+  auto load_task = [&](int k, uint32_t (&u)[8]) {
+    const int64_t blk = g * kDQBlock + ((k * 256 + tid) >> 2);
+    const uint16_t* src = W + blk * kBlock + (tid & 3) * 16;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    const uint4 v0 = (blk < nb) ? __ldg(reinterpret_cast<const uint4*>(src)) : z;
+    const uint4 v1 = (blk < nb) ? __ldg(reinterpret_cast<const uint4*>(src + 8)) : z;
+    u[0] = v0.x; u[1] = v0.y; u[2] = v0.z; u[3] = v0.w; u[4] = v1.x; u[5] = v1.y; u[6] = v1.z; u[7] = v1.w;
   };
-  uint4 raw[8];
-#pragma unroll
-  for (int it = 0; it < 8; ++it) raw[it] = load(it);
-  __syncthreads();
+  __syncthreads();   // the table is in place
   uint32_t bad = 0;
   double sd = 0.0, sw = 0.0;
-  float am_slice[8];
+  float am_k[4];
+  uint32_t cur[8], nxt[8];
+  load_task(0, cur);
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int bi = it * 32 + warp * 4 + (lane >> 3);
-    const uint32_t amb = block_max8_lanes(absmax8_bf16_bits(raw[it]));
+  for (int k = 0; k < 4; ++k) {
+    if (k < 3) load_task(k + 1, nxt);
+    const uint32_t amb = absmax16_lanes(cur);
     bad |= amb >= 0x7F80u;
     const float am = __uint_as_float(amb << 16);
-    am_slice[it] = am;
+    am_k[k] = am;
     if constexpr (DQ) {
-      if ((lane & 7) == 0) s_amax[bi] = am;
+      if ((tid & 3) == 0) s_amax[(k * 256 + tid) >> 2] = am;
     } else {
-      float sd8 = 0.f, sw8 = 0.f;
-      err8_bf16(raw[it], am, am, s_cells, s_code, sd8, sw8);
-      sd += double(sd8);
-      sw += double(sw8);
+      err16_bf16(cur, am, am, tbl, sd, sw);
+    }
+    if (k < 3) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
     }
   }
-  if (bad) set_status(status, QLORA_ERR_NONFINITE);
+  if (bad && status) set_status(status, QLORA_ERR_NONFINITE);
   if constexpr (DQ) {
     __syncthreads();
     const int64_t nblk_g = (int64_t(kDQBlock) < nb - g * kDQBlock ? int64_t(kDQBlock) : nb - g * kDQBlock);
@@ -117,13 +163,17 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
     }
     s_ahat[tid] = ah;
     __syncthreads();
+    // second pass over the chunk (from L2): codes use the exact absmax, the
+    // reconstruction the double-quantized scale
+    load_task(0, cur);
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int bi = it * 32 + warp * 4 + (lane >> 3);
-      float sd8 = 0.f, sw8 = 0.f;
-      err8_bf16(raw[it], am_slice[it], s_ahat[bi], s_cells, s_code, sd8, sw8);
-      sd += double(sd8);
-      sw += double(sw8);
+    for (int k = 0; k < 4; ++k) {
+      if (k < 3) load_task(k + 1, nxt);
+      err16_bf16(cur, am_k[k], s_ahat[(k * 256 + tid) >> 2], tbl, sd, sw);
+      if (k < 3) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
+      }
     }
   }
 #pragma unroll
@@ -138,6 +188,39 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
     for (int i = 0; i < 8; ++i) { a += s_sum[0][i]; b += s_sum[1][i]; }
     partial[chunk] = make_double2(a, b);
   }
+  if (counters == nullptr) return;
+  // ---- fused finish: last chunk of the layer -> err[layer]; last layer -> ranks
+  if (tid == 0) {
+    __threadfence();
+    const int nchunks = tab.first_chunk[layer + 1] - tab.first_chunk[layer];
+    const int done = atomicAdd(counters + 1 + layer, 1);
+    s_flag = (done == nchunks - 1);
+    if (s_flag) atomicExch(counters + 1 + layer, 0);
+  }
+  __syncthreads();
+  if (!s_flag) return;
+  __threadfence();
+  finish_layer(partial, tab.first_chunk[layer], tab.first_chunk[layer + 1], err + layer);
+  if (tid == 0) {
+    __threadfence();
+    const int done = atomicAdd(counters, 1);
+    s_flag = (done == tab.n_layers - 1);
+    if (s_flag) atomicExch(counters, 0);
+  }
+  __syncthreads();
+  if (!s_flag) return;
+  __threadfence();
+  const int n = tab.n_layers;
+  for (int l = tid; l < n; l += 256) {
+    const double e = __ldcg(err + l);
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const double f = __ldcg(err + j);
+      rank += (f > e || (f == e && j < l)) ? 1 : 0;
+    }
+    order[rank] = l;
+    keep[l] = rank < K ? 1 : 0;
+  }
 }
 
 // One CTA per layer: thread t sums chunks first+t, first+t+256, ... in order, then a
@@ -146,7 +229,11 @@ __device__ __forceinline__ void finish_layer(const double2* __restrict__ partial
                                              double* __restrict__ err_out) {
   __shared__ double s_a[256], s_b[256];
   double a = 0.0, b = 0.0;
-  for (int c = c0 + threadIdx.x; c < c1; c += 256) { a += partial[c].x; b += partial[c].y; }
+  for (int c = c0 + threadIdx.x; c < c1; c += 256) {
+    const double2 v = __ldcg(partial + c);
+    a += v.x;
+    b += v.y;
+  }
   s_a[threadIdx.x] = a;
   s_b[threadIdx.x] = b;
   __syncthreads();
@@ -208,11 +295,9 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
   tab.first_chunk[n_layers] = c;
   if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
   double2* partial = reinterpret_cast<double2*>(static_cast<char*>(ws) + kReservedBytes);
-  if (dq) layer_error_chunk_kernel<true><<<unsigned(c), 256, 0, s>>>(tab, partial, status);
-  else layer_error_chunk_kernel<false><<<unsigned(c), 256, 0, s>>>(tab, partial, status);
-  if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
-  layer_error_finish_table_kernel<<<n_layers, 256, 0, s>>>(partial, tab, err);
-  rank_topk_kernel<<<1, 1024, 0, s>>>(err, n_layers, K, order, keep);
+  int* counters = reinterpret_cast<int*>(static_cast<char*>(ws) + kStatusBytes);   // 1 + n_layers, zero
+  if (dq) layer_error_chunk_kernel<true><<<unsigned(c), 256, 0, s>>>(tab, partial, status, counters, err, K, order, keep);
+  else layer_error_chunk_kernel<false><<<unsigned(c), 256, 0, s>>>(tab, partial, status, counters, err, K, order, keep);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -278,8 +363,8 @@ qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const
     c += chunks_of(numel[i]);
   }
   tab.first_chunk[n_layers] = c;
-  if (dq) layer_error_chunk_kernel<true><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr);
-  else layer_error_chunk_kernel<false><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr);
+  if (dq) layer_error_chunk_kernel<true><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr, nullptr, err, K, order, keep);
+  else layer_error_chunk_kernel<false><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr, nullptr, err, K, order, keep);
   if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
   layer_error_finish_table_kernel<<<n_layers, 256, 0, s>>>(partial, tab, err);
   rank_topk_kernel<<<1, 1024, 0, s>>>(err, n_layers, K, order, keep);

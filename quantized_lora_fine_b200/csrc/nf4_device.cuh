@@ -136,6 +136,80 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: two IEEE fp32 operations in one
+// instruction, round to nearest, subnormals kept)
+__device__ __forceinline__ uint64_t f2_from_bf16x2(uint32_t u) {
+  // (element 0, element 1) of a bf16 pair as a packed fp32 pair
+  return (uint64_t(u & 0xFFFF0000u) << 32) | uint64_t(u << 16);
+}
+__device__ __forceinline__ uint64_t f2_splat(float x) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(uint32_t(v)); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(uint32_t(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// RN(w / a) for both elements of a pair, from r = RN(1/a) and na = -a (Markstein
+// step, as div_by_recip).
+__device__ __forceinline__ uint64_t f2_div_by_recip(uint64_t w, uint64_t na, uint64_t r) {
+  const uint64_t q0 = f2_mul(w, r);
+  const uint64_t e = f2_fma(q0, na, w);
+  return f2_fma(e, r, q0);
+}
+
+// ---- fine-cell code lookup, evaluated on the FMA pipe
+// Cell c = bits(n) >> 21 (2048 cells of 1/4 binade; each holds at most one
+// midpoint). s = sat(n * 2^100 + T_c) is exactly 1.0 when n is above the cell's
+// midpoint and 0.0 otherwise; the code index is base_c + s.
+__device__ __forceinline__ float sat_fma(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float2 fine_q_entry(const float2* tbl, float n) {
+  return tbl[__float_as_uint(n) >> 21];
+}
+// Coarse cell c = floor(16 (n + 1)) for n in [-1, 1], as a shared-memory address
+// without integer ALU work: bits(RZ(16 n + 16 + 2^23)) = 0x4B000000 + c, and one
+// integer multiply-add (mod 2^32) turns that into tbl + c * entry_bytes.
+template <uint32_t kEntryBytes>
+__device__ __forceinline__ uint32_t coarse_addr(float n, uint32_t tbl) {
+  float v;
+  asm("fma.rz.f32 %0, %1, 0f41800000, 0f4B000010;" : "=f"(v) : "f"(n));   // 16 n + (2^23 + 16)
+  return __float_as_uint(v) * kEntryBytes + (tbl - 0x4B000000u * kEntryBytes);
+}
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+// Four code indices accumulated as sum idx_p * 16^p in fp32 (exact below 2^16)
+// turn into integer bits through the 2^23 bias: low 16 bits of bits(h + 2^23).
+__device__ __forceinline__ uint32_t nibbles_from_f32(float h) {
+  return __float_as_uint(__fadd_rn(h, 8388608.0f));
+}
+
 // Per-block dequantization table: the 16 products bf16_rn(fp32_rn(c_j * a)) split
 // into a low-byte table (lo[0..3], byte j = low byte of entry j) and a high-byte
 // table (hi[0..3]).
