@@ -123,7 +123,9 @@ __device__ __forceinline__ uint2 quant16_bf16(const uint32_t (&u)[8], float am, 
     for (int i = 0; i < 4; ++i) {
       const uint64_t q = f2_div_by_recip(wp[4 * h + i], na2, r2);
       const float n0 = f2_lo(q), n1 = f2_hi(q);
-      const float2 t0 = lds_f2(coarse_addr<8>(n0, tbl)), t1 = lds_f2(coarse_addr<8>(n1, tbl));
+      const uint64_t cells = coarse_cells2(q);
+      const float2 t0 = lds_f2(coarse_addr_bits<8>(uint32_t(cells), tbl));
+      const float2 t1 = lds_f2(coarse_addr_bits<8>(uint32_t(cells >> 32), tbl));
       const float w0 = (i & 1) ? 4096.f : 16.f, w1 = (i & 1) ? 256.f : 1.f;
       acc[i >> 1] = __fmaf_rn(t0.y + sat_fma(n0, 0x1p100f, t0.x), w0, acc[i >> 1]);
       acc[i >> 1] = __fmaf_rn(t1.y + sat_fma(n1, 0x1p100f, t1.x), w1, acc[i >> 1]);

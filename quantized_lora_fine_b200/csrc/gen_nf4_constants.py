@@ -309,6 +309,10 @@ def render():
         "// first without a midpoint): s = sat(n 2^100 - RN(lo + hi) 2^99), code = lo + s (hi - lo).",
         "__device__ constexpr uint32_t kNF4CoarseC[33 * 2] = {",
         "    " + ", ".join("0x%08Xu, 0x%08Xu" % v for v in cc) + "};",
+        "// kNF4CoarseD[c] = {code[base], code[base + 1] - code[base]} (exact difference):",
+        "// RN(2 lo + diff) = RN(lo + hi) = twice the midpoint, code = lo + s diff.",
+        "__device__ constexpr uint32_t kNF4CoarseD[33 * 2] = {",
+        "    " + ", ".join("0x%08Xu, 0x%08Xu" % (v[1], v[2]) for v in ce) + "};",
         "// Arithmetic lookup on the FMA pipe: s = sat(n * 2^100 + T) is 1 iff n is above",
         "// the cell's midpoint. kNF4FineQ[c] = {T, base} (fp32 bits): idx = base + s.",
         "__device__ constexpr uint32_t kNF4FineQ[2048 * 2] = {",

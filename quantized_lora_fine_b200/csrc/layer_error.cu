@@ -43,13 +43,16 @@ __device__ __forceinline__ void err16_core(const uint32_t (&u)[8], float a, floa
   for (int i = 0; i < 8; ++i) {
     const uint64_t w = f2_from_bf16x2(u[i]);
     const uint64_t q = f2_div_by_recip(kTiny ? f2_mul(w, f2_splat(0x1p64f)) : w, na2, r2);
-    const float n0 = f2_lo(q), n1 = f2_hi(q);
-    // cell entry {code[base], code[base + 1]}; RN(lo + hi) is twice the cell's midpoint
-    const float2 e0 = lds_f2(coarse_addr<8>(n0, tbl)), e1 = lds_f2(coarse_addr<8>(n1, tbl));
-    const float s0 = sat_fma(__fadd_rn(e0.x, e0.y), -0x1p99f, __fmul_rn(n0, 0x1p100f));
-    const float s1 = sat_fma(__fadd_rn(e1.x, e1.y), -0x1p99f, __fmul_rn(n1, 0x1p100f));
-    const float c0 = __fmaf_rn(s0, __fsub_rn(e0.y, e0.x), e0.x);   // code value (exact)
-    const float c1 = __fmaf_rn(s1, __fsub_rn(e1.y, e1.x), e1.x);
+    // cell entries {code[base], code[base + 1] - code[base]}; RN(2 lo + diff) is twice
+    // the cell's midpoint, so s = sat(n 2^100 - RN(2 lo + diff) 2^99) tests n > m
+    const uint64_t cells = coarse_cells2(q);
+    const uint64_t n2 = f2_mul(q, 0x7180000071800000ull);   // n * 2^100, both lanes
+    const float2 e0 = lds_f2(coarse_addr_bits<8>(uint32_t(cells), tbl));
+    const float2 e1 = lds_f2(coarse_addr_bits<8>(uint32_t(cells >> 32), tbl));
+    const float s0 = sat_fma(__fmaf_rn(e0.x, 2.f, e0.y), -0x1p99f, f2_lo(n2));
+    const float s1 = sat_fma(__fmaf_rn(e1.x, 2.f, e1.y), -0x1p99f, f2_hi(n2));
+    const float c0 = __fmaf_rn(s0, e0.y, e0.x);   // code value (exact)
+    const float c1 = __fmaf_rn(s1, e1.y, e1.x);
     const uint64_t p = f2_mul((uint64_t(__float_as_uint(c1)) << 32) | __float_as_uint(c0), ah2);
     const uint64_t wh = f2_from_bf16x2(pack_bf16x2(f2_lo(p), f2_hi(p)));
     const uint64_t d = f2_sub(w, wh);
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
   __shared__ double s_sum[2][8];
   __shared__ int s_flag;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid < 33) s_tbl[tid] = make_float2(__uint_as_float(kNF4CoarseC[2 * tid]), __uint_as_float(kNF4CoarseC[2 * tid + 1]));
+  if (tid < 33) s_tbl[tid] = make_float2(__uint_as_float(kNF4CoarseD[2 * tid]), __uint_as_float(kNF4CoarseD[2 * tid + 1]));
   const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(s_tbl));
   const int chunk = blockIdx.x;
   int lo = 0, hi = tab.n_layers - 1;  // layer owning this chunk

@@ -194,6 +194,16 @@ __device__ __forceinline__ uint32_t coarse_addr(float n, uint32_t tbl) {
   asm("fma.rz.f32 %0, %1, 0f41800000, 0f4B000010;" : "=f"(v) : "f"(n));   // 16 n + (2^23 + 16)
   return __float_as_uint(v) * kEntryBytes + (tbl - 0x4B000000u * kEntryBytes);
 }
+// Both cells of a packed pair: bits of RZ(16 n + 16 + 2^23) per lane.
+__device__ __forceinline__ uint64_t coarse_cells2(uint64_t n2) {
+  uint64_t v;
+  asm("fma.rz.f32x2 %0, %1, %2, %3;" : "=l"(v) : "l"(n2), "l"(0x4180000041800000ull), "l"(0x4B0000104B000010ull));
+  return v;
+}
+template <uint32_t kEntryBytes>
+__device__ __forceinline__ uint32_t coarse_addr_bits(uint32_t cell_bits, uint32_t tbl) {
+  return cell_bits * kEntryBytes + (tbl - 0x4B000000u * kEntryBytes);
+}
 __device__ __forceinline__ float2 lds_f2(uint32_t addr) {
   float2 v;
   asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));

@@ -133,6 +133,20 @@ def cases_mlp(seed: int = 0, M: int = 8192) -> List[LinearCase]:
     ]
 
 
+def cases_14b(r: int, M: int = 16384, seed: int = 0, kinds=("q", "gate", "down"), layer: int = 0) -> List[LinearCase]:
+    """14B-shaped decoder linears (hidden 5120, intermediate 13824) with double
+    quant, rank r, alpha = 2r, X of M tokens; weights are the stack's per-matrix
+    scale * Student-t(nu) draws of the given layer."""
+    mats = {m.name: m for m in stack_matrices(n_layers=layer + 1, linears=QWEN14B_LINEARS, seed=seed)
+            if m.layer == layer}
+    out = []
+    for k in kinds:
+        m = mats[k]
+        out.append(LinearCase(f"14b-{k}-r{r}", M=M, out=m.out, inp=m.inp, r=r, alpha=2.0 * r, double_quant=True,
+                              w_dist="t", nu=m.nu, w_std=m.scale, seed=seed, index=m.index))
+    return out
+
+
 LLAMA7B_LINEARS = (("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
                    ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008))
 QWEN14B_LINEARS = (("q", 5120, 5120), ("k", 5120, 5120), ("v", 5120, 5120), ("o", 5120, 5120),

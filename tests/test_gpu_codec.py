@@ -104,3 +104,12 @@ def test_quant_every_bf16_pair(cuda_device, exp, sigs):
     W32 = _exhaustive_blocks(exp, sigs)
     Wb = synth.from_bf16_bits(nf4.bf16_bits_from_f32(W32))
     _check_quant(Wb, dq=False)
+
+
+def test_quant_stack_gate_matrix_full_size(cuda_device):
+    """A full 11008 x 4096 gate matrix of the stack (scale * Student-t), with and
+    without double quant."""
+    m = synth.stack_matrices()[4]
+    W = synth.stack_weight(m)
+    _check_quant(W, dq=False)
+    _check_quant(W, dq=True)

@@ -50,3 +50,25 @@ def test_llama_stack_sampled_layers(cuda_device):
     pick = [mats[i] for i in (0, 4, 6, 100, 223)]
     Ws = [synth.stack_weight(m) for m in pick]
     _compare(Ws, K=3, dq=False)
+
+
+def test_llama_stack_all_224_matrices(cuda_device):
+    """The whole 32-layer stack (224 matrices, 6.48 G weights) in one call: errors of
+    sampled matrices (the top- and bottom-ranked ones among them) match the oracle
+    within 1e-6; the order is the (error desc, index asc) sort of the errors and
+    keep marks the first K = 16."""
+    mats = synth.stack_matrices()
+    Ws = [synth.stack_weight(m, device="cuda") for m in mats]
+    err, order, keep = api.layer_error_rank(Ws, 16, double_quant=False)
+    torch.cuda.synchronize()
+    assert api.status() == 0
+    err = err.cpu().numpy()
+    order = order.cpu().numpy()
+    keep = keep.cpu().numpy()
+    assert np.array_equal(order, np.lexsort((np.arange(len(err)), -err)))
+    assert np.array_equal(np.flatnonzero(keep), np.sort(order[:16]))
+    for i in sorted({int(order[0]), int(order[-1]), 3, 117}):
+        ref = layer_error.layer_error(bits(Ws[i].cpu()), False)
+        assert abs(err[i] - ref) <= 1e-6 * ref, (i, err[i], ref)
+    del Ws
+    torch.cuda.empty_cache()

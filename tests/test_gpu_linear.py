@@ -102,3 +102,22 @@ def test_mlp_full_size_sampled(cuda_device, idx):
     rows = np.random.default_rng(1).choice(8192, 96, replace=False)
     rows.sort()
     run_and_compare(synth.cases_mlp()[idx], rows=rows)
+
+
+@pytest.mark.parametrize("kind,r", [("q", 16), ("gate", 32), ("down", 64), ("q", 128)])
+def test_14b_shapes_full_size_sampled(cuda_device, kind, r):
+    """14B-shaped linears (hidden 5120, intermediate 13824), double quant, X of
+    16384 tokens, the sweep's ranks: Y and dX on sampled rows, dL1 / dL2 over all
+    rows."""
+    case = synth.cases_14b(r, kinds=(kind,))[0]
+    rows = np.random.default_rng(2).choice(case.M, 48, replace=False)
+    rows.sort()
+    run_and_compare(case, rows=rows)
+
+
+def test_14b_protected_layer_full_size_sampled(cuda_device):
+    """A layer the allocation keeps in bf16 (no dequantization) at the 14B gate shape."""
+    case = synth.cases_14b(16, kinds=("gate",))[0]
+    rows = np.random.default_rng(3).choice(case.M, 32, replace=False)
+    rows.sort()
+    run_and_compare(case, protected=True, rows=rows)
