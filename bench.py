@@ -180,9 +180,10 @@ class ClockSampler:
                 "reasons": sorted(seen), "samples": len(rows)}
 
 
-def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3):
-    """Quantize-all and error/rank over the 224-matrix Llama-7B-shaped stack."""
-    mats = synth.stack_matrices()
+def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int = 32):
+    """Quantize-all and error/rank over the Llama-7B-shaped stack (32 layers, 224
+    matrices by default; fewer layers for small profiler captures)."""
+    mats = synth.stack_matrices(n_layers=layers)
     Ws = [synth.stack_weight(m, device=str(dev)) for m in mats]
     numel = sum(w.numel() for w in Ws)
     nb = numel // 64
@@ -213,13 +214,14 @@ def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3):
     qm, em = min(q_ms), min(e_ms)
     del Ws, outs
     torch.cuda.empty_cache()
-    return {"workload": "llama7b stack: 224 matrices (32 x q,k,v,o 4096^2, gate/up 11008x4096, down 4096x11008), "
-                        "6.48 G weights, per-matrix scale * Student-t(nu), NF4 blocksize 64, no double quant",
+    return {"workload": f"llama7b stack: {len(mats)} matrices ({layers} x q,k,v,o 4096^2, gate/up 11008x4096, "
+                        f"down 4096x11008), {numel / 1e9:.2f} G weights, per-matrix scale * Student-t(nu), "
+                        "NF4 blocksize 64, no double quant",
             "quantize_all": {"ms": qm, "bytes": q_bytes, "GB/s": q_bytes / (qm * 1e-3) / 1e9,
                              "frac_hbm": q_bytes / (qm * 1e-3) / 1e9 / peaks["hbm"], "launches": len(mats)},
             "error_rank_all": {"ms": em, "bytes": e_bytes, "GB/s": e_bytes / (em * 1e-3) / 1e9,
                                "frac_hbm": e_bytes / (em * 1e-3) / 1e9 / peaks["hbm"], "launches": 1},
-            "timing": f"best of {reps} (inputs 12.95 GB, far above L2)"}
+            "timing": f"best of {reps} (inputs {numel * 2 / 1e9:.2f} GB)"}
 
 
 def gpu_main(args):
@@ -428,7 +430,7 @@ def gpu_main(args):
     # all of them, as the allocation pass does.
     hbm = None
     if rank == 0 and world == 1 and not args.no_hbm_legs:
-        hbm = hbm_legs(api, synth, torch, dev, stream, peaks)
+        hbm = hbm_legs(api, synth, torch, dev, stream, peaks, layers=args.hbm_layers)
 
     # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
@@ -466,6 +468,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-hbm-legs", action="store_true", help="skip the full-stack quantizer / error-pass legs")
+    ap.add_argument("--hbm-layers", type=int, default=32, help="decoder layers of the stack for those legs")
     ap.add_argument("--eager", action="store_true", help="time eager API calls instead of CUDA-graph replays")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "gemm.cuh"
 #include "internal.cuh"
@@ -75,7 +76,7 @@ FwdLayout fwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
 }
 
 struct BwdLayout {
-  size_t scales, l1s, t, u, su, part, counters, total;
+  size_t scales, l1s, t, u, su, part, part2, counters, total;
 };
 
 BwdLayout bwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
@@ -92,6 +93,7 @@ BwdLayout bwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
   size_t part = std::max({size_t(a.splits) * M * r, size_t(b.splits) * M * r, size_t(c.splits) * out * r,
                           size_t(d.splits) * in * r}) * 4;
   L.part = off;   off += up256(part);
+  L.part2 = off;  off += up256(size_t(c.splits) * out * r * 4);   // dL2 partials on the side stream
   L.total = off;
   return L;
 }
@@ -286,6 +288,53 @@ qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
   return st;
 }
 
+
+// ---- side stream for independent small kernels (fork / join with events)
+//
+// One non-blocking stream and two events per device, created on first use. A
+// call records `fork` on the caller's stream, makes the side stream wait on it,
+// launches independent work there, records `join` on the side stream and makes
+// the caller's stream wait on it before the dependent work. Works inside CUDA
+// graph capture (the side stream joins the capture through the event). Calls
+// from several host threads serialize on the mutex while they enqueue.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxSideDevices = 64;
+std::mutex g_side_mu;
+SideStream g_side[kMaxSideDevices];
+
+// Returns nullptr (run everything on the caller's stream) when no side stream
+// can be made.
+SideStream* side_stream() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return nullptr;
+  SideStream& ss = g_side[dev];
+  if (!ss.stream) {
+    if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      ss = SideStream();
+      return nullptr;
+    }
+  }
+  return &ss;
+}
+
+qlora_status fork_to(SideStream* ss, cudaStream_t s) {
+  if (cudaEventRecord(ss->fork, s) != cudaSuccess || cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
+
+qlora_status join_from(SideStream* ss, cudaStream_t s) {
+  if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess || cudaStreamWaitEvent(s, ss->join, 0) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -401,13 +450,22 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t 
   float* part = reinterpret_cast<float*>(ws + L.part);
   const int64_t h = w->in, o_ = w->out;
   int* counters = reinterpret_cast<int*>(ws + L.counters);
-  // T = X L1 : A = X (K-major), B = L1 as [h x r] (MN-major for B)
+  // T = X L1 : A = X (K-major), B = L1 as [h x r] (MN-major for B); the scale
+  // expansion and s.L2^T are independent of it and run beside it
   Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* ss = side_stream();
+  cudaStream_t aux = s;
+  if (ss) {
+    QLB_TRY(fork_to(ss, s));
+    aux = ss->stream;
+  }
   if (!w->is_bf16)
     QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
-                                 scales_t, s));
-  QLB_TRY(launch_scale_lora(L2, r, o_, scale, /*transpose=*/true, l2t, s));
+                                 scales_t, aux));
+  QLB_TRY(launch_scale_lora(L2, r, o_, scale, /*transpose=*/true, l2t, aux));
   QLB_TRY(run_thin(tt, part, counters, T, 0, 1.f, status, s));
+  if (ss) QLB_TRY(join_from(ss, s));
   if (!w->is_bf16 && use_pair_kernel()) return run_pair(false, w, X, M, T, l2t, r, scales_t, Y, status, s);
   return run_main(false, w, X, M, T, l2t, r, scales_t, Y, status, s);
 }
@@ -442,28 +500,37 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const ui
     QLB_TRY(run_thin(tt, part, counters, Tw, 0, 1.f, status, s));
     T = Tw;
   }
-  // U = dY L2^T : A = dY (K-major, K = out), B = L2 [r x out] (K-major); with
-  // the pair engine also s.U, the dX LoRA step's A
+  // dL2 = s (dY^T T)^T (A = dY^T MN-major, B = T MN-major, K = M, written
+  // transposed) and the scale expansion run on the side stream, beside
+  // U = dY L2^T (A = dY K-major, B = L2 [r x out] K-major; with the pair engine
+  // also s.U, the dX LoRA step's A) and dL1 = s X^T U on the caller's stream. The
+  // side products use their own partial buffer and counter range.
   const bool pair = !w->is_bf16 && use_pair_kernel();
   uint16_t* sU = reinterpret_cast<uint16_t*>(ws + L.su);
+  float* part2 = reinterpret_cast<float*>(ws + L.part2);
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* ss = ((M + 127) / 128 <= kMaxCounterTiles / 2 && (o_ + 127) / 128 <= kMaxCounterTiles / 2)
+                       ? side_stream() : nullptr;
+  cudaStream_t aux = s;
+  int* counters2 = counters;
+  if (ss) {
+    QLB_TRY(fork_to(ss, s));
+    aux = ss->stream;
+    counters2 = counters + kMaxCounterTiles / 2;
+  }
+  Thin t2{GemmKind::ThinMM, dY, o_, M, T, r, M, o_, mk, r};
+  QLB_TRY(run_thin(t2, ss ? part2 : part, counters2, dL2, 2, scale, status, aux));
+  if (dX && !w->is_bf16)
+    QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
+                                 scales_t, aux));
   Thin tu{GemmKind::ThinKK, dY, o_, M, L2, o_, r, M, o_ / 64, r};
   if (pair && dX) QLB_TRY(run_thin(tu, part, counters, U, 3, scale, status, s, sU));
   else QLB_TRY(run_thin(tu, part, counters, U, 0, 1.f, status, s));
-  // dL2 = s (dY^T T)^T : A = dY^T (MN-major), B = T (MN-major); K = M; written transposed
-  Thin t2{GemmKind::ThinMM, dY, o_, M, T, r, M, o_, mk, r};
-  QLB_TRY(run_thin(t2, part, counters, dL2, 2, scale, status, s));
-  // dL1 = s X^T U (in x r): A = X^T (MN-major), B = U (MN-major); K = M
   Thin t1{GemmKind::ThinMM, X, h, M, U, r, M, h, mk, r};
   QLB_TRY(run_thin(t1, part, counters, dL1, 1, scale, status, s));
-  if (dX && pair) {
-    QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
-                                 scales_t, s));
-    return run_pair(true, w, dY, M, sU, L1, r, scales_t, dX, status, s);
-  }
+  if (ss) QLB_TRY(join_from(ss, s));
+  if (dX && pair) return run_pair(true, w, dY, M, sU, L1, r, scales_t, dX, status, s);
   if (dX) {
-    if (!w->is_bf16)
-      QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
-                                   scales_t, s));
     QLB_TRY(launch_scale_lora(L1, h, r, scale, /*transpose=*/false, l1s, s));
     QLB_TRY(run_main(true, w, dY, M, U, l1s, r, scales_t, dX, status, s));
   }
