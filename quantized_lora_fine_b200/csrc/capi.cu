@@ -185,6 +185,23 @@ void record_prof(cudaEvent_t e, cudaStream_t s) {
     cudaEventRecord(e, s);
 }
 
+}  // namespace
+
+namespace qlb {
+// Programmatic dependent launch is on unless QLORA_B200_PDL=0 (kept switchable for
+// measurement: the results are the same either way).
+bool pdl_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("QLORA_B200_PDL");
+    v = (e && std::strcmp(e, "0") == 0) ? 0 : 1;
+  }
+  return v == 1;
+}
+}  // namespace qlb
+
+namespace {
+
 // The NF4 GEMMs run on the CTA-pair kernel unless QLORA_B200_GEMM=1cta selects
 // the single-CTA kernel (both compute the same values; kept side by side for
 // measurement).

@@ -6,6 +6,7 @@
 
 #include "internal.cuh"
 #include "nf4_device.cuh"
+#include "ptx.cuh"
 
 namespace qlb {
 
@@ -144,6 +145,8 @@ __global__ void __launch_bounds__(256) nf4_quantize_bf16_kernel(const uint16_t* 
   __shared__ __align__(16) float2 s_tbl[33];
   __shared__ float s_amax[256];
   __shared__ float s_red[8];
+  pdl_wait();
+  pdl_launch();
   const int tid = threadIdx.x, lane = tid & 31;
   if (tid < 33) s_tbl[tid] = make_float2(__uint_as_float(kNF4CoarseQ[2 * tid]), __uint_as_float(kNF4CoarseQ[2 * tid + 1]));
   const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(s_tbl));
@@ -253,8 +256,9 @@ qlora_status launch_quantize(const void* W, int w_dtype, int64_t numel, bool dq,
   if (groups <= 0) return QLORA_OK;
   dim3 grid(static_cast<unsigned>(groups));
   if (w_dtype == QLORA_DTYPE_BF16) {
-    if (dq) nf4_quantize_bf16_kernel<true><<<grid, 256, 0, s>>>((const uint16_t*)W, numel, codes, absmax, absmax_q, absmax2, status);
-    else nf4_quantize_bf16_kernel<false><<<grid, 256, 0, s>>>((const uint16_t*)W, numel, codes, absmax, absmax_q, absmax2, status);
+    const uint16_t* Wb = static_cast<const uint16_t*>(W);
+    if (dq) launch_pdl(nf4_quantize_bf16_kernel<true>, grid, dim3(256), 0, s, Wb, numel, codes, absmax, absmax_q, absmax2, status);
+    else launch_pdl(nf4_quantize_bf16_kernel<false>, grid, dim3(256), 0, s, Wb, numel, codes, absmax, absmax_q, absmax2, status);
   } else {
     if (dq) nf4_quantize_f32_kernel<true><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
     else nf4_quantize_f32_kernel<false><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
@@ -318,6 +322,8 @@ __global__ void expand_scales_kernel(const float* __restrict__ absmax, const uin
                                      float* __restrict__ scales_t) {
   // scales_t[kb][o] = scale of block (o, kb)
   __shared__ float tile[32][33];
+  pdl_wait();
+  pdl_launch();
   const int64_t o0 = int64_t(blockIdx.x) * 32, k0 = int64_t(blockIdx.y) * 32;
   const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
   for (int j = ty; j < 32; j += 8) {
@@ -338,7 +344,7 @@ qlora_status launch_expand_scales(const uint8_t*, const float* absmax, const uin
                                   cudaStream_t s) {
   const int64_t nbr = in / kBlock;
   dim3 grid(unsigned((out + 31) / 32), unsigned((nbr + 31) / 32));
-  expand_scales_kernel<<<grid, dim3(32, 8), 0, s>>>(absmax, absmax_q, absmax2, dq ? 1 : 0, out, nbr, scales_t);
+  launch_pdl(expand_scales_kernel, grid, dim3(32, 8), 0, s, absmax, absmax_q, absmax2, dq ? 1 : 0, out, nbr, scales_t);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -346,6 +352,8 @@ qlora_status launch_expand_scales(const uint8_t*, const float* absmax, const uin
 
 __global__ void scale_lora_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t cols, float scale,
                                   int transpose, uint16_t* __restrict__ dst) {
+  pdl_wait();
+  pdl_launch();
   const int64_t n = rows * cols;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
     // non-transposed: dst[i] = s*src[i]; transposed: src is rows x cols, dst is cols x rows
@@ -364,7 +372,7 @@ qlora_status launch_scale_lora(const uint16_t* src, int64_t rows, int64_t cols, 
                                uint16_t* dst, cudaStream_t s) {
   const int64_t n = rows * cols;
   const int64_t blocks = std::min<int64_t>((n + 255) / 256, 4096);
-  scale_lora_kernel<<<unsigned(blocks), 256, 0, s>>>(src, rows, cols, scale, transpose ? 1 : 0, dst);
+  launch_pdl(scale_lora_kernel, dim3(unsigned(blocks)), dim3(256), 0, s, src, rows, cols, scale, transpose ? 1 : 0, dst);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

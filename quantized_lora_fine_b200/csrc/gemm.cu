@@ -165,6 +165,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_launch();
 
   const int num_tiles = p.tiles_m * p.tiles_n * p.splits;
 
@@ -556,6 +558,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_launch();
 
   const int num_tiles = p.tiles_m * p.tiles_n;   // tiles of 256 x 256
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
@@ -793,7 +797,9 @@ static qlora_status launch_cfg(const GemmOperands& o, GemmParams p, int ctas_per
   p.bn = C::BN;
   const int num_tiles = p.tiles_m * p.tiles_n * p.splits;
   const int grid = std::max(1, std::min(num_tiles, num_sms() * ctas_per_sm));
-  tc_gemm_kernel<C><<<grid, C::kThreads, C::kSmem, s>>>(o.A, o.B, o.codes, o.scales, o.Ax, o.Bx, p);
+  if (launch_pdl(tc_gemm_kernel<C>, dim3(grid), dim3(C::kThreads), C::kSmem, s, o.A, o.B, o.codes, o.scales, o.Ax,
+                 o.Bx, p) != cudaSuccess)
+    return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -828,17 +834,19 @@ static qlora_status launch_pair_cfg(const GemmOperands& o, GemmParams p, cudaStr
   const int num_tiles = p.tiles_m * p.tiles_n;
   const int pairs = std::max(1, std::min(num_tiles, max_pairs));
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   if (cudaLaunchKernelEx(&cfg, tc_gemm_nf4_pair_kernel<C>, o.A, o.Ax, o.Bx, p) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;

@@ -18,6 +18,27 @@ constexpr size_t kCounterBytes = 65536;
 constexpr size_t kReservedBytes = kStatusBytes + kCounterBytes;
 constexpr int64_t kMaxCounterTiles = int64_t(kCounterBytes / 4);
 
+// Launch with programmatic dependent launch allowed (unless QLORA_B200_PDL=0):
+// the kernel may begin while the previous kernel in the stream finishes, so every
+// kernel launched this way calls pdl_wait() before it touches global memory.
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 __device__ __forceinline__ void set_status(int* st, int code) {
   if (st) atomicCAS(st, 0, code);
 }

@@ -16,6 +16,7 @@
 
 #include "internal.cuh"
 #include "nf4_device.cuh"
+#include "ptx.cuh"
 
 namespace qlb {
 
@@ -101,6 +102,8 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
   __shared__ float s_red[8];
   __shared__ double s_sum[2][8];
   __shared__ int s_flag;
+  pdl_wait();
+  pdl_launch();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid < 33) s_tbl[tid] = make_float2(__uint_as_float(kNF4CoarseD[2 * tid]), __uint_as_float(kNF4CoarseD[2 * tid + 1]));
   const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(s_tbl));
@@ -299,8 +302,8 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
   if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
   double2* partial = reinterpret_cast<double2*>(static_cast<char*>(ws) + kReservedBytes);
   int* counters = reinterpret_cast<int*>(static_cast<char*>(ws) + kStatusBytes);   // 1 + n_layers, zero
-  if (dq) layer_error_chunk_kernel<true><<<unsigned(c), 256, 0, s>>>(tab, partial, status, counters, err, K, order, keep);
-  else layer_error_chunk_kernel<false><<<unsigned(c), 256, 0, s>>>(tab, partial, status, counters, err, K, order, keep);
+  if (dq) launch_pdl(layer_error_chunk_kernel<true>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status, counters, err, K, order, keep);
+  else launch_pdl(layer_error_chunk_kernel<false>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status, counters, err, K, order, keep);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

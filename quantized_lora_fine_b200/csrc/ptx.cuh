@@ -104,6 +104,12 @@ __device__ __forceinline__ void st_async_signal(uint32_t dst_cluster, uint32_t b
                : "memory");
 }
 
+// Programmatic dependent launch: wait until the previous kernel of the stream has
+// completed and its memory is visible (returns at once without one), and let the
+// next kernel of the stream start launching (its CTAs then wait in pdl_wait()).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
