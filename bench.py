@@ -194,7 +194,8 @@ def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int =
     for w in Ws:   # outputs allocated once, outside the timed region
         outs.append((torch.empty(w.numel() // 2, dtype=torch.uint8, device=dev),
                      torch.empty(w.numel() // 64, dtype=torch.float32, device=dev)))
-    q_ms, e_ms = [], []
+    q_ms, e_ms, f_ms = [], [], []
+    fused_outs = [api.NF4Weight(w.shape[0], w.shape[1], False, codes=c, absmax=a) for w, (c, a) in zip(Ws, outs)]
     for i in range(reps + 1):
         torch.cuda.synchronize()
         e0.record(stream)
@@ -210,8 +211,14 @@ def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int =
         e1.synchronize()
         if i:
             e_ms.append(e0.elapsed_time(e1))
+        e0.record(stream)
+        api.quantize_error_rank(Ws, 16, double_quant=False, outs=fused_outs)
+        e1.record(stream)
+        e1.synchronize()
+        if i:
+            f_ms.append(e0.elapsed_time(e1))
     assert api.status() == 0, "device status set in the codec legs"
-    qm, em = min(q_ms), min(e_ms)
+    qm, em, fm = min(q_ms), min(e_ms), min(f_ms)
     del Ws, outs
     torch.cuda.empty_cache()
     return {"workload": f"llama7b stack: {len(mats)} matrices ({layers} x q,k,v,o 4096^2, gate/up 11008x4096, "
@@ -221,6 +228,9 @@ def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int =
                              "frac_hbm": q_bytes / (qm * 1e-3) / 1e9 / peaks["hbm"], "launches": len(mats)},
             "error_rank_all": {"ms": em, "bytes": e_bytes, "GB/s": e_bytes / (em * 1e-3) / 1e9,
                                "frac_hbm": e_bytes / (em * 1e-3) / 1e9 / peaks["hbm"], "launches": 1},
+            "quantize_error_rank_all": {"ms": fm, "bytes": q_bytes, "GB/s": q_bytes / (fm * 1e-3) / 1e9,
+                                        "frac_hbm": q_bytes / (fm * 1e-3) / 1e9 / peaks["hbm"], "launches": 1,
+                                        "note": "one pass: codes, absmax, errors, ranks"},
             "timing": f"best of {reps} (inputs {numel * 2 / 1e9:.2f} GB)"}
 
 
@@ -256,8 +266,8 @@ def gpu_main(args):
     stream = torch.cuda.current_stream()
 
     def run_step(W, X, dY, L1, L2):
-        w = api.quantize(W, double_quant=True)
-        api.layer_error_rank([W], 0, double_quant=True)
+        # quantize + double quant + error + rank in one pass over W
+        _, _, _, (w,) = api.quantize_error_rank([W], 0, double_quant=True)
         Y, T = api.linear_fwd(w, X, L1, L2, s)
         dX, dL1, dL2 = api.linear_bwd(w, X, dY, L1, L2, s, T=T)
         if world > 1:
@@ -284,10 +294,7 @@ def gpu_main(args):
     state = {}
 
     def leg_quant():
-        state["w"] = api.quantize(g["W"], double_quant=True)
-
-    def leg_err():
-        api.layer_error_rank([g["W"]], 0, double_quant=True)
+        _, _, _, (state["w"],) = api.quantize_error_rank([g["W"]], 0, double_quant=True)
 
     def leg_fwd():
         state["Y"], state["T"] = api.linear_fwd(state["w"], g["X"], g["L1"], g["L2"], s)
@@ -300,13 +307,13 @@ def gpu_main(args):
             dist.all_reduce(state["dL2"])
 
     def whole_step():
-        leg_quant(); leg_err(); leg_fwd(); leg_bwd()
+        leg_quant(); leg_fwd(); leg_bwd()
 
     use_graphs = not args.eager and world == 1
     graphs = {}
     if use_graphs:
         try:
-            for name, fn in (("step", whole_step), ("quantize", leg_quant), ("error_rank", leg_err),
+            for name, fn in (("step", whole_step), ("quantize_error_rank", leg_quant),
                              ("fwd", leg_fwd), ("bwd", leg_bwd)):
                 gr = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(gr):
@@ -323,7 +330,7 @@ def gpu_main(args):
         else:
             fn()
 
-    step_ms, legs = [], {"quantize": [], "error_rank": [], "fwd": [], "bwd": [], "fwd_gemm": [], "dx_gemm": []}
+    step_ms, legs = [], {"quantize_error_rank": [], "fwd": [], "bwd": [], "fwd_gemm": [], "dx_gemm": []}
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -340,7 +347,7 @@ def gpu_main(args):
         legs["fwd_gemm"].append(prof[0].elapsed_time(prof[1]))
         legs["dx_gemm"].append(prof[2].elapsed_time(prof[3]))
     clk = clocks.stop()
-    for name, fn in (("quantize", leg_quant), ("error_rank", leg_err), ("fwd", leg_fwd), ("bwd", leg_bwd)):
+    for name, fn in (("quantize_error_rank", leg_quant), ("fwd", leg_fwd), ("bwd", leg_bwd)):
         for i in range(max(5, min(args.steps, 50))):
             flush.zero_()
             ev[2].record(stream)
@@ -372,18 +379,16 @@ def gpu_main(args):
     dom = (f"qlora_fwd_gemm ({engine} fwd)", fwd_tf, med["fwd_gemm"]) if med["fwd_gemm"] >= med["dx_gemm"] \
         else (f"qlora_bwd_dx_gemm ({engine} dX)", dx_tf, med["dx_gemm"])
     numel = h * o
-    quant_bytes = numel * 2 + numel // 2 + numel // 64 + 4 * (numel // 64 // 256)
-    err_bytes = numel * 2
+    qer_bytes = numel * 2 + numel // 2 + numel // 64 + 4 * (numel // 64 // 256)   # bf16 in; codes, E4M3, fp32 out
     roofline = {"kernel": dom[0], "bound": "tensor", "achieved": dom[1], "peak": peaks["bf16_sus"],
                 "unit": "TFLOP/s", "frac": dom[1] / peaks["bf16_sus"],
                 "peak_kind": f"bf16 sustained ({peaks['source']})",
                 "frac_of_burst": dom[1] / peaks["bf16"], "traffic": None,
                 "per_launch_flops": fl_fwd_gemm if dom[0].startswith("qlora_fwd") else fl_dx_gemm}
     legs_out = {
-        "quantize": {"ms": med["quantize"], "GB/s": quant_bytes / (med["quantize"] * 1e-3) / 1e9,
-                     "frac_hbm": quant_bytes / (med["quantize"] * 1e-3) / 1e9 / peaks["hbm"]},
-        "error_rank": {"ms": med["error_rank"], "GB/s": err_bytes / (med["error_rank"] * 1e-3) / 1e9,
-                       "frac_hbm": err_bytes / (med["error_rank"] * 1e-3) / 1e9 / peaks["hbm"]},
+        "quantize_error_rank": {"ms": med["quantize_error_rank"],
+                                "GB/s": qer_bytes / (med["quantize_error_rank"] * 1e-3) / 1e9,
+                                "frac_hbm": qer_bytes / (med["quantize_error_rank"] * 1e-3) / 1e9 / peaks["hbm"]},
         "fwd": {"ms": med["fwd"]}, "bwd": {"ms": med["bwd"]},
         "fwd_gemm": {"ms": med["fwd_gemm"], "TFLOP/s": fwd_tf}, "dx_gemm": {"ms": med["dx_gemm"], "TFLOP/s": dx_tf},
     }
@@ -439,7 +444,7 @@ def gpu_main(args):
         cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": desc + f"; repeated for {secs:.1f} s", "seconds": secs}
 
-    launches_per_step = 1 + 1 + 4 + 5  # quantize; error/rank; fwd (scales, s.L2^T, T, GEMM); bwd (U + s.U, dL2, dL1, scales, dX GEMM)
+    launches_per_step = 1 + 4 + 5  # quantize+error/rank; fwd (scales, s.L2^T, T, GEMM); bwd (U + s.U, dL2, dL1, scales, dX GEMM)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args, world),

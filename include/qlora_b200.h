@@ -206,6 +206,29 @@ qlora_status nf4_layer_error_rank(int32_t n_layers, const uint16_t* const* W_ptr
                                   double* err, int32_t* order, uint8_t* keep,
                                   void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
+/* The allocation pass fused with the quantization it measures ("AQLoRA: A
+ * Zero-Search Recipe for Fast Quantized LoRA Fine-Tuning", section 3.1-3.2: one
+ * pass quantizes every linear layer to NF4 and scores its reconstruction error;
+ * "QLoRA: How to fine-tune large language models with less memory", sections
+ * "1. NormalFloat" and "2. Double quantization", for the storage). One read of
+ * every matrix gives err / order / keep exactly as nf4_layer_error_rank and the
+ * NF4 storage exactly as nf4_quantize, so the layers that are not kept need no
+ * second pass.
+ *   codes     HOST array of n_layers DEVICE pointers, uint8 [numel / 2] each,
+ *             16-byte aligned
+ *   absmax    HOST array of DEVICE pointers, fp32 [numel / 64]: required without
+ *             double quant; with it the array, or any entry, may be NULL
+ *   absmax_q, absmax2   HOST arrays of DEVICE pointers, E4M3 [numel / 64] and fp32
+ *             [ceil(numel / 16384)]: required with double quant, else ignored
+ * Other arguments, the workspace (nf4_layer_error_rank_workspace_size) and the
+ * errors as for nf4_layer_error_rank; 1 <= n_layers <= 512 (the per-layer
+ * pointers travel as one kernel parameter). */
+qlora_status nf4_quantize_error_rank(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
+                                     int32_t w_dtype, nf4_qconfig q, int32_t K, uint8_t* const* codes,
+                                     float* const* absmax, uint8_t* const* absmax_q, float* const* absmax2,
+                                     double* err, int32_t* order, uint8_t* keep, void* workspace,
+                                     size_t workspace_bytes, qlora_stream_t stream);
+
 /* Allocation-free variant of nf4_layer_error_rank (the paper has no
  * counterpart; this is a convenience of the library).
  *

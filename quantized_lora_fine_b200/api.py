@@ -185,6 +185,41 @@ def layer_error_rank(Ws: Sequence[torch.Tensor], K: int, double_quant: bool = Fa
     return err, order, keep
 
 
+def quantize_error_rank(Ws: Sequence[torch.Tensor], K: int, double_quant: bool = False, keep_absmax: bool = False,
+                        outs: Optional[Sequence[NF4Weight]] = None):
+    """The allocation pass fused with the quantization: one read of every matrix
+    gives (err, order, keep) as layer_error_rank and every layer's NF4Weight as
+    quantize. `outs` may supply preallocated weights (same shapes and settings)."""
+    lib = _lib.load()
+    L = len(Ws)
+    for i, W in enumerate(Ws):
+        _need(W, torch.bfloat16, f"W[{i}]")
+    dev = Ws[0].device
+    if outs is None:
+        outs = []
+        for W in Ws:
+            n = W.numel()
+            nb = n // 64
+            outs.append(NF4Weight(
+                W.shape[0], W.shape[1], double_quant,
+                codes=torch.empty(n // 2, dtype=torch.uint8, device=dev),
+                absmax=torch.empty(nb, dtype=torch.float32, device=dev) if (not double_quant or keep_absmax) else None,
+                absmax_q=torch.empty(nb, dtype=torch.uint8, device=dev) if double_quant else None,
+                absmax2=torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev) if double_quant else None))
+    ptrs = (ctypes.c_void_p * L)(*[W.data_ptr() for W in Ws])
+    numel = (ctypes.c_int64 * L)(*[W.numel() for W in Ws])
+    arr = lambda name: (ctypes.c_void_p * L)(*[_ptr(getattr(w, name)) for w in outs])
+    err = torch.empty(L, dtype=torch.float64, device=dev)
+    order = torch.empty(L, dtype=torch.int32, device=dev)
+    keep = torch.empty(L, dtype=torch.uint8, device=dev)
+    ws = Workspace.get(lib.nf4_layer_error_rank_workspace_size(L, numel), dev)
+    check(lib.nf4_quantize_error_rank(L, ptrs, numel, DTYPE_BF16, NF4QConfig(64, 1 if double_quant else 0, 256), K,
+                                      arr("codes"), arr("absmax"), arr("absmax_q"), arr("absmax2"),
+                                      _ptr(err), _ptr(order), _ptr(keep), _ptr(ws), ws.numel(), _stream()),
+          "nf4_quantize_error_rank")
+    return err, order, keep, list(outs)
+
+
 def status() -> int:
     """Device status word of this device's shared workspace (synchronizes)."""
     dev = torch.device("cuda", torch.cuda.current_device())

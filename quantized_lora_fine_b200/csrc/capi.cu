@@ -577,6 +577,31 @@ qlora_status nf4_layer_error_rank(int32_t n_layers, const uint16_t* const* W_ptr
                                  workspace_bytes, static_cast<int*>(workspace), S(stream));
 }
 
+qlora_status nf4_quantize_error_rank(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
+                                    int32_t w_dtype, nf4_qconfig q, int32_t K, uint8_t* const* codes,
+                                    float* const* absmax, uint8_t* const* absmax_q, float* const* absmax2,
+                                    double* err, int32_t* order, uint8_t* keep, void* workspace,
+                                    size_t workspace_bytes, qlora_stream_t stream) {
+  if (w_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_DTYPE;
+  if (!qconfig_ok(q)) return QLORA_ERR_UNSUPPORTED;
+  if (n_layers < 1 || n_layers > 512 || K < 0 || K > n_layers) return QLORA_ERR_SHAPE;
+  if (!W_ptrs || !numel || !err || !order || !keep || !codes) return QLORA_ERR_NULL;
+  const bool dq = q.double_quant != 0;
+  if (dq && (!absmax_q || !absmax2)) return QLORA_ERR_NULL;
+  if (!dq && !absmax) return QLORA_ERR_NULL;
+  for (int i = 0; i < n_layers; ++i) {
+    if (!W_ptrs[i] || !codes[i]) return QLORA_ERR_NULL;
+    if (dq && (!absmax_q[i] || !absmax2[i])) return QLORA_ERR_NULL;
+    if (!dq && !absmax[i]) return QLORA_ERR_NULL;
+    if (numel[i] <= 0 || numel[i] % 64) return QLORA_ERR_SHAPE;
+    if (!aligned16(W_ptrs[i]) || !aligned16(codes[i])) return QLORA_ERR_ALIGN;
+  }
+  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  QLB_TRY(check_device());
+  return launch_quantize_error_rank(n_layers, W_ptrs, numel, dq, K, codes, absmax, absmax_q, absmax2, err, order,
+                                    keep, workspace, workspace_bytes, static_cast<int*>(workspace), S(stream));
+}
+
 qlora_status nf4_layer_error_rank_noalloc(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
                                           int32_t w_dtype, nf4_qconfig q, int32_t K, double* err, int32_t* order,
                                           uint8_t* keep, qlora_stream_t stream) {

@@ -64,6 +64,10 @@ qlora_status launch_scale_lora(const uint16_t* src, int64_t rows, int64_t cols, 
                                uint16_t* dst, cudaStream_t s);
 // ---- layer_error.cu
 size_t layer_error_ws_bytes(int n_layers, const int64_t* numel);
+qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
+                                       int K, uint8_t* const* codes, float* const* absmax, uint8_t* const* absmax_q,
+                                       float* const* absmax2, double* err, int32_t* order, uint8_t* keep, void* ws,
+                                       size_t ws_bytes, int* status, cudaStream_t s);
 qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
                                      int K, double* err, int32_t* order, uint8_t* keep, void* ws, size_t ws_bytes,
                                      int* status, cudaStream_t s);

@@ -23,19 +23,41 @@ namespace qlb {
 constexpr int kMaxLayers = 1024;
 
 struct LayerTable {
+  static constexpr bool kWrite = false;
   const uint16_t* ptr[kMaxLayers];
   int64_t numel[kMaxLayers];
   int32_t first_chunk[kMaxLayers + 1];
   int32_t n_layers;
 };
 
+// The fused pass also writes every layer's NF4 storage; its table (a by-value
+// kernel parameter, at most 32 KB) holds fewer layers.
+constexpr int kMaxFusedLayers = 512;
+struct FusedTable {
+  static constexpr bool kWrite = true;
+  const uint16_t* ptr[kMaxFusedLayers];
+  int64_t numel[kMaxFusedLayers];
+  uint8_t* codes[kMaxFusedLayers];
+  float* absmax[kMaxFusedLayers];       // may be null with double quant
+  uint8_t* absmax_q[kMaxFusedLayers];   // double quant only
+  float* absmax2[kMaxFusedLayers];      // double quant only
+  int32_t first_chunk[kMaxFusedLayers + 1];
+  int32_t n_layers;
+};
+static_assert(sizeof(FusedTable) <= 32000, "kernel parameter limit");
+
 // Error contribution of 16 bf16 weights (8 packed pairs) of one block: codes
 // from the exact absmax a (same arithmetic as the quantizer), reconstruction
 // w_hat = bf16(fp32(code * ahat)) with ahat = a, or the double-quantized scale.
 // Squares are summed per pair lane in fp32 (8 terms) before the fp64 total.
-template <bool kTiny>
-__device__ __forceinline__ void err16_core(const uint32_t (&u)[8], float a, float ahat, uint32_t tbl, double& sd,
-                                           double& sw) {
+// With kCodes, also the 16 codes in storage order (byte k = idx[2k] << 4 |
+// idx[2k + 1]): idx = base + sat(n 2^100 + T) from the quantizer's {T, base}
+// table (tbl_base), the four indices of a 16-bit half accumulated as fp32
+// nibble weights.
+template <bool kTiny, bool kCodes>
+__device__ __forceinline__ void err16_core(const uint32_t (&u)[8], float a, float ahat, uint32_t tbl,
+                                           uint32_t tbl_base, double& sd, double& sw, uint2& codes) {
+  float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
   // tiny blocks: the division operands are rescaled by 2^64 (exact) so 1/a stays normal
   const float as = kTiny ? a * 0x1p64f : a;
   const uint64_t r2 = f2_splat(__frcp_rn(as)), na2 = f2_splat(-as), ah2 = f2_splat(ahat);
@@ -54,6 +76,17 @@ __device__ __forceinline__ void err16_core(const uint32_t (&u)[8], float a, floa
     const float s1 = sat_fma(__fmaf_rn(e1.x, 2.f, e1.y), -0x1p99f, f2_hi(n2));
     const float c0 = __fmaf_rn(s0, e0.y, e0.x);   // code value (exact)
     const float c1 = __fmaf_rn(s1, e1.y, e1.x);
+    if constexpr (kCodes) {
+      // the index needs the midpoint test of the quantizer's table: in a cell
+      // without a midpoint s above may be 1 (harmless for the value, not for idx)
+      const float2 t0 = lds_f2(coarse_addr_bits<8>(uint32_t(cells), tbl_base));
+      const float2 t1 = lds_f2(coarse_addr_bits<8>(uint32_t(cells >> 32), tbl_base));
+      const float i0 = t0.y + sat_fma(f2_lo(q), 0x1p100f, t0.x);
+      const float i1 = t1.y + sat_fma(f2_hi(q), 0x1p100f, t1.x);
+      const int h = i >> 2, j = i & 3;
+      acc[h][j >> 1] = __fmaf_rn(i0, (j & 1) ? 4096.f : 16.f, acc[h][j >> 1]);
+      acc[h][j >> 1] = __fmaf_rn(i1, (j & 1) ? 256.f : 1.f, acc[h][j >> 1]);
+    }
     const uint64_t p = f2_mul((uint64_t(__float_as_uint(c1)) << 32) | __float_as_uint(c0), ah2);
     const uint64_t wh = f2_from_bf16x2(pack_bf16x2(f2_lo(p), f2_hi(p)));
     const uint64_t d = f2_sub(w, wh);
@@ -62,13 +95,21 @@ __device__ __forceinline__ void err16_core(const uint32_t (&u)[8], float a, floa
   }
   sd += double(f2_lo(sd2)) + double(f2_hi(sd2));
   sw += double(f2_lo(sw2)) + double(f2_hi(sw2));
+  if constexpr (kCodes) {
+    codes.x = prmt(nibbles_from_f32(acc[0][0]), nibbles_from_f32(acc[0][1]), 0x5410u);
+    codes.y = prmt(nibbles_from_f32(acc[1][0]), nibbles_from_f32(acc[1][1]), 0x5410u);
+  }
 }
 
-__device__ __forceinline__ void err16_bf16(const uint32_t (&u)[8], float a, float ahat, uint32_t tbl, double& sd,
-                                           double& sw) {
-  if (!(a > 0.f)) return;   // all-zero block: every w and w_hat is 0
-  if (a < 0x1p-100f) err16_core<true>(u, a, ahat, tbl, sd, sw);
-  else err16_core<false>(u, a, ahat, tbl, sd, sw);
+template <bool kCodes>
+__device__ __forceinline__ void err16_bf16(const uint32_t (&u)[8], float a, float ahat, uint32_t tbl,
+                                           uint32_t tbl_base, double& sd, double& sw, uint2& codes) {
+  if (!(a > 0.f)) {   // all-zero block: every w and w_hat is 0, every code the zero code
+    codes = make_uint2(0x77777777u, 0x77777777u);
+    return;
+  }
+  if (a < 0x1p-100f) err16_core<true, kCodes>(u, a, ahat, tbl, tbl_base, sd, sw, codes);
+  else err16_core<false, kCodes>(u, a, ahat, tbl, tbl_base, sd, sw, codes);
 }
 
 // absmax (bf16 bits) of 16 weights, over the 4 lanes that share the block
@@ -91,12 +132,14 @@ __device__ __forceinline__ void finish_layer(const double2* __restrict__ partial
 // counters (zero on entry, left zero): the last chunk CTA of a layer sums that
 // layer's partials in chunk order into err[layer], and the last layer to finish
 // ranks all layers and writes order / keep.
-template <bool DQ>
-__global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_constant__ LayerTable tab,
+template <bool DQ, class Tab>
+__global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_constant__ Tab tab,
                                                                 double2* __restrict__ partial, int* status,
                                                                 int* counters, double* __restrict__ err, int K,
                                                                 int32_t* __restrict__ order, uint8_t* __restrict__ keep) {
+  constexpr bool kW = Tab::kWrite;
   __shared__ __align__(16) float2 s_tbl[33];
+  __shared__ __align__(16) float2 s_base[33];
   __shared__ float s_amax[256];
   __shared__ float s_ahat[256];
   __shared__ float s_red[8];
@@ -105,8 +148,13 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
   pdl_wait();
   pdl_launch();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid < 33) s_tbl[tid] = make_float2(__uint_as_float(kNF4CoarseD[2 * tid]), __uint_as_float(kNF4CoarseD[2 * tid + 1]));
+  if (tid < 33) {
+    s_tbl[tid] = make_float2(__uint_as_float(kNF4CoarseD[2 * tid]), __uint_as_float(kNF4CoarseD[2 * tid + 1]));
+    if constexpr (kW)
+      s_base[tid] = make_float2(__uint_as_float(kNF4CoarseQ[2 * tid]), __uint_as_float(kNF4CoarseQ[2 * tid + 1]));
+  }
   const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(s_tbl));
+  const uint32_t tbl_base = static_cast<uint32_t>(__cvta_generic_to_shared(s_base));
   const int chunk = blockIdx.x;
   int lo = 0, hi = tab.n_layers - 1;  // layer owning this chunk
   while (lo < hi) {
@@ -139,10 +187,21 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
     bad |= amb >= 0x7F80u;
     const float am = __uint_as_float(amb << 16);
     am_k[k] = am;
+    const int64_t blk = g * kDQBlock + ((k * 256 + tid) >> 2);
     if constexpr (DQ) {
       if ((tid & 3) == 0) s_amax[(k * 256 + tid) >> 2] = am;
+      if constexpr (kW) {
+        if ((tid & 3) == 0 && blk < nb && tab.absmax[layer] != nullptr) tab.absmax[layer][blk] = am;
+      }
     } else {
-      err16_bf16(cur, am, am, tbl, sd, sw);
+      uint2 cw;
+      err16_bf16<kW>(cur, am, am, tbl, tbl_base, sd, sw, cw);
+      if constexpr (kW) {
+        if (blk < nb) {
+          if ((tid & 3) == 0) tab.absmax[layer][blk] = am;
+          *reinterpret_cast<uint2*>(tab.codes[layer] + blk * (kBlock / 2) + (tid & 3) * 8) = cw;
+        }
+      }
     }
     if (k < 3) {
 #pragma unroll
@@ -168,6 +227,11 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
       ah = __fmul_rn(e4m3_to_f32(q), __fdiv_rn(G, 448.f));
     }
     s_ahat[tid] = ah;
+    if constexpr (kW) {
+      if (tid < nblk_g) tab.absmax_q[layer][g * kDQBlock + tid] =
+          (G > 0.f) ? f32_to_e4m3_satfinite(__fmul_rn(s_amax[tid], __fdiv_rn(448.f, G))) : uint8_t(0);
+      if (tid == 0) tab.absmax2[layer][g] = (G > 0.f) ? __fdiv_rn(G, 448.f) : 0.f;
+    }
     __syncthreads();
     // second pass over the chunk (from L2): codes use the exact absmax, the
     // reconstruction the double-quantized scale
@@ -175,7 +239,12 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       if (k < 3) load_task(k + 1, nxt);
-      err16_bf16(cur, am_k[k], s_ahat[(k * 256 + tid) >> 2], tbl, sd, sw);
+      uint2 cw;
+      err16_bf16<kW>(cur, am_k[k], s_ahat[(k * 256 + tid) >> 2], tbl, tbl_base, sd, sw, cw);
+      if constexpr (kW) {
+        const int64_t blk = g * kDQBlock + ((k * 256 + tid) >> 2);
+        if (blk < nb) *reinterpret_cast<uint2*>(tab.codes[layer] + blk * (kBlock / 2) + (tid & 3) * 8) = cw;
+      }
       if (k < 3) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
@@ -302,9 +371,43 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
   if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
   double2* partial = reinterpret_cast<double2*>(static_cast<char*>(ws) + kReservedBytes);
   int* counters = reinterpret_cast<int*>(static_cast<char*>(ws) + kStatusBytes);   // 1 + n_layers, zero
-  if (dq) launch_pdl(layer_error_chunk_kernel<true>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status, counters, err, K, order, keep);
-  else launch_pdl(layer_error_chunk_kernel<false>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status, counters, err, K, order, keep);
+  if (dq) launch_pdl(layer_error_chunk_kernel<true, LayerTable>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status, counters, err, K, order, keep);
+  else launch_pdl(layer_error_chunk_kernel<false, LayerTable>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status, counters, err, K, order, keep);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
+                                       int K, uint8_t* const* codes, float* const* absmax, uint8_t* const* absmax_q,
+                                       float* const* absmax2, double* err, int32_t* order, uint8_t* keep, void* ws,
+                                       size_t ws_bytes, int* status, cudaStream_t s) {
+  if (n_layers > kMaxFusedLayers) return QLORA_ERR_SHAPE;
+  static std::mutex mu;
+  static FusedTable tab;
+  std::lock_guard<std::mutex> lock(mu);
+  tab.n_layers = n_layers;
+  int32_t c = 0;
+  for (int i = 0; i < n_layers; ++i) {
+    tab.ptr[i] = W_ptrs[i];
+    tab.numel[i] = numel[i];
+    tab.codes[i] = codes[i];
+    tab.absmax[i] = absmax ? absmax[i] : nullptr;
+    tab.absmax_q[i] = dq ? absmax_q[i] : nullptr;
+    tab.absmax2[i] = dq ? absmax2[i] : nullptr;
+    tab.first_chunk[i] = c;
+    c += chunks_of(numel[i]);
+  }
+  tab.first_chunk[n_layers] = c;
+  if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
+  double2* partial = reinterpret_cast<double2*>(static_cast<char*>(ws) + kReservedBytes);
+  int* counters = reinterpret_cast<int*>(static_cast<char*>(ws) + kStatusBytes);
+  cudaError_t e;
+  if (dq)
+    e = launch_pdl(layer_error_chunk_kernel<true, FusedTable>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status,
+                   counters, err, K, order, keep);
+  else
+    e = launch_pdl(layer_error_chunk_kernel<false, FusedTable>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial,
+                   status, counters, err, K, order, keep);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------------
@@ -369,8 +472,8 @@ qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const
     c += chunks_of(numel[i]);
   }
   tab.first_chunk[n_layers] = c;
-  if (dq) layer_error_chunk_kernel<true><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr, nullptr, err, K, order, keep);
-  else layer_error_chunk_kernel<false><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr, nullptr, err, K, order, keep);
+  if (dq) layer_error_chunk_kernel<true, LayerTable><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr, nullptr, err, K, order, keep);
+  else layer_error_chunk_kernel<false, LayerTable><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr, nullptr, err, K, order, keep);
   if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
   layer_error_finish_table_kernel<<<n_layers, 256, 0, s>>>(partial, tab, err);
   rank_topk_kernel<<<1, 1024, 0, s>>>(err, n_layers, K, order, keep);

@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import layer_error
+from oracle import layer_error, nf4
 from quantized_lora_fine_b200 import api, synth
 from tests.gpu_helpers import bits
 
@@ -72,3 +72,40 @@ def test_llama_stack_all_224_matrices(cuda_device):
         assert abs(err[i] - ref) <= 1e-6 * ref, (i, err[i], ref)
     del Ws
     torch.cuda.empty_cache()
+
+
+def _compare_fused(Ws, K, dq):
+    err, order, keep, outs = api.quantize_error_rank([W.cuda() for W in Ws], K, double_quant=dq, keep_absmax=dq)
+    torch.cuda.synchronize()
+    assert api.status() == 0
+    ref_err = np.array([layer_error.layer_error(bits(W), dq) for W in Ws])
+    ref_order = layer_error.rank_layers(ref_err)
+    e = err.cpu().numpy()
+    nz = ref_err > 0
+    assert np.all(np.abs(e[nz] - ref_err[nz]) <= 1e-6 * ref_err[nz])
+    assert np.all(e[~nz] == 0)
+    assert np.array_equal(order.cpu().numpy(), ref_order)
+    assert np.array_equal(keep.cpu().numpy(), layer_error.keep_mask(ref_order, K))
+    for W, w in zip(Ws, outs):
+        qw = nf4.quantize(nf4.f32_from_bf16_bits(bits(W)).reshape(W.shape), double_quant=dq)
+        assert np.array_equal(w.codes.cpu().numpy(), qw["codes"]), "codes differ"
+        assert np.array_equal(w.absmax.cpu().numpy().view(np.uint32), qw["absmax"].view(np.uint32))
+        if dq:
+            assert np.array_equal(w.absmax_q.cpu().numpy(), qw["absmax_q"])
+            assert np.array_equal(w.absmax2.cpu().numpy().view(np.uint32), qw["absmax2"].view(np.uint32))
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_fused_quantize_error_rank_small_stack(cuda_device, dq):
+    """One pass: the same errors and ranks as the oracle's error pass and the same
+    codes and scales as the oracle's quantizer, for every layer."""
+    mats = synth.stack_matrices(n_layers=3, linears=(("a", 256, 512), ("b", 512, 256), ("c", 64, 320)))
+    Ws = [synth.stack_weight(m) for m in mats]
+    Ws.append(torch.zeros((64, 64), dtype=torch.bfloat16))
+    _compare_fused(Ws, K=4, dq=dq)
+
+
+def test_fused_quantize_error_rank_full_gate(cuda_device):
+    mats = synth.stack_matrices()
+    Ws = [synth.stack_weight(mats[i]) for i in (4, 7)]   # an 11008 x 4096 gate and a 4096^2 q
+    _compare_fused(Ws, K=1, dq=True)
