@@ -70,122 +70,119 @@ __device__ __forceinline__ void dq_group(const float* s_amax, float* s_red, int6
   if (tid == 0) absmax2[g] = (G > 0.f) ? __fdiv_rn(G, 448.f) : 0.f;
 }
 
-// bf16 weights. One CTA of 256 threads per group of 256 blocks (16384 elements);
-// in each of 4 passes a thread takes 16 consecutive elements (4 threads per block,
-// a CTA covers 8 KB contiguous per pass), loading the next pass while it codes the
-// current one. Per block: integer absmax on packed bf16 pairs (4-lane shuffle
-// max) and one IEEE reciprocal. Per element pair: Markstein division in packed
-// fp32 (exact RN(w / a) for bf16 operands); per element the code index comes from
-// the 33-cell table on the FMA pipe (cell address by RZ multiply-add, one
-// shared-memory load, a saturating FMA for the midpoint test) and is accumulated
-// as fp32 nibble weights.
-__device__ __forceinline__ void quant_load16(const uint16_t* __restrict__ W, int64_t e, int64_t numel,
-                                             uint4 (&r)[2]) {
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int64_t eh = e + 8 * h;
-    if (eh + 8 <= numel) {
-      r[h] = __ldg(reinterpret_cast<const uint4*>(W + eh));
-    } else {
-      uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;
-      if (eh + 0 < numel) t0 |= uint32_t(W[eh + 0]);
-      if (eh + 1 < numel) t0 |= uint32_t(W[eh + 1]) << 16;
-      if (eh + 2 < numel) t1 |= uint32_t(W[eh + 2]);
-      if (eh + 3 < numel) t1 |= uint32_t(W[eh + 3]) << 16;
-      if (eh + 4 < numel) t2 |= uint32_t(W[eh + 4]);
-      if (eh + 5 < numel) t2 |= uint32_t(W[eh + 5]) << 16;
-      if (eh + 6 < numel) t3 |= uint32_t(W[eh + 6]);
-      if (eh + 7 < numel) t3 |= uint32_t(W[eh + 7]) << 16;
-      r[h] = make_uint4(t0, t1, t2, t3);
-    }
-  }
-}
-
-// Codes of 16 bf16 weights (8 packed pairs) of a block with absmax am > 0, as two
-// words in storage order (byte k = idx[2k] << 4 | idx[2k + 1]).
-__device__ __forceinline__ uint2 quant16_bf16(const uint32_t (&u)[8], float am, uint32_t tbl) {
-  float a = am;
-  uint64_t wp[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) wp[i] = f2_from_bf16x2(u[i]);
-  if (am < 0x1p-100f) {   // tiny block: rescale by 2^64 (exact) so that 1/a stays normal
-    a = am * 0x1p64f;
-    const uint64_t s64 = f2_splat(0x1p64f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) wp[i] = f2_mul(wp[i], s64);
-  }
-  const uint64_t r2 = f2_splat(__frcp_rn(a)), na2 = f2_splat(-a);
-  uint32_t word[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    // within a 16-bit half the 4 elements weigh 16, 1, 4096, 256 (storage order)
-    float acc[2] = {0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint64_t q = f2_div_by_recip(wp[4 * h + i], na2, r2);
-      const float n0 = f2_lo(q), n1 = f2_hi(q);
-      const uint64_t cells = coarse_cells2(q);
-      const float2 t0 = lds_f2(coarse_addr_bits<8>(uint32_t(cells), tbl));
-      const float2 t1 = lds_f2(coarse_addr_bits<8>(uint32_t(cells >> 32), tbl));
-      const float w0 = (i & 1) ? 4096.f : 16.f, w1 = (i & 1) ? 256.f : 1.f;
-      acc[i >> 1] = __fmaf_rn(t0.y + sat_fma(n0, 0x1p100f, t0.x), w0, acc[i >> 1]);
-      acc[i >> 1] = __fmaf_rn(t1.y + sat_fma(n1, 0x1p100f, t1.x), w1, acc[i >> 1]);
-    }
-    word[h] = prmt(nibbles_from_f32(acc[0]), nibbles_from_f32(acc[1]), 0x5410u);
-  }
-  return make_uint2(word[0], word[1]);
-}
-
+// bf16 weights. One CTA of 256 threads per group of 256 blocks (16384 elements, the
+// double-quant group); thread t owns block t. The group's weights (up to 32 KB)
+// reach shared memory by one bulk copy (an odd tail of fewer than 8 elements by
+// plain loads); thread t reads its block as eight 16-byte pieces, piece j ^ (t mod 8)
+// at step j, so that the 8 lanes of a quarter warp touch 8 different bank groups.
+// Per block: absmax over packed bf16 pairs and one reciprocal r = RN(1/a). Per
+// element pair: one packed fp32 multiply n~ = RN(w r). For every pair of bf16
+// values with |w| <= a, n~ lies on the same side of every code midpoint as the
+// IEEE quotient RN(w / a) (an exhaustive check over all significand pairs and
+// exponent gaps; the GPU tests repeat it through this kernel), so n~ picks the
+// same code. Per element the code index comes from a 32-cell lookup held in the
+// warp's registers: cell = floor(15.75 n~ + 16) from the bits of an RZ multiply-add,
+// the cell's base index B and the midpoint above it by two warp shuffles, s =
+// sat(n~ 2^36 + T) in {0, 1}, and bits(B + s) carry the index; a multiply-add chain
+// packs 8 of them into a code word. Three exchange stages put the thread's 8 code
+// words back in order, and the block's 32 bytes leave in two 16-byte stores.
 template <bool DQ>
-__global__ void __launch_bounds__(256) nf4_quantize_bf16_kernel(const uint16_t* __restrict__ W, int64_t numel,
-                                                                uint8_t* __restrict__ codes,
-                                                                float* __restrict__ absmax,
-                                                                uint8_t* __restrict__ absmax_q,
-                                                                float* __restrict__ absmax2, int* status) {
-  __shared__ __align__(16) float2 s_tbl[33];
-  __shared__ float s_amax[256];
+__global__ void __launch_bounds__(256, 4) nf4_quantize_bf16_kernel(const uint16_t* __restrict__ W, int64_t numel,
+                                                                   uint8_t* __restrict__ codes,
+                                                                   float* __restrict__ absmax,
+                                                                   uint8_t* __restrict__ absmax_q,
+                                                                   float* __restrict__ absmax2, int* status) {
+  __shared__ __align__(128) uint32_t s_w[kChunkBytes / 4];   // the group's bf16 pairs
+  __shared__ float s_amax[kDQBlock];
   __shared__ float s_red[8];
-  pdl_wait();
-  pdl_launch();
-  const int tid = threadIdx.x, lane = tid & 31;
-  if (tid < 33) s_tbl[tid] = make_float2(__uint_as_float(kNF4CoarseQ[2 * tid]), __uint_as_float(kNF4CoarseQ[2 * tid + 1]));
-  const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(s_tbl));
-  __syncthreads();
+  __shared__ __align__(8) uint64_t s_bar;
+  const int tid = threadIdx.x;
+  const uint32_t bar = smem_u32(&s_bar);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbarrier_init();
+  }
+  const LaneTables lt = lane_tables(tid & 31);
   const int64_t nb = (numel + kBlock - 1) / kBlock;
   const int64_t g = blockIdx.x;
-  const int64_t g0 = g * int64_t(kDQBlock * kBlock);   // first element of the group
-  uint32_t bad = 0;
-  uint4 cur[2], nxt[2];
-  quant_load16(W, g0 + int64_t(tid) * 16, numel, cur);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    if (k < 3) quant_load16(W, g0 + int64_t((k + 1) * 256 + tid) * 16, numel, nxt);
-    const int bi = (k * 256 + tid) >> 2;               // block within the group
-    const int64_t blk = g * kDQBlock + bi;
-    const int64_t e0 = g0 + int64_t(k * 256 + tid) * 16;
-    const uint32_t u[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
-    uint32_t m = __vmaxu2(u[0] & 0x7FFF7FFFu, u[1] & 0x7FFF7FFFu);
-#pragma unroll
-    for (int i = 2; i < 8; ++i) m = __vmaxu2(m, u[i] & 0x7FFF7FFFu);
-    uint32_t amb = max(m >> 16, m & 0xFFFFu);
-    amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 1));
-    amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 2));
-    bad |= amb >= 0x7F80u;
-    const float am = __uint_as_float(amb << 16);
-    if ((lane & 3) == 0) {
-      if constexpr (DQ) s_amax[bi] = am;
-      if (absmax != nullptr && blk < nb) absmax[blk] = am;
+  const int64_t e_g = g * int64_t(kDQBlock * kBlock);                 // first element of the group
+  const int n_g = int(min(int64_t(kDQBlock * kBlock), numel - e_g));  // its elements (even, > 0)
+  const int nblk = (n_g + kBlock - 1) / kBlock;
+  const uint32_t bulk = uint32_t(n_g * 2) & ~15u;                     // bytes the bulk copy moves
+  __syncthreads();
+  pdl_wait();
+  pdl_launch();
+  if (bulk > 0) {
+    if (tid == 0) {
+      mbar_arrive_expect_tx(bar, bulk);
+      bulk_load(smem_u32(s_w), W + e_g, bulk, bar);
     }
-    if (e0 < numel) {
-      const uint2 word = (am > 0.f) ? quant16_bf16(u, am, tbl) : make_uint2(0x77777777u, 0x77777777u);
-      if (e0 + 16 <= numel) {
-        *reinterpret_cast<uint2*>(codes + e0 / 2) = word;
-      } else {
-        const uint64_t both = (uint64_t(word.y) << 32) | word.x;
-        for (int kb = 0; 2 * kb < numel - e0; ++kb) codes[e0 / 2 + kb] = uint8_t(both >> (8 * kb));
-      }
+    const bool landed = mbar_wait(bar, 0);
+    if (!__syncthreads_and(landed)) {   // every thread leaves together
+      if (tid == 0) set_status(status, QLORA_ERR_TIMEOUT);
+      if (!landed) mbar_wait(bar, 0, 20000000000ull);   // the copy must land before the CTA's memory is released
+      return;
     }
-    if (k < 3) { cur[0] = nxt[0]; cur[1] = nxt[1]; }
+  }
+  // the last block of a ragged group: elements past the bulk copy by plain loads
+  // (whole bf16 pairs: numel is even), zeros to the end of the block
+  const int tail0 = int(bulk / 2);
+  if (tail0 < nblk * kBlock && tid == tail0 / kBlock) {
+    for (int e = tail0; e < nblk * kBlock; e += 2)
+      s_w[e / 2] = (e < n_g) ? __ldg(reinterpret_cast<const uint32_t*>(W + e_g + e)) : 0u;
+  }
+  const bool valid = tid < nblk;
+  const uint32_t rot = uint32_t(tid & 7);
+  uint32_t u[8][4];
+  if (valid) {
+    const uint32_t src = smem_u32(s_w) + uint32_t(tid) * 128u + rot * 16u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) lds_u4(src ^ (uint32_t(j) << 4), u[j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+  }
+  uint32_t m = bf16x2_maxabs(u[0][0], u[0][1]);
+#pragma unroll
+  for (int k = 2; k < 32; ++k) m = bf16x2_maxabs(m, u[k >> 2][k & 3]);
+  m &= 0x7FFF7FFFu;
+  const uint32_t amb = max(m >> 16, m & 0xFFFFu);
+  const bool bad = amb >= 0x7F80u;
+  const float am = __uint_as_float(amb << 16);
+  if (valid) {
+    if constexpr (DQ) s_amax[tid] = am;
+    if (absmax != nullptr) absmax[g * kDQBlock + tid] = am;
+  }
+  // Every lane runs the lookup (it holds warp shuffles). Lanes without a live block
+  // (past the group, all-zero or non-finite) run it on zeros with a = 1, which keeps
+  // every quotient finite; their code words are the zero code (a non-finite block
+  // sets the status word).
+  const bool live = am > 0.f && !bad;
+  if (bad) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+  }
+  const CellScale cs(live ? am : 1.f);
+  uint32_t cw[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint32_t x[8];
+    piece_index_bits(u[j], cs, lt, x);
+    cw[j] = live ? pack_code_word(x) : 0x77777777u;
+  }
+  if (valid) {
+    unrotate8(cw, rot);
+    // the block's 32 code bytes (fewer in a ragged last block)
+    const int cb = min(32, n_g / 2 - 32 * tid);
+    uint8_t* dst = codes + e_g / 2 + 32 * tid;
+    if (cb == 32) {
+      reinterpret_cast<uint4*>(dst)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      reinterpret_cast<uint4*>(dst)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    } else {
+#pragma unroll
+      for (int b = 0; b < 32; ++b)   // static indices keep cw in registers
+        if (b < cb) dst[b] = uint8_t(cw[b >> 2] >> (8 * (b & 3)));
+    }
   }
   if (bad) set_status(status, QLORA_ERR_NONFINITE);
   if constexpr (DQ) dq_group(s_amax, s_red, nb, g, absmax_q, absmax2);

@@ -39,6 +39,12 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+int num_sms();
+
+// The quantizer and the error pass stage one chunk of 256 blocks (32 KB of bf16,
+// the double-quant group) per CTA in shared memory.
+constexpr uint32_t kChunkBytes = uint32_t(kDQBlock) * kBlock * 2u;
+
 __device__ __forceinline__ void set_status(int* st, int code) {
   if (st) atomicCAS(st, 0, code);
 }
@@ -79,7 +85,6 @@ qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const
                                              cudaStream_t s);
 
 // ---- gemm.cu
-int num_sms();
 // Operand descriptions for the tcgen05 GEMM engine.
 struct GemmPlan;
 }  // namespace qlb

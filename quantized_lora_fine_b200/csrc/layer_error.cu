@@ -46,173 +46,106 @@ struct FusedTable {
 };
 static_assert(sizeof(FusedTable) <= 32000, "kernel parameter limit");
 
-// Error contribution of 16 bf16 weights (8 packed pairs) of one block: codes
-// from the exact absmax a (same arithmetic as the quantizer), reconstruction
-// w_hat = bf16(fp32(code * ahat)) with ahat = a, or the double-quantized scale.
-// Squares are summed per pair lane in fp32 (8 terms) before the fp64 total.
-// With kCodes, also the 16 codes in storage order (byte k = idx[2k] << 4 |
-// idx[2k + 1]): idx = base + sat(n 2^100 + T) from the quantizer's {T, base}
-// table (tbl_base), the four indices of a 16-bit half accumulated as fp32
-// nibble weights.
-template <bool kTiny, bool kCodes>
-__device__ __forceinline__ void err16_core(const uint32_t (&u)[8], float a, float ahat, uint32_t tbl,
-                                           uint32_t tbl_base, double& sd, double& sw, uint2& codes) {
-  float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-  // tiny blocks: the division operands are rescaled by 2^64 (exact) so 1/a stays normal
-  const float as = kTiny ? a * 0x1p64f : a;
-  const uint64_t r2 = f2_splat(__frcp_rn(as)), na2 = f2_splat(-as), ah2 = f2_splat(ahat);
-  uint64_t sd2 = 0, sw2 = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint64_t w = f2_from_bf16x2(u[i]);
-    const uint64_t q = f2_div_by_recip(kTiny ? f2_mul(w, f2_splat(0x1p64f)) : w, na2, r2);
-    // cell entries {code[base], code[base + 1] - code[base]}; RN(2 lo + diff) is twice
-    // the cell's midpoint, so s = sat(n 2^100 - RN(2 lo + diff) 2^99) tests n > m
-    const uint64_t cells = coarse_cells2(q);
-    const uint64_t n2 = f2_mul(q, 0x7180000071800000ull);   // n * 2^100, both lanes
-    const float2 e0 = lds_f2(coarse_addr_bits<8>(uint32_t(cells), tbl));
-    const float2 e1 = lds_f2(coarse_addr_bits<8>(uint32_t(cells >> 32), tbl));
-    const float s0 = sat_fma(__fmaf_rn(e0.x, 2.f, e0.y), -0x1p99f, f2_lo(n2));
-    const float s1 = sat_fma(__fmaf_rn(e1.x, 2.f, e1.y), -0x1p99f, f2_hi(n2));
-    const float c0 = __fmaf_rn(s0, e0.y, e0.x);   // code value (exact)
-    const float c1 = __fmaf_rn(s1, e1.y, e1.x);
-    if constexpr (kCodes) {
-      // the index needs the midpoint test of the quantizer's table: in a cell
-      // without a midpoint s above may be 1 (harmless for the value, not for idx)
-      const float2 t0 = lds_f2(coarse_addr_bits<8>(uint32_t(cells), tbl_base));
-      const float2 t1 = lds_f2(coarse_addr_bits<8>(uint32_t(cells >> 32), tbl_base));
-      const float i0 = t0.y + sat_fma(f2_lo(q), 0x1p100f, t0.x);
-      const float i1 = t1.y + sat_fma(f2_hi(q), 0x1p100f, t1.x);
-      const int h = i >> 2, j = i & 3;
-      acc[h][j >> 1] = __fmaf_rn(i0, (j & 1) ? 4096.f : 16.f, acc[h][j >> 1]);
-      acc[h][j >> 1] = __fmaf_rn(i1, (j & 1) ? 256.f : 1.f, acc[h][j >> 1]);
+__device__ __forceinline__ void finish_layer_warp(const double2* __restrict__ partial, int c0, int c1,
+                                                  double* __restrict__ err_out);
+
+// Chunk c of the table: its layer (binary search over first_chunk), index within
+// the layer and number of blocks.
+template <class Tab>
+struct ChunkRef {
+  int layer;
+  int64_t g;
+  int nblk;
+  __device__ __forceinline__ ChunkRef(const Tab& tab, int64_t c) {
+    int lo = 0, hi = tab.n_layers - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tab.first_chunk[mid] <= c) lo = mid; else hi = mid - 1;
     }
-    const uint64_t p = f2_mul((uint64_t(__float_as_uint(c1)) << 32) | __float_as_uint(c0), ah2);
-    const uint64_t wh = f2_from_bf16x2(pack_bf16x2(f2_lo(p), f2_hi(p)));
-    const uint64_t d = f2_sub(w, wh);
-    sd2 = f2_fma(d, d, sd2);
-    sw2 = f2_fma(w, w, sw2);
+    layer = lo;
+    g = c - tab.first_chunk[lo];
+    const int64_t nb = tab.numel[lo] / kBlock;
+    nblk = int(min(int64_t(kDQBlock), nb - g * kDQBlock));
   }
-  sd += double(f2_lo(sd2)) + double(f2_hi(sd2));
-  sw += double(f2_lo(sw2)) + double(f2_hi(sw2));
-  if constexpr (kCodes) {
-    codes.x = prmt(nibbles_from_f32(acc[0][0]), nibbles_from_f32(acc[0][1]), 0x5410u);
-    codes.y = prmt(nibbles_from_f32(acc[1][0]), nibbles_from_f32(acc[1][1]), 0x5410u);
-  }
-}
-
-template <bool kCodes>
-__device__ __forceinline__ void err16_bf16(const uint32_t (&u)[8], float a, float ahat, uint32_t tbl,
-                                           uint32_t tbl_base, double& sd, double& sw, uint2& codes) {
-  if (!(a > 0.f)) {   // all-zero block: every w and w_hat is 0, every code the zero code
-    codes = make_uint2(0x77777777u, 0x77777777u);
-    return;
-  }
-  if (a < 0x1p-100f) err16_core<true, kCodes>(u, a, ahat, tbl, tbl_base, sd, sw, codes);
-  else err16_core<false, kCodes>(u, a, ahat, tbl, tbl_base, sd, sw, codes);
-}
-
-// absmax (bf16 bits) of 16 weights, over the 4 lanes that share the block
-__device__ __forceinline__ uint32_t absmax16_lanes(const uint32_t (&u)[8]) {
-  uint32_t m = __vmaxu2(u[0] & 0x7FFF7FFFu, u[1] & 0x7FFF7FFFu);
-#pragma unroll
-  for (int i = 2; i < 8; ++i) m = __vmaxu2(m, u[i] & 0x7FFF7FFFu);
-  uint32_t amb = max(m >> 16, m & 0xFFFFu);
-  amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 1));
-  amb = max(amb, __shfl_xor_sync(0xffffffffu, amb, 2));
-  return amb;
-}
-
-__device__ __forceinline__ void finish_layer(const double2* __restrict__ partial, int c0, int c1,
-                                             double* __restrict__ err_out);
+};
 
 // Pass 1 (and, with counters, passes 2-3 fused): one CTA per chunk of 256 blocks
-// of some layer; in each of 4 passes a thread takes 16 consecutive weights (4
-// threads per block). The chunk's (sum d^2, sum w^2) goes to partial[chunk]. With
-// counters (zero on entry, left zero): the last chunk CTA of a layer sums that
-// layer's partials in chunk order into err[layer], and the last layer to finish
-// ranks all layers and writes order / keep.
+// (16384 weights, the double-quant group) of some layer; thread t owns block t. The
+// chunk's bf16 weights reach shared memory by one bulk copy; thread t reads its
+// block as eight 16-byte pieces, piece j ^ (t mod 8) at step j (the 8 lanes of a
+// quarter warp touch 8 different bank groups). Per block: absmax over packed bf16
+// pairs; with double quant the chunk's max G of the absmax values gives the
+// reconstruction scale ahat = e4m3(a 448 / G) G / 448 (the codes use the exact a).
+// Per element: the code index from the one-multiply quotient and the shuffle
+// lookup (as the quantizer), the code value by one more warp shuffle from the lane
+// that holds it (lane l holds code[l mod 16]; the index bits select the lane),
+// w_hat = bf16(fp32(code ahat)), and (w_hat - w)^2 (a mixed bf16 - fp32
+// subtraction), w^2 summed in packed fp32 (16 terms per accumulator) before the
+// fp64 chunk total. With Tab::kWrite (the fused pass) the thread's 8 code words go
+// back in order and out in two 16-byte stores, with the scales. Warp 0 sums the
+// 256 per-thread totals in a fixed order into partial[chunk]; with counters (zero
+// on entry, left zero) it also finishes: the chunk that completes a layer sums
+// that layer's partials in chunk order into err[layer], and the one that
+// completes the last layer ranks all layers and writes order / keep. The other
+// warps leave as soon as their totals are in shared memory.
 template <bool DQ, class Tab>
-__global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_constant__ Tab tab,
-                                                                double2* __restrict__ partial, int* status,
-                                                                int* counters, double* __restrict__ err, int K,
-                                                                int32_t* __restrict__ order, uint8_t* __restrict__ keep) {
+__global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_constant__ Tab tab,
+                                                                   double2* __restrict__ partial, int* status,
+                                                                   int* counters, double* __restrict__ err, int K,
+                                                                   int32_t* __restrict__ order,
+                                                                   uint8_t* __restrict__ keep) {
   constexpr bool kW = Tab::kWrite;
-  __shared__ __align__(16) float2 s_tbl[33];
-  __shared__ __align__(16) float2 s_base[33];
-  __shared__ float s_amax[256];
-  __shared__ float s_ahat[256];
+  __shared__ __align__(128) uint32_t s_w[kChunkBytes / 4];
+  __shared__ double2 s_part[256];
   __shared__ float s_red[8];
-  __shared__ double s_sum[2][8];
-  __shared__ int s_flag;
+  __shared__ __align__(8) uint64_t s_bar;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t bar = smem_u32(&s_bar);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbarrier_init();
+  }
+  const LaneTables lt = lane_tables(lane);
+  const int64_t chunk = blockIdx.x;
+  const ChunkRef<Tab> cr(tab, chunk);
+  const int layer = cr.layer, nblk = cr.nblk;
+  const int64_t g = cr.g;
+  __syncthreads();   // barrier in place
   pdl_wait();
   pdl_launch();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid < 33) {
-    s_tbl[tid] = make_float2(__uint_as_float(kNF4CoarseD[2 * tid]), __uint_as_float(kNF4CoarseD[2 * tid + 1]));
-    if constexpr (kW)
-      s_base[tid] = make_float2(__uint_as_float(kNF4CoarseQ[2 * tid]), __uint_as_float(kNF4CoarseQ[2 * tid + 1]));
+  if (tid == 0) {
+    const uint32_t bytes = uint32_t(nblk) * kBlock * 2u;
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(smem_u32(s_w), tab.ptr[layer] + g * (kDQBlock * kBlock), bytes, bar);
   }
-  const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(s_tbl));
-  const uint32_t tbl_base = static_cast<uint32_t>(__cvta_generic_to_shared(s_base));
-  const int chunk = blockIdx.x;
-  int lo = 0, hi = tab.n_layers - 1;  // layer owning this chunk
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (tab.first_chunk[mid] <= chunk) lo = mid; else hi = mid - 1;
+  const bool landed = mbar_wait(bar, 0);
+  if (!__syncthreads_and(landed)) {   // every thread leaves together
+    if (tid == 0 && status) set_status(status, QLORA_ERR_TIMEOUT);
+    if (!landed) mbar_wait(bar, 0, 20000000000ull);   // the copy must land before the CTA's memory is released
+    return;
   }
-  const int layer = lo;
-  const uint16_t* W = tab.ptr[layer];
-  const int64_t nb = tab.numel[layer] / kBlock;
-  const int64_t g = chunk - tab.first_chunk[layer];
-  // task k of this thread: weights [16 (tid & 3), +16) of block 64 k + tid / 4
-  auto load_task = [&](int k, uint32_t (&u)[8]) {
-    const int64_t blk = g * kDQBlock + ((k * 256 + tid) >> 2);
-    const uint16_t* src = W + blk * kBlock + (tid & 3) * 16;
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    const uint4 v0 = (blk < nb) ? __ldg(reinterpret_cast<const uint4*>(src)) : z;
-    const uint4 v1 = (blk < nb) ? __ldg(reinterpret_cast<const uint4*>(src + 8)) : z;
-    u[0] = v0.x; u[1] = v0.y; u[2] = v0.z; u[3] = v0.w; u[4] = v1.x; u[5] = v1.y; u[6] = v1.z; u[7] = v1.w;
-  };
-  __syncthreads();   // the table is in place
-  uint32_t bad = 0;
-  double sd = 0.0, sw = 0.0;
-  float am_k[4];
-  uint32_t cur[8], nxt[8];
-  load_task(0, cur);
+  const bool valid = tid < nblk;
+  const uint32_t rot = uint32_t(tid & 7);
+  uint32_t u[8][4];
+  if (valid) {
+    const uint32_t src = smem_u32(s_w) + uint32_t(tid) * 128u + rot * 16u;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    if (k < 3) load_task(k + 1, nxt);
-    const uint32_t amb = absmax16_lanes(cur);
-    bad |= amb >= 0x7F80u;
-    const float am = __uint_as_float(amb << 16);
-    am_k[k] = am;
-    const int64_t blk = g * kDQBlock + ((k * 256 + tid) >> 2);
-    if constexpr (DQ) {
-      if ((tid & 3) == 0) s_amax[(k * 256 + tid) >> 2] = am;
-      if constexpr (kW) {
-        if ((tid & 3) == 0 && blk < nb && tab.absmax[layer] != nullptr) tab.absmax[layer][blk] = am;
-      }
-    } else {
-      uint2 cw;
-      err16_bf16<kW>(cur, am, am, tbl, tbl_base, sd, sw, cw);
-      if constexpr (kW) {
-        if (blk < nb) {
-          if ((tid & 3) == 0) tab.absmax[layer][blk] = am;
-          *reinterpret_cast<uint2*>(tab.codes[layer] + blk * (kBlock / 2) + (tid & 3) * 8) = cw;
-        }
-      }
-    }
-    if (k < 3) {
+    for (int j = 0; j < 8; ++j) lds_u4(src ^ (uint32_t(j) << 4), u[j]);
+  } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
-    }
+    for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
   }
-  if (bad && status) set_status(status, QLORA_ERR_NONFINITE);
+  uint32_t m = bf16x2_maxabs(u[0][0], u[0][1]);
+#pragma unroll
+  for (int k = 2; k < 32; ++k) m = bf16x2_maxabs(m, u[k >> 2][k & 3]);
+  m &= 0x7FFF7FFFu;
+  const uint32_t amb = max(m >> 16, m & 0xFFFFu);
+  const bool bad = amb >= 0x7F80u;
+  const float am = __uint_as_float(amb << 16);
+  const int64_t blk = g * kDQBlock + tid;
+  float ahat = am;
   if constexpr (DQ) {
-    __syncthreads();
-    const int64_t nblk_g = (int64_t(kDQBlock) < nb - g * kDQBlock ? int64_t(kDQBlock) : nb - g * kDQBlock);
-    float v = (tid < nblk_g) ? s_amax[tid] : 0.f;
+    float v = valid ? am : 0.f;   // max over the chunk (NaN blocks compare false and drop out)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     if (lane == 0) s_red[warp] = v;
@@ -220,77 +153,115 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
     float G = s_red[0];
 #pragma unroll
     for (int i = 1; i < 8; ++i) G = fmaxf(G, s_red[i]);
-    float ah = 0.f;
-    if (G > 0.f && tid < nblk_g) {
-      const float inv = __fdiv_rn(448.f, G);
-      const uint8_t q = f32_to_e4m3_satfinite(__fmul_rn(s_amax[tid], inv));
-      ah = __fmul_rn(e4m3_to_f32(q), __fdiv_rn(G, 448.f));
+    uint8_t q8 = 0;
+    ahat = 0.f;
+    if (G > 0.f) {
+      q8 = f32_to_e4m3_satfinite(__fmul_rn(am, __fdiv_rn(448.f, G)));
+      ahat = __fmul_rn(e4m3_to_f32(q8), __fdiv_rn(G, 448.f));
     }
-    s_ahat[tid] = ah;
     if constexpr (kW) {
-      if (tid < nblk_g) tab.absmax_q[layer][g * kDQBlock + tid] =
-          (G > 0.f) ? f32_to_e4m3_satfinite(__fmul_rn(s_amax[tid], __fdiv_rn(448.f, G))) : uint8_t(0);
+      if (valid) {
+        tab.absmax_q[layer][blk] = q8;
+        if (tab.absmax[layer] != nullptr) tab.absmax[layer][blk] = am;
+      }
       if (tid == 0) tab.absmax2[layer][g] = (G > 0.f) ? __fdiv_rn(G, 448.f) : 0.f;
     }
-    __syncthreads();
-    // second pass over the chunk (from L2): codes use the exact absmax, the
-    // reconstruction the double-quantized scale
-    load_task(0, cur);
+  } else if constexpr (kW) {
+    if (valid) tab.absmax[layer][blk] = am;
+  }
+  // Every lane runs the element loop (it holds warp shuffles). Lanes without a live
+  // block (past the chunk, all-zero or non-finite) run it on zeros with a = 1, which
+  // keeps every quotient finite and adds nothing to the sums; their code words are
+  // the zero code.
+  const bool live = valid && am > 0.f && !bad;
+  if (bad) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      if (k < 3) load_task(k + 1, nxt);
-      uint2 cw;
-      err16_bf16<kW>(cur, am_k[k], s_ahat[(k * 256 + tid) >> 2], tbl, tbl_base, sd, sw, cw);
-      if constexpr (kW) {
-        const int64_t blk = g * kDQBlock + ((k * 256 + tid) >> 2);
-        if (blk < nb) *reinterpret_cast<uint2*>(tab.codes[layer] + blk * (kBlock / 2) + (tid & 3) * 8) = cw;
-      }
-      if (k < 3) {
+    for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+  }
+  const CellScale cs(live ? am : 1.f);
+  const uint64_t ah2 = f2_splat(ahat);
+  uint64_t sd2[2] = {0ull, 0ull}, sw2[2] = {0ull, 0ull};
+  uint32_t cw[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
-      }
+  for (int j = 0; j < 8; ++j) {
+    uint32_t x[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint64_t w = f2_from_bf16x2(u[j][i]);
+      const uint64_t q = f2_mul(w, cs.r2);
+      const uint64_t c = cells2(q, cs.cmul2);
+      x[2 * i] = index_bits(f2_lo(q), uint32_t(c), cs.M, lt);
+      x[2 * i + 1] = index_bits(f2_hi(q), uint32_t(c >> 32), cs.M, lt);
+      const float c0 = code_value(x[2 * i], lt), c1 = code_value(x[2 * i + 1], lt);
+      const uint64_t p = f2_mul((uint64_t(__float_as_uint(c1)) << 32) | __float_as_uint(c0), ah2);
+      const uint64_t d = f2_bf16x2_minus(pack_bf16x2(f2_lo(p), f2_hi(p)), w);
+      sd2[j >> 2] = f2_fma(d, d, sd2[j >> 2]);
+      sw2[j >> 2] = f2_fma(w, w, sw2[j >> 2]);
     }
+    if constexpr (kW) cw[j] = live ? pack_code_word(x) : 0x77777777u;
+  }
+  if constexpr (kW) {
+    if (valid) {
+      unrotate8(cw, rot);
+      uint4* dst = reinterpret_cast<uint4*>(tab.codes[layer] + blk * (kBlock / 2));
+      dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    }
+  }
+  if (bad && status) set_status(status, QLORA_ERR_NONFINITE);
+  double sd = 0.0, sw = 0.0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    sd += double(f2_lo(sd2[h])) + double(f2_hi(sd2[h]));
+    sw += double(f2_lo(sw2[h])) + double(f2_hi(sw2[h]));
+  }
+  s_part[tid] = make_double2(sd, sw);
+  __syncthreads();
+  if (warp != 0) return;
+  // ---- warp 0: the chunk total in a fixed order, then the fused finish
+  double a = 0.0, b = 0.0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const double2 v = s_part[lane * 8 + k];
+    a += v.x;
+    b += v.y;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    sd += __shfl_xor_sync(0xffffffffu, sd, o);
-    sw += __shfl_xor_sync(0xffffffffu, sw, o);
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
   }
-  if (lane == 0) { s_sum[0][warp] = sd; s_sum[1][warp] = sw; }
-  __syncthreads();
-  if (tid == 0) {
-    double a = 0.0, b = 0.0;
-    for (int i = 0; i < 8; ++i) { a += s_sum[0][i]; b += s_sum[1][i]; }
-    partial[chunk] = make_double2(a, b);
-  }
+  if (lane == 0) partial[chunk] = make_double2(a, b);
   if (counters == nullptr) return;
-  // ---- fused finish: last chunk of the layer -> err[layer]; last layer -> ranks
-  if (tid == 0) {
+  int last = 0;
+  if (lane == 0) {
     __threadfence();
-    const int nchunks = tab.first_chunk[layer + 1] - tab.first_chunk[layer];
+    const int nchunks_l = tab.first_chunk[layer + 1] - tab.first_chunk[layer];
     const int done = atomicAdd(counters + 1 + layer, 1);
-    s_flag = (done == nchunks - 1);
-    if (s_flag) atomicExch(counters + 1 + layer, 0);
+    last = (done == nchunks_l - 1);
+    if (last) atomicExch(counters + 1 + layer, 0);
   }
-  __syncthreads();
-  if (!s_flag) return;
+  if (!__shfl_sync(0xffffffffu, last, 0)) return;
   __threadfence();
-  finish_layer(partial, tab.first_chunk[layer], tab.first_chunk[layer + 1], err + layer);
-  if (tid == 0) {
+  finish_layer_warp(partial, tab.first_chunk[layer], tab.first_chunk[layer + 1], err + layer);
+  if (lane == 0) {
     __threadfence();
     const int done = atomicAdd(counters, 1);
-    s_flag = (done == tab.n_layers - 1);
-    if (s_flag) atomicExch(counters, 0);
+    last = (done == tab.n_layers - 1);
+    if (last) atomicExch(counters, 0);
   }
-  __syncthreads();
-  if (!s_flag) return;
+  if (!__shfl_sync(0xffffffffu, last, 0)) return;
   __threadfence();
+  // rank all layers (err desc, id asc); the errors are staged in the chunk buffer
   const int n = tab.n_layers;
-  for (int l = tid; l < n; l += 256) {
-    const double e = __ldcg(err + l);
+  double* s_err = reinterpret_cast<double*>(s_w);
+  for (int l = lane; l < n; l += 32) s_err[l] = __ldcg(err + l);
+  __syncwarp();
+  for (int l = lane; l < n; l += 32) {
+    const double e = s_err[l];
     int rank = 0;
     for (int j = 0; j < n; ++j) {
-      const double f = __ldcg(err + j);
+      const double f = s_err[j];
       rank += (f > e || (f == e && j < l)) ? 1 : 0;
     }
     order[rank] = l;
@@ -298,25 +269,24 @@ __global__ void __launch_bounds__(256) layer_error_chunk_kernel(const __grid_con
   }
 }
 
-// One CTA per layer: thread t sums chunks first+t, first+t+256, ... in order, then a
-// fixed-shape tree combines the 256 partials -- deterministic for a given layout.
-__device__ __forceinline__ void finish_layer(const double2* __restrict__ partial, int c0, int c1,
-                                             double* __restrict__ err_out) {
-  __shared__ double s_a[256], s_b[256];
+// One warp per layer: lane l sums chunks first+l, first+l+32, ... in order; the 32
+// lane sums combine by a fixed shuffle pattern, so the result is deterministic for
+// a given layout.
+__device__ __forceinline__ void finish_layer_warp(const double2* __restrict__ partial, int c0, int c1,
+                                                  double* __restrict__ err_out) {
+  const int lane = threadIdx.x & 31;
   double a = 0.0, b = 0.0;
-  for (int c = c0 + threadIdx.x; c < c1; c += 256) {
+  for (int c = c0 + lane; c < c1; c += 32) {
     const double2 v = __ldcg(partial + c);
     a += v.x;
     b += v.y;
   }
-  s_a[threadIdx.x] = a;
-  s_b[threadIdx.x] = b;
-  __syncthreads();
-  for (int o = 128; o > 0; o >>= 1) {
-    if (threadIdx.x < o) { s_a[threadIdx.x] += s_a[threadIdx.x + o]; s_b[threadIdx.x] += s_b[threadIdx.x + o]; }
-    __syncthreads();
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
   }
-  if (threadIdx.x == 0) *err_out = (s_b[0] > 0.0) ? sqrt(s_a[0] / s_b[0]) : 0.0;
+  if (lane == 0) *err_out = (b > 0.0) ? sqrt(a / b) : 0.0;
 }
 
 __global__ void __launch_bounds__(1024) rank_topk_kernel(const double* __restrict__ err, int n_layers, int K,
@@ -336,7 +306,7 @@ __global__ void __launch_bounds__(1024) rank_topk_kernel(const double* __restric
   }
 }
 
-__global__ void __launch_bounds__(256) layer_error_finish_table_kernel(const double2* __restrict__ partial,
+__global__ void __launch_bounds__(32) layer_error_finish_table_kernel(const double2* __restrict__ partial,
                                                                        const __grid_constant__ LayerTable tab,
                                                                        double* __restrict__ err);
 
@@ -349,6 +319,17 @@ size_t layer_error_ws_bytes(int n_layers, const int64_t* numel) {
   int64_t chunks = 0;
   for (int i = 0; i < n_layers; ++i) chunks += chunks_of(numel[i]);
   return kReservedBytes + size_t(chunks) * sizeof(double2);
+}
+
+// Launch of the chunk kernel over c chunks.
+template <bool DQ, class Tab>
+static cudaError_t launch_chunks(const Tab& tab, int64_t c, double2* partial, int* status, int* counters,
+                                 double* err, int K, int32_t* order, uint8_t* keep, cudaStream_t s, bool pdl) {
+  auto kern = layer_error_chunk_kernel<DQ, Tab>;
+  if (pdl)
+    return launch_pdl(kern, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status, counters, err, K, order, keep);
+  kern<<<unsigned(c), 256, 0, s>>>(tab, partial, status, counters, err, K, order, keep);
+  return cudaGetLastError();
 }
 
 qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
@@ -371,9 +352,9 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
   if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
   double2* partial = reinterpret_cast<double2*>(static_cast<char*>(ws) + kReservedBytes);
   int* counters = reinterpret_cast<int*>(static_cast<char*>(ws) + kStatusBytes);   // 1 + n_layers, zero
-  if (dq) launch_pdl(layer_error_chunk_kernel<true, LayerTable>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status, counters, err, K, order, keep);
-  else launch_pdl(layer_error_chunk_kernel<false, LayerTable>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status, counters, err, K, order, keep);
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  const cudaError_t e = dq ? launch_chunks<true>(tab, c, partial, status, counters, err, K, order, keep, s, true)
+                           : launch_chunks<false>(tab, c, partial, status, counters, err, K, order, keep, s, true);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
@@ -400,13 +381,8 @@ qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_p
   if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
   double2* partial = reinterpret_cast<double2*>(static_cast<char*>(ws) + kReservedBytes);
   int* counters = reinterpret_cast<int*>(static_cast<char*>(ws) + kStatusBytes);
-  cudaError_t e;
-  if (dq)
-    e = launch_pdl(layer_error_chunk_kernel<true, FusedTable>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status,
-                   counters, err, K, order, keep);
-  else
-    e = launch_pdl(layer_error_chunk_kernel<false, FusedTable>, dim3(unsigned(c)), dim3(256), 0, s, tab, partial,
-                   status, counters, err, K, order, keep);
+  const cudaError_t e = dq ? launch_chunks<true>(tab, c, partial, status, counters, err, K, order, keep, s, true)
+                           : launch_chunks<false>(tab, c, partial, status, counters, err, K, order, keep, s, true);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
@@ -425,12 +401,12 @@ qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_p
 constexpr int64_t kNoAllocMaxChunks = int64_t(1) << 20;
 static __device__ __align__(256) double2 g_noalloc_partials[kNoAllocMaxChunks];
 
-__global__ void __launch_bounds__(256) layer_error_finish_table_kernel(const double2* __restrict__ partial,
+__global__ void __launch_bounds__(32) layer_error_finish_table_kernel(const double2* __restrict__ partial,
                                                                        const __grid_constant__ LayerTable tab,
                                                                        double* __restrict__ err) {
   const int l = blockIdx.x;
   if (l >= tab.n_layers) return;
-  finish_layer(partial, tab.first_chunk[l], tab.first_chunk[l + 1], err + l);
+  finish_layer_warp(partial, tab.first_chunk[l], tab.first_chunk[l + 1], err + l);
 }
 
 namespace {
@@ -472,10 +448,10 @@ qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const
     c += chunks_of(numel[i]);
   }
   tab.first_chunk[n_layers] = c;
-  if (dq) layer_error_chunk_kernel<true, LayerTable><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr, nullptr, err, K, order, keep);
-  else layer_error_chunk_kernel<false, LayerTable><<<unsigned(c), 256, 0, s>>>(tab, partial, nullptr, nullptr, err, K, order, keep);
-  if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
-  layer_error_finish_table_kernel<<<n_layers, 256, 0, s>>>(partial, tab, err);
+  const cudaError_t e = dq ? launch_chunks<true>(tab, c, partial, nullptr, nullptr, err, K, order, keep, s, false)
+                           : launch_chunks<false>(tab, c, partial, nullptr, nullptr, err, K, order, keep, s, false);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  layer_error_finish_table_kernel<<<n_layers, 32, 0, s>>>(partial, tab, err);
   rank_topk_kernel<<<1, 1024, 0, s>>>(err, n_layers, K, order, keep);
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }

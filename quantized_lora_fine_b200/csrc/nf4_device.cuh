@@ -18,103 +18,6 @@ __device__ __forceinline__ uint32_t nf4_index(float n) {
   return idx;
 }
 
-// Shared-memory copy of the cell tables (64 thresholds + 64 base indices).
-struct NF4CellSmem {
-  float thr[64];
-  uint32_t base[64];
-};
-
-__device__ __forceinline__ void nf4_cells_load(NF4CellSmem& t, int tid) {
-  if (tid < 64) {
-    t.thr[tid] = __uint_as_float(kNF4CellThrBits[tid]);
-    t.base[tid] = kNF4CellBase[tid];
-  }
-}
-
-// Same result as nf4_index(n) for every fp32 n (NaN maps to some index; callers
-// flag non-finite input separately): the cell of n holds at most one midpoint.
-__device__ __forceinline__ uint32_t nf4_index_cell(float n, const NF4CellSmem& t) {
-  const uint32_t c = (__float_as_uint(__fadd_rn(n, 3.0f)) >> 18) & 63u;
-  return t.base[c] + ((n > t.thr[c]) ? 1u : 0u);
-}
-
-// Correctly rounded w / a from r = RN(1/a) with one residual correction
-// (Markstein's division step: q0 = RN(w r), e = w - q0 a exactly by FMA,
-// q = RN(q0 + e r)). Requires a normal, finite a with 1/a normal; the callers
-// rescale tiny blocks by 2^64 first. Checked against IEEE division for every
-// (bf16 w, bf16 a) significand / exponent-gap combination by the GPU tests.
-__device__ __forceinline__ float div_by_recip(float w, float a, float r) {
-  const float q0 = __fmul_rn(w, r);
-  const float e = __fmaf_rn(-q0, a, w);
-  return __fmaf_rn(e, r, q0);
-}
-
-// Normalised value n = RN(w / a) for a block with absmax a > 0. bf16 inputs take
-// the reciprocal path (exact for every bf16 pair, see div_by_recip); fp32 inputs
-// use IEEE division directly.
-template <typename T>
-struct BlockDiv {
-  float a, r;
-  __device__ __forceinline__ BlockDiv(float am) {
-    // Tiny blocks: rescale by 2^64 (exact) so that 1/a stays a normal number.
-    a = (am < 0x1p-100f) ? am * 0x1p64f : am;
-    r = __frcp_rn(a);
-  }
-  __device__ __forceinline__ float operator()(float w, float am) const {
-    if constexpr (sizeof(T) == 2) {
-      return div_by_recip((am < 0x1p-100f) ? w * 0x1p64f : w, a, r);
-    } else {
-      return __fdiv_rn(w, am);
-    }
-  }
-};
-
-// bf16 bit pattern of max |w| over 8 elements held as 4 packed bf16 pairs.
-// Comparing magnitudes as unsigned integers orders +Inf and NaN above every
-// finite value, so a result >= 0x7F80 flags a non-finite element.
-__device__ __forceinline__ uint32_t absmax8_bf16_bits(uint4 v) {
-  const uint32_t a = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
-  const uint32_t b = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
-  const uint32_t m = __vmaxu2(a, b);
-  return max(m >> 16, m & 0xFFFFu);
-}
-
-// Max over the 8 lanes (l ^ 1, l ^ 2, l ^ 4) that share one 64-element block.
-__device__ __forceinline__ uint32_t block_max8_lanes(uint32_t v) {
-  v = max(v, __shfl_xor_sync(0xffffffffu, v, 1));
-  v = max(v, __shfl_xor_sync(0xffffffffu, v, 2));
-  v = max(v, __shfl_xor_sync(0xffffffffu, v, 4));
-  return v;
-}
-
-// Codes of 8 bf16 weights (4 packed pairs) of a block with absmax a > 0, packed in
-// storage order (byte k = idx[2k] << 4 | idx[2k + 1]).
-__device__ __forceinline__ uint32_t quant8_bf16(uint4 v, float a, const NF4CellSmem& cells, uint32_t (&idx)[8]) {
-  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-  float w[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) { w[2 * i] = __uint_as_float(u[i] << 16); w[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u); }
-  float as = a;
-  if (a < 0x1p-100f) {  // tiny block: rescale by 2^64 (exact) so that 1/a stays normal
-    as = a * 0x1p64f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] *= 0x1p64f;
-  }
-  const float r = __frcp_rn(as);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) idx[i] = nf4_index_cell(div_by_recip(w[i], as, r), cells);
-  // byte k = idx[2k] << 4 | idx[2k+1]; integer multiply-adds keep this off the ALU pipe
-  uint32_t word = idx[1];
-  word = idx[0] * 16u + word;
-  word = idx[3] * 256u + word;
-  word = idx[2] * 4096u + word;
-  word = idx[5] * 65536u + word;
-  word = idx[4] * 1048576u + word;
-  word = idx[7] * 16777216u + word;
-  word = idx[6] * 268435456u + word;
-  return word;
-}
-
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -134,6 +37,15 @@ __device__ __forceinline__ uint32_t bitselect(uint32_t a, uint32_t b, uint32_t m
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// max(|a|, |b|) per bf16 lane (the sign bit holds the xor of the operands' signs);
+// a NaN operand gives NaN, so the masked magnitude of a chain flags any NaN or Inf
+// by being >= 0x7F80.
+__device__ __forceinline__ uint32_t bf16x2_maxabs(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
 // ---- packed fp32 pairs (sm_100 f32x2 arithmetic: two IEEE fp32 operations in one
@@ -165,64 +77,109 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   return d;
 }
 
-// RN(w / a) for both elements of a pair, from r = RN(1/a) and na = -a (Markstein
-// step, as div_by_recip).
-__device__ __forceinline__ uint64_t f2_div_by_recip(uint64_t w, uint64_t na, uint64_t r) {
-  const uint64_t q0 = f2_mul(w, r);
-  const uint64_t e = f2_fma(q0, na, w);
-  return f2_fma(e, r, q0);
+// ---- code index of a normalised value: FMA-pipe arithmetic and warp shuffles
+// A block with absmax a is processed with a power-of-two scale sc (1, or 2^64 /
+// 2^-64 for tiny / huge blocks) so that r = RN(1/(a sc)) is a normal number; a
+// weight's scaled quotient is n_s = RN(w r) = n~ / sc with n~ = RN(w RN(1/a)).
+// Cell c = floor(15.75 n~ + 16) in [0, 31] of both elements of a pair: the low 5
+// bits of RZ(n_s (15.75 sc) + 2^23 + 16).
+__device__ __forceinline__ uint64_t cells2(uint64_t ns2, uint64_t cmul2) {
+  uint64_t v;
+  asm("fma.rz.f32x2 %0, %1, %2, %3;" : "=l"(v) : "l"(ns2), "l"(cmul2), "l"(0x4B0000104B000010ull));
+  return v;
 }
-
-// ---- fine-cell code lookup, evaluated on the FMA pipe
-// Cell c = bits(n) >> 21 (2048 cells of 1/4 binade; each holds at most one
-// midpoint). s = sat(n * 2^100 + T_c) is exactly 1.0 when n is above the cell's
-// midpoint and 0.0 otherwise; the code index is base_c + s.
 __device__ __forceinline__ float sat_fma(float a, float b, float c) {
   float d;
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-__device__ __forceinline__ float2 fine_q_entry(const float2* tbl, float n) {
-  return tbl[__float_as_uint(n) >> 21];
+// This lane's entries of the lookup tables: lane l holds B[l] (cell l), T[l]
+// (midpoint l) and code[l mod 16].
+struct LaneTables {
+  float B, T, code;
+};
+__device__ __forceinline__ LaneTables lane_tables(int lane) {
+  LaneTables t;
+  t.B = __uint_as_float(kNF4LaneB[lane]);
+  t.T = __uint_as_float(kNF4LaneT[lane]);
+  t.code = __uint_as_float(kNF4CodeBits[lane & 15]);
+  return t;
 }
-// Coarse cell c = floor(16 (n + 1)) for n in [-1, 1], as a shared-memory address
-// without integer ALU work: bits(RZ(16 n + 16 + 2^23)) = 0x4B000000 + c, and one
-// integer multiply-add (mod 2^32) turns that into tbl + c * entry_bytes.
-template <uint32_t kEntryBytes>
-__device__ __forceinline__ uint32_t coarse_addr(float n, uint32_t tbl) {
-  float v;
-  asm("fma.rz.f32 %0, %1, 0f41800000, 0f4B000010;" : "=f"(v) : "f"(n));   // 16 n + (2^23 + 16)
-  return __float_as_uint(v) * kEntryBytes + (tbl - 0x4B000000u * kEntryBytes);
+// Index bits 0x4B000000 + idx of one element from its scaled quotient and cell bits:
+// b = B[cell], t = T[base] by shuffles (a shuffle uses the low 5 bits of its lane
+// operand), s = sat(n_s M + t) in {0, 1} with M = 2^36 sc, bits(b + s). Every lane of
+// the warp must call it.
+__device__ __forceinline__ uint32_t index_bits(float ns, uint32_t cell_bits, float M, const LaneTables& lt) {
+  const float b = __shfl_sync(0xffffffffu, lt.B, int(cell_bits));
+  const float t = __shfl_sync(0xffffffffu, lt.T, int(__float_as_uint(b)));
+  return __float_as_uint(b + sat_fma(ns, M, t));
 }
-// Both cells of a packed pair: bits of RZ(16 n + 16 + 2^23) per lane.
-__device__ __forceinline__ uint64_t coarse_cells2(uint64_t n2) {
-  uint64_t v;
-  asm("fma.rz.f32x2 %0, %1, %2, %3;" : "=l"(v) : "l"(n2), "l"(0x4180000041800000ull), "l"(0x4B0000104B000010ull));
-  return v;
+// Code value of index bits x (lane x mod 32 holds code[x mod 16]).
+__device__ __forceinline__ float code_value(uint32_t x, const LaneTables& lt) {
+  return __shfl_sync(0xffffffffu, lt.code, int(x));
 }
-template <uint32_t kEntryBytes>
-__device__ __forceinline__ uint32_t coarse_addr_bits(uint32_t cell_bits, uint32_t tbl) {
-  return cell_bits * kEntryBytes + (tbl - 0x4B000000u * kEntryBytes);
+// Per-block constants of the lookup: r = RN(1/(a sc)) and the two multipliers.
+struct CellScale {
+  uint64_t r2, cmul2;
+  float M;
+  __device__ __forceinline__ explicit CellScale(float a) {
+    const float sc = (a < 0x1p-100f) ? 0x1p64f : (a > 0x1p100f) ? 0x1p-64f : 1.f;
+    r2 = f2_splat(__frcp_rn(a * sc));
+    cmul2 = f2_splat(15.75f * sc);
+    M = 0x1p36f * sc;
+  }
+};
+// The 8 elements of a piece (4 packed bf16 pairs, storage order) -> index bits x[k].
+// Every lane of the warp must call it.
+__device__ __forceinline__ void piece_index_bits(const uint32_t (&u)[4], const CellScale& cs, const LaneTables& lt,
+                                                 uint32_t (&x)[8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint64_t q = f2_mul(f2_from_bf16x2(u[i]), cs.r2);
+    const uint64_t c = cells2(q, cs.cmul2);
+    x[2 * i] = index_bits(f2_lo(q), uint32_t(c), cs.M, lt);
+    x[2 * i + 1] = index_bits(f2_hi(q), uint32_t(c >> 32), cs.M, lt);
+  }
 }
-__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
+// {bf16 lo(h) - a.x, bf16 hi(h) - a.y} in fp32: the bf16 halves enter exactly
+// (mixed-precision subtraction), one rounding each.
+__device__ __forceinline__ uint64_t f2_bf16x2_minus(uint32_t h, uint64_t a) {
+  uint64_t d;
+  asm("{\n\t.reg .b16 l, u;\n\t.reg .f32 a0, a1, d0, d1;\n\t"
+      "mov.b32 {l, u}, %1;\n\tmov.b64 {a0, a1}, %2;\n\t"
+      "sub.rn.f32.bf16 d0, l, a0;\n\tsub.rn.f32.bf16 d1, u, a1;\n\t"
+      "mov.b64 %0, {d0, d1};\n\t}"
+      : "=l"(d) : "r"(h), "l"(a));
+  return d;
 }
-__device__ __forceinline__ float lds_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
+// Undo a thread's piece rotation: word j was computed for position j ^ rot; after
+// this, w[p] holds position p (three conditional exchange stages, one per bit).
+__device__ __forceinline__ void unrotate8(uint32_t (&w)[8], uint32_t rot) {
+#pragma unroll
+  for (int b = 0; b < 3; ++b) {
+    const bool sw = (rot >> b) & 1u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i & (1 << b)) continue;
+      const uint32_t x = w[i], y = w[i | (1 << b)];
+      w[i] = sw ? y : x;
+      w[i | (1 << b)] = sw ? x : y;
+    }
+  }
 }
-__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-  return v;
-}
-// Four code indices accumulated as sum idx_p * 16^p in fp32 (exact below 2^16)
-// turn into integer bits through the 2^23 bias: low 16 bits of bits(h + 2^23).
-__device__ __forceinline__ uint32_t nibbles_from_f32(float h) {
-  return __float_as_uint(__fadd_rn(h, 8388608.0f));
+// Code word of a piece (byte k = idx[2k] << 4 | idx[2k + 1]) from its index bits by a
+// multiply-add chain mod 2^32: the 0x4B000000 of each term survives only from the
+// last two terms (0x4B000000 + 0xB0000000), which the final add cancels.
+__device__ __forceinline__ uint32_t pack_code_word(const uint32_t (&x)[8]) {
+  uint32_t acc = x[6];
+  acc = acc * 16u + x[7];
+  acc = acc * 16u + x[4];
+  acc = acc * 16u + x[5];
+  acc = acc * 16u + x[2];
+  acc = acc * 16u + x[3];
+  acc = acc * 16u + x[0];
+  acc = acc * 16u + x[1];
+  return acc + 0x05000000u;
 }
 
 // Per-block dequantization table: the 16 products bf16_rn(fp32_rn(c_j * a)) split

@@ -96,11 +96,13 @@ def _exhaustive_blocks(exp: int, sigs) -> np.ndarray:
     return np.concatenate(blocks)
 
 
-@pytest.mark.parametrize("exp,sigs", [(0, range(128)), (-120, range(0, 128, 9)), (100, range(0, 128, 13))])
+@pytest.mark.parametrize("exp,sigs", [(0, range(128)), (-120, range(0, 128, 9)), (-126, range(0, 128, 17)),
+                                      (100, range(0, 128, 13)), (127, range(0, 128, 11))])
 def test_quant_every_bf16_pair(cuda_device, exp, sigs):
     """Every (bf16 w, bf16 absmax) significand pair and exponent gap: the GPU's
-    reciprocal-based division and cell-table code lookup give the oracle's codes
-    (IEEE division, 15 midpoint comparisons)."""
+    reciprocal-based quotient and cell-table code lookup give the oracle's codes
+    (IEEE division, 15 midpoint comparisons); tiny (2^-126, 2^-120) and huge
+    (2^100, 2^127) absmax take the rescaled path."""
     W32 = _exhaustive_blocks(exp, sigs)
     Wb = synth.from_bf16_bits(nf4.bf16_bits_from_f32(W32))
     _check_quant(Wb, dq=False)
