@@ -45,35 +45,42 @@ def lane_cell(n, sc=1.0):
     return int(v) - 2 ** 23
 
 
-def lane_tables(mids):
-    """Per lane l = cell l (32 cells of width 1/15.75; the midpoints lie at least
-    0.08 apart, so a cell holds at most one): B[l] = 2^23 + base (fp32), base = the
-    number of midpoints below every value of the cell. Per lane j: T[j] = -m_j 2^36
-    for j < 15, else -2^38 (below every n 2^36). A value n of cell c then has code
-    index base + [n > m_base]: m_base is the only midpoint that can lie in the cell."""
+def lane_tables(codes, mids):
+    """Per lane l = cell l (32 cells of width 1/15.75; the midpoints lie at least 0.08
+    apart, so a cell holds at most one), with base = the number of midpoints below
+    every value of the cell: B[l] = 2^23 + base (fp32); T[l] = -m_base 2^36 if
+    base < 15, else -2^38 (below every n 2^36); LO[l] = code[base]; D[l] =
+    code[base + 1] - code[base] (exact in fp32), 0 if base = 15. A value n of the
+    cell has code index base + s with s = [n > m_base]: m_base is the only midpoint
+    that can lie in the cell (the one below it lies below the cell, the one above it
+    above the cell). Its code value is LO + s D."""
     cells = [lane_cell(float(m)) for m in mids]
     assert len(set(cells)) == len(cells), "a cell holds two midpoints"
-    B = []
+    B, T, LO, D = [], [], [], []
     for c in range(32):
         lo = fractions.Fraction(c - 16) / fractions.Fraction(CELL_MUL)   # smallest value of the cell
         base = sum(1 for m in mids if fractions.Fraction(float(m)) < lo)
         B.append(int(np.float32(base + 2 ** 23).view(np.uint32)))
-    T = []
-    for j in range(32):
-        t = -float(mids[j]) * 2.0 ** 36 if j < 15 else -(2.0 ** 38)
+        t = -float(mids[base]) * 2.0 ** 36 if base < 15 else -(2.0 ** 38)
         assert float(np.float32(t)) == t   # exact
         T.append(int(np.float32(t).view(np.uint32)))
-    return B, T
+        c_lo = np.float32(codes[base])
+        d = np.float32(codes[base + 1] - c_lo) if base < 15 else np.float32(0)
+        if base < 15:
+            assert float(d) == float(codes[base + 1]) - float(c_lo)   # exact difference
+        LO.append(int(c_lo.view(np.uint32)))
+        D.append(int(d.view(np.uint32)))
+    return B, T, LO, D
 
 
-def check_lane_tables(codes, mids, B, T, rng=np.random.default_rng(2)):
+def check_lane_tables(codes, mids, B, T, LO, D, rng=np.random.default_rng(2)):
     """Brute force against #{j : n > m_j}, for the three block scalings the kernels
     use (sc = 1, 2^64 for tiny blocks, 2^-64 for huge ones): the kernel holds
-    n_s = n / sc, reads b = B[cell] and t = T[bits(b) mod 32] (warp shuffles by lane
-    index; only the low 5 bits of the lane operand count), s = sat(n_s (2^36 sc) + t),
-    and takes the index from the low bits of bits(b + s). The code value is then
-    code[index] (lane index & 15). Below |n| = 2^-62 the scaled n_s of a tiny block
-    is subnormal and must still give the zero code."""
+    n_s = n / sc, reads b = B[cell], t = T[cell] (warp shuffles by lane index; only
+    the low 5 bits of the lane operand count), s = sat(n_s (2^36 sc) + t), takes the
+    index from the low bits of bits(b + s) and the code value as code[index] (lane
+    index & 15) or LO[cell] + s D[cell] (one rounding, an FMA). Below |n| = 2^-62 the
+    scaled n_s of a tiny block is subnormal and must still give the zero code."""
     f = lambda bits: float(np.uint32(bits).view(np.float32))
     tests = [np.float32(x) for x in (0.0, -0.0, 1.0, -1.0)]
     for m in mids:
@@ -93,10 +100,9 @@ def check_lane_tables(codes, mids, B, T, rng=np.random.default_rng(2)):
                 assert ref == ZERO_CODE, float(n)    # the kernel's subnormal n_s: |n| < 2^-62
                 ns = fractions.Fraction(0)
             v = ns * fractions.Fraction(CELL_MUL) * fractions.Fraction(sc) + 16 + 2 ** 23
-            c = (int(v) - 2 ** 23) & 31
             assert 0 <= int(v) - 2 ** 23 <= 31
-            b = f(B[c])
-            t = f(T[int(np.float32(b).view(np.uint32)) & 31])
+            c = (int(v) - 2 ** 23) & 31
+            b, t = f(B[c]), f(T[c])
             w = ns * fractions.Fraction(2) ** 36 * fractions.Fraction(sc) + fractions.Fraction(t)
             w = float(np.float32(float(w))) if w != 0 else 0.0      # one rounding (FMA)
             s = min(max(w, 0.0), 1.0)
@@ -104,12 +110,14 @@ def check_lane_tables(codes, mids, B, T, rng=np.random.default_rng(2)):
             x = int(np.float32(b + s).view(np.uint32))
             assert x - 0x4B000000 == ref, (float(n), sc, c, x, ref)
             assert codes[x & 15] == codes[ref]
+            val = np.float32(fractions.Fraction(s) * fractions.Fraction(f(D[c])) + fractions.Fraction(f(LO[c])))
+            assert val == codes[ref], (float(n), sc, c)
 
 
 def render():
     codes, mids = constants()
-    B, T = lane_tables(mids)
-    check_lane_tables(codes, mids, B, T)
+    B, T, LO, D = lane_tables(codes, mids)
+    check_lane_tables(codes, mids, B, T, LO, D)
     cb = [int(v) for v in codes.view(np.uint32)]
     mb = [int(v) for v in mids.view(np.uint32)]
     lines = [
@@ -123,15 +131,20 @@ def render():
         "__device__ constexpr uint32_t kNF4MidBits[15] = {",
         "    " + ", ".join("0x%08Xu" % b for b in mb) + "};",
         "// values, for reading: " + ", ".join("%.9g" % v for v in codes),
-        "// Lane tables for the warp-shuffle code lookup. Cell c = floor(15.75 n + 16) in",
-        "// [0, 31] (the low bits of RZ(15.75 n + 2^23 + 16)). kNF4LaneB[c] = 2^23 + base_c",
-        "// (fp32 bits), base_c = the number of midpoints below the cell; kNF4LaneT[j] =",
-        "// -m_j 2^36 (j < 15), else -2^38. s = sat(n 2^36 + T[base_c]) and",
-        "// bits(B[c] + s) = 0x4B000000 + code index.",
+        "// Lane tables for the warp-shuffle code lookup: lane c = cell c = floor(15.75 n + 16)",
+        "// in [0, 31] (the low bits of RZ(15.75 n + 2^23 + 16)), base_c = the number of",
+        "// midpoints below the cell. kNF4LaneB[c] = 2^23 + base_c; kNF4LaneT[c] = -m_base 2^36",
+        "// (-2^38 if base_c = 15); kNF4LaneLo[c] = code[base_c]; kNF4LaneD[c] = code[base_c + 1]",
+        "// - code[base_c] (exact; 0 if base_c = 15). With s = sat(n 2^36 + T[c]):",
+        "// bits(B[c] + s) = 0x4B000000 + code index, and the code value is Lo[c] + s D[c].",
         "__device__ constexpr uint32_t kNF4LaneB[32] = {",
         "    " + ", ".join("0x%08Xu" % v for v in B) + "};",
         "__device__ constexpr uint32_t kNF4LaneT[32] = {",
         "    " + ", ".join("0x%08Xu" % v for v in T) + "};",
+        "__device__ constexpr uint32_t kNF4LaneLo[32] = {",
+        "    " + ", ".join("0x%08Xu" % v for v in LO) + "};",
+        "__device__ constexpr uint32_t kNF4LaneD[32] = {",
+        "    " + ", ".join("0x%08Xu" % v for v in D) + "};",
         "}  // namespace qlb",
         "",
     ]

@@ -3,12 +3,12 @@
 //
 // Pass 1: one CTA per chunk of 256 blocks (16384 elements) of some layer;
 //         quantizes, dequantizes and accumulates sum (w - w_hat)^2 and sum w^2
-//         in fp64; writes one partial pair per chunk.
-// Pass 2: per layer, sums its chunk partials in chunk order -> err.
+//         in fp64; writes one partial pair per chunk (the fused entry also
+//         writes the codes and scales).
+// Pass 2: one warp per layer sums its chunk partials in chunk order -> err.
 // Pass 3: one CTA ranks all layers by (err desc, id asc).
-// The workspace entry point runs all three in one launch (the last chunk CTA of a
-// layer does pass 2 for it, the last layer's finisher does pass 3); the
-// allocation-free entry point, which has no counters, launches them separately.
+// The three kernels follow each other on the stream with programmatic dependent
+// launch: each waits for its predecessor's memory before reading it.
 #include <cfloat>
 #include <cuda_bf16.h>
 
@@ -46,8 +46,12 @@ struct FusedTable {
 };
 static_assert(sizeof(FusedTable) <= 32000, "kernel parameter limit");
 
-__device__ __forceinline__ void finish_layer_warp(const double2* __restrict__ partial, int c0, int c1,
-                                                  double* __restrict__ err_out);
+// Chunk ranges of the layers, for the finish pass (a by-value kernel parameter).
+struct ChunkRanges {
+  int32_t first_chunk[kMaxLayers + 1];
+  int32_t n_layers;
+};
+
 
 // Chunk c of the table: its layer (binary search over first_chunk), index within
 // the layer and number of blocks.
@@ -69,35 +73,30 @@ struct ChunkRef {
   }
 };
 
-// Pass 1 (and, with counters, passes 2-3 fused): one CTA per chunk of 256 blocks
+// Pass 1: one CTA per chunk of 256 blocks
 // (16384 weights, the double-quant group) of some layer; thread t owns block t. The
 // chunk's bf16 weights reach shared memory by one bulk copy; thread t reads its
 // block as eight 16-byte pieces, piece j ^ (t mod 8) at step j (the 8 lanes of a
 // quarter warp touch 8 different bank groups). Per block: absmax over packed bf16
 // pairs; with double quant the chunk's max G of the absmax values gives the
 // reconstruction scale ahat = e4m3(a 448 / G) G / 448 (the codes use the exact a).
-// Per element: the code index from the one-multiply quotient and the shuffle
-// lookup (as the quantizer), the code value by one more warp shuffle from the lane
-// that holds it (lane l holds code[l mod 16]; the index bits select the lane),
+// Per element: the code index from the one-multiply quotient and the shuffle lookup
+// (as the quantizer), the code value by one more warp shuffle from the lane that
+// holds it (lane l holds code[l mod 16]; the index bits select the lane),
 // w_hat = bf16(fp32(code ahat)), and (w_hat - w)^2 (a mixed bf16 - fp32
 // subtraction), w^2 summed in packed fp32 (16 terms per accumulator) before the
 // fp64 chunk total. With Tab::kWrite (the fused pass) the thread's 8 code words go
 // back in order and out in two 16-byte stores, with the scales. Warp 0 sums the
-// 256 per-thread totals in a fixed order into partial[chunk]; with counters (zero
-// on entry, left zero) it also finishes: the chunk that completes a layer sums
-// that layer's partials in chunk order into err[layer], and the one that
-// completes the last layer ranks all layers and writes order / keep. The other
-// warps leave as soon as their totals are in shared memory.
+// 256 per-thread totals in a fixed order into partial[chunk]; the other warps
+// leave as soon as their totals are in shared memory.
 template <bool DQ, class Tab>
 __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_constant__ Tab tab,
-                                                                   double2* __restrict__ partial, int* status,
-                                                                   int* counters, double* __restrict__ err, int K,
-                                                                   int32_t* __restrict__ order,
-                                                                   uint8_t* __restrict__ keep) {
+                                                                   double2* __restrict__ partial, int* status) {
   constexpr bool kW = Tab::kWrite;
   __shared__ __align__(128) uint32_t s_w[kChunkBytes / 4];
   __shared__ double2 s_part[256];
   __shared__ float s_red[8];
+  __shared__ int s_ref[3];
   __shared__ __align__(8) uint64_t s_bar;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t bar = smem_u32(&s_bar);
@@ -107,10 +106,15 @@ __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_
   }
   const LaneTables lt = lane_tables(lane);
   const int64_t chunk = blockIdx.x;
-  const ChunkRef<Tab> cr(tab, chunk);
-  const int layer = cr.layer, nblk = cr.nblk;
-  const int64_t g = cr.g;
-  __syncthreads();   // barrier in place
+  if (tid == 0) {   // the chunk's layer, by one thread
+    const ChunkRef<Tab> cr(tab, chunk);
+    s_ref[0] = cr.layer;
+    s_ref[1] = cr.nblk;
+    s_ref[2] = int(cr.g);
+  }
+  __syncthreads();   // barrier and chunk reference in place
+  const int layer = s_ref[0], nblk = s_ref[1];
+  const int64_t g = s_ref[2];
   pdl_wait();
   pdl_launch();
   if (tid == 0) {
@@ -218,7 +222,7 @@ __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_
   s_part[tid] = make_double2(sd, sw);
   __syncthreads();
   if (warp != 0) return;
-  // ---- warp 0: the chunk total in a fixed order, then the fused finish
+  // ---- warp 0: the chunk total in a fixed order
   double a = 0.0, b = 0.0;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -232,41 +236,6 @@ __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_
     b += __shfl_xor_sync(0xffffffffu, b, o);
   }
   if (lane == 0) partial[chunk] = make_double2(a, b);
-  if (counters == nullptr) return;
-  int last = 0;
-  if (lane == 0) {
-    __threadfence();
-    const int nchunks_l = tab.first_chunk[layer + 1] - tab.first_chunk[layer];
-    const int done = atomicAdd(counters + 1 + layer, 1);
-    last = (done == nchunks_l - 1);
-    if (last) atomicExch(counters + 1 + layer, 0);
-  }
-  if (!__shfl_sync(0xffffffffu, last, 0)) return;
-  __threadfence();
-  finish_layer_warp(partial, tab.first_chunk[layer], tab.first_chunk[layer + 1], err + layer);
-  if (lane == 0) {
-    __threadfence();
-    const int done = atomicAdd(counters, 1);
-    last = (done == tab.n_layers - 1);
-    if (last) atomicExch(counters, 0);
-  }
-  if (!__shfl_sync(0xffffffffu, last, 0)) return;
-  __threadfence();
-  // rank all layers (err desc, id asc); the errors are staged in the chunk buffer
-  const int n = tab.n_layers;
-  double* s_err = reinterpret_cast<double*>(s_w);
-  for (int l = lane; l < n; l += 32) s_err[l] = __ldcg(err + l);
-  __syncwarp();
-  for (int l = lane; l < n; l += 32) {
-    const double e = s_err[l];
-    int rank = 0;
-    for (int j = 0; j < n; ++j) {
-      const double f = s_err[j];
-      rank += (f > e || (f == e && j < l)) ? 1 : 0;
-    }
-    order[rank] = l;
-    keep[l] = rank < K ? 1 : 0;
-  }
 }
 
 // One warp per layer: lane l sums chunks first+l, first+l+32, ... in order; the 32
@@ -291,6 +260,8 @@ __device__ __forceinline__ void finish_layer_warp(const double2* __restrict__ pa
 
 __global__ void __launch_bounds__(1024) rank_topk_kernel(const double* __restrict__ err, int n_layers, int K,
                                                          int32_t* __restrict__ order, uint8_t* __restrict__ keep) {
+  pdl_wait();
+  pdl_launch();
   __shared__ double s_err[kMaxLayers];
   for (int i = threadIdx.x; i < n_layers; i += blockDim.x) s_err[i] = err[i];
   __syncthreads();
@@ -306,9 +277,16 @@ __global__ void __launch_bounds__(1024) rank_topk_kernel(const double* __restric
   }
 }
 
-__global__ void __launch_bounds__(32) layer_error_finish_table_kernel(const double2* __restrict__ partial,
-                                                                       const __grid_constant__ LayerTable tab,
-                                                                       double* __restrict__ err);
+// Pass 2: one warp per layer.
+__global__ void __launch_bounds__(32) layer_error_finish_kernel(const double2* __restrict__ partial,
+                                                                const __grid_constant__ ChunkRanges r,
+                                                                double* __restrict__ err) {
+  pdl_wait();
+  pdl_launch();
+  const int l = blockIdx.x;
+  if (l >= r.n_layers) return;
+  finish_layer_warp(partial, r.first_chunk[l], r.first_chunk[l + 1], err + l);
+}
 
 static int32_t chunks_of(int64_t numel) {
   const int64_t nb = numel / kBlock;
@@ -321,15 +299,31 @@ size_t layer_error_ws_bytes(int n_layers, const int64_t* numel) {
   return kReservedBytes + size_t(chunks) * sizeof(double2);
 }
 
-// Launch of the chunk kernel over c chunks.
+// The three passes on stream s. tab.first_chunk / n_layers are filled in; the chunk
+// and rank kernels need nothing else from the host. With pdl, each kernel may start
+// while its predecessor drains (the allocation-free entry launches plainly).
 template <bool DQ, class Tab>
-static cudaError_t launch_chunks(const Tab& tab, int64_t c, double2* partial, int* status, int* counters,
-                                 double* err, int K, int32_t* order, uint8_t* keep, cudaStream_t s, bool pdl) {
-  auto kern = layer_error_chunk_kernel<DQ, Tab>;
-  if (pdl)
-    return launch_pdl(kern, dim3(unsigned(c)), dim3(256), 0, s, tab, partial, status, counters, err, K, order, keep);
-  kern<<<unsigned(c), 256, 0, s>>>(tab, partial, status, counters, err, K, order, keep);
-  return cudaGetLastError();
+static qlora_status launch_passes(const Tab& tab, double2* partial, int* status, double* err, int K,
+                                  int32_t* order, uint8_t* keep, cudaStream_t s, bool pdl) {
+  static std::mutex mu;
+  static ChunkRanges r;   // host staging of the by-value parameter
+  std::lock_guard<std::mutex> lock(mu);
+  const int n = tab.n_layers;
+  r.n_layers = n;
+  for (int i = 0; i <= n; ++i) r.first_chunk[i] = tab.first_chunk[i];
+  const unsigned c = unsigned(tab.first_chunk[n]);
+  cudaError_t e;
+  if (pdl) {
+    e = launch_pdl(layer_error_chunk_kernel<DQ, Tab>, dim3(c), dim3(256), 0, s, tab, partial, status);
+    if (e == cudaSuccess) e = launch_pdl(layer_error_finish_kernel, dim3(unsigned(n)), dim3(32), 0, s, partial, r, err);
+    if (e == cudaSuccess) e = launch_pdl(rank_topk_kernel, dim3(1), dim3(1024), 0, s, err, n, K, order, keep);
+  } else {
+    layer_error_chunk_kernel<DQ, Tab><<<c, 256, 0, s>>>(tab, partial, status);
+    layer_error_finish_kernel<<<unsigned(n), 32, 0, s>>>(partial, r, err);
+    rank_topk_kernel<<<1, 1024, 0, s>>>(err, n, K, order, keep);
+    e = cudaSuccess;
+  }
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
@@ -340,6 +334,7 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
   static std::mutex mu;
   static LayerTable tab;
   std::lock_guard<std::mutex> lock(mu);
+  if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
   tab.n_layers = n_layers;
   int32_t c = 0;
   for (int i = 0; i < n_layers; ++i) {
@@ -349,12 +344,9 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
     c += chunks_of(numel[i]);
   }
   tab.first_chunk[n_layers] = c;
-  if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
   double2* partial = reinterpret_cast<double2*>(static_cast<char*>(ws) + kReservedBytes);
-  int* counters = reinterpret_cast<int*>(static_cast<char*>(ws) + kStatusBytes);   // 1 + n_layers, zero
-  const cudaError_t e = dq ? launch_chunks<true>(tab, c, partial, status, counters, err, K, order, keep, s, true)
-                           : launch_chunks<false>(tab, c, partial, status, counters, err, K, order, keep, s, true);
-  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
+  return dq ? launch_passes<true>(tab, partial, status, err, K, order, keep, s, true)
+            : launch_passes<false>(tab, partial, status, err, K, order, keep, s, true);
 }
 
 qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
@@ -365,6 +357,7 @@ qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_p
   static std::mutex mu;
   static FusedTable tab;
   std::lock_guard<std::mutex> lock(mu);
+  if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
   tab.n_layers = n_layers;
   int32_t c = 0;
   for (int i = 0; i < n_layers; ++i) {
@@ -378,21 +371,17 @@ qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_p
     c += chunks_of(numel[i]);
   }
   tab.first_chunk[n_layers] = c;
-  if (layer_error_ws_bytes(n_layers, numel) > ws_bytes) return QLORA_ERR_WORKSPACE;
   double2* partial = reinterpret_cast<double2*>(static_cast<char*>(ws) + kReservedBytes);
-  int* counters = reinterpret_cast<int*>(static_cast<char*>(ws) + kStatusBytes);
-  const cudaError_t e = dq ? launch_chunks<true>(tab, c, partial, status, counters, err, K, order, keep, s, true)
-                           : launch_chunks<false>(tab, c, partial, status, counters, err, K, order, keep, s, true);
-  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
+  return dq ? launch_passes<true>(tab, partial, status, err, K, order, keep, s, true)
+            : launch_passes<false>(tab, partial, status, err, K, order, keep, s, true);
 }
 
 // ------------------------------------------------------------------------
 // Allocation-free variant.
 //
 // Same three passes, but the per-chunk partial sums live in a file-scope device
-// array instead of a caller workspace, and the chunk table reaches the finish
-// pass as a kernel parameter, so a call needs no device memory beyond its
-// inputs and outputs. The array is 16 MiB (2^20 chunks of 16384 weights, i.e.
+// array instead of a caller workspace, so a call needs no device memory beyond
+// its inputs and outputs. The array is 16 MiB (2^20 chunks of 16384 weights, i.e.
 // up to 2^34 weights per call); every GPU that loads the library keeps it
 // until the process exits. All calls share it: calls that overlap on the GPU
 // (two streams, two host threads) race on it. Each call overwrites every
@@ -400,14 +389,6 @@ qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_p
 
 constexpr int64_t kNoAllocMaxChunks = int64_t(1) << 20;
 static __device__ __align__(256) double2 g_noalloc_partials[kNoAllocMaxChunks];
-
-__global__ void __launch_bounds__(32) layer_error_finish_table_kernel(const double2* __restrict__ partial,
-                                                                       const __grid_constant__ LayerTable tab,
-                                                                       double* __restrict__ err) {
-  const int l = blockIdx.x;
-  if (l >= tab.n_layers) return;
-  finish_layer_warp(partial, tab.first_chunk[l], tab.first_chunk[l + 1], err + l);
-}
 
 namespace {
 constexpr int kNoAllocMaxDevices = 64;
@@ -448,12 +429,8 @@ qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const
     c += chunks_of(numel[i]);
   }
   tab.first_chunk[n_layers] = c;
-  const cudaError_t e = dq ? launch_chunks<true>(tab, c, partial, nullptr, nullptr, err, K, order, keep, s, false)
-                           : launch_chunks<false>(tab, c, partial, nullptr, nullptr, err, K, order, keep, s, false);
-  if (e != cudaSuccess) return QLORA_ERR_CUDA;
-  layer_error_finish_table_kernel<<<n_layers, 32, 0, s>>>(partial, tab, err);
-  rank_topk_kernel<<<1, 1024, 0, s>>>(err, n_layers, K, order, keep);
-  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return dq ? launch_passes<true>(tab, partial, nullptr, err, K, order, keep, s, false)
+            : launch_passes<false>(tab, partial, nullptr, err, K, order, keep, s, false);
 }
 
 }  // namespace qlb

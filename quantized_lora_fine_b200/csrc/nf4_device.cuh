@@ -93,30 +93,40 @@ __device__ __forceinline__ float sat_fma(float a, float b, float c) {
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// This lane's entries of the lookup tables: lane l holds B[l] (cell l), T[l]
-// (midpoint l) and code[l mod 16].
+// This lane's entries of the lookup tables: lane l holds cell l's B, T, Lo, D and
+// code[l mod 16] (a kernel loads the ones it uses).
 struct LaneTables {
-  float B, T, code;
+  float B, T, lo, d, code;
 };
 __device__ __forceinline__ LaneTables lane_tables(int lane) {
   LaneTables t;
   t.B = __uint_as_float(kNF4LaneB[lane]);
   t.T = __uint_as_float(kNF4LaneT[lane]);
+  t.lo = __uint_as_float(kNF4LaneLo[lane]);
+  t.d = __uint_as_float(kNF4LaneD[lane]);
   t.code = __uint_as_float(kNF4CodeBits[lane & 15]);
   return t;
 }
 // Index bits 0x4B000000 + idx of one element from its scaled quotient and cell bits:
-// b = B[cell], t = T[base] by shuffles (a shuffle uses the low 5 bits of its lane
-// operand), s = sat(n_s M + t) in {0, 1} with M = 2^36 sc, bits(b + s). Every lane of
-// the warp must call it.
+// b = B[cell] and t = T[cell] by two independent shuffles (a shuffle uses the low 5
+// bits of its lane operand), s = sat(n_s M + t) in {0, 1} with M = 2^36 sc, bits(b + s).
+// Every lane of the warp must call it.
 __device__ __forceinline__ uint32_t index_bits(float ns, uint32_t cell_bits, float M, const LaneTables& lt) {
   const float b = __shfl_sync(0xffffffffu, lt.B, int(cell_bits));
-  const float t = __shfl_sync(0xffffffffu, lt.T, int(__float_as_uint(b)));
+  const float t = __shfl_sync(0xffffffffu, lt.T, int(cell_bits));
   return __float_as_uint(b + sat_fma(ns, M, t));
 }
 // Code value of index bits x (lane x mod 32 holds code[x mod 16]).
 __device__ __forceinline__ float code_value(uint32_t x, const LaneTables& lt) {
   return __shfl_sync(0xffffffffu, lt.code, int(x));
+}
+// Code value of one element straight from its cell: Lo + s D with s = sat(n_s M + T)
+// (three independent shuffles; exact). Every lane of the warp must call it.
+__device__ __forceinline__ float code_value_of_cell(float ns, uint32_t cell_bits, float M, const LaneTables& lt) {
+  const float t = __shfl_sync(0xffffffffu, lt.T, int(cell_bits));
+  const float lo = __shfl_sync(0xffffffffu, lt.lo, int(cell_bits));
+  const float d = __shfl_sync(0xffffffffu, lt.d, int(cell_bits));
+  return __fmaf_rn(sat_fma(ns, M, t), d, lo);
 }
 // Per-block constants of the lookup: r = RN(1/(a sc)) and the two multipliers.
 struct CellScale {
