@@ -262,6 +262,10 @@ def gpu_main(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     lib = _lib.load()
     peaks = load_peaks()
+    if args.hbm_only:   # the codec legs alone (profiling aid; not a bench line)
+        print(json.dumps({"hbm_legs": hbm_legs(api, synth, torch, dev, torch.cuda.current_stream(), peaks,
+                                                layers=args.hbm_layers)}), flush=True)
+        return
 
     M, h, o, r, alpha = args.M, 4096, 4096, 16, 32.0
     s = alpha / r
@@ -489,6 +493,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-hbm-legs", action="store_true", help="skip the full-stack quantizer / error-pass legs")
     ap.add_argument("--hbm-layers", type=int, default=32, help="decoder layers of the stack for those legs")
+    ap.add_argument("--hbm-only", action="store_true",
+                    help="run only the full-stack codec legs and print them (for profiler captures)")
     ap.add_argument("--eager", action="store_true", help="time eager API calls instead of CUDA-graph replays")
     args = ap.parse_args()
     if args.warmup < 3:
