@@ -170,6 +170,26 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t 
                               uint16_t* Y, uint16_t* T_save,
                               void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
+/* The forward in two parts, for callers that overlap T = X L1 with other work
+ * (e.g. the weight's quantization on another stream):
+ *   qlora_lora_down    T = X L1 (M x r, fp32 accumulation, rounded once to bf16),
+ *                      the LoRA down-projection of eq. (3) on its own. Shapes as for
+ *                      the linear (in % 256 == 0, r % 8 == 0, 8 <= r <= 256);
+ *                      workspace of qlora_lora_down_workspace_size bytes, zeroed
+ *                      once before first use (status word + split-K counters).
+ *                      X device bf16 [M x in], L1 device bf16 [in x r], T device out
+ *                      bf16 [M x r]; all 16-byte aligned.
+ *   qlora_linear_fwd_t Y = X W_s^T + s T L2 with T supplied (device bf16 [M x r],
+ *                      from qlora_lora_down or the caller); otherwise as
+ *                      qlora_linear_fwd (same workspace size). Gives the bits of
+ *                      qlora_linear_fwd when T is the same. */
+size_t qlora_lora_down_workspace_size(int64_t M, int64_t in, int32_t r);
+qlora_status qlora_lora_down(const uint16_t* X, int64_t M, int64_t in, const uint16_t* L1, int32_t r,
+                             uint16_t* T, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+qlora_status qlora_linear_fwd_t(const qlora_weight* w, const uint16_t* X, int64_t M, const uint16_t* T,
+                                const uint16_t* L2, int32_t r, float scale, uint16_t* Y,
+                                void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
 /* Backward of the forward above (no gradient for W):
  *   U   = dY L2^T                 (M x r, bf16 after fp32 accumulation)
  *   dX  = dY W_s + s U L1^T       (M x in, bf16)          -- skipped if dX == NULL

@@ -44,6 +44,10 @@ SIGNATURES = {
     "qlora_bwd_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int32]),
     "qlora_linear_fwd": (c_int, [POINTER(QLoraWeight), c_void_p, c_int64, c_void_p, c_void_p, c_int32, c_float,
                                  c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qlora_lora_down_workspace_size": (c_size_t, [c_int64, c_int64, c_int32]),
+    "qlora_lora_down": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qlora_linear_fwd_t": (c_int, [POINTER(QLoraWeight), c_void_p, c_int64, c_void_p, c_void_p, c_int32, c_float,
+                                   c_void_p, c_void_p, c_size_t, c_void_p]),
     "qlora_linear_bwd": (c_int, [POINTER(QLoraWeight), c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_int32,
                                  c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "nf4_layer_error_rank_workspace_size": (c_size_t, [c_int32, POINTER(c_int64)]),

@@ -39,19 +39,26 @@ def _need(t: torch.Tensor, dtype, name: str):
 
 
 class Workspace:
-    """A grow-only device scratch buffer per device, zeroed at allocation (its
-    first 4 bytes are the library's sticky device status word)."""
+    """A grow-only device scratch buffer per (device, stream), zeroed at allocation
+    (its first 4 bytes are the library's sticky device status word). Calls on
+    different streams get different buffers, so they may run at the same time."""
 
     _bufs = {}
 
     @classmethod
     def get(cls, nbytes: int, device: torch.device) -> torch.Tensor:
-        key = torch.device(device).index or 0
+        dev = torch.device(device)
+        idx = dev.index if dev.index is not None else torch.cuda.current_device()
+        key = (idx, torch.cuda.current_stream(idx).cuda_stream)
         buf = cls._bufs.get(key)
         if buf is None or buf.numel() < nbytes:
-            buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+            buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
             cls._bufs[key] = buf
         return buf
+
+    @classmethod
+    def all(cls, index: int):
+        return [b for (i, _), b in cls._bufs.items() if i == index]
 
 
 def read_status(ws: torch.Tensor) -> int:
@@ -134,7 +141,10 @@ def dequantize(w: NF4Weight) -> torch.Tensor:
 
 
 def linear_fwd(w: NF4Weight, X: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, scale: float,
-               save_T: bool = True, Y: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+               save_T: bool = True, Y: Optional[torch.Tensor] = None,
+               T: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Y = X W^T + s (X L1) L2. With T given (from lora_down), X L1 is not
+    recomputed and T is returned as is."""
     for t, nm in ((X, "X"), (L1, "L1"), (L2, "L2")):
         _need(t, torch.bfloat16, nm)
     lib = _lib.load()
@@ -142,12 +152,33 @@ def linear_fwd(w: NF4Weight, X: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor
     dev = X.device
     if Y is None:
         Y = torch.empty((M, w.out), dtype=torch.bfloat16, device=dev)
-    T = torch.empty((M, r), dtype=torch.bfloat16, device=dev) if save_T else None
     ws = Workspace.get(lib.qlora_fwd_workspace_size(M, w.out, w.inp, r), dev)
     cs = w.c_struct()
+    if T is not None:
+        _need(T, torch.bfloat16, "T")
+        check(lib.qlora_linear_fwd_t(ctypes.byref(cs), _ptr(X), M, _ptr(T), _ptr(L2), r, float(scale), _ptr(Y),
+                                     _ptr(ws), ws.numel(), _stream()), "qlora_linear_fwd_t")
+        return Y, T
+    T = torch.empty((M, r), dtype=torch.bfloat16, device=dev) if save_T else None
     check(lib.qlora_linear_fwd(ctypes.byref(cs), _ptr(X), M, _ptr(L1), _ptr(L2), r, float(scale), _ptr(Y), _ptr(T),
                                _ptr(ws), ws.numel(), _stream()), "qlora_linear_fwd")
     return Y, T
+
+
+def lora_down(X: torch.Tensor, L1: torch.Tensor, T: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """T = X L1 (bf16 [M x r]): the LoRA down-projection alone, for overlapping it
+    with other work; pass the result to linear_fwd(..., T=T)."""
+    _need(X, torch.bfloat16, "X")
+    _need(L1, torch.bfloat16, "L1")
+    lib = _lib.load()
+    M, r = X.shape[0], L1.shape[1]
+    dev = X.device
+    if T is None:
+        T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+    ws = Workspace.get(lib.qlora_lora_down_workspace_size(M, X.shape[1], r), dev)
+    check(lib.qlora_lora_down(_ptr(X), M, X.shape[1], _ptr(L1), r, _ptr(T), _ptr(ws), ws.numel(), _stream()),
+          "qlora_lora_down")
+    return T
 
 
 def linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, scale: float,
@@ -221,6 +252,12 @@ def quantize_error_rank(Ws: Sequence[torch.Tensor], K: int, double_quant: bool =
 
 
 def status() -> int:
-    """Device status word of this device's shared workspace (synchronizes)."""
-    dev = torch.device("cuda", torch.cuda.current_device())
-    return read_status(Workspace.get(256, dev))
+    """First nonzero device status word among this device's workspaces (one per
+    stream the library was called on); synchronizes."""
+    idx = torch.cuda.current_device()
+    dev = torch.device("cuda", idx)
+    for ws in Workspace.all(idx) or [Workspace.get(256, dev)]:
+        st = read_status(ws)
+        if st:
+            return st
+    return 0

@@ -447,29 +447,24 @@ size_t qlora_bwd_workspace_size(int64_t M, int64_t out, int64_t in, int32_t r) {
   return bwd_layout(M, out, in, r).total;
 }
 
-qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t M, const uint16_t* L1,
-                              const uint16_t* L2, int32_t r, float scale, uint16_t* Y, uint16_t* T_save,
-                              void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
-  QLB_TRY(check_linear(w, M, r));
-  if (!X || !L1 || !L2 || !Y) return QLORA_ERR_NULL;
-  if (!aligned16(X) || !aligned16(L1) || !aligned16(L2) || !aligned16(Y) || (T_save && !aligned16(T_save)))
-    return QLORA_ERR_ALIGN;
-  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+namespace {
+// The forward with T either computed here (T_in == NULL: T = X L1 into T_save or
+// the workspace) or supplied by the caller.
+qlora_status linear_fwd_impl(const qlora_weight* w, const uint16_t* X, int64_t M, const uint16_t* L1,
+                             const uint16_t* T_in, const uint16_t* L2, int32_t r, float scale, uint16_t* Y,
+                             uint16_t* T_save, void* workspace, size_t workspace_bytes, cudaStream_t s) {
   const FwdLayout L = fwd_layout(M, w->out, w->in, r);
   if (workspace_bytes < L.total) return QLORA_ERR_WORKSPACE;
   QLB_TRY(check_device());
-  cudaStream_t s = S(stream);
   char* ws = static_cast<char*>(workspace);
   int* status = reinterpret_cast<int*>(ws);
   float* scales_t = reinterpret_cast<float*>(ws + L.scales);
   uint16_t* l2t = reinterpret_cast<uint16_t*>(ws + L.l2t);
-  uint16_t* T = T_save ? T_save : reinterpret_cast<uint16_t*>(ws + L.t);
   float* part = reinterpret_cast<float*>(ws + L.part);
   const int64_t h = w->in, o_ = w->out;
   int* counters = reinterpret_cast<int*>(ws + L.counters);
   // T = X L1 : A = X (K-major), B = L1 as [h x r] (MN-major for B); the scale
   // expansion and s.L2^T are independent of it and run beside it
-  Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
   std::lock_guard<std::mutex> lock(g_side_mu);
   SideStream* ss = side_stream();
   cudaStream_t aux = s;
@@ -481,10 +476,63 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t 
     QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
                                  scales_t, aux));
   QLB_TRY(launch_scale_lora(L2, r, o_, scale, /*transpose=*/true, l2t, aux));
-  QLB_TRY(run_thin(tt, part, counters, T, 0, 1.f, status, s));
+  const uint16_t* T = T_in;
+  if (!T) {
+    uint16_t* Tw = T_save ? T_save : reinterpret_cast<uint16_t*>(ws + L.t);
+    Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
+    QLB_TRY(run_thin(tt, part, counters, Tw, 0, 1.f, status, s));
+    T = Tw;
+  }
   if (ss) QLB_TRY(join_from(ss, s));
   if (!w->is_bf16 && use_pair_kernel()) return run_pair(false, w, X, M, T, l2t, r, scales_t, Y, status, s);
   return run_main(false, w, X, M, T, l2t, r, scales_t, Y, status, s);
+}
+
+bool lora_shape_ok(int64_t M, int64_t in, int32_t r) {
+  return M > 0 && in > 0 && in % 256 == 0 && in <= (int64_t(1) << 30) && M <= (int64_t(1) << 30) &&
+         (std::max(M, in) + 127) / 128 <= kMaxCounterTiles && r >= 8 && r <= 256 && r % 8 == 0;
+}
+}  // namespace
+
+qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t M, const uint16_t* L1,
+                              const uint16_t* L2, int32_t r, float scale, uint16_t* Y, uint16_t* T_save,
+                              void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  QLB_TRY(check_linear(w, M, r));
+  if (!X || !L1 || !L2 || !Y) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(L1) || !aligned16(L2) || !aligned16(Y) || (T_save && !aligned16(T_save)))
+    return QLORA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  return linear_fwd_impl(w, X, M, L1, nullptr, L2, r, scale, Y, T_save, workspace, workspace_bytes, S(stream));
+}
+
+qlora_status qlora_linear_fwd_t(const qlora_weight* w, const uint16_t* X, int64_t M, const uint16_t* T,
+                                const uint16_t* L2, int32_t r, float scale, uint16_t* Y, void* workspace,
+                                size_t workspace_bytes, qlora_stream_t stream) {
+  QLB_TRY(check_linear(w, M, r));
+  if (!X || !T || !L2 || !Y) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(T) || !aligned16(L2) || !aligned16(Y)) return QLORA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  return linear_fwd_impl(w, X, M, nullptr, T, L2, r, scale, Y, nullptr, workspace, workspace_bytes, S(stream));
+}
+
+size_t qlora_lora_down_workspace_size(int64_t M, int64_t in, int32_t r) {
+  if (!lora_shape_ok(M, in, r)) return 0;
+  const ThinSplit ts = thin_split(M, in / 64);
+  return kReservedBytes + up256(size_t(ts.splits) * size_t(M) * r * 4);
+}
+
+qlora_status qlora_lora_down(const uint16_t* X, int64_t M, int64_t in, const uint16_t* L1, int32_t r, uint16_t* T,
+                             void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  if (!lora_shape_ok(M, in, r)) return QLORA_ERR_SHAPE;
+  if (!X || !L1 || !T) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(L1) || !aligned16(T)) return QLORA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  if (workspace_bytes < qlora_lora_down_workspace_size(M, in, r)) return QLORA_ERR_WORKSPACE;
+  QLB_TRY(check_device());
+  char* ws = static_cast<char*>(workspace);
+  Thin tt{GemmKind::ThinKM, X, in, M, L1, r, in, M, in / 64, r};
+  return run_thin(tt, reinterpret_cast<float*>(ws + kReservedBytes), reinterpret_cast<int*>(ws + kStatusBytes), T, 0,
+                  1.f, reinterpret_cast<int*>(ws), S(stream));
 }
 
 qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const uint16_t* dY, int64_t M,

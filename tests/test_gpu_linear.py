@@ -121,3 +121,44 @@ def test_14b_protected_layer_full_size_sampled(cuda_device):
     rows = np.random.default_rng(3).choice(case.M, 32, replace=False)
     rows.sort()
     run_and_compare(case, protected=True, rows=rows)
+
+
+def test_two_part_forward_matches_forward(cuda_device):
+    """lora_down + linear_fwd(T=...) is the forward split in two: the same bits as
+    the one-call forward (same kernels, same T)."""
+    case = synth.case_small()
+    d = case.make()
+    g, w = gpu_case(d, case.double_quant, False)
+    Y1, T1 = api.linear_fwd(w, g["X"], g["L1"], g["L2"], case.scale)
+    T2 = api.lora_down(g["X"], g["L1"])
+    Y2, T2r = api.linear_fwd(w, g["X"], g["L1"], g["L2"], case.scale, T=T2)
+    torch.cuda.synchronize()
+    assert api.status() == 0
+    assert T2r is T2
+    assert torch.equal(T1, T2)
+    assert torch.equal(Y1, Y2)
+
+
+def test_quantize_on_side_stream_beside_lora_down(cuda_device):
+    """The allocation pass on a second stream while T = X L1 runs on the first (each
+    stream has its own workspace): the same codes, scales and outputs as in order."""
+    case = synth.case_small()
+    d = case.make()
+    g = {k: v.cuda() for k, v in d.items()}
+    ref_w = api.quantize(g["W"], double_quant=True)
+    Yref, Tref = api.linear_fwd(ref_w, g["X"], g["L1"], g["L2"], case.scale)
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side.wait_stream(main)
+    with torch.cuda.stream(side):
+        _, _, _, (w,) = api.quantize_error_rank([g["W"]], 0, double_quant=True)
+    T = api.lora_down(g["X"], g["L1"])
+    main.wait_stream(side)
+    for t in (w.codes, w.absmax_q, w.absmax2):
+        t.record_stream(main)
+    Y, _ = api.linear_fwd(w, g["X"], g["L1"], g["L2"], case.scale, T=T)
+    torch.cuda.synchronize()
+    assert api.status() == 0
+    assert torch.equal(w.codes, ref_w.codes) and torch.equal(w.absmax_q, ref_w.absmax_q)
+    assert torch.equal(w.absmax2, ref_w.absmax2)
+    assert torch.equal(T, Tref) and torch.equal(Y, Yref)
