@@ -196,9 +196,12 @@ def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int =
                      torch.empty(w.numel() // 64, dtype=torch.float32, device=dev)))
     fused_outs = [api.NF4Weight(w.shape[0], w.shape[1], False, codes=c, absmax=a) for w, (c, a) in zip(Ws, outs)]
 
-    def q_all():
+    def q_each():
         for w, (c, a) in zip(Ws, outs):
             api.quantize(w, codes=c, absmax=a)
+
+    def q_all():
+        api.quantize_batch(Ws, double_quant=False, outs=fused_outs)
 
     def e_all():
         api.layer_error_rank(Ws, min(16, len(Ws)), double_quant=False)
@@ -209,7 +212,7 @@ def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int =
     # each leg is captured once into a CUDA graph (after an eager warm-up call) and
     # replayed, so host launch work for the 224 matrices is not in the timed region
     times = {}
-    for name, fn in (("q", q_all), ("e", e_all), ("f", f_all)):
+    for name, fn in (("qe", q_each), ("q", q_all), ("e", e_all), ("f", f_all)):
         fn()
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -226,16 +229,20 @@ def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int =
                 ts.append(e0.elapsed_time(e1))
         times[name] = ts
         del g
-    q_ms, e_ms, f_ms = times["q"], times["e"], times["f"]
+    qe_ms, q_ms, e_ms, f_ms = times["qe"], times["q"], times["e"], times["f"]
     assert api.status() == 0, "device status set in the codec legs"
-    qm, em, fm = min(q_ms), min(e_ms), min(f_ms)
+    qem, qm, em, fm = min(qe_ms), min(q_ms), min(e_ms), min(f_ms)
     del Ws, outs
     torch.cuda.empty_cache()
     return {"workload": f"llama7b stack: {len(mats)} matrices ({layers} x q,k,v,o 4096^2, gate/up 11008x4096, "
                         f"down 4096x11008), {numel / 1e9:.2f} G weights, per-matrix scale * Student-t(nu), "
                         "NF4 blocksize 64, no double quant",
             "quantize_all": {"ms": qm, "bytes": q_bytes, "GB/s": q_bytes / (qm * 1e-3) / 1e9,
-                             "frac_hbm": q_bytes / (qm * 1e-3) / 1e9 / peaks["hbm"], "launches": len(mats)},
+                             "frac_hbm": q_bytes / (qm * 1e-3) / 1e9 / peaks["hbm"], "launches": 1,
+                             "note": "nf4_quantize_batch over all matrices"},
+            "quantize_each": {"ms": qem, "bytes": q_bytes, "GB/s": q_bytes / (qem * 1e-3) / 1e9,
+                              "frac_hbm": q_bytes / (qem * 1e-3) / 1e9 / peaks["hbm"], "launches": len(mats),
+                              "note": "one nf4_quantize call per matrix"},
             "error_rank_all": {"ms": em, "bytes": e_bytes, "GB/s": e_bytes / (em * 1e-3) / 1e9,
                                "frac_hbm": e_bytes / (em * 1e-3) / 1e9 / peaks["hbm"], "launches": 3},
             "quantize_error_rank_all": {"ms": fm, "bytes": q_bytes, "GB/s": q_bytes / (fm * 1e-3) / 1e9,

@@ -138,6 +138,21 @@ qlora_status nf4_quantize(const void* W, int32_t w_dtype, int64_t out, int64_t i
                           uint8_t* codes, float* absmax, uint8_t* absmax_q, float* absmax2,
                           void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
+/* The same quantization for n bf16 matrices in one launch (a whole model at
+ * load time): matrix i is W_ptrs[i] (numel[i] elements, even) with its own
+ * codes[i], absmax[i] / absmax_q[i], absmax2[i] laid out as for nf4_quantize;
+ * every bit is the one nf4_quantize gives that matrix alone.
+ *   n        1 <= n <= 512
+ *   W_ptrs, numel, codes, absmax, absmax_q, absmax2   HOST arrays of n entries
+ *            (device pointers inside; absmax may be NULL or hold NULLs with
+ *            double quant, absmax_q / absmax2 may be NULL without it)
+ *   w_dtype  QLORA_DTYPE_BF16
+ * Errors and workspace as nf4_quantize. */
+qlora_status nf4_quantize_batch(int32_t n, const uint16_t* const* W_ptrs, const int64_t* numel, int32_t w_dtype,
+                                nf4_qconfig q, uint8_t* const* codes, float* const* absmax,
+                                uint8_t* const* absmax_q, float* const* absmax2, void* workspace,
+                                size_t workspace_bytes, qlora_stream_t stream);
+
 /* Dequantization to bf16: W_out[i] = bf16_rn(fp32_rn(code[idx_i] * a)) with a the
  * block's absmax, or with double quantization a = fp32_rn(fp32(q_b) * absmax2[g]).
  *   w      host pointer to a descriptor with is_bf16 = 0 (device buffers inside)

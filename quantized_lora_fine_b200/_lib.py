@@ -39,6 +39,9 @@ SIGNATURES = {
     "nf4_quantize_workspace_size": (c_size_t, [c_int64]),
     "nf4_quantize": (c_int, [c_void_p, c_int32, c_int64, c_int64, NF4QConfig, c_void_p, c_void_p, c_void_p,
                              c_void_p, c_void_p, c_size_t, c_void_p]),
+    "nf4_quantize_batch": (c_int, [c_int32, POINTER(c_void_p), POINTER(c_int64), c_int32, NF4QConfig,
+                                   POINTER(c_void_p), POINTER(c_void_p), POINTER(c_void_p), POINTER(c_void_p),
+                                   c_void_p, c_size_t, c_void_p]),
     "nf4_dequantize": (c_int, [POINTER(QLoraWeight), c_void_p, c_void_p]),
     "qlora_fwd_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int32]),
     "qlora_bwd_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int32]),

@@ -132,6 +132,39 @@ def quantize(W: torch.Tensor, double_quant: bool = False, keep_absmax: bool = Fa
     return NF4Weight(out, inp, double_quant, codes=codes, absmax=absmax, absmax_q=absmax_q, absmax2=absmax2)
 
 
+def quantize_batch(Ws: Sequence[torch.Tensor], double_quant: bool = False, keep_absmax: bool = False,
+                   outs: Optional[Sequence[NF4Weight]] = None) -> list:
+    """quantize() for up to 512 bf16 matrices in one launch (same bits per matrix).
+    `outs` may supply preallocated weights (same shapes and settings)."""
+    lib = _lib.load()
+    L = len(Ws)
+    for i, W in enumerate(Ws):
+        _need(W, torch.bfloat16, f"W[{i}]")
+    dev = Ws[0].device
+    if outs is None:
+        outs = []
+        for W in Ws:
+            n = W.numel()
+            nb = (n + 63) // 64
+            outs.append(NF4Weight(
+                W.shape[0], W.shape[1], double_quant,
+                codes=torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev),
+                absmax=torch.empty(nb, dtype=torch.float32, device=dev) if (not double_quant or keep_absmax) else None,
+                absmax_q=torch.empty(nb, dtype=torch.uint8, device=dev) if double_quant else None,
+                absmax2=torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev) if double_quant else None))
+    ptrs = (ctypes.c_void_p * L)(*[W.data_ptr() for W in Ws])
+    numel = (ctypes.c_int64 * L)(*[W.numel() for W in Ws])
+
+    def arr(name):
+        return (ctypes.c_void_p * L)(*[(_ptr(getattr(o, name)) or 0) for o in outs])
+
+    ws = Workspace.get(lib.nf4_quantize_workspace_size(0), dev)
+    check(lib.nf4_quantize_batch(L, ptrs, numel, DTYPE_BF16, NF4QConfig(64, 1 if double_quant else 0, 256),
+                                 arr("codes"), arr("absmax"), arr("absmax_q"), arr("absmax2"), _ptr(ws), ws.numel(),
+                                 _stream()), "nf4_quantize_batch")
+    return list(outs)
+
+
 def dequantize(w: NF4Weight) -> torch.Tensor:
     lib = _lib.load()
     out = torch.empty((w.out, w.inp), dtype=torch.bfloat16, device=w.codes.device)

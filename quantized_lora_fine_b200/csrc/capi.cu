@@ -422,6 +422,28 @@ qlora_status nf4_quantize(const void* W, int32_t w_dtype, int64_t out, int64_t i
                          static_cast<int*>(workspace), S(stream));
 }
 
+qlora_status nf4_quantize_batch(int32_t n, const uint16_t* const* W_ptrs, const int64_t* numel, int32_t w_dtype,
+                                nf4_qconfig q, uint8_t* const* codes, float* const* absmax,
+                                uint8_t* const* absmax_q, float* const* absmax2, void* workspace,
+                                size_t workspace_bytes, qlora_stream_t stream) {
+  if (w_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_DTYPE;
+  if (!qconfig_ok(q)) return QLORA_ERR_UNSUPPORTED;
+  if (n < 1 || n > 512) return QLORA_ERR_SHAPE;
+  if (!W_ptrs || !numel || !codes) return QLORA_ERR_NULL;
+  const bool dq = q.double_quant != 0;
+  if (dq ? (!absmax_q || !absmax2) : !absmax) return QLORA_ERR_NULL;
+  for (int i = 0; i < n; ++i) {
+    if (!W_ptrs[i] || !codes[i]) return QLORA_ERR_NULL;
+    if (dq ? (!absmax_q[i] || !absmax2[i]) : !absmax[i]) return QLORA_ERR_NULL;
+    if (numel[i] <= 0 || numel[i] % 2) return QLORA_ERR_SHAPE;
+    if (!aligned16(W_ptrs[i]) || !aligned16(codes[i])) return QLORA_ERR_ALIGN;
+  }
+  if (!workspace || workspace_bytes < kStatusBytes || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  QLB_TRY(check_device());
+  return launch_quantize_batch(n, W_ptrs, numel, dq, codes, absmax, absmax_q, absmax2,
+                               static_cast<int*>(workspace), S(stream));
+}
+
 qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream_t stream) {
   if (!w || !W_out) return QLORA_ERR_NULL;
   if (w->is_bf16) return QLORA_ERR_UNSUPPORTED;

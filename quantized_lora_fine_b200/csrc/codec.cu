@@ -4,6 +4,8 @@
 #include <cfloat>
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "internal.cuh"
 #include "nf4_device.cuh"
 #include "ptx.cuh"
@@ -86,12 +88,46 @@ __device__ __forceinline__ void dq_group(const float* s_amax, float* s_red, int6
 // sat(n~ 2^36 + T) in {0, 1}, and bits(B + s) carry the index; a multiply-add chain
 // packs 8 of them into a code word. Three exchange stages put the thread's 8 code
 // words back in order, and the block's 32 bytes leave in two 16-byte stores.
-template <bool DQ>
-__global__ void __launch_bounds__(256, 4) nf4_quantize_bf16_kernel(const uint16_t* __restrict__ W, int64_t numel,
-                                                                   uint8_t* __restrict__ codes,
-                                                                   float* __restrict__ absmax,
-                                                                   uint8_t* __restrict__ absmax_q,
-                                                                   float* __restrict__ absmax2, int* status) {
+// The matrices one launch quantizes: a single one (QuantOne, one CTA per group) or
+// up to kMaxQuantBatch of them (QuantBatch; the CTA's matrix is found by a binary
+// search over first_group).
+struct QuantOne {
+  const uint16_t* W;
+  int64_t numel;
+  uint8_t* codes;
+  float* absmax;
+  uint8_t* absmax_q;
+  float* absmax2;
+};
+constexpr int kMaxQuantBatch = 512;
+struct QuantBatch {
+  const uint16_t* W[kMaxQuantBatch];
+  int64_t numel[kMaxQuantBatch];
+  uint8_t* codes[kMaxQuantBatch];
+  float* absmax[kMaxQuantBatch];   // may be null with double quant
+  uint8_t* absmax_q[kMaxQuantBatch];
+  float* absmax2[kMaxQuantBatch];
+  int32_t first_group[kMaxQuantBatch + 1];
+  int32_t n;
+};
+static_assert(sizeof(QuantBatch) <= 32000, "kernel parameter limit");
+
+__device__ __forceinline__ QuantOne quant_target(const QuantOne& t, int64_t cta, int64_t& g) {
+  g = cta;
+  return t;
+}
+__device__ __forceinline__ QuantOne quant_target(const QuantBatch& t, int64_t cta, int64_t& g) {
+  int lo = 0, hi = t.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (t.first_group[mid] <= cta) lo = mid; else hi = mid - 1;
+  }
+  g = cta - t.first_group[lo];
+  return QuantOne{t.W[lo], t.numel[lo], t.codes[lo], t.absmax[lo], t.absmax_q[lo], t.absmax2[lo]};
+}
+
+template <bool DQ, class Tab>
+__global__ void __launch_bounds__(256, 4) nf4_quantize_bf16_kernel(const __grid_constant__ Tab tab, int* status) {
   __shared__ __align__(128) uint32_t s_w[kChunkBytes / 4];   // the group's bf16 pairs
   __shared__ float s_amax[kDQBlock];
   __shared__ float s_red[8];
@@ -103,8 +139,15 @@ __global__ void __launch_bounds__(256, 4) nf4_quantize_bf16_kernel(const uint16_
     fence_mbarrier_init();
   }
   const LaneTables lt = lane_tables(tid & 31);
+  int64_t g;
+  const QuantOne q = quant_target(tab, blockIdx.x, g);
+  const uint16_t* __restrict__ W = q.W;
+  const int64_t numel = q.numel;
+  uint8_t* __restrict__ codes = q.codes;
+  float* __restrict__ absmax = q.absmax;
+  uint8_t* __restrict__ absmax_q = q.absmax_q;
+  float* __restrict__ absmax2 = q.absmax2;
   const int64_t nb = (numel + kBlock - 1) / kBlock;
-  const int64_t g = blockIdx.x;
   const int64_t e_g = g * int64_t(kDQBlock * kBlock);                 // first element of the group
   const int n_g = int(min(int64_t(kDQBlock * kBlock), numel - e_g));  // its elements (even, > 0)
   const int nblk = (n_g + kBlock - 1) / kBlock;
@@ -254,13 +297,42 @@ qlora_status launch_quantize(const void* W, int w_dtype, int64_t numel, bool dq,
   dim3 grid(static_cast<unsigned>(groups));
   if (w_dtype == QLORA_DTYPE_BF16) {
     const uint16_t* Wb = static_cast<const uint16_t*>(W);
-    if (dq) launch_pdl(nf4_quantize_bf16_kernel<true>, grid, dim3(256), 0, s, Wb, numel, codes, absmax, absmax_q, absmax2, status);
-    else launch_pdl(nf4_quantize_bf16_kernel<false>, grid, dim3(256), 0, s, Wb, numel, codes, absmax, absmax_q, absmax2, status);
+    const QuantOne one{Wb, numel, codes, absmax, absmax_q, absmax2};
+    if (dq) launch_pdl(nf4_quantize_bf16_kernel<true, QuantOne>, grid, dim3(256), 0, s, one, status);
+    else launch_pdl(nf4_quantize_bf16_kernel<false, QuantOne>, grid, dim3(256), 0, s, one, status);
   } else {
     if (dq) nf4_quantize_f32_kernel<true><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
     else nf4_quantize_f32_kernel<false><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
   }
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status launch_quantize_batch(int n, const uint16_t* const* W, const int64_t* numel, bool dq,
+                                   uint8_t* const* codes, float* const* absmax, uint8_t* const* absmax_q,
+                                   float* const* absmax2, int* status, cudaStream_t s) {
+  if (n < 1 || n > kMaxQuantBatch) return QLORA_ERR_SHAPE;
+  static std::mutex mu;
+  static QuantBatch tab;   // host staging of the by-value parameter
+  std::lock_guard<std::mutex> lock(mu);
+  tab.n = n;
+  int64_t c = 0;
+  for (int i = 0; i < n; ++i) {
+    tab.W[i] = W[i];
+    tab.numel[i] = numel[i];
+    tab.codes[i] = codes[i];
+    tab.absmax[i] = absmax ? absmax[i] : nullptr;
+    tab.absmax_q[i] = dq ? absmax_q[i] : nullptr;
+    tab.absmax2[i] = dq ? absmax2[i] : nullptr;
+    tab.first_group[i] = int32_t(c);
+    const int64_t nb = (numel[i] + kBlock - 1) / kBlock;
+    c += (nb + kDQBlock - 1) / kDQBlock;
+    if (c > (int64_t(1) << 31) - 1) return QLORA_ERR_SHAPE;
+  }
+  tab.first_group[n] = int32_t(c);
+  const dim3 grid(static_cast<unsigned>(c));
+  const cudaError_t e = dq ? launch_pdl(nf4_quantize_bf16_kernel<true, QuantBatch>, grid, dim3(256), 0, s, tab, status)
+                           : launch_pdl(nf4_quantize_bf16_kernel<false, QuantBatch>, grid, dim3(256), 0, s, tab, status);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- dequantize

@@ -58,6 +58,10 @@ __device__ __forceinline__ void set_status_site(int* st, int code, int site) {
 // ---- codec.cu
 qlora_status launch_quantize(const void* W, int w_dtype, int64_t numel, bool dq, uint8_t* codes, float* absmax,
                              uint8_t* absmax_q, float* absmax2, int* status, cudaStream_t s);
+// Up to 512 bf16 matrices in one launch (same double-quant setting for all).
+qlora_status launch_quantize_batch(int n, const uint16_t* const* W, const int64_t* numel, bool dq,
+                                   uint8_t* const* codes, float* const* absmax, uint8_t* const* absmax_q,
+                                   float* const* absmax2, int* status, cudaStream_t s);
 qlora_status launch_dequantize(const uint8_t* codes, const float* absmax, const uint8_t* absmax_q,
                                const float* absmax2, bool dq, int64_t numel, uint16_t* out, cudaStream_t s);
 // Scales of an out x in NF4 weight, expanded to fp32 and laid out [in/64][out].

@@ -81,6 +81,19 @@ def test_host_validation_before_any_launch(lib):
     n = (ctypes.c_int64 * 1)(100)
     assert lib.nf4_layer_error_rank(1, ptrs, n, 0, q, 2, None, None, None, None, 0, None) == 2
     assert lib.nf4_layer_error_rank(1, ptrs, n, 0, q, 1, 0x10, 0x10, 0x10, None, 0, None) == 2
+    # batch quantize: n out of range, odd element count, misaligned codes, missing absmax
+    cp = (ctypes.c_void_p * 1)(0x2000)
+    am = (ctypes.c_void_p * 1)(0x3000)
+    none = (ctypes.c_void_p * 1)(0)
+    assert lib.nf4_quantize_batch(0, ptrs, n, 0, q, cp, am, none, none, 0x4000, 256, None) == 2
+    n_odd = (ctypes.c_int64 * 1)(101)
+    assert lib.nf4_quantize_batch(1, ptrs, n_odd, 0, q, cp, am, none, none, 0x4000, 256, None) == 2
+    cp_bad = (ctypes.c_void_p * 1)(0x2001)
+    assert lib.nf4_quantize_batch(1, ptrs, n, 0, q, cp_bad, am, none, none, 0x4000, 256, None) == 3
+    assert lib.nf4_quantize_batch(1, ptrs, n, 0, q, cp, none, none, none, 0x4000, 256, None) == 1
+    # two-part forward: bad rank; the misaligned weight above
+    assert lib.qlora_lora_down(None, 8, 4096, None, 12, None, None, 0, None) == 2
+    assert lib.qlora_linear_fwd_t(ctypes.byref(w), 0x1000, 8, None, 0x1000, 16, 2.0, 0x1000, None, 0, None) == 3
 
 
 def test_product_path_refuses_without_library(tmp_path, monkeypatch):

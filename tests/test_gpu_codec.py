@@ -115,3 +115,33 @@ def test_quant_stack_gate_matrix_full_size(cuda_device):
     W = synth.stack_weight(m)
     _check_quant(W, dq=False)
     _check_quant(W, dq=True)
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_quantize_batch_matches_single_calls(cuda_device, dq):
+    """One batched launch over matrices of several shapes (one with a ragged last
+    block, one smaller than a group) gives every matrix the bits of its own call."""
+    shapes = [(512, 512), (11, 66), (3, 20000), (64, 256), (1, 6)]
+    Ws = [synth.normal_bf16(sh, 0.02, 0, 1, i, device="cuda") for i, sh in enumerate(shapes)]
+    outs = api.quantize_batch(Ws, double_quant=dq, keep_absmax=True)
+    for W, o in zip(Ws, outs):
+        ref = api.quantize(W, double_quant=dq, keep_absmax=True)
+        assert torch.equal(o.codes, ref.codes)
+        assert torch.equal(o.absmax.view(torch.int32), ref.absmax.view(torch.int32))
+        if dq:
+            assert torch.equal(o.absmax_q, ref.absmax_q)
+            assert torch.equal(o.absmax2.view(torch.int32), ref.absmax2.view(torch.int32))
+    assert api.status() == 0
+
+
+def test_quantize_batch_stack_layer(cuda_device):
+    """The seven matrices of one decoder layer of the 7B stack in one launch give the
+    bits of seven single calls (which the tests above hold to the oracle)."""
+    mats = synth.stack_matrices(n_layers=1)
+    Ws = [synth.stack_weight(m, device="cuda") for m in mats]
+    outs = api.quantize_batch(Ws, double_quant=True)
+    for W, o in zip(Ws, outs):
+        ref = api.quantize(W, double_quant=True)
+        assert torch.equal(o.codes, ref.codes) and torch.equal(o.absmax_q, ref.absmax_q)
+        assert torch.equal(o.absmax2.view(torch.int32), ref.absmax2.view(torch.int32))
+    assert api.status() == 0
