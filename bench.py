@@ -495,7 +495,7 @@ def gpu_main(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args, world),
-            "roofline": roofline, "legs": legs_out, "hbm_legs": hbm, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "gemm_pairs": int(lib.qlora_pair_clusters()), "legs": legs_out, "hbm_legs": hbm, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
             "timing": "cuda-graph replay of the step" if use_graphs else "eager API calls",
             "peaks": {"bf16_tflops": peaks["bf16"], "bf16_tflops_sustained": peaks["bf16_sus"],

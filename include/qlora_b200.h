@@ -115,6 +115,11 @@ qlora_status qlora_device_check(int device);
  * (dx_*). Pass NULL to disable. Process-wide; not thread-safe. */
 qlora_status qlora_profile_events(void* fwd_begin, void* fwd_end, void* dx_begin, void* dx_end);
 
+/* Diagnostic (not part of the method): the number of 2-SM CTA pairs the last NF4
+ * GEMM launch used (0 before any). The 256 x 256 output tiles are spread over
+ * them, so a part that co-schedules fewer pairs takes more rounds of tiles. */
+int32_t qlora_pair_clusters(void);
+
 /* ------------------------------------------------------------ NF4 codec */
 
 /* Bytes of workspace nf4_quantize needs (the status word only). */

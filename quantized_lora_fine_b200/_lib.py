@@ -36,6 +36,7 @@ SIGNATURES = {
     "qlora_reset_status": (c_int, [c_void_p, c_void_p]),
     "qlora_device_check": (c_int, [c_int]),
     "qlora_profile_events": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p]),
+    "qlora_pair_clusters": (c_int32, []),
     "nf4_quantize_workspace_size": (c_size_t, [c_int64]),
     "nf4_quantize": (c_int, [c_void_p, c_int32, c_int64, c_int64, NF4QConfig, c_void_p, c_void_p, c_void_p,
                              c_void_p, c_void_p, c_size_t, c_void_p]),

@@ -372,6 +372,8 @@ const char* qlora_status_str(qlora_status s) {
   return "unknown status";
 }
 
+int32_t qlora_pair_clusters(void) { return last_pair_clusters(); }
+
 qlora_status qlora_profile_events(void* fwd_begin, void* fwd_end, void* dx_begin, void* dx_end) {
   g_prof[0] = static_cast<cudaEvent_t>(fwd_begin);
   g_prof[1] = static_cast<cudaEvent_t>(fwd_end);

@@ -803,6 +803,12 @@ static qlora_status launch_cfg(const GemmOperands& o, GemmParams p, int ctas_per
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// CTA pairs of the last pair launch (0 before any): the co-resident 2-SM clusters the
+// occupancy calculator reports for the kernel (74 on a 148-SM part when every GPC can
+// pair all of its SMs), capped by the tile count.
+static int g_last_pairs = 0;
+int last_pair_clusters() { return g_last_pairs; }
+
 template <class C>
 static qlora_status launch_pair_cfg(const GemmOperands& o, GemmParams p, cudaStream_t s) {
   static bool attr_set = false;
@@ -833,6 +839,7 @@ static qlora_status launch_pair_cfg(const GemmOperands& o, GemmParams p, cudaStr
   p.bn = 256;
   const int num_tiles = p.tiles_m * p.tiles_n;
   const int pairs = std::max(1, std::min(num_tiles, max_pairs));
+  g_last_pairs = pairs;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -89,6 +89,7 @@ qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const
                                              cudaStream_t s);
 
 // ---- gemm.cu
+int last_pair_clusters();
 // Operand descriptions for the tcgen05 GEMM engine.
 struct GemmPlan;
 }  // namespace qlb
