@@ -205,6 +205,17 @@ namespace {
 // The NF4 GEMMs run on the CTA-pair kernel unless QLORA_B200_GEMM=1cta selects
 // the single-CTA kernel (both compute the same values; kept side by side for
 // measurement).
+// Backward schedule: QLORA_B200_BWD=beside or =serial forces one of the two (read on
+// every call, so tests can cover both on any part); otherwise it follows the SMs the
+// dX GEMM leaves free.
+int bwd_schedule_override() {
+  const char* e = std::getenv("QLORA_B200_BWD");
+  if (!e) return 0;
+  if (std::strcmp(e, "beside") == 0) return 1;
+  if (std::strcmp(e, "serial") == 0) return 2;
+  return 0;
+}
+
 bool use_pair_kernel() {
   static int v = -1;
   if (v < 0) {
@@ -315,8 +326,9 @@ qlora_status run_main(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
 // graph capture (the side stream joins the capture through the event). Calls
 // from several host threads serialize on the mutex while they enqueue.
 struct SideStream {
-  cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaStream_t stream = nullptr;   // default priority: small independent kernels
+  cudaStream_t hi = nullptr;       // highest priority: a GEMM that shares the GPU
+  cudaEvent_t fork = nullptr, mid = nullptr, join = nullptr;
 };
 constexpr int kMaxSideDevices = 64;
 std::mutex g_side_mu;
@@ -329,8 +341,14 @@ SideStream* side_stream() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return nullptr;
   SideStream& ss = g_side[dev];
   if (!ss.stream) {
+    // hi: when its tensor-core GEMM and a caller-stream kernel become ready together,
+    // the GEMM's CTAs are placed first
+    int least = 0, greatest = 0;
+    cudaDeviceGetStreamPriorityRange(&least, &greatest);
     if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&ss.hi, cudaStreamNonBlocking, greatest) != cudaSuccess ||
         cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.mid, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
       cudaGetLastError();
       ss = SideStream();
@@ -340,14 +358,25 @@ SideStream* side_stream() {
   return &ss;
 }
 
-qlora_status fork_to(SideStream* ss, cudaStream_t s) {
-  if (cudaEventRecord(ss->fork, s) != cudaSuccess || cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
+// side waits for the work enqueued on s so far (side = ss->stream by default, or ss->hi)
+qlora_status fork_to(SideStream* ss, cudaStream_t s, cudaStream_t side = nullptr) {
+  if (cudaEventRecord(ss->fork, s) != cudaSuccess ||
+      cudaStreamWaitEvent(side ? side : ss->stream, ss->fork, 0) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return QLORA_OK;
 }
 
-qlora_status join_from(SideStream* ss, cudaStream_t s) {
-  if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess || cudaStreamWaitEvent(s, ss->join, 0) != cudaSuccess)
+// A second fork point: side waits for the work enqueued on s so far.
+qlora_status handoff_to(SideStream* ss, cudaStream_t s, cudaStream_t side) {
+  if (cudaEventRecord(ss->mid, s) != cudaSuccess || cudaStreamWaitEvent(side, ss->mid, 0) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
+
+// s waits for everything enqueued on side (ss->stream by default, or ss->hi)
+qlora_status join_from(SideStream* ss, cudaStream_t s, cudaStream_t side = nullptr) {
+  if (cudaEventRecord(ss->join, side ? side : ss->stream) != cudaSuccess ||
+      cudaStreamWaitEvent(s, ss->join, 0) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return QLORA_OK;
 }
@@ -589,33 +618,51 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const ui
     QLB_TRY(run_thin(tt, part, counters, Tw, 0, 1.f, status, s));
     T = Tw;
   }
-  // dL2 = s (dY^T T)^T (A = dY^T MN-major, B = T MN-major, K = M, written
-  // transposed) and the scale expansion run on the side stream, beside
-  // U = dY L2^T (A = dY K-major, B = L2 [r x out] K-major; with the pair engine
-  // also s.U, the dX LoRA step's A) and dL1 = s X^T U on the caller's stream. The
-  // side products use their own partial buffer and counter range.
+  // U = dY L2^T (A = dY K-major, B = L2 [r x out] K-major; with the pair engine also
+  // s.U, the dX LoRA step's A), dL1 = s X^T U and dL2 = s (dY^T T)^T (A = dY^T
+  // MN-major, B = T MN-major, K = M, written transposed) are thin HBM-bound products;
+  // dX is the tensor-core GEMM. dL2 uses its own partial buffer and counter range so
+  // it can run beside the others. Two schedules:
+  //  * the pair GEMM leaves SMs free (its pair count is the fewest that keeps its
+  //    number of rounds of tiles, see pair_spare_sms): U, then dX on the side stream
+  //    (highest priority) while dL1 and dL2 run on the caller's stream on the free
+  //    SMs and, later, on the GEMM's idle SMs in its last round;
+  //  * otherwise dL2 and the scale expansion run on the side stream beside U and dL1,
+  //    and dX follows on the caller's stream.
   const bool pair = !w->is_bf16 && use_pair_kernel();
   uint16_t* sU = reinterpret_cast<uint16_t*>(ws + L.su);
   float* part2 = reinterpret_cast<float*>(ws + L.part2);
   std::lock_guard<std::mutex> lock(g_side_mu);
   SideStream* ss = ((M + 127) / 128 <= kMaxCounterTiles / 2 && (o_ + 127) / 128 <= kMaxCounterTiles / 2)
                        ? side_stream() : nullptr;
+  const int dx_tiles = int((M + 255) / 256) * int(h / 256);
+  const int forced = bwd_schedule_override();
+  const bool beside_gemm = ss && dX && pair && forced != 2 && (forced == 1 || pair_spare_sms(true, dx_tiles) >= 16);
   cudaStream_t aux = s;
   int* counters2 = counters;
   if (ss) {
-    QLB_TRY(fork_to(ss, s));
-    aux = ss->stream;
+    aux = beside_gemm ? ss->hi : ss->stream;
+    QLB_TRY(fork_to(ss, s, aux));
     counters2 = counters + kMaxCounterTiles / 2;
   }
+  float* part_b = ss ? part2 : part;
+  Thin tu{GemmKind::ThinKK, dY, o_, M, L2, o_, r, M, o_ / 64, r};
+  Thin t1{GemmKind::ThinMM, X, h, M, U, r, M, h, mk, r};
   Thin t2{GemmKind::ThinMM, dY, o_, M, T, r, M, o_, mk, r};
-  QLB_TRY(run_thin(t2, ss ? part2 : part, counters2, dL2, 2, scale, status, aux));
   if (dX && !w->is_bf16)
     QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
                                  scales_t, aux));
-  Thin tu{GemmKind::ThinKK, dY, o_, M, L2, o_, r, M, o_ / 64, r};
+  if (beside_gemm) {
+    QLB_TRY(run_thin(tu, part, counters, U, 3, scale, status, s, sU));
+    QLB_TRY(handoff_to(ss, s, aux));   // the GEMM needs s.U
+    QLB_TRY(run_pair(true, w, dY, M, sU, L1, r, scales_t, dX, status, aux));
+    QLB_TRY(run_thin(t1, part, counters, dL1, 1, scale, status, s));
+    QLB_TRY(run_thin(t2, part_b, counters2, dL2, 2, scale, status, s));
+    return join_from(ss, s, aux);
+  }
+  QLB_TRY(run_thin(t2, part_b, counters2, dL2, 2, scale, status, aux));
   if (pair && dX) QLB_TRY(run_thin(tu, part, counters, U, 3, scale, status, s, sU));
   else QLB_TRY(run_thin(tu, part, counters, U, 0, 1.f, status, s));
-  Thin t1{GemmKind::ThinMM, X, h, M, U, r, M, h, mk, r};
   QLB_TRY(run_thin(t1, part, counters, dL1, 1, scale, status, s));
   if (ss) QLB_TRY(join_from(ss, s));
   if (dX && pair) return run_pair(true, w, dY, M, sU, L1, r, scales_t, dX, status, s);

@@ -809,14 +809,15 @@ static qlora_status launch_cfg(const GemmOperands& o, GemmParams p, int ctas_per
 static int g_last_pairs = 0;
 int last_pair_clusters() { return g_last_pairs; }
 
+// Co-resident 2-SM clusters of the pair kernel (occupancy calculator; sets the
+// kernel's shared-memory limit on first use), 0 on failure.
 template <class C>
-static qlora_status launch_pair_cfg(const GemmOperands& o, GemmParams p, cudaStream_t s) {
-  static bool attr_set = false;
-  static int max_pairs = 0;
-  if (!attr_set) {
+static int pair_max_clusters() {
+  static int max_pairs = -1;
+  if (max_pairs < 0) {
     if (cudaFuncSetAttribute(tc_gemm_nf4_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
         cudaSuccess)
-      return QLORA_ERR_CUDA;
+      return 0;
     cudaLaunchConfig_t qc = {};
     cudaLaunchAttribute qa[1];
     qa[0].id = cudaLaunchAttributeClusterDimension;
@@ -834,11 +835,30 @@ static qlora_status launch_pair_cfg(const GemmOperands& o, GemmParams p, cudaStr
       n = num_sms() / 2;
     }
     max_pairs = n;
-    attr_set = true;
   }
+  return max_pairs;
+}
+
+// The fewest pairs that still finish num_tiles tiles in the least number of rounds:
+// the same time for the GEMM, and the SMs left over stay free for concurrent work.
+static int pairs_for(int num_tiles, int max_pairs) {
+  const int rounds = (num_tiles + max_pairs - 1) / max_pairs;
+  return std::max(1, (num_tiles + rounds - 1) / rounds);
+}
+
+int pair_spare_sms(bool dx, int num_tiles) {
+  const int mp = dx ? pair_max_clusters<PairCfg<true>>() : pair_max_clusters<PairCfg<false>>();
+  if (mp <= 0) return 0;
+  return num_sms() - 2 * pairs_for(num_tiles, mp);
+}
+
+template <class C>
+static qlora_status launch_pair_cfg(const GemmOperands& o, GemmParams p, cudaStream_t s) {
+  const int max_pairs = pair_max_clusters<C>();
+  if (max_pairs <= 0) return QLORA_ERR_CUDA;
   p.bn = 256;
   const int num_tiles = p.tiles_m * p.tiles_n;
-  const int pairs = std::max(1, std::min(num_tiles, max_pairs));
+  const int pairs = pairs_for(num_tiles, max_pairs);
   g_last_pairs = pairs;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];

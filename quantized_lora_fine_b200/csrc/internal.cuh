@@ -90,6 +90,8 @@ qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const
 
 // ---- gemm.cu
 int last_pair_clusters();
+// SMs a pair GEMM over num_tiles 256 x 256 tiles leaves free (see pairs_for).
+int pair_spare_sms(bool dx, int num_tiles);
 // Operand descriptions for the tcgen05 GEMM engine.
 struct GemmPlan;
 }  // namespace qlb

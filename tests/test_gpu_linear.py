@@ -162,3 +162,28 @@ def test_quantize_on_side_stream_beside_lora_down(cuda_device):
     assert torch.equal(w.codes, ref_w.codes) and torch.equal(w.absmax_q, ref_w.absmax_q)
     assert torch.equal(w.absmax2, ref_w.absmax2)
     assert torch.equal(T, Tref) and torch.equal(Y, Yref)
+
+
+@pytest.mark.parametrize("schedule", ["beside", "serial"])
+def test_backward_schedules_give_the_same_bits(cuda_device, monkeypatch, schedule):
+    """Both backward schedules (dX beside dL1 / dL2, or dL2 beside U and dL1 before
+    dX) compute the same products with the same reductions: identical bits, and
+    within the oracle's tolerance."""
+    case = dataclasses.replace(synth.case_q_proj(seed=3, M=1024), double_quant=True)
+    monkeypatch.delenv("QLORA_B200_BWD", raising=False)
+    ref = run_and_compare(case, rows=np.arange(0, case.M, 97))
+    d = case.make()
+    g, w = gpu_case(d, case.double_quant, False)
+    Y, T = api.linear_fwd(w, g["X"], g["L1"], g["L2"], case.scale)
+    outs = {}
+    for sch in ("auto", schedule):
+        if sch == "auto":
+            monkeypatch.delenv("QLORA_B200_BWD", raising=False)
+        else:
+            monkeypatch.setenv("QLORA_B200_BWD", sch)
+        outs[sch] = api.linear_bwd(w, g["X"], g["dY"], g["L1"], g["L2"], case.scale, T=T)
+    torch.cuda.synchronize()
+    assert api.status() == 0
+    for a, b in zip(outs["auto"], outs[schedule]):
+        assert torch.equal(a, b)
+    assert ref is not None
