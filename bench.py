@@ -180,6 +180,26 @@ class ClockSampler:
                 "reasons": sorted(seen), "samples": len(rows)}
 
 
+def pair_gemm_traffic(name: str):
+    """DRAM bytes per launch of a fused pair GEMM from the committed ncu capture in
+    profiles/roofline_traffic.json, or None when the GEMM's sources changed since the
+    capture (their hash no longer matches)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    try:
+        d = json.load(open(path))
+        h = hashlib.sha256()
+        for f in d["sources"]:
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                h.update(fh.read())
+        if h.hexdigest() != d["sources_sha256"]:
+            return None
+        k = d["kernels"][name]
+        return k["dram_bytes_read"] + k["dram_bytes_write"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int = 32):
     """Quantize-all and error/rank over the Llama-7B-shaped stack (32 layers, 224
     matrices by default; fewer layers for small profiler captures)."""
@@ -429,7 +449,8 @@ def gpu_main(args):
                 "unit": "TFLOP/s", "frac": dom[1] / peaks[peak_key],
                 "peak_kind": f"{peak_kind} ({peaks['source']}; power cap {'seen' if capped else 'not seen'})",
                 "frac_of_burst": dom[1] / peaks["bf16"], "frac_of_sustained": dom[1] / peaks["bf16_sus"],
-                "traffic": None,
+                "traffic": pair_gemm_traffic("qlora_fwd_gemm" if dom[0].startswith("qlora_fwd") else "qlora_bwd_dx_gemm"),
+                "traffic_unit": "bytes per launch (ncu dram read + write)",
                 "per_launch_flops": fl_fwd_gemm if dom[0].startswith("qlora_fwd") else fl_dx_gemm}
     legs_out = {
         "quantize_error_rank": {"ms": med["quantize_error_rank"],
