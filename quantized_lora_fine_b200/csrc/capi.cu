@@ -14,8 +14,8 @@ using namespace qlb;
 
 namespace {
 
-constexpr int kThinTargetCtas = 296;  // split-K target for the thin LoRA products (fixed: results do not
-                                      // depend on the device's SM count)
+constexpr int kThinTargetCtas = 148;  // split-K target for the thin LoRA products, about one CTA per SM
+                                      // (fixed: results do not depend on the device's SM count)
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }

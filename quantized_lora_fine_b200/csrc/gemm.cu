@@ -890,17 +890,18 @@ qlora_status launch_gemm(GemmKind kind, int bn, const GemmOperands& o, const Gem
     case GemmKind::DxNF4: return launch_cfg<GemmCfg<256, false, true, true, false, 3>>(o, p, 1, s);
     case GemmKind::FwdBF16: return launch_cfg<GemmCfg<256, false, false, false, false, 4>>(o, p, 1, s);
     case GemmKind::DxBF16: return launch_cfg<GemmCfg<256, false, true, false, false, 4>>(o, p, 1, s);
+    // thin products: one CTA per SM with a deep ring (HBM-bound streaming of A)
     case GemmKind::ThinKK:  // A K-major, B K-major, fp32 partials
-      if (bn <= 64) return launch_cfg<GemmCfg<64, false, false, false, true, 4>>(o, p, 2, s);
-      if (bn <= 128) return launch_cfg<GemmCfg<128, false, false, false, true, 4>>(o, p, 2, s);
+      if (bn <= 64) return launch_cfg<GemmCfg<64, false, false, false, true, 8>>(o, p, 1, s);
+      if (bn <= 128) return launch_cfg<GemmCfg<128, false, false, false, true, 6>>(o, p, 1, s);
       return launch_cfg<GemmCfg<256, false, false, false, true, 4>>(o, p, 1, s);
     case GemmKind::ThinKM:  // A K-major, B MN-major
-      if (bn <= 64) return launch_cfg<GemmCfg<64, false, true, false, true, 4>>(o, p, 2, s);
-      if (bn <= 128) return launch_cfg<GemmCfg<128, false, true, false, true, 4>>(o, p, 2, s);
+      if (bn <= 64) return launch_cfg<GemmCfg<64, false, true, false, true, 8>>(o, p, 1, s);
+      if (bn <= 128) return launch_cfg<GemmCfg<128, false, true, false, true, 6>>(o, p, 1, s);
       return launch_cfg<GemmCfg<256, false, true, false, true, 4>>(o, p, 1, s);
     case GemmKind::ThinMM:  // A MN-major, B MN-major
-      if (bn <= 64) return launch_cfg<GemmCfg<64, true, true, false, true, 4>>(o, p, 2, s);
-      if (bn <= 128) return launch_cfg<GemmCfg<128, true, true, false, true, 4>>(o, p, 2, s);
+      if (bn <= 64) return launch_cfg<GemmCfg<64, true, true, false, true, 8>>(o, p, 1, s);
+      if (bn <= 128) return launch_cfg<GemmCfg<128, true, true, false, true, 6>>(o, p, 1, s);
       return launch_cfg<GemmCfg<256, true, true, false, true, 4>>(o, p, 1, s);
   }
   return QLORA_ERR_UNSUPPORTED;
