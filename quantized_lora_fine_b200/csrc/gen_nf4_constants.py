@@ -134,17 +134,12 @@ def render():
         "// Lane tables for the warp-shuffle code lookup: lane c = cell c = floor(15.75 n + 16)",
         "// in [0, 31] (the low bits of RZ(15.75 n + 2^23 + 16)), base_c = the number of",
         "// midpoints below the cell. kNF4LaneB[c] = 2^23 + base_c; kNF4LaneT[c] = -m_base 2^36",
-        "// (-2^38 if base_c = 15); kNF4LaneLo[c] = code[base_c]; kNF4LaneD[c] = code[base_c + 1]",
-        "// - code[base_c] (exact; 0 if base_c = 15). With s = sat(n 2^36 + T[c]):",
-        "// bits(B[c] + s) = 0x4B000000 + code index, and the code value is Lo[c] + s D[c].",
+        "// (-2^38 if base_c = 15). With s = sat(n 2^36 + T[c]): bits(B[c] + s) = 0x4B000000 +",
+        "// code index.",
         "__device__ constexpr uint32_t kNF4LaneB[32] = {",
         "    " + ", ".join("0x%08Xu" % v for v in B) + "};",
         "__device__ constexpr uint32_t kNF4LaneT[32] = {",
         "    " + ", ".join("0x%08Xu" % v for v in T) + "};",
-        "__device__ constexpr uint32_t kNF4LaneLo[32] = {",
-        "    " + ", ".join("0x%08Xu" % v for v in LO) + "};",
-        "__device__ constexpr uint32_t kNF4LaneD[32] = {",
-        "    " + ", ".join("0x%08Xu" % v for v in D) + "};",
         "}  // namespace qlb",
         "",
     ]

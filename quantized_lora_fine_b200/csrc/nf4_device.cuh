@@ -71,12 +71,6 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
 // ---- code index of a normalised value: FMA-pipe arithmetic and warp shuffles
 // A block with absmax a is processed with a power-of-two scale sc (1, or 2^64 /
 // 2^-64 for tiny / huge blocks) so that r = RN(1/(a sc)) is a normal number; a
@@ -93,17 +87,15 @@ __device__ __forceinline__ float sat_fma(float a, float b, float c) {
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// This lane's entries of the lookup tables: lane l holds cell l's B, T, Lo, D and
+// This lane's entries of the lookup tables: lane l holds cell l's B and T and
 // code[l mod 16] (a kernel loads the ones it uses).
 struct LaneTables {
-  float B, T, lo, d, code;
+  float B, T, code;
 };
 __device__ __forceinline__ LaneTables lane_tables(int lane) {
   LaneTables t;
   t.B = __uint_as_float(kNF4LaneB[lane]);
   t.T = __uint_as_float(kNF4LaneT[lane]);
-  t.lo = __uint_as_float(kNF4LaneLo[lane]);
-  t.d = __uint_as_float(kNF4LaneD[lane]);
   t.code = __uint_as_float(kNF4CodeBits[lane & 15]);
   return t;
 }
@@ -119,14 +111,6 @@ __device__ __forceinline__ uint32_t index_bits(float ns, uint32_t cell_bits, flo
 // Code value of index bits x (lane x mod 32 holds code[x mod 16]).
 __device__ __forceinline__ float code_value(uint32_t x, const LaneTables& lt) {
   return __shfl_sync(0xffffffffu, lt.code, int(x));
-}
-// Code value of one element straight from its cell: Lo + s D with s = sat(n_s M + T)
-// (three independent shuffles; exact). Every lane of the warp must call it.
-__device__ __forceinline__ float code_value_of_cell(float ns, uint32_t cell_bits, float M, const LaneTables& lt) {
-  const float t = __shfl_sync(0xffffffffu, lt.T, int(cell_bits));
-  const float lo = __shfl_sync(0xffffffffu, lt.lo, int(cell_bits));
-  const float d = __shfl_sync(0xffffffffu, lt.d, int(cell_bits));
-  return __fmaf_rn(sat_fma(ns, M, t), d, lo);
 }
 // Per-block constants of the lookup: r = RN(1/(a sc)) and the two multipliers.
 struct CellScale {
