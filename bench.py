@@ -200,6 +200,52 @@ def pair_gemm_traffic(name: str):
         return None
 
 
+def mlp_leg(api, synth, torch, dev, peaks, reps: int = 5):
+    """The Llama-7B MLP at M = 8192 (gate and up 4096 -> 11008, down 11008 -> 4096;
+    NF4 blocks of 64 without double quant; r = 64, alpha = 128): fwd+bwd of the three
+    linears, weights quantized once outside the timed region, captured in one CUDA
+    graph and replayed (L2 flushed before each replay)."""
+    items = []
+    fl = 0.0
+    for c in synth.cases_mlp():
+        d = c.make(device=str(dev))
+        w = api.quantize(d["W"], double_quant=False)
+        items.append((c, w, d))
+        fl += flops_fwd_bwd(c.M, c.inp, c.out, c.r)
+
+    def run():
+        for c, w, d in items:
+            T = api.lora_down(d["X"], d["L1"])
+            api.linear_fwd(w, d["X"], d["L1"], d["L2"], c.scale, T=T)
+            api.linear_bwd(w, d["X"], d["dY"], d["L1"], d["L2"], c.scale, T=T)
+
+    run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for i in range(reps + 1):
+        flush.zero_()
+        e0.record()
+        g.replay()
+        e1.record()
+        e1.synchronize()
+        if i:
+            ts.append(e0.elapsed_time(e1))
+    assert api.status() == 0, "device status set in the MLP leg"
+    ms = statistics.median(ts)
+    tf = fl / (ms * 1e-3) / 1e12
+    del g, items
+    torch.cuda.empty_cache()
+    return {"workload": "llama7b MLP: gate/up 4096->11008, down 11008->4096, M=8192, NF4 (no double quant), "
+                        "r=64, alpha=128, fwd+bwd of the three linears",
+            "ms": ms, "TFLOP/s": tf, "frac_of_burst": tf / peaks["bf16"],
+            "timing": f"CUDA-graph replay, median of {reps}, L2 flushed before each"}
+
+
 def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int = 32):
     """Quantize-all and error/rank over the Llama-7B-shaped stack (32 layers, 224
     matrices by default; fewer layers for small profiler captures)."""
@@ -368,12 +414,15 @@ def gpu_main(args):
         state["w"], state["T"] = alloc_and_down(g["W"], g["X"], g["L1"])
         leg_fwd(); leg_bwd()
 
+    def fwd_bwd():     # the linear's fwd+bwd alone (weights already quantized)
+        leg_down(); leg_fwd(); leg_bwd()
+
     use_graphs = not args.eager and world == 1
     graphs = {}
     if use_graphs:
         try:
             for name, fn in (("step", whole_step), ("quantize_error_rank", leg_quant), ("lora_down", leg_down),
-                             ("fwd", leg_fwd), ("bwd", leg_bwd)):
+                             ("fwd", leg_fwd), ("bwd", leg_bwd), ("fwd_bwd", fwd_bwd)):
                 gr = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(gr):
                     fn()
@@ -389,8 +438,8 @@ def gpu_main(args):
         else:
             fn()
 
-    step_ms, legs = [], {"quantize_error_rank": [], "lora_down": [], "fwd": [], "bwd": [], "fwd_gemm": [],
-                         "dx_gemm": []}
+    step_ms, legs = [], {"quantize_error_rank": [], "lora_down": [], "fwd": [], "bwd": [], "fwd_bwd": [],
+                         "fwd_gemm": [], "dx_gemm": []}
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -408,7 +457,7 @@ def gpu_main(args):
         legs["dx_gemm"].append(prof[2].elapsed_time(prof[3]))
     clk = clocks.stop()
     for name, fn in (("quantize_error_rank", leg_quant), ("lora_down", leg_down), ("fwd", leg_fwd),
-                     ("bwd", leg_bwd)):
+                     ("bwd", leg_bwd), ("fwd_bwd", fwd_bwd)):
         for i in range(max(5, min(args.steps, 50))):
             flush.zero_()
             ev[2].record(stream)
@@ -458,6 +507,9 @@ def gpu_main(args):
                                 "frac_hbm": qer_bytes / (med["quantize_error_rank"] * 1e-3) / 1e9 / peaks["hbm"]},
         "lora_down": {"ms": med["lora_down"], "note": "T = X L1; in the step it runs beside the allocation pass"},
         "fwd": {"ms": med["fwd"], "note": "with T given"}, "bwd": {"ms": med["bwd"]},
+        "fwd_bwd": {"ms": med["fwd_bwd"], "TFLOP/s": fl / (med["fwd_bwd"] * 1e-3) / 1e12,
+                    "frac_of_burst": fl / (med["fwd_bwd"] * 1e-3) / 1e12 / peaks["bf16"],
+                    "note": "T, forward and backward of the linear without the allocation pass"},
         "fwd_gemm": {"ms": med["fwd_gemm"], "TFLOP/s": fwd_tf}, "dx_gemm": {"ms": med["dx_gemm"], "TFLOP/s": dx_tf},
     }
 
@@ -504,6 +556,9 @@ def gpu_main(args):
     hbm = None
     if rank == 0 and world == 1 and not args.no_hbm_legs:
         hbm = hbm_legs(api, synth, torch, dev, stream, peaks, layers=args.hbm_layers)
+    mlp = None
+    if rank == 0 and world == 1 and not args.no_mlp_leg:
+        mlp = mlp_leg(api, synth, torch, dev, peaks)
 
     # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
@@ -516,7 +571,7 @@ def gpu_main(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args, world),
-            "roofline": roofline, "gemm_pairs": int(lib.qlora_pair_clusters()), "legs": legs_out, "hbm_legs": hbm, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "gemm_pairs": int(lib.qlora_pair_clusters()), "legs": legs_out, "mlp": mlp, "hbm_legs": hbm, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
             "timing": "cuda-graph replay of the step" if use_graphs else "eager API calls",
             "peaks": {"bf16_tflops": peaks["bf16"], "bf16_tflops_sustained": peaks["bf16_sus"],
@@ -541,6 +596,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-hbm-legs", action="store_true", help="skip the full-stack quantizer / error-pass legs")
+    ap.add_argument("--no-mlp-leg", action="store_true", help="skip the Llama-7B MLP (gate, up, down) fwd+bwd leg")
     ap.add_argument("--hbm-layers", type=int, default=32, help="decoder layers of the stack for those legs")
     ap.add_argument("--hbm-only", action="store_true",
                     help="run only the full-stack codec legs and print them (for profiler captures)")
