@@ -53,6 +53,14 @@ def merged_weight(W_s, L1, L2, s: float) -> np.ndarray:
     return f64(W_s) + s * (f64(L1) @ f64(L2)).T
 
 
+def merged_weight_bf16_bits(W_s, L1, L2, s: float) -> np.ndarray:
+    """The merged weight stored in bf16: each element of merged_weight rounded once,
+    to nearest even (reading: the merge is formed exactly and stored in the compute
+    dtype; a negative s unmerges)."""
+    from oracle import nf4
+    return nf4.bf16_bits_from_f64(merged_weight(W_s, L1, L2, s))
+
+
 def trainable_params(h: int, o: int, r: int) -> int:
     """LoRA parameter count r (h + o) ([LoRA-blog] "How much smaller is the trainable part?")."""
     return r * (h + o)

@@ -124,6 +124,21 @@ def bf16_bits_from_f32(x: np.ndarray) -> np.ndarray:
     return out.astype(np.uint16)
 
 
+def bf16_bits_from_f64(x: np.ndarray) -> np.ndarray:
+    """fp64 -> bf16 bit patterns with one rounding (to nearest, ties to even), not
+    through fp32: x = m 2^e (frexp); the bf16 quantum is 2^(e - 8), and 2^-133 below
+    the normal range; rint (ties to even) on the exactly scaled value, then the
+    result (a bf16 value, or an overflow to inf) is read through fp32."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)
+    q = np.maximum(e.astype(np.int64) - 8, -133)
+    with np.errstate(over="ignore", invalid="ignore"):
+        v = np.ldexp(np.rint(np.ldexp(x, -q)), q)
+        f = v.astype(np.float32)
+    out = (f.view(np.uint32) >> 16).astype(np.uint16)
+    return np.where(np.isnan(x), np.uint16(0x7FC0), out).astype(np.uint16)
+
+
 def f32_from_bf16_bits(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
 

@@ -7,7 +7,7 @@ differences, adjoint identities and the pages' parameter counts.
 import numpy as np
 import pytest
 
-from oracle import lora
+from oracle import lora, nf4
 from tests.conftest import load_golden
 
 
@@ -151,3 +151,17 @@ def test_pins_catch_planted_mistakes():
         pin_backward_fd(bwd=bwd_sign_slip)
     with pytest.raises(AssertionError):
         pin_backward_fd(bwd=bwd_dropped_term)
+
+
+def test_merged_bf16_is_the_rounded_merge():
+    """merged_weight_bf16_bits rounds merged_weight once; merging with s and then -s
+    from an exact merge returns the weight; a zero adapter merges to the weight."""
+    rng = np.random.default_rng(7)
+    W = nf4.f32_from_bf16_bits(nf4.bf16_bits_from_f32(rng.standard_normal((32, 64)).astype(np.float32) * 0.02))
+    L1 = nf4.f32_from_bf16_bits(nf4.bf16_bits_from_f32(rng.standard_normal((64, 4)).astype(np.float32) * 0.01))
+    L2 = nf4.f32_from_bf16_bits(nf4.bf16_bits_from_f32(rng.standard_normal((4, 32)).astype(np.float32) * 0.01))
+    Wm = lora.merged_weight(W, L1, L2, 2.0)
+    assert np.array_equal(lora.merged_weight_bf16_bits(W, L1, L2, 2.0), nf4.bf16_bits_from_f64(Wm))
+    assert np.array_equal(lora.merged_weight(Wm, L1, L2, -2.0), W.astype(np.float64))
+    zero = np.zeros_like(L2)
+    assert np.array_equal(lora.merged_weight_bf16_bits(W, L1, zero, 2.0), nf4.bf16_bits_from_f32(W))

@@ -297,3 +297,45 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     with pytest.raises(AssertionError):
         pin_bruteforce_codes(np.concatenate([MID, -MID]))
     monkeypatch.setattr(nf4, "code_indices", orig_ci)
+
+
+def _bf16_rne_exact(x: float) -> int:
+    """Round a float (exactly, as a rational) to bf16 with ties to even, by brute
+    force over the two neighbouring bf16 values."""
+    from fractions import Fraction
+    v = Fraction(x)
+    lo_bits = int(nf4.bf16_bits_from_f32(np.array([np.float32(x)], np.float32))[0])
+    cands = {lo_bits, (lo_bits + 1) & 0xFFFF, (lo_bits - 1) & 0xFFFF}
+    best = None
+    for b in cands:
+        f = float(nf4.f32_from_bf16_bits(np.array([b], np.uint16))[0])
+        if not np.isfinite(f):
+            continue
+        d = abs(Fraction(f) - v)
+        key = (d, b & 1)
+        if best is None or key < best[0]:
+            best = (key, b)
+    return best[1]
+
+
+def test_bf16_from_f64_rounds_once():
+    """fp64 -> bf16 in one rounding: equal to the fp32 route when the value is an fp32
+    number, equal to brute force on random fp64 values, and right where the fp32
+    route rounds twice (a value just above a bf16 midpoint that fp32 rounds onto it)."""
+    rng = np.random.default_rng(5)
+    f = rng.standard_normal(20000).astype(np.float32) * np.float32(2.0) ** rng.integers(-30, 30, 20000)
+    assert np.array_equal(nf4.bf16_bits_from_f64(f.astype(np.float64)), nf4.bf16_bits_from_f32(f))
+    x = rng.standard_normal(3000) * 2.0 ** rng.integers(-20, 20, 3000)
+    got = nf4.bf16_bits_from_f64(x)
+    for xi, g in zip(x[:3000], got[:3000]):
+        assert int(g) == _bf16_rne_exact(float(xi)), xi
+    # 1 + 2^-8 (a bf16 midpoint) + 2^-30: rounds up in one step; via fp32 it would first
+    # land exactly on the midpoint and then go to the even neighbour, 1.0
+    y = 1.0 + 2.0 ** -8 + 2.0 ** -30
+    assert int(nf4.bf16_bits_from_f64(np.array([y]))[0]) == 0x3F81
+    assert int(nf4.bf16_bits_from_f32(np.array([np.float32(y)]))[0]) == 0x3F80
+    # exact midpoints go to the even neighbour; the subnormal range and zero signs
+    assert int(nf4.bf16_bits_from_f64(np.array([1.0 + 2.0 ** -8]))[0]) == 0x3F80
+    assert int(nf4.bf16_bits_from_f64(np.array([1.0 + 3 * 2.0 ** -8]))[0]) == 0x3F82
+    assert int(nf4.bf16_bits_from_f64(np.array([3 * 2.0 ** -134]))[0]) == 0x0002
+    assert int(nf4.bf16_bits_from_f64(np.array([-0.0]))[0]) == 0x8000
