@@ -317,6 +317,73 @@ def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int =
             "timing": f"CUDA-graph replay, best of {reps} (inputs {numel * 2 / 1e9:.2f} GB, above L2)"}
 
 
+def merge_leg(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int = 4, r: int = 16):
+    """LoRA merge (W_hat + s (L1 L2)^T, bf16 out) and merge + NF4 re-quantization over
+    the first `layers` decoder layers of the Llama-7B-shaped stack (7 matrices per
+    layer), weights NF4 with double quant, r = 16, alpha = 32."""
+    mats = synth.stack_matrices(n_layers=layers)
+    Ws = [synth.stack_weight(m, device=str(dev)) for m in mats]
+    ws = api.quantize_batch(Ws, double_quant=True)
+    numel = sum(w.numel() for w in Ws)
+    del Ws
+    torch.cuda.empty_cache()
+    ads = [(synth.normal_bf16((m.inp, r), 0.01, 0, synth.STREAM_L1, m.index, str(dev)),
+            synth.normal_bf16((r, m.out), 0.01, 0, synth.STREAM_L2, m.index, str(dev))) for m in mats]
+    nb = numel // 64
+    l_bytes = sum(2 * r * (m.inp + m.out) for m in mats)
+    in_bytes = numel // 2 + nb + 4 * ((nb + 255) // 256) + l_bytes  # codes, e4m3 scales, group scales, adapters
+    m_bytes = in_bytes + 2 * numel                                    # + bf16 merged weight out
+    rq_bytes = in_bytes + numel // 2 + nb + 4 * ((nb + 255) // 256)   # + re-quantized codes and scales out
+    flops = 2.0 * r * numel                                           # fp64 rank sums
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def merge():
+        for w, (L1, L2) in zip(ws, ads):
+            api.lora_merge(w, L1, L2, 2.0)
+
+    def merge_rq():
+        for w, (L1, L2) in zip(ws, ads):
+            api.lora_merge_requantize(w, L1, L2, 2.0, double_quant=True)
+
+    # warm-up and capture on one stream, so the re-quantize workspace (the bf16 merged
+    # weight, keyed by stream) is allocated before the capture and not inside the graph
+    cap = torch.cuda.Stream(device=dev)
+    times = {}
+    for name, fn in (("m", merge), ("rq", merge_rq)):
+        with torch.cuda.stream(cap):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for i in range(reps + 1):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            e1.synchronize()
+            if i:
+                ts.append(e0.elapsed_time(e1))
+        times[name] = min(ts)
+        del g
+    assert api.status() == 0, "device status set in the merge legs"
+    del ws, ads
+    torch.cuda.empty_cache()
+    mm, rm = times["m"], times["rq"]
+    return {"workload": f"llama7b stack, first {layers} layers: {len(mats)} matrices, {numel / 1e9:.2f} G weights, "
+                        f"NF4 with double quant, r={r}, s=2",
+            "merge": {"ms": mm, "bytes": m_bytes, "GB/s": m_bytes / (mm * 1e-3) / 1e9,
+                      "frac_hbm": m_bytes / (mm * 1e-3) / 1e9 / peaks["hbm"],
+                      "fp64_TFLOP/s": flops / (mm * 1e-3) / 1e12, "launches": len(mats)},
+            "merge_requantize": {"ms": rm, "bytes": rq_bytes, "GB/s": rq_bytes / (rm * 1e-3) / 1e9,
+                                 "frac_hbm": rq_bytes / (rm * 1e-3) / 1e9 / peaks["hbm"],
+                                 "fp64_TFLOP/s": flops / (rm * 1e-3) / 1e12, "launches": 2 * len(mats),
+                                 "note": "NF4 in, NF4 out: each block is quantized where it is merged (exact "
+                                         "fp32 scales to a scratch array), then one double-quant pass over the scales"},
+            "timing": f"CUDA-graph replay, best of {reps} (outputs {2 * numel / 1e9:.2f} GB, above L2)"}
+
+
 def gpu_main(args):
     import ctypes
 
@@ -335,6 +402,10 @@ def gpu_main(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     lib = _lib.load()
     peaks = load_peaks()
+    if args.merge_only:   # the merge legs alone (profiling aid; not a bench line)
+        print(json.dumps({"merge": merge_leg(api, synth, torch, dev, torch.cuda.current_stream(), peaks,
+                                             layers=args.merge_layers)}), flush=True)
+        return
     if args.hbm_only:   # the codec legs alone (profiling aid; not a bench line)
         print(json.dumps({"hbm_legs": hbm_legs(api, synth, torch, dev, torch.cuda.current_stream(), peaks,
                                                 layers=args.hbm_layers)}), flush=True)
@@ -559,6 +630,9 @@ def gpu_main(args):
     mlp = None
     if rank == 0 and world == 1 and not args.no_mlp_leg:
         mlp = mlp_leg(api, synth, torch, dev, peaks)
+    merge = None
+    if rank == 0 and world == 1 and not args.no_merge_leg:
+        merge = merge_leg(api, synth, torch, dev, stream, peaks, layers=args.merge_layers)
 
     # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
@@ -571,7 +645,7 @@ def gpu_main(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args, world),
-            "roofline": roofline, "gemm_pairs": int(lib.qlora_pair_clusters()), "legs": legs_out, "mlp": mlp, "hbm_legs": hbm, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "gemm_pairs": int(lib.qlora_pair_clusters()), "legs": legs_out, "mlp": mlp, "hbm_legs": hbm, "merge": merge, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
             "timing": "cuda-graph replay of the step" if use_graphs else "eager API calls",
             "peaks": {"bf16_tflops": peaks["bf16"], "bf16_tflops_sustained": peaks["bf16_sus"],
@@ -597,6 +671,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-hbm-legs", action="store_true", help="skip the full-stack quantizer / error-pass legs")
     ap.add_argument("--no-mlp-leg", action="store_true", help="skip the Llama-7B MLP (gate, up, down) fwd+bwd leg")
+    ap.add_argument("--no-merge-leg", action="store_true", help="skip the LoRA merge / merge + re-quantize leg")
+    ap.add_argument("--merge-layers", type=int, default=4, help="decoder layers of the stack for the merge leg")
+    ap.add_argument("--merge-only", action="store_true",
+                    help="run only the merge legs and print them (profiling aid; not a bench line)")
     ap.add_argument("--hbm-layers", type=int, default=32, help="decoder layers of the stack for those legs")
     ap.add_argument("--hbm-only", action="store_true",
                     help="run only the full-stack codec legs and print them (for profiler captures)")

@@ -164,6 +164,37 @@ qlora_status nf4_quantize_batch(int32_t n, const uint16_t* const* W_ptrs, const 
  *   W_out  device out, bf16 [out*in], 16-byte aligned */
 qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream_t stream);
 
+/* ------------------------------------------------------------ LoRA merge */
+
+/* Merging the adapter into the frozen weight after training ("LoRA: Fine-tuning a
+ * model by learning a small update", section "Serving models and switching tasks":
+ * W_merged = W_0 + (alpha / r) B A, no extra inference latency; "QLoRA: How to
+ * fine-tune large language models with less memory", eq. (3)), in the stored
+ * out x in layout:
+ *   W_out = bf16_rn(W_hat + s (L1 L2)^T)
+ * with W_hat the dequantized NF4 weight (bf16_rn(fp32_rn(code * scale)), as
+ * nf4_dequantize) or the protected bf16 one. The rank-r product is summed in fp64
+ * and the sum rounded to bf16 once (exact for bf16 adapters and weights of ordinary
+ * ranges: every product is exact in fp64). A negative scale unmerges.
+ *   w      host pointer to the weight descriptor; in % 64 == 0
+ *   L1     device bf16 [in x r]     L2 device bf16 [r x out]     1 <= r <= 256
+ *   W_out  device out, bf16 [out x in], 16-byte aligned
+ * qlora_lora_merge_requantize NF4-quantizes the merged bf16 weight exactly as
+ * nf4_quantize would (codes / scales laid out as there; config q) without storing
+ * it: each 64-block is quantized where it is merged, then the scales are
+ * double-quantized when q.double_quant is set. absmax (fp32 [out*in/64]) may be
+ * NULL with double quant; the exact scales then live in the workspace
+ * (qlora_lora_merge_requantize_workspace_size bytes, 16-byte aligned; its first
+ * bytes are the status word, which gets QLORA_ERR_NONFINITE if a merged value is
+ * not finite). */
+qlora_status qlora_lora_merge(const qlora_weight* w, const uint16_t* L1, const uint16_t* L2, int32_t r, float scale,
+                              uint16_t* W_out, qlora_stream_t stream);
+size_t qlora_lora_merge_requantize_workspace_size(int64_t out, int64_t in);
+qlora_status qlora_lora_merge_requantize(const qlora_weight* w, const uint16_t* L1, const uint16_t* L2, int32_t r,
+                                         float scale, nf4_qconfig q, uint8_t* codes, float* absmax,
+                                         uint8_t* absmax_q, float* absmax2, void* workspace,
+                                         size_t workspace_bytes, qlora_stream_t stream);
+
 /* --------------------------------------------------------- NF4-LoRA linear */
 
 /* Shape rules for the linear: in % 256 == 0, out % 256 == 0, 1 <= M <= 2^21,

@@ -44,6 +44,10 @@ SIGNATURES = {
                                    POINTER(c_void_p), POINTER(c_void_p), POINTER(c_void_p), POINTER(c_void_p),
                                    c_void_p, c_size_t, c_void_p]),
     "nf4_dequantize": (c_int, [POINTER(QLoraWeight), c_void_p, c_void_p]),
+    "qlora_lora_merge": (c_int, [POINTER(QLoraWeight), c_void_p, c_void_p, c_int32, c_float, c_void_p, c_void_p]),
+    "qlora_lora_merge_requantize_workspace_size": (c_size_t, [c_int64, c_int64]),
+    "qlora_lora_merge_requantize": (c_int, [POINTER(QLoraWeight), c_void_p, c_void_p, c_int32, c_float, NF4QConfig,
+                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "qlora_fwd_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int32]),
     "qlora_bwd_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, c_int32]),
     "qlora_linear_fwd": (c_int, [POINTER(QLoraWeight), c_void_p, c_int64, c_void_p, c_void_p, c_int32, c_float,

@@ -173,6 +173,42 @@ def dequantize(w: NF4Weight) -> torch.Tensor:
     return out
 
 
+def lora_merge(w: NF4Weight, L1: torch.Tensor, L2: torch.Tensor, scale: float) -> torch.Tensor:
+    """bf16 [out x in] = W_hat + scale (L1 L2)^T (a negative scale unmerges)."""
+    _need(L1, torch.bfloat16, "L1")
+    _need(L2, torch.bfloat16, "L2")
+    lib = _lib.load()
+    dev = L1.device
+    out = torch.empty((w.out, w.inp), dtype=torch.bfloat16, device=dev)
+    cs = w.c_struct()
+    check(lib.qlora_lora_merge(ctypes.byref(cs), _ptr(L1), _ptr(L2), L1.shape[1], float(scale), _ptr(out), _stream()),
+          "qlora_lora_merge")
+    return out
+
+
+def lora_merge_requantize(w: NF4Weight, L1: torch.Tensor, L2: torch.Tensor, scale: float,
+                          double_quant: bool = False, keep_absmax: bool = False) -> NF4Weight:
+    """The merged weight W_hat + scale (L1 L2)^T, NF4-quantized as quantize() would."""
+    _need(L1, torch.bfloat16, "L1")
+    _need(L2, torch.bfloat16, "L2")
+    lib = _lib.load()
+    dev = L1.device
+    n = w.out * w.inp
+    nb = (n + 63) // 64
+    o = NF4Weight(w.out, w.inp, double_quant,
+                  codes=torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev),
+                  absmax=torch.empty(nb, dtype=torch.float32, device=dev) if (not double_quant or keep_absmax) else None,
+                  absmax_q=torch.empty(nb, dtype=torch.uint8, device=dev) if double_quant else None,
+                  absmax2=torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev) if double_quant else None)
+    ws = Workspace.get(lib.qlora_lora_merge_requantize_workspace_size(w.out, w.inp), dev)
+    cs = w.c_struct()
+    check(lib.qlora_lora_merge_requantize(ctypes.byref(cs), _ptr(L1), _ptr(L2), L1.shape[1], float(scale),
+                                          NF4QConfig(64, 1 if double_quant else 0, 256), _ptr(o.codes),
+                                          _ptr(o.absmax), _ptr(o.absmax_q), _ptr(o.absmax2), _ptr(ws), ws.numel(),
+                                          _stream()), "qlora_lora_merge_requantize")
+    return o
+
+
 def linear_fwd(w: NF4Weight, X: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, scale: float,
                save_T: bool = True, Y: Optional[torch.Tensor] = None,
                T: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:

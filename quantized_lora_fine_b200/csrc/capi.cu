@@ -475,6 +475,65 @@ qlora_status nf4_quantize_batch(int32_t n, const uint16_t* const* W_ptrs, const 
                                static_cast<int*>(workspace), S(stream));
 }
 
+namespace {
+qlora_status check_merge(const qlora_weight* w, const uint16_t* L1, const uint16_t* L2, int32_t r) {
+  if (!w || !L1 || !L2) return QLORA_ERR_NULL;
+  if (w->out <= 0 || w->in <= 0 || w->in % 64) return QLORA_ERR_SHAPE;
+  if (w->in > (int64_t(1) << 30) || w->out > (int64_t(1) << 30)) return QLORA_ERR_SHAPE;
+  if (w->in / 64 > 65535 * int64_t(1) || (w->out + 63) / 64 > 65535) return QLORA_ERR_SHAPE;
+  if (r < 1 || r > 256) return QLORA_ERR_SHAPE;
+  if (w->is_bf16) {
+    if (!w->w_bf16) return QLORA_ERR_NULL;
+    if (!aligned16(w->w_bf16)) return QLORA_ERR_ALIGN;
+  } else {
+    if (!qconfig_ok(w->q)) return QLORA_ERR_UNSUPPORTED;
+    if (!w->codes || (w->q.double_quant ? (!w->absmax_q || !w->absmax2) : !w->absmax)) return QLORA_ERR_NULL;
+    if (!aligned16(w->codes)) return QLORA_ERR_ALIGN;
+  }
+  return QLORA_OK;
+}
+
+qlora_status merge_into(const qlora_weight* w, const uint16_t* L1, const uint16_t* L2, int32_t r, float scale,
+                        uint16_t* W_out, uint8_t* q_codes, float* q_absmax, int* status, cudaStream_t s) {
+  return launch_lora_merge(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0,
+                           w->is_bf16 ? w->w_bf16 : nullptr, w->out, w->in, L1, L2, r, double(scale), W_out, q_codes,
+                           q_absmax, status, s);
+}
+}  // namespace
+
+qlora_status qlora_lora_merge(const qlora_weight* w, const uint16_t* L1, const uint16_t* L2, int32_t r, float scale,
+                              uint16_t* W_out, qlora_stream_t stream) {
+  QLB_TRY(check_merge(w, L1, L2, r));
+  if (!W_out) return QLORA_ERR_NULL;
+  if (!aligned16(W_out)) return QLORA_ERR_ALIGN;
+  QLB_TRY(check_device());
+  return merge_into(w, L1, L2, r, scale, W_out, nullptr, nullptr, nullptr, S(stream));
+}
+
+size_t qlora_lora_merge_requantize_workspace_size(int64_t out, int64_t in) {
+  if (out <= 0 || in <= 0) return 0;
+  return kStatusBytes + up256(size_t(out) * size_t(in / 64) * sizeof(float));
+}
+
+qlora_status qlora_lora_merge_requantize(const qlora_weight* w, const uint16_t* L1, const uint16_t* L2, int32_t r,
+                                         float scale, nf4_qconfig q, uint8_t* codes, float* absmax,
+                                         uint8_t* absmax_q, float* absmax2, void* workspace,
+                                         size_t workspace_bytes, qlora_stream_t stream) {
+  QLB_TRY(check_merge(w, L1, L2, r));
+  if (!qconfig_ok(q)) return QLORA_ERR_UNSUPPORTED;
+  if (!codes || (q.double_quant ? (!absmax_q || !absmax2) : !absmax)) return QLORA_ERR_NULL;
+  if (!aligned16(codes)) return QLORA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < qlora_lora_merge_requantize_workspace_size(w->out, w->in))
+    return QLORA_ERR_WORKSPACE;
+  QLB_TRY(check_device());
+  // the exact fp32 scales go to the caller's absmax when given, else to the workspace
+  float* amax = absmax ? absmax : reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  QLB_TRY(merge_into(w, L1, L2, r, scale, nullptr, codes, amax, static_cast<int*>(workspace), S(stream)));
+  if (q.double_quant) return launch_dq_scales(amax, w->out * (w->in / 64), absmax_q, absmax2, S(stream));
+  return QLORA_OK;
+}
+
 qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream_t stream) {
   if (!w || !W_out) return QLORA_ERR_NULL;
   if (w->is_bf16) return QLORA_ERR_UNSUPPORTED;

@@ -384,6 +384,237 @@ qlora_status launch_dequantize(const uint8_t* codes, const float* absmax, const 
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ LoRA merge
+//
+// W_out = bf16_rn(W_hat + s (L1 L2)^T) in the stored out x in layout, W_hat the
+// dequantized NF4 weight (or the protected bf16 one). The rank-r product is summed in
+// fp64 (the products of bf16 values are exact there, and so are the sums for weights
+// and adapters of ordinary ranges) and rounded to bf16 once.
+//
+// One CTA per 128 x 64 tile (rows n, columns k; each tile row is one NF4 block);
+// thread (tn, tk) = (tid / 8, tid % 8) owns rows 4 tn .. 4 tn + 3 and columns
+// 8 tk .. 8 tk + 7, so the 8 lanes of a block are 8 consecutive lanes of one warp.
+// The adapter slices of the tile go through shared memory 16 ranks at a time, as
+// fp64: L1 as [q][k], L2 as [q][n]. Per rank a thread reads its 8 L1 values as four
+// 16-byte pieces and its 4 L2 values as two; the pieces of each 8-column group are
+// stored rotated by (group / 2) so that the 8 groups a warp reads at once sit in 8
+// different 16-byte bank groups (no conflicts), and the 4 row groups of a warp read
+// 64 contiguous bytes. 32 fp64 FMAs per 6 shared loads.
+//
+// The tile's weight (32 code bytes or 128 bf16 bytes per row) is copied to shared
+// memory by cp.async when the CTA starts and the block scales are read into
+// registers, so their latency hides behind the adapter loads and the fp64 loop.
+//
+// QUANT epilogue: the merged block is NF4-quantized in place of the bf16 store, with
+// the quantizer's rule (absmax over the block's 64 merged bf16 values by shuffles
+// among its 8 lanes, IEEE quotient, nearest code by midpoint count, element 2k in
+// the high nibble of byte k); codes always use the exact fp32 absmax, which goes to
+// `q_absmax` for the double-quant pass.
+constexpr int kMergeRows = 128, kMergeCols = 64, kMergeQ = 16;
+
+struct MergeArgs {
+  const uint8_t* codes;
+  const float* absmax;
+  const uint8_t* absmax_q;
+  const float* absmax2;
+  int dq;
+  const uint16_t* Wbf;        // protected bf16 weight, or null
+  int64_t out, in;
+  const uint16_t* L1;         // in x r
+  const uint16_t* L2;         // r x out
+  int r;
+  double s;
+  uint16_t* W_out;            // bf16 out x in (bf16 epilogue)
+  uint8_t* q_codes;           // NF4 codes out (QUANT epilogue)
+  float* q_absmax;            // fp32 absmax out (QUANT epilogue)
+  int* status;
+};
+
+__device__ __forceinline__ double bf16_to_f64(uint16_t b) { return double(__uint_as_float(uint32_t(b) << 16)); }
+
+// Position of column k of an 8-column group inside its shared-memory row: the four
+// 2-column pieces of group g are stored rotated by g / 2.
+__device__ __forceinline__ int merge_col_slot(int k) {
+  const int g = k >> 3, p = (k >> 1) & 3;
+  return (g << 3) | (((p + (g >> 1)) & 3) << 1) | (k & 1);
+}
+
+template <bool BF16W, bool QUANT>
+__global__ void __launch_bounds__(256, 2) lora_merge_kernel(const __grid_constant__ MergeArgs m) {
+  __shared__ __align__(16) double s_a[kMergeQ][kMergeCols];   // L1 slice, [q][slot(k)]
+  __shared__ __align__(16) double s_b[kMergeQ][kMergeRows];   // L2 slice, [q][n]
+  constexpr int kRowBytes = BF16W ? kMergeCols * 2 : kMergeCols / 2;
+  __shared__ __align__(16) uint8_t s_w[kMergeRows * kRowBytes];  // the tile's weight rows
+  pdl_wait();
+  pdl_launch();
+  const int tid = threadIdx.x, tn = tid >> 3, tk = tid & 7;
+  const int64_t n0 = int64_t(blockIdx.y) * kMergeRows, k0 = int64_t(blockIdx.x) * kMergeCols;
+  const int r = m.r;
+  {
+    constexpr int kPieces = kRowBytes / 16;   // 16-byte pieces per row: 8 (bf16) or 2 (codes)
+    const uint8_t* src = BF16W ? reinterpret_cast<const uint8_t*>(m.Wbf) : m.codes;
+#pragma unroll
+    for (int j = 0; j < kMergeRows * kPieces / 256; ++j) {
+      const int i = tid + 256 * j, row = i / kPieces, piece = i % kPieces;
+      if (n0 + row < m.out)
+        cp_async16(smem_u32(s_w + row * kRowBytes + piece * 16),
+                   src + ((n0 + row) * m.in + k0) * kRowBytes / kMergeCols + piece * 16);
+    }
+  }
+  float scale[4] = {0.f, 0.f, 0.f, 0.f};
+  if constexpr (!BF16W) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t n = n0 + 4 * tn + i;
+      if (n < m.out) scale[i] = block_scale((n * m.in + k0) / kBlock, m.absmax, m.absmax_q, m.absmax2, m.dq != 0);
+    }
+  }
+  double acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+  for (int q0 = 0; q0 < r; q0 += kMergeQ) {
+    const int qn = min(kMergeQ, r - q0);
+#pragma unroll
+    for (int j = 0; j < kMergeQ * kMergeCols / 256; ++j) {
+      const int i = tid + 256 * j, q = i >> 6, k = i & 63;
+      s_a[q][merge_col_slot(k)] = (q < qn) ? bf16_to_f64(m.L1[(k0 + k) * r + q0 + q]) : 0.0;
+    }
+#pragma unroll
+    for (int j = 0; j < kMergeQ * kMergeRows / 256; ++j) {
+      const int i = tid + 256 * j, q = i >> 7, n = i & 127;
+      s_b[q][n] = (q < qn && n0 + n < m.out) ? bf16_to_f64(m.L2[int64_t(q0 + q) * m.out + n0 + n]) : 0.0;
+    }
+    __syncthreads();
+    const double2* ra = reinterpret_cast<const double2*>(&s_a[0][8 * tk]);
+    const double2* rb = reinterpret_cast<const double2*>(&s_b[0][4 * tn]);
+    const int rot = tk >> 1;
+    for (int q = 0; q < qn; ++q) {
+      double a[8];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const double2 v = ra[q * (kMergeCols / 2) + ((p + rot) & 3)];
+        a[2 * p] = v.x;
+        a[2 * p + 1] = v.y;
+      }
+      const double2 b01 = rb[q * (kMergeRows / 2)], b23 = rb[q * (kMergeRows / 2) + 1];
+      const double b[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[j], b[i], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = 4 * tn + i;
+    const int64_t n = n0 + row;
+    const bool live = n < m.out;                              // same for the 8 lanes of a block
+    const int64_t e = n * m.in + k0 + 8 * tk;                 // first of this thread's 8 elements
+    uint4 wv = make_uint4(0u, 0u, 0u, 0u);
+    if (live) {
+      if constexpr (BF16W) {
+        wv = *reinterpret_cast<const uint4*>(s_w + row * kRowBytes + 16 * tk);
+      } else {
+        wv = nf4_dequant_word(*reinterpret_cast<const uint32_t*>(s_w + row * kRowBytes + 4 * tk),
+                              nf4_make_lut(scale[i]));
+      }
+    }
+    const uint32_t wh[4] = {wv.x, wv.y, wv.z, wv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      uint16_t lo, hi;
+      const double v0 = double(__uint_as_float(wh[p] << 16)) + m.s * acc[i][2 * p];
+      const double v1 = double(__uint_as_float(wh[p] & 0xFFFF0000u)) + m.s * acc[i][2 * p + 1];
+      asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(lo) : "d"(v0));
+      asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(hi) : "d"(v1));
+      o[p] = live ? (uint32_t(lo) | (uint32_t(hi) << 16)) : 0u;
+    }
+    if constexpr (!QUANT) {
+      if (live) *reinterpret_cast<uint4*>(m.W_out + e) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+      float w[8];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        w[2 * p] = bf16_lo(o[p]);
+        w[2 * p + 1] = bf16_hi(o[p]);
+      }
+      float am = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float aw = fabsf(w[j]);
+        bad |= !(aw <= FLT_MAX);
+        am = fmaxf(am, aw);
+      }
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+      if (live) {
+        const bool use = am > 0.f && am <= FLT_MAX;
+        uint32_t word = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t hi_idx = use ? nf4_index(__fdiv_rn(w[2 * k], am)) : 7u;
+          const uint32_t lo_idx = use ? nf4_index(__fdiv_rn(w[2 * k + 1], am)) : 7u;
+          word |= ((hi_idx << 4) | lo_idx) << (8 * k);
+        }
+        *reinterpret_cast<uint32_t*>(m.q_codes + e / 2) = word;
+        if (tk == 0) m.q_absmax[e / kBlock] = am;
+      }
+    }
+  }
+  if constexpr (QUANT) {
+    if (bad) set_status(m.status, QLORA_ERR_NONFINITE);
+  }
+}
+
+// Double quantization of a finished absmax array: one CTA of 256 threads per group
+// of 256 scales, the same arithmetic as the quantizer's own double-quant tail.
+__global__ void __launch_bounds__(256) dq_scales_kernel(const float* __restrict__ absmax, int64_t nb,
+                                                        uint8_t* __restrict__ absmax_q,
+                                                        float* __restrict__ absmax2) {
+  __shared__ float s_amax[kDQBlock];
+  __shared__ float s_red[8];
+  pdl_wait();
+  pdl_launch();
+  const int64_t g = blockIdx.x;
+  const int64_t b = g * kDQBlock + threadIdx.x;
+  s_amax[threadIdx.x] = b < nb ? absmax[b] : 0.f;
+  dq_group(s_amax, s_red, nb, g, absmax_q, absmax2);
+}
+
+qlora_status launch_lora_merge(const uint8_t* codes, const float* absmax, const uint8_t* absmax_q,
+                               const float* absmax2, bool dq, const uint16_t* Wbf, int64_t out, int64_t in,
+                               const uint16_t* L1, const uint16_t* L2, int r, double s, uint16_t* W_out,
+                               uint8_t* q_codes, float* q_absmax, int* status, cudaStream_t st) {
+  const MergeArgs m{codes, absmax, absmax_q, absmax2, dq ? 1 : 0, Wbf, out, in, L1, L2, r, s, W_out,
+                    q_codes, q_absmax, status};
+  const dim3 grid(unsigned(in / kMergeCols), unsigned((out + kMergeRows - 1) / kMergeRows));
+  const bool quant = q_codes != nullptr;
+  cudaError_t e;
+  if (Wbf)
+    e = quant ? launch_pdl(lora_merge_kernel<true, true>, grid, dim3(256), 0, st, m)
+              : launch_pdl(lora_merge_kernel<true, false>, grid, dim3(256), 0, st, m);
+  else
+    e = quant ? launch_pdl(lora_merge_kernel<false, true>, grid, dim3(256), 0, st, m)
+              : launch_pdl(lora_merge_kernel<false, false>, grid, dim3(256), 0, st, m);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status launch_dq_scales(const float* absmax, int64_t nb, uint8_t* absmax_q, float* absmax2, cudaStream_t st) {
+  const int64_t groups = (nb + kDQBlock - 1) / kDQBlock;
+  if (groups <= 0) return QLORA_OK;
+  const cudaError_t e = launch_pdl(dq_scales_kernel, dim3(unsigned(groups)), dim3(256), 0, st, absmax, nb, absmax_q,
+                                   absmax2);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 // ------------------------------------------------------- expanded GEMM scales
 
 __global__ void expand_scales_kernel(const float* __restrict__ absmax, const uint8_t* __restrict__ absmax_q,

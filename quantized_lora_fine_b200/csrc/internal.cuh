@@ -72,6 +72,16 @@ qlora_status launch_expand_scales(const uint8_t* unused, const float* absmax, co
 // dst[n][q] = bf16(s * src[q][n]), src r x cols (transpose = 1)
 qlora_status launch_scale_lora(const uint16_t* src, int64_t rows, int64_t cols, float scale, bool transpose,
                                uint16_t* dst, cudaStream_t s);
+// W_out = bf16(W_hat + s (L1 L2)^T) (stored layout; W_hat from the NF4 fields, or Wbf
+// when it is non-null); in % 64 == 0. With q_codes non-null the merged weight is
+// NF4-quantized instead of stored: codes to q_codes, exact fp32 absmax to q_absmax,
+// non-finite merged values set QLORA_ERR_NONFINITE in *status.
+qlora_status launch_lora_merge(const uint8_t* codes, const float* absmax, const uint8_t* absmax_q,
+                               const float* absmax2, bool dq, const uint16_t* Wbf, int64_t out, int64_t in,
+                               const uint16_t* L1, const uint16_t* L2, int r, double s, uint16_t* W_out,
+                               uint8_t* q_codes, float* q_absmax, int* status, cudaStream_t st);
+// Double-quantize a finished fp32 absmax array (nb scales, groups of 256).
+qlora_status launch_dq_scales(const float* absmax, int64_t nb, uint8_t* absmax_q, float* absmax2, cudaStream_t st);
 // ---- layer_error.cu
 size_t layer_error_ws_bytes(int n_layers, const int64_t* numel);
 qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,

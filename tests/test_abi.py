@@ -95,6 +95,25 @@ def test_host_validation_before_any_launch(lib):
     assert lib.qlora_lora_down(None, 8, 4096, None, 12, None, None, 0, None) == 2
     assert lib.qlora_linear_fwd_t(ctypes.byref(w), 0x1000, 8, None, 0x1000, 16, 2.0, 0x1000, None, 0, None) == 3
 
+    # merge: in not a multiple of 64, rank out of range, misaligned codes / output, short workspace
+    m = _lib.QLoraWeight()
+    m.out, m.in_, m.q = 128, 100, q
+    m.codes, m.absmax = 0x2000, 0x3000
+    assert lib.qlora_lora_merge(ctypes.byref(m), 0x1000, 0x1000, 8, 2.0, 0x4000, None) == 2
+    m.in_ = 128
+    assert lib.qlora_lora_merge(ctypes.byref(m), 0x1000, 0x1000, 0, 2.0, 0x4000, None) == 2
+    assert lib.qlora_lora_merge(ctypes.byref(m), None, 0x1000, 8, 2.0, 0x4000, None) == 1
+    assert lib.qlora_lora_merge(ctypes.byref(m), 0x1000, 0x1000, 8, 2.0, 0x4001, None) == 3
+    m.codes = 0x2001
+    assert lib.qlora_lora_merge(ctypes.byref(m), 0x1000, 0x1000, 8, 2.0, 0x4000, None) == 3
+    m.codes = 0x2000
+    need = lib.qlora_lora_merge_requantize_workspace_size(128, 128)
+    assert need >= 128 * 2 * 4          # the fp32 scales (status word in front)
+    assert lib.qlora_lora_merge_requantize_workspace_size(0, 128) == 0
+    assert lib.qlora_lora_merge_requantize(ctypes.byref(m), 0x1000, 0x1000, 8, 2.0, q, 0x5000, 0x6000, None, None,
+                                           0x7000, need - 1, None) == 7
+    assert lib.qlora_lora_merge_requantize(ctypes.byref(m), 0x1000, 0x1000, 8, 2.0, q, 0x5000, None, None, None,
+                                           0x7000, need, None) == 1
 
 def test_product_path_refuses_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "_lib", None)
