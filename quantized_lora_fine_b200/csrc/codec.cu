@@ -391,26 +391,40 @@ qlora_status launch_dequantize(const uint8_t* codes, const float* absmax, const 
 // fp64 (the products of bf16 values are exact there, and so are the sums for weights
 // and adapters of ordinary ranges) and rounded to bf16 once.
 //
-// One CTA per 128 x 64 tile (rows n, columns k; each tile row is one NF4 block);
-// thread (tn, tk) = (tid / 8, tid % 8) owns rows 4 tn .. 4 tn + 3 and columns
-// 8 tk .. 8 tk + 7, so the 8 lanes of a block are 8 consecutive lanes of one warp.
-// The adapter slices of the tile go through shared memory 16 ranks at a time, as
-// fp64: L1 as [q][k], L2 as [q][n]. Per rank a thread reads its 8 L1 values as four
-// 16-byte pieces and its 4 L2 values as two; the pieces of each 8-column group are
-// stored rotated by (group / 2) so that the 8 groups a warp reads at once sit in 8
-// different 16-byte bank groups (no conflicts), and the 4 row groups of a warp read
-// 64 contiguous bytes. 32 fp64 FMAs per 6 shared loads.
+// Tiles of 128 x 64 (rows n, columns k; each tile row is one NF4 block); thread
+// (tn, tk) = (tid / 8, tid % 8) owns rows 4 tn .. 4 tn + 3 and columns 8 tk .. 8 tk + 7,
+// so the 8 lanes of a block are 8 consecutive lanes of one warp. The adapter slices
+// of a tile go through shared memory 16 ranks at a time, as fp64: L1 as [q][k], L2
+// as [q][n]. Per rank a thread reads its 8 L1 values as four 16-byte pieces and its
+// 4 L2 values as two; the pieces of each 8-column group are stored rotated by
+// (group / 2) so that the 8 groups a warp reads at once sit in 8 different 16-byte
+// bank groups (no conflicts), and the 4 row groups of a warp read 64 contiguous
+// bytes. 32 fp64 FMAs per 6 shared loads.
 //
-// The tile's weight (32 code bytes or 128 bf16 bytes per row) is copied to shared
-// memory by cp.async when the CTA starts and the block scales are read into
-// registers, so their latency hides behind the adapter loads and the fp64 loop.
+// Persistent: two CTAs per SM walk the work items (tile, 16-rank chunk) of their
+// tiles. While item i is converted to fp64, summed and (after a tile's last chunk)
+// written out, the raw bf16 adapter slices of item i + 1 and, at a tile's first
+// chunk, the tile's weight rows (32 code bytes or 128 bf16 bytes per row) arrive by
+// cp.async in the other buffer. Buffer reuse is ordered by the two barriers of each
+// item: staging buffer (i + 1) % 2 was last read by the conversion of item i - 1,
+// and weight slot j % 2 (j = the CTA's tile count) by the epilogue of tile j - 2;
+// both precede the first barrier of item i, after which the copies are issued.
+// Block scales are read into registers at a tile's first chunk and used in its
+// epilogue.
 //
 // QUANT epilogue: the merged block is NF4-quantized in place of the bf16 store, with
 // the quantizer's rule (absmax over the block's 64 merged bf16 values by shuffles
-// among its 8 lanes, IEEE quotient, nearest code by midpoint count, element 2k in
-// the high nibble of byte k); codes always use the exact fp32 absmax, which goes to
-// `q_absmax` for the double-quant pass.
+// among its 8 lanes; the code the IEEE quotient selects, found as the quantizer finds
+// it; element 2k in the high nibble of byte k); codes always use the exact fp32
+// absmax, which goes to `q_absmax` for the double-quant pass.
 constexpr int kMergeRows = 128, kMergeCols = 64, kMergeQ = 16;
+constexpr int kMergeStageBytes = kMergeCols * kMergeQ * 2 + kMergeQ * kMergeRows * 2;   // raw L1 + L2 chunk
+template <bool BF16W>
+__host__ __device__ constexpr int merge_w_bytes() { return kMergeRows * (BF16W ? kMergeCols * 2 : kMergeCols / 2); }
+template <bool BF16W>
+__host__ __device__ constexpr int merge_smem_bytes() {
+  return (kMergeQ * kMergeCols + kMergeQ * kMergeRows) * 8 + 2 * kMergeStageBytes + 2 * merge_w_bytes<BF16W>();
+}
 
 struct MergeArgs {
   const uint8_t* codes;
@@ -441,56 +455,124 @@ __device__ __forceinline__ int merge_col_slot(int k) {
 
 template <bool BF16W, bool QUANT>
 __global__ void __launch_bounds__(256, 2) lora_merge_kernel(const __grid_constant__ MergeArgs m) {
-  __shared__ __align__(16) double s_a[kMergeQ][kMergeCols];   // L1 slice, [q][slot(k)]
-  __shared__ __align__(16) double s_b[kMergeQ][kMergeRows];   // L2 slice, [q][n]
-  constexpr int kRowBytes = BF16W ? kMergeCols * 2 : kMergeCols / 2;
-  __shared__ __align__(16) uint8_t s_w[kMergeRows * kRowBytes];  // the tile's weight rows
+  extern __shared__ __align__(16) uint8_t smem[];
+  double(*s_a)[kMergeCols] = reinterpret_cast<double(*)[kMergeCols]>(smem);                       // [q][slot(k)]
+  double(*s_b)[kMergeRows] = reinterpret_cast<double(*)[kMergeRows]>(smem + kMergeQ * kMergeCols * 8);  // [q][n]
+  uint8_t* const stage0 = smem + (kMergeQ * kMergeCols + kMergeQ * kMergeRows) * 8;    // 2 x {L1 [k][16], L2 [16][n]}
+  uint8_t* const wbuf0 = stage0 + 2 * kMergeStageBytes;                                // 2 x weight rows
+  constexpr int kRowBytes = merge_w_bytes<BF16W>() / kMergeRows;
   pdl_wait();
   pdl_launch();
   const int tid = threadIdx.x, tn = tid >> 3, tk = tid & 7;
-  const int64_t n0 = int64_t(blockIdx.y) * kMergeRows, k0 = int64_t(blockIdx.x) * kMergeCols;
   const int r = m.r;
-  {
-    constexpr int kPieces = kRowBytes / 16;   // 16-byte pieces per row: 8 (bf16) or 2 (codes)
-    const uint8_t* src = BF16W ? reinterpret_cast<const uint8_t*>(m.Wbf) : m.codes;
-#pragma unroll
-    for (int j = 0; j < kMergeRows * kPieces / 256; ++j) {
-      const int i = tid + 256 * j, row = i / kPieces, piece = i % kPieces;
-      if (n0 + row < m.out)
-        cp_async16(smem_u32(s_w + row * kRowBytes + piece * 16),
-                   src + ((n0 + row) * m.in + k0) * kRowBytes / kMergeCols + piece * 16);
+  const int nchunk = (r + kMergeQ - 1) / kMergeQ;
+  const int64_t tiles_k = m.in / kMergeCols, tiles_n = (m.out + kMergeRows - 1) / kMergeRows;
+  const int64_t my_tiles = (tiles_k * tiles_n - blockIdx.x + gridDim.x - 1) / gridDim.x;
+  const int64_t n_items = my_tiles * nchunk;
+  // 16-byte copies need 16-byte aligned rows: L1 rows are r bf16 long, L2 rows out bf16
+  const bool l1_async = (r % 8) == 0 && (reinterpret_cast<uintptr_t>(m.L1) & 15) == 0;
+  const bool l2_async = (m.out % 8) == 0 && (reinterpret_cast<uintptr_t>(m.L2) & 15) == 0;
+
+  // Copies for item `it` into staging buffer it % 2 (and, at a first chunk, the tile's
+  // weight rows into slot (it / nchunk) % 2); one commit group per item.
+  auto issue = [&](int64_t it) {
+    const int64_t j = it / nchunk;
+    const int c = int(it % nchunk);
+    const int64_t t = blockIdx.x + j * gridDim.x;
+    const int64_t n0 = (t / tiles_k) * kMergeRows, k0 = (t % tiles_k) * kMergeCols;
+    const int q0 = c * kMergeQ, qn = min(kMergeQ, r - q0);
+    uint8_t* st = stage0 + (it & 1) * kMergeStageBytes;
+    uint16_t* st_l1 = reinterpret_cast<uint16_t*>(st);                       // [k][16]
+    uint16_t* st_l2 = reinterpret_cast<uint16_t*>(st + kMergeCols * kMergeQ * 2);   // [16][n]
+    if (l1_async) {
+      // row k: qn ranks = qn / 8 pieces of 16 bytes
+      const int pieces = qn / 8;
+      for (int i = tid; i < kMergeCols * pieces; i += 256) {
+        const int k = i / pieces, pc = i % pieces;
+        cp_async16(smem_u32(st_l1 + k * kMergeQ + pc * 8), m.L1 + (k0 + k) * r + q0 + pc * 8);
+      }
+    } else {
+      for (int i = tid; i < kMergeCols * kMergeQ; i += 256) {
+        const int k = i >> 4, q = i & 15;
+        if (q < qn) st_l1[k * kMergeQ + q] = m.L1[(k0 + k) * r + q0 + q];
+      }
     }
-  }
-  float scale[4] = {0.f, 0.f, 0.f, 0.f};
-  if constexpr (!BF16W) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int64_t n = n0 + 4 * tn + i;
-      if (n < m.out) scale[i] = block_scale((n * m.in + k0) / kBlock, m.absmax, m.absmax_q, m.absmax2, m.dq != 0);
+    const int64_t ncols = min(int64_t(kMergeRows), m.out - n0);
+    if (l2_async) {
+      const int pieces = int(ncols / 8);                                      // per L2 row
+      for (int i = tid; i < qn * pieces; i += 256) {
+        const int q = i / pieces, pc = i % pieces;
+        cp_async16(smem_u32(st_l2 + q * kMergeRows + pc * 8), m.L2 + int64_t(q0 + q) * m.out + n0 + pc * 8);
+      }
+    } else {
+      for (int i = tid; i < kMergeQ * kMergeRows; i += 256) {
+        const int q = i >> 7, n = i & 127;
+        if (q < qn && n < ncols) st_l2[q * kMergeRows + n] = m.L2[int64_t(q0 + q) * m.out + n0 + n];
+      }
     }
-  }
+    if (c == 0) {
+      constexpr int kPieces = kRowBytes / 16;   // 16-byte pieces per weight row: 8 (bf16) or 2 (codes)
+      uint8_t* wb = wbuf0 + (j & 1) * merge_w_bytes<BF16W>();
+      const uint8_t* src = BF16W ? reinterpret_cast<const uint8_t*>(m.Wbf) : m.codes;
+#pragma unroll
+      for (int u = 0; u < kMergeRows * kPieces / 256; ++u) {
+        const int i = tid + 256 * u, row = i / kPieces, piece = i % kPieces;
+        if (n0 + row < m.out)
+          cp_async16(smem_u32(wb + row * kRowBytes + piece * 16),
+                     src + ((n0 + row) * m.in + k0) * kRowBytes / kMergeCols + piece * 16);
+      }
+    }
+    cp_async_commit();
+  };
+
   double acc[4][8];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
-  for (int q0 = 0; q0 < r; q0 += kMergeQ) {
-    const int qn = min(kMergeQ, r - q0);
+  float scale[4] = {0.f, 0.f, 0.f, 0.f};
+  bool bad = false;
+  if (n_items > 0) issue(0);
+  for (int64_t it = 0; it < n_items; ++it) {
+    const int64_t j = it / nchunk;
+    const int c = int(it % nchunk);
+    const int64_t t = blockIdx.x + j * gridDim.x;
+    const int64_t n0 = (t / tiles_k) * kMergeRows, k0 = (t % tiles_k) * kMergeCols;
+    const int q0 = c * kMergeQ, qn = min(kMergeQ, r - q0);
+    cp_async_wait_all();
+    __syncthreads();                                           // item it has landed; item it - 1 is done
+    if (it + 1 < n_items) issue(it + 1);
+    if constexpr (!BF16W) {
+      if (c == 0) {
 #pragma unroll
-    for (int j = 0; j < kMergeQ * kMergeCols / 256; ++j) {
-      const int i = tid + 256 * j, q = i >> 6, k = i & 63;
-      s_a[q][merge_col_slot(k)] = (q < qn) ? bf16_to_f64(m.L1[(k0 + k) * r + q0 + q]) : 0.0;
+        for (int i = 0; i < 4; ++i) {
+          const int64_t n = n0 + 4 * tn + i;
+          scale[i] = n < m.out ? block_scale((n * m.in + k0) / kBlock, m.absmax, m.absmax_q, m.absmax2, m.dq != 0)
+                               : 0.f;
+        }
+      }
     }
+    {
+      const uint8_t* st = stage0 + (it & 1) * kMergeStageBytes;
+      const uint16_t* st_l1 = reinterpret_cast<const uint16_t*>(st);
+      const uint16_t* st_l2 = reinterpret_cast<const uint16_t*>(st + kMergeCols * kMergeQ * 2);
+      const int64_t ncols = min(int64_t(kMergeRows), m.out - n0);
 #pragma unroll
-    for (int j = 0; j < kMergeQ * kMergeRows / 256; ++j) {
-      const int i = tid + 256 * j, q = i >> 7, n = i & 127;
-      s_b[q][n] = (q < qn && n0 + n < m.out) ? bf16_to_f64(m.L2[int64_t(q0 + q) * m.out + n0 + n]) : 0.0;
+      for (int u = 0; u < kMergeQ * kMergeCols / 256; ++u) {
+        const int i = tid + 256 * u, q = i >> 6, k = i & 63;
+        s_a[q][merge_col_slot(k)] = (q < qn) ? bf16_to_f64(st_l1[k * kMergeQ + q]) : 0.0;
+      }
+#pragma unroll
+      for (int u = 0; u < kMergeQ * kMergeRows / 256; ++u) {
+        const int i = tid + 256 * u, q = i >> 7, n = i & 127;
+        s_b[q][n] = (q < qn && n < ncols) ? bf16_to_f64(st_l2[q * kMergeRows + n]) : 0.0;
+      }
     }
-    __syncthreads();
+    __syncthreads();                                           // fp64 slices ready
     const double2* ra = reinterpret_cast<const double2*>(&s_a[0][8 * tk]);
     const double2* rb = reinterpret_cast<const double2*>(&s_b[0][4 * tn]);
     const int rot = tk >> 1;
-    for (int q = 0; q < qn; ++q) {
+    auto rank_step = [&](int q) {
       double a[8];
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
@@ -503,69 +585,74 @@ __global__ void __launch_bounds__(256, 2) lora_merge_kernel(const __grid_constan
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[j], b[i], acc[i][j]);
-    }
-    __syncthreads();
-  }
-  cp_async_wait_all();
-  __syncthreads();
-  bool bad = false;
+        for (int jj = 0; jj < 8; ++jj) acc[i][jj] = fma(a[jj], b[i], acc[i][jj]);
+    };
+    if (qn == kMergeQ) {   // a full chunk, unrolled so that the next rank's loads overlap this rank's FMAs
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int row = 4 * tn + i;
-    const int64_t n = n0 + row;
-    const bool live = n < m.out;                              // same for the 8 lanes of a block
-    const int64_t e = n * m.in + k0 + 8 * tk;                 // first of this thread's 8 elements
-    uint4 wv = make_uint4(0u, 0u, 0u, 0u);
-    if (live) {
-      if constexpr (BF16W) {
-        wv = *reinterpret_cast<const uint4*>(s_w + row * kRowBytes + 16 * tk);
-      } else {
-        wv = nf4_dequant_word(*reinterpret_cast<const uint32_t*>(s_w + row * kRowBytes + 4 * tk),
-                              nf4_make_lut(scale[i]));
-      }
-    }
-    const uint32_t wh[4] = {wv.x, wv.y, wv.z, wv.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      uint16_t lo, hi;
-      const double v0 = double(__uint_as_float(wh[p] << 16)) + m.s * acc[i][2 * p];
-      const double v1 = double(__uint_as_float(wh[p] & 0xFFFF0000u)) + m.s * acc[i][2 * p + 1];
-      asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(lo) : "d"(v0));
-      asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(hi) : "d"(v1));
-      o[p] = live ? (uint32_t(lo) | (uint32_t(hi) << 16)) : 0u;
-    }
-    if constexpr (!QUANT) {
-      if (live) *reinterpret_cast<uint4*>(m.W_out + e) = make_uint4(o[0], o[1], o[2], o[3]);
+      for (int q = 0; q < kMergeQ; ++q) rank_step(q);
     } else {
-      float w[8];
+      for (int q = 0; q < qn; ++q) rank_step(q);
+    }
+    if (c != nchunk - 1) continue;
+    // ---- epilogue of tile t: its weight rows are in slot j % 2
+    const uint8_t* wb = wbuf0 + (j & 1) * merge_w_bytes<BF16W>();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = 4 * tn + i;
+      const int64_t n = n0 + row;
+      const bool live = n < m.out;                              // same for the 8 lanes of a block
+      const int64_t e = n * m.in + k0 + 8 * tk;                 // first of this thread's 8 elements
+      uint4 wv = make_uint4(0u, 0u, 0u, 0u);
+      if (live) {
+        if constexpr (BF16W) {
+          wv = *reinterpret_cast<const uint4*>(wb + row * kRowBytes + 16 * tk);
+        } else {
+          wv = nf4_dequant_word(*reinterpret_cast<const uint32_t*>(wb + row * kRowBytes + 4 * tk),
+                                nf4_make_lut(scale[i]));
+        }
+      }
+      const uint32_t wh[4] = {wv.x, wv.y, wv.z, wv.w};
+      uint32_t o[4];
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
-        w[2 * p] = bf16_lo(o[p]);
-        w[2 * p + 1] = bf16_hi(o[p]);
+        uint16_t lo, hi;
+        const double v0 = double(__uint_as_float(wh[p] << 16)) + m.s * acc[i][2 * p];
+        const double v1 = double(__uint_as_float(wh[p] & 0xFFFF0000u)) + m.s * acc[i][2 * p + 1];
+        asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(lo) : "d"(v0));
+        asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(hi) : "d"(v1));
+        o[p] = live ? (uint32_t(lo) | (uint32_t(hi) << 16)) : 0u;
+        acc[i][2 * p] = 0.0;
+        acc[i][2 * p + 1] = 0.0;
       }
-      float am = 0.f;
+      if constexpr (!QUANT) {
+        if (live) *reinterpret_cast<uint4*>(m.W_out + e) = make_uint4(o[0], o[1], o[2], o[3]);
+      } else {
+        float w[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float aw = fabsf(w[j]);
-        bad |= !(aw <= FLT_MAX);
-        am = fmaxf(am, aw);
-      }
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
-      if (live) {
-        const bool use = am > 0.f && am <= FLT_MAX;
-        uint32_t word = 0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t hi_idx = use ? nf4_index(__fdiv_rn(w[2 * k], am)) : 7u;
-          const uint32_t lo_idx = use ? nf4_index(__fdiv_rn(w[2 * k + 1], am)) : 7u;
-          word |= ((hi_idx << 4) | lo_idx) << (8 * k);
+        for (int p = 0; p < 4; ++p) {
+          w[2 * p] = bf16_lo(o[p]);
+          w[2 * p + 1] = bf16_hi(o[p]);
         }
-        *reinterpret_cast<uint32_t*>(m.q_codes + e / 2) = word;
-        if (tk == 0) m.q_absmax[e / kBlock] = am;
+        float am = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const float aw = fabsf(w[jj]);
+          bad |= !(aw <= FLT_MAX);
+          am = fmaxf(am, aw);
+        }
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+        // the quantizer's code lookup (cell of the one-multiply quotient, then two lane
+        // table shuffles); every lane runs it, for a dead row too
+        const bool use = am > 0.f && am <= FLT_MAX;
+        uint32_t x[8];
+        piece_index_bits(o, CellScale(use ? am : 1.f), lane_tables(tid & 31), x);
+        if (live) {
+          const uint32_t word = use ? pack_code_word(x) : 0x77777777u;
+          *reinterpret_cast<uint32_t*>(m.q_codes + e / 2) = word;
+          if (tk == 0) m.q_absmax[e / kBlock] = am;
+        }
       }
     }
   }
@@ -589,21 +676,32 @@ __global__ void __launch_bounds__(256) dq_scales_kernel(const float* __restrict_
   dq_group(s_amax, s_red, nb, g, absmax_q, absmax2);
 }
 
+template <bool BF16W, bool QUANT>
+static cudaError_t launch_merge_cfg(const MergeArgs& m, cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(lora_merge_kernel<BF16W, QUANT>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, merge_smem_bytes<BF16W>());
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int64_t tiles = (m.in / kMergeCols) * ((m.out + kMergeRows - 1) / kMergeRows);
+  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(tiles, int64_t(num_sms()) * 2)));
+  return launch_pdl(lora_merge_kernel<BF16W, QUANT>, dim3(unsigned(grid)), dim3(256), merge_smem_bytes<BF16W>(), st, m);
+}
+
 qlora_status launch_lora_merge(const uint8_t* codes, const float* absmax, const uint8_t* absmax_q,
                                const float* absmax2, bool dq, const uint16_t* Wbf, int64_t out, int64_t in,
                                const uint16_t* L1, const uint16_t* L2, int r, double s, uint16_t* W_out,
                                uint8_t* q_codes, float* q_absmax, int* status, cudaStream_t st) {
   const MergeArgs m{codes, absmax, absmax_q, absmax2, dq ? 1 : 0, Wbf, out, in, L1, L2, r, s, W_out,
                     q_codes, q_absmax, status};
-  const dim3 grid(unsigned(in / kMergeCols), unsigned((out + kMergeRows - 1) / kMergeRows));
   const bool quant = q_codes != nullptr;
   cudaError_t e;
   if (Wbf)
-    e = quant ? launch_pdl(lora_merge_kernel<true, true>, grid, dim3(256), 0, st, m)
-              : launch_pdl(lora_merge_kernel<true, false>, grid, dim3(256), 0, st, m);
+    e = quant ? launch_merge_cfg<true, true>(m, st) : launch_merge_cfg<true, false>(m, st);
   else
-    e = quant ? launch_pdl(lora_merge_kernel<false, true>, grid, dim3(256), 0, st, m)
-              : launch_pdl(lora_merge_kernel<false, false>, grid, dim3(256), 0, st, m);
+    e = quant ? launch_merge_cfg<false, true>(m, st) : launch_merge_cfg<false, false>(m, st);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

@@ -76,6 +76,30 @@ def test_merge_ragged_rows_and_ranks(cuda_device, dq):
                                       seed=3))
 
 
+@pytest.mark.parametrize("dq", [False, True])
+def test_merge_unaligned_adapter_rows(cuda_device, dq):
+    # r = 12 and out = 100: adapter rows are not whole 16-byte pieces (plain-load staging)
+    case = synth.LinearCase("merge-odd", M=1, out=100, inp=192, r=12, alpha=24.0, double_quant=dq, seed=9)
+    _check_merge(case)
+    _check_requant(case, dq_out=dq, keep_absmax=True)
+
+
+def test_merge_misaligned_adapter_pointers(cuda_device):
+    """Adapters that start 2 bytes past a 16-byte boundary take the plain-load path and
+    give the same bits."""
+    case = synth.LinearCase("merge-misaligned", M=1, out=256, inp=256, r=16, alpha=32.0, double_quant=True, seed=10)
+    d, g, w, W_s, L1, L2, ref = _check_merge(case)
+    def shifted(t):
+        buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+        v = buf[1:].view(t.shape)
+        v.copy_(t)
+        assert v.data_ptr() % 16 != 0
+        return v
+    got = api.lora_merge(w, shifted(g["L1"]), shifted(g["L2"]), case.scale)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(got).reshape(ref.shape), ref)
+
+
 def test_merge_q_proj_shape(cuda_device):
     _check_merge(synth.LinearCase("merge-q_proj", M=1, out=4096, inp=4096, r=16, alpha=32.0, double_quant=True))
 
@@ -185,3 +209,23 @@ def test_zero_adapter_merge_is_the_dequantized_weight(cuda_device):
     got = api.lora_merge(w, g["L1"], z, case.scale)
     torch.cuda.synchronize()
     assert np.array_equal(bits(got).reshape(-1), nf4.dequantize_bf16_bits(oracle_qweight(d["W"], True)).reshape(-1))
+
+
+@pytest.mark.parametrize("exp,sigs", [(0, range(0, 128, 3)), (-120, range(0, 128, 9)), (-126, range(0, 128, 17)),
+                                      (100, range(0, 128, 13)), (127, range(0, 128, 11))])
+def test_merge_requantize_every_bf16_value(cuda_device, exp, sigs):
+    """Blocks [a, x_1..x_63] holding every bf16 x with |x| <= a (a = (1 + s/128) 2^exp),
+    merged with a zero adapter and re-quantized: codes and scales equal the oracle's
+    quantization of the same values (this covers the power-of-two rescale that keeps
+    the block reciprocal normal for tiny and huge blocks)."""
+    from tests.test_gpu_codec import _exhaustive_blocks
+    blocks = _exhaustive_blocks(exp, sigs)
+    W = torch.from_numpy(nf4.bf16_bits_from_f32(blocks).view(np.int16)).view(torch.bfloat16).cuda()
+    L1 = torch.zeros((64, 8), dtype=torch.bfloat16, device="cuda")
+    L2 = torch.zeros((8, W.shape[0]), dtype=torch.bfloat16, device="cuda")
+    qw = nf4.quantize(blocks, double_quant=False)
+    o = api.lora_merge_requantize(api.NF4Weight.protected(W), L1, L2, 2.0, keep_absmax=True)
+    torch.cuda.synchronize()
+    assert api.status() == 0
+    assert np.array_equal(o.codes.cpu().numpy(), qw["codes"])
+    assert np.array_equal(o.absmax.cpu().numpy().view(np.uint32), qw["absmax"].view(np.uint32))
