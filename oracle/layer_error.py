@@ -16,6 +16,10 @@ Readings (the design doc lists them):
 * "layer" = one linear matrix (the page counts 144 linear layers in phi-1.5);
 * ranking: error descending, ties by matrix index ascending;
 * K from rho: round half up of rho * L (the only pin: 0.2 * 144 -> 29).
+* K from a memory budget ([AQLoRA] keeps the top-K in 16-bit "under a memory
+  budget"): the budget counts the bytes a kept layer adds to the all-NF4 model,
+  i.e. its bf16 size minus its NF4 storage (codes and scales, as the format
+  stores them); K is the longest prefix of the ranking whose added bytes fit.
 """
 from __future__ import annotations
 
@@ -24,7 +28,7 @@ from typing import Sequence, Tuple
 
 import numpy as np
 
-from . import nf4
+from . import nf4, storage
 
 
 def layer_sums(w_bf16_bits: np.ndarray, double_quant: bool = False) -> Tuple[float, float]:
@@ -59,3 +63,20 @@ def k_from_budget(rho, n_layers: int) -> int:
     """K = round half up of rho * L, in exact rational arithmetic."""
     x = Fraction(str(rho)) * n_layers
     return int((x + Fraction(1, 2)) // 1)
+
+
+def protect_cost_bytes(numel: int, double_quant: bool) -> int:
+    """Bytes that keeping one layer in bf16 adds to its NF4 storage."""
+    return 2 * numel - storage.buffer_bytes(numel, double_quant)["total"]
+
+
+def k_under_memory_budget(order: Sequence[int], numel: Sequence[int], double_quant: bool,
+                          budget_bytes: int) -> int:
+    """Largest K such that the top-K layers of ``order`` add at most budget_bytes."""
+    used, K = 0, 0
+    for l in order:
+        used += protect_cost_bytes(int(numel[int(l)]), double_quant)
+        if used > budget_bytes:
+            break
+        K += 1
+    return K

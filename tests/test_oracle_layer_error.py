@@ -108,3 +108,34 @@ def test_storage_matches_oracle_buffers():
             assert qw["absmax_q"].nbytes == bb["absmax_q"] and qw["absmax2"].nbytes == bb["absmax2"]
         else:
             assert qw["absmax"].nbytes == bb["absmax"]
+
+
+def test_memory_budget_rule_by_hand():
+    """Three 64 x 64 layers without double quant: NF4 storage 2048 code bytes + 64
+    fp32 scales = 2304 bytes, bf16 8192 bytes, so each kept layer adds 5888 bytes;
+    with double quant 2048 + 64 + 4 = 2116 bytes, adding 6076. The budget is
+    inclusive and the cut follows the ranking, not the layer ids."""
+    assert layer_error.protect_cost_bytes(4096, False) == 5888
+    assert layer_error.protect_cost_bytes(4096, True) == 6076
+    order = [2, 0, 1]
+    numel = [4096, 4096 * 4, 4096]
+    # ranked costs: layer 2 -> 5888, layer 0 -> 5888, layer 1 (16384 weights) -> 4 * 5888
+    for budget, K in [(0, 0), (5887, 0), (5888, 1), (11775, 1), (11776, 2), (11776 + 4 * 5888 - 1, 2),
+                      (11776 + 4 * 5888, 3), (10 ** 12, 3)]:
+        assert layer_error.k_under_memory_budget(order, numel, False, budget) == K, budget
+    assert layer_error.k_under_memory_budget([1, 0, 2], numel, False, 4 * 5888 - 1) == 0   # big layer ranked first
+
+
+def test_memory_budget_rule_is_monotone_and_a_prefix():
+    rng = np.random.default_rng(3)
+    numel = [int(64 * rng.integers(1, 5000)) for _ in range(40)]
+    err = rng.random(40)
+    order = layer_error.rank_layers(err)
+    costs = [layer_error.protect_cost_bytes(n, True) for n in numel]
+    prev = 0
+    for budget in sorted(rng.integers(0, sum(costs) + 10, 200).tolist()):
+        K = layer_error.k_under_memory_budget(order, numel, True, budget)
+        assert K >= prev
+        prev = K
+        assert sum(costs[l] for l in order[:K]) <= budget
+        assert K == len(order) or sum(costs[l] for l in order[:K + 1]) > budget
