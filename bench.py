@@ -317,6 +317,73 @@ def hbm_legs(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int =
             "timing": f"CUDA-graph replay, best of {reps} (inputs {numel * 2 / 1e9:.2f} GB, above L2)"}
 
 
+def protect_leg(api, synth, torch, dev, peaks, reps: int = 3, K: int = 8):
+    """What keeping layers in bf16 does to the step time on this part (the speed
+    effect the AQLoRA page attributes to protected layers). The fwd+bwd of one
+    linear (T, forward, backward; M = 16384, r = 16) is timed for the three
+    14B-stack shapes with the NF4 weight (double quant) and with the same weight
+    kept in bf16; the 280-matrix stack (40 layers of q, k, v, o, gate, up, down) is
+    ranked by the error pass, and the step over all its linears is composed from
+    the per-shape times with no layer kept and with the top K kept."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    shapes = {}
+    for c in synth.cases_14b(16, M=16384):
+        d = c.make(device=str(dev))
+        kind = c.name.split("-")[1]
+        row = {"out": c.out, "in": c.inp}
+        for mode in ("nf4", "bf16"):
+            w = api.quantize(d["W"], double_quant=True) if mode == "nf4" else api.NF4Weight.protected(d["W"])
+
+            def run():
+                T = api.lora_down(d["X"], d["L1"])
+                api.linear_fwd(w, d["X"], d["L1"], d["L2"], c.scale, T=T)
+                api.linear_bwd(w, d["X"], d["dY"], d["L1"], d["L2"], c.scale, T=T)
+
+            run()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                run()
+            ts = []
+            for i in range(reps + 1):
+                flush.zero_()
+                e0.record()
+                g.replay()
+                e1.record()
+                e1.synchronize()
+                if i:
+                    ts.append(e0.elapsed_time(e1))
+            ms = statistics.median(ts)
+            row[f"{mode}_ms"] = ms
+            row[f"{mode}_TFLOP/s"] = flops_fwd_bwd(c.M, c.inp, c.out, c.r) / (ms * 1e-3) / 1e12
+            del g, w
+        shapes[kind] = row
+        del d
+        torch.cuda.empty_cache()
+    assert api.status() == 0, "device status set in the protection leg"
+    # rank the whole stack (12.7 G weights) once with the error pass
+    mats = synth.stack_matrices(n_layers=40, linears=synth.QWEN14B_LINEARS)
+    Ws = [synth.stack_weight(m, device=str(dev)) for m in mats]
+    _, order, _ = api.layer_error_rank(Ws, K, double_quant=True)
+    order = order.cpu().tolist()
+    del Ws
+    torch.cuda.empty_cache()
+    kind_of = {"q": "q", "k": "q", "v": "q", "o": "q", "gate": "gate", "up": "gate", "down": "down"}
+    all_nf4 = sum(shapes[kind_of[m.name]]["nf4_ms"] for m in mats)
+    kept = [mats[l] for l in order[:K]]
+    with_k = all_nf4 + sum(shapes[kind_of[m.name]]["bf16_ms"] - shapes[kind_of[m.name]]["nf4_ms"] for m in kept)
+    return {"workload": "14B-stack linears (hidden 5120, intermediate 13824), M = 16384, r = 16, alpha = 32, "
+                        "NF4 with double quant vs the same weight kept in bf16; fwd+bwd = T, forward, backward",
+            "per_shape": shapes,
+            "stack": {"matrices": len(mats), "K": K,
+                      "kept": [f"layer {m.layer} {m.name}" for m in kept],
+                      "step_ms_no_layer_kept": all_nf4, "step_ms_top_K_kept": with_k,
+                      "change": with_k / all_nf4 - 1.0,
+                      "note": "composed from the per-shape times (each linear timed alone, L2 flushed)"},
+            "timing": f"CUDA-graph replay, median of {reps}, L2 flushed before each"}
+
+
 def merge_leg(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int = 4, r: int = 16):
     """LoRA merge (W_hat + s (L1 L2)^T, bf16 out) and merge + NF4 re-quantization over
     the first `layers` decoder layers of the Llama-7B-shaped stack (7 matrices per
@@ -402,6 +469,9 @@ def gpu_main(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     lib = _lib.load()
     peaks = load_peaks()
+    if args.protect_only:   # the protected-layer leg alone (not a bench line)
+        print(json.dumps({"protect": protect_leg(api, synth, torch, dev, peaks)}), flush=True)
+        return
     if args.merge_only:   # the merge legs alone (profiling aid; not a bench line)
         print(json.dumps({"merge": merge_leg(api, synth, torch, dev, torch.cuda.current_stream(), peaks,
                                              layers=args.merge_layers)}), flush=True)
@@ -630,6 +700,9 @@ def gpu_main(args):
     mlp = None
     if rank == 0 and world == 1 and not args.no_mlp_leg:
         mlp = mlp_leg(api, synth, torch, dev, peaks)
+    protect = None
+    if rank == 0 and world == 1 and not args.no_protect_leg:
+        protect = protect_leg(api, synth, torch, dev, peaks)
     merge = None
     if rank == 0 and world == 1 and not args.no_merge_leg:
         merge = merge_leg(api, synth, torch, dev, stream, peaks, layers=args.merge_layers)
@@ -645,7 +718,7 @@ def gpu_main(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args, world),
-            "roofline": roofline, "gemm_pairs": int(lib.qlora_pair_clusters()), "legs": legs_out, "mlp": mlp, "hbm_legs": hbm, "merge": merge, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "gemm_pairs": int(lib.qlora_pair_clusters()), "legs": legs_out, "mlp": mlp, "hbm_legs": hbm, "merge": merge, "protect": protect, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
             "timing": "cuda-graph replay of the step" if use_graphs else "eager API calls",
             "peaks": {"bf16_tflops": peaks["bf16"], "bf16_tflops_sustained": peaks["bf16_sus"],
@@ -672,6 +745,10 @@ def main():
     ap.add_argument("--no-hbm-legs", action="store_true", help="skip the full-stack quantizer / error-pass legs")
     ap.add_argument("--no-mlp-leg", action="store_true", help="skip the Llama-7B MLP (gate, up, down) fwd+bwd leg")
     ap.add_argument("--no-merge-leg", action="store_true", help="skip the LoRA merge / merge + re-quantize leg")
+    ap.add_argument("--no-protect-leg", action="store_true",
+                    help="skip the protected-layer (bf16 vs NF4) step-time leg on the 14B-stack shapes")
+    ap.add_argument("--protect-only", action="store_true",
+                    help="run only the protected-layer leg and print it (not a bench line)")
     ap.add_argument("--merge-layers", type=int, default=4, help="decoder layers of the stack for the merge leg")
     ap.add_argument("--merge-only", action="store_true",
                     help="run only the merge legs and print them (profiling aid; not a bench line)")

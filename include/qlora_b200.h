@@ -277,6 +277,29 @@ qlora_status nf4_layer_error_rank(int32_t n_layers, const uint16_t* const* W_ptr
                                   double* err, int32_t* order, uint8_t* keep,
                                   void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
+/* The same pass with K taken from a memory budget ("AQLoRA: A Zero-Search Recipe
+ * for Fast Quantized LoRA Fine-Tuning", section 3.2: the top-K layers are kept in
+ * 16-bit under a memory budget). Keeping layer l in bf16 adds
+ *   cost_l = 2 numel_l - (NF4 bytes of layer l: numel_l / 2 code bytes plus
+ *            4 numel_l / 64 scale bytes, or with double quant numel_l / 64 E4M3
+ *            bytes plus 4 ceil(numel_l / 16384) bytes)
+ * to the all-NF4 model. K is the largest count such that the first K layers of
+ * `order` add at most budget_bytes in total (0 <= budget_bytes; the budget is
+ * inclusive).
+ *   K_out    device out, int32 [1]
+ * Other arguments, the workspace and the errors as for nf4_layer_error_rank;
+ * numel_l <= 2^40. */
+qlora_status nf4_layer_error_rank_budget(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
+                                         int32_t w_dtype, nf4_qconfig q, int64_t budget_bytes, double* err,
+                                         int32_t* order, uint8_t* keep, int32_t* K_out, void* workspace,
+                                         size_t workspace_bytes, qlora_stream_t stream);
+
+/* K from a protection fraction rho = num / den of n_layers layers (same page,
+ * section 3.2, where rho = 0.2 of 144 linear layers keeps 29): round half up of
+ * rho * n_layers, in exact integer arithmetic. Host only (no device work).
+ *   0 <= num <= den, 0 < den <= 2^31, 0 <= n_layers <= 2^30; K host out. */
+qlora_status nf4_k_from_fraction(int64_t num, int64_t den, int32_t n_layers, int32_t* K);
+
 /* The allocation pass fused with the quantization it measures ("AQLoRA: A
  * Zero-Search Recipe for Fast Quantized LoRA Fine-Tuning", section 3.1-3.2: one
  * pass quantizes every linear layer to NF4 and scores its reconstruction error;

@@ -61,6 +61,10 @@ SIGNATURES = {
     "nf4_layer_error_rank_workspace_size": (c_size_t, [c_int32, POINTER(c_int64)]),
     "nf4_layer_error_rank": (c_int, [c_int32, POINTER(c_void_p), POINTER(c_int64), c_int32, NF4QConfig, c_int32,
                                      c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "nf4_layer_error_rank_budget": (c_int, [c_int32, POINTER(c_void_p), POINTER(c_int64), c_int32, NF4QConfig,
+                                            c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                            c_void_p]),
+    "nf4_k_from_fraction": (c_int, [c_int64, c_int64, c_int32, POINTER(c_int32)]),
     "nf4_layer_error_rank_noalloc": (c_int, [c_int32, POINTER(c_void_p), POINTER(c_int64), c_int32, NF4QConfig,
                                              c_int32, c_void_p, c_void_p, c_void_p, c_void_p]),
     "nf4_quantize_error_rank": (c_int, [c_int32, POINTER(c_void_p), POINTER(c_int64), c_int32, NF4QConfig, c_int32,

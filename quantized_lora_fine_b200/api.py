@@ -285,6 +285,35 @@ def layer_error_rank(Ws: Sequence[torch.Tensor], K: int, double_quant: bool = Fa
     return err, order, keep
 
 
+def layer_error_rank_budget(Ws: Sequence[torch.Tensor], budget_bytes: int, double_quant: bool = False):
+    """layer_error_rank with K from a memory budget: the longest prefix of the
+    ranking whose bf16 copies add at most budget_bytes to the NF4 storage.
+    Returns (err, order, keep, K) with K a one-element device int32 tensor."""
+    lib = _lib.load()
+    L = len(Ws)
+    for i, W in enumerate(Ws):
+        _need(W, torch.bfloat16, f"W[{i}]")
+    dev = Ws[0].device
+    ptrs = (ctypes.c_void_p * L)(*[W.data_ptr() for W in Ws])
+    numel = (ctypes.c_int64 * L)(*[W.numel() for W in Ws])
+    err = torch.empty(L, dtype=torch.float64, device=dev)
+    order = torch.empty(L, dtype=torch.int32, device=dev)
+    keep = torch.empty(L, dtype=torch.uint8, device=dev)
+    K = torch.empty(1, dtype=torch.int32, device=dev)
+    ws = Workspace.get(lib.nf4_layer_error_rank_workspace_size(L, numel), dev)
+    check(lib.nf4_layer_error_rank_budget(L, ptrs, numel, DTYPE_BF16, NF4QConfig(64, 1 if double_quant else 0, 256),
+                                          int(budget_bytes), _ptr(err), _ptr(order), _ptr(keep), _ptr(K), _ptr(ws),
+                                          ws.numel(), _stream()), "nf4_layer_error_rank_budget")
+    return err, order, keep, K
+
+
+def k_from_fraction(num: int, den: int, n_layers: int) -> int:
+    """K = round half up of (num / den) * n_layers (host only)."""
+    k = ctypes.c_int32(0)
+    check(_lib.load().nf4_k_from_fraction(int(num), int(den), int(n_layers), ctypes.byref(k)), "nf4_k_from_fraction")
+    return int(k.value)
+
+
 def quantize_error_rank(Ws: Sequence[torch.Tensor], K: int, double_quant: bool = False, keep_absmax: bool = False,
                         outs: Optional[Sequence[NF4Weight]] = None):
     """The allocation pass fused with the quantization: one read of every matrix

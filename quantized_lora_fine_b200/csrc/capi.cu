@@ -755,6 +755,33 @@ qlora_status nf4_layer_error_rank(int32_t n_layers, const uint16_t* const* W_ptr
                                  workspace_bytes, static_cast<int*>(workspace), S(stream));
 }
 
+qlora_status nf4_layer_error_rank_budget(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
+                                         int32_t w_dtype, nf4_qconfig q, int64_t budget_bytes, double* err,
+                                         int32_t* order, uint8_t* keep, int32_t* K_out, void* workspace,
+                                         size_t workspace_bytes, qlora_stream_t stream) {
+  if (w_dtype != QLORA_DTYPE_BF16) return QLORA_ERR_DTYPE;
+  if (!qconfig_ok(q)) return QLORA_ERR_UNSUPPORTED;
+  if (n_layers < 1 || n_layers > 1024 || budget_bytes < 0) return QLORA_ERR_SHAPE;
+  if (!W_ptrs || !numel || !err || !order || !keep || !K_out) return QLORA_ERR_NULL;
+  for (int i = 0; i < n_layers; ++i) {
+    if (!W_ptrs[i]) return QLORA_ERR_NULL;
+    if (numel[i] <= 0 || numel[i] % 64 || numel[i] > (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
+    if (!aligned16(W_ptrs[i])) return QLORA_ERR_ALIGN;
+  }
+  if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
+  QLB_TRY(check_device());
+  return launch_layer_error_rank(n_layers, W_ptrs, numel, q.double_quant != 0, 0, err, order, keep, workspace,
+                                 workspace_bytes, static_cast<int*>(workspace), S(stream), budget_bytes, K_out);
+}
+
+qlora_status nf4_k_from_fraction(int64_t num, int64_t den, int32_t n_layers, int32_t* K) {
+  if (!K) return QLORA_ERR_NULL;
+  if (den <= 0 || num < 0 || num > den || den > (int64_t(1) << 31) || n_layers < 0 || n_layers > (1 << 30))
+    return QLORA_ERR_SHAPE;
+  *K = int32_t((2 * num * n_layers + den) / (2 * den));   // floor(num L / den + 1/2)
+  return QLORA_OK;
+}
+
 qlora_status nf4_quantize_error_rank(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
                                     int32_t w_dtype, nf4_qconfig q, int32_t K, uint8_t* const* codes,
                                     float* const* absmax, uint8_t* const* absmax_q, float* const* absmax2,

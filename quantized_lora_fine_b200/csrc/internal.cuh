@@ -88,9 +88,14 @@ qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_p
                                        int K, uint8_t* const* codes, float* const* absmax, uint8_t* const* absmax_q,
                                        float* const* absmax2, double* err, int32_t* order, uint8_t* keep, void* ws,
                                        size_t ws_bytes, int* status, cudaStream_t s);
+// With K_out non-null the keep rule is the memory budget (K ignored): the longest
+// prefix of the order whose added bf16 bytes fit in budget_bytes; K goes to *K_out.
 qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
                                      int K, double* err, int32_t* order, uint8_t* keep, void* ws, size_t ws_bytes,
-                                     int* status, cudaStream_t s);
+                                     int* status, cudaStream_t s, int64_t budget_bytes = 0,
+                                     int32_t* K_out = nullptr);
+// Stored bytes of one NF4 matrix (codes + scales; double quant as configured).
+int64_t nf4_storage_bytes(int64_t numel, bool dq);
 
 // Allocation-free variant: partial sums in a file-scope device array (see layer_error.cu).
 int64_t noalloc_chunks(int n_layers, const int64_t* numel);

@@ -258,6 +258,17 @@ __device__ __forceinline__ void finish_layer_warp(const double2* __restrict__ pa
   if (lane == 0) *err_out = (b > 0.0) ? sqrt(a / b) : 0.0;
 }
 
+// Position of layer l in the order (error descending, index ascending).
+__device__ __forceinline__ int rank_of(const double* s_err, int n_layers, int l) {
+  const double e = s_err[l];
+  int rank = 0;
+  for (int j = 0; j < n_layers; ++j) {
+    const double f = s_err[j];
+    rank += (f > e || (f == e && j < l)) ? 1 : 0;
+  }
+  return rank;
+}
+
 __global__ void __launch_bounds__(1024) rank_topk_kernel(const double* __restrict__ err, int n_layers, int K,
                                                          int32_t* __restrict__ order, uint8_t* __restrict__ keep) {
   pdl_wait();
@@ -266,15 +277,50 @@ __global__ void __launch_bounds__(1024) rank_topk_kernel(const double* __restric
   for (int i = threadIdx.x; i < n_layers; i += blockDim.x) s_err[i] = err[i];
   __syncthreads();
   for (int l = threadIdx.x; l < n_layers; l += blockDim.x) {
-    const double e = s_err[l];
-    int rank = 0;
-    for (int j = 0; j < n_layers; ++j) {
-      const double f = s_err[j];
-      rank += (f > e || (f == e && j < l)) ? 1 : 0;
-    }
+    const int rank = rank_of(s_err, n_layers, l);
     order[rank] = l;
     keep[l] = rank < K ? 1 : 0;
   }
+}
+
+// Keep rule by memory budget: the longest prefix of the order whose added bytes
+// (cost[l]: what keeping layer l in bf16 adds to its NF4 storage, always > 0) sum
+// to at most `budget`. One thread per layer (n_layers <= 1024 = block size):
+// costs are placed at their rank, an inclusive prefix sum runs in shared memory,
+// and since the prefixes grow, K is the number of them within the budget.
+struct BudgetTable {
+  int64_t cost[kMaxLayers];
+  int64_t budget;
+};
+
+__global__ void __launch_bounds__(1024) rank_budget_kernel(const double* __restrict__ err, int n_layers,
+                                                           const __grid_constant__ BudgetTable bt,
+                                                           int32_t* __restrict__ order, uint8_t* __restrict__ keep,
+                                                           int32_t* __restrict__ K_out) {
+  pdl_wait();
+  pdl_launch();
+  __shared__ double s_err[kMaxLayers];
+  __shared__ int64_t s_pre[kMaxLayers];
+  __shared__ int32_t s_rank[kMaxLayers];
+  const int t = threadIdx.x;
+  if (t < n_layers) s_err[t] = err[t];
+  __syncthreads();
+  if (t < n_layers) {
+    const int rank = rank_of(s_err, n_layers, t);
+    s_rank[t] = rank;
+    order[rank] = t;
+    s_pre[rank] = bt.cost[t];
+  }
+  __syncthreads();
+  for (int off = 1; off < n_layers; off <<= 1) {
+    const int64_t v = (t < n_layers && t >= off) ? s_pre[t - off] : 0;
+    __syncthreads();
+    if (t < n_layers) s_pre[t] += v;
+    __syncthreads();
+  }
+  const int K = __syncthreads_count(t < n_layers && s_pre[t] <= bt.budget);
+  if (t < n_layers) keep[t] = s_rank[t] < K ? 1 : 0;
+  if (t == 0) *K_out = K;
 }
 
 // Pass 2: one warp per layer.
@@ -293,6 +339,13 @@ static int32_t chunks_of(int64_t numel) {
   return static_cast<int32_t>((nb + kDQBlock - 1) / kDQBlock);
 }
 
+// Bytes of one NF4 matrix as stored: packed codes plus fp32 scales, or with double
+// quant one E4M3 byte per block plus one fp32 factor per 256 blocks.
+int64_t nf4_storage_bytes(int64_t numel, bool dq) {
+  const int64_t nb = (numel + kBlock - 1) / kBlock;
+  return (numel + 1) / 2 + (dq ? nb + 4 * ((nb + kDQBlock - 1) / kDQBlock) : 4 * nb);
+}
+
 size_t layer_error_ws_bytes(int n_layers, const int64_t* numel) {
   int64_t chunks = 0;
   for (int i = 0; i < n_layers; ++i) chunks += chunks_of(numel[i]);
@@ -304,7 +357,8 @@ size_t layer_error_ws_bytes(int n_layers, const int64_t* numel) {
 // while its predecessor drains (the allocation-free entry launches plainly).
 template <bool DQ, class Tab>
 static qlora_status launch_passes(const Tab& tab, double2* partial, int* status, double* err, int K,
-                                  int32_t* order, uint8_t* keep, cudaStream_t s, bool pdl) {
+                                  int32_t* order, uint8_t* keep, cudaStream_t s, bool pdl,
+                                  const BudgetTable* budget = nullptr, int32_t* K_out = nullptr) {
   static std::mutex mu;
   static ChunkRanges r;   // host staging of the by-value parameter
   std::lock_guard<std::mutex> lock(mu);
@@ -316,11 +370,16 @@ static qlora_status launch_passes(const Tab& tab, double2* partial, int* status,
   if (pdl) {
     e = launch_pdl(layer_error_chunk_kernel<DQ, Tab>, dim3(c), dim3(256), 0, s, tab, partial, status);
     if (e == cudaSuccess) e = launch_pdl(layer_error_finish_kernel, dim3(unsigned(n)), dim3(32), 0, s, partial, r, err);
-    if (e == cudaSuccess) e = launch_pdl(rank_topk_kernel, dim3(1), dim3(1024), 0, s, err, n, K, order, keep);
+    if (e == cudaSuccess)
+      e = budget ? launch_pdl(rank_budget_kernel, dim3(1), dim3(1024), 0, s, err, n, *budget, order, keep, K_out)
+                 : launch_pdl(rank_topk_kernel, dim3(1), dim3(1024), 0, s, err, n, K, order, keep);
   } else {
     layer_error_chunk_kernel<DQ, Tab><<<c, 256, 0, s>>>(tab, partial, status);
     layer_error_finish_kernel<<<unsigned(n), 32, 0, s>>>(partial, r, err);
-    rank_topk_kernel<<<1, 1024, 0, s>>>(err, n, K, order, keep);
+    if (budget)
+      rank_budget_kernel<<<1, 1024, 0, s>>>(err, n, *budget, order, keep, K_out);
+    else
+      rank_topk_kernel<<<1, 1024, 0, s>>>(err, n, K, order, keep);
     e = cudaSuccess;
   }
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
@@ -328,7 +387,7 @@ static qlora_status launch_passes(const Tab& tab, double2* partial, int* status,
 
 qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
                                      int K, double* err, int32_t* order, uint8_t* keep, void* ws, size_t ws_bytes,
-                                     int* status, cudaStream_t s) {
+                                     int* status, cudaStream_t s, int64_t budget_bytes, int32_t* K_out) {
   // The chunk table travels as a by-value kernel parameter (no host-to-device
   // copy), so this call can be captured into a CUDA graph.
   static std::mutex mu;
@@ -345,6 +404,13 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
   }
   tab.first_chunk[n_layers] = c;
   double2* partial = reinterpret_cast<double2*>(static_cast<char*>(ws) + kReservedBytes);
+  if (K_out) {   // keep rule by memory budget
+    static BudgetTable bt;
+    for (int i = 0; i < n_layers; ++i) bt.cost[i] = 2 * numel[i] - nf4_storage_bytes(numel[i], dq);
+    bt.budget = budget_bytes;
+    return dq ? launch_passes<true>(tab, partial, status, err, 0, order, keep, s, true, &bt, K_out)
+              : launch_passes<false>(tab, partial, status, err, 0, order, keep, s, true, &bt, K_out);
+  }
   return dq ? launch_passes<true>(tab, partial, status, err, K, order, keep, s, true)
             : launch_passes<false>(tab, partial, status, err, K, order, keep, s, true);
 }

@@ -119,3 +119,30 @@ def test_product_path_refuses_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "_lib", None)
     with pytest.raises(RuntimeError):
         _lib.load(str(tmp_path / "missing.so"))
+
+
+def test_k_from_fraction_is_round_half_up(lib):
+    """The host-only fraction rule agrees with the oracle's exact rational rule
+    (0.2 of 144 keeps 29) and rejects bad fractions."""
+    from fractions import Fraction
+    from oracle import layer_error
+    k = ctypes.c_int32(0)
+    assert lib.nf4_k_from_fraction(1, 5, 144, ctypes.byref(k)) == 0 and k.value == 29
+    assert lib.nf4_k_from_fraction(7, 20, 10, ctypes.byref(k)) == 0 and k.value == 4      # 3.5 rounds up
+    import random
+    rnd = random.Random(1)
+    for _ in range(2000):
+        den = rnd.randint(1, 10 ** 6)
+        num = rnd.randint(0, den)
+        L = rnd.randint(0, 5000)
+        assert lib.nf4_k_from_fraction(num, den, L, ctypes.byref(k)) == 0
+        assert k.value == layer_error.k_from_budget(Fraction(num, den), L), (num, den, L)
+    assert lib.nf4_k_from_fraction(1, 0, 10, ctypes.byref(k)) == 2
+    assert lib.nf4_k_from_fraction(3, 2, 10, ctypes.byref(k)) == 2
+    assert lib.nf4_k_from_fraction(1, 2, 10, None) == 1
+    # budget rule: negative budget, missing K output
+    q = _lib.NF4QConfig(64, 0, 256)
+    ptrs = (ctypes.c_void_p * 1)(0x1000)
+    n = (ctypes.c_int64 * 1)(4096)
+    assert lib.nf4_layer_error_rank_budget(1, ptrs, n, 0, q, -1, 0x10, 0x10, 0x10, 0x10, 0x2000, 1 << 20, None) == 2
+    assert lib.nf4_layer_error_rank_budget(1, ptrs, n, 0, q, 100, 0x10, 0x10, 0x10, None, 0x2000, 1 << 20, None) == 1

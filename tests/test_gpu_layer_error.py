@@ -109,3 +109,34 @@ def test_fused_quantize_error_rank_full_gate(cuda_device):
     mats = synth.stack_matrices()
     Ws = [synth.stack_weight(mats[i]) for i in (4, 7)]   # an 11008 x 4096 gate and a 4096^2 q
     _compare_fused(Ws, K=1, dq=True)
+
+
+def _compare_budget(Ws, dq, budgets):
+    ref_err = np.array([layer_error.layer_error(bits(W), dq) for W in Ws])
+    ref_order = layer_error.rank_layers(ref_err)
+    numel = [W.numel() for W in Ws]
+    g = [W.cuda() for W in Ws]
+    for budget in budgets:
+        K_ref = layer_error.k_under_memory_budget(ref_order, numel, dq, budget)
+        err, order, keep, K = api.layer_error_rank_budget(g, budget, double_quant=dq)
+        torch.cuda.synchronize()
+        assert int(K.item()) == K_ref, (budget, int(K.item()), K_ref)
+        assert np.array_equal(order.cpu().numpy(), ref_order)
+        assert np.array_equal(keep.cpu().numpy(), layer_error.keep_mask(ref_order, K_ref))
+        nz = ref_err > 0
+        assert np.all(np.abs(err.cpu().numpy()[nz] - ref_err[nz]) <= 1e-6 * ref_err[nz])
+    assert api.status() == 0
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_memory_budget_keep_rule(cuda_device, dq):
+    """K from a byte budget: the budget at each exact prefix sum of the ranked costs
+    keeps that prefix, one byte less keeps one layer fewer; zero keeps none and a
+    large budget keeps all."""
+    mats = synth.stack_matrices(n_layers=3, linears=(("a", 256, 512), ("b", 512, 256), ("c", 64, 320)))
+    Ws = [synth.stack_weight(m) for m in mats]
+    ref_err = np.array([layer_error.layer_error(bits(W), dq) for W in Ws])
+    order = layer_error.rank_layers(ref_err)
+    costs = np.cumsum([layer_error.protect_cost_bytes(Ws[l].numel(), dq) for l in order])
+    budgets = [0, 1, int(costs[-1]) * 10] + [int(c) for c in costs[:5]] + [int(c) - 1 for c in costs[:5]]
+    _compare_budget(Ws, dq, budgets)
