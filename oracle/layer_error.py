@@ -8,7 +8,7 @@ reconstruction error (the equation itself is missing from the extracted page).
 [AQLoRA] 3.2: layers are ranked by that error and a fixed top-K cut keeps the
 highest-error layers in 16-bit; K comes from the protection budget rho.
 
-Readings (the design doc lists them):
+Readings (where the pages are silent):
 * error = relative Frobenius norm e = sqrt(sum (w - w_hat)^2 / sum w^2) over
   the whole matrix, w the bf16 input widened to fp64 and w_hat the bf16
   dequantized value the GEMM would consume, with the layer's double-quant

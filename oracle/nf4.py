@@ -13,7 +13,7 @@ What the pages fix ([QLoRA-blog] "1. NormalFloat", "2. Double quantization";
 * double quantization stores the first-level (per 64) scales in 8 bits with a
   higher-precision scale per group of 256 first-level scales.
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 * code values: asymmetric normal quantiles (construction in ``nf4_code_table``);
 * absmax scaling, IEEE fp32 division, nearest code by fp32 midpoints, ties to
   the lower code;
