@@ -146,3 +146,29 @@ def test_k_from_fraction_is_round_half_up(lib):
     n = (ctypes.c_int64 * 1)(4096)
     assert lib.nf4_layer_error_rank_budget(1, ptrs, n, 0, q, -1, 0x10, 0x10, 0x10, 0x10, 0x2000, 1 << 20, None) == 2
     assert lib.nf4_layer_error_rank_budget(1, ptrs, n, 0, q, 100, 0x10, 0x10, 0x10, None, 0x2000, 1 << 20, None) == 1
+
+
+def test_empty_inputs_are_refused_on_the_host(lib):
+    """Empty inputs (no rows, no columns, no tokens, no layers, rank 0) return
+    QLORA_ERR_SHAPE before any device work; workspace sizes for them are 0."""
+    q = _lib.NF4QConfig(64, 0, 256)
+    for out, inp in ((0, 64), (64, 0), (0, 0)):
+        assert lib.nf4_quantize(0x1000, 0, out, inp, q, 0x2000, 0x3000, None, None, 0x4000, 256, None) == 2
+    w = _lib.QLoraWeight()
+    w.out, w.in_, w.q = 256, 256, q
+    w.codes, w.absmax = 0x2000, 0x3000
+    assert lib.qlora_linear_fwd(ctypes.byref(w), 0x1000, 0, 0x1000, 0x1000, 16, 2.0, 0x1000, None, 0x4000,
+                                1 << 20, None) == 2
+    assert lib.qlora_linear_bwd(ctypes.byref(w), 0x1000, 0x1000, 0, 0x1000, 0x1000, 16, 2.0, 0x1000, 0x1000,
+                                0x1000, 0x1000, 0x4000, 1 << 20, None) == 2
+    assert lib.qlora_fwd_workspace_size(0, 256, 256, 16) == 0
+    assert lib.qlora_bwd_workspace_size(0, 256, 256, 16) == 0
+    ptrs = (ctypes.c_void_p * 1)(0x1000)
+    n = (ctypes.c_int64 * 1)(0)
+    assert lib.nf4_layer_error_rank(0, ptrs, n, 0, q, 0, 0x10, 0x10, 0x10, 0x2000, 1 << 20, None) == 2
+    assert lib.nf4_layer_error_rank(1, ptrs, n, 0, q, 0, 0x10, 0x10, 0x10, 0x2000, 1 << 20, None) == 2
+    m = _lib.QLoraWeight()
+    m.out, m.in_, m.q = 0, 64, q
+    m.codes, m.absmax = 0x2000, 0x3000
+    assert lib.qlora_lora_merge(ctypes.byref(m), 0x1000, 0x1000, 8, 2.0, 0x4000, None) == 2
+    assert lib.qlora_lora_merge_requantize_workspace_size(0, 64) == 0
