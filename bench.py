@@ -332,13 +332,17 @@ def protect_leg(api, synth, torch, dev, peaks, reps: int = 3, K: int = 8):
         d = c.make(device=str(dev))
         kind = c.name.split("-")[1]
         row = {"out": c.out, "in": c.inp}
-        for mode in ("nf4", "bf16"):
+        for mode in ("nf4", "bf16", "two_stage"):
+            if mode == "two_stage":   # two NF4 stages, reconstructed to bf16 once per step
+                w1 = api.quantize(d["W"], double_quant=True)
+                w2 = api.quantize_residual(d["W"], w1, double_quant=True)
             w = api.quantize(d["W"], double_quant=True) if mode == "nf4" else api.NF4Weight.protected(d["W"])
 
             def run():
+                ww = api.NF4Weight.protected(api.dequantize_two_stage(w1, w2)) if mode == "two_stage" else w
                 T = api.lora_down(d["X"], d["L1"])
-                api.linear_fwd(w, d["X"], d["L1"], d["L2"], c.scale, T=T)
-                api.linear_bwd(w, d["X"], d["dY"], d["L1"], d["L2"], c.scale, T=T)
+                api.linear_fwd(ww, d["X"], d["L1"], d["L2"], c.scale, T=T)
+                api.linear_bwd(ww, d["X"], d["dY"], d["L1"], d["L2"], c.scale, T=T)
 
             run()
             torch.cuda.synchronize()
@@ -359,6 +363,7 @@ def protect_leg(api, synth, torch, dev, peaks, reps: int = 3, K: int = 8):
             row[f"{mode}_TFLOP/s"] = flops_fwd_bwd(c.M, c.inp, c.out, c.r) / (ms * 1e-3) / 1e12
             del g, w
         shapes[kind] = row
+        row["two_stage_vs_bf16"] = row["two_stage_ms"] / row["bf16_ms"] - 1.0
         del d
         torch.cuda.empty_cache()
     assert api.status() == 0, "device status set in the protection leg"
@@ -373,13 +378,16 @@ def protect_leg(api, synth, torch, dev, peaks, reps: int = 3, K: int = 8):
     all_nf4 = sum(shapes[kind_of[m.name]]["nf4_ms"] for m in mats)
     kept = [mats[l] for l in order[:K]]
     with_k = all_nf4 + sum(shapes[kind_of[m.name]]["bf16_ms"] - shapes[kind_of[m.name]]["nf4_ms"] for m in kept)
+    with_k2 = all_nf4 + sum(shapes[kind_of[m.name]]["two_stage_ms"] - shapes[kind_of[m.name]]["nf4_ms"] for m in kept)
     return {"workload": "14B-stack linears (hidden 5120, intermediate 13824), M = 16384, r = 16, alpha = 32, "
-                        "NF4 with double quant vs the same weight kept in bf16; fwd+bwd = T, forward, backward",
+                        "NF4 with double quant vs the same weight kept in bf16 vs two NF4 stages (reconstructed "
+                        "to bf16 once per step); fwd+bwd = T, forward, backward",
             "per_shape": shapes,
             "stack": {"matrices": len(mats), "K": K,
                       "kept": [f"layer {m.layer} {m.name}" for m in kept],
                       "step_ms_no_layer_kept": all_nf4, "step_ms_top_K_kept": with_k,
                       "change": with_k / all_nf4 - 1.0,
+                      "step_ms_top_K_two_stage": with_k2, "change_two_stage": with_k2 / all_nf4 - 1.0,
                       "note": "composed from the per-shape times (each linear timed alone, L2 flushed)"},
             "timing": f"CUDA-graph replay, median of {reps}, L2 flushed before each"}
 
@@ -729,18 +737,26 @@ def gpu_main(args):
     # on the Llama-7B-shaped stack instead: 224 matrices, 6.48 G weights (12.95 GB
     # of bf16), quantize every matrix (one call each) and one error/rank call over
     # all of them, as the allocation pass does.
+    # The side legs run after the step's own numbers are taken; one that fails is
+    # reported in its own entry and does not cost the line.
+    def side_leg(fn, *a, **k):
+        try:
+            return fn(*a, **k)
+        except Exception as e:   # noqa: BLE001 -- reported, not hidden
+            return {"error": f"{type(e).__name__}: {e}"}
+
     hbm = None
     if rank == 0 and world == 1 and not args.no_hbm_legs:
-        hbm = hbm_legs(api, synth, torch, dev, stream, peaks, layers=args.hbm_layers)
+        hbm = side_leg(hbm_legs, api, synth, torch, dev, stream, peaks, layers=args.hbm_layers)
     mlp = None
     if rank == 0 and world == 1 and not args.no_mlp_leg:
-        mlp = mlp_leg(api, synth, torch, dev, peaks)
+        mlp = side_leg(mlp_leg, api, synth, torch, dev, peaks)
     protect = None
     if rank == 0 and world == 1 and not args.no_protect_leg:
-        protect = protect_leg(api, synth, torch, dev, peaks)
+        protect = side_leg(protect_leg, api, synth, torch, dev, peaks)
     merge = None
     if rank == 0 and world == 1 and not args.no_merge_leg:
-        merge = merge_leg(api, synth, torch, dev, stream, peaks, layers=args.merge_layers)
+        merge = side_leg(merge_leg, api, synth, torch, dev, stream, peaks, layers=args.merge_layers)
 
     # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1 only)
     cpu = None

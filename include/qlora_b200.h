@@ -35,6 +35,11 @@
  *     out) are recorded in an int32 status word at the start of the
  *     workspace. The word is sticky: it keeps the first error until
  *     qlora_reset_status(). A fresh workspace must be zeroed (or reset) once.
+ *   - One workspace may serve every entry point on a stream: its first 256
+ *     bytes hold the status word, the next 64 KiB split-K tile counters that
+ *     must be zero when a call starts and that every call leaves zero; a
+ *     call's other scratch comes after them. Zeroing a workspace once keeps
+ *     this true for any sequence of calls.
  *   - No call aborts the process or throws.
  */
 #ifndef QLORA_B200_H
@@ -163,6 +168,37 @@ qlora_status nf4_quantize_batch(int32_t n, const uint16_t* const* W_ptrs, const 
  *   w      host pointer to a descriptor with is_bf16 = 0 (device buffers inside)
  *   W_out  device out, bf16 [out*in], 16-byte aligned */
 qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream_t stream);
+
+/* ------------------------------------------ residual NF4 second stage */
+
+/* A protected layer stored as two NF4 stages instead of bf16 ("AQLoRA: A
+ * Zero-Search Recipe for Fast Quantized LoRA Fine-Tuning", "Additional controls"
+ * and section 8: a second NF4 stage over the protected layers' residuals matched
+ * 16-bit protection at +3.6 % step time). The second stage quantizes
+ *   R = fp32_rn(w - fp32_rn(c1 * a1))
+ * (w the original bf16 weight, c1 * a1 the first stage's value) exactly as
+ * nf4_quantize quantizes an fp32 tensor (config q, its own double-quant setting).
+ *   W        device bf16 [out x in], 16-byte aligned: the weight the first stage
+ *            was made from
+ *   w1       host pointer to the first stage's descriptor (is_bf16 = 0);
+ *            out * in % 64 == 0
+ *   codes, absmax, absmax_q, absmax2   device outs for the second stage, laid out
+ *            as nf4_quantize's
+ *   workspace  nf4_quantize_residual_workspace_size(out * in) bytes, 16-byte
+ *            aligned (status word, counters, then R) */
+size_t nf4_quantize_residual_workspace_size(int64_t numel);
+qlora_status nf4_quantize_residual(const uint16_t* W, const qlora_weight* w1, nf4_qconfig q, uint8_t* codes,
+                                   float* absmax, uint8_t* absmax_q, float* absmax2, void* workspace,
+                                   size_t workspace_bytes, qlora_stream_t stream);
+
+/* The two-stage reconstruction the GEMM consumes:
+ *   W_out[i] = bf16_rn(fp32_rn(fp32_rn(c1 * a1) + fp32_rn(c2 * a2)))
+ *   w1, w2   host pointers to the two stages' descriptors (same out, in)
+ *   W_out    device out, bf16 [out x in], 16-byte aligned
+ * A layer stored this way runs the linear through the protected-layer (bf16)
+ * path on W_out. */
+qlora_status nf4_dequantize_two_stage(const qlora_weight* w1, const qlora_weight* w2, uint16_t* W_out,
+                                      qlora_stream_t stream);
 
 /* ------------------------------------------------------------ LoRA merge */
 

@@ -65,6 +65,10 @@ SIGNATURES = {
                                             c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                             c_void_p]),
     "nf4_k_from_fraction": (c_int, [c_int64, c_int64, c_int32, POINTER(c_int32)]),
+    "nf4_quantize_residual_workspace_size": (c_size_t, [c_int64]),
+    "nf4_quantize_residual": (c_int, [c_void_p, POINTER(QLoraWeight), NF4QConfig, c_void_p, c_void_p, c_void_p,
+                                      c_void_p, c_void_p, c_size_t, c_void_p]),
+    "nf4_dequantize_two_stage": (c_int, [POINTER(QLoraWeight), POINTER(QLoraWeight), c_void_p, c_void_p]),
     "nf4_layer_error_rank_noalloc": (c_int, [c_int32, POINTER(c_void_p), POINTER(c_int64), c_int32, NF4QConfig,
                                              c_int32, c_void_p, c_void_p, c_void_p, c_void_p]),
     "nf4_quantize_error_rank": (c_int, [c_int32, POINTER(c_void_p), POINTER(c_int64), c_int32, NF4QConfig, c_int32,

@@ -173,6 +173,40 @@ def dequantize(w: NF4Weight) -> torch.Tensor:
     return out
 
 
+def quantize_residual(W: torch.Tensor, w1: NF4Weight, double_quant: bool = False,
+                      keep_absmax: bool = False) -> NF4Weight:
+    """Second NF4 stage of W over the first stage w1: quantizes
+    R = fp32_rn(W - fp32_rn(c1 a1)) as quantize() would quantize an fp32 tensor."""
+    _need(W, torch.bfloat16, "W")
+    if tuple(W.shape) != (w1.out, w1.inp):
+        raise ValueError("W must have the first stage's shape")
+    lib = _lib.load()
+    dev = W.device
+    n = W.numel()
+    nb = (n + 63) // 64
+    o = NF4Weight(w1.out, w1.inp, double_quant,
+                  codes=torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev),
+                  absmax=torch.empty(nb, dtype=torch.float32, device=dev) if (not double_quant or keep_absmax) else None,
+                  absmax_q=torch.empty(nb, dtype=torch.uint8, device=dev) if double_quant else None,
+                  absmax2=torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev) if double_quant else None)
+    ws = Workspace.get(lib.nf4_quantize_residual_workspace_size(n), dev)
+    cs = w1.c_struct()
+    check(lib.nf4_quantize_residual(_ptr(W), ctypes.byref(cs), NF4QConfig(64, 1 if double_quant else 0, 256),
+                                    _ptr(o.codes), _ptr(o.absmax), _ptr(o.absmax_q), _ptr(o.absmax2), _ptr(ws),
+                                    ws.numel(), _stream()), "nf4_quantize_residual")
+    return o
+
+
+def dequantize_two_stage(w1: NF4Weight, w2: NF4Weight) -> torch.Tensor:
+    """bf16_rn(fp32_rn(v1 + v2)) of two NF4 stages, stored out x in."""
+    lib = _lib.load()
+    out = torch.empty((w1.out, w1.inp), dtype=torch.bfloat16, device=w1.codes.device)
+    c1, c2 = w1.c_struct(), w2.c_struct()
+    check(lib.nf4_dequantize_two_stage(ctypes.byref(c1), ctypes.byref(c2), _ptr(out), _stream()),
+          "nf4_dequantize_two_stage")
+    return out
+
+
 def lora_merge(w: NF4Weight, L1: torch.Tensor, L2: torch.Tensor, scale: float) -> torch.Tensor:
     """bf16 [out x in] = W_hat + scale (L1 L2)^T (a negative scale unmerges)."""
     _need(L1, torch.bfloat16, "L1")

@@ -512,7 +512,7 @@ qlora_status qlora_lora_merge(const qlora_weight* w, const uint16_t* L1, const u
 
 size_t qlora_lora_merge_requantize_workspace_size(int64_t out, int64_t in) {
   if (out <= 0 || in <= 0) return 0;
-  return kStatusBytes + up256(size_t(out) * size_t(in / 64) * sizeof(float));
+  return kReservedBytes + up256(size_t(out) * size_t(in / 64) * sizeof(float));
 }
 
 qlora_status qlora_lora_merge_requantize(const qlora_weight* w, const uint16_t* L1, const uint16_t* L2, int32_t r,
@@ -528,10 +528,62 @@ qlora_status qlora_lora_merge_requantize(const qlora_weight* w, const uint16_t* 
     return QLORA_ERR_WORKSPACE;
   QLB_TRY(check_device());
   // the exact fp32 scales go to the caller's absmax when given, else to the workspace
-  float* amax = absmax ? absmax : reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+  // (scratch after the split-K counters, which other calls on this workspace expect to find zero)
+  float* amax = absmax ? absmax : reinterpret_cast<float*>(static_cast<char*>(workspace) + kReservedBytes);
   QLB_TRY(merge_into(w, L1, L2, r, scale, nullptr, codes, amax, static_cast<int*>(workspace), S(stream)));
   if (q.double_quant) return launch_dq_scales(amax, w->out * (w->in / 64), absmax_q, absmax2, S(stream));
   return QLORA_OK;
+}
+
+namespace {
+qlora_status check_stage(const qlora_weight* w) {
+  if (!w) return QLORA_ERR_NULL;
+  if (w->is_bf16) return QLORA_ERR_UNSUPPORTED;
+  if (!qconfig_ok(w->q)) return QLORA_ERR_UNSUPPORTED;
+  if (w->out <= 0 || w->in <= 0 || (w->out * w->in) % 64) return QLORA_ERR_SHAPE;
+  if (!w->codes || (w->q.double_quant ? (!w->absmax_q || !w->absmax2) : !w->absmax)) return QLORA_ERR_NULL;
+  if (!aligned16(w->codes)) return QLORA_ERR_ALIGN;
+  return QLORA_OK;
+}
+}  // namespace
+
+size_t nf4_quantize_residual_workspace_size(int64_t numel) {
+  if (numel <= 0) return 0;
+  return kReservedBytes + up256(size_t(numel) * sizeof(float));
+}
+
+qlora_status nf4_quantize_residual(const uint16_t* W, const qlora_weight* w1, nf4_qconfig q, uint8_t* codes,
+                                   float* absmax, uint8_t* absmax_q, float* absmax2, void* workspace,
+                                   size_t workspace_bytes, qlora_stream_t stream) {
+  QLB_TRY(check_stage(w1));
+  if (!W) return QLORA_ERR_NULL;
+  if (!aligned16(W)) return QLORA_ERR_ALIGN;
+  if (!qconfig_ok(q)) return QLORA_ERR_UNSUPPORTED;
+  if (!codes || (q.double_quant ? (!absmax_q || !absmax2) : !absmax)) return QLORA_ERR_NULL;
+  if (!aligned16(codes)) return QLORA_ERR_ALIGN;
+  const int64_t numel = w1->out * w1->in;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < nf4_quantize_residual_workspace_size(numel))
+    return QLORA_ERR_WORKSPACE;
+  QLB_TRY(check_device());
+  // R after the split-K counters, which other calls on this workspace expect to find zero
+  float* R = reinterpret_cast<float*>(static_cast<char*>(workspace) + kReservedBytes);
+  QLB_TRY(launch_nf4_residual(W, w1->codes, w1->absmax, w1->absmax_q, w1->absmax2, w1->q.double_quant != 0, numel, R,
+                              S(stream)));
+  return launch_quantize(R, QLORA_DTYPE_F32, numel, q.double_quant != 0, codes, absmax, absmax_q, absmax2,
+                         static_cast<int*>(workspace), S(stream));
+}
+
+qlora_status nf4_dequantize_two_stage(const qlora_weight* w1, const qlora_weight* w2, uint16_t* W_out,
+                                      qlora_stream_t stream) {
+  QLB_TRY(check_stage(w1));
+  QLB_TRY(check_stage(w2));
+  if (w1->out != w2->out || w1->in != w2->in) return QLORA_ERR_SHAPE;
+  if (!W_out) return QLORA_ERR_NULL;
+  if (!aligned16(W_out)) return QLORA_ERR_ALIGN;
+  QLB_TRY(check_device());
+  return launch_dequantize_two_stage(w1->codes, w1->absmax, w1->absmax_q, w1->absmax2, w1->q.double_quant != 0,
+                                     w2->codes, w2->absmax, w2->absmax_q, w2->absmax2, w2->q.double_quant != 0,
+                                     w1->out * w1->in, W_out, S(stream));
 }
 
 qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream_t stream) {

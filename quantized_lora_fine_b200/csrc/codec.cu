@@ -713,6 +713,95 @@ qlora_status launch_dq_scales(const float* absmax, int64_t nb, uint8_t* absmax_q
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// ------------------------------------------------- residual NF4 second stage
+//
+// A protected layer may be stored as two NF4 stages instead of bf16: the second
+// quantizes what the first missed, R = fp32_rn(w - fp32_rn(c1 a1)), with the fp32
+// quantizer; the GEMM then consumes bf16_rn(fp32_rn(v1 + v2)), vi = fp32_rn(ci ai).
+// Both kernels: one thread per 8 elements (one code word), grid-stride, the 16 code
+// values in shared memory; numel % 64 == 0.
+struct NF4Stage {
+  const uint8_t* codes;
+  const float* absmax;
+  const uint8_t* absmax_q;
+  const float* absmax2;
+  int dq;
+};
+
+__global__ void __launch_bounds__(256) nf4_residual_kernel(const uint16_t* __restrict__ W, const NF4Stage s1,
+                                                           int64_t numel, float* __restrict__ R) {
+  __shared__ float s_code[16];
+  pdl_wait();
+  pdl_launch();
+  if (threadIdx.x < 16) s_code[threadIdx.x] = nf4_code(int(threadIdx.x));
+  __syncthreads();
+  const int64_t units = numel / 8;
+  for (int64_t u = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; u < units; u += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t e = u * 8;
+    const float a = block_scale(e / kBlock, s1.absmax, s1.absmax_q, s1.absmax2, s1.dq != 0);
+    const uint32_t cw = *reinterpret_cast<const uint32_t*>(s1.codes + e / 2);
+    const uint4 wv = *reinterpret_cast<const uint4*>(W + e);
+    const uint32_t wh[4] = {wv.x, wv.y, wv.z, wv.w};
+    float r[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {   // byte k: element 2k in the high nibble
+      const uint32_t b = (cw >> (8 * k)) & 0xFFu;
+      r[2 * k] = __fsub_rn(bf16_lo(wh[k]), __fmul_rn(s_code[b >> 4], a));
+      r[2 * k + 1] = __fsub_rn(bf16_hi(wh[k]), __fmul_rn(s_code[b & 15u], a));
+    }
+    float4* dst = reinterpret_cast<float4*>(R + e);
+    dst[0] = make_float4(r[0], r[1], r[2], r[3]);
+    dst[1] = make_float4(r[4], r[5], r[6], r[7]);
+  }
+}
+
+__global__ void __launch_bounds__(256) nf4_dequantize2_kernel(const NF4Stage s1, const NF4Stage s2, int64_t numel,
+                                                              uint16_t* __restrict__ out) {
+  __shared__ float s_code[16];
+  pdl_wait();
+  pdl_launch();
+  if (threadIdx.x < 16) s_code[threadIdx.x] = nf4_code(int(threadIdx.x));
+  __syncthreads();
+  const int64_t units = numel / 8;
+  for (int64_t u = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; u < units; u += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t e = u * 8;
+    const float a1 = block_scale(e / kBlock, s1.absmax, s1.absmax_q, s1.absmax2, s1.dq != 0);
+    const float a2 = block_scale(e / kBlock, s2.absmax, s2.absmax_q, s2.absmax2, s2.dq != 0);
+    const uint32_t c1 = *reinterpret_cast<const uint32_t*>(s1.codes + e / 2);
+    const uint32_t c2 = *reinterpret_cast<const uint32_t*>(s2.codes + e / 2);
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t b1 = (c1 >> (8 * k)) & 0xFFu, b2 = (c2 >> (8 * k)) & 0xFFu;
+      const float even = __fadd_rn(__fmul_rn(s_code[b1 >> 4], a1), __fmul_rn(s_code[b2 >> 4], a2));
+      const float odd = __fadd_rn(__fmul_rn(s_code[b1 & 15u], a1), __fmul_rn(s_code[b2 & 15u], a2));
+      o[k] = pack_bf16x2(even, odd);
+    }
+    *reinterpret_cast<uint4*>(out + e) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+qlora_status launch_nf4_residual(const uint16_t* W, const uint8_t* codes, const float* absmax,
+                                 const uint8_t* absmax_q, const float* absmax2, bool dq, int64_t numel, float* R,
+                                 cudaStream_t st) {
+  const NF4Stage s1{codes, absmax, absmax_q, absmax2, dq ? 1 : 0};
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((numel / 8 + 255) / 256, int64_t(num_sms()) * 8));
+  const cudaError_t e = launch_pdl(nf4_residual_kernel, dim3(unsigned(blocks)), dim3(256), 0, st, W, s1, numel, R);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status launch_dequantize_two_stage(const uint8_t* codes1, const float* absmax1, const uint8_t* absmax_q1,
+                                         const float* absmax2_1, bool dq1, const uint8_t* codes2,
+                                         const float* absmax_2, const uint8_t* absmax_q2, const float* absmax2_2,
+                                         bool dq2, int64_t numel, uint16_t* out, cudaStream_t st) {
+  const NF4Stage s1{codes1, absmax1, absmax_q1, absmax2_1, dq1 ? 1 : 0};
+  const NF4Stage s2{codes2, absmax_2, absmax_q2, absmax2_2, dq2 ? 1 : 0};
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((numel / 8 + 255) / 256, int64_t(num_sms()) * 8));
+  const cudaError_t e =
+      launch_pdl(nf4_dequantize2_kernel, dim3(unsigned(blocks)), dim3(256), 0, st, s1, s2, numel, out);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 // ------------------------------------------------------- expanded GEMM scales
 
 __global__ void expand_scales_kernel(const float* __restrict__ absmax, const uint8_t* __restrict__ absmax_q,

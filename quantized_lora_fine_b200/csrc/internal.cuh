@@ -80,6 +80,15 @@ qlora_status launch_lora_merge(const uint8_t* codes, const float* absmax, const 
                                const float* absmax2, bool dq, const uint16_t* Wbf, int64_t out, int64_t in,
                                const uint16_t* L1, const uint16_t* L2, int r, double s, uint16_t* W_out,
                                uint8_t* q_codes, float* q_absmax, int* status, cudaStream_t st);
+// R = fp32_rn(w - fp32_rn(c1 a1)) for the first NF4 stage (codes, scales); numel % 64 == 0.
+qlora_status launch_nf4_residual(const uint16_t* W, const uint8_t* codes, const float* absmax,
+                                 const uint8_t* absmax_q, const float* absmax2, bool dq, int64_t numel, float* R,
+                                 cudaStream_t st);
+// out = bf16_rn(fp32_rn(v1 + v2)) of two NF4 stages; numel % 64 == 0.
+qlora_status launch_dequantize_two_stage(const uint8_t* codes1, const float* absmax1, const uint8_t* absmax_q1,
+                                         const float* absmax2_1, bool dq1, const uint8_t* codes2,
+                                         const float* absmax_2, const uint8_t* absmax_q2, const float* absmax2_2,
+                                         bool dq2, int64_t numel, uint16_t* out, cudaStream_t st);
 // Double-quantize a finished fp32 absmax array (nb scales, groups of 256).
 qlora_status launch_dq_scales(const float* absmax, int64_t nb, uint8_t* absmax_q, float* absmax2, cudaStream_t st);
 // ---- layer_error.cu

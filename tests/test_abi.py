@@ -172,3 +172,27 @@ def test_empty_inputs_are_refused_on_the_host(lib):
     m.codes, m.absmax = 0x2000, 0x3000
     assert lib.qlora_lora_merge(ctypes.byref(m), 0x1000, 0x1000, 8, 2.0, 0x4000, None) == 2
     assert lib.qlora_lora_merge_requantize_workspace_size(0, 64) == 0
+
+
+def test_residual_stage_host_validation(lib):
+    q = _lib.NF4QConfig(64, 0, 256)
+    w1 = _lib.QLoraWeight()
+    w1.out, w1.in_, w1.q = 128, 64, q
+    w1.codes, w1.absmax = 0x2000, 0x3000
+    need = lib.nf4_quantize_residual_workspace_size(128 * 64)
+    assert need >= 128 * 64 * 4
+    assert lib.nf4_quantize_residual(0x1000, ctypes.byref(w1), q, 0x5000, 0x6000, None, None, 0x7000, need - 1,
+                                     None) == 7
+    assert lib.nf4_quantize_residual(0x1001, ctypes.byref(w1), q, 0x5000, 0x6000, None, None, 0x7000, need,
+                                     None) == 3
+    assert lib.nf4_quantize_residual(None, ctypes.byref(w1), q, 0x5000, 0x6000, None, None, 0x7000, need, None) == 1
+    w1.is_bf16 = 1
+    assert lib.nf4_quantize_residual(0x1000, ctypes.byref(w1), q, 0x5000, 0x6000, None, None, 0x7000, need,
+                                     None) == 5
+    w1.is_bf16 = 0
+    w2 = _lib.QLoraWeight()
+    w2.out, w2.in_, w2.q = 64, 128, q
+    w2.codes, w2.absmax = 0x2000, 0x3000
+    assert lib.nf4_dequantize_two_stage(ctypes.byref(w1), ctypes.byref(w2), 0x8000, None) == 2
+    w1.in_ = 63
+    assert lib.nf4_dequantize_two_stage(ctypes.byref(w1), ctypes.byref(w2), 0x8000, None) == 2

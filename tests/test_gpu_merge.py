@@ -229,3 +229,20 @@ def test_merge_requantize_every_bf16_value(cuda_device, exp, sigs):
     assert api.status() == 0
     assert np.array_equal(o.codes.cpu().numpy(), qw["codes"])
     assert np.array_equal(o.absmax.cpu().numpy().view(np.uint32), qw["absmax"].view(np.uint32))
+
+
+def test_linear_after_requantize_on_the_same_workspace(cuda_device):
+    """Calls on one stream share one workspace: a merge + re-quantize (whose scratch
+    holds fp32 scales) followed by the linear still gives the oracle's Y, i.e. the
+    scratch stays clear of the split-K counters the linear relies on."""
+    case = synth.LinearCase("after-requant", M=512, out=512, inp=768, r=16, alpha=32.0, double_quant=True, seed=11)
+    d = case.make()
+    g, w = gpu_case(d, True)
+    api.lora_merge_requantize(w, g["L1"], g["L2"], case.scale, double_quant=True)
+    Y, _ = api.linear_fwd(w, g["X"], g["L1"], g["L2"], case.scale)
+    torch.cuda.synchronize()
+    What = oracle_what(oracle_qweight(d["W"], True))
+    X, L1, L2 = (f64_of_bf16(d[k]) for k in ("X", "L1", "L2"))
+    Yref, _ = lora.forward(X, What, L1, L2, case.scale)
+    from tests.gpu_helpers import assert_close
+    assert_close(f64_of_bf16(Y), Yref, "Y")
