@@ -233,10 +233,12 @@ qlora_status qlora_lora_merge_requantize(const qlora_weight* w, const uint16_t* 
 
 /* --------------------------------------------------------- NF4-LoRA linear */
 
-/* Shape rules for the linear: in % 256 == 0, out % 256 == 0, 1 <= M <= 2^21,
- * r % 8 == 0 and 8 <= r <= 256; every pointer 16-byte aligned. The workspace
- * holds, after the status word, 64 KiB of split-K tile counters that the
- * kernels leave at zero: zero a fresh workspace once before its first use. */
+/* Shape rules for the linear: in % 256 == 0, out % 256 == 0, 1 <= M <= 2^20
+ * and in, out <= 2^20, r % 8 == 0 and 8 <= r <= 256; every pointer 16-byte
+ * aligned. The workspace holds, after the status word, 64 KiB of split-K tile
+ * counters that the kernels leave at zero: zero a fresh workspace once before
+ * its first use. A workspace serves one call at a time: calls that may run at
+ * the same time (on different streams) need different workspaces. */
 size_t qlora_fwd_workspace_size(int64_t M, int64_t out, int64_t in, int32_t r);
 size_t qlora_bwd_workspace_size(int64_t M, int64_t out, int64_t in, int32_t r);
 

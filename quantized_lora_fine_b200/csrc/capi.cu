@@ -103,8 +103,9 @@ qlora_status check_linear(const qlora_weight* w, int64_t M, int32_t r) {
   if (w->out <= 0 || w->in <= 0 || M <= 0) return QLORA_ERR_SHAPE;
   if (w->in % 256 || w->out % 256) return QLORA_ERR_SHAPE;
   if (w->in > (int64_t(1) << 30) || w->out > (int64_t(1) << 30) || M > (int64_t(1) << 30)) return QLORA_ERR_SHAPE;
-  // split-K tile counters: one per 128 rows of M, out or in
-  if ((std::max({M, w->out, w->in}) + 127) / 128 > kMaxCounterTiles) return QLORA_ERR_SHAPE;
+  // split-K tile counters: one per 128 rows of M, out or in; the backward runs two
+  // products at once, each on its own half of the counters
+  if ((std::max({M, w->out, w->in}) + 127) / 128 > kMaxCounterTiles / 2) return QLORA_ERR_SHAPE;
   if (r < 8 || r > 256 || r % 8) return QLORA_ERR_SHAPE;
   if (w->is_bf16) {
     if (!w->w_bf16) return QLORA_ERR_NULL;

@@ -196,3 +196,20 @@ def test_residual_stage_host_validation(lib):
     assert lib.nf4_dequantize_two_stage(ctypes.byref(w1), ctypes.byref(w2), 0x8000, None) == 2
     w1.in_ = 63
     assert lib.nf4_dequantize_two_stage(ctypes.byref(w1), ctypes.byref(w2), 0x8000, None) == 2
+
+
+def test_linear_size_limits(lib):
+    """M, in and out are limited to 2^20 (8192 counter tiles each: the backward's two
+    concurrent split-K products use one half of the 16384 counters each)."""
+    q = _lib.NF4QConfig(64, 0, 256)
+    w = _lib.QLoraWeight()
+    w.out, w.in_, w.q = 256, 256, q
+    w.codes, w.absmax = 0x2000, 0x3000
+    big = (1 << 20) + 128
+    assert lib.qlora_linear_fwd(ctypes.byref(w), 0x1000, big, 0x1000, 0x1000, 16, 2.0, 0x1000, None, 0x4000,
+                                1 << 40, None) == 2
+    assert lib.qlora_linear_bwd(ctypes.byref(w), 0x1000, 0x1000, big, 0x1000, 0x1000, 16, 2.0, 0x1000, 0x1000,
+                                0x1000, 0x1000, 0x4000, 1 << 40, None) == 2
+    w.in_ = (1 << 20) + 256
+    assert lib.qlora_linear_fwd(ctypes.byref(w), 0x1000, 8, 0x1000, 0x1000, 16, 2.0, 0x1000, None, 0x4000,
+                                1 << 40, None) == 2
