@@ -213,3 +213,20 @@ def test_linear_size_limits(lib):
     w.in_ = (1 << 20) + 256
     assert lib.qlora_linear_fwd(ctypes.byref(w), 0x1000, 8, 0x1000, 0x1000, 16, 2.0, 0x1000, None, 0x4000,
                                 1 << 40, None) == 2
+
+
+def test_workspace_sizes_reserve_the_counter_region(lib):
+    """Entry points share one workspace per stream: bytes [256, 256 + 64 KiB) hold
+    split-K counters that every call must find zero, so any call with scratch
+    sizes its workspace past them (status 256 + counters 65536 + scratch)."""
+    reserved = 256 + 65536
+    n = 4096 * 4096
+    assert lib.nf4_quantize_residual_workspace_size(n) >= reserved + 4 * n
+    assert lib.qlora_lora_merge_requantize_workspace_size(4096, 4096) >= reserved + 4 * n // 64
+    assert lib.qlora_fwd_workspace_size(8192, 4096, 4096, 16) >= reserved + 4096 * 64 * 4
+    assert lib.qlora_bwd_workspace_size(8192, 4096, 4096, 16) >= reserved
+    assert lib.qlora_lora_down_workspace_size(8192, 4096, 16) >= reserved + 8192 * 16 * 4
+    nn = (ctypes.c_int64 * 2)(n, n)
+    assert lib.nf4_layer_error_rank_workspace_size(2, nn) >= reserved + 2 * (n // 16384) * 16
+    # the quantizer keeps only the status word and no scratch
+    assert lib.nf4_quantize_workspace_size(n) == 256
