@@ -541,7 +541,8 @@ qlora_status check_stage(const qlora_weight* w) {
   if (!w) return QLORA_ERR_NULL;
   if (w->is_bf16) return QLORA_ERR_UNSUPPORTED;
   if (!qconfig_ok(w->q)) return QLORA_ERR_UNSUPPORTED;
-  if (w->out <= 0 || w->in <= 0 || (w->out * w->in) % 64) return QLORA_ERR_SHAPE;
+  if (w->out <= 0 || w->in <= 0 || w->out > (int64_t(1) << 30) || w->in > (int64_t(1) << 30)) return QLORA_ERR_SHAPE;
+  if ((w->out * w->in) % 64) return QLORA_ERR_SHAPE;
   if (!w->codes || (w->q.double_quant ? (!w->absmax_q || !w->absmax2) : !w->absmax)) return QLORA_ERR_NULL;
   if (!aligned16(w->codes)) return QLORA_ERR_ALIGN;
   return QLORA_OK;

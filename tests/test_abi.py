@@ -196,6 +196,8 @@ def test_residual_stage_host_validation(lib):
     assert lib.nf4_dequantize_two_stage(ctypes.byref(w1), ctypes.byref(w2), 0x8000, None) == 2
     w1.in_ = 63
     assert lib.nf4_dequantize_two_stage(ctypes.byref(w1), ctypes.byref(w2), 0x8000, None) == 2
+    w1.in_ = (1 << 30) + 64
+    assert lib.nf4_dequantize_two_stage(ctypes.byref(w1), ctypes.byref(w2), 0x8000, None) == 2
 
 
 def test_linear_size_limits(lib):
