@@ -130,8 +130,8 @@ int32_t qlora_pair_clusters(void);
 /* Bytes of workspace nf4_quantize needs (the status word only). */
 size_t nf4_quantize_workspace_size(int64_t numel);
 
-/* Blockwise NF4 quantization of W (numel = out*in elements, any even count;
- * a short last block uses the elements present).
+/* Blockwise NF4 quantization of W (numel = out*in elements, any even count up to
+ * 2^40, else QLORA_ERR_SHAPE; a short last block uses the elements present).
  *   W        device, bf16 (w_dtype QLORA_DTYPE_BF16) or fp32, 16-byte aligned
  *   codes    device out, uint8 [numel/2]
  *   absmax   device out, fp32 [ceil(numel/64)]; required when double_quant = 0,
@@ -149,7 +149,7 @@ qlora_status nf4_quantize(const void* W, int32_t w_dtype, int64_t out, int64_t i
                           void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
 /* The same quantization for n bf16 matrices in one launch (a whole model at
- * load time): matrix i is W_ptrs[i] (numel[i] elements, even) with its own
+ * load time): matrix i is W_ptrs[i] (numel[i] elements, even, <= 2^40) with its own
  * codes[i], absmax[i] / absmax_q[i], absmax2[i] laid out as for nf4_quantize;
  * every bit is the one nf4_quantize gives that matrix alone.
  *   n        1 <= n <= 512
@@ -165,7 +165,8 @@ qlora_status nf4_quantize_batch(int32_t n, const uint16_t* const* W_ptrs, const 
 
 /* Dequantization to bf16: W_out[i] = bf16_rn(fp32_rn(code[idx_i] * a)) with a the
  * block's absmax, or with double quantization a = fp32_rn(fp32(q_b) * absmax2[g]).
- *   w      host pointer to a descriptor with is_bf16 = 0 (device buffers inside)
+ *   w      host pointer to a descriptor with is_bf16 = 0 (device buffers inside);
+ *          out * in even and at most 2^40
  *   W_out  device out, bf16 [out*in], 16-byte aligned */
 qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream_t stream);
 
@@ -181,7 +182,7 @@ qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream
  *   W        device bf16 [out x in], 16-byte aligned: the weight the first stage
  *            was made from
  *   w1       host pointer to the first stage's descriptor (is_bf16 = 0);
- *            out * in % 64 == 0
+ *            out, in <= 2^30, out * in % 64 == 0 and out * in <= 2^40
  *   codes, absmax, absmax_q, absmax2   device outs for the second stage, laid out
  *            as nf4_quantize's
  *   workspace  nf4_quantize_residual_workspace_size(out * in) bytes, 16-byte
@@ -302,11 +303,14 @@ size_t nf4_layer_error_rank_workspace_size(int32_t n_layers, const int64_t* nume
 /* Per-layer NF4 reconstruction error, ranking and top-K selection.
  *   W_ptrs   HOST array of n_layers DEVICE pointers, each a bf16 matrix
  *            (w_dtype must be QLORA_DTYPE_BF16), 16-byte aligned
- *   numel    HOST array of element counts (each a positive multiple of 64)
+ *   numel    HOST array of element counts (each a positive multiple of 64, at
+ *            most 2^40; at most 2^31 - 1 chunks of 16384 in all)
  *   q        quantization config used for every layer (double_quant 0 or 1)
  *   K        number of layers to keep (0 <= K <= n_layers)
  *   err      device out, fp64 [n_layers]: e = sqrt(sum (w - w_hat)^2 / sum w^2)
  *            with w_hat the bf16 dequantized weight (0 for an all-zero matrix)
+ *            A NaN or +-Inf weight sets QLORA_ERR_NONFINITE in the status word and
+ *            leaves that layer's err unspecified (NaN errors rank first, by id).
  *   order    device out, int32 [n_layers]: layer ids by (err desc, id asc)
  *   keep     device out, uint8 [n_layers]: 1 for the first K of `order`
  * 1 <= n_layers <= 1024. Sums run in fp64 in a fixed order (deterministic). */
@@ -383,8 +387,10 @@ qlora_status nf4_quantize_error_rank(int32_t n_layers, const uint16_t* const* W_
  *   - every call on a device uses the same array, so calls that overlap on the
  *     GPU (different streams or host threads) race and must be serialized by the
  *     caller; nothing needs clearing between calls;
- *   - there is no device status word: a layer that contains NaN or +-Inf gets
- *     err = NaN.
+ *   - there is no device status word. A layer that contains NaN or +-Inf, or a
+ *     chunk of it whose bulk copy into shared memory timed out, gets err = NaN;
+ *     NaN errors rank ahead of every finite error (among themselves by layer
+ *     id), so `order` stays a permutation and such layers are the first kept.
  * Allocates no device memory and calls no allocating routine. */
 qlora_status nf4_layer_error_rank_noalloc(int32_t n_layers, const uint16_t* const* W_ptrs, const int64_t* numel,
                                           int32_t w_dtype, nf4_qconfig q, int32_t K,

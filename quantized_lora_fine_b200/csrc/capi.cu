@@ -18,6 +18,13 @@ constexpr int kThinTargetCtas = 148;  // split-K target for the thin LoRA produc
                                       // (fixed: results do not depend on the device's SM count)
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// out x in matrices of the codec entry points: both positive and at most 2^40
+// elements in all (the grids count chunks of 16384 elements in 32 bits, and
+// every byte count stays far inside 64 bits).
+constexpr int64_t kMaxCodecNumel = int64_t(1) << 40;
+inline bool codec_dims_ok(int64_t out, int64_t in) {
+  return out > 0 && in > 0 && out <= kMaxCodecNumel && in <= kMaxCodecNumel / out;
+}
 inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 inline cudaStream_t S(qlora_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -441,7 +448,7 @@ qlora_status nf4_quantize(const void* W, int32_t w_dtype, int64_t out, int64_t i
                           qlora_stream_t stream) {
   if (w_dtype != QLORA_DTYPE_BF16 && w_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
   if (!qconfig_ok(q)) return QLORA_ERR_UNSUPPORTED;
-  if (out <= 0 || in <= 0) return QLORA_ERR_SHAPE;
+  if (!codec_dims_ok(out, in)) return QLORA_ERR_SHAPE;
   const int64_t numel = out * in;
   if (numel % 2) return QLORA_ERR_SHAPE;
   if (!W || !codes) return QLORA_ERR_NULL;
@@ -467,7 +474,7 @@ qlora_status nf4_quantize_batch(int32_t n, const uint16_t* const* W_ptrs, const 
   for (int i = 0; i < n; ++i) {
     if (!W_ptrs[i] || !codes[i]) return QLORA_ERR_NULL;
     if (dq ? (!absmax_q[i] || !absmax2[i]) : !absmax[i]) return QLORA_ERR_NULL;
-    if (numel[i] <= 0 || numel[i] % 2) return QLORA_ERR_SHAPE;
+    if (numel[i] <= 0 || numel[i] % 2 || numel[i] > kMaxCodecNumel) return QLORA_ERR_SHAPE;
     if (!aligned16(W_ptrs[i]) || !aligned16(codes[i])) return QLORA_ERR_ALIGN;
   }
   if (!workspace || workspace_bytes < kStatusBytes || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
@@ -542,6 +549,7 @@ qlora_status check_stage(const qlora_weight* w) {
   if (w->is_bf16) return QLORA_ERR_UNSUPPORTED;
   if (!qconfig_ok(w->q)) return QLORA_ERR_UNSUPPORTED;
   if (w->out <= 0 || w->in <= 0 || w->out > (int64_t(1) << 30) || w->in > (int64_t(1) << 30)) return QLORA_ERR_SHAPE;
+  if (!codec_dims_ok(w->out, w->in)) return QLORA_ERR_SHAPE;
   if ((w->out * w->in) % 64) return QLORA_ERR_SHAPE;
   if (!w->codes || (w->q.double_quant ? (!w->absmax_q || !w->absmax2) : !w->absmax)) return QLORA_ERR_NULL;
   if (!aligned16(w->codes)) return QLORA_ERR_ALIGN;
@@ -592,7 +600,7 @@ qlora_status nf4_dequantize(const qlora_weight* w, uint16_t* W_out, qlora_stream
   if (!w || !W_out) return QLORA_ERR_NULL;
   if (w->is_bf16) return QLORA_ERR_UNSUPPORTED;
   if (!qconfig_ok(w->q)) return QLORA_ERR_UNSUPPORTED;
-  if (w->out <= 0 || w->in <= 0) return QLORA_ERR_SHAPE;
+  if (!codec_dims_ok(w->out, w->in)) return QLORA_ERR_SHAPE;
   const int64_t numel = w->out * w->in;
   if (numel % 2) return QLORA_ERR_SHAPE;
   if (!w->codes) return QLORA_ERR_NULL;
@@ -800,9 +808,10 @@ qlora_status nf4_layer_error_rank(int32_t n_layers, const uint16_t* const* W_ptr
   if (!W_ptrs || !numel || !err || !order || !keep) return QLORA_ERR_NULL;
   for (int i = 0; i < n_layers; ++i) {
     if (!W_ptrs[i]) return QLORA_ERR_NULL;
-    if (numel[i] <= 0 || numel[i] % 64) return QLORA_ERR_SHAPE;
+    if (numel[i] <= 0 || numel[i] % 64 || numel[i] > kMaxCodecNumel) return QLORA_ERR_SHAPE;
     if (!aligned16(W_ptrs[i])) return QLORA_ERR_ALIGN;
   }
+  if (noalloc_chunks(n_layers, numel) > int64_t(INT32_MAX)) return QLORA_ERR_SHAPE;   // chunk ids are 32-bit
   if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
   QLB_TRY(check_device());
   return launch_layer_error_rank(n_layers, W_ptrs, numel, q.double_quant != 0, K, err, order, keep, workspace,
@@ -822,6 +831,7 @@ qlora_status nf4_layer_error_rank_budget(int32_t n_layers, const uint16_t* const
     if (numel[i] <= 0 || numel[i] % 64 || numel[i] > (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
     if (!aligned16(W_ptrs[i])) return QLORA_ERR_ALIGN;
   }
+  if (noalloc_chunks(n_layers, numel) > int64_t(INT32_MAX)) return QLORA_ERR_SHAPE;   // chunk ids are 32-bit
   if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
   QLB_TRY(check_device());
   return launch_layer_error_rank(n_layers, W_ptrs, numel, q.double_quant != 0, 0, err, order, keep, workspace,
@@ -852,9 +862,10 @@ qlora_status nf4_quantize_error_rank(int32_t n_layers, const uint16_t* const* W_
     if (!W_ptrs[i] || !codes[i]) return QLORA_ERR_NULL;
     if (dq && (!absmax_q[i] || !absmax2[i])) return QLORA_ERR_NULL;
     if (!dq && !absmax[i]) return QLORA_ERR_NULL;
-    if (numel[i] <= 0 || numel[i] % 64) return QLORA_ERR_SHAPE;
+    if (numel[i] <= 0 || numel[i] % 64 || numel[i] > kMaxCodecNumel) return QLORA_ERR_SHAPE;
     if (!aligned16(W_ptrs[i]) || !aligned16(codes[i])) return QLORA_ERR_ALIGN;
   }
+  if (noalloc_chunks(n_layers, numel) > int64_t(INT32_MAX)) return QLORA_ERR_SHAPE;   // chunk ids are 32-bit
   if (!workspace || !aligned16(workspace)) return QLORA_ERR_WORKSPACE;
   QLB_TRY(check_device());
   return launch_quantize_error_rank(n_layers, W_ptrs, numel, dq, K, codes, absmax, absmax_q, absmax2, err, order,
@@ -870,7 +881,7 @@ qlora_status nf4_layer_error_rank_noalloc(int32_t n_layers, const uint16_t* cons
   if (!W_ptrs || !numel || !err || !order || !keep) return QLORA_ERR_NULL;
   for (int i = 0; i < n_layers; ++i) {
     if (!W_ptrs[i]) return QLORA_ERR_NULL;
-    if (numel[i] <= 0 || numel[i] % 64) return QLORA_ERR_SHAPE;
+    if (numel[i] <= 0 || numel[i] % 64 || numel[i] > kMaxCodecNumel) return QLORA_ERR_SHAPE;
     if (!aligned16(W_ptrs[i])) return QLORA_ERR_ALIGN;
   }
   if (noalloc_chunks(n_layers, numel) > (int64_t(1) << 20)) return QLORA_ERR_SHAPE;

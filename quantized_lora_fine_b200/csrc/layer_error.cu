@@ -124,7 +124,13 @@ __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_
   }
   const bool landed = mbar_wait(bar, 0);
   if (!__syncthreads_and(landed)) {   // every thread leaves together
-    if (tid == 0 && status) set_status(status, QLORA_ERR_TIMEOUT);
+    if (tid == 0) {
+      if (status) set_status(status, QLORA_ERR_TIMEOUT);
+      // the chunk's partial still gets written: NaN, so the layer's error shows the
+      // failure instead of a sum left over from an earlier call
+      partial[chunk] = make_double2(__longlong_as_double(0x7FF8000000000000ll),
+                                    __longlong_as_double(0x7FF8000000000000ll));
+    }
     if (!landed) mbar_wait(bar, 0, 20000000000ull);   // the copy must land before the CTA's memory is released
     return;
   }
@@ -219,6 +225,12 @@ __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_
     sd += double(f2_lo(sd2[h])) + double(f2_hi(sd2[h]));
     sw += double(f2_lo(sw2[h])) + double(f2_hi(sw2[h]));
   }
+  if (bad && !status) {
+    // without a status word the non-finite block is reported through the sums:
+    // NaN reaches the chunk's partial and the layer's error
+    sd = __longlong_as_double(0x7FF8000000000000ll);
+    sw = sd;
+  }
   s_part[tid] = make_double2(sd, sw);
   __syncthreads();
   if (warp != 0) return;
@@ -255,16 +267,23 @@ __device__ __forceinline__ void finish_layer_warp(const double2* __restrict__ pa
     a += __shfl_xor_sync(0xffffffffu, a, o);
     b += __shfl_xor_sync(0xffffffffu, b, o);
   }
-  if (lane == 0) *err_out = (b > 0.0) ? sqrt(a / b) : 0.0;
+  // an all-zero layer has error 0; a NaN sum (non-finite block or timed-out copy on
+  // the path without a status word) gives NaN
+  if (lane == 0) *err_out = (b == 0.0) ? 0.0 : sqrt(a / b);
 }
 
-// Position of layer l in the order (error descending, index ascending).
+// Position of layer l in the order (error descending, index ascending). A NaN
+// error (only the path without a status word produces one) ranks ahead of every
+// number, NaN layers among themselves by index, so the order stays a permutation.
 __device__ __forceinline__ int rank_of(const double* s_err, int n_layers, int l) {
   const double e = s_err[l];
+  const bool en = isnan(e);
   int rank = 0;
   for (int j = 0; j < n_layers; ++j) {
     const double f = s_err[j];
-    rank += (f > e || (f == e && j < l)) ? 1 : 0;
+    const bool fn = isnan(f);
+    const bool before = (fn != en) ? fn : (en ? (j < l) : (f > e || (f == e && j < l)));
+    rank += before ? 1 : 0;
   }
   return rank;
 }
@@ -451,7 +470,9 @@ qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_p
 // up to 2^34 weights per call); every GPU that loads the library keeps it
 // until the process exits. All calls share it: calls that overlap on the GPU
 // (two streams, two host threads) race on it. Each call overwrites every
-// partial it reads, so nothing has to be cleared between calls.
+// partial it reads (a chunk whose copy timed out writes NaN), so nothing has to be
+// cleared between calls. There is no status word on this path: a non-finite block
+// or a timed-out copy turns its chunk's partial, and so the layer's error, into NaN.
 
 constexpr int64_t kNoAllocMaxChunks = int64_t(1) << 20;
 static __device__ __align__(256) double2 g_noalloc_partials[kNoAllocMaxChunks];

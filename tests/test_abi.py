@@ -198,6 +198,26 @@ def test_residual_stage_host_validation(lib):
     assert lib.nf4_dequantize_two_stage(ctypes.byref(w1), ctypes.byref(w2), 0x8000, None) == 2
     w1.in_ = (1 << 30) + 64
     assert lib.nf4_dequantize_two_stage(ctypes.byref(w1), ctypes.byref(w2), 0x8000, None) == 2
+    # each side within 2^30 but their product past the 2^40-element limit: refused,
+    # not quantized in part
+    w1.out, w1.in_ = 1 << 30, (1 << 10) + 64
+    assert lib.nf4_quantize_residual(0x1000, ctypes.byref(w1), q, 0x5000, 0x6000, None, None, 0x7000, 1 << 62,
+                                     None) == 2
+    w2.out, w2.in_ = w1.out, w1.in_
+    assert lib.nf4_dequantize_two_stage(ctypes.byref(w1), ctypes.byref(w2), 0x8000, None) == 2
+
+
+def test_codec_element_limit(lib):
+    """Quantize and dequantize take at most 2^40 elements (out * in), checked without
+    overflow however large each side is."""
+    q = _lib.NF4QConfig(64, 0, 256)
+    for out, inn in (((1 << 40) + 64, 1), (1 << 21, (1 << 19) + 64), ((1 << 62), 1 << 62)):
+        assert lib.nf4_quantize(0x1000, _lib.DTYPE_BF16, out, inn, q, 0x2000, 0x3000, None, None, 0x4000, 256,
+                                None) == 2
+        w = _lib.QLoraWeight()
+        w.out, w.in_, w.q = out, inn, q
+        w.codes, w.absmax = 0x2000, 0x3000
+        assert lib.nf4_dequantize(ctypes.byref(w), 0x5000, None) == 2
 
 
 def test_linear_size_limits(lib):
