@@ -42,6 +42,27 @@ def test_quant_student_t_ragged_groups(cuda_device):
     _check_quant(synth.student_t_bf16((300, 192), 3.0, 0.02, 1, synth.STREAM_W), dq=True)
 
 
+def test_double_quant_hand_worked_group(cuda_device):
+    """The hand-worked double-quant group of the oracle's pins (block maxima
+    203 * 2^-20 and 49 * 2^-12): E4M3 scale bytes 0x4F and 0x7E, factor 7 * 2^-18,
+    through the GPU quantizer and through the fused allocation pass."""
+    W = torch.zeros((2, 64), dtype=torch.float32)
+    W[0, 11] = -203 * 2.0 ** -20
+    W[1, 40] = 49 * 2.0 ** -12
+    W[0, 3] = 2.0 ** -20          # a smaller weight in each block, so the codes are not all zero
+    W[1, 5] = -2.0 ** -9
+    Wb = W.to(torch.bfloat16)
+    g = api.quantize(Wb.cuda(), double_quant=True)
+    torch.cuda.synchronize()
+    assert g.absmax_q.cpu().tolist() == [0x4F, 0x7E]
+    assert g.absmax2.cpu().tolist() == [7 * 2.0 ** -18]
+    _check_quant(Wb, dq=True)
+    _, _, _, outs = api.quantize_error_rank([Wb.cuda()], 0, double_quant=True)
+    torch.cuda.synchronize()
+    assert outs[0].absmax_q.cpu().tolist() == [0x4F, 0x7E]
+    assert outs[0].absmax2.cpu().tolist() == [7 * 2.0 ** -18]
+
+
 def test_quant_partial_tail_block(cuda_device):
     W = synth.normal_bf16((7, 38), 0.5, 2, synth.STREAM_W)   # 266 elements: 4 full blocks + 10
     _check_quant(W, dq=False)

@@ -254,6 +254,56 @@ def test_double_quant_group_structure():
     assert np.all(np.abs(ahat[nz] - a[nz]) <= a[nz] * 2.0 ** -4 * 1.0001)
 
 
+def pin_double_quant_hand_case():
+    """A two-block group worked by hand in exact arithmetic (bf16 inputs).
+
+    G = 49 * 2^-12 (bf16 0x3C44) is the group maximum and a = 203 * 2^-20 (bf16
+    0x394B) the other scale.
+      448 / G = 37449 + 1/7; fp32 spacing there is 2^-8, and 1/7 = 36.57 * 2^-8,
+      so inv = fp32(448 / G) = 37449 + 37/256 (above 448 / G by 3/1792).
+      a * inv = 7.25 + 87 * 2^-28 exactly; fp32 spacing in [4, 8) is 2^-21 =
+      128 * 2^-28, so fp32(a * inv) = 7.25 + 2^-21. E4M3 spacing in [4, 8) is 0.5:
+      7.25 is the midpoint of 7.0 and 7.5, and the value lies above it -> 7.5
+      (exponent 2 + 7 = 9, mantissa 7: byte 0x4F).
+      G * inv = 448.0000086 -> fp32 448.000030517578125 -> saturates to 448 (0x7E).
+      f = fp32(G / 448) = 7 * 2^-18 exactly; a_hat = 7.5 * 7 * 2^-18 = 52.5 * 2^-18.
+    Two plausible slips land exactly on the midpoint instead and round to the even
+    neighbour 7.0 (0x4E): a * (448 / G) without rounding 448 / G first (= 7.25), and
+    a / f (= 7.25)."""
+    a = np.array([203 * 2.0 ** -20, 49 * 2.0 ** -12], np.float32)
+    assert nf4.bf16_bits_from_f32(a).tolist() == [0x394B, 0x3C44]
+    q, f = nf4.double_quantize(a)
+    assert q.tolist() == [0x4F, 0x7E], [hex(v) for v in q]
+    assert f.tolist() == [7 * 2.0 ** -18]
+    assert nf4.dq_scales(q, f).tolist() == [52.5 * 2.0 ** -18, 448 * 7 * 2.0 ** -18]
+
+
+def test_double_quant_hand_worked_group():
+    pin_double_quant_hand_case()
+
+
+def test_double_quant_pin_catches_planted_slips(monkeypatch):
+    """The hand-worked group fails for the two slips it was chosen against (CPU)."""
+    orig = nf4.double_quantize
+
+    def make(rule):
+        def dq(absmax, dq_blocksize=nf4.DQ_BLOCKSIZE):
+            a = np.asarray(absmax, np.float32).reshape(-1)
+            G = np.float32(a.max())
+            if rule == "unrounded":   # a * 448 / G in fp64, one rounding to fp32
+                scaled = (a.astype(np.float64) * 448.0 / np.float64(G)).astype(np.float32)
+            else:                     # a / fp32(G / 448)
+                scaled = (a / np.float32(G / np.float32(448))).astype(np.float32)
+            return nf4.e4m3_encode_satfinite(scaled), np.array([G / np.float32(448)], np.float32)
+        return dq
+    for rule in ("unrounded", "divide"):
+        monkeypatch.setattr(nf4, "double_quantize", make(rule))
+        with pytest.raises(AssertionError):
+            pin_double_quant_hand_case()
+    monkeypatch.setattr(nf4, "double_quantize", orig)
+    pin_double_quant_hand_case()
+
+
 def test_double_quant_codes_use_exact_absmax():
     rng = np.random.default_rng(8)
     w = (rng.standard_normal((16, 1024)) * 0.02).astype(np.float32)
