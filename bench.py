@@ -368,7 +368,7 @@ def protect_leg(api, synth, torch, dev, peaks, reps: int = 3, K: int = 8):
         torch.cuda.empty_cache()
     assert api.status() == 0, "device status set in the protection leg"
     # rank the whole stack (12.7 G weights) once with the error pass
-    mats = synth.stack_matrices(n_layers=40, linears=synth.QWEN14B_LINEARS)
+    mats = synth.stack_matrices_14b()
     Ws = [synth.stack_weight(m, device=str(dev)) for m in mats]
     _, order, _ = api.layer_error_rank(Ws, K, double_quant=True)
     order = order.cpu().tolist()

@@ -137,13 +137,12 @@ def cases_14b(r: int, M: int = 16384, seed: int = 0, kinds=("q", "gate", "down")
     """14B-shaped decoder linears (hidden 5120, intermediate 13824) with double
     quant, rank r, alpha = 2r, X of M tokens; weights are the stack's per-matrix
     scale * Student-t(nu) draws of the given layer."""
-    mats = {m.name: m for m in stack_matrices(n_layers=layer + 1, linears=QWEN14B_LINEARS, seed=seed)
-            if m.layer == layer}
+    mats = {m.name: m for m in stack_matrices_14b(n_layers=layer + 1) if m.layer == layer}
     out = []
     for k in kinds:
         m = mats[k]
         out.append(LinearCase(f"14b-{k}-r{r}", M=M, out=m.out, inp=m.inp, r=r, alpha=2.0 * r, double_quant=True,
-                              w_dist="t", nu=m.nu, w_std=m.scale, seed=seed, index=m.index))
+                              w_dist="t", nu=m.nu, w_std=m.scale, seed=m.seed + seed, index=m.index))
     return out
 
 
@@ -162,6 +161,11 @@ class StackMatrix:
     nu: float
     scale: float
     index: int
+    seed: int = 0               # seed of the stack's draws and of its weights
+
+
+# The 14B-shaped stack draws from its own seed (the Llama-7B-shaped stack uses 0).
+STACK_14B_SEED = 1
 
 
 def stack_matrices(n_layers: int = 32, linears=LLAMA7B_LINEARS, seed: int = 0) -> List[StackMatrix]:
@@ -172,12 +176,19 @@ def stack_matrices(n_layers: int = 32, linears=LLAMA7B_LINEARS, seed: int = 0) -
         for j, (nm, o, i) in enumerate(linears):
             idx = l * len(linears) + j
             nu, sc = draws[idx]
-            mats.append(StackMatrix(l, nm, o, i, nu, sc, idx))
+            mats.append(StackMatrix(l, nm, o, i, nu, sc, idx, seed))
     return mats
 
 
-def stack_weight(m: StackMatrix, seed: int = 0, device: str = "cpu") -> torch.Tensor:
-    return student_t_bf16((m.out, m.inp), m.nu, m.scale, seed, STREAM_W, m.index, device)
+def stack_matrices_14b(n_layers: int = 40) -> List[StackMatrix]:
+    """The 14B-shaped stack: hidden 5120, intermediate 13824, MHA, its own seed."""
+    return stack_matrices(n_layers=n_layers, linears=QWEN14B_LINEARS, seed=STACK_14B_SEED)
+
+
+def stack_weight(m: StackMatrix, seed: Optional[int] = None, device: str = "cpu") -> torch.Tensor:
+    """``scale * t_nu`` weights of one stack matrix (seed defaults to the stack's)."""
+    sd = m.seed if seed is None else seed
+    return student_t_bf16((m.out, m.inp), m.nu, m.scale, sd, STREAM_W, m.index, device)
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:

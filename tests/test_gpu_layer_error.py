@@ -6,6 +6,8 @@ import torch
 
 from oracle import layer_error, nf4
 from quantized_lora_fine_b200 import api, synth
+from tests import stack_pool
+from tests.conftest import load_golden
 from tests.gpu_helpers import bits
 
 pytestmark = pytest.mark.gpu
@@ -52,25 +54,47 @@ def test_llama_stack_sampled_layers(cuda_device):
     _compare(Ws, K=3, dq=False)
 
 
-def test_llama_stack_all_224_matrices(cuda_device):
-    """The whole 32-layer stack (224 matrices, 6.48 G weights) in one call: errors of
-    sampled matrices (the top- and bottom-ranked ones among them) match the oracle
-    within 1e-6; the order is the (error desc, index asc) sort of the errors and
-    keep marks the first K = 16."""
-    mats = synth.stack_matrices()
-    Ws = [synth.stack_weight(m, device="cuda") for m in mats]
-    err, order, keep = api.layer_error_rank(Ws, 16, double_quant=False)
+def _golden_stack(name, mats):
+    """The oracle's errors, order and keep for a full stack (tests/golden, written by
+    make_stack_rank_goldens.py from the host-drawn weights), and the same weights on
+    the GPU, drawn on the host the same way."""
+    gold = load_golden(name)
+    assert [(m["out"], m["in"]) for m in gold["matrices"]] == [(m.out, m.inp) for m in mats]
+    Ws = [None] * len(mats)
+    for idx, b in stack_pool.stack_bits(mats):
+        Ws[idx] = synth.from_bf16_bits(b, device="cuda")
+    return gold, Ws
+
+
+def _check_against_golden(gold, err, order, keep):
+    ref = np.array(gold["err"], np.float64)
+    e = err.cpu().numpy()
+    assert np.all(ref > 0)
+    rel = np.abs(e - ref) / ref
+    assert rel.max() <= 1e-6, (int(rel.argmax()), float(rel.max()))
+    assert np.array_equal(order.cpu().numpy(), np.array(gold["order"], np.int32))
+    assert np.array_equal(keep.cpu().numpy(), np.array(gold["keep"], np.uint8))
+
+
+@pytest.mark.parametrize("name,mats_of", [
+    ("stack_rank_llama7b.json", lambda: synth.stack_matrices()),
+    ("stack_rank_14b.json", lambda: synth.stack_matrices_14b())])
+def test_full_stack_ranking_against_oracle_golden(cuda_device, name, mats_of):
+    """Every matrix of the 224-matrix Llama-7B-shaped stack (fp32 absmax, K = 16) and
+    of the 280-matrix 14B-shaped stack (double quant, K = 8): all errors within 1e-6
+    relative of the oracle's, order and keep bit-exact, through the error pass and
+    through the fused quantize + error pass."""
+    gold, Ws = _golden_stack(name, mats_of())
+    dq, K = gold["double_quant"], gold["K"]
+    err, order, keep = api.layer_error_rank(Ws, K, double_quant=dq)
     torch.cuda.synchronize()
     assert api.status() == 0
-    err = err.cpu().numpy()
-    order = order.cpu().numpy()
-    keep = keep.cpu().numpy()
-    assert np.array_equal(order, np.lexsort((np.arange(len(err)), -err)))
-    assert np.array_equal(np.flatnonzero(keep), np.sort(order[:16]))
-    for i in sorted({int(order[0]), int(order[-1]), 3, 117}):
-        ref = layer_error.layer_error(bits(Ws[i].cpu()), False)
-        assert abs(err[i] - ref) <= 1e-6 * ref, (i, err[i], ref)
-    del Ws
+    _check_against_golden(gold, err, order, keep)
+    err, order, keep, outs = api.quantize_error_rank(Ws, K, double_quant=dq)
+    torch.cuda.synchronize()
+    assert api.status() == 0
+    _check_against_golden(gold, err, order, keep)
+    del Ws, outs
     torch.cuda.empty_cache()
 
 

@@ -97,7 +97,7 @@ def test_q_proj_full_size_sampled(cuda_device):
     run_and_compare(synth.case_q_proj(), rows=rows)
 
 
-@pytest.mark.parametrize("idx", [0, 2])
+@pytest.mark.parametrize("idx", [0, 1, 2])   # gate, up, down
 def test_mlp_full_size_sampled(cuda_device, idx):
     rows = np.random.default_rng(1).choice(8192, 96, replace=False)
     rows.sort()

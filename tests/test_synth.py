@@ -36,7 +36,7 @@ def test_stack_draws_and_sizes():
     mats7 = synth.stack_matrices()
     assert len(mats7) == 224
     assert sum(m.out * m.inp for m in mats7) == 32 * (4 * 4096 * 4096 + 3 * 11008 * 4096)   # 6.48 G weights
-    mats14 = synth.stack_matrices(n_layers=40, linears=synth.QWEN14B_LINEARS)
+    mats14 = synth.stack_matrices_14b()
     assert len(mats14) == 280
     assert sum(m.out * m.inp for m in mats14) == 12_687_769_600
     for m in mats7 + mats14:
@@ -44,8 +44,13 @@ def test_stack_draws_and_sizes():
     assert [m.index for m in mats7] == list(range(224))
     assert [(m.layer, m.name) for m in mats7[:8]] == [(0, "q"), (0, "k"), (0, "v"), (0, "o"), (0, "gate"),
                                                      (0, "up"), (0, "down"), (1, "q")]
-    # the draws are a fixed sequence: the first matrices of both stacks share them
-    assert [(m.nu, m.scale) for m in mats7[:7]] == [(m.nu, m.scale) for m in mats14[:7]]
+    # each stack draws from its own seed, and a stack matrix's weights follow it
+    assert all(m.seed == 0 for m in mats7) and all(m.seed == synth.STACK_14B_SEED for m in mats14)
+    assert synth.STACK_14B_SEED != 0
+    assert [(m.nu, m.scale) for m in mats7[:7]] != [(m.nu, m.scale) for m in mats14[:7]]
+    small = synth.stack_matrices(n_layers=1, linears=(("a", 64, 128),), seed=synth.STACK_14B_SEED)[0]
+    assert torch.equal(synth.stack_weight(small), synth.stack_weight(small, seed=synth.STACK_14B_SEED))
+    assert not torch.equal(synth.stack_weight(small), synth.stack_weight(small, seed=0))
 
 
 def test_bf16_bits_round_trip():
