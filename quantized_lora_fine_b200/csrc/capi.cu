@@ -65,8 +65,10 @@ int thin_bn(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
 
 // ---- workspace layouts
 
+static_assert(size_t(kPair2CounterInts) * sizeof(int) <= kGemmCounterBytes, "pair-GEMM counters fit their region");
+
 struct FwdLayout {
-  size_t scales, l2t, t, part, counters, total;
+  size_t scales, l2t, t, part, gpart, counters, total;
 };
 
 FwdLayout fwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
@@ -78,12 +80,13 @@ FwdLayout fwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
   L.t = off;      off += up256(size_t(M) * r * 2);
   const ThinSplit ts = thin_split(M, in / 64);
   L.part = off;   off += up256(size_t(ts.splits) * size_t(M) * r * 4);
+  L.gpart = off;  off += up256(pair2_partial_bytes(M, out));   // pair GEMM: split last round
   L.total = off;
   return L;
 }
 
 struct BwdLayout {
-  size_t scales, l1s, t, u, su, part, part2, counters, total;
+  size_t scales, l1s, t, u, su, part, part2, gpart, counters, total;
 };
 
 BwdLayout bwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
@@ -101,6 +104,7 @@ BwdLayout bwd_layout(int64_t M, int64_t out, int64_t in, int32_t r) {
                           size_t(d.splits) * in * r}) * 4;
   L.part = off;   off += up256(part);
   L.part2 = off;  off += up256(size_t(c.splits) * out * r * 4);   // dL2 partials on the side stream
+  L.gpart = off;  off += up256(pair2_partial_bytes(M, in));         // pair GEMM: split last round
   L.total = off;
   return L;
 }
@@ -224,14 +228,18 @@ int bwd_schedule_override() {
   return 0;
 }
 
-bool use_pair_kernel() {
+// NF4 GEMM engine: 2 = CTA pairs with 512 x 256 tiles (default), 1 = CTA pairs with
+// 256 x 256 tiles (QLORA_B200_GEMM=pair256), 0 = single CTAs (QLORA_B200_GEMM=1cta).
+// All compute the same products within rounding; the others are kept for measurement.
+int gemm_engine() {
   static int v = -1;
   if (v < 0) {
     const char* e = std::getenv("QLORA_B200_GEMM");
-    v = (e && std::strcmp(e, "1cta") == 0) ? 0 : 1;
+    v = (e && std::strcmp(e, "1cta") == 0) ? 0 : (e && std::strcmp(e, "pair256") == 0) ? 1 : 2;
   }
-  return v == 1;
+  return v;
 }
+bool use_pair_kernel() { return gemm_engine() >= 1; }
 
 // Fused NF4 GEMM on CTA pairs (256 x 256 tiles): out = A . W' + Ax . Bx^T, where
 // the LoRA step reads Bx as [N x r] rows: Ax = T with Bx = s.L2^T (fwd), or
@@ -240,7 +248,7 @@ bool use_pair_kernel() {
 // per forward GEMM on the q_proj workload than this transposed copy.)
 qlora_status run_pair(bool dx, const qlora_weight* w, const uint16_t* A, int64_t M, const uint16_t* Ax,
                       const uint16_t* Bx, int32_t r, const float* scales_t, uint16_t* out, int* status,
-                      cudaStream_t s) {
+                      float* gpart, int* gcount, cudaStream_t s) {
   const int64_t o_ = w->out, h = w->in;
   const int64_t Kdim = dx ? o_ : h;
   const int64_t Ndim = dx ? h : o_;
@@ -266,8 +274,15 @@ qlora_status run_pair(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
   p.codes_ld = h / 2;
   p.scales = scales_t;
   p.scales_ld = o_;
+  if (gemm_engine() == 2) {
+    p.tiles_m = int((M + 511) / 512);
+    p.sk_part = gpart;
+    p.sk_count = gcount;
+    // output written by TMA: 128-row x 64-column boxes, 128-byte swizzle
+    if (!make_tmap_2d(&pp.Y, out, TmapType::BF16, Ndim, M, Ndim * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+  }
   record_prof(g_prof[dx ? 2 : 0], s);
-  const qlora_status st = launch_gemm_pair(dx, pp, p, s);
+  const qlora_status st = gemm_engine() == 2 ? launch_gemm_pair2(dx, pp, p, s) : launch_gemm_pair(dx, pp, p, s);
   record_prof(g_prof[dx ? 3 : 1], s);
   return st;
 }
@@ -658,7 +673,9 @@ qlora_status linear_fwd_impl(const qlora_weight* w, const uint16_t* X, int64_t M
     T = Tw;
   }
   if (ss) QLB_TRY(join_from(ss, s));
-  if (!w->is_bf16 && use_pair_kernel()) return run_pair(false, w, X, M, T, l2t, r, scales_t, Y, status, s);
+  if (!w->is_bf16 && use_pair_kernel())
+    return run_pair(false, w, X, M, T, l2t, r, scales_t, Y, status, reinterpret_cast<float*>(ws + L.gpart),
+                    reinterpret_cast<int*>(ws + kStatusBytes + kCounterBytes), s);
   return run_main(false, w, X, M, T, l2t, r, scales_t, Y, status, s);
 }
 
@@ -756,9 +773,14 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const ui
   std::lock_guard<std::mutex> lock(g_side_mu);
   SideStream* ss = ((M + 127) / 128 <= kMaxCounterTiles / 2 && (o_ + 127) / 128 <= kMaxCounterTiles / 2)
                        ? side_stream() : nullptr;
-  const int dx_tiles = int((M + 255) / 256) * int(h / 256);
   const int forced = bwd_schedule_override();
-  const bool beside_gemm = ss && dX && pair && forced != 2 && (forced == 1 || pair_spare_sms(true, dx_tiles) >= 16);
+  const int spare = !pair ? 0
+                    : gemm_engine() == 2 ? pair2_spare_sms(true, int((M + 511) / 512) * int(h / 256),
+                                                           int(o_ / 64) + (r + 63) / 64)
+                                         : pair_spare_sms(true, int((M + 255) / 256) * int(h / 256));
+  const bool beside_gemm = ss && dX && pair && forced != 2 && (forced == 1 || spare >= 16);
+  float* gpart = reinterpret_cast<float*>(ws + L.gpart);
+  int* gcount = reinterpret_cast<int*>(ws + kStatusBytes + kCounterBytes);
   cudaStream_t aux = s;
   int* counters2 = counters;
   if (ss) {
@@ -776,7 +798,7 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const ui
   if (beside_gemm) {
     QLB_TRY(run_thin(tu, part, counters, U, 3, scale, status, s, sU));
     QLB_TRY(handoff_to(ss, s, aux));   // the GEMM needs s.U
-    QLB_TRY(run_pair(true, w, dY, M, sU, L1, r, scales_t, dX, status, aux));
+    QLB_TRY(run_pair(true, w, dY, M, sU, L1, r, scales_t, dX, status, gpart, gcount, aux));
     QLB_TRY(run_thin(t1, part, counters, dL1, 1, scale, status, s));
     QLB_TRY(run_thin(t2, part_b, counters2, dL2, 2, scale, status, s));
     return join_from(ss, s, aux);
@@ -786,7 +808,7 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const ui
   else QLB_TRY(run_thin(tu, part, counters, U, 0, 1.f, status, s));
   QLB_TRY(run_thin(t1, part, counters, dL1, 1, scale, status, s));
   if (ss) QLB_TRY(join_from(ss, s));
-  if (dX && pair) return run_pair(true, w, dY, M, sU, L1, r, scales_t, dX, status, s);
+  if (dX && pair) return run_pair(true, w, dY, M, sU, L1, r, scales_t, dX, status, gpart, gcount, s);
   if (dX) {
     QLB_TRY(launch_scale_lora(L1, h, r, scale, /*transpose=*/false, l1s, s));
     QLB_TRY(run_main(true, w, dY, M, U, l1s, r, scales_t, dX, status, s));

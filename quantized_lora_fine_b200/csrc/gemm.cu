@@ -25,6 +25,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "gemm.cuh"
@@ -735,6 +736,405 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   }
 }
 
+// =============================================================== CTA-pair kernel, 512-row tiles
+//
+// Same pair MMA (cluster of 2, tcgen05 cta_group::2, M = 256, N = 256) as above, but a
+// pair tile is 512 (M) x 256 (N): each K step stages two 128-row A sub-tiles per CTA
+// and issues two pair MMAs per 16-wide K slice against the same dequantized B half,
+// into two accumulators (TMEM columns 0-255: rows m0 .. m0 + 255 of the tile, columns
+// 256-511: rows m0 + 256 .. m0 + 511). Every decoded weight therefore meets 512 token
+// rows instead of 256: the dequantizers' ALU work and shared-memory stores per MMA
+// are halved. The two accumulators fill TMEM, so there is no second buffer: the MMA
+// issuer commits accumulator 0 before the last step's accumulator-1 MMAs, the
+// epilogue drains it first (TMEM -> registers -> bf16 in a swizzled staging buffer ->
+// TMA store), and the next tile's first MMAs wait only for accumulator 0.
+//
+// Schedule (GemmParams::sk_*): sk_R rounds of whole tiles, then the remaining tiles'
+// steps cut into ranges of sk_L steps, one range per pair (so a part that can co-run
+// fewer pairs than a multiple of the tile count does not idle through a last partial
+// round). A tile cut into parts is finished by the pair holding its first step, which
+// is the last range of that pair: the other parts (the first range of their pairs,
+// done before it) write fp32 partials and count themselves in; the finishing pair
+// waits for the count (bounded), adds the partials in pair order to its accumulator
+// and writes the tile.
+//
+// Shared memory per CTA: 4 ring slots of 48 KB (A rows 0-127 and 256-383 of this
+// CTA's half of the tile, i.e. tile rows 128 rank + {0, 256} + 0..127, and this
+// CTA's B half), two 16 KB epilogue staging buffers, barriers.
+// Warp roles: 0 A producer, 1 MMA issuer (even CTA) and TMEM allocation, 2-5
+// epilogue, 6-13 dequantizers (two per ring slot).
+
+template <bool B_MN_>
+struct Pair2Cfg {
+  static constexpr bool B_MN = B_MN_;
+  static constexpr int S = 4;                     // ring slots (one K step each)
+  static constexpr int kA = 128 * 64 * 2;         // one 128-row A sub-tile: 16 KB
+  static constexpr int kB = 128 * 64 * 2;         // this CTA's B half: 16 KB
+  static constexpr int kSlot = 2 * kA + kB;       // 48 KB
+  static constexpr int kStageOff = S * kSlot;     // epilogue staging
+  static constexpr int kStageBytes = 128 * 64 * 2;   // 128 rows x 64 bf16 columns
+  static constexpr int kBarOff = kStageOff + 2 * kStageBytes;
+  static constexpr int kWarpsPerSlot = 2;
+  static constexpr int kDeqWarps = S * kWarpsPerSlot;
+  static constexpr int kFirstDeqWarp = 6;
+  static constexpr int kThreads = (kFirstDeqWarp + kDeqWarps) * 32;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kNumBars = 2 * S + 5;      // ready, empty, tfull[2], tempty[2], drain
+  static constexpr int kTmemSlotOff = kBarOff + 8 * kNumBars;
+  static constexpr int kSigOff = kTmemSlotOff + 8;                 // 4 bytes per dequantizer warp
+  static constexpr int kSigBytes = 4;
+  static constexpr int kSmem = kSigOff + kDeqWarps * kSigBytes + 1024;
+  static constexpr int kEpiThreads = 128;
+  static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(kStageOff % 1024 == 0, "swizzled staging must be 1024-byte aligned");
+};
+
+// Steps of pair `pr` and the (tile, k step) of its step i (see GemmParams::sk_*).
+__device__ __forceinline__ uint32_t sk_num_steps(const GemmParams& p, int pr) {
+  const int S = p.num_k_main + p.num_k_ext;
+  uint32_t n = uint32_t(p.sk_R) * uint32_t(S);
+  const int b = pr * p.sk_L, e = min(b + p.sk_L, p.sk_W);
+  if (e > b) n += uint32_t(e - b);
+  return n;
+}
+__device__ __forceinline__ void sk_step(const GemmParams& p, int pr, uint32_t i, int& tile, int& k) {
+  const int S = p.num_k_main + p.num_k_ext;
+  const uint32_t dp = uint32_t(p.sk_R) * uint32_t(S);
+  if (i < dp) {
+    const int r = int(i / uint32_t(S));
+    tile = pr + r * p.sk_P;
+    k = int(i) - r * S;
+  } else {
+    const int ti = pr * p.sk_L + int(i - dp);
+    const int u = ti / S;
+    tile = p.sk_base + u;
+    k = ti - u * S;
+  }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1)
+    tc_gemm_nf4_pair2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAx,
+                             const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmY,
+                             const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_base = smem_base + C::kBarOff;
+  auto ready = [&](int i) { return bar_base + 8u * i; };
+  auto empty = [&](int i) { return bar_base + 8u * (C::S + i); };
+  const int kT0 = 2 * C::S;
+  auto tfull = [&](int h) { return bar_base + 8u * (kT0 + h); };
+  auto tempty = [&](int h) { return bar_base + 8u * (kT0 + 2 + h); };
+  const uint32_t drain_bar = bar_base + 8u * (kT0 + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kTmemSlotOff);
+  auto slot = [&](uint32_t i) { return smem_base + (i % C::S) * C::kSlot; };   // A0 | A1 | B half
+
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::S; ++i) {
+      mbar_init(ready(i), 1 + C::kWarpsPerSlot);   // used in the even CTA only
+      mbar_init(empty(i), 1);
+    }
+    for (int h = 0; h < 2; ++h) { mbar_init(tfull(h), 1); mbar_init(tempty(h), 8); }
+    mbar_init(drain_bar, 1);
+    fence_mbarrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_launch();
+
+  const int pr = int(blockIdx.x >> 1);
+  const int S = p.num_k_main + p.num_k_ext;
+  const uint32_t nsteps = sk_num_steps(p, pr);
+  const uint32_t dp_steps = uint32_t(p.sk_R) * uint32_t(S);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ A producer (both CTAs)
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmAx);
+      uint32_t it = 0;
+      for (; it < nsteps; ++it) {
+        int tile, k;
+        sk_step(p, pr, it, tile, k);
+        if (!mbar_wait(empty(it % C::S), ((it / C::S) & 1u) ^ 1u)) {
+          set_status_site(p.status, QLORA_ERR_TIMEOUT, 201);
+          break;
+        }
+        const int m0 = (tile / p.tiles_n) * 512 + int(rank) * 128;
+        const bool main_step = k < p.num_k_main;
+        const uint32_t dst = slot(it), bar = ready(it % C::S);
+        const CUtensorMap* m = main_step ? &tmA : &tmAx;
+        const int kx = (main_step ? k : k - p.num_k_main) * 64;
+        if (rank == 0) {
+          // bytes of the whole step: both CTAs' two A sub-tiles and, in LoRA steps, B halves
+          mbar_arrive_expect_tx(bar, 4 * C::kA + (main_step ? uint32_t(C::kWarpsPerSlot * C::kSigBytes)
+                                                            : uint32_t(2 * C::kB)));
+          tma_load_2d(dst, m, bar, kx, m0);
+          tma_load_2d(dst + C::kA, m, bar, kx, m0 + 256);
+        } else {
+          const uint32_t bar0 = mapa_shared(bar, 0);
+          tma_load_2d_pair(dst, m, bar0, kx, m0);
+          tma_load_2d_pair(dst + C::kA, m, bar0, kx, m0 + 256);
+        }
+      }
+      // let the last copies land before leaving
+      if (it > 0) mbar_wait(empty(it % C::S), ((it / C::S) & 1u) ^ 1u, 100000000ull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc_main = make_idesc_bf16(256, 256, 0, C::B_MN ? 1 : 0);
+      constexpr uint32_t idesc_ext = make_idesc_bf16(256, 256, 0, 0);   // LoRA B is [N x r], K-major
+      constexpr uint32_t b_adv = C::B_MN ? (2048u >> 4) : (32u >> 4);
+      constexpr uint32_t b_adv_ext = 32u >> 4;
+      const uint64_t da_base = make_smem_desc(slot(0), 16u, 1024u, kSwizzle128B);
+      const uint64_t db_base = make_smem_desc(slot(0) + 2 * C::kA, 8192u, 1024u, kSwizzle128B);
+      constexpr uint64_t kSlotAdv = uint64_t(C::kSlot >> 4);
+      constexpr uint64_t kA1 = uint64_t(C::kA >> 4);
+      uint32_t seg = 0;
+      for (uint32_t it = 0; it < nsteps; ++it) {
+        int tile, k;
+        sk_step(p, pr, it, tile, k);
+        const bool first = (k == 0) || (it == dp_steps);
+        const bool last = (k == S - 1) || (it + 1 == nsteps);
+        const uint32_t par = (seg & 1u) ^ 1u;
+        if (first) {
+          if (!mbar_wait_cluster(tempty(0), par)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 204); break; }
+          tc_fence_after();
+        }
+        const uint32_t si = it % C::S;
+        if (!mbar_wait_cluster(ready(si), (it / C::S) & 1u)) {
+          set_status_site(p.status, QLORA_ERR_TIMEOUT, 205);
+          break;
+        }
+        tc_fence_after();
+        const bool ext = k >= p.num_k_main;
+        const uint64_t ad = da_base + si * kSlotAdv, bd = db_base + si * kSlotAdv;
+        const uint32_t badv = ext ? b_adv_ext : b_adv;
+        const uint32_t idesc = ext ? idesc_ext : idesc_main;
+#pragma unroll
+        for (uint32_t kk = 0; kk < 4; ++kk)
+          tc_mma_bf16_pair(tmem_base, ad + 2 * kk, bd + kk * badv, idesc, (!first || kk > 0) ? 1u : 0u);
+        if (last) tc_commit_pair_mc(tfull(0), 0x3);
+        if (first) {
+          if (!mbar_wait_cluster(tempty(1), par)) { set_status_site(p.status, QLORA_ERR_TIMEOUT, 206); break; }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (uint32_t kk = 0; kk < 4; ++kk)
+          tc_mma_bf16_pair(tmem_base + 256u, ad + kA1 + 2 * kk, bd + kk * badv, idesc, (!first || kk > 0) ? 1u : 0u);
+        tc_commit_pair_mc(empty(si), 0x3);
+        if (last) {
+          tc_commit_pair_mc(tfull(1), 0x3);
+          ++seg;
+        }
+      }
+      tc_commit_pair_mc(drain_bar, 0x1);
+      mbar_wait(drain_bar, 0, 100000000ull);
+    }
+  } else if (warp < uint32_t(C::kFirstDeqWarp)) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const uint32_t q = warp & 3u;
+    const uint32_t row = q * 32 + lane;              // TMEM lane = row of this CTA's sub-tiles
+    const bool leader = (warp == 2 && lane == 0);    // issues the TMA stores and counts in
+    const uint32_t tempty_remote[2] = {mapa_shared(tempty(0), 0), mapa_shared(tempty(1), 0)};
+    const uint32_t stage0 = smem_base + C::kStageOff;
+    const uint32_t tl = tmem_base + ((q * 32u) << 16);
+    constexpr size_t kRankFloats = size_t(2) * 256 * 128;   // one rank's partial: 2 halves x 256 cols x 128 rows
+    // Every epilogue warp walks the same segments and named barriers even after a
+    // wait has timed out (ok = false then skips the remaining waits), so no warp is
+    // left alone at a barrier.
+    uint32_t seg = 0, chunk = 0;
+    bool ok = true;
+    auto wait_full = [&](int h, uint32_t par, int site) {
+      if (ok && !__all_sync(0xffffffffu, mbar_wait_cluster(tfull(h), par))) {
+        set_status_site(p.status, QLORA_ERR_TIMEOUT, site);
+        ok = false;
+      }
+    };
+    for (uint32_t i = 0; i < nsteps;) {
+      int tile, kb;
+      sk_step(p, pr, i, tile, kb);
+      const int len = (i < dp_steps) ? S : min(S - kb, int(nsteps - i));
+      i += uint32_t(len);
+      const int ke = kb + len;
+      const int mb = tile / p.tiles_n, nb = tile - mb * p.tiles_n;
+      const uint32_t par = seg & 1u;
+      ++seg;
+      int extra = 0, pf1 = 0;     // partials of later parts to add, from pair slots pf1, pf1 + 1, ...
+      if (kb > 0 || ke < S) {
+        // ---- a tile cut into parts (pairs pf .. pl, in step order)
+        const int u = tile - p.sk_base;
+        const int pf = (u * S) / p.sk_L, pl = ((u + 1) * S - 1) / p.sk_L;
+        int* counter = p.sk_count + 2 * u + int(rank);
+        if (kb > 0) {
+          // a later part: fp32 partial to this pair's slot (column-major in 128-row
+          // columns, so every warp store is one 128-byte line), then count in
+          float* dst = p.sk_part + (size_t(pr) * 2 + rank) * kRankFloats + row;
+          for (int h = 0; h < 2; ++h) {
+            wait_full(h, par, 207);
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+              uint32_t v[32];
+              tmem_ld_32x32b_x32(tl + uint32_t(h) * 256u + uint32_t(c) * 32u, v);
+              tmem_ld_wait();
+              float* d = dst + (size_t(h) * 256 + c * 32) * 128;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) __stcg(d + size_t(j) * 128, __uint_as_float(v[j]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_remote[h]);
+          }
+          __threadfence();
+          named_bar_sync(1, C::kEpiThreads);
+          if (leader) atomicAdd(counter, 1);
+          continue;
+        }
+        // the first part: wait (bounded) until the pl - pf later parts have counted in
+        extra = pl - pf;
+        pf1 = pf + 1;
+        if (ok && ld_acquire_gpu(counter) < extra) {
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_gpu(counter) < extra) {
+            if (globaltimer_ns() - t0 > 2000000000ull) {
+              set_status_site(p.status, QLORA_ERR_TIMEOUT, 208);
+              break;
+            }
+          }
+        }
+      }
+      for (int h = 0; h < 2; ++h) {
+        wait_full(h, par, 209);
+        tc_fence_after();
+        const int y = mb * 512 + h * 256 + int(rank) * 128;   // first output row of this store box
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c, ++chunk) {
+          const uint32_t buf = chunk & 1u;
+          uint32_t v[64];
+          tmem_ld_32x32b_x32(tl + uint32_t(h) * 256u + uint32_t(c) * 64u, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld_32x32b_x32(tl + uint32_t(h) * 256u + uint32_t(c) * 64u + 32u,
+                             *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_ld_wait();
+          if (c == 3) {
+            // the accumulator is in registers: the next tile's MMAs may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_remote[h]);
+          }
+          for (int e = 0; e < extra; ++e) {
+            const float* src = p.sk_part + (size_t(pf1 + e) * 2 + rank) * kRankFloats +
+                               (size_t(h) * 256 + c * 64) * 128 + row;
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+              v[j] = __float_as_uint(__uint_as_float(v[j]) + __ldcg(src + size_t(j) * 128));
+          }
+          // the store that used this staging buffer two chunks ago must have read it
+          if (leader) bulk_wait_group_read<1>();
+          named_bar_sync(1, C::kEpiThreads);
+          const uint32_t sbase = stage0 + buf * C::kStageBytes + row * 128u;
+          const uint32_t sw = row & 7u;
+#pragma unroll
+          for (uint32_t j = 0; j < 8; ++j) {
+            const uint32_t a0 = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+            const uint32_t a1 = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+            const uint32_t a2 = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+            const uint32_t a3 = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + ((j ^ sw) << 4)), "r"(a0),
+                         "r"(a1), "r"(a2), "r"(a3)
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1, C::kEpiThreads);
+          if (leader && y < p.M) {   // rows past M are clipped by the store; a box wholly past M is skipped
+            tma_store_2d(&tmY, stage0 + buf * C::kStageBytes, nb * 256 + c * 64, y);
+          }
+          if (leader) bulk_commit_group();
+        }
+      }
+      if (extra > 0 && leader) {
+        // every later part has been read: the counter goes back to zero for the next call
+        p.sk_count[2 * (tile - p.sk_base) + int(rank)] = 0;
+      }
+    }
+    if (leader) bulk_wait_group<0>();
+  } else {
+    // ------------------------------------------------------------ dequantizers (both CTAs)
+    const uint32_t dw = warp - uint32_t(C::kFirstDeqWarp);
+    const uint32_t own = dw / C::kWarpsPerSlot;   // ring slot this warp fills
+    const uint32_t sub = dw % C::kWarpsPerSlot;   // threads t in [32 sub, 32 sub + 32)
+    const uint32_t row = sub * 32 + lane;
+    const uint32_t ready_even = mapa_shared(ready(own), 0);
+    const uint32_t sig_even = mapa_shared(smem_base + C::kSigOff + dw * C::kSigBytes, 0);
+    auto nc0_of = [&](int t) { return (t % p.tiles_n) * 256 + int(rank) * 128; };
+    PairRaw raw;
+    if (own < nsteps) {
+      int t, k;
+      sk_step(p, pr, own, t, k);
+      if (k < p.num_k_main) pair_load_raw<C::B_MN>(p, row, k, nc0_of(t), raw);
+    }
+    for (uint32_t it = own; it < nsteps; it += C::S) {
+      int t, k;
+      sk_step(p, pr, it, t, k);
+      const uint32_t round = it / C::S;
+      const uint32_t b_tile = slot(it) + 2 * C::kA;
+      if (!__all_sync(0xffffffffu, mbar_wait(empty(own), (round & 1u) ^ 1u))) {
+        set_status_site(p.status, QLORA_ERR_TIMEOUT, 218);
+        break;
+      }
+      if (k < p.num_k_main) {
+        pair_store_block<C::B_MN>(row, 0, raw, b_tile);
+        pair_store_block<C::B_MN>(row, 1, raw, b_tile);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(ready(own));
+          else st_async_signal(sig_even, ready_even);
+        }
+      } else if (lane == 0) {
+        // LoRA step: B half by TMA; its bytes were posted by the even A producer
+        const int kx = (k - p.num_k_main) * 64, n0 = nc0_of(t);
+        const uint32_t bar = rank == 0 ? ready(own) : ready_even;
+        if (sub == 0) {   // [N x r] rows n0.. (s.L2^T for the forward pass, L1 for dX)
+          if (rank == 0) tma_load_2d(b_tile, &tmBx, bar, kx, n0);
+          else tma_load_2d_pair(b_tile, &tmBx, bar, kx, n0);
+        }
+        if (rank == 0) mbar_arrive(ready(own));
+      }
+      // codes of this warp's next step, in flight while it waits for that slot
+      const uint32_t nx = it + C::S;
+      if (nx < nsteps) {
+        int t2, k2;
+        sk_step(p, pr, nx, t2, k2);
+        if (k2 < p.num_k_main) pair_load_raw<C::B_MN>(p, row, k2, nc0_of(t2), raw);
+      }
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+}
+
 // --------------------------------------------------------------- host side
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -877,6 +1277,122 @@ static qlora_status launch_pair_cfg(const GemmOperands& o, GemmParams p, cudaStr
   if (cudaLaunchKernelEx(&cfg, tc_gemm_nf4_pair_kernel<C>, o.A, o.Ax, o.Bx, p) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// ---- 512 x 256 pair kernel
+
+template <class C>
+static int pair2_max_clusters() {
+  static int max_pairs = -1;
+  if (max_pairs < 0) {
+    if (cudaFuncSetAttribute(tc_gemm_nf4_pair2_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+        cudaSuccess)
+      return 0;
+    cudaLaunchConfig_t qc = {};
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    qc.gridDim = dim3(2 * 74, 1, 1);
+    qc.blockDim = dim3(C::kThreads, 1, 1);
+    qc.dynamicSmemBytes = C::kSmem;
+    qc.attrs = qa;
+    qc.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_nf4_pair2_kernel<C>, &qc) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    max_pairs = n;
+  }
+  return max_pairs;
+}
+
+// QLORA_B200_MAX_PAIRS=n caps the pairs of the 512 x 256 kernel (read on every call, so
+// tests can force a given schedule of whole rounds and split tiles on any part).
+static int pair2_pair_cap() {
+  const char* e = std::getenv("QLORA_B200_MAX_PAIRS");
+  if (!e) return kPair2MaxPairs;
+  const int v = std::atoi(e);
+  return (v >= 1 && v <= kPair2MaxPairs) ? v : kPair2MaxPairs;
+}
+
+// Schedule over P co-resident pairs: R = T / P rounds of whole tiles, then the
+// remaining T - R P tiles' W steps in ranges of L = ceil(W / P) steps (at least a
+// third of a tile, so a tile has at most four parts). When cutting saves less than a
+// twentieth of a tile, L = S: the remaining tiles run whole, one per pair.
+struct Pair2Sched {
+  int P, R, L, W, base, launch;
+};
+static Pair2Sched pair2_schedule(int T, int S, int P) {
+  Pair2Sched sc;
+  sc.P = P;
+  sc.R = T / P;
+  const int Tr = T - sc.R * P;
+  sc.base = sc.R * P;
+  sc.W = Tr * S;
+  sc.L = 0;
+  if (Tr > 0) {
+    int L = std::max((sc.W + P - 1) / P, (S + 2) / 3);
+    if (L >= S || (S - L) * 20 < S) L = S;
+    sc.L = L;
+  }
+  sc.launch = sc.R > 0 ? P : (sc.L > 0 ? (sc.W + sc.L - 1) / sc.L : 0);
+  return sc;
+}
+
+size_t pair2_partial_bytes(int64_t M, int64_t N) {
+  const int64_t T = ((M + 511) / 512) * (N / 256);
+  const int64_t slots = std::min<int64_t>(kPair2MaxPairs, 4 * T);
+  return size_t(slots) * (size_t(2) * 2 * 256 * 128 * sizeof(float));
+}
+
+template <class C>
+static qlora_status launch_pair2_cfg(const GemmOperands& o, GemmParams p, cudaStream_t s) {
+  const int max_pairs = std::min(pair2_max_clusters<C>(), pair2_pair_cap());
+  if (max_pairs <= 0) return QLORA_ERR_CUDA;
+  p.bn = 256;
+  const int T = p.tiles_m * p.tiles_n;
+  const int S = p.num_k_main + p.num_k_ext;
+  if (T <= 0 || S <= 0) return QLORA_OK;
+  const Pair2Sched sc = pair2_schedule(T, S, max_pairs);
+  p.sk_P = sc.P;
+  p.sk_R = sc.R;
+  p.sk_L = sc.L;
+  p.sk_W = sc.W;
+  p.sk_base = sc.base;
+  if (sc.launch > kPair2MaxPairs || (sc.L > 0 && sc.L < S && (!p.sk_part || !p.sk_count))) return QLORA_ERR_CUDA;
+  g_last_pairs = sc.launch;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(2 * sc.launch, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  if (cudaLaunchKernelEx(&cfg, tc_gemm_nf4_pair2_kernel<C>, o.A, o.Ax, o.Bx, o.Y, p) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status launch_gemm_pair2(bool dx, const GemmOperands& o, GemmParams p, cudaStream_t s) {
+  if (!dx) return launch_pair2_cfg<Pair2Cfg<false>>(o, p, s);
+  return launch_pair2_cfg<Pair2Cfg<true>>(o, p, s);
+}
+
+int pair2_spare_sms(bool dx, int num_tiles, int steps) {
+  const int mp = std::min(dx ? pair2_max_clusters<Pair2Cfg<true>>() : pair2_max_clusters<Pair2Cfg<false>>(),
+                          pair2_pair_cap());
+  if (mp <= 0) return 0;
+  return num_sms() - 2 * pair2_schedule(num_tiles, steps, mp).launch;
 }
 
 qlora_status launch_gemm_pair(bool dx, const GemmOperands& o, const GemmParams& p, cudaStream_t s) {

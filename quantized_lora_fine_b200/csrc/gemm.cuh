@@ -38,10 +38,20 @@ struct GemmParams {
   int64_t codes_ld;   // bytes between code rows (in / 2)
   const float* scales;
   int64_t scales_ld;  // floats between S_t rows (out)
+  // Schedule of the 512 x 256 pair kernel (set by its launcher): sk_R rounds of whole
+  // tiles (pair p takes tiles p + r sk_P), then the remaining tiles' steps as ranges of
+  // sk_L steps, pair p taking [p sk_L, min((p + 1) sk_L, sk_W)) of the sk_W tail steps
+  // (tail tile u is tile sk_base + u). A tile split over several pairs is finished by
+  // the pair that holds its first step: it adds the others' fp32 partials (sk_part,
+  // one slot per pair) in pair order once their counter (sk_count, two per tail tile,
+  // left at zero) says they are written.
+  int sk_P, sk_R, sk_L, sk_W, sk_base;
+  float* sk_part;
+  int* sk_count;
 };
 
 struct GemmOperands {
-  CUtensorMap A, B, codes, scales, Ax, Bx;
+  CUtensorMap A, B, codes, scales, Ax, Bx, Y;
 };
 
 enum class GemmKind {
@@ -71,5 +81,16 @@ qlora_status launch_gemm(GemmKind kind, int bn, const GemmOperands& o, const Gem
 // scales (fwd: box 128 x 1; dX: box 64 x 2), Ax (box 64 x 128), Bx (box 64 x 128).
 // Requires N % 256 == 0.
 qlora_status launch_gemm_pair(bool dx, const GemmOperands& o, const GemmParams& p, cudaStream_t s);
+
+// Fused NF4 GEMM on CTA pairs with 512 x 256 tiles (two M = 256 accumulators per
+// decoded B stage) and a split last round. Operands as launch_gemm_pair plus Y (the
+// output, box 64 x 128, 128-byte swizzle, written by TMA). The caller provides
+// p.sk_part (pair2_partial_bytes(...) bytes) and p.sk_count (pair2_counter_ints(...)
+// ints, zero); requires N % 256 == 0.
+qlora_status launch_gemm_pair2(bool dx, const GemmOperands& o, GemmParams p, cudaStream_t s);
+// Upper bounds of the split-round scratch for a D[M x N] product (host only).
+size_t pair2_partial_bytes(int64_t M, int64_t N);
+constexpr int kPair2MaxPairs = 80;                 // pairs launched at most
+constexpr int kPair2CounterInts = 2 * kPair2MaxPairs;   // two per split tile
 
 }  // namespace qlb

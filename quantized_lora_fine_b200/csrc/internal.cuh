@@ -12,10 +12,13 @@ constexpr int kBlock = 64;        // NF4 block (elements per absmax)
 constexpr int kDQBlock = 256;     // absmax values per second-level scale
 constexpr size_t kStatusBytes = 256;
 // Workspace layout shared by every entry point: [0, 256) status word,
-// [256, 256 + 64 KiB) split-K tile counters (only ever used as counters, which
-// the kernels return to zero), then per-call scratch.
+// [256, 256 + 64 KiB) split-K tile counters and the next 1 KiB of pair-GEMM tile
+// counters (only ever used as counters, which the kernels return to zero), then
+// per-call scratch.
 constexpr size_t kCounterBytes = 65536;
-constexpr size_t kReservedBytes = kStatusBytes + kCounterBytes;
+// then 1 KiB of tile counters of the pair GEMM's split last round (also left at zero)
+constexpr size_t kGemmCounterBytes = 1024;
+constexpr size_t kReservedBytes = kStatusBytes + kCounterBytes + kGemmCounterBytes;
 constexpr int64_t kMaxCounterTiles = int64_t(kCounterBytes / 4);
 
 // Launch with programmatic dependent launch allowed (unless QLORA_B200_PDL=0):
@@ -116,6 +119,8 @@ qlora_status launch_layer_error_rank_noalloc(int n_layers, const uint16_t* const
 int last_pair_clusters();
 // SMs a pair GEMM over num_tiles 256 x 256 tiles leaves free (see pairs_for).
 int pair_spare_sms(bool dx, int num_tiles);
+// The same for the 512 x 256 pair kernel over num_tiles tiles of `steps` K steps.
+int pair2_spare_sms(bool dx, int num_tiles, int steps);
 // Operand descriptions for the tcgen05 GEMM engine.
 struct GemmPlan;
 }  // namespace qlb

@@ -59,6 +59,20 @@ def test_ranks(cuda_device, r):
     run_and_compare(c)
 
 
+@pytest.mark.parametrize("pairs", [1, 2, 3, 4, 5, 7])
+def test_split_last_round_schedules(cuda_device, monkeypatch, pairs):
+    """The GEMMs' schedule with the co-resident pairs capped: whole rounds of 512 x 256
+    tiles, then the remaining tiles cut into step ranges over the pairs (a tile in up
+    to four parts, finished by the pair holding its first step) or run whole. Six
+    output tiles of 1024 x 768 with 9 steps each (8 K steps + the LoRA step) give a
+    different mix of whole rounds and split tiles for every cap; ragged M covers a
+    box wholly past the last row."""
+    monkeypatch.setenv("QLORA_B200_MAX_PAIRS", str(pairs))
+    c = dataclasses.replace(synth.case_small(), M=1024, out=768, inp=512, r=16, alpha=32.0, double_quant=True)
+    run_and_compare(c)
+    run_and_compare(dataclasses.replace(c, M=700))
+
+
 def test_protected_bf16_layer(cuda_device):
     c = dataclasses.replace(synth.case_small(), M=300, out=512, inp=768, r=16, alpha=32.0)
     run_and_compare(c, protected=True)
