@@ -392,6 +392,80 @@ def protect_leg(api, synth, torch, dev, peaks, reps: int = 3, K: int = 8):
             "timing": f"CUDA-graph replay, median of {reps}, L2 flushed before each"}
 
 
+def linear_set_leg(api, synth, torch, dev, peaks, ranks=(16, 32, 64, 128), K: int = 8, alpha_frac: float = 0.85,
+                   M: int = 16384):
+    """The 14B-shaped decoder's whole linear set, run for real: 40 layers x {q, k, v, o
+    5120^2, gate/up 13824x5120, down 5120x13824} = 280 NF4 linears (double quant),
+    X of M = 16384 tokens per linear, r in `ranks` with alpha = 2r. The allocation
+    pass ranks all 280 matrices and the top K = 8 are kept in bf16. Three settings
+    (AQLoRA summary page, section 3.3: adapters on every block, or only on the top
+    blocks with the backward stopped below the cut; AQLoRA-s uses alpha = .85):
+      qlora        every linear NF4, adapters everywhere, full backward (dX everywhere)
+      protect      the top K in bf16, adapters everywhere, full backward
+      protect_top  the top K in bf16, adapters on the top alpha_frac of the blocks: the
+                   blocks below run the forward only, the lowest adapted block runs
+                   its backward without dX (early stop)
+    Inputs are shared per shape (one X and dY per input / output width); every
+    linear has its own weight. Each setting runs once untimed, then once timed with
+    CUDA events around the 280 linears (eager calls; every linear lasts milliseconds).
+    The forward of a block without adapters still adds its rank-r term, as every
+    call of the library does."""
+    mats = synth.stack_matrices_14b()
+    Ws = [synth.stack_weight(m, device=str(dev)) for m in mats]
+    _, order, keep, nf4 = api.quantize_error_rank(Ws, K, double_quant=True)
+    keep = keep.cpu().tolist()
+    weights = [api.NF4Weight.protected(W) if keep[i] else None for i, W in enumerate(Ws)]
+    del Ws
+    torch.cuda.empty_cache()
+    shapes = sorted({(m.inp, m.out) for m in mats})
+    n_layers = 1 + max(m.layer for m in mats)
+    cut = n_layers - int(round(alpha_frac * n_layers))   # blocks [cut, n_layers) carry adapters
+    X = {h: synth.normal_bf16((M, h), 1.0, 0, synth.STREAM_X, h, device=str(dev)) for h in {h for h, _ in shapes}}
+    dY = {o: synth.normal_bf16((M, o), 1.0, 0, synth.STREAM_DY, o, device=str(dev)) for o in {o for _, o in shapes}}
+    Y = {o: torch.empty((M, o), dtype=torch.bfloat16, device=dev) for o in dY}
+    out = {"workload": f"14B-shaped stack: {len(mats)} linears (hidden 5120, intermediate 13824), NF4 + double "
+                       f"quant, M = {M} tokens per linear, alpha = 2r; top {K} of the error ranking kept in bf16; "
+                       f"adapters on blocks {cut}..{n_layers - 1} in the protect_top setting",
+           "kept": [f"layer {mats[l].layer} {mats[l].name}" for l in order[:K].tolist()],
+           "timing": "CUDA events around the 280 linears (eager calls), after one untimed pass", "per_rank": {}}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for r in ranks:
+        s = 2.0
+        L1 = {h: synth.normal_bf16((h, r), 0.01, 0, synth.STREAM_L1, h, device=str(dev)) for h in X}
+        L2 = {o: synth.normal_bf16((r, o), 0.01, 0, synth.STREAM_L2, o, device=str(dev)) for o in dY}
+        fl_full = sum(flops_fwd_bwd(M, m.inp, m.out, r) for m in mats)
+
+        def run(setting):
+            for i, m in enumerate(mats):
+                w = weights[i] if (setting != "qlora" and keep[i]) else nf4[i]
+                T = api.lora_down(X[m.inp], L1[m.inp])
+                api.linear_fwd(w, X[m.inp], L1[m.inp], L2[m.out], s, Y=Y[m.out], T=T)
+                if setting == "protect_top" and m.layer < cut:
+                    continue                        # no adapter below the cut: no backward
+                early = setting == "protect_top" and m.layer == cut
+                api.linear_bwd(w, X[m.inp], dY[m.out], L1[m.inp], L2[m.out], s, T=T, need_dX=not early)
+
+        row = {}
+        for setting in ("qlora", "protect", "protect_top"):
+            run(setting)
+            torch.cuda.synchronize()
+            e0.record()
+            run(setting)
+            e1.record()
+            e1.synchronize()
+            row[f"{setting}_ms"] = e0.elapsed_time(e1)
+        row["qlora_TFLOP/s"] = fl_full / (row["qlora_ms"] * 1e-3) / 1e12
+        row["qlora_frac_of_burst"] = row["qlora_TFLOP/s"] / peaks["bf16"]
+        row["protect_TFLOP/s"] = fl_full / (row["protect_ms"] * 1e-3) / 1e12
+        row["protect_vs_qlora"] = row["protect_ms"] / row["qlora_ms"] - 1.0
+        row["protect_top_vs_qlora"] = row["protect_top_ms"] / row["qlora_ms"] - 1.0
+        out["per_rank"][str(r)] = row
+    assert api.status() == 0, "device status set in the linear-set leg"
+    del nf4, weights, X, dY, Y
+    torch.cuda.empty_cache()
+    return out
+
+
 def merge_leg(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int = 4, r: int = 16):
     """LoRA merge (W_hat + s (L1 L2)^T, bf16 out) and merge + NF4 re-quantization over
     the first `layers` decoder layers of the Llama-7B-shaped stack (7 matrices per
@@ -459,6 +533,29 @@ def merge_leg(api, synth, torch, dev, stream, peaks, reps: int = 3, layers: int 
             "timing": f"CUDA-graph replay, best of {reps} (outputs {2 * numel / 1e9:.2f} GB, above L2)"}
 
 
+def summary_of(line):
+    """Short form of the legs' headline rates (the end of the line)."""
+    def g(*path):
+        v = line
+        for k in path:
+            if not isinstance(v, dict) or k not in v:
+                return None
+            v = v[k]
+        return round(v, 4) if isinstance(v, float) else v
+    out = {"step_TFLOP/s": g("value"), "fwd_bwd_TFLOP/s": g("legs", "fwd_bwd", "TFLOP/s"),
+           "fwd_bwd_frac_of_burst": g("legs", "fwd_bwd", "frac_of_burst"),
+           "fwd_gemm_TFLOP/s": g("legs", "fwd_gemm", "TFLOP/s"), "dx_gemm_TFLOP/s": g("legs", "dx_gemm", "TFLOP/s"),
+           "mlp_TFLOP/s": g("mlp", "TFLOP/s"), "mlp_frac_of_burst": g("mlp", "frac_of_burst")}
+    for leg in ("quantize_all", "quantize_each", "error_rank_all", "quantize_error_rank_all"):
+        out[f"{leg}_GB/s"] = g("hbm_legs", leg, "GB/s")
+        out[f"{leg}_frac_hbm"] = g("hbm_legs", leg, "frac_hbm")
+    for r in ("16", "32", "64", "128"):
+        out[f"linear_set_r{r}_TFLOP/s"] = g("linear_set", "per_rank", r, "qlora_TFLOP/s")
+        out[f"linear_set_r{r}_protect_top_vs_qlora"] = g("linear_set", "per_rank", r, "protect_top_vs_qlora")
+    out["merge_fp64_TFLOP/s"] = g("merge", "merge", "fp64_TFLOP/s")
+    return {k: v for k, v in out.items() if v is not None}
+
+
 def gpu_main(args):
     import ctypes
 
@@ -477,6 +574,9 @@ def gpu_main(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     lib = _lib.load()
     peaks = load_peaks()
+    if args.linear_set_only:   # the linear-set leg alone (not a bench line)
+        print(json.dumps({"linear_set": linear_set_leg(api, synth, torch, dev, peaks)}), flush=True)
+        return
     if args.protect_only:   # the protected-layer leg alone (not a bench line)
         print(json.dumps({"protect": protect_leg(api, synth, torch, dev, peaks)}), flush=True)
         return
@@ -634,7 +734,8 @@ def gpu_main(args):
     fwd_tf = fl_fwd_gemm / (med["fwd_gemm"] * 1e-3) / 1e12
     dx_tf = fl_dx_gemm / (med["dx_gemm"] * 1e-3) / 1e12
     # dominant kernel = the longer of the two fused GEMMs
-    engine = "tc_gemm_kernel" if os.environ.get("QLORA_B200_GEMM") == "1cta" else "tc_gemm_nf4_pair_kernel"
+    engine = {"1cta": "tc_gemm_kernel", "pair256": "tc_gemm_nf4_pair_kernel"}.get(
+        os.environ.get("QLORA_B200_GEMM", ""), "tc_gemm_nf4_pair2_kernel")
     dom = (f"qlora_fwd_gemm ({engine} fwd)", fwd_tf, med["fwd_gemm"]) if med["fwd_gemm"] >= med["dx_gemm"] \
         else (f"qlora_bwd_dx_gemm ({engine} dX)", dx_tf, med["dx_gemm"])
     numel = h * o
@@ -757,6 +858,9 @@ def gpu_main(args):
     merge = None
     if rank == 0 and world == 1 and not args.no_merge_leg:
         merge = side_leg(merge_leg, api, synth, torch, dev, stream, peaks, layers=args.merge_layers)
+    linear_set = None
+    if rank == 0 and world == 1 and not args.no_linear_set_leg:
+        linear_set = side_leg(linear_set_leg, api, synth, torch, dev, peaks)
 
     # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
@@ -769,11 +873,14 @@ def gpu_main(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args, world),
-            "roofline": roofline, "gemm_pairs": int(lib.qlora_pair_clusters()), "legs": legs_out, "mlp": mlp, "hbm_legs": hbm, "merge": merge, "protect": protect, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps, "clocks": clk,
+            "roofline": roofline, "gemm_pairs": int(lib.qlora_pair_clusters()), "legs": legs_out, "mlp": mlp,
+            "hbm_legs": hbm, "merge": merge, "protect": protect, "linear_set": linear_set, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
             "timing": "cuda-graph replay of the step" if use_graphs else "eager API calls",
             "peaks": {"bf16_tflops": peaks["bf16"], "bf16_tflops_sustained": peaks["bf16_sus"],
                       "hbm_gbs": peaks["hbm"], "source": peaks["source"]}}
+    # the headline figures of every leg again, last, in a short form
+    line["summary"] = summary_of(line)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -798,6 +905,10 @@ def main():
     ap.add_argument("--no-merge-leg", action="store_true", help="skip the LoRA merge / merge + re-quantize leg")
     ap.add_argument("--no-protect-leg", action="store_true",
                     help="skip the protected-layer (bf16 vs NF4) step-time leg on the 14B-stack shapes")
+    ap.add_argument("--no-linear-set-leg", action="store_true",
+                    help="skip the 280-linear 14B-shaped linear set (all NF4 / top 8 in bf16 / top-block adapters)")
+    ap.add_argument("--linear-set-only", action="store_true",
+                    help="run only the linear-set leg and print it (not a bench line)")
     ap.add_argument("--protect-only", action="store_true",
                     help="run only the protected-layer leg and print it (not a bench line)")
     ap.add_argument("--merge-layers", type=int, default=4, help="decoder layers of the stack for the merge leg")

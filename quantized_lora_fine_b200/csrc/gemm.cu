@@ -26,6 +26,7 @@
 
 #include <algorithm>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "gemm.cuh"
@@ -758,22 +759,26 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 // waits for the count (bounded), adds the partials in pair order to its accumulator
 // and writes the tile.
 //
-// Shared memory per CTA: 4 ring slots of 48 KB (A rows 0-127 and 256-383 of this
-// CTA's half of the tile, i.e. tile rows 128 rank + {0, 256} + 0..127, and this
-// CTA's B half), two 16 KB epilogue staging buffers, barriers.
+// Shared memory per CTA: S ring slots of 48 KB (the A rows 128 rank + {0, 256} +
+// 0..127 of the tile, and this CTA's B half) and kNumStage 16 KB epilogue staging
+// buffers (128 rows x 64 bf16 columns, 128-byte swizzle, written out by TMA store),
+// barriers. The epilogue's stores leave the SM slowly while every pair drains at
+// once (a store held its buffer about 2000 cycles before it had read it), so the
+// default gives the staging a whole accumulator (3 slots, 4 buffers).
 // Warp roles: 0 A producer, 1 MMA issuer (even CTA) and TMEM allocation, 2-5
-// epilogue, 6-13 dequantizers (two per ring slot).
+// epilogue, then the dequantizers (two per ring slot).
 
-template <bool B_MN_>
+template <bool B_MN_, int S_, int NST_>
 struct Pair2Cfg {
   static constexpr bool B_MN = B_MN_;
-  static constexpr int S = 4;                     // ring slots (one K step each)
+  static constexpr int S = S_;                    // ring slots (one K step each)
+  static constexpr int kNumStage = NST_;          // epilogue staging buffers of 16 KB
   static constexpr int kA = 128 * 64 * 2;         // one 128-row A sub-tile: 16 KB
   static constexpr int kB = 128 * 64 * 2;         // this CTA's B half: 16 KB
   static constexpr int kSlot = 2 * kA + kB;       // 48 KB
   static constexpr int kStageOff = S * kSlot;     // epilogue staging
   static constexpr int kStageBytes = 128 * 64 * 2;   // 128 rows x 64 bf16 columns
-  static constexpr int kBarOff = kStageOff + 2 * kStageBytes;
+  static constexpr int kBarOff = kStageOff + kNumStage * kStageBytes;
   static constexpr int kWarpsPerSlot = 2;
   static constexpr int kDeqWarps = S * kWarpsPerSlot;
   static constexpr int kFirstDeqWarp = 6;
@@ -1024,7 +1029,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         const int y = mb * 512 + h * 256 + int(rank) * 128;   // first output row of this store box
 #pragma unroll 1
         for (int c = 0; c < 4; ++c, ++chunk) {
-          const uint32_t buf = chunk & 1u;
+          const uint32_t buf = chunk % uint32_t(C::kNumStage);
           uint32_t v[64];
           tmem_ld_32x32b_x32(tl + uint32_t(h) * 256u + uint32_t(c) * 64u, *reinterpret_cast<uint32_t(*)[32]>(v));
           tmem_ld_32x32b_x32(tl + uint32_t(h) * 256u + uint32_t(c) * 64u + 32u,
@@ -1043,8 +1048,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             for (int j = 0; j < 64; ++j)
               v[j] = __float_as_uint(__uint_as_float(v[j]) + __ldcg(src + size_t(j) * 128));
           }
-          // the store that used this staging buffer two chunks ago must have read it
-          if (leader) bulk_wait_group_read<1>();
+          // the store that used this staging buffer kNumStage chunks ago must have read it
+          if (leader) bulk_wait_group_read<C::kNumStage - 1>();
           named_bar_sync(1, C::kEpiThreads);
           const uint32_t sbase = stage0 + buf * C::kStageBytes + row * 128u;
           const uint32_t sw = row & 7u;
@@ -1383,14 +1388,29 @@ static qlora_status launch_pair2_cfg(const GemmOperands& o, GemmParams p, cudaSt
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
+// Ring and staging: 3 slots and 4 staging buffers by default (64 KB of staging holds a
+// whole accumulator's bf16 rows, so accumulator 0 leaves TMEM without waiting for any
+// store); QLORA_B200_PAIR2=4x2 selects 4 slots and 2 buffers (read on every call, for
+// measurement). On the q_proj workload 3 x 4 ran the forward and dX GEMMs in 198 and
+// 199 us against 214 and 217 us for 4 x 2 on the same B200.
+static bool pair2_shallow_stage() {
+  const char* e = std::getenv("QLORA_B200_PAIR2");
+  return e && std::strcmp(e, "4x2") == 0;
+}
+using Pair2Fwd = Pair2Cfg<false, 3, 4>;
+using Pair2Dx = Pair2Cfg<true, 3, 4>;
+
 qlora_status launch_gemm_pair2(bool dx, const GemmOperands& o, GemmParams p, cudaStream_t s) {
-  if (!dx) return launch_pair2_cfg<Pair2Cfg<false>>(o, p, s);
-  return launch_pair2_cfg<Pair2Cfg<true>>(o, p, s);
+  if (pair2_shallow_stage()) {
+    if (!dx) return launch_pair2_cfg<Pair2Cfg<false, 4, 2>>(o, p, s);
+    return launch_pair2_cfg<Pair2Cfg<true, 4, 2>>(o, p, s);
+  }
+  if (!dx) return launch_pair2_cfg<Pair2Fwd>(o, p, s);
+  return launch_pair2_cfg<Pair2Dx>(o, p, s);
 }
 
 int pair2_spare_sms(bool dx, int num_tiles, int steps) {
-  const int mp = std::min(dx ? pair2_max_clusters<Pair2Cfg<true>>() : pair2_max_clusters<Pair2Cfg<false>>(),
-                          pair2_pair_cap());
+  const int mp = std::min(dx ? pair2_max_clusters<Pair2Dx>() : pair2_max_clusters<Pair2Fwd>(), pair2_pair_cap());
   if (mp <= 0) return 0;
   return num_sms() - 2 * pair2_schedule(num_tiles, steps, mp).launch;
 }

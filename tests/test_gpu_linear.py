@@ -73,6 +73,32 @@ def test_split_last_round_schedules(cuda_device, monkeypatch, pairs):
     run_and_compare(dataclasses.replace(c, M=700))
 
 
+_ENGINE_CHECK = """
+import dataclasses, sys
+sys.path.insert(0, {root!r})
+from quantized_lora_fine_b200 import synth
+from tests.test_gpu_linear import run_and_compare
+c = dataclasses.replace(synth.case_small(), M=700, out=768, inp=512, r=16, alpha=32.0, double_quant=True)
+run_and_compare(c)
+print("ok")
+"""
+
+
+@pytest.mark.parametrize("env", [{"QLORA_B200_PAIR2": "4x2"}, {"QLORA_B200_GEMM": "pair256"},
+                                 {"QLORA_B200_GEMM": "1cta"}])
+def test_other_gemm_engines(cuda_device, env):
+    """The NF4 GEMM engines kept for measurement (4 ring slots with 2 staging buffers,
+    the 256 x 256 pair kernel, the single-CTA kernel) give the same products within
+    the tolerances. The engine is chosen once per process, so each runs in a child."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, "-c", _ENGINE_CHECK.format(root=root)], env={**os.environ, **env},
+                         capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0 and res.stdout.strip().endswith("ok"), res.stdout[-2000:] + res.stderr[-2000:]
+
+
 def test_protected_bf16_layer(cuda_device):
     c = dataclasses.replace(synth.case_small(), M=300, out=512, inp=768, r=16, alpha=32.0)
     run_and_compare(c, protected=True)
