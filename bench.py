@@ -574,6 +574,17 @@ def gpu_main(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     lib = _lib.load()
     peaks = load_peaks()
+    if args.gemm_only:   # two forward + backward calls of the q_proj linear (profiler captures; not a bench line)
+        c = synth.case_q_proj()
+        dd = {k: v.to(dev) for k, v in c.make().items()}
+        w = api.quantize(dd["W"], double_quant=True)
+        for _ in range(2):
+            _, T = api.linear_fwd(w, dd["X"], dd["L1"], dd["L2"], c.scale)
+            api.linear_bwd(w, dd["X"], dd["dY"], dd["L1"], dd["L2"], c.scale, T=T)
+        torch.cuda.synchronize()
+        assert api.status() == 0, "device status set"
+        print(json.dumps({"gemm_only": "ok", "pairs": int(lib.qlora_pair_clusters())}), flush=True)
+        return
     if args.linear_set_only:   # the linear-set leg alone (not a bench line)
         print(json.dumps({"linear_set": linear_set_leg(api, synth, torch, dev, peaks)}), flush=True)
         return
@@ -905,6 +916,8 @@ def main():
     ap.add_argument("--no-merge-leg", action="store_true", help="skip the LoRA merge / merge + re-quantize leg")
     ap.add_argument("--no-protect-leg", action="store_true",
                     help="skip the protected-layer (bf16 vs NF4) step-time leg on the 14B-stack shapes")
+    ap.add_argument("--gemm-only", action="store_true",
+                    help="two forward + backward calls of the q_proj linear, nothing timed (profiler captures)")
     ap.add_argument("--no-linear-set-leg", action="store_true",
                     help="skip the 280-linear 14B-shaped linear set (all NF4 / top 8 in bf16 / top-block adapters)")
     ap.add_argument("--linear-set-only", action="store_true",

@@ -10,6 +10,7 @@
 // The three kernels follow each other on the stream with programmatic dependent
 // launch: each waits for its predecessor's memory before reading it.
 #include <cfloat>
+#include <cstdlib>
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -91,7 +92,8 @@ struct ChunkRef {
 // leave as soon as their totals are in shared memory.
 template <bool DQ, class Tab>
 __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_constant__ Tab tab,
-                                                                   double2* __restrict__ partial, int* status) {
+                                                                   double2* __restrict__ partial, int* status,
+                                                                   uint64_t copy_wait_ns) {
   constexpr bool kW = Tab::kWrite;
   __shared__ __align__(128) uint32_t s_w[kChunkBytes / 4];
   __shared__ double2 s_part[256];
@@ -122,7 +124,8 @@ __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_
     mbar_arrive_expect_tx(bar, bytes);
     bulk_load(smem_u32(s_w), tab.ptr[layer] + g * (kDQBlock * kBlock), bytes, bar);
   }
-  const bool landed = mbar_wait(bar, 0);
+  // the chunk's copy must land within copy_wait_ns (0: one try, no waiting)
+  const bool landed = copy_wait_ns ? mbar_wait(bar, 0, copy_wait_ns) : mbar_try_wait(bar, 0);
   if (!__syncthreads_and(landed)) {   // every thread leaves together
     if (tid == 0) {
       if (status) set_status(status, QLORA_ERR_TIMEOUT);
@@ -353,6 +356,16 @@ __global__ void __launch_bounds__(32) layer_error_finish_kernel(const double2* _
   finish_layer_warp(partial, r.first_chunk[l], r.first_chunk[l + 1], err + l);
 }
 
+// Limit of the chunk kernel's wait for its bulk copy: 2 s, or QLORA_B200_COPY_WAIT_NS
+// (read on every call; 0 = a single try). A limit that runs out records
+// QLORA_ERR_TIMEOUT (or a NaN error without a status word) and the kernel still waits
+// for its copy to land before it exits; the failure-detection tests use 0.
+static uint64_t copy_wait_ns() {
+  const char* e = std::getenv("QLORA_B200_COPY_WAIT_NS");
+  if (!e) return 2000000000ull;
+  return std::strtoull(e, nullptr, 10);
+}
+
 static int32_t chunks_of(int64_t numel) {
   const int64_t nb = numel / kBlock;
   return static_cast<int32_t>((nb + kDQBlock - 1) / kDQBlock);
@@ -387,13 +400,13 @@ static qlora_status launch_passes(const Tab& tab, double2* partial, int* status,
   const unsigned c = unsigned(tab.first_chunk[n]);
   cudaError_t e;
   if (pdl) {
-    e = launch_pdl(layer_error_chunk_kernel<DQ, Tab>, dim3(c), dim3(256), 0, s, tab, partial, status);
+    e = launch_pdl(layer_error_chunk_kernel<DQ, Tab>, dim3(c), dim3(256), 0, s, tab, partial, status, copy_wait_ns());
     if (e == cudaSuccess) e = launch_pdl(layer_error_finish_kernel, dim3(unsigned(n)), dim3(32), 0, s, partial, r, err);
     if (e == cudaSuccess)
       e = budget ? launch_pdl(rank_budget_kernel, dim3(1), dim3(1024), 0, s, err, n, *budget, order, keep, K_out)
                  : launch_pdl(rank_topk_kernel, dim3(1), dim3(1024), 0, s, err, n, K, order, keep);
   } else {
-    layer_error_chunk_kernel<DQ, Tab><<<c, 256, 0, s>>>(tab, partial, status);
+    layer_error_chunk_kernel<DQ, Tab><<<c, 256, 0, s>>>(tab, partial, status, copy_wait_ns());
     layer_error_finish_kernel<<<unsigned(n), 32, 0, s>>>(partial, r, err);
     if (budget)
       rank_budget_kernel<<<1, 1024, 0, s>>>(err, n, *budget, order, keep, K_out);

@@ -164,3 +164,25 @@ def test_memory_budget_keep_rule(cuda_device, dq):
     costs = np.cumsum([layer_error.protect_cost_bytes(Ws[l].numel(), dq) for l in order])
     budgets = [0, 1, int(costs[-1]) * 10] + [int(c) for c in costs[:5]] + [int(c) - 1 for c in costs[:5]]
     _compare_budget(Ws, dq, budgets)
+
+
+def test_copy_wait_timeout_is_reported(cuda_device, monkeypatch):
+    """Failure detection without a GPU fault: with the chunk kernel's bulk-copy wait
+    limited to a single try, every chunk gives up before its copy lands. The call
+    returns, the status word reads QLORA_ERR_TIMEOUT and the errors are NaN (each
+    timed-out chunk writes a NaN partial); every copy still lands before its CTA exits,
+    so after the status is cleared the same call with the normal limit matches the
+    oracle on the same context."""
+    mats = synth.stack_matrices(n_layers=2, linears=(("a", 256, 512), ("b", 512, 256)))
+    Ws = [synth.stack_weight(m) for m in mats]
+    g = [W.cuda() for W in Ws]
+    monkeypatch.setenv("QLORA_B200_COPY_WAIT_NS", "0")
+    err, order, keep = api.layer_error_rank(g, 2, double_quant=False)
+    torch.cuda.synchronize()
+    assert api.status() == 9          # QLORA_ERR_TIMEOUT
+    assert np.all(np.isnan(err.cpu().numpy()))
+    assert sorted(order.cpu().tolist()) == list(range(len(Ws)))   # still a permutation
+    for ws in api.Workspace.all(torch.cuda.current_device()):
+        api.reset_status(ws)
+    monkeypatch.delenv("QLORA_B200_COPY_WAIT_NS")
+    _compare(Ws, K=2, dq=False)
