@@ -1431,8 +1431,9 @@ qlora_status launch_gemm(GemmKind kind, int bn, const GemmOperands& o, const Gem
       if (bn <= 64) return launch_cfg<GemmCfg<64, false, false, false, true, 8>>(o, p, 1, s);
       if (bn <= 128) return launch_cfg<GemmCfg<128, false, false, false, true, 6>>(o, p, 1, s);
       return launch_cfg<GemmCfg<256, false, false, false, true, 4>>(o, p, 1, s);
-    case GemmKind::ThinKM:  // A K-major, B MN-major
-      if (bn <= 64) return launch_cfg<GemmCfg<64, false, true, false, true, 8>>(o, p, 1, s);
+    case GemmKind::ThinKM:  // A K-major, B MN-major (T = X L1: 4 stages for r <= 64, so the
+                            // allocation pass's CTAs fit beside it on an SM)
+      if (bn <= 64) return launch_cfg<GemmCfg<64, false, true, false, true, 4>>(o, p, 1, s);
       if (bn <= 128) return launch_cfg<GemmCfg<128, false, true, false, true, 6>>(o, p, 1, s);
       return launch_cfg<GemmCfg<256, false, true, false, true, 4>>(o, p, 1, s);
     case GemmKind::ThinMM:  // A MN-major, B MN-major

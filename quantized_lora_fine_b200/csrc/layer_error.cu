@@ -124,8 +124,8 @@ __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_
     mbar_arrive_expect_tx(bar, bytes);
     bulk_load(smem_u32(s_w), tab.ptr[layer] + g * (kDQBlock * kBlock), bytes, bar);
   }
-  // the chunk's copy must land within copy_wait_ns (0: one try, no waiting)
-  const bool landed = copy_wait_ns ? mbar_wait(bar, 0, copy_wait_ns) : mbar_try_wait(bar, 0);
+  // the chunk's copy must land within copy_wait_ns (0: one non-blocking check)
+  const bool landed = copy_wait_ns ? mbar_wait(bar, 0, copy_wait_ns) : mbar_test_wait(bar, 0);
   if (!__syncthreads_and(landed)) {   // every thread leaves together
     if (tid == 0) {
       if (status) set_status(status, QLORA_ERR_TIMEOUT);
@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(32) layer_error_finish_kernel(const double2* _
 }
 
 // Limit of the chunk kernel's wait for its bulk copy: 2 s, or QLORA_B200_COPY_WAIT_NS
-// (read on every call; 0 = a single try). A limit that runs out records
+// (read on every call; 0 = one non-blocking check). A limit that runs out records
 // QLORA_ERR_TIMEOUT (or a NaN error without a status word) and the kernel still waits
 // for its copy to land before it exits; the failure-detection tests use 0.
 static uint64_t copy_wait_ns() {
