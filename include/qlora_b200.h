@@ -125,6 +125,16 @@ qlora_status qlora_profile_events(void* fwd_begin, void* fwd_end, void* dx_begin
  * them, so a part that co-schedules fewer pairs takes more rounds of tiles. */
 int32_t qlora_pair_clusters(void);
 
+/* Diagnostic, host only (no device work): the schedule the NF4 pair GEMM (512 x 256
+ * tiles) uses for `tiles` output tiles of `steps` K steps (K / 64 plus the LoRA
+ * steps) over `pairs` co-resident CTA pairs (1..80):
+ *   out[0] P = pairs, out[1] R = whole rounds (pair p takes tiles p + r P, r < R),
+ *   out[2] L = steps per pair in the remaining tiles (0: none remain), out[3] W =
+ *   their total steps (pair p takes steps [p L, min((p + 1) L, W)) of them, tile
+ *   base + step / steps), out[4] base = R P, out[5] pairs launched.
+ * A tile cut into parts is finished by the pair holding its first step. */
+qlora_status qlora_pair_schedule(int32_t tiles, int32_t steps, int32_t pairs, int32_t* out);
+
 /* ------------------------------------------------------------ NF4 codec */
 
 /* Bytes of workspace nf4_quantize needs (the status word only). */
@@ -335,6 +345,18 @@ qlora_status nf4_layer_error_rank_budget(int32_t n_layers, const uint16_t* const
                                          int32_t w_dtype, nf4_qconfig q, int64_t budget_bytes, double* err,
                                          int32_t* order, uint8_t* keep, int32_t* K_out, void* workspace,
                                          size_t workspace_bytes, qlora_stream_t stream);
+
+/* The ranking step alone ("AQLoRA: A Zero-Search Recipe for Fast Quantized LoRA
+ * Fine-Tuning", section 3.2: layers ranked by their error, the top K kept in 16-bit)
+ * over errors already on the device, e.g. gathered from several GPUs that each
+ * scored their own matrices:
+ *   err    device fp64 [n_layers] (NaN ranks ahead of every number, by id)
+ *   order  device out, int32 [n_layers]: layer ids by (err desc, id asc)
+ *   keep   device out, uint8 [n_layers]: 1 for the first K of `order`
+ * 1 <= n_layers <= 1024, 0 <= K <= n_layers. Deterministic: every caller with the
+ * same errors gets the same order. No workspace. */
+qlora_status nf4_rank_errors(int32_t n_layers, const double* err, int32_t K, int32_t* order, uint8_t* keep,
+                             qlora_stream_t stream);
 
 /* K from a protection fraction rho = num / den of n_layers layers (same page,
  * section 3.2, where rho = 0.2 of 144 linear layers keeps 29): round half up of

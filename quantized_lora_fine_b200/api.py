@@ -383,6 +383,18 @@ def quantize_error_rank(Ws: Sequence[torch.Tensor], K: int, double_quant: bool =
     return err, order, keep, list(outs)
 
 
+def rank_errors(err: torch.Tensor, K: int):
+    """(order, keep) of per-layer errors already on the device (fp64): the ranking
+    step alone, (error desc, index asc), NaN first."""
+    _need(err, torch.float64, "err")
+    lib = _lib.load()
+    L = err.numel()
+    order = torch.empty(L, dtype=torch.int32, device=err.device)
+    keep = torch.empty(L, dtype=torch.uint8, device=err.device)
+    check(lib.nf4_rank_errors(L, _ptr(err), int(K), _ptr(order), _ptr(keep), _stream()), "nf4_rank_errors")
+    return order, keep
+
+
 def status() -> int:
     """First nonzero device status word among this device's workspaces (one per
     stream the library was called on); synchronizes."""

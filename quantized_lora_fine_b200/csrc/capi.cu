@@ -426,6 +426,13 @@ const char* qlora_status_str(qlora_status s) {
 
 int32_t qlora_pair_clusters(void) { return last_pair_clusters(); }
 
+qlora_status qlora_pair_schedule(int32_t tiles, int32_t steps, int32_t pairs, int32_t* out) {
+  if (!out) return QLORA_ERR_NULL;
+  if (tiles < 1 || steps < 1 || pairs < 1 || pairs > kPair2MaxPairs) return QLORA_ERR_SHAPE;
+  pair2_schedule_of(tiles, steps, pairs, out);
+  return QLORA_OK;
+}
+
 qlora_status qlora_profile_events(void* fwd_begin, void* fwd_end, void* dx_begin, void* dx_end) {
   g_prof[0] = static_cast<cudaEvent_t>(fwd_begin);
   g_prof[1] = static_cast<cudaEvent_t>(fwd_end);
@@ -858,6 +865,14 @@ qlora_status nf4_layer_error_rank_budget(int32_t n_layers, const uint16_t* const
   QLB_TRY(check_device());
   return launch_layer_error_rank(n_layers, W_ptrs, numel, q.double_quant != 0, 0, err, order, keep, workspace,
                                  workspace_bytes, static_cast<int*>(workspace), S(stream), budget_bytes, K_out);
+}
+
+qlora_status nf4_rank_errors(int32_t n_layers, const double* err, int32_t K, int32_t* order, uint8_t* keep,
+                            qlora_stream_t stream) {
+  if (n_layers < 1 || n_layers > 1024 || K < 0 || K > n_layers) return QLORA_ERR_SHAPE;
+  if (!err || !order || !keep) return QLORA_ERR_NULL;
+  QLB_TRY(check_device());
+  return launch_rank_errors(n_layers, err, K, order, keep, S(stream));
 }
 
 qlora_status nf4_k_from_fraction(int64_t num, int64_t den, int32_t n_layers, int32_t* K) {

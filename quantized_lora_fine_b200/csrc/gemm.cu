@@ -1347,6 +1347,16 @@ static Pair2Sched pair2_schedule(int T, int S, int P) {
   return sc;
 }
 
+void pair2_schedule_of(int tiles, int steps, int pairs, int32_t* out) {
+  const Pair2Sched sc = pair2_schedule(tiles, steps, pairs);
+  out[0] = sc.P;
+  out[1] = sc.R;
+  out[2] = sc.L;
+  out[3] = sc.W;
+  out[4] = sc.base;
+  out[5] = sc.launch;
+}
+
 size_t pair2_partial_bytes(int64_t M, int64_t N) {
   const int64_t T = ((M + 511) / 512) * (N / 256);
   const int64_t slots = std::min<int64_t>(kPair2MaxPairs, 4 * T);

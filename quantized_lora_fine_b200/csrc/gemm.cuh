@@ -88,6 +88,8 @@ qlora_status launch_gemm_pair(bool dx, const GemmOperands& o, const GemmParams& 
 // p.sk_part (pair2_partial_bytes(...) bytes) and p.sk_count (pair2_counter_ints(...)
 // ints, zero); requires N % 256 == 0.
 qlora_status launch_gemm_pair2(bool dx, const GemmOperands& o, GemmParams p, cudaStream_t s);
+// The schedule over `pairs` co-resident pairs: {P, R, L, W, base, launch} (host only).
+void pair2_schedule_of(int tiles, int steps, int pairs, int32_t* out);
 // Upper bounds of the split-round scratch for a D[M x N] product (host only).
 size_t pair2_partial_bytes(int64_t M, int64_t N);
 constexpr int kPair2MaxPairs = 80;                 // pairs launched at most

@@ -106,6 +106,8 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
                                      int K, double* err, int32_t* order, uint8_t* keep, void* ws, size_t ws_bytes,
                                      int* status, cudaStream_t s, int64_t budget_bytes = 0,
                                      int32_t* K_out = nullptr);
+// The ranking alone over errors already on the device (1 <= n <= 1024).
+qlora_status launch_rank_errors(int n, const double* err, int K, int32_t* order, uint8_t* keep, cudaStream_t s);
 // Stored bytes of one NF4 matrix (codes + scales; double quant as configured).
 int64_t nf4_storage_bytes(int64_t numel, bool dq);
 

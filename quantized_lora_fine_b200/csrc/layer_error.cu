@@ -447,6 +447,11 @@ qlora_status launch_layer_error_rank(int n_layers, const uint16_t* const* W_ptrs
             : launch_passes<false>(tab, partial, status, err, K, order, keep, s, true);
 }
 
+qlora_status launch_rank_errors(int n, const double* err, int K, int32_t* order, uint8_t* keep, cudaStream_t s) {
+  const cudaError_t e = launch_pdl(rank_topk_kernel, dim3(1), dim3(1024), 0, s, err, n, K, order, keep);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 qlora_status launch_quantize_error_rank(int n_layers, const uint16_t* const* W_ptrs, const int64_t* numel, bool dq,
                                        int K, uint8_t* const* codes, float* const* absmax, uint8_t* const* absmax_q,
                                        float* const* absmax2, double* err, int32_t* order, uint8_t* keep, void* ws,

@@ -186,3 +186,24 @@ def test_copy_wait_timeout_is_reported(cuda_device, monkeypatch):
         api.reset_status(ws)
     monkeypatch.delenv("QLORA_B200_COPY_WAIT_NS")
     _compare(Ws, K=2, dq=False)
+
+
+def test_rank_errors_alone_and_sharded_on_one_gpu(cuda_device):
+    """The ranking step alone (nf4_rank_errors) on oracle errors gives the oracle's
+    order and keep; the sharded pass with one rank (the library's error pass and
+    ranking) gives the unsharded call's results."""
+    from quantized_lora_fine_b200 import dist as qdist
+    mats = synth.stack_matrices(n_layers=2, linears=(("a", 256, 512), ("b", 512, 256), ("c", 64, 320)))
+    Ws = [synth.stack_weight(m) for m in mats]
+    ref = np.array([layer_error.layer_error(bits(W), True) for W in Ws])
+    ref_order = layer_error.rank_layers(ref)
+    order, keep = api.rank_errors(torch.tensor(ref, dtype=torch.float64, device="cuda"), 3)
+    torch.cuda.synchronize()
+    assert np.array_equal(order.cpu().numpy(), ref_order)
+    assert np.array_equal(keep.cpu().numpy(), layer_error.keep_mask(ref_order, 3))
+    g = {i: W.cuda() for i, W in enumerate(Ws)}
+    err, order, keep = qdist.sharded_layer_error_rank(g, [W.numel() for W in Ws], 3, double_quant=True)
+    e1, o1, k1 = api.layer_error_rank(list(g.values()), 3, double_quant=True)
+    torch.cuda.synchronize()
+    assert torch.equal(err, e1) and torch.equal(order, o1) and torch.equal(keep, k1)
+    assert api.status() == 0

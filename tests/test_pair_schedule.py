@@ -1,0 +1,92 @@
+"""The NF4 pair GEMM's schedule (host side, from the library) walked with the
+kernel's own step and segment arithmetic (CPU, no device): whole rounds of 512 x 256
+tiles, then the remaining tiles' K steps in equal ranges over the pairs. Every
+(tile, step) is covered exactly once; a tile cut into parts is finished by the pair
+holding its first step, which is that pair's last range, while the later parts are
+their pairs' first ranges (done before it, so the finishing pair's bounded wait
+always ends); no tile has more than four parts; the per-tile counters (two per
+tile) and the per-pair partial slots stay inside their regions."""
+import ctypes
+
+import pytest
+
+from quantized_lora_fine_b200 import _lib, build
+
+MAX_PAIRS = 80          # partial slots and counter pairs reserved in the workspace
+COUNTER_INTS = 2 * MAX_PAIRS
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def schedule(lib, tiles, steps, pairs):
+    out = (ctypes.c_int32 * 6)()
+    assert lib.qlora_pair_schedule(tiles, steps, pairs, out) == 0
+    return list(out)
+
+
+def walk(P, R, L, W, base, launch, tiles, steps):
+    """The kernel's per-pair step sequence and its segments (as the epilogue walks them)."""
+    seen = set()
+    for pr in range(launch):
+        dp = R * steps
+        n = dp + max(0, min(pr * L + L, W) - pr * L)
+        assert n > 0, "a launched pair without work"
+        seq = []
+        for i in range(n):
+            if i < dp:
+                r = i // steps
+                tile, k = pr + r * P, i - r * steps
+            else:
+                ti = pr * L + (i - dp)
+                u = ti // steps
+                tile, k = base + u, ti - u * steps
+            assert 0 <= tile < tiles and 0 <= k < steps
+            assert (tile, k) not in seen
+            seen.add((tile, k))
+            seq.append((tile, k))
+        segs, i = [], 0
+        while i < n:
+            tile, kb = seq[i]
+            ln = steps if i < dp else min(steps - kb, n - i)
+            segs.append((tile, kb, kb + ln))
+            i += ln
+        for si, (tile, kb, ke) in enumerate(segs):
+            if kb == 0 and ke == steps:
+                continue
+            u = tile - base
+            pf, pl = (u * steps) // L, ((u + 1) * steps - 1) // L
+            assert pf <= pr <= pl < launch and pl - pf + 1 <= 4
+            assert 2 * u + 1 < COUNTER_INTS
+            if kb == 0:
+                assert pr == pf and si == len(segs) - 1     # finishing part: the pair's last range
+            else:
+                assert si == R                              # later part: the pair's first range
+    assert len(seen) == tiles * steps
+
+
+@pytest.mark.parametrize("pairs", [1, 2, 3, 5, 7, 16, 37, 64, 72, 73, 74, 80])
+def test_schedule_covers_every_step_once(lib, pairs):
+    for tiles in list(range(1, 48)) + [64, 97, 256, 512, 688, 1280]:
+        for steps in (1, 2, 3, 5, 9, 13, 65, 66, 81, 173, 217):
+            P, R, L, W, base, launch = schedule(lib, tiles, steps, pairs)
+            assert P == pairs and launch <= MAX_PAIRS and launch <= 4 * tiles
+            walk(P, R, L, W, base, launch, tiles, steps)
+
+
+def test_q_proj_last_round_is_split(lib):
+    """q_proj (8192 x 4096 output: 256 tiles of 64 K steps + 1 LoRA step): 3 whole
+    rounds, then 30 or 33 steps per pair on 74 or 73 pairs, instead of a fourth round."""
+    assert schedule(lib, 256, 65, 74)[1:4] == [3, 30, 34 * 65]
+    assert schedule(lib, 256, 65, 73)[1:4] == [3, 33, 37 * 65]
+    assert schedule(lib, 256, 65, 64)[1:3] == [4, 0]
+
+
+def test_schedule_refuses_bad_arguments(lib):
+    out = (ctypes.c_int32 * 6)()
+    assert lib.qlora_pair_schedule(0, 5, 4, out) == 2
+    assert lib.qlora_pair_schedule(5, 5, 81, out) == 2
+    assert lib.qlora_pair_schedule(5, 5, 4, None) == 1
