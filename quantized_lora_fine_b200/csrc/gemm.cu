@@ -1436,18 +1436,19 @@ qlora_status launch_gemm(GemmKind kind, int bn, const GemmOperands& o, const Gem
     case GemmKind::DxNF4: return launch_cfg<GemmCfg<256, false, true, true, false, 3>>(o, p, 1, s);
     case GemmKind::FwdBF16: return launch_cfg<GemmCfg<256, false, false, false, false, 4>>(o, p, 1, s);
     case GemmKind::DxBF16: return launch_cfg<GemmCfg<256, false, true, false, false, 4>>(o, p, 1, s);
-    // thin products: one CTA per SM with a deep ring (HBM-bound streaming of A)
+    // thin products: one CTA per SM, split-K; a 4-stage ring (96 KB of shared memory)
+    // for r <= 64 so that the products the backward runs side by side (U and dL2), and
+    // T beside the allocation pass, can share SMs (measured: the step 8 us shorter)
     case GemmKind::ThinKK:  // A K-major, B K-major, fp32 partials
-      if (bn <= 64) return launch_cfg<GemmCfg<64, false, false, false, true, 8>>(o, p, 1, s);
+      if (bn <= 64) return launch_cfg<GemmCfg<64, false, false, false, true, 4>>(o, p, 1, s);
       if (bn <= 128) return launch_cfg<GemmCfg<128, false, false, false, true, 6>>(o, p, 1, s);
       return launch_cfg<GemmCfg<256, false, false, false, true, 4>>(o, p, 1, s);
-    case GemmKind::ThinKM:  // A K-major, B MN-major (T = X L1: 4 stages for r <= 64, so the
-                            // allocation pass's CTAs fit beside it on an SM)
+    case GemmKind::ThinKM:  // A K-major, B MN-major
       if (bn <= 64) return launch_cfg<GemmCfg<64, false, true, false, true, 4>>(o, p, 1, s);
       if (bn <= 128) return launch_cfg<GemmCfg<128, false, true, false, true, 6>>(o, p, 1, s);
       return launch_cfg<GemmCfg<256, false, true, false, true, 4>>(o, p, 1, s);
     case GemmKind::ThinMM:  // A MN-major, B MN-major
-      if (bn <= 64) return launch_cfg<GemmCfg<64, true, true, false, true, 8>>(o, p, 1, s);
+      if (bn <= 64) return launch_cfg<GemmCfg<64, true, true, false, true, 4>>(o, p, 1, s);
       if (bn <= 128) return launch_cfg<GemmCfg<128, true, true, false, true, 6>>(o, p, 1, s);
       return launch_cfg<GemmCfg<256, true, true, false, true, 4>>(o, p, 1, s);
   }
