@@ -665,6 +665,9 @@ def gpu_main(args):
     def leg_fwd():
         state["Y"], state["T"] = api.linear_fwd(state["w"], g["X"], g["L1"], g["L2"], s, T=state["T"])
 
+    def leg_fwd_fused_t():   # the one-call forward: T = X L1 in the GEMM's own tiles
+        state["Y"], state["T"] = api.linear_fwd(state["w"], g["X"], g["L1"], g["L2"], s)
+
     def leg_bwd():
         state["dX"], state["dL1"], state["dL2"] = api.linear_bwd(state["w"], g["X"], g["dY"], g["L1"], g["L2"], s,
                                                                   T=state["T"])
@@ -684,7 +687,8 @@ def gpu_main(args):
     if use_graphs:
         try:
             for name, fn in (("step", whole_step), ("quantize_error_rank", leg_quant), ("lora_down", leg_down),
-                             ("fwd", leg_fwd), ("bwd", leg_bwd), ("fwd_bwd", fwd_bwd)):
+                             ("fwd", leg_fwd), ("fwd_fused_t", leg_fwd_fused_t), ("bwd", leg_bwd),
+                             ("fwd_bwd", fwd_bwd)):
                 gr = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(gr):
                     fn()
@@ -700,8 +704,8 @@ def gpu_main(args):
         else:
             fn()
 
-    step_ms, legs = [], {"quantize_error_rank": [], "lora_down": [], "fwd": [], "bwd": [], "fwd_bwd": [],
-                         "fwd_gemm": [], "dx_gemm": []}
+    step_ms, legs = [], {"quantize_error_rank": [], "lora_down": [], "fwd": [], "fwd_fused_t": [], "bwd": [],
+                         "fwd_bwd": [], "fwd_gemm": [], "dx_gemm": [], "fwd_fused_t_gemm": []}
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -719,7 +723,7 @@ def gpu_main(args):
         legs["dx_gemm"].append(prof[2].elapsed_time(prof[3]))
     clk = clocks.stop()
     for name, fn in (("quantize_error_rank", leg_quant), ("lora_down", leg_down), ("fwd", leg_fwd),
-                     ("bwd", leg_bwd), ("fwd_bwd", fwd_bwd)):
+                     ("fwd_fused_t", leg_fwd_fused_t), ("bwd", leg_bwd), ("fwd_bwd", fwd_bwd)):
         for i in range(max(5, min(args.steps, 50))):
             flush.zero_()
             ev[2].record(stream)
@@ -727,6 +731,8 @@ def gpu_main(args):
             ev[3].record(stream)
             ev[3].synchronize()
             legs[name].append(ev[2].elapsed_time(ev[3]))
+            if name == "fwd_fused_t":
+                legs["fwd_fused_t_gemm"].append(prof[0].elapsed_time(prof[1]))
     lib.qlora_profile_events(None, None, None, None)
     torch.cuda.synchronize()
     assert api.status() == 0, "device status set during timing"
@@ -769,7 +775,11 @@ def gpu_main(args):
                                 "GB/s": qer_bytes / (med["quantize_error_rank"] * 1e-3) / 1e9,
                                 "frac_hbm": qer_bytes / (med["quantize_error_rank"] * 1e-3) / 1e9 / peaks["hbm"]},
         "lora_down": {"ms": med["lora_down"], "note": "T = X L1; in the step the allocation pass runs beside it"},
-        "fwd": {"ms": med["fwd"], "note": "with T given"}, "bwd": {"ms": med["bwd"]},
+        "fwd": {"ms": med["fwd"], "note": "with T given"},
+        "fwd_fused_t": {"ms": med["fwd_fused_t"], "gemm_ms": med["fwd_fused_t_gemm"],
+                        "note": "the one-call forward: T = X L1 in the GEMM's own tiles (the step instead runs "
+                                "T beside the allocation pass, which measured faster)"},
+        "bwd": {"ms": med["bwd"]},
         "fwd_bwd": {"ms": med["fwd_bwd"], "TFLOP/s": fl / (med["fwd_bwd"] * 1e-3) / 1e12,
                     "frac_of_burst": fl / (med["fwd_bwd"] * 1e-3) / 1e12 / peaks["bf16"],
                     "note": "T, forward and backward of the linear without the allocation pass"},

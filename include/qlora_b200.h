@@ -36,10 +36,12 @@
  *     workspace. The word is sticky: it keeps the first error until
  *     qlora_reset_status(). A fresh workspace must be zeroed (or reset) once.
  *   - One workspace may serve every entry point on a stream: its first 256
- *     bytes hold the status word, the next 64 KiB split-K tile counters that
- *     must be zero when a call starts and that every call leaves zero; a
- *     call's other scratch comes after them. Zeroing a workspace once keeps
- *     this true for any sequence of calls.
+ *     bytes hold the status word, the next 64 KiB + 4 KiB split-K tile
+ *     counters and the forward GEMM's per-row-block flags, which must be zero
+ *     when a call starts and which every call that ends with status 0 leaves
+ *     zero; a call's other scratch comes after them. Zeroing a workspace once
+ *     keeps this true for any sequence of successful calls; after an error,
+ *     qlora_reset_workspace() restores it.
  *   - No call aborts the process or throws.
  */
 #ifndef QLORA_B200_H
@@ -110,6 +112,14 @@ qlora_status qlora_read_status(const void* workspace, qlora_stream_t stream);
 
 /* Clears the device status word (stream-ordered). */
 qlora_status qlora_reset_status(void* workspace, qlora_stream_t stream);
+
+/* Clears the status word and the tile counters and block flags that follow it
+ * (the workspace's first min(workspace_bytes, 256 + 64 KiB + 4 KiB) bytes;
+ * stream-ordered). A call that ended with a nonzero status may have stopped
+ * between setting and clearing those, so reset this way (not only the status
+ * word) before the workspace serves a GEMM again. QLORA_ERR_WORKSPACE when
+ * workspace is NULL or smaller than 256 bytes. */
+qlora_status qlora_reset_workspace(void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
 /* Checks that device `device` is an sm_100 (B200-class) part. */
 qlora_status qlora_device_check(int device);

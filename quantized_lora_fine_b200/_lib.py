@@ -34,6 +34,7 @@ SIGNATURES = {
     "qlora_status_str": (c_char_p, [c_int]),
     "qlora_read_status": (c_int, [c_void_p, c_void_p]),
     "qlora_reset_status": (c_int, [c_void_p, c_void_p]),
+    "qlora_reset_workspace": (c_int, [c_void_p, c_size_t, c_void_p]),
     "qlora_device_check": (c_int, [c_int]),
     "qlora_profile_events": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p]),
     "qlora_pair_clusters": (c_int32, []),

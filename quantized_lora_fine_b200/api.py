@@ -66,7 +66,10 @@ def read_status(ws: torch.Tensor) -> int:
 
 
 def reset_status(ws: torch.Tensor) -> None:
-    check(_lib.load().qlora_reset_status(ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(_stream())), "reset_status")
+    """Clears the status word and the tile counters / block flags after it (an
+    interrupted GEMM can leave those set)."""
+    check(_lib.load().qlora_reset_workspace(ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(),
+                                            ctypes.c_void_p(_stream())), "reset_status")
 
 
 @dataclasses.dataclass

@@ -65,7 +65,8 @@ int thin_bn(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
 
 // ---- workspace layouts
 
-static_assert(size_t(kPair2CounterInts) * sizeof(int) <= kGemmCounterBytes, "pair-GEMM counters fit their region");
+static_assert(size_t(kPair2CounterInts + 4 * kPair2MaxTBlocks) * sizeof(int) <= kGemmCounterBytes,
+              "pair-GEMM counters and T flags fit their region");
 
 struct FwdLayout {
   size_t scales, l2t, t, part, gpart, counters, total;
@@ -240,15 +241,24 @@ int gemm_engine() {
   return v;
 }
 bool use_pair_kernel() { return gemm_engine() >= 1; }
+// T = X L1 inside the forward GEMM unless QLORA_B200_FUSED_T=0 (read on every call; the
+// separate T pass is kept for measurement).
+bool fused_t_enabled() {
+  const char* e = std::getenv("QLORA_B200_FUSED_T");
+  return !(e && std::strcmp(e, "0") == 0);
+}
 
 // Fused NF4 GEMM on CTA pairs (256 x 256 tiles): out = A . W' + Ax . Bx^T, where
 // the LoRA step reads Bx as [N x r] rows: Ax = T with Bx = s.L2^T (fwd), or
 // Ax = s.U with Bx = L1 as stored (dX). Codes are read in place, scales from S_t.
 // (An MN-major LoRA B read straight from L2 [r x out] was measured 12 us slower
 // per forward GEMM on the q_proj workload than this transposed copy.)
+// With t_out (forward, 512 x 256 engine) the GEMM also computes T = X L1 into t_out
+// (its T tiles, before the output tiles' LoRA steps read it; Ax must be t_out).
 qlora_status run_pair(bool dx, const qlora_weight* w, const uint16_t* A, int64_t M, const uint16_t* Ax,
                       const uint16_t* Bx, int32_t r, const float* scales_t, uint16_t* out, int* status,
-                      float* gpart, int* gcount, cudaStream_t s) {
+                      float* gpart, int* gcount, cudaStream_t s, const uint16_t* L1 = nullptr,
+                      uint16_t* t_out = nullptr) {
   const int64_t o_ = w->out, h = w->in;
   const int64_t Kdim = dx ? o_ : h;
   const int64_t Ndim = dx ? h : o_;
@@ -280,6 +290,14 @@ qlora_status run_pair(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
     p.sk_count = gcount;
     // output written by TMA: 128-row x 64-column boxes, 128-byte swizzle
     if (!make_tmap_2d(&pp.Y, out, TmapType::BF16, Ndim, M, Ndim * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+    if (t_out) {
+      // T tiles: B = L1 [in x r] as MN-major 64 x 64 chunks; T [M x r] stored in 128 x 64 boxes
+      if (!make_tmap_2d(&pp.L1, L1, TmapType::BF16, r, h, int64_t(r) * 2, 64, 64, true)) return QLORA_ERR_CUDA;
+      if (!make_tmap_2d(&pp.Tout, t_out, TmapType::BF16, r, M, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+      p.aux_tiles = p.tiles_m;
+      p.t_chunks = (r + 63) / 64;
+      p.t_flags = gcount + kPair2CounterInts;
+    }
   }
   record_prof(g_prof[dx ? 2 : 0], s);
   const qlora_status st = gemm_engine() == 2 ? launch_gemm_pair2(dx, pp, p, s) : launch_gemm_pair(dx, pp, p, s);
@@ -461,6 +479,12 @@ qlora_status qlora_read_status(const void* workspace, qlora_stream_t stream) {
 qlora_status qlora_reset_status(void* workspace, qlora_stream_t stream) {
   if (!workspace) return QLORA_ERR_WORKSPACE;
   return cudaMemsetAsync(workspace, 0, sizeof(int), S(stream)) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_reset_workspace(void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  if (!workspace || workspace_bytes < kStatusBytes) return QLORA_ERR_WORKSPACE;
+  const size_t n = std::min(workspace_bytes, kReservedBytes);
+  return cudaMemsetAsync(workspace, 0, n, S(stream)) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
 size_t nf4_quantize_workspace_size(int64_t) { return kStatusBytes; }
@@ -673,13 +697,20 @@ qlora_status linear_fwd_impl(const qlora_weight* w, const uint16_t* X, int64_t M
                                  scales_t, aux));
   QLB_TRY(launch_scale_lora(L2, r, o_, scale, /*transpose=*/true, l2t, aux));
   const uint16_t* T = T_in;
-  if (!T) {
-    uint16_t* Tw = T_save ? T_save : reinterpret_cast<uint16_t*>(ws + L.t);
+  // T = X L1 inside the NF4 GEMM (its T tiles read X while it is in L2), unless T is
+  // given, the weight is protected, another engine runs, or M has too many row blocks
+  const bool fuse_t = !T_in && !w->is_bf16 && gemm_engine() == 2 && fused_t_enabled() &&
+                      (M + 511) / 512 <= kPair2MaxTBlocks;
+  uint16_t* Tw = T_save ? T_save : reinterpret_cast<uint16_t*>(ws + L.t);
+  if (!T && !fuse_t) {
     Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
     QLB_TRY(run_thin(tt, part, counters, Tw, 0, 1.f, status, s));
     T = Tw;
   }
   if (ss) QLB_TRY(join_from(ss, s));
+  if (fuse_t)
+    return run_pair(false, w, X, M, Tw, l2t, r, scales_t, Y, status, reinterpret_cast<float*>(ws + L.gpart),
+                    reinterpret_cast<int*>(ws + kStatusBytes + kCounterBytes), s, L1, Tw);
   if (!w->is_bf16 && use_pair_kernel())
     return run_pair(false, w, X, M, T, l2t, r, scales_t, Y, status, reinterpret_cast<float*>(ws + L.gpart),
                     reinterpret_cast<int*>(ws + kStatusBytes + kCounterBytes), s);

@@ -817,10 +817,24 @@ __device__ __forceinline__ void sk_step(const GemmParams& p, int pr, uint32_t i,
   }
 }
 
+// Block and column tile of a tile id: the aux_tiles leading T tiles (block = id,
+// column -1), then the output tiles row-block-major.
+__device__ __forceinline__ void sk_tile(const GemmParams& p, int tile, int& mb, int& nb) {
+  if (tile < p.aux_tiles) {
+    mb = tile;
+    nb = -1;
+  } else {
+    const int t2 = tile - p.aux_tiles;
+    mb = t2 / p.tiles_n;
+    nb = t2 - mb * p.tiles_n;
+  }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, 1)
     tc_gemm_nf4_pair2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAx,
                              const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmY,
+                             const __grid_constant__ CUtensorMap tmL1, const __grid_constant__ CUtensorMap tmT,
                              const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -864,6 +878,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   const int S = p.num_k_main + p.num_k_ext;
   const uint32_t nsteps = sk_num_steps(p, pr);
   const uint32_t dp_steps = uint32_t(p.sk_R) * uint32_t(S);
+  // MMA width of the T tiles: 128 columns hold r <= 128, else 256
+  const int t_n = p.t_chunks <= 2 ? 128 : 256;
 
   if (warp == 0) {
     // ------------------------------------------------------------ A producer (both CTAs)
@@ -878,15 +894,42 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           set_status_site(p.status, QLORA_ERR_TIMEOUT, 201);
           break;
         }
-        const int m0 = (tile / p.tiles_n) * 512 + int(rank) * 128;
+        int mb, nb;
+        sk_tile(p, tile, mb, nb);
+        const bool ttile = nb < 0;
+        const int m0 = mb * 512 + int(rank) * 128;
         const bool main_step = k < p.num_k_main;
         const uint32_t dst = slot(it), bar = ready(it % C::S);
-        const CUtensorMap* m = main_step ? &tmA : &tmAx;
-        const int kx = (main_step ? k : k - p.num_k_main) * 64;
+        // a T tile reads X in every step (its extra step starts past the K extent: zeros)
+        const bool x_step = main_step || ttile;
+        const CUtensorMap* m = x_step ? &tmA : &tmAx;
+        const int kx = (x_step ? k : k - p.num_k_main) * 64;
+        if (!x_step && p.aux_tiles > 0 && k == p.num_k_main) {
+          // the first LoRA step of an output tile needs its block's T: wait for the flag
+          int* fl = p.t_flags + (mb * 2 + int(rank)) * 2;
+          if (ld_acquire_gpu(fl) == 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_gpu(fl) == 0) {
+              if (globaltimer_ns() - t0 > 2000000000ull) {
+                set_status_site(p.status, QLORA_ERR_TIMEOUT, 202);
+                break;
+              }
+            }
+          }
+          fence_proxy_async_global();
+          // the block's last reader clears the flag for the next call
+          if (atomicAdd(fl + 1, 1) == p.tiles_n - 1) {
+            fl[1] = 0;
+            fl[0] = 0;
+          }
+        }
         if (rank == 0) {
-          // bytes of the whole step: both CTAs' two A sub-tiles and, in LoRA steps, B halves
-          mbar_arrive_expect_tx(bar, 4 * C::kA + (main_step ? uint32_t(C::kWarpsPerSlot * C::kSigBytes)
-                                                            : uint32_t(2 * C::kB)));
+          // bytes of the whole step: both CTAs' two A sub-tiles and, in LoRA steps and T
+          // tiles, B halves by TMA
+          // (a T tile's B is its MMA width t_n x 64 rows of L1, split over the pair)
+          mbar_arrive_expect_tx(bar, 4 * C::kA + (main_step && !ttile ? uint32_t(C::kWarpsPerSlot * C::kSigBytes)
+                                                  : ttile             ? uint32_t(t_n * 128)
+                                                                      : uint32_t(2 * C::kB)));
           tma_load_2d(dst, m, bar, kx, m0);
           tma_load_2d(dst + C::kA, m, bar, kx, m0 + 256);
         } else {
@@ -903,6 +946,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     if (rank == 0 && lane == 0) {
       constexpr uint32_t idesc_main = make_idesc_bf16(256, 256, 0, C::B_MN ? 1 : 0);
       constexpr uint32_t idesc_ext = make_idesc_bf16(256, 256, 0, 0);   // LoRA B is [N x r], K-major
+      // T tiles: L1 [K x r], MN-major, N = t_n
+      const uint32_t idesc_t = t_n == 128 ? make_idesc_bf16(256, 128, 0, 1) : make_idesc_bf16(256, 256, 0, 1);
       constexpr uint32_t b_adv = C::B_MN ? (2048u >> 4) : (32u >> 4);
       constexpr uint32_t b_adv_ext = 32u >> 4;
       const uint64_t da_base = make_smem_desc(slot(0), 16u, 1024u, kSwizzle128B);
@@ -928,8 +973,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         tc_fence_after();
         const bool ext = k >= p.num_k_main;
         const uint64_t ad = da_base + si * kSlotAdv, bd = db_base + si * kSlotAdv;
-        const uint32_t badv = ext ? b_adv_ext : b_adv;
-        const uint32_t idesc = ext ? idesc_ext : idesc_main;
+        // a T tile's B (L1 as stored) is MN-major in every step
+        const bool ttile = tile < p.aux_tiles;
+        const uint32_t badv = ttile ? (2048u >> 4) : ext ? b_adv_ext : b_adv;
+        const uint32_t idesc = ttile ? idesc_t : ext ? idesc_ext : idesc_main;
 #pragma unroll
         for (uint32_t kk = 0; kk < 4; ++kk)
           tc_mma_bf16_pair(tmem_base, ad + 2 * kk, bd + kk * badv, idesc, (!first || kk > 0) ? 1u : 0u);
@@ -976,7 +1023,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       const int len = (i < dp_steps) ? S : min(S - kb, int(nsteps - i));
       i += uint32_t(len);
       const int ke = kb + len;
-      const int mb = tile / p.tiles_n, nb = tile - mb * p.tiles_n;
+      int mb, nb;
+      sk_tile(p, tile, mb, nb);
+      const bool ttile = nb < 0;                         // a T tile: T = X L1 of block mb
+      const int nchunks = ttile ? p.t_chunks : 4;        // 64-column chunks written
       const uint32_t par = seg & 1u;
       ++seg;
       int extra = 0, pf1 = 0;     // partials of later parts to add, from pair slots pf1, pf1 + 1, ...
@@ -1028,14 +1078,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         tc_fence_after();
         const int y = mb * 512 + h * 256 + int(rank) * 128;   // first output row of this store box
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c, ++chunk) {
+        for (int c = 0; c < nchunks; ++c, ++chunk) {
           const uint32_t buf = chunk % uint32_t(C::kNumStage);
           uint32_t v[64];
           tmem_ld_32x32b_x32(tl + uint32_t(h) * 256u + uint32_t(c) * 64u, *reinterpret_cast<uint32_t(*)[32]>(v));
           tmem_ld_32x32b_x32(tl + uint32_t(h) * 256u + uint32_t(c) * 64u + 32u,
                              *reinterpret_cast<uint32_t(*)[32]>(v + 32));
           tmem_ld_wait();
-          if (c == 3) {
+          if (c == nchunks - 1) {
             // the accumulator is in registers: the next tile's MMAs may overwrite it
             tc_fence_before();
             __syncwarp();
@@ -1066,7 +1116,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           fence_proxy_async_smem();
           named_bar_sync(1, C::kEpiThreads);
           if (leader && y < p.M) {   // rows past M are clipped by the store; a box wholly past M is skipped
-            tma_store_2d(&tmY, stage0 + buf * C::kStageBytes, nb * 256 + c * 64, y);
+            if (ttile) tma_store_2d(&tmT, stage0 + buf * C::kStageBytes, c * 64, y);   // columns past r clipped
+            else tma_store_2d(&tmY, stage0 + buf * C::kStageBytes, nb * 256 + c * 64, y);
           }
           if (leader) bulk_commit_group();
         }
@@ -1074,6 +1125,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       if (extra > 0 && leader) {
         // every later part has been read: the counter goes back to zero for the next call
         p.sk_count[2 * (tile - p.sk_base) + int(rank)] = 0;
+      }
+      if (ttile && leader) {
+        // this CTA's T rows of the block are in global memory: raise its flag for the
+        // output tiles' LoRA steps (they read T with TMA after an acquire of the flag)
+        bulk_wait_group<0>();
+        fence_proxy_async_global();
+        __threadfence();
+        st_release_gpu(p.t_flags + (mb * 2 + int(rank)) * 2, 1);
       }
     }
     if (leader) bulk_wait_group<0>();
@@ -1085,12 +1144,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     const uint32_t row = sub * 32 + lane;
     const uint32_t ready_even = mapa_shared(ready(own), 0);
     const uint32_t sig_even = mapa_shared(smem_base + C::kSigOff + dw * C::kSigBytes, 0);
-    auto nc0_of = [&](int t) { return (t % p.tiles_n) * 256 + int(rank) * 128; };
+    auto nc0_of = [&](int t) { return ((t - p.aux_tiles) % p.tiles_n) * 256 + int(rank) * 128; };
     PairRaw raw;
     if (own < nsteps) {
       int t, k;
       sk_step(p, pr, own, t, k);
-      if (k < p.num_k_main) pair_load_raw<C::B_MN>(p, row, k, nc0_of(t), raw);
+      if (k < p.num_k_main && t >= p.aux_tiles) pair_load_raw<C::B_MN>(p, row, k, nc0_of(t), raw);
     }
     for (uint32_t it = own; it < nsteps; it += C::S) {
       int t, k;
@@ -1101,7 +1160,22 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         set_status_site(p.status, QLORA_ERR_TIMEOUT, 218);
         break;
       }
-      if (k < p.num_k_main) {
+      if (t < p.aux_tiles) {
+        if (lane == 0) {
+          // T tile: this CTA's B half is L1 rows 64 k.. (zeros past the K extent), columns
+          // (t_n / 2) rank .. + t_n / 2 - 1 (zeros past r), as MN-major 64-column chunks by
+          // TMA; the even A producer posted its bytes
+          const uint32_t bar = rank == 0 ? ready(own) : ready_even;
+          if (sub == 0) {
+            for (int c = 0; c < t_n / 128; ++c) {
+              const int x = int(rank) * (t_n / 2) + 64 * c;
+              if (rank == 0) tma_load_2d(b_tile + c * 8192, &tmL1, bar, x, k * 64);
+              else tma_load_2d_pair(b_tile + c * 8192, &tmL1, bar, x, k * 64);
+            }
+          }
+          if (rank == 0) mbar_arrive(ready(own));
+        }
+      } else if (k < p.num_k_main) {
         pair_store_block<C::B_MN>(row, 0, raw, b_tile);
         pair_store_block<C::B_MN>(row, 1, raw, b_tile);
         fence_proxy_async_smem();
@@ -1125,7 +1199,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       if (nx < nsteps) {
         int t2, k2;
         sk_step(p, pr, nx, t2, k2);
-        if (k2 < p.num_k_main) pair_load_raw<C::B_MN>(p, row, k2, nc0_of(t2), raw);
+        if (k2 < p.num_k_main && t2 >= p.aux_tiles) pair_load_raw<C::B_MN>(p, row, k2, nc0_of(t2), raw);
       }
       __syncwarp();
     }
@@ -1358,7 +1432,7 @@ void pair2_schedule_of(int tiles, int steps, int pairs, int32_t* out) {
 }
 
 size_t pair2_partial_bytes(int64_t M, int64_t N) {
-  const int64_t T = ((M + 511) / 512) * (N / 256);
+  const int64_t T = ((M + 511) / 512) * (N / 256 + 1);   // with the forward's T tiles
   const int64_t slots = std::min<int64_t>(kPair2MaxPairs, 4 * T);
   return size_t(slots) * (size_t(2) * 2 * 256 * 128 * sizeof(float));
 }
@@ -1368,8 +1442,11 @@ static qlora_status launch_pair2_cfg(const GemmOperands& o, GemmParams p, cudaSt
   const int max_pairs = std::min(pair2_max_clusters<C>(), pair2_pair_cap());
   if (max_pairs <= 0) return QLORA_ERR_CUDA;
   p.bn = 256;
-  const int T = p.tiles_m * p.tiles_n;
+  const int T = p.aux_tiles + p.tiles_m * p.tiles_n;
   const int S = p.num_k_main + p.num_k_ext;
+  if (p.aux_tiles > 0 && (p.aux_tiles != p.tiles_m || p.aux_tiles > kPair2MaxTBlocks || !p.t_flags ||
+                          p.t_chunks < 1 || p.t_chunks > 4))
+    return QLORA_ERR_CUDA;
   if (T <= 0 || S <= 0) return QLORA_OK;
   const Pair2Sched sc = pair2_schedule(T, S, max_pairs);
   p.sk_P = sc.P;
@@ -1393,7 +1470,7 @@ static qlora_status launch_pair2_cfg(const GemmOperands& o, GemmParams p, cudaSt
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 2 : 1;
-  if (cudaLaunchKernelEx(&cfg, tc_gemm_nf4_pair2_kernel<C>, o.A, o.Ax, o.Bx, o.Y, p) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, tc_gemm_nf4_pair2_kernel<C>, o.A, o.Ax, o.Bx, o.Y, o.L1, o.Tout, p) != cudaSuccess)
     return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }

@@ -48,10 +48,18 @@ struct GemmParams {
   int sk_P, sk_R, sk_L, sk_W, sk_base;
   float* sk_part;
   int* sk_count;
+  // Forward of the 512 x 256 pair kernel with T = X L1 fused in: aux_tiles leading
+  // "T tiles" (one per 512-row block, tile id = block) multiply the block's X rows by
+  // L1 (loaded by TMA in place of a dequantized B) and store T (t_chunks 64-column
+  // chunks) before raising the block's flag in t_flags; a main tile's first LoRA step
+  // waits (bounded) for its block's flag. t_flags holds [flag, readers] per block and
+  // CTA rank, left at zero (the last reader clears them). aux_tiles = 0: no T tiles.
+  int aux_tiles, t_chunks;
+  int* t_flags;
 };
 
 struct GemmOperands {
-  CUtensorMap A, B, codes, scales, Ax, Bx, Y;
+  CUtensorMap A, B, codes, scales, Ax, Bx, Y, L1, Tout;
 };
 
 enum class GemmKind {
@@ -94,5 +102,8 @@ void pair2_schedule_of(int tiles, int steps, int pairs, int32_t* out);
 size_t pair2_partial_bytes(int64_t M, int64_t N);
 constexpr int kPair2MaxPairs = 80;                 // pairs launched at most
 constexpr int kPair2CounterInts = 2 * kPair2MaxPairs;   // two per split tile
+// T fused into the forward: 4 ints per 512-row block after the split-tile counters, so
+// at most this many blocks (M <= 110592 tokens); larger M runs T as its own pass.
+constexpr int kPair2MaxTBlocks = 216;
 
 }  // namespace qlb

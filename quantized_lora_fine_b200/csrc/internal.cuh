@@ -16,8 +16,9 @@ constexpr size_t kStatusBytes = 256;
 // counters (only ever used as counters, which the kernels return to zero), then
 // per-call scratch.
 constexpr size_t kCounterBytes = 65536;
-// then 1 KiB of tile counters of the pair GEMM's split last round (also left at zero)
-constexpr size_t kGemmCounterBytes = 1024;
+// then 4 KiB of pair-GEMM counters and flags (the split last round's tile counters and
+// the fused forward's per-block T flags; also left at zero)
+constexpr size_t kGemmCounterBytes = 4096;
 constexpr size_t kReservedBytes = kStatusBytes + kCounterBytes + kGemmCounterBytes;
 constexpr int64_t kMaxCounterTiles = int64_t(kCounterBytes / 4);
 

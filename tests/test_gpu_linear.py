@@ -163,9 +163,11 @@ def test_14b_protected_layer_full_size_sampled(cuda_device):
     run_and_compare(case, protected=True, rows=rows)
 
 
-def test_two_part_forward_matches_forward(cuda_device):
+def test_two_part_forward_matches_forward(cuda_device, monkeypatch):
     """lora_down + linear_fwd(T=...) is the forward split in two: the same bits as
-    the one-call forward (same kernels, same T)."""
+    the one-call forward when that one computes T in its own pass (same kernels,
+    same T)."""
+    monkeypatch.setenv("QLORA_B200_FUSED_T", "0")
     case = synth.case_small()
     d = case.make()
     g, w = gpu_case(d, case.double_quant, False)
@@ -179,9 +181,10 @@ def test_two_part_forward_matches_forward(cuda_device):
     assert torch.equal(Y1, Y2)
 
 
-def test_quantize_on_side_stream_beside_lora_down(cuda_device):
+def test_quantize_on_side_stream_beside_lora_down(cuda_device, monkeypatch):
     """The allocation pass on a second stream while T = X L1 runs on the first (each
     stream has its own workspace): the same codes, scales and outputs as in order."""
+    monkeypatch.setenv("QLORA_B200_FUSED_T", "0")
     case = synth.case_small()
     d = case.make()
     g = {k: v.cuda() for k, v in d.items()}
@@ -202,6 +205,34 @@ def test_quantize_on_side_stream_beside_lora_down(cuda_device):
     assert torch.equal(w.codes, ref_w.codes) and torch.equal(w.absmax_q, ref_w.absmax_q)
     assert torch.equal(w.absmax2, ref_w.absmax2)
     assert torch.equal(T, Tref) and torch.equal(Y, Yref)
+
+
+@pytest.mark.parametrize("M,r,pairs", [(1300, 16, None), (1300, 72, None), (600, 256, None), (2048, 64, None),
+                                       (1300, 16, 3), (2048, 64, 5)])
+def test_fused_t_tiles(cuda_device, monkeypatch, M, r, pairs):
+    """The forward GEMM computes T = X L1 itself: one extra tile per 512-row block
+    (A = the X rows, B = L1), whose rows the output tiles' LoRA step waits for. T and
+    Y are within the oracle's tolerance, and T differs from the separate T = X L1
+    pass by at most one bf16 rounding (the fp32 sums are added in another order).
+    Ragged M and r (a partial 64-column chunk of T), r = 256 (four chunks), and a
+    capped pair count (T tiles cut into step ranges) are covered."""
+    if pairs is not None:
+        monkeypatch.setenv("QLORA_B200_MAX_PAIRS", str(pairs))
+    c = dataclasses.replace(synth.case_small(), M=M, out=768, inp=512, r=r, alpha=2.0 * r, double_quant=True)
+    monkeypatch.delenv("QLORA_B200_FUSED_T", raising=False)
+    run_and_compare(c)
+    d = c.make()
+    g, w = gpu_case(d, c.double_quant, False)
+    Yf, Tf = api.linear_fwd(w, g["X"], g["L1"], g["L2"], c.scale)
+    monkeypatch.setenv("QLORA_B200_FUSED_T", "0")
+    Yu, Tu = api.linear_fwd(w, g["X"], g["L1"], g["L2"], c.scale)
+    torch.cuda.synchronize()
+    assert api.status() == 0
+    tf, tu = Tf.double(), Tu.double()
+    # one bf16 rounding, plus fp32 summation-order slack where T nearly cancels
+    slack = 2.0 ** -7 * tu.abs() + 2.0 ** -16 * tu.abs().max()
+    assert torch.all((tf - tu).abs() <= slack), "fused T off by more than one rounding"
+    assert_close(f64_of_bf16(Yf), f64_of_bf16(Yu), "Y fused vs separate T")
 
 
 @pytest.mark.parametrize("schedule", ["beside", "serial"])
