@@ -54,7 +54,12 @@ struct ThinSplit {
 ThinSplit thin_split(int64_t rows, int64_t ksteps) {
   ThinSplit t;
   t.tiles = int((rows + 127) / 128);
-  int sp = std::max(1, int(kThinTargetCtas / t.tiles));  // one wave of CTAs
+  static const int target = [] {
+    const char* e = std::getenv("QLORA_B200_THIN_CTAS");
+    const int v = e ? std::atoi(e) : 0;
+    return v > 0 ? v : kThinTargetCtas;
+  }();
+  int sp = std::max(1, int(target / t.tiles));  // one wave of CTAs
   sp = int(std::min<int64_t>(sp, ksteps));
   t.kps = int((ksteps + sp - 1) / sp);
   t.splits = int((ksteps + t.kps - 1) / t.kps);
@@ -247,18 +252,25 @@ bool fused_t_enabled() {
   const char* e = std::getenv("QLORA_B200_FUSED_T");
   return !(e && std::strcmp(e, "0") == 0);
 }
+// U = dY L2^T inside the dX GEMM unless QLORA_B200_FUSED_U=0 (read on every call).
+bool fused_u_enabled() {
+  const char* e = std::getenv("QLORA_B200_FUSED_U");
+  return !(e && std::strcmp(e, "0") == 0);
+}
 
 // Fused NF4 GEMM on CTA pairs (256 x 256 tiles): out = A . W' + Ax . Bx^T, where
 // the LoRA step reads Bx as [N x r] rows: Ax = T with Bx = s.L2^T (fwd), or
 // Ax = s.U with Bx = L1 as stored (dX). Codes are read in place, scales from S_t.
 // (An MN-major LoRA B read straight from L2 [r x out] was measured 12 us slower
 // per forward GEMM on the q_proj workload than this transposed copy.)
-// With t_out (forward, 512 x 256 engine) the GEMM also computes T = X L1 into t_out
-// (its T tiles, before the output tiles' LoRA steps read it; Ax must be t_out).
+// With aux_out (512 x 256 engine) the GEMM also computes the LoRA product its
+// output tiles' LoRA step reads, in its own aux tiles before them: forward, T = X L1
+// into aux_out (aux_b = L1; Ax must be aux_out); dX, U = dY L2^T into aux_out and
+// bf16(aux_scale * U) into aux_out2 (aux_b = L2; Ax must be aux_out2).
 qlora_status run_pair(bool dx, const qlora_weight* w, const uint16_t* A, int64_t M, const uint16_t* Ax,
                       const uint16_t* Bx, int32_t r, const float* scales_t, uint16_t* out, int* status,
-                      float* gpart, int* gcount, cudaStream_t s, const uint16_t* L1 = nullptr,
-                      uint16_t* t_out = nullptr) {
+                      float* gpart, int* gcount, cudaStream_t s, const uint16_t* aux_b = nullptr,
+                      uint16_t* aux_out = nullptr, uint16_t* aux_out2 = nullptr, float aux_scale = 0.f) {
   const int64_t o_ = w->out, h = w->in;
   const int64_t Kdim = dx ? o_ : h;
   const int64_t Ndim = dx ? h : o_;
@@ -290,13 +302,25 @@ qlora_status run_pair(bool dx, const qlora_weight* w, const uint16_t* A, int64_t
     p.sk_count = gcount;
     // output written by TMA: 128-row x 64-column boxes, 128-byte swizzle
     if (!make_tmap_2d(&pp.Y, out, TmapType::BF16, Ndim, M, Ndim * 2, 64, 128, true)) return QLORA_ERR_CUDA;
-    if (t_out) {
-      // T tiles: B = L1 [in x r] as MN-major 64 x 64 chunks; T [M x r] stored in 128 x 64 boxes
-      if (!make_tmap_2d(&pp.L1, L1, TmapType::BF16, r, h, int64_t(r) * 2, 64, 64, true)) return QLORA_ERR_CUDA;
-      if (!make_tmap_2d(&pp.Tout, t_out, TmapType::BF16, r, M, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
+    if (aux_out) {
       p.aux_tiles = p.tiles_m;
       p.t_chunks = (r + 63) / 64;
       p.t_flags = gcount + kPair2CounterInts;
+      const int t_n = p.t_chunks <= 2 ? 128 : 256;   // the aux tiles' MMA width (as the kernel)
+      if (!dx) {
+        // T tiles: B = L1 [in x r] as MN-major 64 x 64 chunks
+        if (!make_tmap_2d(&pp.L1, aux_b, TmapType::BF16, r, h, int64_t(r) * 2, 64, 64, true)) return QLORA_ERR_CUDA;
+      } else {
+        // U tiles: B = L2 [r x out] K-major, one box of t_n / 2 rows per CTA
+        if (!make_tmap_2d(&pp.L1, aux_b, TmapType::BF16, o_, r, o_ * 2, 64, t_n / 2, true)) return QLORA_ERR_CUDA;
+        if (!aux_out2) return QLORA_ERR_CUDA;
+        if (!make_tmap_2d(&pp.Tout2, aux_out2, TmapType::BF16, r, M, int64_t(r) * 2, 64, 128, true))
+          return QLORA_ERR_CUDA;
+        p.aux_dual = 1;
+        p.aux_scale = aux_scale;
+      }
+      // T or U [M x r] stored in 128 x 64 boxes
+      if (!make_tmap_2d(&pp.Tout, aux_out, TmapType::BF16, r, M, int64_t(r) * 2, 64, 128, true)) return QLORA_ERR_CUDA;
     }
   }
   record_prof(g_prof[dx ? 2 : 0], s);
@@ -817,6 +841,11 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const ui
                                                            int(o_ / 64) + (r + 63) / 64)
                                          : pair_spare_sms(true, int((M + 255) / 256) * int(h / 256));
   const bool beside_gemm = ss && dX && pair && forced != 2 && (forced == 1 || spare >= 16);
+  // With every pair busy in the dX GEMM, U = dY L2^T (and s.U) is computed inside it
+  // (its U tiles, before the output tiles' LoRA steps read s.U), and dL1 and dL2 follow
+  // side by side on the two streams.
+  const bool fuse_u = !beside_gemm && ss && dX && pair && forced == 0 && gemm_engine() == 2 && fused_u_enabled() &&
+                      (M + 511) / 512 <= kPair2MaxTBlocks;
   float* gpart = reinterpret_cast<float*>(ws + L.gpart);
   int* gcount = reinterpret_cast<int*>(ws + kStatusBytes + kCounterBytes);
   cudaStream_t aux = s;
@@ -833,6 +862,14 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const ui
   if (dX && !w->is_bf16)
     QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
                                  scales_t, aux));
+  if (fuse_u) {
+    QLB_TRY(join_from(ss, s, aux));    // the GEMM reads the expanded scales
+    QLB_TRY(run_pair(true, w, dY, M, sU, L1, r, scales_t, dX, status, gpart, gcount, s, L2, U, sU, scale));
+    QLB_TRY(handoff_to(ss, s, aux));   // dL2 (T, dY) beside dL1 (X, U), after the GEMM
+    QLB_TRY(run_thin(t2, part_b, counters2, dL2, 2, scale, status, aux));
+    QLB_TRY(run_thin(t1, part, counters, dL1, 1, scale, status, s));
+    return join_from(ss, s, aux);
+  }
   if (beside_gemm) {
     QLB_TRY(run_thin(tu, part, counters, U, 3, scale, status, s, sU));
     QLB_TRY(handoff_to(ss, s, aux));   // the GEMM needs s.U

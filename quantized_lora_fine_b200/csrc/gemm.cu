@@ -835,7 +835,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     tc_gemm_nf4_pair2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAx,
                              const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmY,
                              const __grid_constant__ CUtensorMap tmL1, const __grid_constant__ CUtensorMap tmT,
-                             const GemmParams p) {
+                             const __grid_constant__ CUtensorMap tmT2, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t smem_base = smem_u32(smem);
@@ -946,8 +946,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     if (rank == 0 && lane == 0) {
       constexpr uint32_t idesc_main = make_idesc_bf16(256, 256, 0, C::B_MN ? 1 : 0);
       constexpr uint32_t idesc_ext = make_idesc_bf16(256, 256, 0, 0);   // LoRA B is [N x r], K-major
-      // T tiles: L1 [K x r], MN-major, N = t_n
-      const uint32_t idesc_t = t_n == 128 ? make_idesc_bf16(256, 128, 0, 1) : make_idesc_bf16(256, 256, 0, 1);
+      // aux tiles, N = t_n: forward T tiles read L1 [K x r] (MN-major), dX U tiles L2
+      // [r x K] (K-major)
+      constexpr uint32_t t_bmn = C::B_MN ? 0u : 1u;
+      const uint32_t idesc_t = t_n == 128 ? make_idesc_bf16(256, 128, 0, t_bmn) : make_idesc_bf16(256, 256, 0, t_bmn);
+      constexpr uint32_t b_adv_t = C::B_MN ? (32u >> 4) : (2048u >> 4);
       constexpr uint32_t b_adv = C::B_MN ? (2048u >> 4) : (32u >> 4);
       constexpr uint32_t b_adv_ext = 32u >> 4;
       const uint64_t da_base = make_smem_desc(slot(0), 16u, 1024u, kSwizzle128B);
@@ -973,9 +976,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         tc_fence_after();
         const bool ext = k >= p.num_k_main;
         const uint64_t ad = da_base + si * kSlotAdv, bd = db_base + si * kSlotAdv;
-        // a T tile's B (L1 as stored) is MN-major in every step
+        // an aux tile's B is the same operand in every step
         const bool ttile = tile < p.aux_tiles;
-        const uint32_t badv = ttile ? (2048u >> 4) : ext ? b_adv_ext : b_adv;
+        const uint32_t badv = ttile ? b_adv_t : ext ? b_adv_ext : b_adv;
         const uint32_t idesc = ttile ? idesc_t : ext ? idesc_ext : idesc_main;
 #pragma unroll
         for (uint32_t kk = 0; kk < 4; ++kk)
@@ -1078,8 +1081,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         tc_fence_after();
         const int y = mb * 512 + h * 256 + int(rank) * 128;   // first output row of this store box
 #pragma unroll 1
-        for (int c = 0; c < nchunks; ++c, ++chunk) {
-          const uint32_t buf = chunk % uint32_t(C::kNumStage);
+        for (int c = 0; c < nchunks; ++c) {
           uint32_t v[64];
           tmem_ld_32x32b_x32(tl + uint32_t(h) * 256u + uint32_t(c) * 64u, *reinterpret_cast<uint32_t(*)[32]>(v));
           tmem_ld_32x32b_x32(tl + uint32_t(h) * 256u + uint32_t(c) * 64u + 32u,
@@ -1098,28 +1100,42 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             for (int j = 0; j < 64; ++j)
               v[j] = __float_as_uint(__uint_as_float(v[j]) + __ldcg(src + size_t(j) * 128));
           }
-          // the store that used this staging buffer kNumStage chunks ago must have read it
-          if (leader) bulk_wait_group_read<C::kNumStage - 1>();
-          named_bar_sync(1, C::kEpiThreads);
-          const uint32_t sbase = stage0 + buf * C::kStageBytes + row * 128u;
-          const uint32_t sw = row & 7u;
+          // a U tile writes the chunk twice: U, then bf16(aux_scale * bf16(U))
+          const int npass = (ttile && p.aux_dual) ? 2 : 1;
+#pragma unroll 1
+          for (int pass = 0; pass < npass; ++pass) {
+            const uint32_t buf = chunk++ % uint32_t(C::kNumStage);
+            // the store that used this staging buffer kNumStage uses ago must have read it
+            if (leader) bulk_wait_group_read<C::kNumStage - 1>();
+            named_bar_sync(1, C::kEpiThreads);
+            const uint32_t sbase = stage0 + buf * C::kStageBytes + row * 128u;
+            const uint32_t sw = row & 7u;
+            auto pk = [&](uint32_t x0, uint32_t x1) {
+              const uint32_t a = pack_bf16x2(__uint_as_float(x0), __uint_as_float(x1));
+              if (pass == 0) return a;
+              return pack_bf16x2(__fmul_rn(__uint_as_float(a << 16), p.aux_scale),
+                                 __fmul_rn(__uint_as_float(a & 0xFFFF0000u), p.aux_scale));
+            };
 #pragma unroll
-          for (uint32_t j = 0; j < 8; ++j) {
-            const uint32_t a0 = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
-            const uint32_t a1 = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
-            const uint32_t a2 = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
-            const uint32_t a3 = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + ((j ^ sw) << 4)), "r"(a0),
-                         "r"(a1), "r"(a2), "r"(a3)
-                         : "memory");
+            for (uint32_t j = 0; j < 8; ++j) {
+              const uint32_t a0 = pk(v[8 * j + 0], v[8 * j + 1]);
+              const uint32_t a1 = pk(v[8 * j + 2], v[8 * j + 3]);
+              const uint32_t a2 = pk(v[8 * j + 4], v[8 * j + 5]);
+              const uint32_t a3 = pk(v[8 * j + 6], v[8 * j + 7]);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + ((j ^ sw) << 4)), "r"(a0),
+                           "r"(a1), "r"(a2), "r"(a3)
+                           : "memory");
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, C::kEpiThreads);
+            if (leader && y < p.M) {   // rows past M are clipped by the store; a box wholly past M is skipped
+              const uint32_t sb = stage0 + buf * C::kStageBytes;
+              if (!ttile) tma_store_2d(&tmY, sb, nb * 256 + c * 64, y);
+              else if (pass == 0) tma_store_2d(&tmT, sb, c * 64, y);   // columns past r clipped
+              else tma_store_2d(&tmT2, sb, c * 64, y);
+            }
+            if (leader) bulk_commit_group();
           }
-          fence_proxy_async_smem();
-          named_bar_sync(1, C::kEpiThreads);
-          if (leader && y < p.M) {   // rows past M are clipped by the store; a box wholly past M is skipped
-            if (ttile) tma_store_2d(&tmT, stage0 + buf * C::kStageBytes, c * 64, y);   // columns past r clipped
-            else tma_store_2d(&tmY, stage0 + buf * C::kStageBytes, nb * 256 + c * 64, y);
-          }
-          if (leader) bulk_commit_group();
         }
       }
       if (extra > 0 && leader) {
@@ -1165,12 +1181,20 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           // T tile: this CTA's B half is L1 rows 64 k.. (zeros past the K extent), columns
           // (t_n / 2) rank .. + t_n / 2 - 1 (zeros past r), as MN-major 64-column chunks by
           // TMA; the even A producer posted its bytes
+          // (a U tile: L2 rows (t_n / 2) rank .. + t_n / 2 - 1, K columns 64 k.., one
+          // K-major box)
           const uint32_t bar = rank == 0 ? ready(own) : ready_even;
           if (sub == 0) {
-            for (int c = 0; c < t_n / 128; ++c) {
-              const int x = int(rank) * (t_n / 2) + 64 * c;
-              if (rank == 0) tma_load_2d(b_tile + c * 8192, &tmL1, bar, x, k * 64);
-              else tma_load_2d_pair(b_tile + c * 8192, &tmL1, bar, x, k * 64);
+            if constexpr (!C::B_MN) {
+              for (int c = 0; c < t_n / 128; ++c) {
+                const int x = int(rank) * (t_n / 2) + 64 * c;
+                if (rank == 0) tma_load_2d(b_tile + c * 8192, &tmL1, bar, x, k * 64);
+                else tma_load_2d_pair(b_tile + c * 8192, &tmL1, bar, x, k * 64);
+              }
+            } else {
+              const int y = int(rank) * (t_n / 2);
+              if (rank == 0) tma_load_2d(b_tile, &tmL1, bar, k * 64, y);
+              else tma_load_2d_pair(b_tile, &tmL1, bar, k * 64, y);
             }
           }
           if (rank == 0) mbar_arrive(ready(own));
@@ -1470,7 +1494,8 @@ static qlora_status launch_pair2_cfg(const GemmOperands& o, GemmParams p, cudaSt
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 2 : 1;
-  if (cudaLaunchKernelEx(&cfg, tc_gemm_nf4_pair2_kernel<C>, o.A, o.Ax, o.Bx, o.Y, o.L1, o.Tout, p) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, tc_gemm_nf4_pair2_kernel<C>, o.A, o.Ax, o.Bx, o.Y, o.L1, o.Tout, o.Tout2, p) !=
+      cudaSuccess)
     return QLORA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }

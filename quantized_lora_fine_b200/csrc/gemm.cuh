@@ -54,12 +54,17 @@ struct GemmParams {
   // chunks) before raising the block's flag in t_flags; a main tile's first LoRA step
   // waits (bounded) for its block's flag. t_flags holds [flag, readers] per block and
   // CTA rank, left at zero (the last reader clears them). aux_tiles = 0: no T tiles.
+  // The dX kernel's aux tiles are "U tiles" the same way: U = dY L2^T of the block
+  // (A = the dY rows, B = L2 [r x out] read K-major), stored as U and, with aux_dual,
+  // also as bf16(aux_scale * bf16(U)) to the second aux output (the LoRA step's A).
   int aux_tiles, t_chunks;
   int* t_flags;
+  int aux_dual;
+  float aux_scale;
 };
 
 struct GemmOperands {
-  CUtensorMap A, B, codes, scales, Ax, Bx, Y, L1, Tout;
+  CUtensorMap A, B, codes, scales, Ax, Bx, Y, L1, Tout, Tout2;
 };
 
 enum class GemmKind {

@@ -235,6 +235,33 @@ def test_fused_t_tiles(cuda_device, monkeypatch, M, r, pairs):
     assert_close(f64_of_bf16(Yf), f64_of_bf16(Yu), "Y fused vs separate T")
 
 
+@pytest.mark.parametrize("M,r,pairs", [(1300, 16, None), (1300, 72, None), (600, 256, None), (2048, 64, None),
+                                       (1300, 16, 3), (2048, 128, 5)])
+def test_fused_u_tiles(cuda_device, monkeypatch, M, r, pairs):
+    """The dX GEMM computes U = dY L2^T itself: one extra tile per 512-row block (A =
+    the dY rows, B = L2 read K-major) that stores U and s.U, whose rows the output
+    tiles' LoRA step waits for; dL1 and dL2 run after it. Gradients are within the
+    oracle's tolerance, dL2 (which does not read U) has the same bits as with U as
+    its own pass, and dX and dL1 agree with that path within one bf16 rounding of U."""
+    if pairs is not None:
+        monkeypatch.setenv("QLORA_B200_MAX_PAIRS", str(pairs))
+    c = dataclasses.replace(synth.case_small(), M=M, out=768, inp=512, r=r, alpha=2.0 * r, double_quant=True)
+    monkeypatch.delenv("QLORA_B200_FUSED_U", raising=False)
+    monkeypatch.delenv("QLORA_B200_BWD", raising=False)
+    run_and_compare(c)
+    d = c.make()
+    g, w = gpu_case(d, c.double_quant, False)
+    _, T = api.linear_fwd(w, g["X"], g["L1"], g["L2"], c.scale)
+    fused = api.linear_bwd(w, g["X"], g["dY"], g["L1"], g["L2"], c.scale, T=T)
+    monkeypatch.setenv("QLORA_B200_FUSED_U", "0")
+    sep = api.linear_bwd(w, g["X"], g["dY"], g["L1"], g["L2"], c.scale, T=T)
+    torch.cuda.synchronize()
+    assert api.status() == 0
+    assert torch.equal(fused[2], sep[2]), "dL2 does not read U"
+    assert_close(f64_of_bf16(fused[0]), f64_of_bf16(sep[0]), "dX fused vs separate U")
+    assert_close(fused[1].double().cpu().numpy(), sep[1].double().cpu().numpy(), "dL1 fused vs separate U")
+
+
 @pytest.mark.parametrize("schedule", ["beside", "serial"])
 def test_backward_schedules_give_the_same_bits(cuda_device, monkeypatch, schedule):
     """Both backward schedules (dX beside dL1 / dL2, or dL2 beside U and dL1 before
@@ -243,6 +270,7 @@ def test_backward_schedules_give_the_same_bits(cuda_device, monkeypatch, schedul
     case = dataclasses.replace(synth.case_q_proj(seed=3, M=1024), double_quant=True)
     monkeypatch.delenv("QLORA_B200_BWD", raising=False)
     ref = run_and_compare(case, rows=np.arange(0, case.M, 97))
+    monkeypatch.setenv("QLORA_B200_FUSED_U", "0")   # U as its own pass in every schedule
     d = case.make()
     g, w = gpu_case(d, case.double_quant, False)
     Y, T = api.linear_fwd(w, g["X"], g["L1"], g["L2"], case.scale)
