@@ -252,10 +252,17 @@ bool fused_t_enabled() {
   const char* e = std::getenv("QLORA_B200_FUSED_T");
   return !(e && std::strcmp(e, "0") == 0);
 }
-// U = dY L2^T inside the dX GEMM unless QLORA_B200_FUSED_U=0 (read on every call).
-bool fused_u_enabled() {
+// U = dY L2^T inside the dX GEMM: QLORA_B200_FUSED_U=1 always, =0 never, unset when
+// the output has at least 32 column tiles of 256 (read on every call). A U tile
+// takes a whole tile's turn in the schedule but does about half its MMA work, so it
+// pays where its share of the tiles is small: on q_proj (16 column tiles) the dX
+// GEMM took 233.5 us with U tiles against 218.8 us, and the backward 280.6 us
+// against 277.1 us with U as its own pass.
+bool fused_u_wanted(int64_t n_cols) {
   const char* e = std::getenv("QLORA_B200_FUSED_U");
-  return !(e && std::strcmp(e, "0") == 0);
+  if (e && std::strcmp(e, "0") == 0) return false;
+  if (e && std::strcmp(e, "1") == 0) return true;
+  return n_cols / 256 >= 32;
 }
 
 // Fused NF4 GEMM on CTA pairs (256 x 256 tiles): out = A . W' + Ax . Bx^T, where
@@ -707,8 +714,14 @@ qlora_status linear_fwd_impl(const qlora_weight* w, const uint16_t* X, int64_t M
   float* part = reinterpret_cast<float*>(ws + L.part);
   const int64_t h = w->in, o_ = w->out;
   int* counters = reinterpret_cast<int*>(ws + L.counters);
-  // T = X L1 : A = X (K-major), B = L1 as [h x r] (MN-major for B); the scale
-  // expansion and s.L2^T are independent of it and run beside it
+  // T = X L1 inside the NF4 GEMM (its T tiles read X while it is in L2), unless T is
+  // given, the weight is protected, another engine runs, or M has too many row blocks
+  const bool fuse_t = !T_in && !w->is_bf16 && gemm_engine() == 2 && fused_t_enabled() &&
+                      (M + 511) / 512 <= kPair2MaxTBlocks;
+  const bool thin_t = !T_in && !fuse_t;
+  // The scale expansion and s.L2^T are independent of T and of each other: the
+  // expansion runs on the side stream, s.L2^T beside it on this stream, or beside T
+  // when T = X L1 runs here as its own pass (A = X K-major, B = L1 [h x r] MN-major)
   std::lock_guard<std::mutex> lock(g_side_mu);
   SideStream* ss = side_stream();
   cudaStream_t aux = s;
@@ -719,14 +732,10 @@ qlora_status linear_fwd_impl(const qlora_weight* w, const uint16_t* X, int64_t M
   if (!w->is_bf16)
     QLB_TRY(launch_expand_scales(w->codes, w->absmax, w->absmax_q, w->absmax2, w->q.double_quant != 0, o_, h,
                                  scales_t, aux));
-  QLB_TRY(launch_scale_lora(L2, r, o_, scale, /*transpose=*/true, l2t, aux));
+  QLB_TRY(launch_scale_lora(L2, r, o_, scale, /*transpose=*/true, l2t, thin_t ? aux : s));
   const uint16_t* T = T_in;
-  // T = X L1 inside the NF4 GEMM (its T tiles read X while it is in L2), unless T is
-  // given, the weight is protected, another engine runs, or M has too many row blocks
-  const bool fuse_t = !T_in && !w->is_bf16 && gemm_engine() == 2 && fused_t_enabled() &&
-                      (M + 511) / 512 <= kPair2MaxTBlocks;
   uint16_t* Tw = T_save ? T_save : reinterpret_cast<uint16_t*>(ws + L.t);
-  if (!T && !fuse_t) {
+  if (thin_t) {
     Thin tt{GemmKind::ThinKM, X, h, M, L1, r, h, M, h / 64, r};
     QLB_TRY(run_thin(tt, part, counters, Tw, 0, 1.f, status, s));
     T = Tw;
@@ -844,7 +853,7 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const ui
   // With every pair busy in the dX GEMM, U = dY L2^T (and s.U) is computed inside it
   // (its U tiles, before the output tiles' LoRA steps read s.U), and dL1 and dL2 follow
   // side by side on the two streams.
-  const bool fuse_u = !beside_gemm && ss && dX && pair && forced == 0 && gemm_engine() == 2 && fused_u_enabled() &&
+  const bool fuse_u = !beside_gemm && ss && dX && pair && forced == 0 && gemm_engine() == 2 && fused_u_wanted(h) &&
                       (M + 511) / 512 <= kPair2MaxTBlocks;
   float* gpart = reinterpret_cast<float*>(ws + L.gpart);
   int* gcount = reinterpret_cast<int*>(ws + kStatusBytes + kCounterBytes);

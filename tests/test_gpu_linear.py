@@ -238,15 +238,17 @@ def test_fused_t_tiles(cuda_device, monkeypatch, M, r, pairs):
 @pytest.mark.parametrize("M,r,pairs", [(1300, 16, None), (1300, 72, None), (600, 256, None), (2048, 64, None),
                                        (1300, 16, 3), (2048, 128, 5)])
 def test_fused_u_tiles(cuda_device, monkeypatch, M, r, pairs):
-    """The dX GEMM computes U = dY L2^T itself: one extra tile per 512-row block (A =
-    the dY rows, B = L2 read K-major) that stores U and s.U, whose rows the output
-    tiles' LoRA step waits for; dL1 and dL2 run after it. Gradients are within the
+    """The dX GEMM computes U = dY L2^T itself (forced on: by default only for outputs
+    of at least 32 column tiles, as the full-size MLP down and 14B down cases are):
+    one extra tile per 512-row block (A = the dY rows, B = L2 read K-major) that
+    stores U and s.U, whose rows the output tiles' LoRA step waits for; dL1 and dL2
+    run after it. Gradients are within the
     oracle's tolerance, dL2 (which does not read U) has the same bits as with U as
     its own pass, and dX and dL1 agree with that path within one bf16 rounding of U."""
     if pairs is not None:
         monkeypatch.setenv("QLORA_B200_MAX_PAIRS", str(pairs))
     c = dataclasses.replace(synth.case_small(), M=M, out=768, inp=512, r=r, alpha=2.0 * r, double_quant=True)
-    monkeypatch.delenv("QLORA_B200_FUSED_U", raising=False)
+    monkeypatch.setenv("QLORA_B200_FUSED_U", "1")   # by default only outputs of >= 32 column tiles
     monkeypatch.delenv("QLORA_B200_BWD", raising=False)
     run_and_compare(c)
     d = c.make()
