@@ -203,8 +203,9 @@ def pair_gemm_traffic(name: str):
 def mlp_leg(api, synth, torch, dev, peaks, reps: int = 5):
     """The Llama-7B MLP at M = 8192 (gate and up 4096 -> 11008, down 11008 -> 4096;
     NF4 blocks of 64 without double quant; r = 64, alpha = 128): fwd+bwd of the three
-    linears, weights quantized once outside the timed region, captured in one CUDA
-    graph and replayed (L2 flushed before each replay)."""
+    linears (the one-call forward, T in the GEMM's T tiles), weights quantized once
+    outside the timed region, captured in one CUDA graph and replayed (L2 flushed
+    before each replay)."""
     items = []
     fl = 0.0
     for c in synth.cases_mlp():
@@ -215,8 +216,7 @@ def mlp_leg(api, synth, torch, dev, peaks, reps: int = 5):
 
     def run():
         for c, w, d in items:
-            T = api.lora_down(d["X"], d["L1"])
-            api.linear_fwd(w, d["X"], d["L1"], d["L2"], c.scale, T=T)
+            _, T = api.linear_fwd(w, d["X"], d["L1"], d["L2"], c.scale)   # one call: T in the GEMM's T tiles
             api.linear_bwd(w, d["X"], d["dY"], d["L1"], d["L2"], c.scale, T=T)
 
     run()
@@ -340,8 +340,7 @@ def protect_leg(api, synth, torch, dev, peaks, reps: int = 3, K: int = 8):
 
             def run():
                 ww = api.NF4Weight.protected(api.dequantize_two_stage(w1, w2)) if mode == "two_stage" else w
-                T = api.lora_down(d["X"], d["L1"])
-                api.linear_fwd(ww, d["X"], d["L1"], d["L2"], c.scale, T=T)
+                _, T = api.linear_fwd(ww, d["X"], d["L1"], d["L2"], c.scale)
                 api.linear_bwd(ww, d["X"], d["dY"], d["L1"], d["L2"], c.scale, T=T)
 
             run()
@@ -381,7 +380,8 @@ def protect_leg(api, synth, torch, dev, peaks, reps: int = 3, K: int = 8):
     with_k2 = all_nf4 + sum(shapes[kind_of[m.name]]["two_stage_ms"] - shapes[kind_of[m.name]]["nf4_ms"] for m in kept)
     return {"workload": "14B-stack linears (hidden 5120, intermediate 13824), M = 16384, r = 16, alpha = 32, "
                         "NF4 with double quant vs the same weight kept in bf16 vs two NF4 stages (reconstructed "
-                        "to bf16 once per step); fwd+bwd = T, forward, backward",
+                        "to bf16 once per step); fwd+bwd = the one-call forward (T in the NF4 GEMM's T tiles; "
+                        "a bf16 layer computes T as its own pass) and the backward",
             "per_shape": shapes,
             "stack": {"matrices": len(mats), "K": K,
                       "kept": [f"layer {m.layer} {m.name}" for m in kept],
@@ -438,8 +438,7 @@ def linear_set_leg(api, synth, torch, dev, peaks, ranks=(16, 32, 64, 128), K: in
         def run(setting):
             for i, m in enumerate(mats):
                 w = weights[i] if (setting != "qlora" and keep[i]) else nf4[i]
-                T = api.lora_down(X[m.inp], L1[m.inp])
-                api.linear_fwd(w, X[m.inp], L1[m.inp], L2[m.out], s, Y=Y[m.out], T=T)
+                _, T = api.linear_fwd(w, X[m.inp], L1[m.inp], L2[m.out], s, Y=Y[m.out])
                 if setting == "protect_top" and m.layer < cut:
                     continue                        # no adapter below the cut: no backward
                 early = setting == "protect_top" and m.layer == cut
