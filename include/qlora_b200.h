@@ -274,7 +274,11 @@ size_t qlora_bwd_workspace_size(int64_t M, int64_t out, int64_t in, int32_t r);
  *   T_save  device out, bf16 [M x r] (T, unscaled), or NULL to keep it in the
  *           workspace only.
  * The NF4 weight is dequantized tile by tile inside the GEMM; no dequantized
- * copy of W is written to memory. */
+ * copy of W is written to memory. With an NF4 weight (and M <= 110592) T is
+ * computed inside the same GEMM, in one leading tile per 512 rows of X whose rows
+ * the LoRA step of the output tiles waits for (QLORA_B200_FUSED_T=0: as its own
+ * pass); a protected weight computes T as its own pass. The two ways sum the fp32
+ * products in different orders, so T may differ in the last bf16 bit. */
 qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t M,
                               const uint16_t* L1, const uint16_t* L2, int32_t r, float scale,
                               uint16_t* Y, uint16_t* T_save,
