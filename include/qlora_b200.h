@@ -296,7 +296,8 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const uint16_t* X, int64_t 
  *   qlora_linear_fwd_t Y = X W_s^T + s T L2 with T supplied (device bf16 [M x r],
  *                      from qlora_lora_down or the caller); otherwise as
  *                      qlora_linear_fwd (same workspace size). Gives the bits of
- *                      qlora_linear_fwd when T is the same. */
+ *                      qlora_linear_fwd when T is the same (as it is when that
+ *                      call computes T as its own pass). */
 size_t qlora_lora_down_workspace_size(int64_t M, int64_t in, int32_t r);
 qlora_status qlora_lora_down(const uint16_t* X, int64_t M, int64_t in, const uint16_t* L1, int32_t r,
                              uint16_t* T, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
@@ -312,7 +313,11 @@ qlora_status qlora_linear_fwd_t(const qlora_weight* w, const uint16_t* X, int64_
  *   T_saved  device bf16 [M x r] from the forward, or NULL to recompute T = X L1.
  * dX == NULL expresses an early backward stop below the lowest adapted layer
  * (AQLoRA section 3.3). dL1/dL2 are overwritten, not accumulated. Their
- * reductions run in a fixed order, so repeated calls give identical bits. */
+ * reductions run in a fixed order, so repeated calls give identical bits. With an
+ * NF4 weight, U (and s U, the dX LoRA step's operand) can be computed inside the
+ * dX GEMM, in one leading tile per 512 rows of dY: by default when in >= 8192 (32
+ * column tiles of the output), QLORA_B200_FUSED_U=1 always, =0 never; U may then
+ * differ in the last bf16 bit from U as its own pass, and dX and dL1 with it. */
 qlora_status qlora_linear_bwd(const qlora_weight* w, const uint16_t* X, const uint16_t* dY, int64_t M,
                               const uint16_t* L1, const uint16_t* L2, int32_t r, float scale,
                               const uint16_t* T_saved, uint16_t* dX, float* dL1, float* dL2,
