@@ -252,3 +252,12 @@ def test_workspace_sizes_reserve_the_counter_region(lib):
     assert lib.nf4_layer_error_rank_workspace_size(2, nn) >= reserved + 2 * (n // 16384) * 16
     # the quantizer keeps only the status word and no scratch
     assert lib.nf4_quantize_workspace_size(n) == 256
+
+
+def test_workspace_reset_argument_checks(lib):
+    """qlora_reset_workspace (status word, split-K counters and the forward GEMM's
+    block flags) refuses a missing or too-small workspace on the host; no device
+    work is queued then."""
+    assert lib.qlora_reset_workspace(None, 1 << 20, None) == 7     # QLORA_ERR_WORKSPACE
+    buf = ctypes.create_string_buffer(64)
+    assert lib.qlora_reset_workspace(ctypes.cast(buf, ctypes.c_void_p), 64, None) == 7
