@@ -541,7 +541,8 @@ def summary_of(line):
                 return None
             v = v[k]
         return round(v, 4) if isinstance(v, float) else v
-    out = {"step_TFLOP/s": g("value"), "fwd_bwd_TFLOP/s": g("legs", "fwd_bwd", "TFLOP/s"),
+    out = {"step_TFLOP/s": g("value"), "e2e_TFLOP/s": g("e2e", "value"),
+           "fwd_bwd_TFLOP/s": g("legs", "fwd_bwd", "TFLOP/s"),
            "fwd_bwd_frac_of_burst": g("legs", "fwd_bwd", "frac_of_burst"),
            "fwd_gemm_TFLOP/s": g("legs", "fwd_gemm", "TFLOP/s"), "dx_gemm_TFLOP/s": g("legs", "dx_gemm", "TFLOP/s"),
            "mlp_TFLOP/s": g("mlp", "TFLOP/s"), "mlp_frac_of_burst": g("mlp", "frac_of_burst")}
@@ -789,11 +790,13 @@ def gpu_main(args):
 
     # ------------------------------------------------ end to end with host buffers
     # Every step copies its inputs (W, X, dY, L1, L2) from pinned host memory and its
-    # results (Y, dX, dL1, dL2) back to pinned host memory. The steps are pipelined
-    # on three streams: the host-to-device copies of step k + 1 (into the second of
-    # two device input sets) and the device-to-host copies of step k - 1 run while
-    # step k computes; the timed region spans all steps, from the first input copy
-    # to the last result copy.
+    # result, the adapter gradients dL1 and dL2, back to pinned host memory (Y and dX
+    # are what the neighbouring layers consume on the device; a second run also
+    # copies them back and is reported beside). The steps are pipelined on three
+    # streams: the host-to-device copies of step k + 1 (into the second of two device
+    # input sets) and the device-to-host copies of step k - 1 run while step k
+    # computes; the timed region spans all steps, from the first input copy to the
+    # last result copy.
     e2e = None
     if args.e2e_steps > 0:
         pin = {k: v.cpu().pin_memory() for k, v in d.items()}
@@ -802,12 +805,14 @@ def gpu_main(args):
                  "dL1": torch.empty((h, r), dtype=torch.float32).pin_memory(),
                  "dL2": torch.empty((r, o), dtype=torch.float32).pin_memory()} for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in pin.values())
-        d2h = sum(t.numel() * t.element_size() for t in outs[0].values())
+        result_names = ("dL1", "dL2")
+        d2h = sum(outs[0][k].numel() * outs[0][k].element_size() for k in result_names)
+        d2h_all = sum(t.numel() * t.element_size() for t in outs[0].values())
         dev_in = [{k: torch.empty_like(v, device=dev) for k, v in pin.items()} for _ in range(2)]
         s_in = torch.cuda.Stream(device=dev)
         s_out = torch.cuda.Stream(device=dev)
 
-        def pipeline(n_steps):
+        def pipeline(n_steps, names):
             ready = [torch.cuda.Event() for _ in range(n_steps)]
             done = [torch.cuda.Event() for _ in range(n_steps)]
             copied = [torch.cuda.Event() for _ in range(n_steps)]
@@ -831,28 +836,38 @@ def gpu_main(args):
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(done[k])
                     for name, t in zip(("Y", "dX", "dL1", "dL2"), res):
+                        if name not in names:
+                            continue
                         t.record_stream(s_out)
                         outs[k % 2][name].copy_(t, non_blocking=True)
                     copied[k].record(s_out)
             stream.wait_event(copied[n_steps - 1])
 
-        pipeline(3)   # warm-up
-        torch.cuda.synchronize()
-        flush.zero_()
-        s_in.wait_stream(stream)
-        ev[0].record(stream)
-        s_in.wait_event(ev[0])
-        pipeline(args.e2e_steps)
-        ev[1].record(stream)
-        ev[1].synchronize()
-        em = ev[0].elapsed_time(ev[1]) / args.e2e_steps
-        assert api.status() == 0, "device status set in the end-to-end run"
-        if world > 1:
-            t = torch.tensor([em], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            em = float(t.item())
+        def timed(names):
+            pipeline(3, names)   # warm-up
+            torch.cuda.synchronize()
+            flush.zero_()
+            s_in.wait_stream(stream)
+            ev[0].record(stream)
+            s_in.wait_event(ev[0])
+            pipeline(args.e2e_steps, names)
+            ev[1].record(stream)
+            ev[1].synchronize()
+            em = ev[0].elapsed_time(ev[1]) / args.e2e_steps
+            assert api.status() == 0, "device status set in the end-to-end run"
+            if world > 1:
+                t = torch.tensor([em], dtype=torch.float64, device=dev)
+                dist.all_reduce(t, op=dist.ReduceOp.MAX)
+                em = float(t.item())
+            return em
+
+        em = timed(result_names)
+        em_all = timed(("Y", "dX", "dL1", "dL2"))
         e2e = {"value": fl * world / (em * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": em,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "result": "dL1, dL2 (the adapter gradients)",
+               "with_Y_dX_back": {"ms_per_step": em_all, "TFLOP/s": fl * world / (em_all * 1e-3) / 1e12,
+                                  "d2h_bytes_per_step": d2h_all},
                "timing": f"{args.e2e_steps} steps pipelined over three streams (input copies of the next step and "
                          "result copies of the previous one beside each step), one event pair around all of them"}
 
