@@ -11,6 +11,7 @@
 // launch: each waits for its predecessor's memory before reading it.
 #include <cfloat>
 #include <cstdlib>
+#include <cstring>
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -90,10 +91,13 @@ struct ChunkRef {
 // back in order and out in two 16-byte stores, with the scales. Warp 0 sums the
 // 256 per-thread totals in a fixed order into partial[chunk]; the other warps
 // leave as soon as their totals are in shared memory.
-template <bool DQ, class Tab>
-__global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_constant__ Tab tab,
-                                                                   double2* __restrict__ partial, int* status,
-                                                                   uint64_t copy_wait_ns) {
+// With RELOAD the thread reads its pieces from shared memory twice (once for the
+// absmax, once in the element loop) instead of holding all eight in registers, so
+// six CTAs fit an SM instead of four.
+template <bool DQ, class Tab, bool RELOAD = false>
+__global__ void __launch_bounds__(256, RELOAD ? 6 : 4) layer_error_chunk_kernel(const __grid_constant__ Tab tab,
+                                                                                double2* __restrict__ partial,
+                                                                                int* status, uint64_t copy_wait_ns) {
   constexpr bool kW = Tab::kWrite;
   __shared__ __align__(128) uint32_t s_w[kChunkBytes / 4];
   __shared__ double2 s_part[256];
@@ -139,18 +143,31 @@ __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_
   }
   const bool valid = tid < nblk;
   const uint32_t rot = uint32_t(tid & 7);
-  uint32_t u[8][4];
-  if (valid) {
-    const uint32_t src = smem_u32(s_w) + uint32_t(tid) * 128u + rot * 16u;
+  const uint32_t src = smem_u32(s_w) + uint32_t(tid) * 128u + rot * 16u;
+  uint32_t u[RELOAD ? 1 : 8][4];
+  uint32_t m = 0u;
+  if constexpr (RELOAD) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) lds_u4(src ^ (uint32_t(j) << 4), u[j]);
+    for (int j = 0; j < 8; ++j) {
+      uint32_t v[4] = {0u, 0u, 0u, 0u};
+      if (valid) lds_u4(src ^ (uint32_t(j) << 4), v);
+      m = bf16x2_maxabs(m, v[0]);
+      m = bf16x2_maxabs(m, v[1]);
+      m = bf16x2_maxabs(m, v[2]);
+      m = bf16x2_maxabs(m, v[3]);
+    }
   } else {
+    if (valid) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+      for (int j = 0; j < 8; ++j) lds_u4(src ^ (uint32_t(j) << 4), u[j]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+    }
+    m = bf16x2_maxabs(u[0][0], u[0][1]);
+#pragma unroll
+    for (int k = 2; k < 32; ++k) m = bf16x2_maxabs(m, u[k >> 2][k & 3]);
   }
-  uint32_t m = bf16x2_maxabs(u[0][0], u[0][1]);
-#pragma unroll
-  for (int k = 2; k < 32; ++k) m = bf16x2_maxabs(m, u[k >> 2][k & 3]);
   m &= 0x7FFF7FFFu;
   const uint32_t amb = max(m >> 16, m & 0xFFFFu);
   const bool bad = amb >= 0x7F80u;
@@ -187,9 +204,11 @@ __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_
   // keeps every quotient finite and adds nothing to the sums; their code words are
   // the zero code.
   const bool live = valid && am > 0.f && !bad;
-  if (bad) {
+  if constexpr (!RELOAD) {
+    if (bad) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+      for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+    }
   }
   const CellScale cs(live ? am : 1.f);
   const uint64_t ah2 = f2_splat(ahat);
@@ -198,9 +217,14 @@ __global__ void __launch_bounds__(256, 4) layer_error_chunk_kernel(const __grid_
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     uint32_t x[8];
+    uint32_t* uj = u[RELOAD ? 0 : j];
+    if constexpr (RELOAD) {
+      uj[0] = uj[1] = uj[2] = uj[3] = 0u;
+      if (valid && !bad) lds_u4(src ^ (uint32_t(j) << 4), u[0]);
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint64_t w = f2_from_bf16x2(u[j][i]);
+      const uint64_t w = f2_from_bf16x2(uj[i]);
       const uint64_t q = f2_mul(w, cs.r2);
       const uint64_t c = cells2(q, cs.cmul2);
       x[2 * i] = index_bits(f2_lo(q), uint32_t(c), cs.M, lt);
@@ -384,6 +408,15 @@ size_t layer_error_ws_bytes(int n_layers, const int64_t* numel) {
   return kReservedBytes + size_t(chunks) * sizeof(double2);
 }
 
+// Chunk kernel variant: six CTAs per SM, each thread reading its pieces twice, unless
+// QLORA_B200_ERR_RELOAD=0 (four CTAs, pieces held in registers; read on every call).
+// On the 224-matrix stack: error pass 3.51 against 3.38 TB/s, fused quantize + error
+// 4.02 against 3.78 TB/s.
+static bool err_reload() {
+  const char* e = std::getenv("QLORA_B200_ERR_RELOAD");
+  return !(e && std::strcmp(e, "0") == 0);
+}
+
 // The three passes on stream s. tab.first_chunk / n_layers are filled in; the chunk
 // and rank kernels need nothing else from the host. With pdl, each kernel may start
 // while its predecessor drains (the allocation-free entry launches plainly).
@@ -400,13 +433,19 @@ static qlora_status launch_passes(const Tab& tab, double2* partial, int* status,
   const unsigned c = unsigned(tab.first_chunk[n]);
   cudaError_t e;
   if (pdl) {
-    e = launch_pdl(layer_error_chunk_kernel<DQ, Tab>, dim3(c), dim3(256), 0, s, tab, partial, status, copy_wait_ns());
+    e = err_reload() ? launch_pdl(layer_error_chunk_kernel<DQ, Tab, true>, dim3(c), dim3(256), 0, s, tab, partial,
+                                  status, copy_wait_ns())
+                     : launch_pdl(layer_error_chunk_kernel<DQ, Tab>, dim3(c), dim3(256), 0, s, tab, partial, status,
+                                  copy_wait_ns());
     if (e == cudaSuccess) e = launch_pdl(layer_error_finish_kernel, dim3(unsigned(n)), dim3(32), 0, s, partial, r, err);
     if (e == cudaSuccess)
       e = budget ? launch_pdl(rank_budget_kernel, dim3(1), dim3(1024), 0, s, err, n, *budget, order, keep, K_out)
                  : launch_pdl(rank_topk_kernel, dim3(1), dim3(1024), 0, s, err, n, K, order, keep);
   } else {
-    layer_error_chunk_kernel<DQ, Tab><<<c, 256, 0, s>>>(tab, partial, status, copy_wait_ns());
+    if (err_reload())
+      layer_error_chunk_kernel<DQ, Tab, true><<<c, 256, 0, s>>>(tab, partial, status, copy_wait_ns());
+    else
+      layer_error_chunk_kernel<DQ, Tab><<<c, 256, 0, s>>>(tab, partial, status, copy_wait_ns());
     layer_error_finish_kernel<<<unsigned(n), 32, 0, s>>>(partial, r, err);
     if (budget)
       rank_budget_kernel<<<1, 1024, 0, s>>>(err, n, *budget, order, keep, K_out);
