@@ -2,6 +2,8 @@
 // the LoRA path. All HBM-bound: 128-bit loads and stores, warp shuffles.
 #include <algorithm>
 #include <cfloat>
+#include <cstdlib>
+#include <cstring>
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -126,8 +128,12 @@ __device__ __forceinline__ QuantOne quant_target(const QuantBatch& t, int64_t ct
   return QuantOne{t.W[lo], t.numel[lo], t.codes[lo], t.absmax[lo], t.absmax_q[lo], t.absmax2[lo]};
 }
 
-template <bool DQ, class Tab>
-__global__ void __launch_bounds__(256, 4) nf4_quantize_bf16_kernel(const __grid_constant__ Tab tab, int* status) {
+// With RELOAD each thread reads its eight pieces from shared memory twice (for the
+// absmax, then for the codes) instead of holding them in registers, so more CTAs fit
+// an SM.
+template <bool DQ, class Tab, bool RELOAD = false>
+__global__ void __launch_bounds__(256, RELOAD ? 6 : 4) nf4_quantize_bf16_kernel(const __grid_constant__ Tab tab,
+                                                                                int* status) {
   __shared__ __align__(128) uint32_t s_w[kChunkBytes / 4];   // the group's bf16 pairs
   __shared__ float s_amax[kDQBlock];
   __shared__ float s_red[8];
@@ -176,18 +182,31 @@ __global__ void __launch_bounds__(256, 4) nf4_quantize_bf16_kernel(const __grid_
   }
   const bool valid = tid < nblk;
   const uint32_t rot = uint32_t(tid & 7);
-  uint32_t u[8][4];
-  if (valid) {
-    const uint32_t src = smem_u32(s_w) + uint32_t(tid) * 128u + rot * 16u;
+  const uint32_t src = smem_u32(s_w) + uint32_t(tid) * 128u + rot * 16u;
+  uint32_t u[RELOAD ? 1 : 8][4];
+  uint32_t m = 0u;
+  if constexpr (RELOAD) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) lds_u4(src ^ (uint32_t(j) << 4), u[j]);
+    for (int j = 0; j < 8; ++j) {
+      uint32_t v[4] = {0u, 0u, 0u, 0u};
+      if (valid) lds_u4(src ^ (uint32_t(j) << 4), v);
+      m = bf16x2_maxabs(m, v[0]);
+      m = bf16x2_maxabs(m, v[1]);
+      m = bf16x2_maxabs(m, v[2]);
+      m = bf16x2_maxabs(m, v[3]);
+    }
   } else {
+    if (valid) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+      for (int j = 0; j < 8; ++j) lds_u4(src ^ (uint32_t(j) << 4), u[j]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+    }
+    m = bf16x2_maxabs(u[0][0], u[0][1]);
+#pragma unroll
+    for (int k = 2; k < 32; ++k) m = bf16x2_maxabs(m, u[k >> 2][k & 3]);
   }
-  uint32_t m = bf16x2_maxabs(u[0][0], u[0][1]);
-#pragma unroll
-  for (int k = 2; k < 32; ++k) m = bf16x2_maxabs(m, u[k >> 2][k & 3]);
   m &= 0x7FFF7FFFu;
   const uint32_t amb = max(m >> 16, m & 0xFFFFu);
   const bool bad = amb >= 0x7F80u;
@@ -201,16 +220,24 @@ __global__ void __launch_bounds__(256, 4) nf4_quantize_bf16_kernel(const __grid_
   // every quotient finite; their code words are the zero code (a non-finite block
   // sets the status word).
   const bool live = am > 0.f && !bad;
-  if (bad) {
+  if constexpr (!RELOAD) {
+    if (bad) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+      for (int j = 0; j < 8; ++j) u[j][0] = u[j][1] = u[j][2] = u[j][3] = 0u;
+    }
   }
   const CellScale cs(live ? am : 1.f);
   uint32_t cw[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     uint32_t x[8];
-    piece_index_bits(u[j], cs, lt, x);
+    if constexpr (RELOAD) {
+      u[0][0] = u[0][1] = u[0][2] = u[0][3] = 0u;
+      if (valid && !bad) lds_u4(src ^ (uint32_t(j) << 4), u[0]);
+      piece_index_bits(u[0], cs, lt, x);
+    } else {
+      piece_index_bits(u[j], cs, lt, x);
+    }
     cw[j] = live ? pack_code_word(x) : 0x77777777u;
   }
   if (valid) {
@@ -289,6 +316,13 @@ __global__ void __launch_bounds__(256) nf4_quantize_f32_kernel(const float* __re
   if constexpr (DQ) dq_group(s_amax, s_red, nb, g, absmax_q, absmax2);
 }
 
+// Quantizer variant: each thread reads its block from shared memory twice (more CTAs
+// per SM), unless QLORA_B200_QUANT_RELOAD=0 (read on every call).
+static bool quant_reload() {
+  const char* e = std::getenv("QLORA_B200_QUANT_RELOAD");
+  return !(e && std::strcmp(e, "0") == 0);
+}
+
 qlora_status launch_quantize(const void* W, int w_dtype, int64_t numel, bool dq, uint8_t* codes, float* absmax,
                              uint8_t* absmax_q, float* absmax2, int* status, cudaStream_t s) {
   const int64_t nb = (numel + kBlock - 1) / kBlock;
@@ -298,8 +332,13 @@ qlora_status launch_quantize(const void* W, int w_dtype, int64_t numel, bool dq,
   if (w_dtype == QLORA_DTYPE_BF16) {
     const uint16_t* Wb = static_cast<const uint16_t*>(W);
     const QuantOne one{Wb, numel, codes, absmax, absmax_q, absmax2};
-    if (dq) launch_pdl(nf4_quantize_bf16_kernel<true, QuantOne>, grid, dim3(256), 0, s, one, status);
-    else launch_pdl(nf4_quantize_bf16_kernel<false, QuantOne>, grid, dim3(256), 0, s, one, status);
+    if (quant_reload()) {
+      if (dq) launch_pdl(nf4_quantize_bf16_kernel<true, QuantOne, true>, grid, dim3(256), 0, s, one, status);
+      else launch_pdl(nf4_quantize_bf16_kernel<false, QuantOne, true>, grid, dim3(256), 0, s, one, status);
+    } else {
+      if (dq) launch_pdl(nf4_quantize_bf16_kernel<true, QuantOne>, grid, dim3(256), 0, s, one, status);
+      else launch_pdl(nf4_quantize_bf16_kernel<false, QuantOne>, grid, dim3(256), 0, s, one, status);
+    }
   } else {
     if (dq) nf4_quantize_f32_kernel<true><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
     else nf4_quantize_f32_kernel<false><<<grid, 256, 0, s>>>((const float*)W, numel, codes, absmax, absmax_q, absmax2, status);
@@ -330,8 +369,12 @@ qlora_status launch_quantize_batch(int n, const uint16_t* const* W, const int64_
   }
   tab.first_group[n] = int32_t(c);
   const dim3 grid(static_cast<unsigned>(c));
-  const cudaError_t e = dq ? launch_pdl(nf4_quantize_bf16_kernel<true, QuantBatch>, grid, dim3(256), 0, s, tab, status)
-                           : launch_pdl(nf4_quantize_bf16_kernel<false, QuantBatch>, grid, dim3(256), 0, s, tab, status);
+  const bool rl = quant_reload();
+  const cudaError_t e =
+      dq ? (rl ? launch_pdl(nf4_quantize_bf16_kernel<true, QuantBatch, true>, grid, dim3(256), 0, s, tab, status)
+               : launch_pdl(nf4_quantize_bf16_kernel<true, QuantBatch>, grid, dim3(256), 0, s, tab, status))
+         : (rl ? launch_pdl(nf4_quantize_bf16_kernel<false, QuantBatch, true>, grid, dim3(256), 0, s, tab, status)
+               : launch_pdl(nf4_quantize_bf16_kernel<false, QuantBatch>, grid, dim3(256), 0, s, tab, status));
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
