@@ -380,6 +380,64 @@ __global__ void __launch_bounds__(32) layer_error_finish_kernel(const double2* _
   finish_layer_warp(partial, r.first_chunk[l], r.first_chunk[l + 1], err + l);
 }
 
+// Passes 2 and 3 in one CTA for a few layers (the allocation pass of one matrix, or
+// of a layer's handful): all 1024 threads sum a layer's chunk partials (thread t
+// takes chunks first + t, first + t + 1024, ...; warps then the 32 warp sums
+// combine by a fixed shuffle pattern, so the result is deterministic for a given
+// layout), then every thread ranks layers as rank_topk_kernel does.
+constexpr int kSmallLayers = 16;
+__global__ void __launch_bounds__(1024) finish_rank_small_kernel(const double2* __restrict__ partial,
+                                                                 const __grid_constant__ ChunkRanges r,
+                                                                 double* __restrict__ err, int K,
+                                                                 int32_t* __restrict__ order,
+                                                                 uint8_t* __restrict__ keep) {
+  pdl_wait();
+  pdl_launch();
+  __shared__ double s_a[32], s_b[32];
+  __shared__ double s_err[kSmallLayers];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = r.n_layers;
+  for (int l = 0; l < n; ++l) {
+    double a = 0.0, b = 0.0;
+    for (int c = r.first_chunk[l] + tid; c < r.first_chunk[l + 1]; c += 1024) {
+      const double2 v = __ldcg(partial + c);
+      a += v.x;
+      b += v.y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a += __shfl_xor_sync(0xffffffffu, a, o);
+      b += __shfl_xor_sync(0xffffffffu, b, o);
+    }
+    if (lane == 0) {
+      s_a[warp] = a;
+      s_b[warp] = b;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      a = s_a[lane];
+      b = s_b[lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b += __shfl_xor_sync(0xffffffffu, b, o);
+      }
+      // as finish_layer_warp: an all-zero layer has error 0, a NaN sum gives NaN
+      if (lane == 0) {
+        const double e = (b == 0.0) ? 0.0 : sqrt(a / b);
+        s_err[l] = e;
+        err[l] = e;
+      }
+    }
+    __syncthreads();
+  }
+  for (int l = tid; l < n; l += blockDim.x) {
+    const int rank = rank_of(s_err, n, l);
+    order[rank] = l;
+    keep[l] = rank < K ? 1 : 0;
+  }
+}
+
 // Limit of the chunk kernel's wait for its bulk copy: 2 s, or QLORA_B200_COPY_WAIT_NS
 // (read on every call; 0 = one non-blocking check). A limit that runs out records
 // QLORA_ERR_TIMEOUT (or a NaN error without a status word) and the kernel still waits
@@ -437,20 +495,29 @@ static qlora_status launch_passes(const Tab& tab, double2* partial, int* status,
                                   status, copy_wait_ns())
                      : launch_pdl(layer_error_chunk_kernel<DQ, Tab>, dim3(c), dim3(256), 0, s, tab, partial, status,
                                   copy_wait_ns());
-    if (e == cudaSuccess) e = launch_pdl(layer_error_finish_kernel, dim3(unsigned(n)), dim3(32), 0, s, partial, r, err);
-    if (e == cudaSuccess)
-      e = budget ? launch_pdl(rank_budget_kernel, dim3(1), dim3(1024), 0, s, err, n, *budget, order, keep, K_out)
-                 : launch_pdl(rank_topk_kernel, dim3(1), dim3(1024), 0, s, err, n, K, order, keep);
+    if (e == cudaSuccess && !budget && n <= kSmallLayers) {
+      e = launch_pdl(finish_rank_small_kernel, dim3(1), dim3(1024), 0, s, partial, r, err, K, order, keep);
+    } else {
+      if (e == cudaSuccess)
+        e = launch_pdl(layer_error_finish_kernel, dim3(unsigned(n)), dim3(32), 0, s, partial, r, err);
+      if (e == cudaSuccess)
+        e = budget ? launch_pdl(rank_budget_kernel, dim3(1), dim3(1024), 0, s, err, n, *budget, order, keep, K_out)
+                   : launch_pdl(rank_topk_kernel, dim3(1), dim3(1024), 0, s, err, n, K, order, keep);
+    }
   } else {
     if (err_reload())
       layer_error_chunk_kernel<DQ, Tab, true><<<c, 256, 0, s>>>(tab, partial, status, copy_wait_ns());
     else
       layer_error_chunk_kernel<DQ, Tab><<<c, 256, 0, s>>>(tab, partial, status, copy_wait_ns());
-    layer_error_finish_kernel<<<unsigned(n), 32, 0, s>>>(partial, r, err);
-    if (budget)
-      rank_budget_kernel<<<1, 1024, 0, s>>>(err, n, *budget, order, keep, K_out);
-    else
-      rank_topk_kernel<<<1, 1024, 0, s>>>(err, n, K, order, keep);
+    if (!budget && n <= kSmallLayers) {
+      finish_rank_small_kernel<<<1, 1024, 0, s>>>(partial, r, err, K, order, keep);
+    } else {
+      layer_error_finish_kernel<<<unsigned(n), 32, 0, s>>>(partial, r, err);
+      if (budget)
+        rank_budget_kernel<<<1, 1024, 0, s>>>(err, n, *budget, order, keep, K_out);
+      else
+        rank_topk_kernel<<<1, 1024, 0, s>>>(err, n, K, order, keep);
+    }
     e = cudaSuccess;
   }
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? QLORA_OK : QLORA_ERR_CUDA;
