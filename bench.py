@@ -908,7 +908,7 @@ def gpu_main(args):
         cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": desc + f"; repeated for {secs:.1f} s", "seconds": secs}
 
-    launches_per_step = 3 + 1 + 3 + 5  # quantize+error, finish, rank; T; fwd (scales, s.L2^T, GEMM); bwd (U + s.U, dL2, dL1, scales, dX GEMM)
+    launches_per_step = 2 + 1 + 3 + 5  # quantize+error, finish+rank; T; fwd (scales, s.L2^T, GEMM); bwd (U + s.U, dL2, dL1, scales, dX GEMM)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args, world),
