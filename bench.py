@@ -180,6 +180,23 @@ class ClockSampler:
                 "reasons": sorted(seen), "samples": len(rows)}
 
 
+def cpus_near_gpu(torch, dev):
+    """The host CPUs NVML lists as local to `dev` (its NUMA node), or None."""
+    try:
+        import pynvml
+        props = torch.cuda.get_device_properties(dev)
+        pynvml.nvmlInit()
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        words = (os.cpu_count() + 63) // 64
+        mask = pynvml.nvmlDeviceGetCpuAffinity(h, words)
+        cpus = {w * 64 + b for w, m in enumerate(mask) for b in range(64) if (int(m) >> b) & 1}
+        cpus &= set(os.sched_getaffinity(0))
+        return cpus or None
+    except Exception:
+        return None
+
+
 def pair_gemm_traffic(name: str):
     """DRAM bytes per launch of a fused pair GEMM from the committed ncu capture in
     profiles/roofline_traffic.json, or None when the GEMM's sources changed since the
@@ -799,11 +816,18 @@ def gpu_main(args):
     # last result copy.
     e2e = None
     if args.e2e_steps > 0:
+        # the pinned buffers are placed while this thread runs on the GPU's own NUMA
+        # node, so the copy engines read local memory
+        near, before = cpus_near_gpu(torch, dev), os.sched_getaffinity(0)
+        if near:
+            os.sched_setaffinity(0, near)
         pin = {k: v.cpu().pin_memory() for k, v in d.items()}
         outs = [{"Y": torch.empty((M, o), dtype=torch.bfloat16).pin_memory(),
                  "dX": torch.empty((M, h), dtype=torch.bfloat16).pin_memory(),
                  "dL1": torch.empty((h, r), dtype=torch.float32).pin_memory(),
                  "dL2": torch.empty((r, o), dtype=torch.float32).pin_memory()} for _ in range(2)]
+        if near:
+            os.sched_setaffinity(0, before)
         h2d = sum(t.numel() * t.element_size() for t in pin.values())
         result_names = ("dL1", "dL2")
         d2h = sum(outs[0][k].numel() * outs[0][k].element_size() for k in result_names)
@@ -866,6 +890,7 @@ def gpu_main(args):
         e2e = {"value": fl * world / (em * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": em,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "result": "dL1, dL2 (the adapter gradients)",
+               "host_buffers": "pinned on the GPU's NUMA node" if near else "pinned (NUMA node not known)",
                "with_Y_dX_back": {"ms_per_step": em_all, "TFLOP/s": fl * world / (em_all * 1e-3) / 1e12,
                                   "d2h_bytes_per_step": d2h_all},
                "timing": f"{args.e2e_steps} steps pipelined over three streams (input copies of the next step and "
