@@ -759,6 +759,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 // waits for the count (bounded), adds the partials in pair order to its accumulator
 // and writes the tile.
 //
+// Aux tiles (GemmParams::aux_tiles): the LoRA product the output tiles' LoRA step
+// reads can be computed in the same launch, one leading tile per 512-row block: the
+// forward's T = X L1 (B = L1 by TMA) or the dX pass's U = dY L2^T (B = L2 by TMA,
+// stored as U and s.U). An aux tile takes A like an output tile, stores through the
+// same staging, then releases a per-block flag; an output tile's producer acquires
+// that flag before its LoRA step loads the aux rows. Aux tiles wait on nothing and
+// come first in every pair's order, so no wait closes a cycle.
+//
 // Shared memory per CTA: S ring slots of 48 KB (the A rows 128 rank + {0, 256} +
 // 0..127 of the tile, and this CTA's B half) and kNumStage 16 KB epilogue staging
 // buffers (128 rows x 64 bf16 columns, 128-byte swizzle, written out by TMA store),
@@ -817,8 +825,8 @@ __device__ __forceinline__ void sk_step(const GemmParams& p, int pr, uint32_t i,
   }
 }
 
-// Block and column tile of a tile id: the aux_tiles leading T tiles (block = id,
-// column -1), then the output tiles row-block-major.
+// Block and column tile of a tile id: the aux_tiles leading aux tiles (T or U;
+// block = id, column -1), then the output tiles row-block-major.
 __device__ __forceinline__ void sk_tile(const GemmParams& p, int tile, int& mb, int& nb) {
   if (tile < p.aux_tiles) {
     mb = tile;
@@ -878,7 +886,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
   const int S = p.num_k_main + p.num_k_ext;
   const uint32_t nsteps = sk_num_steps(p, pr);
   const uint32_t dp_steps = uint32_t(p.sk_R) * uint32_t(S);
-  // MMA width of the T tiles: 128 columns hold r <= 128, else 256
+  // MMA width of the aux tiles: 128 columns hold r <= 128, else 256
   const int t_n = p.t_chunks <= 2 ? 128 : 256;
 
   if (warp == 0) {
@@ -900,12 +908,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         const int m0 = mb * 512 + int(rank) * 128;
         const bool main_step = k < p.num_k_main;
         const uint32_t dst = slot(it), bar = ready(it % C::S);
-        // a T tile reads X in every step (its extra step starts past the K extent: zeros)
+        // an aux tile reads A (X or dY) in every step (its extra step starts past the K
+        // extent: zeros)
         const bool x_step = main_step || ttile;
         const CUtensorMap* m = x_step ? &tmA : &tmAx;
         const int kx = (x_step ? k : k - p.num_k_main) * 64;
         if (!x_step && p.aux_tiles > 0 && k == p.num_k_main) {
-          // the first LoRA step of an output tile needs its block's T: wait for the flag
+          // the first LoRA step of an output tile needs its block's T (or s.U): wait for
+          // the flag
           int* fl = p.t_flags + (mb * 2 + int(rank)) * 2;
           if (ld_acquire_gpu(fl) == 0) {
             const uint64_t t0 = globaltimer_ns();
@@ -924,9 +934,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
           }
         }
         if (rank == 0) {
-          // bytes of the whole step: both CTAs' two A sub-tiles and, in LoRA steps and T
-          // tiles, B halves by TMA
-          // (a T tile's B is its MMA width t_n x 64 rows of L1, split over the pair)
+          // bytes of the whole step: both CTAs' two A sub-tiles and, in LoRA steps and aux
+          // tiles, B halves by TMA (an aux tile's B is its MMA width t_n x 64 K, split
+          // over the pair)
           mbar_arrive_expect_tx(bar, 4 * C::kA + (main_step && !ttile ? uint32_t(C::kWarpsPerSlot * C::kSigBytes)
                                                   : ttile             ? uint32_t(t_n * 128)
                                                                       : uint32_t(2 * C::kB)));
@@ -1028,7 +1038,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       const int ke = kb + len;
       int mb, nb;
       sk_tile(p, tile, mb, nb);
-      const bool ttile = nb < 0;                         // a T tile: T = X L1 of block mb
+      const bool ttile = nb < 0;                         // an aux tile: T or U of block mb
       const int nchunks = ttile ? p.t_chunks : 4;        // 64-column chunks written
       const uint32_t par = seg & 1u;
       ++seg;
@@ -1143,8 +1153,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         p.sk_count[2 * (tile - p.sk_base) + int(rank)] = 0;
       }
       if (ttile && leader) {
-        // this CTA's T rows of the block are in global memory: raise its flag for the
-        // output tiles' LoRA steps (they read T with TMA after an acquire of the flag)
+        // this CTA's aux rows of the block are in global memory: raise its flag for the
+        // output tiles' LoRA steps (they read them with TMA after an acquire of the flag)
         bulk_wait_group<0>();
         fence_proxy_async_global();
         __threadfence();
@@ -1456,7 +1466,7 @@ void pair2_schedule_of(int tiles, int steps, int pairs, int32_t* out) {
 }
 
 size_t pair2_partial_bytes(int64_t M, int64_t N) {
-  const int64_t T = ((M + 511) / 512) * (N / 256 + 1);   // with the forward's T tiles
+  const int64_t T = ((M + 511) / 512) * (N / 256 + 1);   // with the aux tiles
   const int64_t slots = std::min<int64_t>(kPair2MaxPairs, 4 * T);
   return size_t(slots) * (size_t(2) * 2 * 256 * 128 * sizeof(float));
 }
