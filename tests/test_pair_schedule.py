@@ -90,3 +90,78 @@ def test_schedule_refuses_bad_arguments(lib):
     assert lib.qlora_pair_schedule(0, 5, 4, out) == 2
     assert lib.qlora_pair_schedule(5, 5, 81, out) == 2
     assert lib.qlora_pair_schedule(5, 5, 4, None) == 1
+
+
+def simulate_flags(P, R, L, W, base, launch, blocks, per_block, steps, ext, aux_last=False):
+    """Runs the kernel's per-pair step order as a discrete-event model: every pair
+    advances one K step per tick unless blocked. An output tile's first LoRA step
+    (k = steps - ext) waits until its block's aux tile (tile id = block) is finished,
+    i.e. every step of it is done by whichever pairs hold its parts (a split tile's
+    finishing pair adds the other parts once they have counted in; it holds its
+    pair's last range, so its own wait delays nothing else). Returns the number of
+    ticks, or None if the pairs deadlock. aux_last puts the aux tiles after the output
+    tiles instead (an order the kernel does not use; the model must catch it)."""
+    aux = blocks
+    total = aux + blocks * per_block
+    seqs = []
+    for pr in range(launch):
+        dp = R * steps
+        n = dp + max(0, min(pr * L + L, W) - pr * L)
+        seq = []
+        for i in range(n):
+            if i < dp:
+                r = i // steps
+                seq.append((pr + r * P, i - r * steps))
+            else:
+                ti = pr * L + (i - dp)
+                u = ti // steps
+                seq.append((base + u, ti - u * steps))
+        seqs.append(seq)
+    done_steps = [0] * total
+    pos = [0] * launch
+    ticks = 0
+    while any(pos[p] < len(seqs[p]) for p in range(launch)):
+        moved = False
+        for p in range(launch):
+            if pos[p] >= len(seqs[p]):
+                continue
+            tile, k = seqs[p][pos[p]]
+            is_aux = (tile >= total - aux) if aux_last else (tile < aux)
+            if not is_aux and k == steps - ext:
+                mb = (tile if aux_last else tile - aux) // per_block
+                flag_tile = total - aux + mb if aux_last else mb
+                if done_steps[flag_tile] < steps:
+                    continue                      # the LoRA step waits for the block's T / U
+            pos[p] += 1
+            done_steps[tile] += 1
+            moved = True
+        ticks += 1
+        if not moved:
+            return None
+    assert all(d == steps for d in done_steps)
+    return ticks
+
+
+@pytest.mark.parametrize("pairs", [1, 2, 3, 5, 7, 16, 74])
+def test_aux_flag_waits_never_deadlock(lib, pairs):
+    """The aux tiles (T or U, one per 512-row block) set a per-block flag that the
+    output tiles' first LoRA step waits for. Walking the library's schedule with
+    those waits and with split tiles finished only after all their parts, every pair
+    count and shape finishes: no wait closes a cycle."""
+    for blocks in (1, 2, 3, 5, 16, 17):
+        for per_block in (1, 2, 3, 16):
+            for steps, ext in ((2, 1), (5, 1), (9, 1), (66, 2), (65, 1)):
+                tiles = blocks * per_block
+                if (tiles + blocks) * steps > 30000:
+                    continue
+                P, R, L, W, base, launch = schedule(lib, tiles + blocks, steps, pairs)
+                assert simulate_flags(P, R, L, W, base, launch, blocks, per_block, steps, ext) is not None
+
+
+def test_aux_flag_model_catches_a_bad_order(lib):
+    """The model is not vacuous: with the aux tiles after the output tiles, a single
+    pair reaches an output tile's LoRA step before its block's aux tile and waits
+    forever."""
+    P, R, L, W, base, launch = schedule(lib, 2 + 2 * 3, 5, 1)
+    assert simulate_flags(P, R, L, W, base, launch, 2, 3, 5, 1, aux_last=True) is None
+    assert simulate_flags(P, R, L, W, base, launch, 2, 3, 5, 1) is not None
