@@ -136,14 +136,20 @@ qlora_status qlora_profile_events(void* fwd_begin, void* fwd_end, void* dx_begin
 int32_t qlora_pair_clusters(void);
 
 /* Diagnostic, host only (no device work): the schedule the NF4 pair GEMM (512 x 256
- * tiles) uses for `tiles` output tiles of `steps` K steps (K / 64 plus the LoRA
- * steps) over `pairs` co-resident CTA pairs (1..80):
+ * tiles) uses for `tiles` tiles of `steps` K steps (K / 64 plus the LoRA steps), the
+ * first `aux_tiles` of them the T or U tiles (0 when the LoRA product is computed
+ * apart), over `pairs` co-resident CTA pairs (1..80):
  *   out[0] P = pairs, out[1] R = whole rounds (pair p takes tiles p + r P, r < R),
  *   out[2] L = steps per pair in the remaining tiles (0: none remain), out[3] W =
- *   their total steps (pair p takes steps [p L, min((p + 1) L, W)) of them, tile
- *   base + step / steps), out[4] base = R P, out[5] pairs launched.
- * A tile cut into parts is finished by the pair holding its first step. */
-qlora_status qlora_pair_schedule(int32_t tiles, int32_t steps, int32_t pairs, int32_t* out);
+ *   their total steps, out[4] base = R P (tail step s is step s % steps of tile
+ *   base + s / steps), out[5] pairs launched, out[6] A and out[7] La: pair p < A (one
+ *   that ran an aux tile, about half a tile's work) takes tail steps [p La, (p + 1)
+ *   La), pair p >= A takes [A La + (p - A) L, + L), all clipped to W (A = 0: every
+ *   pair [p L, (p + 1) L)).
+ * A tile cut into parts is finished by the pair holding its first step.
+ * QLORA_ERR_SHAPE unless tiles >= 1, 0 <= aux_tiles <= tiles, steps >= 1 and
+ * 1 <= pairs <= 80; QLORA_ERR_NULL when out is NULL. */
+qlora_status qlora_pair_schedule(int32_t tiles, int32_t aux_tiles, int32_t steps, int32_t pairs, int32_t* out);
 
 /* ------------------------------------------------------------ NF4 codec */
 

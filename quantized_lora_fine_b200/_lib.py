@@ -38,7 +38,7 @@ SIGNATURES = {
     "qlora_device_check": (c_int, [c_int]),
     "qlora_profile_events": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p]),
     "qlora_pair_clusters": (c_int32, []),
-    "qlora_pair_schedule": (c_int, [c_int32, c_int32, c_int32, c_void_p]),
+    "qlora_pair_schedule": (c_int, [c_int32, c_int32, c_int32, c_int32, c_void_p]),
     "nf4_rank_errors": (c_int, [c_int32, c_void_p, c_int32, c_void_p, c_void_p, c_void_p]),
     "nf4_quantize_workspace_size": (c_size_t, [c_int64]),
     "nf4_quantize": (c_int, [c_void_p, c_int32, c_int64, c_int64, NF4QConfig, c_void_p, c_void_p, c_void_p,

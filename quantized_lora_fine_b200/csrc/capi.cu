@@ -475,10 +475,11 @@ const char* qlora_status_str(qlora_status s) {
 
 int32_t qlora_pair_clusters(void) { return last_pair_clusters(); }
 
-qlora_status qlora_pair_schedule(int32_t tiles, int32_t steps, int32_t pairs, int32_t* out) {
+qlora_status qlora_pair_schedule(int32_t tiles, int32_t aux_tiles, int32_t steps, int32_t pairs, int32_t* out) {
   if (!out) return QLORA_ERR_NULL;
-  if (tiles < 1 || steps < 1 || pairs < 1 || pairs > kPair2MaxPairs) return QLORA_ERR_SHAPE;
-  pair2_schedule_of(tiles, steps, pairs, out);
+  if (tiles < 1 || aux_tiles < 0 || aux_tiles > tiles || steps < 1 || pairs < 1 || pairs > kPair2MaxPairs)
+    return QLORA_ERR_SHAPE;
+  pair2_schedule_of(tiles, aux_tiles, steps, pairs, out);
   return QLORA_OK;
 }
 

@@ -802,11 +802,23 @@ struct Pair2Cfg {
   static_assert(kStageOff % 1024 == 0, "swizzled staging must be 1024-byte aligned");
 };
 
+// Tail range of pair `pr`: its first tail step and length (see GemmParams::sk_*).
+__device__ __forceinline__ int sk_tail_begin(const GemmParams& p, int pr) {
+  return pr < p.sk_A ? pr * p.sk_La : p.sk_A * p.sk_La + (pr - p.sk_A) * p.sk_L;
+}
+__device__ __forceinline__ int sk_tail_len(const GemmParams& p, int pr) {
+  return pr < p.sk_A ? p.sk_La : p.sk_L;
+}
+// The pair whose tail range holds tail step s (s < sk_W).
+__device__ __forceinline__ int sk_pair_of(const GemmParams& p, int s) {
+  const int a = p.sk_A * p.sk_La;
+  return s < a ? s / p.sk_La : p.sk_A + (s - a) / p.sk_L;
+}
 // Steps of pair `pr` and the (tile, k step) of its step i (see GemmParams::sk_*).
 __device__ __forceinline__ uint32_t sk_num_steps(const GemmParams& p, int pr) {
   const int S = p.num_k_main + p.num_k_ext;
   uint32_t n = uint32_t(p.sk_R) * uint32_t(S);
-  const int b = pr * p.sk_L, e = min(b + p.sk_L, p.sk_W);
+  const int b = sk_tail_begin(p, pr), e = min(b + sk_tail_len(p, pr), p.sk_W);
   if (e > b) n += uint32_t(e - b);
   return n;
 }
@@ -818,7 +830,7 @@ __device__ __forceinline__ void sk_step(const GemmParams& p, int pr, uint32_t i,
     tile = pr + r * p.sk_P;
     k = int(i) - r * S;
   } else {
-    const int ti = pr * p.sk_L + int(i - dp);
+    const int ti = sk_tail_begin(p, pr) + int(i - dp);
     const int u = ti / S;
     tile = p.sk_base + u;
     k = ti - u * S;
@@ -1046,7 +1058,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
       if (kb > 0 || ke < S) {
         // ---- a tile cut into parts (pairs pf .. pl, in step order)
         const int u = tile - p.sk_base;
-        const int pf = (u * S) / p.sk_L, pl = ((u + 1) * S - 1) / p.sk_L;
+        const int pf = sk_pair_of(p, u * S), pl = sk_pair_of(p, (u + 1) * S - 1);
         int* counter = p.sk_count + 2 * u + int(rank);
         if (kb > 0) {
           // a later part: fp32 partial to this pair's slot (column-major in 128-row
@@ -1436,9 +1448,13 @@ static int pair2_pair_cap() {
 // third of a tile, so a tile has at most four parts). When cutting saves less than a
 // twentieth of a tile, L = S: the remaining tiles run whole, one per pair.
 struct Pair2Sched {
-  int P, R, L, W, base, launch;
+  int P, R, L, W, base, launch, A, La;
 };
-static Pair2Sched pair2_schedule(int T, int S, int P) {
+// T tiles (the first A of them aux tiles) of S steps over P pairs. When the aux tiles
+// all fall in the first of at least one whole round, the pairs that ran one (about
+// half an output tile's work: the same A bytes, half the MMA width) take tail
+// ranges longer by 9/20 of a tile, so all pairs end together.
+static Pair2Sched pair2_schedule(int T, int S, int P, int A = 0) {
   Pair2Sched sc;
   sc.P = P;
   sc.R = T / P;
@@ -1446,29 +1462,51 @@ static Pair2Sched pair2_schedule(int T, int S, int P) {
   sc.base = sc.R * P;
   sc.W = Tr * S;
   sc.L = 0;
+  sc.A = 0;
+  sc.La = 0;
+  const int min_range = (S + 2) / 3;   // at most four parts per tile
   if (Tr > 0) {
-    int L = std::max((sc.W + P - 1) / P, (S + 2) / 3);
+    int L = std::max((sc.W + P - 1) / P, min_range);
     if (L >= S || (S - L) * 20 < S) L = S;
     sc.L = L;
+    // (only where the others' ranges stay at least a third of a tile; else even ranges)
+    const int e = (9 * S) / 20;
+    if (A > 0 && A <= P && sc.R >= 1 && L < S && e > 0) {
+      const int Ln = (sc.W - A * e + P - 1) / P;
+      if (Ln >= min_range) {
+        sc.A = A;
+        sc.La = Ln + e;
+        sc.L = Ln;
+      }
+    }
   }
   sc.launch = sc.R > 0 ? P : (sc.L > 0 ? (sc.W + sc.L - 1) / sc.L : 0);
   return sc;
 }
 
-void pair2_schedule_of(int tiles, int steps, int pairs, int32_t* out) {
-  const Pair2Sched sc = pair2_schedule(tiles, steps, pairs);
+void pair2_schedule_of(int tiles, int aux_tiles, int steps, int pairs, int32_t* out) {
+  const Pair2Sched sc = pair2_schedule(tiles, steps, pairs, aux_tiles);
   out[0] = sc.P;
   out[1] = sc.R;
   out[2] = sc.L;
   out[3] = sc.W;
   out[4] = sc.base;
   out[5] = sc.launch;
+  out[6] = sc.A;
+  out[7] = sc.La;
 }
 
 size_t pair2_partial_bytes(int64_t M, int64_t N) {
   const int64_t T = ((M + 511) / 512) * (N / 256 + 1);   // with the aux tiles
   const int64_t slots = std::min<int64_t>(kPair2MaxPairs, 4 * T);
   return size_t(slots) * (size_t(2) * 2 * 256 * 128 * sizeof(float));
+}
+
+// Longer tail ranges for the pairs that ran an aux tile, unless QLORA_B200_AUX_BALANCE=0
+// (read on every call).
+static bool aux_balance() {
+  const char* e = std::getenv("QLORA_B200_AUX_BALANCE");
+  return !(e && std::strcmp(e, "0") == 0);
 }
 
 template <class C>
@@ -1482,13 +1520,16 @@ static qlora_status launch_pair2_cfg(const GemmOperands& o, GemmParams p, cudaSt
                           p.t_chunks < 1 || p.t_chunks > 4))
     return QLORA_ERR_CUDA;
   if (T <= 0 || S <= 0) return QLORA_OK;
-  const Pair2Sched sc = pair2_schedule(T, S, max_pairs);
+  const Pair2Sched sc = pair2_schedule(T, S, max_pairs, aux_balance() ? p.aux_tiles : 0);
   p.sk_P = sc.P;
   p.sk_R = sc.R;
   p.sk_L = sc.L;
   p.sk_W = sc.W;
   p.sk_base = sc.base;
-  if (sc.launch > kPair2MaxPairs || (sc.L > 0 && sc.L < S && (!p.sk_part || !p.sk_count))) return QLORA_ERR_CUDA;
+  p.sk_A = sc.A;
+  p.sk_La = sc.La;
+  const bool may_split = sc.W > 0 && (sc.A > 0 || (sc.L > 0 && sc.L < S));
+  if (sc.launch > kPair2MaxPairs || (may_split && (!p.sk_part || !p.sk_count))) return QLORA_ERR_CUDA;
   g_last_pairs = sc.launch;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];

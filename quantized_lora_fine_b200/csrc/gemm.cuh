@@ -44,8 +44,11 @@ struct GemmParams {
   // (tail tile u is tile sk_base + u). A tile split over several pairs is finished by
   // the pair that holds its first step: it adds the others' fp32 partials (sk_part,
   // one slot per pair) in pair order once their counter (sk_count, two per tail tile,
-  // left at zero) says they are written.
-  int sk_P, sk_R, sk_L, sk_W, sk_base;
+  // left at zero) says they are written. With sk_A > 0 the first sk_A pairs (those
+  // whose first round was an aux tile, about half a tile's work) take tail ranges of
+  // sk_La steps instead: pair p < sk_A takes [p sk_La, (p + 1) sk_La), pair p >= sk_A
+  // [sk_A sk_La + (p - sk_A) sk_L, + sk_L), all clipped to sk_W.
+  int sk_P, sk_R, sk_L, sk_W, sk_base, sk_A, sk_La;
   float* sk_part;
   int* sk_count;
   // Forward of the 512 x 256 pair kernel with T = X L1 fused in: aux_tiles leading
@@ -101,8 +104,8 @@ qlora_status launch_gemm_pair(bool dx, const GemmOperands& o, const GemmParams& 
 // p.sk_part (pair2_partial_bytes(...) bytes) and p.sk_count (pair2_counter_ints(...)
 // ints, zero); requires N % 256 == 0.
 qlora_status launch_gemm_pair2(bool dx, const GemmOperands& o, GemmParams p, cudaStream_t s);
-// The schedule over `pairs` co-resident pairs: {P, R, L, W, base, launch} (host only).
-void pair2_schedule_of(int tiles, int steps, int pairs, int32_t* out);
+// The schedule over `pairs` co-resident pairs: {P, R, L, W, base, launch, A, La} (host only).
+void pair2_schedule_of(int tiles, int aux_tiles, int steps, int pairs, int32_t* out);
 // Upper bounds of the split-round scratch for a D[M x N] product (host only).
 size_t pair2_partial_bytes(int64_t M, int64_t N);
 constexpr int kPair2MaxPairs = 80;                 // pairs launched at most
