@@ -5,9 +5,12 @@ double quantization (E4M3 absmax, groups of 256), X 8192 x 4096 bf16 (batch 4 x
 seq 2048), rank 16, alpha 32, forward + backward (dX, dL1, dL2).
 
 One timed step runs every step of the path once on that batch:
-  nf4_quantize(W, dq)                  quantize + double-quantize the scales
-  nf4_layer_error_rank([W], K=0)       per-layer NF4 error + ranking
-  qlora_linear_fwd                     T = X L1; Y = X W^T + s T L2 (fused dequant GEMM)
+  nf4_quantize_error_rank([W], K=0)    the allocation pass with the quantization it
+                                       measures: codes, double-quantized scales,
+                                       per-layer NF4 error and ranking from one read
+                                       of W (on a second stream, beside T)
+  qlora_lora_down                      T = X L1
+  qlora_linear_fwd_t                   Y = X W^T + s T L2 (fused dequant GEMM)
   qlora_linear_bwd                     U, dL2, dL1, dX = dY W + s U L1^T (fused dequant GEMM)
 `value` counts only the algorithmic fwd+bwd flops (4 M h o + 6 M r (h + o))
 over the whole step time; per-leg times are reported beside it.
